@@ -1,0 +1,198 @@
+/*
+ * ispa.h -- C ABI of the ISPA warmup hot path on B200 (sm_100a).
+ *
+ * Method: "Towards Memory-Efficient Autoregressive Video Generation via
+ * Instance-Specific Parametric Absorption" (technical summary, section 2):
+ *   1. Dual-stream warmup: every layer computes A_full (sink + history +
+ *      current chunk) and A_loc (sink + current chunk) in one decomposed
+ *      attention pass whose two branches are merged by their log-sum-exp.
+ *   2. Layer absorb: Delta W = (A_loc^T A_loc + lambda I)^-1
+ *      A_loc^T (A_full - A_loc) W, the minimiser of
+ *      ||A_loc (W + Delta W) - A_full W||_F^2 + lambda ||Delta W||_F^2.
+ *   3. Layers are ranked by their reconstruction error epsilon; the K with
+ *      the lowest error become local-attention layers (W + Delta W).
+ *
+ * Conventions shared by every call
+ *  - All array arguments are DEVICE pointers unless stated otherwise; the
+ *    caller allocates and owns them. The library allocates no device memory
+ *    of its own: calls that need scratch take a caller-provided workspace
+ *    whose size the matching *_workspace_size() query returns.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream). The return value reports only what the host can check
+ *    before launch; conditions found on the device are OR-ed into a device
+ *    status word (`dev_status`, an int the caller zeroes and reads after
+ *    synchronising) as ISPA_STATUS_* bits.
+ *  - Attention tensors are token-major: a [n, heads, head_dim] bf16 array,
+ *    row stride heads * head_dim elements, the heads concatenated head-major.
+ *    Attention outputs are [nq, d] with d = heads * head_dim.
+ *  - Base pointers must be 16-byte aligned.
+ */
+#ifndef ISPA_H_
+#define ISPA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ISPA_API __attribute__((visibility("default")))
+#else
+#define ISPA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- host-side return codes ------------------------------------------ */
+#define ISPA_OK 0
+#define ISPA_ERR_ARG (-1)         /* null pointer, negative size, bad scale ... */
+#define ISPA_ERR_UNSUPPORTED (-2) /* shape or alignment this build does not handle */
+#define ISPA_ERR_WORKSPACE (-3)   /* workspace missing or smaller than required */
+#define ISPA_ERR_CUDA (-4)        /* a CUDA runtime/driver call failed */
+#define ISPA_ERR_NO_DEVICE (-5)   /* the current device is not sm_100 */
+
+/* ---- device status bits (OR-ed into *dev_status) --------------------- */
+#define ISPA_STATUS_TIMEOUT 1      /* a bounded wait in a kernel gave up */
+#define ISPA_STATUS_FP16_RANGE 2   /* a V value fell outside fp16 range (|v| > 65504) */
+#define ISPA_STATUS_NOT_SPD 4      /* G + lambda I was not positive definite */
+#define ISPA_STATUS_NONFINITE 8    /* a non-finite value reached an output */
+
+/* One branch of the KV cache: keys and values [len, heads, head_dim] bf16.
+ * len may be 0 (then k and v are ignored and may be NULL). */
+typedef struct {
+  const void* k;
+  const void* v;
+  int64_t len;
+} ispa_kv;
+
+/* Text for a return code or a status bit. Never NULL. Host only. */
+ISPA_API const char* ispa_status_string(int code);
+
+/* Library version as major*10000 + minor*100 + patch. */
+ISPA_API int ispa_version(void);
+
+/* ---- 1. dual-stream attention ----------------------------------------
+ * Technical summary section 2, step 1 ("Dual-Stream Warmup", decomposable
+ * attention): for every query row and head, softmax(q k^T * scale) v over
+ * the local branch (sink then local keys) gives A_loc and LSE_loc; the same
+ * pass continues over the history keys as a second online-softmax branch
+ * (A_hist, LSE_hist); the two are merged by their log-sum-exp into A_full:
+ *   LSE_full = log(exp(LSE_loc) + exp(LSE_hist)),
+ *   A_full   = e^(LSE_loc-LSE_full) A_loc + e^(LSE_hist-LSE_full) A_hist.
+ * D = A_full - A_loc is formed in fp32 from the two branch outputs, never
+ * as the difference of two rounded outputs.
+ *
+ * q        [nq, heads, head_dim] bf16.
+ * sink, local, hist: the three key/value branches. sink.len + local.len
+ *          must be >= 1; hist.len may be 0 (then LSE_hist = -inf, D = 0,
+ *          A_full = A_loc).
+ * heads    >= 1; head_dim must be 64 or 128.
+ * scale    softmax scale (> 0), normally 1/sqrt(head_dim).
+ * a_loc    out [nq, d] fp32 (rounded to tf32, nearest-away), required.
+ * d_out    out [nq, d] fp32 (rounded to tf32), required.
+ * a_full   out [nq, d] bf16, optional (NULL: not written).
+ * lse_loc, lse_hist, lse_full: out [heads, nq] fp32, natural log, optional.
+ * workspace: device scratch of >= ispa_dual_attention_workspace_size()
+ *          bytes, 256-byte aligned; holds V converted to fp16 (the P.V
+ *          product runs with fp16 P and fp16 V). Its contents are
+ *          overwritten; it must not be used by another call in flight.
+ * dev_status: device int; ISPA_STATUS_FP16_RANGE if a V value overflowed
+ *          fp16, ISPA_STATUS_TIMEOUT if a kernel wait gave up.
+ * Returns ISPA_OK or an ISPA_ERR_* code (nothing is launched on error).
+ */
+ISPA_API size_t ispa_dual_attention_workspace_size(int64_t sink_len, int64_t local_len, int64_t hist_len,
+                                          int heads, int head_dim);
+ISPA_API int ispa_dual_attention(const void* q, int64_t nq, int heads, int head_dim, ispa_kv sink,
+                        ispa_kv local, ispa_kv hist, float scale, float* a_loc, float* d_out,
+                        void* a_full, float* lse_loc, float* lse_hist, float* lse_full,
+                        void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
+
+/* ---- 1b. local attention (L-Layer after the transition) --------------
+ * Technical summary section 2, step 3: a local-attention layer keeps only
+ * the sink and the current chunk. Same kernel as ispa_dual_attention with
+ * no history branch. out_f32 [nq, d] fp32 and/or out_bf16 [nq, d] bf16
+ * (at least one non-NULL), lse [heads, nq] optional. Workspace as above
+ * with hist_len = 0.
+ */
+ISPA_API int ispa_local_attention(const void* q, int64_t nq, int heads, int head_dim, ispa_kv sink,
+                         ispa_kv local, float scale, float* out_f32, void* out_bf16, float* lse,
+                         void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
+
+/* ---- 2. Gram accumulation --------------------------------------------
+ * Technical summary section 2, step 2: the closed form needs
+ * G = A_loc^T A_loc and R = A_loc^T (A_full - A_loc) over all warmup rows;
+ * the reconstruction error also needs S = D^T D. This call adds the
+ * contribution of `rows` rows:
+ *     M[0:d, 0:d]  (G) += A_loc^T A_loc
+ *     M[0:d, d:2d] (R) += A_loc^T D
+ *     M[d:2d, d:2d] (S) += D^T D          (only if want_s != 0)
+ * M is [2d, 2d] fp32 row-major (leading dimension 2d). G and S are
+ * symmetric and only their 128x128 tiles on or above the diagonal are
+ * written; the tiles below it and the block M[d:2d, 0:d] are not touched.
+ * accumulate = 0 overwrites instead of adding (first chunk).
+ * a_loc, d_in: [rows, dim] fp32 row-major. Products run on the tensor
+ * cores in tf32 (inputs are used as tf32, accumulation in fp32).
+ * dim must be a multiple of 128; rows >= 0 (rows = 0 with accumulate = 0
+ * zeroes the written tiles).
+ */
+ISPA_API int ispa_gram_accumulate(const float* a_loc, const float* d_in, int64_t rows, int dim, float* M,
+                         int accumulate, int want_s, void* stream);
+
+/* ---- 3. absorb solve ---------------------------------------------------
+ * Technical summary section 2, step 2 (closed form): solves
+ *     (G + lambda I) Delta W = R W
+ * with G, R read from M (layout of ispa_gram_accumulate) by a blocked
+ * Cholesky factorisation of G + lambda I in fp32 followed by two triangular
+ * solves.
+ * W        [dim, dim] fp32 row-major, the layer's output projection.
+ * lambda   > 0: used as given. <= 0: lambda = 1e-2 * trace(G) / dim,
+ *          computed on the device.
+ * dW       out [dim, dim] fp32.
+ * B        out [dim, dim] fp32: R W (kept for ispa_layer_error).
+ * lambda_out out, device float, optional: the lambda used.
+ * workspace: >= ispa_absorb_workspace_size(dim) bytes, 256-byte aligned.
+ * dev_status: ISPA_STATUS_NOT_SPD if a Cholesky pivot was not positive
+ *          (dW is then undefined).
+ * dim must be a multiple of 128.
+ */
+ISPA_API size_t ispa_absorb_workspace_size(int dim);
+ISPA_API int ispa_absorb_solve(const float* M, const float* W, int dim, float lambda, float* dW, float* B,
+                      float* lambda_out, void* workspace, size_t workspace_bytes, int* dev_status,
+                      void* stream);
+
+/* ---- 4. reconstruction error and layer ranking -------------------------
+ * Technical summary section 2, "Dynamic layer selection": every layer's
+ * error after absorption, then an ascending ranking over layers; the K
+ * layers with the lowest error become local-attention layers.
+ *
+ * ispa_layer_error: one layer. With E = A_loc (W + Delta W) - A_full W the
+ * error is formed from the Gram blocks, without a pass over the rows:
+ *     ||E||_F^2        = <S, W W^T> - <Delta W, B> - lambda ||Delta W||_F^2
+ *     ||A_full W||_F^2 = <G + R + R^T + S, W W^T>
+ * (both follow from (G + lambda I) Delta W = B = R W); W W^T is formed
+ * tile by tile in fp32 and every reduction is accumulated in fp64.
+ * M        [2d, 2d] from ispa_gram_accumulate with want_s != 0.
+ * W, dW, B [dim, dim] fp32 (dW, B from ispa_absorb_solve).
+ * lambda   device float (the lambda the solve used, e.g. its lambda_out).
+ * err      out, device double[2]: {||E||_F^2, ||E||_F^2 / ||A_full W||_F^2}.
+ * workspace: >= ispa_layer_error_workspace_size() bytes (accumulators).
+ * dim must be a multiple of 128.
+ *
+ * ispa_rank_layers: err is device double[2 * n_layers] (layer l at
+ * err + 2 l); layers are ordered by ascending relative error, ties to the
+ * lower layer index.
+ * perm     out, device int[n_layers]: layer indices in that order.
+ * selected out, device uint8[n_layers], optional: 1 for the first K of perm.
+ * 1 <= n_layers <= 4096, 0 <= K <= n_layers.
+ */
+ISPA_API size_t ispa_layer_error_workspace_size(int dim);
+ISPA_API int ispa_layer_error(const float* M, const float* W, const float* dW, const float* B,
+                     const float* lambda, int dim, double* err, void* workspace,
+                     size_t workspace_bytes, void* stream);
+ISPA_API int ispa_rank_layers(const double* err, int n_layers, int K, int* perm, uint8_t* selected,
+                     void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ISPA_H_ */

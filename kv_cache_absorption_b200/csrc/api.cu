@@ -1,0 +1,284 @@
+// C ABI of the ISPA warmup hot path: argument checks, TMA descriptor
+// encoding, workspace carving and kernel launches. Declarations and the
+// contract of every entry point are in include/ispa.h.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "sm100.cuh"
+#include "attention.h"
+
+namespace ispa {
+size_t absorb_workspace_bytes(int dim);
+cudaError_t absorb_solve(const float* M, const float* W, int dim, float lambda, float* dW,
+                         float* B, float* lambda_out, void* workspace, int* status,
+                         cudaStream_t stream);
+cudaError_t layer_error(const float* M, const float* W, const float* dW, const float* B,
+                        const float* lam, int dim, double* err, double* acc, cudaStream_t stream);
+cudaError_t rank_layers(const double* err, int n, int K, int* perm, uint8_t* selected,
+                        cudaStream_t stream);
+}  // namespace ispa
+
+namespace {
+
+using ispa::AttnParams;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major [rows, cols] matrix, tiles of box_cols x box_rows.
+bool encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t cols,
+               uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (uint64_t)esize};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// The kernels use tcgen05 and TMA: only compute capability 10.0 parts run them.
+int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ISPA_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return ISPA_ERR_CUDA;
+  return (major == 10 && minor == 0) ? ISPA_OK : ISPA_ERR_NO_DEVICE;
+}
+
+int cuda_rc(cudaError_t e) {
+  if (e == cudaSuccess) return ISPA_OK;
+  std::fprintf(stderr, "ispa: CUDA error %s\n", cudaGetErrorString(e));
+  return ISPA_ERR_CUDA;
+}
+
+bool kv_ok(const ispa_kv& b) {
+  if (b.len < 0 || b.len > (int64_t)1 << 31) return false;
+  if (b.len == 0) return true;
+  return b.k && b.v && aligned16(b.k) && aligned16(b.v);
+}
+
+size_t v_half_bytes(int64_t len, int d) { return round256((size_t)len * d * 2); }
+
+int attention_common(const void* q, int64_t nq, int heads, int head_dim, const ispa_kv (&br)[3],
+                     float scale, int round_tf32, float* a_loc, float* d_out, void* a_full,
+                     float* lse_loc, float* lse_hist, float* lse_full, void* workspace,
+                     size_t workspace_bytes, int* dev_status, void* stream) {
+  if (!q || !dev_status || nq < 0 || nq > (int64_t)1 << 30 || heads < 1 || heads > 65535)
+    return ISPA_ERR_ARG;
+  if (head_dim != 64 && head_dim != 128) return ISPA_ERR_UNSUPPORTED;
+  if (!(scale > 0.f) || !(scale < 1e30f)) return ISPA_ERR_ARG;
+  for (const auto& b : br)
+    if (!kv_ok(b)) return ISPA_ERR_ARG;
+  if (br[0].len + br[1].len < 1) return ISPA_ERR_ARG;
+  if (!aligned16(q) || (a_loc && !aligned16(a_loc)) || (d_out && !aligned16(d_out)) ||
+      (a_full && !aligned16(a_full)))
+    return ISPA_ERR_UNSUPPORTED;
+  const int d = heads * head_dim;
+  const size_t need = ispa_dual_attention_workspace_size(br[0].len, br[1].len, br[2].len, heads,
+                                                         head_dim);
+  if (!workspace || workspace_bytes < need || !aligned256(workspace)) return ISPA_ERR_WORKSPACE;
+  int rc = check_device();
+  if (rc != ISPA_OK) return rc;
+  if (nq == 0) return ISPA_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!encode_2d(&p.tm_q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, nq, 64, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return ISPA_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  for (int b = 0; b < 3; ++b) {
+    p.len[b] = br[b].len;
+    if (br[b].len == 0) {  // never read: no tiles of this branch
+      p.tm_k[b] = p.tm_q;
+      p.tm_v[b] = p.tm_q;
+      continue;
+    }
+    void* vh = ws;
+    ws += v_half_bytes(br[b].len, d);
+    cudaError_t e = ispa::launch_v_to_half(br[b].v, vh, br[b].len * d, dev_status, s);
+    if (e != cudaSuccess) return cuda_rc(e);
+    if (!encode_2d(&p.tm_k[b], br[b].k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, br[b].len, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&p.tm_v[b], vh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, br[b].len, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return ISPA_ERR_CUDA;
+  }
+  p.nq = (int)nq;
+  p.heads = heads;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.round_tf32 = round_tf32;
+  p.a_loc = a_loc;
+  p.d_out = d_out;
+  p.a_full = static_cast<__nv_bfloat16*>(a_full);
+  p.lse_loc = lse_loc;
+  p.lse_hist = lse_hist;
+  p.lse_full = lse_full;
+  p.status = dev_status;
+  return cuda_rc(ispa::launch_dual_attention(p, head_dim, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ispa_status_string(int code) {
+  switch (code) {
+    case ISPA_OK: return "ok";
+    case ISPA_ERR_ARG: return "invalid argument";
+    case ISPA_ERR_UNSUPPORTED: return "unsupported shape or alignment";
+    case ISPA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case ISPA_ERR_CUDA: return "CUDA error";
+    case ISPA_ERR_NO_DEVICE: return "current device is not an sm_100 GPU";
+    case ISPA_STATUS_TIMEOUT: return "device: a bounded wait timed out";
+    case ISPA_STATUS_FP16_RANGE: return "device: a value exceeded fp16 range";
+    case ISPA_STATUS_NOT_SPD: return "device: G + lambda I is not positive definite";
+    case ISPA_STATUS_NONFINITE: return "device: non-finite output";
+    default: return "unknown status";
+  }
+}
+
+int ispa_version(void) { return 100; }
+
+size_t ispa_dual_attention_workspace_size(int64_t sink_len, int64_t local_len, int64_t hist_len,
+                                          int heads, int head_dim) {
+  if (sink_len < 0 || local_len < 0 || hist_len < 0 || heads < 1 || head_dim < 1) return 0;
+  const int d = heads * head_dim;
+  return v_half_bytes(sink_len, d) + v_half_bytes(local_len, d) + v_half_bytes(hist_len, d) + 256;
+}
+
+int ispa_dual_attention(const void* q, int64_t nq, int heads, int head_dim, ispa_kv sink,
+                        ispa_kv local, ispa_kv hist, float scale, float* a_loc, float* d_out,
+                        void* a_full, float* lse_loc, float* lse_hist, float* lse_full,
+                        void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+  if (!a_loc || !d_out) return ISPA_ERR_ARG;
+  const ispa_kv br[3] = {sink, local, hist};
+  return attention_common(q, nq, heads, head_dim, br, scale, 1, a_loc, d_out, a_full, lse_loc,
+                          lse_hist, lse_full, workspace, workspace_bytes, dev_status, stream);
+}
+
+int ispa_local_attention(const void* q, int64_t nq, int heads, int head_dim, ispa_kv sink,
+                         ispa_kv local, float scale, float* out_f32, void* out_bf16, float* lse,
+                         void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+  if (!out_f32 && !out_bf16) return ISPA_ERR_ARG;
+  const ispa_kv br[3] = {sink, local, ispa_kv{nullptr, nullptr, 0}};
+  return attention_common(q, nq, heads, head_dim, br, scale, 0, out_f32, nullptr, out_bf16, lse,
+                          nullptr, nullptr, workspace, workspace_bytes, dev_status, stream);
+}
+
+int ispa_gram_accumulate(const float* a_loc, const float* d_in, int64_t rows, int dim, float* M,
+                         int accumulate, int want_s, void* stream) {
+  if (!M || rows < 0 || rows > ((int64_t)1 << 31) - 64 || dim <= 0) return ISPA_ERR_ARG;
+  if (dim % 128 != 0 || dim > 32768 || !aligned16(M)) return ISPA_ERR_UNSUPPORTED;
+  if (rows > 0 && (!a_loc || !d_in)) return ISPA_ERR_ARG;
+  if (rows > 0 && (!aligned16(a_loc) || !aligned16(d_in))) return ISPA_ERR_UNSUPPORTED;
+  int rc = check_device();
+  if (rc != ISPA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t d = (size_t)dim;
+  if (!accumulate) {
+    cudaError_t e = cudaMemsetAsync(M, 0, d * 2 * d * sizeof(float), s);  // G and R rows
+    if (e == cudaSuccess && want_s)
+      e = cudaMemset2DAsync(M + d * 2 * d + d, 2 * d * sizeof(float), 0, d * sizeof(float), d, s);
+    if (e != cudaSuccess) return cuda_rc(e);
+  }
+  if (rows == 0) return ISPA_OK;
+  ispa::GramParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!encode_2d(&p.tm_a, a_loc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dim, rows, 32, 32,
+                 CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) ||
+      !encode_2d(&p.tm_d, d_in, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dim, rows, 32, 32,
+                 CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B))
+    return ISPA_ERR_CUDA;
+  const int bn = (dim % 256 == 0) ? 256 : 128;
+  p.M = M;
+  p.dim = dim;
+  p.k_iters = (int)((rows + 31) / 32);
+  p.want_s = want_s ? 1 : 0;
+  p.n_tiles = ispa::gram_tile_count(dim, bn, p.want_s);
+  p.total_iters = (int64_t)p.n_tiles * p.k_iters;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t grid = p.total_iters < sms ? p.total_iters : sms;
+  p.iters_per_cta = (p.total_iters + grid - 1) / grid;
+  p.status = nullptr;
+  return cuda_rc(ispa::launch_gram(p, bn, (int)grid, s));
+}
+
+size_t ispa_absorb_workspace_size(int dim) {
+  if (dim <= 0) return 0;
+  return ispa::absorb_workspace_bytes(dim);
+}
+
+int ispa_absorb_solve(const float* M, const float* W, int dim, float lambda, float* dW, float* B,
+                      float* lambda_out, void* workspace, size_t workspace_bytes, int* dev_status,
+                      void* stream) {
+  if (!M || !W || !dW || !B || !dev_status || dim <= 0 || lambda != lambda) return ISPA_ERR_ARG;
+  if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
+  if (!aligned16(M) || !aligned16(W) || !aligned16(dW) || !aligned16(B))
+    return ISPA_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < ispa::absorb_workspace_bytes(dim) || !aligned256(workspace))
+    return ISPA_ERR_WORKSPACE;
+  int rc = check_device();
+  if (rc != ISPA_OK) return rc;
+  return cuda_rc(ispa::absorb_solve(M, W, dim, lambda, dW, B, lambda_out, workspace, dev_status,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+size_t ispa_layer_error_workspace_size(int dim) { return dim > 0 ? 256 : 0; }
+
+int ispa_layer_error(const float* M, const float* W, const float* dW, const float* B,
+                     const float* lambda, int dim, double* err, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  if (!M || !W || !dW || !B || !lambda || !err || dim <= 0) return ISPA_ERR_ARG;
+  if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
+  if (!aligned16(M) || !aligned16(W) || !aligned16(dW) || !aligned16(B))
+    return ISPA_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < 256 || (reinterpret_cast<uintptr_t>(workspace) & 7u))
+    return ISPA_ERR_WORKSPACE;
+  int rc = check_device();
+  if (rc != ISPA_OK) return rc;
+  return cuda_rc(ispa::layer_error(M, W, dW, B, lambda, dim, err, static_cast<double*>(workspace),
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+int ispa_rank_layers(const double* err, int n_layers, int K, int* perm, uint8_t* selected,
+                     void* stream) {
+  if (!err || !perm || n_layers < 1 || n_layers > 4096 || K < 0 || K > n_layers)
+    return ISPA_ERR_ARG;
+  int rc = check_device();
+  if (rc != ISPA_OK) return rc;
+  return cuda_rc(ispa::rank_layers(err, n_layers, K, perm, selected,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

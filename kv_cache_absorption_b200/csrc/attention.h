@@ -1,0 +1,58 @@
+// Launch-side declarations shared by the C-ABI layer and the kernels.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+namespace ispa {
+
+// Parameters of one dual-stream attention launch. Tensor maps address
+// [len, heads * head_dim] row-major matrices in 64-column x 128-row boxes
+// with 128-byte swizzle: Q and K in bf16, V in fp16 (converted copies).
+struct AttnParams {
+  CUtensorMap tm_q;
+  CUtensorMap tm_k[3];    // sink, local, history
+  CUtensorMap tm_v[3];
+  int64_t len[3];
+  int nq;
+  int heads;
+  float scale_log2;       // softmax scale * log2(e)
+  int round_tf32;         // round A_loc / D stores to tf32 (nearest, ties away)
+  float* a_loc;           // [nq, d] fp32 or nullptr
+  float* d_out;           // [nq, d] fp32 or nullptr
+  __nv_bfloat16* a_full;  // [nq, d] bf16 or nullptr
+  float* lse_loc;         // [heads, nq] or nullptr
+  float* lse_hist;
+  float* lse_full;
+  int* status;
+};
+
+size_t attention_smem_bytes(int head_dim);
+cudaError_t launch_v_to_half(const void* src, void* dst, int64_t n_elems, int* status,
+                             cudaStream_t stream);
+cudaError_t launch_dual_attention(const AttnParams& p, int head_dim, cudaStream_t stream);
+
+// Gram accumulation: see gram.cu.
+struct GramParams {
+  CUtensorMap tm_a;       // A_loc [rows, dim] fp32, 32-column x 32-row boxes
+  CUtensorMap tm_d;       // D
+  float* M;               // [2 dim, 2 dim]
+  int dim;
+  int k_iters;            // ceil(rows / 32)
+  int want_s;
+  int n_tiles;
+  int64_t total_iters;
+  int64_t iters_per_cta;
+  int* status;
+};
+cudaError_t launch_gram(const GramParams& p, int bn, int grid, cudaStream_t stream);
+int gram_tile_count(int dim, int bn, int want_s);
+
+// Dense fp32 helpers for the solve and the error: see solve.cu / error.cu.
+cudaError_t launch_sgemm(bool ta, bool tb, int M, int N, int K, float alpha, const float* A,
+                         int lda, const float* B, int ldb, float beta, float* C, int ldc,
+                         bool lower_only, cudaStream_t stream);
+
+}  // namespace ispa

@@ -1,0 +1,138 @@
+// Reconstruction error per layer and the instance-specific layer ranking.
+//
+// "Towards Memory-Efficient Autoregressive Video Generation via
+// Instance-Specific Parametric Absorption", technical summary section 2,
+// "Dynamic layer selection": after the warmup all layers are ranked by their
+// reconstruction error epsilon and the lowest-error layers become local-
+// attention layers.
+//
+// With E = A_loc (W + dW) - A_full W and (G + lambda I) dW = B = R W:
+//   ||E||^2        = <S, W W^T> - <dW, B> - lambda ||dW||^2
+//   ||A_full W||^2 = <G, W W^T> + 2 <R, W W^T> + <S, W W^T>
+// so the error needs no pass over the warmup rows. W W^T is never stored:
+// each CTA forms one 128 x 128 tile of it in registers and immediately
+// reduces it against the matching tiles of G, R and S (fp64 accumulation).
+// G and S hold only their tiles on and above the tile diagonal: a tile above
+// the diagonal counts twice (for its mirror image), one below it not at all.
+#include "sm100.cuh"
+#include "attention.h"
+#include "simt_gemm.cuh"
+
+namespace ispa {
+namespace {
+
+__device__ __forceinline__ double block_sum(double v, double* red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  double s = 0.0;
+  if (threadIdx.x == 0)
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) s += red[i];
+  __syncthreads();
+  return s;
+}
+
+// acc[0] += <G, WW^T>, acc[1] += <R, WW^T>, acc[2] += <S, WW^T>
+__global__ void __launch_bounds__(kGemmThreads)
+wwt_reduce_kernel(const float* __restrict__ M, const float* __restrict__ W, int dim,
+                  double* __restrict__ acc) {
+  __shared__ GemmSmem sm;
+  __shared__ double red[kGemmThreads / 32];
+  const int I = blockIdx.y, J = blockIdx.x;
+  const int m0 = I * kGemmTile, n0 = J * kGemmTile;
+  float p[8][8];
+  gemm_tile<false, true>(sm, W, dim, W, dim, dim, dim, dim, m0, n0, p);
+  const size_t ld = 2 * (size_t)dim;
+  const double wsym = I < J ? 2.0 : (I == J ? 1.0 : 0.0);
+  double g = 0.0, r = 0.0, s = 0.0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const size_t row = m0 + gemm_row(i);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const size_t col = n0 + gemm_col(j);
+      const double pij = p[i][j];
+      r += (double)M[row * ld + dim + col] * pij;
+      if (wsym != 0.0) {
+        g += (double)M[row * ld + col] * pij;
+        s += (double)M[(row + dim) * ld + dim + col] * pij;
+      }
+    }
+  }
+  g = block_sum(g, red) * wsym;
+  r = block_sum(r, red);
+  s = block_sum(s, red) * wsym;
+  if (threadIdx.x == 0) {
+    atomicAdd(acc + 0, g);
+    atomicAdd(acc + 1, r);
+    atomicAdd(acc + 2, s);
+  }
+}
+
+// acc[3] += <dW, B>, acc[4] += ||dW||^2
+__global__ void dot_kernel(const float4* __restrict__ dW, const float4* __restrict__ B, size_t n4,
+                           double* __restrict__ acc) {
+  __shared__ double red[8];
+  double db = 0.0, dd = 0.0;
+  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n4;
+       e += (size_t)gridDim.x * blockDim.x) {
+    const float4 a = dW[e], b = B[e];
+    db += (double)a.x * b.x + (double)a.y * b.y + (double)a.z * b.z + (double)a.w * b.w;
+    dd += (double)a.x * a.x + (double)a.y * a.y + (double)a.z * a.z + (double)a.w * a.w;
+  }
+  db = block_sum(db, red);
+  dd = block_sum(dd, red);
+  if (threadIdx.x == 0) {
+    atomicAdd(acc + 3, db);
+    atomicAdd(acc + 4, dd);
+  }
+}
+
+__global__ void finalize_kernel(const double* __restrict__ acc, const float* __restrict__ lam,
+                                double* __restrict__ err) {
+  const double l = *lam;
+  const double e2 = acc[2] - acc[3] - l * acc[4];
+  const double den = acc[0] + 2.0 * acc[1] + acc[2];
+  err[0] = e2;
+  err[1] = e2 / den;
+}
+
+// Stable ascending rank of the relative errors err[2 l + 1]: layer i lands at
+// position #{j : e_j < e_i or (e_j == e_i and j < i)}.
+__global__ void rank_kernel(const double* __restrict__ err, int n, int K, int* __restrict__ perm,
+                            uint8_t* __restrict__ selected) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const double ei = err[2 * i + 1];
+    int pos = 0;
+    for (int j = 0; j < n; ++j) {
+      const double ej = err[2 * j + 1];
+      pos += (ej < ei) || (ej == ei && j < i);
+    }
+    perm[pos] = i;
+    if (selected) selected[i] = pos < K ? 1 : 0;
+  }
+}
+
+}  // namespace
+
+cudaError_t layer_error(const float* M, const float* W, const float* dW, const float* B,
+                        const float* lam, int dim, double* err, double* acc,
+                        cudaStream_t stream) {
+  cudaMemsetAsync(acc, 0, 5 * sizeof(double), stream);
+  dim3 grid(dim / kGemmTile, dim / kGemmTile);
+  wwt_reduce_kernel<<<grid, kGemmThreads, 0, stream>>>(M, W, dim, acc);
+  const size_t n4 = (size_t)dim * dim / 4;
+  dot_kernel<<<148 * 2, 256, 0, stream>>>(reinterpret_cast<const float4*>(dW),
+                                          reinterpret_cast<const float4*>(B), n4, acc);
+  finalize_kernel<<<1, 1, 0, stream>>>(acc, lam, err);
+  return cudaGetLastError();
+}
+
+cudaError_t rank_layers(const double* err, int n, int K, int* perm, uint8_t* selected,
+                        cudaStream_t stream) {
+  rank_kernel<<<1, 256, 0, stream>>>(err, n, K, perm, selected);
+  return cudaGetLastError();
+}
+
+}  // namespace ispa

@@ -1,0 +1,283 @@
+"""Thin ctypes binding of the C ABI in include/ispa.h.
+
+Argument marshalling only: checks dtypes, devices and shapes, allocates
+outputs and workspaces through torch's caching allocator, and passes raw
+device pointers plus the current CUDA stream to the library. Every step of
+the computation runs in the library's CUDA kernels; there is no fallback.
+The function names are those of the C entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libispa.so")
+
+ISPA_OK = 0
+ISPA_ERR_ARG = -1
+ISPA_ERR_UNSUPPORTED = -2
+ISPA_ERR_WORKSPACE = -3
+ISPA_ERR_CUDA = -4
+ISPA_ERR_NO_DEVICE = -5
+ISPA_STATUS_TIMEOUT = 1
+ISPA_STATUS_FP16_RANGE = 2
+ISPA_STATUS_NOT_SPD = 4
+ISPA_STATUS_NONFINITE = 8
+
+EXPORTED = (
+    "ispa_status_string", "ispa_version",
+    "ispa_dual_attention_workspace_size", "ispa_dual_attention", "ispa_local_attention",
+    "ispa_gram_accumulate", "ispa_absorb_workspace_size", "ispa_absorb_solve",
+    "ispa_layer_error_workspace_size", "ispa_layer_error", "ispa_rank_layers",
+)
+
+
+class IspaKV(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("len", ctypes.c_int64)]
+
+
+class IspaError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        super().__init__(f"{what}: {ispa_status_string(code)} ({code})" if what else
+                         f"{ispa_status_string(code)} ({code})")
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m kv_cache_absorption_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, I64, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "ispa_status_string": (ctypes.c_char_p, [I]),
+        "ispa_version": (I, []),
+        "ispa_dual_attention_workspace_size": (SZ, [I64, I64, I64, I, I]),
+        "ispa_dual_attention": (I, [P, I64, I, I, IspaKV, IspaKV, IspaKV, F, P, P, P, P, P, P,
+                                    P, SZ, P, P]),
+        "ispa_local_attention": (I, [P, I64, I, I, IspaKV, IspaKV, F, P, P, P, P, SZ, P, P]),
+        "ispa_gram_accumulate": (I, [P, P, I64, I, P, I, I, P]),
+        "ispa_absorb_workspace_size": (SZ, [I]),
+        "ispa_absorb_solve": (I, [P, P, I, F, P, P, P, P, SZ, P, P]),
+        "ispa_layer_error_workspace_size": (SZ, [I]),
+        "ispa_layer_error": (I, [P, P, P, P, P, I, P, P, SZ, P]),
+        "ispa_rank_layers": (I, [P, I, I, P, P, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def ispa_status_string(code: int) -> str:
+    return _load().ispa_status_string(int(code)).decode()
+
+
+def ispa_version() -> int:
+    return _load().ispa_version()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc: int, what: str):
+    if rc != ISPA_OK:
+        raise IspaError(rc, what)
+
+
+def _dev_tensor(t: torch.Tensor, dtype, name: str, ndim: Optional[int] = None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims")
+    return t
+
+
+def _kv(k: Optional[torch.Tensor], v: Optional[torch.Tensor], heads: int, hd: int, name: str):
+    if k is None or k.shape[0] == 0:
+        return IspaKV(None, None, 0)
+    _dev_tensor(k, torch.bfloat16, name + " keys", 3)
+    _dev_tensor(v, torch.bfloat16, name + " values", 3)
+    if tuple(k.shape[1:]) != (heads, hd) or k.shape != v.shape:
+        raise ValueError(f"{name}: keys/values must be [len, {heads}, {hd}]")
+    return IspaKV(k.data_ptr(), v.data_ptr(), k.shape[0])
+
+
+def new_status(device=None) -> torch.Tensor:
+    """A zeroed device status word for the calls that report device-side
+    conditions."""
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+def read_status(status: torch.Tensor) -> int:
+    """Synchronises and returns the device status bits."""
+    return int(status.item())
+
+
+def ispa_dual_attention_workspace_size(sink_len: int, local_len: int, hist_len: int, heads: int,
+                                       head_dim: int) -> int:
+    return _load().ispa_dual_attention_workspace_size(sink_len, local_len, hist_len, heads, head_dim)
+
+
+def ispa_dual_attention(q, k_sink, v_sink, k_loc, v_loc, k_hist=None, v_hist=None, scale=None,
+                        a_loc=None, d_out=None, want_a_full=True, want_lse=True,
+                        workspace=None, status=None, stream=None) -> dict:
+    """Dual-stream attention of one chunk. q, k_*, v_*: [n, heads, head_dim]
+    bf16 CUDA tensors. Returns a dict with a_loc and d ([nq, d] fp32), and,
+    on request, a_full ([nq, d] bf16), lse_loc/lse_hist/lse_full ([heads, nq]
+    fp32) and the status word."""
+    _dev_tensor(q, torch.bfloat16, "q", 3)
+    nq, heads, hd = q.shape
+    d = heads * hd
+    sink = _kv(k_sink, v_sink, heads, hd, "sink")
+    loc = _kv(k_loc, v_loc, heads, hd, "local")
+    hist = _kv(k_hist, v_hist, heads, hd, "history")
+    dev = q.device
+    if scale is None:
+        scale = hd ** -0.5
+    a_loc = torch.empty(nq, d, dtype=torch.float32, device=dev) if a_loc is None else a_loc
+    d_out = torch.empty(nq, d, dtype=torch.float32, device=dev) if d_out is None else d_out
+    a_full = torch.empty(nq, d, dtype=torch.bfloat16, device=dev) if want_a_full else None
+    lse = [torch.empty(heads, nq, dtype=torch.float32, device=dev) if want_lse else None
+           for _ in range(3)]
+    need = ispa_dual_attention_workspace_size(sink.len, loc.len, hist.len, heads, hd)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    status = new_status(dev) if status is None else status
+    rc = _load().ispa_dual_attention(
+        _ptr(q), nq, heads, hd, sink, loc, hist, float(scale), _ptr(a_loc), _ptr(d_out),
+        _ptr(a_full), _ptr(lse[0]), _ptr(lse[1]), _ptr(lse[2]), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream))
+    _check(rc, "ispa_dual_attention")
+    return {"a_loc": a_loc, "d": d_out, "a_full": a_full, "lse_loc": lse[0], "lse_hist": lse[1],
+            "lse_full": lse[2], "status": status}
+
+
+def ispa_local_attention(q, k_sink, v_sink, k_loc, v_loc, scale=None, out_dtype=torch.bfloat16,
+                         want_lse=False, workspace=None, status=None, stream=None) -> dict:
+    """Local (sink + current chunk) attention of an L-Layer. Returns a dict
+    with out ([nq, d] in out_dtype: bf16 or fp32), lse and the status word."""
+    _dev_tensor(q, torch.bfloat16, "q", 3)
+    nq, heads, hd = q.shape
+    sink = _kv(k_sink, v_sink, heads, hd, "sink")
+    loc = _kv(k_loc, v_loc, heads, hd, "local")
+    dev = q.device
+    if scale is None:
+        scale = hd ** -0.5
+    out = torch.empty(nq, heads * hd, dtype=out_dtype, device=dev)
+    lse = torch.empty(heads, nq, dtype=torch.float32, device=dev) if want_lse else None
+    need = ispa_dual_attention_workspace_size(sink.len, loc.len, 0, heads, hd)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    status = new_status(dev) if status is None else status
+    f32 = out if out_dtype == torch.float32 else None
+    b16 = out if out_dtype == torch.bfloat16 else None
+    if f32 is None and b16 is None:
+        raise TypeError("out_dtype must be torch.float32 or torch.bfloat16")
+    rc = _load().ispa_local_attention(
+        _ptr(q), nq, heads, hd, sink, loc, float(scale), _ptr(f32), _ptr(b16), _ptr(lse),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream(stream))
+    _check(rc, "ispa_local_attention")
+    return {"out": out, "lse": lse, "status": status}
+
+
+def ispa_gram_accumulate(a_loc, d, M=None, accumulate=False, want_s=True, stream=None):
+    """M[0:d,0:d] (G) (+)= A_loc^T A_loc, M[0:d,d:2d] (R) (+)= A_loc^T D,
+    M[d:2d,d:2d] (S) (+)= D^T D; M is [2d, 2d] fp32. Returns M."""
+    _dev_tensor(a_loc, torch.float32, "a_loc", 2)
+    _dev_tensor(d, torch.float32, "d", 2)
+    rows, dim = a_loc.shape
+    if d.shape != a_loc.shape:
+        raise ValueError("a_loc and d must have the same shape")
+    if M is None:
+        M = torch.empty(2 * dim, 2 * dim, dtype=torch.float32, device=a_loc.device)
+        accumulate = False
+    _dev_tensor(M, torch.float32, "M", 2)
+    rc = _load().ispa_gram_accumulate(_ptr(a_loc), _ptr(d), rows, dim, _ptr(M), int(bool(accumulate)),
+                                      int(bool(want_s)), _stream(stream))
+    _check(rc, "ispa_gram_accumulate")
+    return M
+
+
+def ispa_absorb_workspace_size(dim: int) -> int:
+    return _load().ispa_absorb_workspace_size(dim)
+
+
+def ispa_absorb_solve(M, W, lam: float = 0.0, workspace=None, status=None, stream=None) -> dict:
+    """Delta W solving (G + lambda I) Delta W = R W (lam <= 0: 1e-2 tr(G)/d).
+    Returns dW, B = R W, the lambda used (device float) and the status word."""
+    _dev_tensor(M, torch.float32, "M", 2)
+    _dev_tensor(W, torch.float32, "W", 2)
+    dim = W.shape[0]
+    if tuple(M.shape) != (2 * dim, 2 * dim) or W.shape[1] != dim:
+        raise ValueError("M must be [2d, 2d] and W [d, d]")
+    dev = W.device
+    dW = torch.empty(dim, dim, dtype=torch.float32, device=dev)
+    B = torch.empty(dim, dim, dtype=torch.float32, device=dev)
+    lam_out = torch.empty(1, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(ispa_absorb_workspace_size(dim), dtype=torch.uint8, device=dev)
+    status = new_status(dev) if status is None else status
+    rc = _load().ispa_absorb_solve(_ptr(M), _ptr(W), dim, float(lam), _ptr(dW), _ptr(B),
+                                   _ptr(lam_out), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _ptr(status),
+                                   _stream(stream))
+    _check(rc, "ispa_absorb_solve")
+    return {"dW": dW, "B": B, "lam": lam_out, "status": status}
+
+
+def ispa_layer_error_workspace_size(dim: int) -> int:
+    return _load().ispa_layer_error_workspace_size(dim)
+
+
+def ispa_layer_error(M, W, dW, B, lam, err=None, workspace=None, stream=None):
+    """Reconstruction error of one layer: device double[2] =
+    {||E||^2, ||E||^2 / ||A_full W||^2} (written into ``err`` if given)."""
+    for t, n in ((M, "M"), (W, "W"), (dW, "dW"), (B, "B"), (lam, "lam")):
+        _dev_tensor(t, torch.float32, n)
+    dim = W.shape[0]
+    dev = W.device
+    if err is None:
+        err = torch.empty(2, dtype=torch.float64, device=dev)
+    if workspace is None:
+        workspace = torch.empty(ispa_layer_error_workspace_size(dim), dtype=torch.uint8, device=dev)
+    rc = _load().ispa_layer_error(_ptr(M), _ptr(W), _ptr(dW), _ptr(B), _ptr(lam), dim, _ptr(err),
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _stream(stream))
+    _check(rc, "ispa_layer_error")
+    return err
+
+
+def ispa_rank_layers(err, K: int, stream=None):
+    """Stable ascending ranking of layers by relative error (err: device
+    double [n_layers, 2]). Returns (perm int32 [n], selected uint8 [n])."""
+    _dev_tensor(err, torch.float64, "err")
+    n = err.numel() // 2
+    perm = torch.empty(n, dtype=torch.int32, device=err.device)
+    sel = torch.empty(n, dtype=torch.uint8, device=err.device)
+    rc = _load().ispa_rank_layers(_ptr(err), n, int(K), _ptr(perm), _ptr(sel), _stream(stream))
+    _check(rc, "ispa_rank_layers")
+    return perm, sel

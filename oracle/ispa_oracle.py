@@ -37,7 +37,7 @@ def as_f64(x) -> np.ndarray:
 
 def _scores(q: np.ndarray, k: np.ndarray, scale: float) -> np.ndarray:
     """Per-head scaled scores [H, nq, nk] from q [nq, H, hd], k [nk, H, hd]."""
-    return np.einsum("qhc,khc->hqk", q, k) * scale
+    return np.matmul(q.transpose(1, 0, 2), k.transpose(1, 2, 0)) * scale
 
 
 def branch_attention(q, k, v, scale):
@@ -57,7 +57,7 @@ def branch_attention(q, k, v, scale):
     e = np.exp(s - m)
     z = e.sum(axis=2, keepdims=True)
     p = e / z
-    out = np.einsum("hqk,khc->qhc", p, v)
+    out = np.matmul(p, v.transpose(1, 0, 2)).transpose(1, 0, 2)   # [nq, H, hd]
     lse = (m + np.log(z))[:, :, 0]
     return out, lse
 

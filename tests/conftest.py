@@ -19,5 +19,8 @@ def lib():
     import torch
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
+    from kv_cache_absorption_b200 import build
+    build.build()
     from kv_cache_absorption_b200 import ispa
+    ispa._load()
     return ispa

@@ -1,0 +1,129 @@
+"""The C-ABI library: it builds, loads without a GPU, exports exactly what
+include/ispa.h declares, and rejects bad arguments on the host before any
+device work. CPU only."""
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ispa.h")
+
+
+@pytest.fixture(scope="module")
+def ispa():
+    from kv_cache_absorption_b200 import build
+    build.build()
+    from kv_cache_absorption_b200 import ispa as m
+    m._load()
+    return m
+
+
+def declared():
+    text = open(HEADER).read()
+    return set(re.findall(r"^ISPA_API [\w\s\*]+?\b(ispa_\w+)\(", text, flags=re.M))
+
+
+def exported():
+    out = subprocess.run(["nm", "-D", "--defined-only", os.path.join(
+        ROOT, "kv_cache_absorption_b200", "libispa.so")], capture_output=True, text=True).stdout
+    return {line.split()[-1] for line in out.splitlines() if " T " in line}
+
+
+def test_exports_match_header(ispa):
+    names = declared()
+    assert len(names) == 11
+    assert names == exported()
+    assert names == set(ispa.EXPORTED)
+    lib = ctypes.CDLL(ispa.LIB_PATH)
+    for n in names:
+        assert getattr(lib, n) is not None
+
+
+def test_version_and_status_strings(ispa):
+    assert ispa.ispa_version() == 100
+    for code in (0, -1, -2, -3, -4, -5, 1, 2, 4, 8):
+        assert ispa.ispa_status_string(code) != "unknown status"
+    assert ispa.ispa_status_string(12345) == "unknown status"
+
+
+def test_workspace_sizes(ispa):
+    def r256(x):
+        return (x + 255) // 256 * 256
+    d = 12 * 128
+    assert ispa.ispa_dual_attention_workspace_size(1560, 4680, 14040, 12, 128) == \
+        r256(1560 * d * 2) + r256(4680 * d * 2) + r256(14040 * d * 2) + 256
+    assert ispa.ispa_dual_attention_workspace_size(-1, 1, 1, 1, 64) == 0
+    n = 1536
+    assert ispa.ispa_absorb_workspace_size(n) >= 2 * n * n * 4
+    assert ispa.ispa_absorb_workspace_size(0) == 0
+    assert ispa.ispa_layer_error_workspace_size(128) >= 40
+
+
+def _kv(ispa, n, addr=0x10000):
+    return ispa.IspaKV(addr, addr, n)
+
+
+def _dual(ispa, q=0x1000, nq=64, heads=2, hd=64, sink=16, loc=64, hist=256, scale=0.125,
+          a_loc=0x2000, d_out=0x3000, ws=0x100000, ws_bytes=1 << 30, status=0x4000):
+    lib = ispa._load()
+    return lib.ispa_dual_attention(q, nq, heads, hd, _kv(ispa, sink), _kv(ispa, loc),
+                                   _kv(ispa, hist), scale, a_loc, d_out, None, None, None, None,
+                                   ws, ws_bytes, status, None)
+
+
+def test_dual_attention_host_checks(ispa):
+    assert _dual(ispa, q=0) == ispa.ISPA_ERR_ARG
+    assert _dual(ispa, a_loc=0) == ispa.ISPA_ERR_ARG
+    assert _dual(ispa, status=0) == ispa.ISPA_ERR_ARG
+    assert _dual(ispa, nq=-1) == ispa.ISPA_ERR_ARG
+    assert _dual(ispa, heads=0) == ispa.ISPA_ERR_ARG
+    assert _dual(ispa, hd=96) == ispa.ISPA_ERR_UNSUPPORTED
+    assert _dual(ispa, scale=0.0) == ispa.ISPA_ERR_ARG
+    assert _dual(ispa, scale=float("nan")) == ispa.ISPA_ERR_ARG
+    assert _dual(ispa, sink=0, loc=0) == ispa.ISPA_ERR_ARG
+    assert _dual(ispa, hist=-5) == ispa.ISPA_ERR_ARG
+    assert _dual(ispa, q=0x1004) == ispa.ISPA_ERR_UNSUPPORTED
+    assert _dual(ispa, ws=0) == ispa.ISPA_ERR_WORKSPACE
+    assert _dual(ispa, ws_bytes=100) == ispa.ISPA_ERR_WORKSPACE
+    assert _dual(ispa, ws=0x100010) == ispa.ISPA_ERR_WORKSPACE
+    # arguments that pass every host check then need an sm_100 device
+    import torch
+    rc = _dual(ispa)
+    if not torch.cuda.is_available():
+        assert rc in (ispa.ISPA_ERR_CUDA, ispa.ISPA_ERR_NO_DEVICE)
+
+
+def test_other_entry_points_host_checks(ispa):
+    lib = ispa._load()
+    P = 0x1000
+    assert lib.ispa_gram_accumulate(P, P, 100, 100, P, 0, 1, None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert lib.ispa_gram_accumulate(P, P, -1, 128, P, 0, 1, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_gram_accumulate(None, P, 10, 128, P, 0, 1, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_gram_accumulate(P, P, 10, 128, None, 0, 1, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_absorb_solve(P, P, 128, float("nan"), P, P, None, P, 1 << 30, P, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_absorb_solve(P, P, 100, 0.0, P, P, None, P, 1 << 30, P, None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert lib.ispa_absorb_solve(P, P, 128, 0.0, P, P, None, P, 16, P, None) == ispa.ISPA_ERR_WORKSPACE
+    assert lib.ispa_layer_error(P, P, P, P, None, 128, P, P, 256, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_layer_error(P, P, P, P, P, 128, P, P, 8, None) == ispa.ISPA_ERR_WORKSPACE
+    assert lib.ispa_rank_layers(P, 4, 5, P, None, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_rank_layers(P, 0, 0, P, None, None) == ispa.ISPA_ERR_ARG
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    code = ("import kv_cache_absorption_b200.ispa as m; m.LIB_PATH = '/nonexistent/libispa.so';\n"
+            "try:\n    m._load()\nexcept RuntimeError as e:\n    print('LOUD', e)\n")
+    out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True)
+    assert "LOUD" in out.stdout and "missing" in out.stdout
+
+
+def test_product_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "kv_cache_absorption_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in re.sub(r"#.*|//.*", "", text), f

@@ -1,0 +1,313 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle on
+the same seeded inputs.
+
+Tolerances (fixed for this path): attention outputs max-abs <= 2e-2 and
+relative Frobenius <= 5e-3 (bf16 inputs, fp32 accumulation); G and R
+relative Frobenius <= 1e-3; Delta W relative Frobenius <= 2e-3; identical
+layer ranking. LSEs: absolute <= 1e-3 (fp32 running max and sum with an
+approximate exp2 of relative error ~2^-22; derived bound far below this).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from ispa_synth import C0, C1, attention_like, gaussian, layer_streams, scaled
+
+pytestmark = pytest.mark.gpu
+
+ATT_MAXABS, ATT_RELFRO = 2e-2, 5e-3
+GR_RELFRO, DW_RELFRO = 1e-3, 2e-3
+LSE_ABS = 1e-3
+
+
+def rel_fro(got, ref):
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+def f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def check_attention(out, ref, tag=""):
+    for key, gkey in (("a_loc", "a_loc"), ("d", "d"), ("a_full", "a_full")):
+        got = f64(out[gkey])
+        r = ref[key]
+        if key == "d" and np.linalg.norm(r) == 0:
+            assert np.max(np.abs(got)) == 0.0, tag
+            continue
+        assert np.max(np.abs(got - r)) <= ATT_MAXABS, (tag, key)
+        tol = ATT_RELFRO
+        assert rel_fro(got, r) <= tol, (tag, key, rel_fro(got, r))
+    for key in ("lse_loc", "lse_hist", "lse_full"):
+        got, r = f64(out[key]), ref[key]
+        fin = np.isfinite(r)
+        assert np.array_equal(np.isfinite(got), fin), (tag, key)
+        assert np.array_equal(got[~fin], r[~fin]), (tag, key)
+        if fin.any():
+            assert np.max(np.abs(got[fin] - r[fin])) <= LSE_ABS, (tag, key)
+
+
+def to_dev(ch):
+    return {k: v.cuda() for k, v in ch.items()}
+
+
+def run_dual(lib, ch):
+    return lib.ispa_dual_attention(ch["q"], ch["k_sink"], ch["v_sink"], ch["k_loc"], ch["v_loc"],
+                                   ch.get("k_hist"), ch.get("v_hist"))
+
+
+def ref_dual(ch):
+    return oracle.dual_attention(ch["q"], ch["k_sink"], ch["v_sink"], ch["k_loc"], ch["v_loc"],
+                                 ch["k_hist"], ch["v_hist"])
+
+
+def random_chunk(nq, sink, loc, hist, H, hd, seed):
+    g = lambda n, i: gaussian((n, H, hd), seed + 17 * i, 0, "X").to(torch.bfloat16)
+    return {"q": g(nq, 0), "k_sink": g(sink, 1), "v_sink": g(sink, 2), "k_loc": g(loc, 3),
+            "v_loc": g(loc, 4), "k_hist": g(hist, 5), "v_hist": g(hist, 6)}
+
+
+# ---------------------------------------------------------------- attention
+
+def test_dual_attention_tiny_workload_all_chunks(lib):
+    st = layer_streams(C0, 0, seed=0)
+    for c in range(C0.n_chunks):
+        ch = st.chunk(c)
+        out = run_dual(lib, to_dev(ch))
+        torch.cuda.synchronize()
+        assert lib.read_status(out["status"]) == 0
+        check_attention(out, ref_dual(ch), f"chunk {c}")
+
+
+@pytest.mark.parametrize("nq,sink,loc,hist,H,hd", [
+    (200, 16, 100, 300, 3, 128),    # ragged everywhere, several tiles
+    (128, 128, 128, 128, 1, 64),    # exact tiles
+    (1, 1, 0, 0, 1, 64),            # single query, single key
+    (5, 0, 37, 0, 2, 128),          # no sink, no history
+    (300, 24, 0, 1000, 2, 64),      # no local keys, long history
+    (129, 7, 130, 257, 4, 128),     # one row / one key past a tile boundary
+])
+def test_dual_attention_shapes(lib, nq, sink, loc, hist, H, hd):
+    ch = random_chunk(nq, sink, loc, hist, H, hd, seed=nq + sink + hist)
+    out = run_dual(lib, to_dev(ch))
+    torch.cuda.synchronize()
+    assert lib.read_status(out["status"]) == 0
+    check_attention(out, ref_dual(ch), str((nq, sink, loc, hist, H, hd)))
+
+
+def test_empty_history_gives_zero_discrepancy(lib):
+    ch = random_chunk(70, 16, 64, 0, 2, 64, seed=3)
+    out = run_dual(lib, to_dev(ch))
+    torch.cuda.synchronize()
+    assert torch.all(out["d"] == 0)
+    assert torch.all(torch.isneginf(out["lse_hist"]))
+    assert torch.equal(out["lse_full"], out["lse_loc"])
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_local_attention(lib, dtype):
+    ch = random_chunk(150, 16, 140, 0, 2, 128, seed=11)
+    dc = to_dev(ch)
+    out = lib.ispa_local_attention(dc["q"], dc["k_sink"], dc["v_sink"], dc["k_loc"], dc["v_loc"],
+                                   out_dtype=dtype, want_lse=True)
+    torch.cuda.synchronize()
+    ref, lse = oracle.local_attention(ch["q"], ch["k_sink"], ch["v_sink"], ch["k_loc"], ch["v_loc"])
+    got = f64(out["out"])
+    assert np.max(np.abs(got - ref)) <= ATT_MAXABS
+    assert rel_fro(got, ref) <= ATT_RELFRO
+    assert np.max(np.abs(f64(out["lse"]) - lse)) <= LSE_ABS
+
+
+def test_dual_attention_full_size_sampled_rows(lib):
+    """1.3B single chunk at full size (Nq 4680, keys 1560 + 4680 + 14040,
+    12 heads x 128): every output row is produced by the launch the benchmark
+    times; 96 sampled rows are checked against the oracle."""
+    st = layer_streams(C1, 0, seed=0)
+    ch = st.chunk(0)
+    out = run_dual(lib, to_dev(ch))
+    torch.cuda.synchronize()
+    assert lib.read_status(out["status"]) == 0
+    rows = np.sort(np.random.default_rng(0).choice(C1.chunk_tokens, 96, replace=False))
+    rows = np.concatenate([rows, [0, 127, 128, 4679]])
+    sub = dict(ch)
+    sub["q"] = ch["q"][torch.from_numpy(rows)]
+    ref = ref_dual(sub)
+    got = {k: (v[torch.from_numpy(rows).cuda()] if k in ("a_loc", "d", "a_full") else
+               v[:, torch.from_numpy(rows).cuda()]) for k, v in out.items()
+           if k != "status"}
+    check_attention(got, ref, "full-size sample")
+
+
+# ---------------------------------------------------------------- Gram
+
+def upper_tile_mask(dim):
+    I = np.arange(dim)[:, None] // 128
+    J = np.arange(dim)[None, :] // 128
+    return I <= J
+
+
+@pytest.mark.parametrize("rows,dim", [(1000, 256), (777, 384), (64, 128)])
+def test_gram_accumulate_two_calls(lib, rows, dim):
+    a1 = attention_like(rows, dim, seed=1)
+    d1 = 0.3 * attention_like(rows, dim, seed=2)
+    a2 = attention_like(rows + 40, dim, seed=3)
+    d2 = 0.3 * attention_like(rows + 40, dim, seed=4)
+    M = lib.ispa_gram_accumulate(a1.cuda(), d1.cuda())
+    M = lib.ispa_gram_accumulate(a2.cuda(), d2.cuda(), M=M, accumulate=True)
+    torch.cuda.synchronize()
+    G, R, S = oracle.gram(np.concatenate([f64(a1), f64(a2)]), np.concatenate([f64(d1), f64(d2)]))
+    Mg = f64(M)
+    up = upper_tile_mask(dim)
+    assert rel_fro(Mg[:dim, :dim][up], G[up]) <= GR_RELFRO
+    assert rel_fro(Mg[:dim, dim:], R) <= GR_RELFRO
+    assert rel_fro(Mg[dim:, dim:][up], S[up]) <= GR_RELFRO
+
+
+def test_gram_overwrite_and_empty(lib):
+    dim = 256
+    a = attention_like(300, dim, seed=5).cuda()
+    M = torch.full((2 * dim, 2 * dim), 7.0, device="cuda")
+    lib.ispa_gram_accumulate(a[:0], a[:0], M=M, accumulate=False)
+    torch.cuda.synchronize()
+    assert torch.all(M[:dim] == 0) and torch.all(M[dim:, dim:] == 0)
+    assert torch.all(M[dim:, :dim] == 7.0)   # the unused block is not touched
+
+
+# ---------------------------------------------------------------- solve / error / rank
+
+def synthetic_layer(rows, dim, seed):
+    a = attention_like(rows, dim, seed=seed)
+    f = a + 0.4 * attention_like(rows, dim, seed=seed + 1, rho=0.5, common=0.1)
+    W = gaussian((dim, dim), seed, 0, "W") / math.sqrt(dim)
+    return f64(a), f64(f), W
+
+
+def pack_M(G, R, S):
+    d = G.shape[0]
+    M = np.zeros((2 * d, 2 * d), np.float32)
+    M[:d, :d], M[:d, d:], M[d:, d:] = G, R, S
+    return torch.from_numpy(M)
+
+
+@pytest.mark.parametrize("dim", [128, 256, 512])
+def test_absorb_solve_isolated(lib, dim):
+    a, f, W = synthetic_layer(4 * dim + 100, dim, seed=dim)
+    G, R, S = oracle.gram(a, f - a)
+    M = pack_M(G, R, S)
+    out = lib.ispa_absorb_solve(M.cuda(), W.cuda())
+    torch.cuda.synchronize()
+    assert lib.read_status(out["status"]) == 0
+    Gf, Rf = f64(M[:dim, :dim]), f64(M[:dim, dim:])
+    lam = oracle.default_lambda(Gf)
+    assert abs(out["lam"].item() - lam) <= 1e-6 * lam
+    dW, B = oracle.absorb(Gf, Rf, f64(W), lam)
+    assert rel_fro(f64(out["B"]), B) <= 1e-5
+    assert rel_fro(f64(out["dW"]), dW) <= DW_RELFRO
+
+
+def test_absorb_solve_explicit_lambda_and_not_spd(lib):
+    dim = 128
+    a, f, W = synthetic_layer(600, dim, seed=9)
+    G, R, S = oracle.gram(a, f - a)
+    M = pack_M(G, R, S)
+    out = lib.ispa_absorb_solve(M.cuda(), W.cuda(), lam=2.5)
+    torch.cuda.synchronize()
+    assert out["lam"].item() == 2.5
+    dW, _ = oracle.absorb(f64(M[:dim, :dim]), f64(M[:dim, dim:]), f64(W), 2.5)
+    assert rel_fro(f64(out["dW"]), dW) <= DW_RELFRO
+    # a negative ridge weight larger than the smallest eigenvalue of G
+    bad = lib.ispa_absorb_solve(M.cuda(), W.cuda(), lam=-1e6)
+    torch.cuda.synchronize()
+    assert bad["lam"].item() > 0  # lam <= 0 selects the default
+    M0 = torch.zeros_like(M)
+    bad = lib.ispa_absorb_solve(M0.cuda(), W.cuda())   # G = 0 and lambda = 0
+    torch.cuda.synchronize()
+    assert lib.read_status(bad["status"]) & lib.ISPA_STATUS_NOT_SPD
+
+
+@pytest.mark.parametrize("dim", [128, 384])
+def test_layer_error_isolated(lib, dim):
+    a, f, W = synthetic_layer(3 * dim + 50, dim, seed=dim + 1)
+    G, R, S = oracle.gram(a, f - a)
+    M = pack_M(G, R, S)
+    G32, R32 = f64(M[:dim, :dim]), f64(M[:dim, dim:])
+    lam = oracle.default_lambda(G32)
+    dW, B = oracle.absorb(G32, R32, f64(W), lam)
+    err = lib.ispa_layer_error(M.cuda(), W.cuda(), torch.from_numpy(dW).float().cuda(),
+                               torch.from_numpy(B).float().cuda(),
+                               torch.tensor([lam], dtype=torch.float32).cuda())
+    torch.cuda.synchronize()
+    e2, eps = oracle.reconstruction_error(a, f, f64(W), dW)
+    got = err.cpu().numpy()
+    assert abs(got[0] - e2) <= 2e-3 * e2
+    assert abs(got[1] - eps) <= 2e-3 * eps
+
+
+def test_rank_layers_bit_exact(lib):
+    r = np.random.default_rng(4)
+    eps = r.integers(0, 9, size=37) / 10.0
+    err = torch.from_numpy(np.stack([eps * 3, eps], 1)).cuda()
+    perm, sel = lib.ispa_rank_layers(err, 18)
+    torch.cuda.synchronize()
+    ref_perm, ref_sel = oracle.rank_layers(eps, 18)
+    assert perm.cpu().numpy().tolist() == ref_perm.tolist()
+    assert sel.cpu().numpy().astype(bool).tolist() == ref_sel.tolist()
+
+
+# ---------------------------------------------------------------- end to end
+
+def test_warmup_tiny_end_to_end(lib):
+    from kv_cache_absorption_b200.warmup import LayerWarmup, run_warmup
+    st = layer_streams(C0, 0, seed=0)
+    chunks = [st.chunk(c) for c in range(C0.n_chunks)]
+    ref = oracle.warmup_layer(chunks, st.w)
+    runner = LayerWarmup(C0.heads, C0.head_dim, C0.chunk_tokens, C0.sink_tokens,
+                         C0.chunk_tokens, 256)
+    err, perm, sel, dws = run_warmup([([to_dev(c) for c in chunks], st.w.cuda())], 1, runner,
+                                     keep_dw=True)
+    torch.cuda.synchronize()
+    assert lib.read_status(runner.status) == 0
+    d = C0.d
+    Mg = f64(runner.M)
+    up = upper_tile_mask(d)
+    assert rel_fro(Mg[:d, :d][up], ref["G"][up]) <= GR_RELFRO
+    assert rel_fro(Mg[:d, d:], ref["R"]) <= GR_RELFRO
+    assert rel_fro(f64(dws[0]), ref["dW"]) <= DW_RELFRO
+    assert abs(err[0, 1].item() - ref["eps"]) <= 5e-3 * ref["eps"]
+
+
+def test_warmup_multilayer_ranking(lib):
+    """Six layers of a reduced 1.3B geometry (frames of 64 tokens, 2 heads x
+    64, 4 chunks with a growing history); the per-layer AR(1) correlation is
+    spread so that the errors separate."""
+    from kv_cache_absorption_b200.warmup import LayerWarmup, run_warmup
+    L = 6
+    layers_dev, eps_ref = [], []
+    for l in range(L):
+        cfg = scaled(C0, tokens_per_frame=64, sink_tokens=64, chunk_frames=3, first_chunk_frame=1,
+                     n_chunks=4, history_window=None, rho=0.5 + 0.08 * l)
+        st = layer_streams(cfg, l, seed=1)
+        chunks = [st.chunk(c) for c in range(4)]
+        eps_ref.append(oracle.warmup_layer(chunks, st.w)["eps"])
+        layers_dev.append(([to_dev(c) for c in chunks], st.w.cuda()))
+    runner = LayerWarmup(2, 64, 192, 64, 192, 9 * 64)
+    err, perm, sel, _ = run_warmup(layers_dev, 3, runner)
+    torch.cuda.synchronize()
+    ref_perm, ref_sel = oracle.rank_layers(eps_ref, 3)
+    got_eps = err[:, 1].cpu().numpy()
+    assert np.max(np.abs(got_eps - eps_ref) / np.asarray(eps_ref)) <= 5e-3
+    assert perm.cpu().numpy().tolist() == ref_perm.tolist()
+    assert sel.cpu().numpy().astype(bool).tolist() == ref_sel.tolist()
+
+
+def test_fp16_range_flag(lib):
+    ch = random_chunk(32, 8, 32, 16, 1, 64, seed=5)
+    ch["v_hist"] = ch["v_hist"].clone()
+    ch["v_hist"][3, 0, 5] = 1.0e5
+    out = run_dual(lib, to_dev(ch))
+    torch.cuda.synchronize()
+    assert lib.read_status(out["status"]) & lib.ISPA_STATUS_FP16_RANGE
