@@ -45,7 +45,8 @@ struct alignas(1024) Smem {
   uint64_t kv_empty[NSTAGE];
   uint64_t s_full[2];
   uint64_t p_full[2];
-  uint64_t o_done;
+  uint64_t o_done[2];   // PV of tile j done -> o_done[j & 1]
+  uint64_t o_final;     // every MMA of the CTA done
   uint64_t drain;
   uint32_t taddr;
   int abort_flag;
@@ -93,7 +94,9 @@ dual_attention_kernel(const __grid_constant__ AttnParams p) {
     mbar_init(&s.q_full, 1);
     for (int i = 0; i < NSTAGE; ++i) { mbar_init(&s.kv_full[i], 1); mbar_init(&s.kv_empty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&s.s_full[i], 1); mbar_init(&s.p_full[i], 128); }
-    mbar_init(&s.o_done, 1);
+    mbar_init(&s.o_done[0], 1);
+    mbar_init(&s.o_done[1], 1);
+    mbar_init(&s.o_final, 1);
     mbar_init(&s.drain, 1);
     s.abort_flag = 0;
     fence_mbar_init();
@@ -168,8 +171,9 @@ dual_attention_kernel(const __grid_constant__ AttnParams p) {
                  (first && kk == 0) ? 0u : 1u);
         }
         tc_commit(&s.kv_empty[st]);
-        tc_commit(&s.o_done);
+        tc_commit(&s.o_done[j & 1]);
       }
+      if (ok) tc_commit(&s.o_final);
       if (!ok) {  // let issued MMAs finish before TMEM is freed
         tc_commit(&s.drain);
         drain_wait(&s.drain, 0, p.status);
@@ -218,7 +222,10 @@ dual_attention_kernel(const __grid_constant__ AttnParams p) {
         const bool need = m_new > m + kRescaleThreshold;
         if (__any_sync(0xffffffffu, need)) {
           // all PV products into this branch's O must have landed first
-          if (!mbar_wait(&s.o_done, (j - 1) & 1, p.status, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&s.o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const float alpha = need ? ex2(m - m_new) : 1.f;
           if (need) { l *= alpha; m = m_new; }
@@ -253,7 +260,7 @@ dual_attention_kernel(const __grid_constant__ AttnParams p) {
       mbar_arrive(&s.p_full[j & 1]);
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && n_tiles > 0 && mbar_wait(&s.o_done, (n_tiles - 1) & 1, p.status, abort_flag)) {
+    if (ok && n_tiles > 0 && mbar_wait(&s.o_final, 0, p.status, abort_flag)) {
       tc_fence_after();
       const bool has_hist = n_tiles > n_loc;
       if (!has_hist) { m_loc = m; l_loc = l; }
@@ -356,8 +363,11 @@ __global__ void v_to_half_kernel(const uint4* __restrict__ src, uint4* __restric
 
 }  // namespace
 
+// At least 120 KB so that one CTA holds an SM: each CTA allocates all 512
+// TMEM columns.
 size_t attention_smem_bytes(int head_dim) {
-  return (head_dim == 64 ? sizeof(Smem<64>) : sizeof(Smem<128>)) + 1024;
+  const size_t need = (head_dim == 64 ? sizeof(Smem<64>) : sizeof(Smem<128>)) + 1024;
+  return need < 120 * 1024 ? 120 * 1024 : need;
 }
 
 cudaError_t launch_v_to_half(const void* src, void* dst, int64_t n_elems, int* status,
