@@ -1,0 +1,502 @@
+#!/usr/bin/env python
+"""Benchmark of the ISPA warmup hot path on B200.
+
+One step = the whole hot path over one batch of synthetic input: dual-stream
+attention of every chunk, Gram accumulation of its rows, the closed-form
+Delta W solve, the reconstruction error of every layer and the layer ranking.
+Default workload: the 1.3B-class single-layer chunk (12 heads x 128, 4680
+queries, 1560 sink + 4680 local + 14040 history keys). ``--config c2`` /
+``c3`` run the 1.3B / 14B full warmups (30 / 40 layers, 4 chunks each).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). ``value`` is the step's algorithmic TFLOP
+(attention 4*Nq*Nk*d counted once, Gram 4*N*d^2, solve (1/3+4)*d^3, error
+d^3) divided by the device time of the step, summed over all ranks' work;
+attention TFLOP/s and absorb ms per layer are reported alongside.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "dual-stream attention TFLOP/s and absorb ms/layer at 1.3B/14B shapes, % roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dual_attention_1.3B_chunk_traffic.txt")
+L2_FLUSH_BYTES = 512 << 20
+
+
+# ---------------------------------------------------------------- work model
+
+def step_work(cfg):
+    """Algorithmic FLOPs of one step, split by stage."""
+    d = cfg.d
+    attn = 0.0
+    for c in range(cfg.n_chunks):
+        nk = cfg.sink_tokens + cfg.chunk_tokens + len(cfg.history_frames_of(c)) * cfg.tokens_per_frame
+        attn += 4.0 * cfg.chunk_tokens * nk * d
+    gram = 4.0 * cfg.warmup_rows * d * d
+    solve = (1.0 / 3.0 + 4.0) * d ** 3
+    err = float(d) ** 3
+    L = cfg.layers
+    return {"attention": attn * L, "gram": gram * L, "solve": solve * L, "error": err * L}
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p["bf16_tflops"], p["hbm_gbs"], "measured"
+    except Exception:
+        return 1590.0, 6650.0, "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for f in ("attention.cu", "sm100.cuh", "attention.h"):
+        with open(os.path.join(ROOT, "kv_cache_absorption_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_per_launch():
+    """DRAM bytes per attention launch from the committed ncu summary, or None
+    when the kernel source changed since the counters were taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            kv = dict(line.strip().split("=", 1) for line in f if "=" in line and not line.startswith("#"))
+        if kv.get("source_hash") != source_hash():
+            return None
+        return float(kv["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str, period_ms: int = 50):
+        self.bus_id = bus_id.lower()
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", str(period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        rows = []
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            if not parts[0].lower().endswith(self.bus_id[-12:]):
+                continue
+            try:
+                rows.append(parts)
+            except ValueError:
+                pass
+        if not rows:   # bus id not reported: use the only GPU in the list, if there is one
+            ids = {line.split(",")[0].strip() for line in out.splitlines() if line.count(",") >= 8}
+            if len(ids) == 1:
+                rows = [[p.strip() for p in line.split(",")] for line in out.splitlines()
+                        if line.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- oracle timing (host)
+
+_ORACLE_INPUTS = {}
+
+
+def oracle_timing(cfg, sample_rows: int, seed: int = 0):
+    """Times the float64 oracle on a bounded sample of one layer of ``cfg``:
+    dual attention of ``sample_rows`` query rows of the last chunk (all heads,
+    all keys), the Gram of those rows, the full-size closed-form solve and the
+    direct error on the sampled rows. Returns per-stage (flops, seconds)."""
+    import oracle
+    from ispa_synth import layer_streams
+    key = (cfg.name, seed)
+    if key not in _ORACLE_INPUTS:
+        st = layer_streams(cfg, 0, seed=seed)
+        _ORACLE_INPUTS[key] = (st.chunk(cfg.n_chunks - 1), st.w)
+    ch, w = _ORACLE_INPUTS[key]
+    sub = dict(ch)
+    sub["q"] = ch["q"][:sample_rows]
+    nk = ch["k_sink"].shape[0] + ch["k_loc"].shape[0] + ch["k_hist"].shape[0]
+    d = cfg.d
+    t0 = time.perf_counter()
+    o = oracle.dual_attention(sub["q"], sub["k_sink"], sub["v_sink"], sub["k_loc"], sub["v_loc"],
+                              sub["k_hist"], sub["v_hist"])
+    t1 = time.perf_counter()
+    G, R, S = oracle.gram(o["a_loc"], o["d"])
+    t2 = time.perf_counter()
+    W = oracle.as_f64(w)
+    t3 = time.perf_counter()
+    dW, B = oracle.absorb(G, R, W, oracle.default_lambda(G))   # full d x d solve
+    t4 = time.perf_counter()
+    oracle.reconstruction_error(o["a_loc"], o["a_full"], W, dW)
+    t5 = time.perf_counter()
+    return {
+        "attention": (4.0 * sample_rows * nk * d, t1 - t0),
+        "gram": (4.0 * sample_rows * d * d, t2 - t1),
+        "solve": ((1.0 / 3.0 + 4.0) * d ** 3, t4 - t3),
+        "error": (4.0 * sample_rows * d * d, t5 - t4),
+    }
+
+
+def cpu_cores():
+    try:
+        n = len(os.sched_getaffinity(0))
+    except Exception:
+        n = os.cpu_count() or 1
+    blas = None
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max((i.get("num_threads", 0) for i in threadpool_info()), default=None)
+    except Exception:
+        pass
+    return n, blas
+
+
+def oracle_throughput(cfg, budget_s: float):
+    """Oracle throughput on this workload mix, extrapolated stage by stage
+    from bounded samples: t_full = sum_s F_s * (t_s / f_s)."""
+    work = step_work(cfg)
+    rows = 4
+    timing = oracle_timing(cfg, rows)
+    spent = sum(t for _, t in timing.values())
+    while spent < budget_s * 0.5 and rows < 256:
+        rows *= 2
+        timing = oracle_timing(cfg, rows)
+        spent = sum(t for _, t in timing.values())
+    t_full = sum(work[s] * timing[s][1] / max(timing[s][0], 1.0) for s in work)
+    total = sum(work.values())
+    cores, blas = cpu_cores()
+    return {
+        "value": total / t_full / 1e12, "unit": "TFLOP/s", "cores": blas or cores,
+        "kind": "oracle",
+        "sample": (f"float64 oracle on {rows} query rows of one layer's last chunk (all heads, "
+                   f"all keys), their Gram and direct error, plus one full {cfg.d}x{cfg.d} "
+                   f"solve; per-stage rates extrapolated to the full step"),
+        "seconds": spent, "ms_per_full_step": t_full * 1e3,
+    }
+
+
+# ---------------------------------------------------------------- distributed
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- our arm
+
+def make_inputs(cfg, rank, device):
+    from ispa_synth import layer_streams
+    layers = []
+    for l in range(cfg.layers):
+        st = layer_streams(cfg, layer=l + 1000 * rank, seed=0, device=device)
+        chunks = [st.chunk(c) for c in range(cfg.n_chunks)]
+        layers.append((chunks, st.w))
+        del st
+    return layers
+
+
+def run_ours(args):
+    import torch
+    from kv_cache_absorption_b200 import build
+    build.build()
+    from kv_cache_absorption_b200 import ispa
+    from kv_cache_absorption_b200.warmup import LayerWarmup, rank as rank_layers
+    from ispa_synth import CONFIGS
+
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cfg = CONFIGS[args.config]
+    layers = make_inputs(cfg, rank, dev)
+    max_hist = max(len(cfg.history_frames_of(c)) for c in range(cfg.n_chunks)) * cfg.tokens_per_frame
+    runner = LayerWarmup(cfg.heads, cfg.head_dim, cfg.chunk_tokens, cfg.sink_tokens,
+                         cfg.chunk_tokens, max_hist, device=dev)
+    L = cfg.layers
+    K = cfg.select_k if cfg.select_k is not None else L // 2
+    err = torch.empty(L, 2, dtype=torch.float64, device=dev)
+    perm = torch.empty(L, dtype=torch.int32, device=dev)
+    sel = torch.empty(L, dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    E = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step(ev=None):
+        for li, (chunks, W) in enumerate(layers):
+            for c, ch in enumerate(chunks):
+                if ev: ev["a0"].append(E()); ev["a0"][-1].record()
+                runner.attention(ch)
+                if ev: ev["a1"].append(E()); ev["a1"][-1].record()
+                runner.gram(first=(c == 0))
+                if ev: ev["g1"].append(E()); ev["g1"][-1].record()
+            runner.solve(W)
+            runner.error(W, err[li])
+            if ev: ev["s1"].append(E()); ev["s1"][-1].record()
+        rank_layers(err, K, perm, sel)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ispa.read_status(runner.status) != 0:
+        raise RuntimeError(f"device status {ispa.read_status(runner.status)} after warmup")
+
+    bus = torch.cuda.get_device_properties(dev)
+    bus_id = f"{getattr(bus, 'pci_domain_id', 0):08x}:{getattr(bus, 'pci_bus_id', 0):02x}:" \
+             f"{getattr(bus, 'pci_device_id', 0):02x}.0"
+    ev = {"a0": [], "a1": [], "g1": [], "s1": []}
+    starts, ends = [], []
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(bus_id)
+    time.sleep(0.15)
+    launches0 = ispa.ispa_kernel_launches()
+    for _ in range(args.steps):
+        flush.zero_()                       # L2 flush between timed steps, outside the events
+        s, e = E(), E()
+        s.record()
+        step(ev)
+        e.record()
+        starts.append(s), ends.append(e)
+    torch.cuda.synchronize()
+    launches = ispa.ispa_kernel_launches() - launches0
+    clocks = sampler.stop()
+    barrier(world)
+
+    step_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    attn_ms = sum(a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"])) / args.steps
+    gram_ms = sum(a.elapsed_time(b) for a, b in zip(ev["a1"], ev["g1"])) / args.steps
+    solve_ms = 0.0
+    n_chunks = cfg.n_chunks
+    for li in range(len(ev["s1"])):
+        # solve + error of a layer: from the end of its last Gram to s1
+        solve_ms += ev["g1"][(li + 1) * n_chunks - 1].elapsed_time(ev["s1"][li])
+    solve_ms /= args.steps
+    step_ms_max = max_over_ranks(step_ms, world)
+
+    work = step_work(cfg)
+    total = sum(work.values())
+    value = total * world / (step_ms_max * 1e-3) / 1e12
+    attn_tflops = work["attention"] / (attn_ms * 1e-3) / 1e12
+    absorb_ms_layer = (gram_ms + solve_ms) / L
+    bf16_peak, hbm_peak, peak_src = peaks()
+    attn_launches = L * cfg.n_chunks
+    roofline = {
+        "bound": "tensor", "kernel": "dual-stream attention (V fp16 pre-pass + attention kernel)",
+        "achieved": round(attn_tflops, 2), "peak": bf16_peak, "unit": "TFLOP/s",
+        "frac": round(attn_tflops / bf16_peak, 4), "peak_source": f"{peak_src} bf16 dense (burst)",
+        "traffic": traffic_per_launch(),
+        "algorithmic_flops_per_launch": work["attention"] / attn_launches,
+        "ms_per_launch": attn_ms / attn_launches,
+    }
+    absorb_flops = work["gram"] + work["solve"] + work["error"]
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 QK^T, fp16 PV, tf32 Gram, fp32 solve",
+        "data": "synthetic AR(1) rho=0.9 bf16 Q/K/V, W ~ N(0,1/d), seeded",
+        "config": {"workload": cfg.name, "layers": L, "heads": cfg.heads, "head_dim": cfg.head_dim,
+                   "d": cfg.d, "chunks": cfg.n_chunks, "chunk_rows": cfg.chunk_tokens,
+                   "sink": cfg.sink_tokens,
+                   "history": [len(cfg.history_frames_of(c)) * cfg.tokens_per_frame
+                               for c in range(cfg.n_chunks)],
+                   "select_k": K, "l2": "flushed (512 MB write) before every timed step",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "attention_tflops": round(attn_tflops, 2),
+        "attention_ms_per_step": round(attn_ms, 4),
+        "absorb_ms_per_layer": round(absorb_ms_layer, 4),
+        "gram_ms_per_step": round(gram_ms, 4), "solve_error_ms_per_step": round(solve_ms, 4),
+        "absorb_tflops": round(absorb_flops / ((gram_ms + solve_ms) * 1e-3) / 1e12, 2),
+        "roofline": roofline,
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if not args.no_e2e:
+        out["e2e"] = run_e2e(args, cfg, layers, runner, err, perm, sel, K, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = oracle_throughput(cfg, args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(args, cfg, layers, runner, err, perm, sel, K, world):
+    """Same step through the public API with the inputs in pinned host
+    memory: host->device copies of every chunk's Q/K/V and each W, the step,
+    and device->host copies of every Delta W, the errors and the ranking, all
+    inside the timed region."""
+    import torch
+    from kv_cache_absorption_b200.warmup import rank as rank_layers
+    host_layers = [([{k: v.cpu().pin_memory() for k, v in ch.items()} for ch in chunks],
+                    W.cpu().pin_memory()) for chunks, W in layers]
+    dev_layers = layers
+    L = cfg.layers
+    d = cfg.d
+    dW_host = torch.empty(L, d, d, dtype=torch.float32).pin_memory()
+    err_host = torch.empty(L, 2, dtype=torch.float64).pin_memory()
+    perm_host = torch.empty(L, dtype=torch.int32).pin_memory()
+    h2d = sum(W.numel() * 4 + sum(x.numel() * x.element_size() for ch in chunks for x in ch.values())
+              for chunks, W in host_layers)
+    d2h = dW_host.numel() * 4 + err_host.numel() * 8 + perm_host.numel() * 4
+
+    def step():
+        for li, ((hchunks, hW), (dchunks, dW_)) in enumerate(zip(host_layers, dev_layers)):
+            dW_.copy_(hW, non_blocking=True)
+            for c, (hc, dc) in enumerate(zip(hchunks, dchunks)):
+                for k in hc:
+                    dc[k].copy_(hc[k], non_blocking=True)
+                runner.attention(dc)
+                runner.gram(first=(c == 0))
+            runner.solve(dW_)
+            runner.error(dW_, err[li])
+            dW_host[li].copy_(runner.dW, non_blocking=True)
+        rank_layers(err, K, perm, sel)
+        err_host.copy_(err, non_blocking=True)
+        perm_host.copy_(perm, non_blocking=True)
+
+    n = max(3, min(args.steps, 30))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(n):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s.elapsed_time(e) / n, world)
+    total = sum(step_work(cfg).values())
+    return {"value": round(total * world / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 4), "steps": n, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h)}
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The float64 oracle on the host cores: each step times one bounded
+    sample of the workload; the reported rate is the stage-weighted
+    extrapolation to the full step."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from ispa_synth import CONFIGS
+    cfg = CONFIGS[args.config]
+    work = step_work(cfg)
+    total = sum(work.values())
+    rows = 2
+    acc = {s: [0.0, 0.0] for s in work}
+    for i in range(args.warmup + args.steps):
+        timing = oracle_timing(cfg, rows)
+        if i >= args.warmup:
+            for s in acc:
+                acc[s][0] += timing[s][0]
+                acc[s][1] += timing[s][1]
+    t_full = sum(work[s] * acc[s][1] / acc[s][0] for s in work) / 1.0
+    t_full_step = t_full  # seconds per full step at the sampled rates
+    value = total / t_full_step / 1e12
+    cores, blas = cpu_cores()
+    sample = (f"per step: float64 oracle on {rows} query rows of the last chunk (all heads, all "
+              f"keys), their Gram and direct error, one full {cfg.d}x{cfg.d} solve; rates "
+              f"extrapolated stage by stage to the full step")
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": t_full_step * 1e3, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": cfg.name, "d": cfg.d, "layers": cfg.layers},
+           "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas or cores,
+                            "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--config", choices=("c1", "c2", "c3"), default="c1")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

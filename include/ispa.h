@@ -71,6 +71,11 @@ ISPA_API const char* ispa_status_string(int code);
 /* Library version as major*10000 + minor*100 + patch. */
 ISPA_API int ispa_version(void);
 
+/* Number of CUDA kernels this library has launched in this process so far
+ * (all devices and threads; memsets and copies not included). For
+ * instrumentation: the difference across a region counts its launches. */
+ISPA_API uint64_t ispa_kernel_launches(void);
+
 /* ---- 1. dual-stream attention ----------------------------------------
  * Technical summary section 2, step 1 ("Dual-Stream Warmup", decomposable
  * attention): for every query row and head, softmax(q k^T * scale) v over

@@ -1,6 +1,7 @@
 // C ABI of the ISPA warmup hot path: argument checks, TMA descriptor
 // encoding, workspace carving and kernel launches. Declarations and the
 // contract of every entry point are in include/ispa.h.
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -9,6 +10,8 @@
 #include "attention.h"
 
 namespace ispa {
+static std::atomic<unsigned long long> g_launches{0};
+void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 size_t absorb_workspace_bytes(int dim);
 cudaError_t absorb_solve(const float* M, const float* W, int dim, float lambda, float* dW,
                          float* B, float* lambda_out, void* workspace, int* status,
@@ -166,6 +169,8 @@ const char* ispa_status_string(int code) {
 }
 
 int ispa_version(void) { return 100; }
+
+uint64_t ispa_kernel_launches(void) { return ispa::g_launches.load(std::memory_order_relaxed); }
 
 size_t ispa_dual_attention_workspace_size(int64_t sink_len, int64_t local_len, int64_t hist_len,
                                           int heads, int head_dim) {

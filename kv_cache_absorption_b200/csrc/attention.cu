@@ -378,6 +378,7 @@ cudaError_t launch_v_to_half(const void* src, void* dst, int64_t n_elems, int* s
   if (blocks > 148 * 8) blocks = 148 * 8;
   v_to_half_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4*>(src),
                                                static_cast<uint4*>(dst), n8, status);
+  count_launches();
   return cudaGetLastError();
 }
 
@@ -393,6 +394,7 @@ cudaError_t launch_dual_attention(const AttnParams& p, int head_dim, cudaStream_
                          (int)smem);
     dual_attention_kernel<128><<<grid, kThreads, smem, stream>>>(p);
   }
+  count_launches();
   return cudaGetLastError();
 }
 

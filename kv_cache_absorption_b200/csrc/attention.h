@@ -8,6 +8,9 @@
 
 namespace ispa {
 
+// Kernel launches made by the library (read by ispa_kernel_launches).
+void count_launches(unsigned n = 1);
+
 // Parameters of one dual-stream attention launch. Tensor maps address
 // [len, heads * head_dim] row-major matrices in 64-column x 128-row boxes
 // with 128-byte swizzle: Q and K in bf16, V in fp16 (converted copies).

@@ -126,12 +126,14 @@ cudaError_t layer_error(const float* M, const float* W, const float* dW, const f
   dot_kernel<<<148 * 2, 256, 0, stream>>>(reinterpret_cast<const float4*>(dW),
                                           reinterpret_cast<const float4*>(B), n4, acc);
   finalize_kernel<<<1, 1, 0, stream>>>(acc, lam, err);
+  count_launches(3);
   return cudaGetLastError();
 }
 
 cudaError_t rank_layers(const double* err, int n, int K, int* perm, uint8_t* selected,
                         cudaStream_t stream) {
   rank_kernel<<<1, 256, 0, stream>>>(err, n, K, perm, selected);
+  count_launches();
   return cudaGetLastError();
 }
 

@@ -231,6 +231,7 @@ cudaError_t launch_gram(const GramParams& p, int bn, int grid, cudaStream_t stre
     cudaFuncSetAttribute(gram_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     gram_kernel<128><<<grid, kThreads, smem, stream>>>(p);
   }
+  count_launches();
   return cudaGetLastError();
 }
 

@@ -144,6 +144,7 @@ cudaError_t launch_sgemm(bool ta, bool tb, int M, int N, int K, float alpha, con
   else if (!ta && tb) sgemm_kernel<false, true><<<grid, kGemmThreads, 0, stream>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, lo);
   else if (ta && !tb) sgemm_kernel<true, false><<<grid, kGemmThreads, 0, stream>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, lo);
   else sgemm_kernel<true, true><<<grid, kGemmThreads, 0, stream>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, lo);
+  count_launches();
   return cudaGetLastError();
 }
 
@@ -168,6 +169,7 @@ cudaError_t absorb_solve(const float* M, const float* W, int dim, float lambda, 
 
   lambda_kernel<<<1, 256, 0, stream>>>(M, dim, lambda, lam, lambda_out);
   build_shifted_kernel<<<148 * 4, 256, 0, stream>>>(M, dim, lam, A);
+  count_launches(2);
   // B = R W, R = M[0:d, d:2d]
   if ((e = launch_sgemm(false, false, dim, dim, dim, 1.f, M + d, 2 * dim, W, dim, 0.f, B, dim,
                         false, stream)) != cudaSuccess)
@@ -177,6 +179,7 @@ cudaError_t absorb_solve(const float* M, const float* W, int dim, float lambda, 
     const size_t kk = (size_t)k * NB;
     potrf_block_kernel<<<1, 256, 0, stream>>>(A + kk * d + kk, dim, L + kk * d + kk, dim,
                                               Linv + (size_t)k * NB * NB, status);
+    count_launches();
     const int m = dim - (int)kk - NB;
     if (m <= 0) continue;
     // L21 = A21 Linv^T

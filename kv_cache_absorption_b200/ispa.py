@@ -29,7 +29,7 @@ ISPA_STATUS_NOT_SPD = 4
 ISPA_STATUS_NONFINITE = 8
 
 EXPORTED = (
-    "ispa_status_string", "ispa_version",
+    "ispa_status_string", "ispa_version", "ispa_kernel_launches",
     "ispa_dual_attention_workspace_size", "ispa_dual_attention", "ispa_local_attention",
     "ispa_gram_accumulate", "ispa_absorb_workspace_size", "ispa_absorb_solve",
     "ispa_layer_error_workspace_size", "ispa_layer_error", "ispa_rank_layers",
@@ -62,6 +62,7 @@ def _load():
     sig = {
         "ispa_status_string": (ctypes.c_char_p, [I]),
         "ispa_version": (I, []),
+        "ispa_kernel_launches": (ctypes.c_uint64, []),
         "ispa_dual_attention_workspace_size": (SZ, [I64, I64, I64, I, I]),
         "ispa_dual_attention": (I, [P, I64, I, I, IspaKV, IspaKV, IspaKV, F, P, P, P, P, P, P,
                                     P, SZ, P, P]),
@@ -87,6 +88,11 @@ def ispa_status_string(code: int) -> str:
 
 def ispa_version() -> int:
     return _load().ispa_version()
+
+
+def ispa_kernel_launches() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(_load().ispa_kernel_launches())
 
 
 def _ptr(t: Optional[torch.Tensor]):

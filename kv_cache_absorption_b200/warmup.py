@@ -8,7 +8,8 @@ layer's Delta W is solved, every layer's reconstruction error is formed and
 the layers are ranked; the K lowest-error layers become L-Layers.
 
 Orchestration only: buffers and workspaces are allocated once (through
-torch) and every step is a call into the C ABI.
+torch) and every step is a call into the C ABI, so a warmup issues no
+allocation and no host synchronisation.
 """
 from __future__ import annotations
 
@@ -41,41 +42,60 @@ class LayerWarmup:
         self.dW = torch.empty(d, d, **f32)
         self.B = torch.empty(d, d, **f32)
         self.lam = torch.empty(1, **f32)
+        self._rows = 0
 
-    # -- stage 1: one chunk of dual-stream attention, folded into G, R, S
-    def chunk(self, ch: dict, first: bool, stream=None):
-        lib = ispa._load()
+    def attention(self, ch: dict, stream=None):
+        """Dual-stream attention of one chunk into a_loc, d_out, a_full, LSEs."""
         q = ch["q"]
-        nq = q.shape[0]
+        self._rows = nq = q.shape[0]
         kv = [ispa._kv(ch["k_sink"], ch["v_sink"], self.heads, self.head_dim, "sink"),
               ispa._kv(ch["k_loc"], ch["v_loc"], self.heads, self.head_dim, "local"),
               ispa._kv(ch.get("k_hist"), ch.get("v_hist"), self.heads, self.head_dim, "history")]
-        st = ispa._stream(stream)
-        rc = lib.ispa_dual_attention(
+        rc = ispa._load().ispa_dual_attention(
             ispa._ptr(q), nq, self.heads, self.head_dim, kv[0], kv[1], kv[2],
             float(self.head_dim ** -0.5), ispa._ptr(self.a_loc), ispa._ptr(self.d_out),
             ispa._ptr(self.a_full), ispa._ptr(self.lse[0]), ispa._ptr(self.lse[1]),
             ispa._ptr(self.lse[2]), ispa._ptr(self.attn_ws), self.attn_ws.numel(),
-            ispa._ptr(self.status), st)
+            ispa._ptr(self.status), ispa._stream(stream))
         ispa._check(rc, "ispa_dual_attention")
-        rc = lib.ispa_gram_accumulate(ispa._ptr(self.a_loc), ispa._ptr(self.d_out), nq, self.d,
-                                      ispa._ptr(self.M), 0 if first else 1, 1, st)
+
+    def gram(self, first: bool, stream=None):
+        """Fold the last chunk's rows into G, R, S (first chunk overwrites)."""
+        rc = ispa._load().ispa_gram_accumulate(
+            ispa._ptr(self.a_loc), ispa._ptr(self.d_out), self._rows, self.d, ispa._ptr(self.M),
+            0 if first else 1, 1, ispa._stream(stream))
         ispa._check(rc, "ispa_gram_accumulate")
 
-    # -- stages 2-3: Delta W, then the layer's reconstruction error
-    def absorb(self, W: torch.Tensor, err_slot: torch.Tensor, lam: float = 0.0, stream=None):
-        lib = ispa._load()
-        st = ispa._stream(stream)
-        rc = lib.ispa_absorb_solve(ispa._ptr(self.M), ispa._ptr(W), self.d, float(lam),
-                                   ispa._ptr(self.dW), ispa._ptr(self.B), ispa._ptr(self.lam),
-                                   ispa._ptr(self.solve_ws), self.solve_ws.numel(),
-                                   ispa._ptr(self.status), st)
+    def chunk(self, ch: dict, first: bool, stream=None):
+        self.attention(ch, stream)
+        self.gram(first, stream)
+
+    def solve(self, W: torch.Tensor, lam: float = 0.0, stream=None):
+        """Delta W of the layer (and B = R W, lambda)."""
+        rc = ispa._load().ispa_absorb_solve(
+            ispa._ptr(self.M), ispa._ptr(W), self.d, float(lam), ispa._ptr(self.dW),
+            ispa._ptr(self.B), ispa._ptr(self.lam), ispa._ptr(self.solve_ws),
+            self.solve_ws.numel(), ispa._ptr(self.status), ispa._stream(stream))
         ispa._check(rc, "ispa_absorb_solve")
-        rc = lib.ispa_layer_error(ispa._ptr(self.M), ispa._ptr(W), ispa._ptr(self.dW),
-                                  ispa._ptr(self.B), ispa._ptr(self.lam), self.d,
-                                  ispa._ptr(err_slot), ispa._ptr(self.err_ws),
-                                  self.err_ws.numel(), st)
+
+    def error(self, W: torch.Tensor, err_slot: torch.Tensor, stream=None):
+        """The layer's {||E||^2, relative error} into err_slot (device double[2])."""
+        rc = ispa._load().ispa_layer_error(
+            ispa._ptr(self.M), ispa._ptr(W), ispa._ptr(self.dW), ispa._ptr(self.B),
+            ispa._ptr(self.lam), self.d, ispa._ptr(err_slot), ispa._ptr(self.err_ws),
+            self.err_ws.numel(), ispa._stream(stream))
         ispa._check(rc, "ispa_layer_error")
+
+    def absorb(self, W: torch.Tensor, err_slot: torch.Tensor, lam: float = 0.0, stream=None):
+        self.solve(W, lam, stream)
+        self.error(W, err_slot, stream)
+
+
+def rank(err: torch.Tensor, K: int, perm: torch.Tensor, selected: torch.Tensor, stream=None):
+    """Stable ascending ranking of err [L, 2] (relative error in column 1)."""
+    rc = ispa._load().ispa_rank_layers(ispa._ptr(err), err.shape[0], int(K), ispa._ptr(perm),
+                                       ispa._ptr(selected), ispa._stream(stream))
+    ispa._check(rc, "ispa_rank_layers")
 
 
 def run_warmup(layers, K: int, runner: LayerWarmup, keep_dw: bool = False, stream=None):
@@ -84,6 +104,8 @@ def run_warmup(layers, K: int, runner: LayerWarmup, keep_dw: bool = False, strea
     list of Delta W if keep_dw)."""
     n = len(layers)
     err = torch.empty(n, 2, dtype=torch.float64, device=runner.device)
+    perm = torch.empty(n, dtype=torch.int32, device=runner.device)
+    sel = torch.empty(n, dtype=torch.uint8, device=runner.device)
     dws = []
     for li, (chunks, W) in enumerate(layers):
         for c, ch in enumerate(chunks):
@@ -91,5 +113,5 @@ def run_warmup(layers, K: int, runner: LayerWarmup, keep_dw: bool = False, strea
         runner.absorb(W, err[li], stream=stream)
         if keep_dw:
             dws.append(runner.dW.clone())
-    perm, sel = ispa.ispa_rank_layers(err, K, stream=stream)
+    rank(err, K, perm, sel, stream)
     return err, perm, sel, dws

@@ -35,7 +35,7 @@ def exported():
 
 def test_exports_match_header(ispa):
     names = declared()
-    assert len(names) == 11
+    assert len(names) == 12
     assert names == exported()
     assert names == set(ispa.EXPORTED)
     lib = ctypes.CDLL(ispa.LIB_PATH)
@@ -45,6 +45,7 @@ def test_exports_match_header(ispa):
 
 def test_version_and_status_strings(ispa):
     assert ispa.ispa_version() == 100
+    assert ispa.ispa_kernel_launches() == 0   # nothing launched in a CPU-only process
     for code in (0, -1, -2, -3, -4, -5, 1, 2, 4, 8):
         assert ispa.ispa_status_string(code) != "unknown status"
     assert ispa.ispa_status_string(12345) == "unknown status"
