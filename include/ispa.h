@@ -79,13 +79,14 @@ ISPA_API uint64_t ispa_kernel_launches(void);
 /* ---- 1. dual-stream attention ----------------------------------------
  * Technical summary section 2, step 1 ("Dual-Stream Warmup", decomposable
  * attention): for every query row and head, softmax(q k^T * scale) v over
- * the local branch (sink then local keys) gives A_loc and LSE_loc; the same
- * pass continues over the history keys as a second online-softmax branch
- * (A_hist, LSE_hist); the two are merged by their log-sum-exp into A_full:
+ * the local branch (sink then local keys) gives A_loc and LSE_loc; the
+ * history keys form a second online-softmax branch (A_hist, LSE_hist); each
+ * key is visited once. The branches are merged by their log-sum-exp:
  *   LSE_full = log(exp(LSE_loc) + exp(LSE_hist)),
  *   A_full   = e^(LSE_loc-LSE_full) A_loc + e^(LSE_hist-LSE_full) A_hist.
- * D = A_full - A_loc is formed in fp32 from the two branch outputs, never
- * as the difference of two rounded outputs.
+ * D = A_full - A_loc = e^(LSE_hist-LSE_full) (A_hist - A_loc) is formed in
+ * fp32 from the branch outputs, never as the difference of two rounded
+ * outputs.
  *
  * q        [nq, heads, head_dim] bf16.
  * sink, local, hist: the three key/value branches. sink.len + local.len
@@ -99,14 +100,15 @@ ISPA_API uint64_t ispa_kernel_launches(void);
  * lse_loc, lse_hist, lse_full: out [heads, nq] fp32, natural log, optional.
  * workspace: device scratch of >= ispa_dual_attention_workspace_size()
  *          bytes, 256-byte aligned; holds V converted to fp16 (the P.V
- *          product runs with fp16 P and fp16 V). Its contents are
- *          overwritten; it must not be used by another call in flight.
+ *          product runs with fp16 P and fp16 V), the history branch's
+ *          output and both branches' LSEs. Its contents are overwritten; it
+ *          must not be used by another call in flight.
  * dev_status: device int; ISPA_STATUS_FP16_RANGE if a V value overflowed
  *          fp16, ISPA_STATUS_TIMEOUT if a kernel wait gave up.
  * Returns ISPA_OK or an ISPA_ERR_* code (nothing is launched on error).
  */
-ISPA_API size_t ispa_dual_attention_workspace_size(int64_t sink_len, int64_t local_len, int64_t hist_len,
-                                          int heads, int head_dim);
+ISPA_API size_t ispa_dual_attention_workspace_size(int64_t nq, int64_t sink_len, int64_t local_len,
+                                                   int64_t hist_len, int heads, int head_dim);
 ISPA_API int ispa_dual_attention(const void* q, int64_t nq, int heads, int head_dim, ispa_kv sink,
                         ispa_kv local, ispa_kv hist, float scale, float* a_loc, float* d_out,
                         void* a_full, float* lse_loc, float* lse_hist, float* lse_full,

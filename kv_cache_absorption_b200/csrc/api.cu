@@ -103,7 +103,7 @@ int attention_common(const void* q, int64_t nq, int heads, int head_dim, const i
       (a_full && !aligned16(a_full)))
     return ISPA_ERR_UNSUPPORTED;
   const int d = heads * head_dim;
-  const size_t need = ispa_dual_attention_workspace_size(br[0].len, br[1].len, br[2].len, heads,
+  const size_t need = ispa_dual_attention_workspace_size(nq, br[0].len, br[1].len, br[2].len, heads,
                                                          head_dim);
   if (!workspace || workspace_bytes < need || !aligned256(workspace)) return ISPA_ERR_WORKSPACE;
   int rc = check_device();
@@ -134,8 +134,16 @@ int attention_common(const void* q, int64_t nq, int heads, int head_dim, const i
                    CU_TENSOR_MAP_SWIZZLE_128B))
       return ISPA_ERR_CUDA;
   }
+  if (br[2].len > 0) {
+    p.hist_out = reinterpret_cast<float*>(ws);
+    ws += round256((size_t)nq * d * 4);
+  }
+  p.lse_loc_ws = reinterpret_cast<float*>(ws);
+  ws += round256((size_t)heads * nq * 4);
+  p.lse_hist_ws = reinterpret_cast<float*>(ws);
   p.nq = (int)nq;
   p.heads = heads;
+  p.n_pairs = ispa::attention_pairs(nq);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.round_tf32 = round_tf32;
   p.a_loc = a_loc;
@@ -172,11 +180,14 @@ int ispa_version(void) { return 100; }
 
 uint64_t ispa_kernel_launches(void) { return ispa::g_launches.load(std::memory_order_relaxed); }
 
-size_t ispa_dual_attention_workspace_size(int64_t sink_len, int64_t local_len, int64_t hist_len,
-                                          int heads, int head_dim) {
-  if (sink_len < 0 || local_len < 0 || hist_len < 0 || heads < 1 || head_dim < 1) return 0;
+size_t ispa_dual_attention_workspace_size(int64_t nq, int64_t sink_len, int64_t local_len,
+                                          int64_t hist_len, int heads, int head_dim) {
+  if (nq < 0 || sink_len < 0 || local_len < 0 || hist_len < 0 || heads < 1 || head_dim < 1) return 0;
   const int d = heads * head_dim;
-  return v_half_bytes(sink_len, d) + v_half_bytes(local_len, d) + v_half_bytes(hist_len, d) + 256;
+  const size_t lse = round256((size_t)heads * nq * 4);
+  const size_t hist_out = hist_len > 0 ? round256((size_t)nq * d * 4) : 0;
+  return v_half_bytes(sink_len, d) + v_half_bytes(local_len, d) + v_half_bytes(hist_len, d) +
+         hist_out + 2 * lse + 256;
 }
 
 int ispa_dual_attention(const void* q, int64_t nq, int heads, int head_dim, ispa_kv sink,

@@ -2,55 +2,90 @@
 //
 // "Towards Memory-Efficient Autoregressive Video Generation via
 // Instance-Specific Parametric Absorption", technical summary section 2,
-// step 1 (Dual-Stream Warmup, decomposable attention grounded in online
-// softmax): one pass over the keys yields the local output A_loc (sink +
-// current chunk) and, continuing over the history keys as a second branch,
-// the full output A_full by a post-hoc log-sum-exp merge.
+// step 1 (Dual-Stream Warmup): A_loc attends to sink + current chunk, A_full
+// also to the history. The pages obtain both without a second attention pass
+// by splitting the keys into a local and a history branch, each run as an
+// online softmax that keeps its log-sum-exp, and merging the branches post hoc.
 //
-// One CTA owns one head and 128 query rows. Warp roles:
-//   warp 0     TMA producer: Q once, then K/V tiles of 128 keys into a
-//              2-stage ring (K bf16, V fp16 from the conversion pre-pass).
-//   warp 1     owns the TMEM allocation; one lane issues every tcgen05.mma:
-//              S = Q K^T (bf16, SS form) into one of two S buffers, and
-//              O_b += P V (fp16, TS form: P read from TMEM where the softmax
-//              wrote it over S) into O_loc or O_hist.
-//   warps 2-5  softmax warpgroup, one thread per query row (TMEM lane):
-//              online softmax in base 2 with a lazily rescaled running max,
-//              P as fp16 back into TMEM, and the epilogue that merges the
-//              two branches and writes A_loc, D, A_full and the LSEs.
-// TMEM columns: S0 [0,128), S1 [128,256), O_loc [256,256+HD),
-// O_hist [256+HD, 256+2HD); 512 columns are allocated.
+// That decomposition is also the work split here. A unit is one branch of
+// one head for a pair of 128-row query tiles; history units (the longer ones)
+// are scheduled first, local units fill in behind them, and a separate
+// element-wise kernel applies the LSE merge:
+//   LSE_full = log(e^LSE_loc + e^LSE_hist), w = e^(LSE_hist - LSE_full),
+//   D = w (A_hist - A_loc), A_full = A_loc + D.
+//
+// Unit CTA (384 threads), both query tiles t = 0, 1 share every K/V tile:
+//   warp 0      TMA producer: the two Q tiles, then 128-key tiles into a
+//               3-stage K ring (bf16) and a 2-stage V ring (fp16 copies).
+//               K(j) is released after both QK(j), V(j) after both PV(j).
+//   warp 1      owns TMEM; one lane issues every tcgen05.mma in the order
+//               PV_0(j-1), QK_0(j), PV_1(j-1), QK_1(j): S_t = Q_t K^T (bf16,
+//               SS form) and O_t += P_t V (fp16, TS form, P_t read from TMEM
+//               where the softmax wrote it over S_t, in two 64-key halves so
+//               the first half of PV overlaps the second half's exponentials).
+//   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: one thread
+//               per query row; base-2 online softmax with a lazily rescaled
+//               running max; paired fp32 arithmetic (f32x2) where it applies.
+// Because PV_t(j-1) is issued before QK_t(j), S_t(j) being ready means O_t is
+// quiescent, so the softmax may rescale it without another wait.
+// TMEM: S_0 [0,128), O_0 [128,128+HD), S_1 [256,384), O_1 [384,384+HD).
 #include "sm100.cuh"
 #include "attention.h"
 
 namespace ispa {
 namespace {
 
-constexpr int BM = 128;      // query rows per CTA
+constexpr int BM = 128;      // query rows per tile
+constexpr int NQT = 2;       // query tiles per unit
 constexpr int BN = 128;      // keys per tile
-constexpr int NSTAGE = 2;    // K/V ring depth
-constexpr int kThreads = 192;
+constexpr int NK = 3;        // K ring depth
+constexpr int NV = 2;        // V ring depth
+constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 // Rescale O only when the running max grows by more than 2^8: P values stay
 // below 256 (fine for fp16) and most tiles skip the TMEM round trip.
 constexpr float kRescaleThreshold = 8.0f;
+constexpr float kLn2 = 0.6931471805599453f;
 
 template <int HD>
 struct alignas(1024) Smem {
-  uint8_t q[HD / 64][BM * 128];
-  uint8_t k[NSTAGE][HD / 64][BN * 128];
-  uint8_t v[NSTAGE][HD / 64][BN * 128];
+  uint8_t q[NQT][HD / 64][BM * 128];
+  uint8_t k[NK][HD / 64][BN * 128];
+  uint8_t v[NV][HD / 64][BN * 128];
   uint64_t q_full;
-  uint64_t kv_full[NSTAGE];
-  uint64_t kv_empty[NSTAGE];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t o_done[2];   // PV of tile j done -> o_done[j & 1]
-  uint64_t o_final;     // every MMA of the CTA done
+  uint64_t k_full[NK];
+  uint64_t k_empty[NK];
+  uint64_t v_full[NV];
+  uint64_t v_empty[NV];
+  uint64_t s_full[NQT];
+  uint64_t p_full[NQT][2];   // P_t keys [0,64) and [64,128) written
+  uint64_t o_final;          // every MMA of the unit done
   uint64_t drain;
   uint32_t taddr;
   int abort_flag;
 };
+
+struct Unit {
+  int head;
+  int q0;          // first query row of the pair
+  int n_qt;        // query tiles with rows in range (1 or 2)
+  int hist;        // 1 = history branch, 0 = local branch (sink then local)
+  int n_tiles;
+};
+
+__device__ __forceinline__ Unit unit_of(const AttnParams& p) {
+  Unit u;
+  int b = blockIdx.x;
+  const int per = p.heads * p.n_pairs;
+  u.hist = (p.len[2] > 0 && b < per) ? 1 : 0;
+  if (p.len[2] > 0 && b >= per) b -= per;
+  u.head = b / p.n_pairs;
+  u.q0 = (b % p.n_pairs) * (BM * NQT);
+  u.n_qt = (p.nq - u.q0 > BM) ? 2 : 1;
+  u.n_tiles = u.hist ? (int)((p.len[2] + BN - 1) / BN)
+                     : (int)((p.len[0] + BN - 1) / BN) + (int)((p.len[1] + BN - 1) / BN);
+  return u;
+}
 
 struct TileInfo {
   int branch;   // 0 sink, 1 local, 2 history
@@ -58,14 +93,17 @@ struct TileInfo {
   int valid;
 };
 
-__device__ __forceinline__ TileInfo tile_of(int j, const AttnParams& p) {
-  int n0 = (int)((p.len[0] + BN - 1) / BN);
-  int n1 = (int)((p.len[1] + BN - 1) / BN);
+__device__ __forceinline__ TileInfo tile_of(int j, bool hist, const AttnParams& p) {
   TileInfo t;
-  if (j < n0) { t.branch = 0; t.row0 = j * BN; }
-  else if (j < n0 + n1) { t.branch = 1; t.row0 = (j - n0) * BN; }
-  else { t.branch = 2; t.row0 = (j - n0 - n1) * BN; }
-  int64_t rem = p.len[t.branch] - t.row0;
+  if (hist) {
+    t.branch = 2;
+    t.row0 = j * BN;
+  } else {
+    const int n0 = (int)((p.len[0] + BN - 1) / BN);
+    if (j < n0) { t.branch = 0; t.row0 = j * BN; }
+    else { t.branch = 1; t.row0 = (j - n0) * BN; }
+  }
+  const int64_t rem = p.len[t.branch] - t.row0;
   t.valid = rem < BN ? (int)rem : BN;
   return t;
 }
@@ -76,26 +114,54 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* 
   mbar_wait(bar, parity, status, &dummy);
 }
 
+__device__ __forceinline__ void store_f32x32(float* dst, const float (&v)[32], bool tf32) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float4 x;
+    x.x = tf32 ? to_tf32(v[4 * i]) : v[4 * i];
+    x.y = tf32 ? to_tf32(v[4 * i + 1]) : v[4 * i + 1];
+    x.z = tf32 ? to_tf32(v[4 * i + 2]) : v[4 * i + 2];
+    x.w = tf32 ? to_tf32(v[4 * i + 3]) : v[4 * i + 3];
+    d4[i] = x;
+  }
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * i + 2 * k], v[8 * i + 2 * k + 1]);
+      w[k] = *reinterpret_cast<uint32_t*>(&b2);
+    }
+    d4[i] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
-dual_attention_kernel(const __grid_constant__ AttnParams p) {
+branch_attention_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   Smem<HD>& s = *reinterpret_cast<Smem<HD>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int head = blockIdx.y;
-  const int q0 = blockIdx.x * BM;
-  const int n_loc = (int)((p.len[0] + BN - 1) / BN) + (int)((p.len[1] + BN - 1) / BN);
-  const int n_tiles = n_loc + (int)((p.len[2] + BN - 1) / BN);
+  const Unit u = unit_of(p);
+  const int n_tiles = u.n_tiles;
   volatile int* abort_flag = &s.abort_flag;
 
   if (threadIdx.x == 0) {
     mbar_init(&s.q_full, 1);
-    for (int i = 0; i < NSTAGE; ++i) { mbar_init(&s.kv_full[i], 1); mbar_init(&s.kv_empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&s.s_full[i], 1); mbar_init(&s.p_full[i], 128); }
-    mbar_init(&s.o_done[0], 1);
-    mbar_init(&s.o_done[1], 1);
+    for (int i = 0; i < NK; ++i) { mbar_init(&s.k_full[i], 1); mbar_init(&s.k_empty[i], 1); }
+    for (int i = 0; i < NV; ++i) { mbar_init(&s.v_full[i], 1); mbar_init(&s.v_empty[i], 1); }
+    for (int i = 0; i < NQT; ++i) {
+      mbar_init(&s.s_full[i], 1);
+      mbar_init(&s.p_full[i][0], 128);
+      mbar_init(&s.p_full[i][1], 128);
+    }
     mbar_init(&s.o_final, 1);
     mbar_init(&s.drain, 1);
     s.abort_flag = 0;
@@ -106,34 +172,39 @@ dual_attention_kernel(const __grid_constant__ AttnParams p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = s.taddr;
-  // TMEM column bases: S buffer b at 128 b, O of branch b (0 local, 1 history) at 256 + HD b
-  auto t_s = [tbase](int b) { return tbase + 128u * (uint32_t)b; };
-  auto t_o = [tbase](int b) { return tbase + 256u + (uint32_t)(HD * b); };
+  // TMEM column bases of S_t and O_t
+  auto t_s = [tbase](int t) { return tbase + 256u * (uint32_t)t; };
+  auto t_o = [tbase](int t) { return tbase + 256u * (uint32_t)t + 128u; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    int issued = 0;
     if (lane == 0) {
       tma_prefetch(&p.tm_q);
-      mbar_expect_tx(&s.q_full, HD / 64 * BM * 128);
-      for (int b = 0; b < HD / 64; ++b)
-        tma_load_2d(s.q[b], &p.tm_q, &s.q_full, head * HD + b * 64, q0);
+      mbar_expect_tx(&s.q_full, u.n_qt * (HD / 64) * BM * 128);
+      for (int t = 0; t < u.n_qt; ++t)
+        for (int b = 0; b < HD / 64; ++b)
+          tma_load_2d(s.q[t][b], &p.tm_q, &s.q_full, u.head * HD + b * 64, u.q0 + t * BM);
+      int k_issued = 0, v_issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
-        const int st = j % NSTAGE;
-        if (j >= NSTAGE && !mbar_wait(&s.kv_empty[st], ((j / NSTAGE) - 1) & 1, p.status, abort_flag))
-          break;
-        TileInfo t = tile_of(j, p);
-        mbar_expect_tx(&s.kv_full[st], 2 * (HD / 64) * BN * 128);
-        for (int b = 0; b < HD / 64; ++b) {
-          tma_load_2d(s.k[st][b], &p.tm_k[t.branch], &s.kv_full[st], head * HD + b * 64, t.row0);
-          tma_load_2d(s.v[st][b], &p.tm_v[t.branch], &s.kv_full[st], head * HD + b * 64, t.row0);
-        }
-        issued = j + 1;
+        const TileInfo ti = tile_of(j, u.hist, p);
+        const int sk = j % NK, sv = j % NV;
+        if (j >= NK && !mbar_wait(&s.k_empty[sk], ((j / NK) - 1) & 1, p.status, abort_flag)) break;
+        mbar_expect_tx(&s.k_full[sk], (HD / 64) * BN * 128);
+        for (int b = 0; b < HD / 64; ++b)
+          tma_load_2d(s.k[sk][b], &p.tm_k[ti.branch], &s.k_full[sk], u.head * HD + b * 64, ti.row0);
+        k_issued = j + 1;
+        if (j >= NV && !mbar_wait(&s.v_empty[sv], ((j / NV) - 1) & 1, p.status, abort_flag)) break;
+        mbar_expect_tx(&s.v_full[sv], (HD / 64) * BN * 128);
+        for (int b = 0; b < HD / 64; ++b)
+          tma_load_2d(s.v[sv][b], &p.tm_v[ti.branch], &s.v_full[sv], u.head * HD + b * 64, ti.row0);
+        v_issued = j + 1;
       }
       if (*abort_flag) {  // let copies still in flight land before the CTA exits
         drain_wait(&s.q_full, 0, p.status);
-        for (int j = issued - NSTAGE < 0 ? 0 : issued - NSTAGE; j < issued; ++j)
-          drain_wait(&s.kv_full[j % NSTAGE], (j / NSTAGE) & 1, p.status);
+        for (int j = k_issued - NK < 0 ? 0 : k_issued - NK; j < k_issued; ++j)
+          drain_wait(&s.k_full[j % NK], (j / NK) & 1, p.status);
+        for (int j = v_issued - NV < 0 ? 0 : v_issued - NV; j < v_issued; ++j)
+          drain_wait(&s.v_full[j % NV], (j / NV) & 1, p.status);
       }
     }
   } else if (warp == 1) {
@@ -141,37 +212,54 @@ dual_attention_kernel(const __grid_constant__ AttnParams p) {
     if (lane == 0) {
       const uint32_t idesc_qk = instr_desc(1, 1, 0, 0, BM, BN);   // bf16 x bf16, K-major both
       const uint32_t idesc_pv = instr_desc(0, 0, 0, 1, BM, HD);   // f16 P (TMEM) x f16 V (MN-major)
+      // Descriptors are built once; a k-step only adds its byte offset >> 4 to
+      // the start-address field (all offsets stay inside the 14-bit field).
+      uint64_t dq[NQT], dk[NK], dv[NV];
+      for (int t = 0; t < NQT; ++t) dq[t] = smem_desc(smem_u32(s.q[t][0]), 16, 1024);
+      for (int i = 0; i < NK; ++i) dk[i] = smem_desc(smem_u32(s.k[i][0]), 16, 1024);
+      for (int i = 0; i < NV; ++i) dv[i] = smem_desc(smem_u32(s.v[i][0]), BN * 128, 1024);
       bool ok = mbar_wait(&s.q_full, 0, p.status, abort_flag);
-      auto issue_qk = [&](int j) -> bool {
-        const int st = j % NSTAGE;
-        if (!mbar_wait(&s.kv_full[st], (j / NSTAGE) & 1, p.status, abort_flag)) return false;
-        tc_fence_after();
+      for (int j = 0; ok && j <= n_tiles; ++j) {
+        for (int t = 0; ok && t < u.n_qt; ++t) {
+          if (j > 0) {   // O_t += P_t(j-1) V(j-1), one 64-key half at a time
+            const int sv = (j - 1) % NV;
+            if (t == 0 && !mbar_wait(&s.v_full[sv], ((j - 1) / NV) & 1, p.status, abort_flag)) {
+              ok = false;
+              break;
+            }
+            const uint64_t bv = sv == 0 ? dv[0] : dv[1];
+            const uint32_t ao = t_s(t), oo = t_o(t);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk / 4) * (BM * 128) + (kk % 4) * 32;
-          const uint32_t koff = (kk / 4) * (BN * 128) + (kk % 4) * 32;
-          mma_ss(t_s(j & 1), smem_desc(smem_u32(s.q[0]) + off, 16, 1024),
-                 smem_desc(smem_u32(s.k[st][0]) + koff, 16, 1024), idesc_qk, kk > 0);
-        }
-        tc_commit(&s.s_full[j & 1]);
-        return true;
-      };
-      if (ok && n_tiles > 0) ok = issue_qk(0);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + 1 < n_tiles && !issue_qk(j + 1)) { ok = false; break; }
-        if (!mbar_wait(&s.p_full[j & 1], (j >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const int st = j % NSTAGE;
-        const int br = j < n_loc ? 0 : 1;
-        const bool first = (j == 0) || (j == n_loc);
+            for (int h = 0; h < 2; ++h) {
+              if (!mbar_wait(&s.p_full[t][h], (j - 1) & 1, p.status, abort_flag)) { ok = false; break; }
+              tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          mma_ts(t_o(br), t_s(j & 1) + kk * 8,
-                 smem_desc(smem_u32(s.v[st][0]) + kk * 2048, BN * 128, 1024), idesc_pv,
-                 (first && kk == 0) ? 0u : 1u);
+              for (int kk = h * 4; kk < h * 4 + 4; ++kk)
+                mma_ts(oo, ao + kk * 8, bv + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+                       (j == 1 && kk == 0) ? 0u : 1u);
+            }
+            if (!ok) break;
+            if (t == u.n_qt - 1) tc_commit(&s.v_empty[sv]);
+          }
+          if (j < n_tiles) {   // S_t = Q_t K(j)^T
+            const int sk = j % NK;
+            if (t == 0 && !mbar_wait(&s.k_full[sk], (j / NK) & 1, p.status, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t bq = t == 0 ? dq[0] : dq[1];
+            const uint64_t bk = sk == 0 ? dk[0] : (sk == 1 ? dk[1] : dk[2]);
+            const uint32_t so = t_s(t);
+#pragma unroll
+            for (int kk = 0; kk < HD / 16; ++kk) {
+              const uint32_t off = ((kk / 4) * (BN * 128) + (kk % 4) * 32) >> 4;
+              mma_ss(so, bq + off, bk + off, idesc_qk, kk > 0);
+            }
+            tc_commit(&s.s_full[t]);
+            if (t == u.n_qt - 1) tc_commit(&s.k_empty[sk]);
+          }
         }
-        tc_commit(&s.kv_empty[st]);
-        tc_commit(&s.o_done[j & 1]);
       }
       if (ok) tc_commit(&s.o_final);
       if (!ok) {  // let issued MMAs finish before TMEM is freed
@@ -180,57 +268,52 @@ dual_attention_kernel(const __grid_constant__ AttnParams p) {
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp >= 4 && (warp - 4) / 4 < u.n_qt) {
     // ------------------------------------------------------------ softmax
+    const int t = (warp - 4) / 4;                 // query tile of this warpgroup
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;            // row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t ts = t_s(t) + lane_off, to = t_o(t) + lane_off;
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;                 // running max (log2 units), sum
-    float m_loc = -INFINITY, l_loc = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      if (j == n_loc) { m_loc = m; l_loc = l; m = -INFINITY; l = 0.f; }
-      const TileInfo t = tile_of(j, p);
-      if (!mbar_wait(&s.s_full[j & 1], (j >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
+      const TileInfo ti = tile_of(j, u.hist, p);
+      if (!mbar_wait(&s.s_full[t], j & 1, p.status, abort_flag)) { ok = false; break; }
       tc_fence_after();
       float sv[BN];
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t raw[32];
-        tmem_ld32(t_s(j & 1) + lane_off + c * 32, raw);
-        tmem_ld_wait();
+        tmem_ld32(ts + c * 32, raw);
 #pragma unroll
         for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(raw[i]);
       }
-      float mx = -INFINITY;
-      if (t.valid < BN) {
+      tmem_ld_wait();
+      if (ti.valid < BN) {
 #pragma unroll
-        for (int i = 0; i < BN; ++i) {
-          if (i >= t.valid) sv[i] = -INFINITY;
-          mx = fmaxf(mx, sv[i]);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < BN; ++i) mx = fmaxf(mx, sv[i]);
+        for (int i = 0; i < BN; ++i)
+          if (i >= ti.valid) sv[i] = -INFINITY;
       }
+      float mx8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx8[k] = fmax3(sv[k], sv[k + 8], sv[k + 16]);
+#pragma unroll
+      for (int i = 24; i < BN; i += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], sv[i + k], sv[i + k + 8]);
+      const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                             fmaxf(mx8[6], mx8[7]));
       const float m_new = fmaxf(m, mx * sl2);
-      const bool first = (j == 0) || (j == n_loc);
-      if (first) {
+      if (j == 0) {
         m = m_new;
       } else {
         const bool need = m_new > m + kRescaleThreshold;
-        if (__any_sync(0xffffffffu, need)) {
-          // all PV products into this branch's O must have landed first
-          if (!mbar_wait(&s.o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.status, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+        if (__any_sync(0xffffffffu, need)) {   // O_t is quiescent: PV_t(j-1) preceded S_t(j)
           const float alpha = need ? ex2(m - m_new) : 1.f;
           if (need) { l *= alpha; m = m_new; }
-          const uint32_t to = t_o(j < n_loc ? 0 : 1) + lane_off;
-#pragma unroll
+#pragma unroll 1
           for (int c = 0; c < HD / 32; ++c) {
             uint32_t raw[32];
             tmem_ld32(to + c * 32, raw);
@@ -241,103 +324,112 @@ dual_attention_kernel(const __grid_constant__ AttnParams p) {
           }
         }
       }
-      float rs = 0.f;
+      const float2 scl = make_float2(sl2, sl2), nm = make_float2(-m, -m);
+      float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < BN / 64; ++c) {
-        uint32_t pk[32];
+      for (int h = 0; h < 2; ++h) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2(fmaf(sv[c * 64 + 2 * i], sl2, -m));
-          const float p1 = ex2(fmaf(sv[c * 64 + 2 * i + 1], sl2, -m));
-          rs += p0 + p1;
-          pk[i] = pack_half2(p0, p1);
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = h * 64 + c * 32 + 2 * i;
+            const float2 x = ffma2(make_float2(sv[e], sv[e + 1]), scl, nm);
+            const float2 pe = make_float2(ex2(x.x), ex2(x.y));
+            rs2[i & 1] = fadd2(rs2[i & 1], pe);
+            pk[i] = pack_half2(pe.x, pe.y);
+          }
+          tmem_st16(ts + h * 32 + c * 16, pk);
         }
-        tmem_st32(t_s(j & 1) + lane_off + c * 32, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&s.p_full[t][h]);
       }
-      l += rs;
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&s.p_full[j & 1]);
+      l += (rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y);
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && n_tiles > 0 && mbar_wait(&s.o_final, 0, p.status, abort_flag)) {
+    if (ok && mbar_wait(&s.o_final, 0, p.status, abort_flag)) {
       tc_fence_after();
-      const bool has_hist = n_tiles > n_loc;
-      if (!has_hist) { m_loc = m; l_loc = l; }
-      const float kLn2 = 0.6931471805599453f;
-      const float lse_l = (m_loc + log2f(l_loc)) * kLn2;
-      float lse_h = -INFINITY, lse_f = lse_l, w_hist = 0.f, inv_lh = 0.f;
-      if (has_hist) {
-        lse_h = (m + log2f(l)) * kLn2;
-        const float hi = fmaxf(lse_l, lse_h), lo = fminf(lse_l, lse_h);
-        lse_f = hi + log1pf(expf(lo - hi));
-        w_hist = expf(lse_h - lse_f);
-        inv_lh = 1.f / l;
-      }
-      const float inv_ll = 1.f / l_loc;
-      const int row = q0 + r;
+      const int row = u.q0 + t * BM + r;
       const bool row_ok = row < p.nq;
       const int64_t d = (int64_t)p.heads * HD;
-      const int64_t base = (int64_t)row * d + (int64_t)head * HD;
+      const int64_t base = (int64_t)row * d + (int64_t)u.head * HD;
+      const float lse = (m + log2f(l)) * kLn2;
+      const float inv = 1.f / l;
+      const bool direct = !u.hist && p.len[2] == 0;   // no history: write the final outputs
 #pragma unroll 1
       for (int c = 0; c < HD / 32; ++c) {
-        uint32_t ol[32], oh[32];
-        tmem_ld32(t_o(0) + lane_off + c * 32, ol);
-        if (has_hist) tmem_ld32(t_o(1) + lane_off + c * 32, oh);
+        uint32_t raw[32];
+        tmem_ld32(to + c * 32, raw);
         tmem_ld_wait();
         if (!row_ok) continue;
-        float al[32], dd[32];
+        float a[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          al[i] = __uint_as_float(ol[i]) * inv_ll;
-          const float ah = has_hist ? __uint_as_float(oh[i]) * inv_lh : 0.f;
-          dd[i] = has_hist ? w_hist * (ah - al[i]) : 0.f;
-        }
-        if (p.a_loc) {
-          float4* dst = reinterpret_cast<float4*>(p.a_loc + base + c * 32);
+        for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(raw[i]) * inv;
+        if (u.hist) {
+          store_f32x32(p.hist_out + base + c * 32, a, false);
+        } else {
+          if (p.a_loc) store_f32x32(p.a_loc + base + c * 32, a, p.round_tf32 != 0);
+          if (direct && p.a_full) store_bf16x32(p.a_full + base + c * 32, a);
+          if (direct && p.d_out) {
+            float z[32];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float4 v;
-            v.x = p.round_tf32 ? to_tf32(al[4 * i]) : al[4 * i];
-            v.y = p.round_tf32 ? to_tf32(al[4 * i + 1]) : al[4 * i + 1];
-            v.z = p.round_tf32 ? to_tf32(al[4 * i + 2]) : al[4 * i + 2];
-            v.w = p.round_tf32 ? to_tf32(al[4 * i + 3]) : al[4 * i + 3];
-            dst[i] = v;
-          }
-        }
-        if (p.d_out) {
-          float4* dst = reinterpret_cast<float4*>(p.d_out + base + c * 32);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(to_tf32(dd[4 * i]), to_tf32(dd[4 * i + 1]),
-                                 to_tf32(dd[4 * i + 2]), to_tf32(dd[4 * i + 3]));
-        }
-        if (p.a_full) {
-          uint4* dst = reinterpret_cast<uint4*>(p.a_full + base + c * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t w[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(al[8 * i + 2 * k] + dd[8 * i + 2 * k],
-                                                        al[8 * i + 2 * k + 1] + dd[8 * i + 2 * k + 1]);
-              w[k] = *reinterpret_cast<uint32_t*>(&b2);
-            }
-            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int i = 0; i < 32; ++i) z[i] = 0.f;
+            store_f32x32(p.d_out + base + c * 32, z, false);
           }
         }
       }
       if (row_ok) {
-        const int64_t li = (int64_t)head * p.nq + row;
-        if (p.lse_loc) p.lse_loc[li] = lse_l;
-        if (p.lse_hist) p.lse_hist[li] = lse_h;
-        if (p.lse_full) p.lse_full[li] = lse_f;
+        const int64_t li = (int64_t)u.head * p.nq + row;
+        if (u.hist) {
+          p.lse_hist_ws[li] = lse;
+        } else {
+          p.lse_loc_ws[li] = lse;
+          if (direct) {
+            if (p.lse_loc) p.lse_loc[li] = lse;
+            if (p.lse_hist) p.lse_hist[li] = -INFINITY;
+            if (p.lse_full) p.lse_full[li] = lse;
+          }
+        }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tbase, kTmemCols);
+}
+
+// Post-hoc LSE merge of the two branches (element-wise, 4 columns a thread).
+__global__ void lse_merge_kernel(const AttnParams p, int hd) {
+  const int64_t d = (int64_t)p.heads * hd;
+  const int64_t n4 = (int64_t)p.nq * d / 4;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n4;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = (e * 4) / d;
+    const int head = (int)(((e * 4) % d) / hd);
+    const int64_t li = (int64_t)head * p.nq + row;
+    const float ll = p.lse_loc_ws[li], lh = p.lse_hist_ws[li];
+    const float hi = fmaxf(ll, lh), lo = fminf(ll, lh);
+    const float lf = hi + log1pf(expf(lo - hi));
+    const float w = expf(lh - lf);
+    const float4 a = reinterpret_cast<const float4*>(p.a_loc)[e];
+    const float4 h = reinterpret_cast<const float4*>(p.hist_out)[e];
+    const float4 dd = make_float4(w * (h.x - a.x), w * (h.y - a.y), w * (h.z - a.z), w * (h.w - a.w));
+    if (p.d_out)
+      reinterpret_cast<float4*>(p.d_out)[e] =
+          make_float4(to_tf32(dd.x), to_tf32(dd.y), to_tf32(dd.z), to_tf32(dd.w));
+    if (p.a_full) {
+      __nv_bfloat162 b0 = __floats2bfloat162_rn(a.x + dd.x, a.y + dd.y);
+      __nv_bfloat162 b1 = __floats2bfloat162_rn(a.z + dd.z, a.w + dd.w);
+      reinterpret_cast<uint2*>(p.a_full)[e] =
+          make_uint2(*reinterpret_cast<uint32_t*>(&b0), *reinterpret_cast<uint32_t*>(&b1));
+    }
+    if (((e * 4) % hd) == 0) {   // one thread per (row, head) writes the LSEs
+      if (p.lse_loc) p.lse_loc[li] = ll;
+      if (p.lse_hist) p.lse_hist[li] = lh;
+      if (p.lse_full) p.lse_full[li] = lf;
+    }
+  }
 }
 
 // bf16 -> fp16 copy of the value tensors (the P.V product runs in fp16);
@@ -382,18 +474,27 @@ cudaError_t launch_v_to_half(const void* src, void* dst, int64_t n_elems, int* s
   return cudaGetLastError();
 }
 
+int attention_pairs(int64_t nq) { return (int)((nq + BM * NQT - 1) / (BM * NQT)); }
+
 cudaError_t launch_dual_attention(const AttnParams& p, int head_dim, cudaStream_t stream) {
-  dim3 grid((p.nq + BM - 1) / BM, p.heads);
+  const int units = p.heads * p.n_pairs * (p.len[2] > 0 ? 2 : 1);
   const size_t smem = attention_smem_bytes(head_dim);
   if (head_dim == 64) {
-    cudaFuncSetAttribute(dual_attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(branch_attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
-    dual_attention_kernel<64><<<grid, kThreads, smem, stream>>>(p);
+    branch_attention_kernel<64><<<units, kThreads, smem, stream>>>(p);
   } else {
-    cudaFuncSetAttribute(dual_attention_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(branch_attention_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
-    dual_attention_kernel<128><<<grid, kThreads, smem, stream>>>(p);
+    branch_attention_kernel<128><<<units, kThreads, smem, stream>>>(p);
   }
+  count_launches();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || p.len[2] == 0) return e;
+  const int64_t n4 = (int64_t)p.nq * p.heads * head_dim / 4;
+  int blocks = (int)((n4 + 255) / 256);
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  lse_merge_kernel<<<blocks, 256, 0, stream>>>(p, head_dim);
   count_launches();
   return cudaGetLastError();
 }

@@ -21,18 +21,23 @@ struct AttnParams {
   int64_t len[3];
   int nq;
   int heads;
+  int n_pairs;            // ceil(nq / 256): query-tile pairs per head
   float scale_log2;       // softmax scale * log2(e)
   int round_tf32;         // round A_loc / D stores to tf32 (nearest, ties away)
-  float* a_loc;           // [nq, d] fp32 or nullptr
+  float* a_loc;           // [nq, d] fp32 or nullptr (required with history)
   float* d_out;           // [nq, d] fp32 or nullptr
   __nv_bfloat16* a_full;  // [nq, d] bf16 or nullptr
   float* lse_loc;         // [heads, nq] or nullptr
   float* lse_hist;
   float* lse_full;
+  float* hist_out;        // workspace: history-branch output [nq, d] fp32
+  float* lse_loc_ws;      // workspace: [heads, nq]
+  float* lse_hist_ws;     // workspace: [heads, nq]
   int* status;
 };
 
 size_t attention_smem_bytes(int head_dim);
+int attention_pairs(int64_t nq);
 cudaError_t launch_v_to_half(const void* src, void* dst, int64_t n_elems, int* status,
                              cudaStream_t stream);
 cudaError_t launch_dual_attention(const AttnParams& p, int head_dim, cudaStream_t stream);

@@ -63,7 +63,7 @@ def _load():
         "ispa_status_string": (ctypes.c_char_p, [I]),
         "ispa_version": (I, []),
         "ispa_kernel_launches": (ctypes.c_uint64, []),
-        "ispa_dual_attention_workspace_size": (SZ, [I64, I64, I64, I, I]),
+        "ispa_dual_attention_workspace_size": (SZ, [I64, I64, I64, I64, I, I]),
         "ispa_dual_attention": (I, [P, I64, I, I, IspaKV, IspaKV, IspaKV, F, P, P, P, P, P, P,
                                     P, SZ, P, P]),
         "ispa_local_attention": (I, [P, I64, I, I, IspaKV, IspaKV, F, P, P, P, P, SZ, P, P]),
@@ -142,9 +142,10 @@ def read_status(status: torch.Tensor) -> int:
     return int(status.item())
 
 
-def ispa_dual_attention_workspace_size(sink_len: int, local_len: int, hist_len: int, heads: int,
-                                       head_dim: int) -> int:
-    return _load().ispa_dual_attention_workspace_size(sink_len, local_len, hist_len, heads, head_dim)
+def ispa_dual_attention_workspace_size(nq: int, sink_len: int, local_len: int, hist_len: int,
+                                       heads: int, head_dim: int) -> int:
+    return _load().ispa_dual_attention_workspace_size(nq, sink_len, local_len, hist_len, heads,
+                                                      head_dim)
 
 
 def ispa_dual_attention(q, k_sink, v_sink, k_loc, v_loc, k_hist=None, v_hist=None, scale=None,
@@ -168,7 +169,7 @@ def ispa_dual_attention(q, k_sink, v_sink, k_loc, v_loc, k_hist=None, v_hist=Non
     a_full = torch.empty(nq, d, dtype=torch.bfloat16, device=dev) if want_a_full else None
     lse = [torch.empty(heads, nq, dtype=torch.float32, device=dev) if want_lse else None
            for _ in range(3)]
-    need = ispa_dual_attention_workspace_size(sink.len, loc.len, hist.len, heads, hd)
+    need = ispa_dual_attention_workspace_size(nq, sink.len, loc.len, hist.len, heads, hd)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     status = new_status(dev) if status is None else status
@@ -194,7 +195,7 @@ def ispa_local_attention(q, k_sink, v_sink, k_loc, v_loc, scale=None, out_dtype=
         scale = hd ** -0.5
     out = torch.empty(nq, heads * hd, dtype=out_dtype, device=dev)
     lse = torch.empty(heads, nq, dtype=torch.float32, device=dev) if want_lse else None
-    need = ispa_dual_attention_workspace_size(sink.len, loc.len, 0, heads, hd)
+    need = ispa_dual_attention_workspace_size(nq, sink.len, loc.len, 0, heads, hd)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     status = new_status(dev) if status is None else status

@@ -32,7 +32,8 @@ class LayerWarmup:
         self.a_full = torch.empty(chunk_rows, d, dtype=torch.bfloat16, device=device)
         self.lse = [torch.empty(heads, chunk_rows, **f32) for _ in range(3)]
         self.attn_ws = torch.empty(ispa.ispa_dual_attention_workspace_size(
-            max_sink, max_local, max_hist, heads, head_dim), dtype=torch.uint8, device=device)
+            chunk_rows, max_sink, max_local, max_hist, heads, head_dim), dtype=torch.uint8,
+            device=device)
         self.M = torch.zeros(2 * d, 2 * d, **f32)
         self.solve_ws = torch.empty(ispa.ispa_absorb_workspace_size(d), dtype=torch.uint8,
                                     device=device)

@@ -55,9 +55,12 @@ def test_workspace_sizes(ispa):
     def r256(x):
         return (x + 255) // 256 * 256
     d = 12 * 128
-    assert ispa.ispa_dual_attention_workspace_size(1560, 4680, 14040, 12, 128) == \
-        r256(1560 * d * 2) + r256(4680 * d * 2) + r256(14040 * d * 2) + 256
-    assert ispa.ispa_dual_attention_workspace_size(-1, 1, 1, 1, 64) == 0
+    assert ispa.ispa_dual_attention_workspace_size(4680, 1560, 4680, 14040, 12, 128) == \
+        r256(1560 * d * 2) + r256(4680 * d * 2) + r256(14040 * d * 2) + r256(4680 * d * 4) + \
+        2 * r256(12 * 4680 * 4) + 256
+    assert ispa.ispa_dual_attention_workspace_size(10, 1, 1, 0, 1, 64) == \
+        r256(64 * 2) * 2 + 2 * r256(40) + 256
+    assert ispa.ispa_dual_attention_workspace_size(1, -1, 1, 1, 1, 64) == 0
     n = 1536
     assert ispa.ispa_absorb_workspace_size(n) >= 2 * n * n * 4
     assert ispa.ispa_absorb_workspace_size(0) == 0
