@@ -8,6 +8,7 @@
 
 #include "sm100.cuh"
 #include "attention.h"
+#include "host_util.h"
 
 namespace ispa {
 static std::atomic<unsigned long long> g_launches{0};
@@ -25,39 +26,7 @@ cudaError_t rank_layers(const double* err, int n, int K, int* perm, uint8_t* sel
 namespace {
 
 using ispa::AttnParams;
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
-// Row-major [rows, cols] matrix, tiles of box_cols x box_rows.
-bool encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t cols,
-               uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * (uint64_t)esize};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t es[2] = {1, 1};
-  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
+using ispa::encode_2d;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
@@ -113,7 +82,7 @@ int attention_common(const void* q, int64_t nq, int heads, int head_dim, const i
 
   AttnParams p;
   std::memset(&p, 0, sizeof(p));
-  if (!encode_2d(&p.tm_q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, nq, 64, 128,
+  if (!encode_2d(&p.tm_q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, nq, d, 64, 128,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return ISPA_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -128,9 +97,9 @@ int attention_common(const void* q, int64_t nq, int heads, int head_dim, const i
     ws += v_half_bytes(br[b].len, d);
     cudaError_t e = ispa::launch_v_to_half(br[b].v, vh, br[b].len * d, dev_status, s);
     if (e != cudaSuccess) return cuda_rc(e);
-    if (!encode_2d(&p.tm_k[b], br[b].k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, br[b].len, 64, 128,
+    if (!encode_2d(&p.tm_k[b], br[b].k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, br[b].len, d, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&p.tm_v[b], vh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, br[b].len, 64, 128,
+        !encode_2d(&p.tm_v[b], vh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, br[b].len, d, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B))
       return ISPA_ERR_CUDA;
   }
@@ -228,9 +197,9 @@ int ispa_gram_accumulate(const float* a_loc, const float* d_in, int64_t rows, in
   if (rows == 0) return ISPA_OK;
   ispa::GramParams p;
   std::memset(&p, 0, sizeof(p));
-  if (!encode_2d(&p.tm_a, a_loc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dim, rows, 32, 32,
+  if (!encode_2d(&p.tm_a, a_loc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dim, rows, dim, 32, 32,
                  CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) ||
-      !encode_2d(&p.tm_d, d_in, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dim, rows, 32, 32,
+      !encode_2d(&p.tm_d, d_in, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dim, rows, dim, 32, 32,
                  CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B))
     return ISPA_ERR_CUDA;
   const int bn = (dim % 256 == 0) ? 256 : 128;

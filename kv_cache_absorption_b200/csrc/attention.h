@@ -58,9 +58,5 @@ struct GramParams {
 cudaError_t launch_gram(const GramParams& p, int bn, int grid, cudaStream_t stream);
 int gram_tile_count(int dim, int bn, int want_s);
 
-// Dense fp32 helpers for the solve and the error: see solve.cu / error.cu.
-cudaError_t launch_sgemm(bool ta, bool tb, int M, int N, int K, float alpha, const float* A,
-                         int lda, const float* B, int ldb, float beta, float* C, int ldc,
-                         bool lower_only, cudaStream_t stream);
 
 }  // namespace ispa

@@ -10,13 +10,15 @@
 //   ||E||^2        = <S, W W^T> - <dW, B> - lambda ||dW||^2
 //   ||A_full W||^2 = <G, W W^T> + 2 <R, W W^T> + <S, W W^T>
 // so the error needs no pass over the warmup rows. W W^T is never stored:
-// each CTA forms one 128 x 128 tile of it in registers and immediately
-// reduces it against the matching tiles of G, R and S (fp64 accumulation).
-// G and S hold only their tiles on and above the tile diagonal: a tile above
-// the diagonal counts twice (for its mirror image), one below it not at all.
+// each CTA of the 3xTF32 tensor-core GEMM forms one 128 x 128 tile of it in
+// TMEM and immediately reduces it against the matching tiles of G, R and S
+// (fp64 accumulation). G and S hold only their tiles on and above the tile
+// diagonal: a tile above the diagonal counts twice (for its mirror image),
+// one below it not at all.
 #include "sm100.cuh"
 #include "attention.h"
-#include "simt_gemm.cuh"
+#include "host_util.h"
+#include "tgemm.h"
 
 namespace ispa {
 namespace {
@@ -31,43 +33,6 @@ __device__ __forceinline__ double block_sum(double v, double* red) {
     for (int i = 0; i < (int)(blockDim.x >> 5); ++i) s += red[i];
   __syncthreads();
   return s;
-}
-
-// acc[0] += <G, WW^T>, acc[1] += <R, WW^T>, acc[2] += <S, WW^T>
-__global__ void __launch_bounds__(kGemmThreads)
-wwt_reduce_kernel(const float* __restrict__ M, const float* __restrict__ W, int dim,
-                  double* __restrict__ acc) {
-  __shared__ GemmSmem sm;
-  __shared__ double red[kGemmThreads / 32];
-  const int I = blockIdx.y, J = blockIdx.x;
-  const int m0 = I * kGemmTile, n0 = J * kGemmTile;
-  float p[8][8];
-  gemm_tile<false, true>(sm, W, dim, W, dim, dim, dim, dim, m0, n0, p);
-  const size_t ld = 2 * (size_t)dim;
-  const double wsym = I < J ? 2.0 : (I == J ? 1.0 : 0.0);
-  double g = 0.0, r = 0.0, s = 0.0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const size_t row = m0 + gemm_row(i);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const size_t col = n0 + gemm_col(j);
-      const double pij = p[i][j];
-      r += (double)M[row * ld + dim + col] * pij;
-      if (wsym != 0.0) {
-        g += (double)M[row * ld + col] * pij;
-        s += (double)M[(row + dim) * ld + dim + col] * pij;
-      }
-    }
-  }
-  g = block_sum(g, red) * wsym;
-  r = block_sum(r, red);
-  s = block_sum(s, red) * wsym;
-  if (threadIdx.x == 0) {
-    atomicAdd(acc + 0, g);
-    atomicAdd(acc + 1, r);
-    atomicAdd(acc + 2, s);
-  }
 }
 
 // acc[3] += <dW, B>, acc[4] += ||dW||^2
@@ -120,13 +85,30 @@ cudaError_t layer_error(const float* M, const float* W, const float* dW, const f
                         const float* lam, int dim, double* err, double* acc,
                         cudaStream_t stream) {
   cudaMemsetAsync(acc, 0, 5 * sizeof(double), stream);
-  dim3 grid(dim / kGemmTile, dim / kGemmTile);
-  wwt_reduce_kernel<<<grid, kGemmThreads, 0, stream>>>(M, W, dim, acc);
+  {
+    TGemmParams p{};
+    p.nprob = 1;
+    p.dot_M = M;
+    p.dot_dim = dim;
+    p.dot_acc = acc;
+    TGemmProblem& pr = p.prob[0];
+    // P = W W^T: op(A) = W (K-major), op(B) = W^T, i.e. W read K-major
+    if (!encode_f32_operand(&pr.ta, W, dim, dim, dim, false) ||
+        !encode_f32_operand(&pr.tb, W, dim, dim, dim, false))
+      return cudaErrorInvalidValue;
+    pr.a_mn = 0;
+    pr.b_mn = 0;
+    pr.M = pr.N = pr.K = dim;
+    pr.mode = kModeDot3;
+    pr.alpha = 1.f;
+    cudaError_t e = launch_tgemm(p, stream);
+    if (e != cudaSuccess) return e;
+  }
   const size_t n4 = (size_t)dim * dim / 4;
   dot_kernel<<<148 * 2, 256, 0, stream>>>(reinterpret_cast<const float4*>(dW),
                                           reinterpret_cast<const float4*>(B), n4, acc);
   finalize_kernel<<<1, 1, 0, stream>>>(acc, lam, err);
-  count_launches(3);
+  count_launches(2);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,293 @@
+// fp32-accurate GEMM on the tf32 tensor cores (tcgen05 kind::tf32, 3xTF32).
+//
+// The absorb solve of "Towards Memory-Efficient Autoregressive Video
+// Generation via Instance-Specific Parametric Absorption" (technical
+// summary, section 2, step 2) factors G + lambda I, whose condition number
+// amplifies rounding error: single-pass tf32 (10-bit mantissa) is not
+// accurate enough there, fp32 is. Each fp32 operand x is split in shared
+// memory into hi = tf32(x) and lo = tf32(x - hi) (round to nearest), and
+// A B is accumulated in fp32 as A_hi B_hi + A_hi B_lo + A_lo B_hi, whose
+// error is of the order of fp32 rounding.
+//
+// One CTA computes one 128 x 128 tile of C = alpha * op(A) op(B) + beta * C.
+// Operands are row-major fp32 in global memory; each is read either K-major
+// (the K index contiguous) or MN-major (M or N contiguous), so transposes
+// cost nothing. A launch may hold up to 4 independent problems ("grouped");
+// a problem can be restricted to the tiles on or below its diagonal, and to
+// the K range a triangular A operand leaves non-zero.
+//
+// Warp roles (192 threads): warp 0 TMA producer (3-stage ring of 32-deep K
+// slabs), warp 1 TMEM owner and MMA issuer, warps 2-5 split each slab into
+// hi/lo and then run the epilogue.
+#include "sm100.cuh"
+#include "attention.h"
+#include "tgemm.h"
+
+namespace ispa {
+namespace {
+
+constexpr int TM = 128, TN = 128, TK = 32;
+constexpr int NSTAGE = 3;
+constexpr int kThreads = 192;
+constexpr int kSlab = TM * TK * 4;   // 16 KB: one operand slab, fp32
+
+struct alignas(1024) GSmem {
+  uint8_t a_hi[NSTAGE][kSlab];
+  uint8_t a_lo[NSTAGE][kSlab];
+  uint8_t b_hi[NSTAGE][kSlab];
+  uint8_t b_lo[NSTAGE][kSlab];
+  uint64_t full[NSTAGE];    // TMA landed
+  uint64_t split[NSTAGE];   // hi/lo written
+  uint64_t empty[NSTAGE];   // MMAs done reading
+  uint64_t acc_full;
+  uint64_t drain;
+  uint32_t taddr;
+  int abort_flag;
+  int tile_i, tile_j, prob;
+};
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* status) {
+  int dummy = 0;
+  mbar_wait(bar, parity, status, &dummy);
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Tile (i, j) of problem `q` from the launch-wide tile index.
+__device__ __forceinline__ void decode(const TGemmParams& p, int b, int& q, int& i, int& j) {
+  q = 0;
+  while (q + 1 < p.nprob && b >= p.prob[q + 1].tile_base) ++q;
+  const TGemmProblem& pr = p.prob[q];
+  int t = b - pr.tile_base;
+  if (pr.lower) {   // tiles with j <= i, row by row
+    int r = (int)((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
+    while ((r + 1) * (r + 2) / 2 <= t) ++r;
+    while (r * (r + 1) / 2 > t) --r;
+    i = r;
+    j = t - r * (r + 1) / 2;
+  } else {
+    i = t / pr.nt;
+    j = t % pr.nt;
+  }
+}
+
+__device__ __forceinline__ void k_range(const TGemmProblem& pr, int i, int& kb, int& ke) {
+  kb = 0;
+  ke = pr.K / TK;
+  if (pr.tri == kTriLowerA) ke = min(ke, (i + 1) * (TM / TK));
+  if (pr.tri == kTriUpperA) kb = i * (TM / TK);
+}
+
+// Loads one 32-deep slab of a 128-wide operand block (rows/cols starting at
+// `mn0`, K starting at `k0`) into `dst`.
+__device__ __forceinline__ void load_slab(uint8_t* dst, const CUtensorMap* m, bool mn_major,
+                                          int mn0, int k0, uint64_t* bar) {
+  if (mn_major) {   // K rows x MN columns: four 32-wide boxes
+    for (int c = 0; c < 4; ++c) tma_load_2d(dst + c * (TK * 128), m, bar, mn0 + c * 32, k0);
+  } else {          // MN rows x K columns: one box of 128 rows x 32
+    tma_load_2d(dst, m, bar, k0, mn0);
+  }
+}
+
+__device__ __forceinline__ uint64_t slab_desc(const uint8_t* base, bool mn_major) {
+  // K-major: 128-byte rows, 8-row groups 1024 B apart, 128-byte swizzle.
+  // MN-major: 32-wide MN blocks 4 KB apart, 4-row K groups 512 B apart,
+  // 128-byte swizzle of 32-byte atoms (the MN-major tf32 form).
+  return mn_major ? smem_desc(smem_u32(base), TK * 128, 512, 1) : smem_desc(smem_u32(base), 16, 1024, 2);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constant__ TGemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  GSmem& s = *reinterpret_cast<GSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  volatile int* abort_flag = &s.abort_flag;
+  int q, ti, tj;
+  decode(p, blockIdx.x, q, ti, tj);
+  const TGemmProblem& pr = p.prob[q];
+  int kb, ke;
+  k_range(pr, ti, kb, ke);
+  const int nk = ke - kb;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NSTAGE; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.split[i], 128);
+      mbar_init(&s.empty[i], 1);
+    }
+    mbar_init(&s.acc_full, 1);
+    mbar_init(&s.drain, 1);
+    s.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) { tmem_alloc(&s.taddr, TN); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tacc = s.taddr;
+
+  if (warp == 0) {
+    if (lane == 0 && nk > 0) {
+      tma_prefetch(&pr.ta);
+      tma_prefetch(&pr.tb);
+      int n = 0;
+      for (int k = kb; k < ke; ++k, ++n) {
+        const int st = n % NSTAGE;
+        if (n >= NSTAGE && !mbar_wait(&s.empty[st], ((n / NSTAGE) - 1) & 1, p.status, abort_flag)) break;
+        mbar_expect_tx(&s.full[st], 2 * kSlab);
+        load_slab(s.a_hi[st], &pr.ta, pr.a_mn, pr.a_row0 + ti * TM, pr.a_k0 + k * TK, &s.full[st]);
+        load_slab(s.b_hi[st], &pr.tb, pr.b_mn, pr.b_col0 + tj * TN, pr.b_k0 + k * TK, &s.full[st]);
+      }
+      if (*abort_flag)
+        for (int j = n - NSTAGE < 0 ? 0 : n - NSTAGE; j < n; ++j)
+          drain_wait(&s.full[j % NSTAGE], (j / NSTAGE) & 1, p.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && nk > 0) {
+      const uint32_t idesc = instr_desc(2, 2, pr.a_mn, pr.b_mn, TM, TN);
+      const uint32_t a_step = pr.a_mn ? 1024u >> 4 : 32u >> 4;   // one 8-deep k step
+      const uint32_t b_step = pr.b_mn ? 1024u >> 4 : 32u >> 4;
+      bool ok = true;
+      for (int n = 0; n < nk; ++n) {
+        const int st = n % NSTAGE;
+        if (!mbar_wait(&s.split[st], (n / NSTAGE) & 1, p.status, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t ah = slab_desc(s.a_hi[st], pr.a_mn), al = slab_desc(s.a_lo[st], pr.a_mn);
+        const uint64_t bh = slab_desc(s.b_hi[st], pr.b_mn), bl = slab_desc(s.b_lo[st], pr.b_mn);
+#pragma unroll
+        for (int kk = 0; kk < TK / 8; ++kk) {
+          const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
+          mma_ss_tf32(tacc, ah + kk * a_step, bh + kk * b_step, idesc, acc);
+          mma_ss_tf32(tacc, ah + kk * a_step, bl + kk * b_step, idesc, 1u);
+          mma_ss_tf32(tacc, al + kk * a_step, bh + kk * b_step, idesc, 1u);
+        }
+        tc_commit(&s.empty[st]);
+      }
+      if (ok) tc_commit(&s.acc_full);
+      else { tc_commit(&s.drain); drain_wait(&s.drain, 0, p.status); }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------- split, then epilogue
+    const int et = threadIdx.x - 64;   // 0..127
+    bool ok = true;
+    for (int n = 0; n < nk; ++n) {
+      const int st = n % NSTAGE;
+      if (!mbar_wait(&s.full[st], (n / NSTAGE) & 1, p.status, abort_flag)) { ok = false; break; }
+#pragma unroll 4
+      for (int v = et; v < 2 * kSlab / 16; v += 128) {
+        const bool is_b = v >= kSlab / 16;
+        const int off = (is_b ? v - kSlab / 16 : v) * 16;
+        float4* hi = reinterpret_cast<float4*>((is_b ? s.b_hi[st] : s.a_hi[st]) + off);
+        float4* lo = reinterpret_cast<float4*>((is_b ? s.b_lo[st] : s.a_lo[st]) + off);
+        const float4 x = *hi;
+        float4 h, l;
+        h.x = to_tf32(x.x); l.x = to_tf32(x.x - h.x);
+        h.y = to_tf32(x.y); l.y = to_tf32(x.y - h.y);
+        h.z = to_tf32(x.z); l.z = to_tf32(x.z - h.z);
+        h.w = to_tf32(x.w); l.w = to_tf32(x.w - h.w);
+        *hi = h;
+        *lo = l;
+      }
+      fence_proxy_async_smem();   // generic-proxy writes -> visible to the MMA (async proxy)
+      mbar_arrive(&s.split[st]);
+    }
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const int64_t row = (int64_t)pr.c_row0 + (int64_t)ti * TM + r;
+    const int64_t col0 = (int64_t)pr.c_col0 + (int64_t)tj * TN;
+    if (ok && (nk == 0 || mbar_wait(&s.acc_full, 0, p.status, abort_flag))) {
+      tc_fence_after();
+      if (pr.mode == kModeStore) {
+        float* crow = pr.C + row * pr.ldc + col0;
+        const float alpha = pr.alpha, beta = pr.beta;
+#pragma unroll 1
+        for (int c = 0; c < TN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tacc + lane_off + c * 32, v);
+          tmem_ld_wait();
+          float4* dst = reinterpret_cast<float4*>(crow + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float4 o;
+            o.x = nk > 0 ? alpha * __uint_as_float(v[4 * i]) : 0.f;
+            o.y = nk > 0 ? alpha * __uint_as_float(v[4 * i + 1]) : 0.f;
+            o.z = nk > 0 ? alpha * __uint_as_float(v[4 * i + 2]) : 0.f;
+            o.w = nk > 0 ? alpha * __uint_as_float(v[4 * i + 3]) : 0.f;
+            if (beta != 0.f) {
+              const float4 old = dst[i];
+              o.x = fmaf(beta, old.x, o.x);
+              o.y = fmaf(beta, old.y, o.y);
+              o.z = fmaf(beta, old.z, o.z);
+              o.w = fmaf(beta, old.w, o.w);
+            }
+            dst[i] = o;
+          }
+        }
+      } else {
+        // kModeDot3: <P, G>, <P, R>, <P, S> for this tile of P = op(A) op(B),
+        // G and S weighted for their stored upper tiles (2 above, 1 on the
+        // diagonal, 0 below), accumulated in fp64.
+        const int64_t ld = 2 * (int64_t)p.dot_dim;
+        const double wsym = ti < tj ? 2.0 : (ti == tj ? 1.0 : 0.0);
+        double g = 0.0, rr = 0.0, sv = 0.0;
+        const float* Mr = p.dot_M + row * ld;
+        const float* Sr = p.dot_M + (row + p.dot_dim) * ld + p.dot_dim;
+#pragma unroll 1
+        for (int c = 0; c < TN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tacc + lane_off + c * 32, v);
+          tmem_ld_wait();
+          const int64_t cc = col0 + c * 32;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const double pij = __uint_as_float(v[i]);
+            rr += (double)Mr[p.dot_dim + cc + i] * pij;
+            if (wsym != 0.0) {
+              g += (double)Mr[cc + i] * pij;
+              sv += (double)Sr[cc + i] * pij;
+            }
+          }
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+          g += __shfl_xor_sync(0xffffffffu, g, o);
+          rr += __shfl_xor_sync(0xffffffffu, rr, o);
+          sv += __shfl_xor_sync(0xffffffffu, sv, o);
+        }
+        if (lane == 0) {
+          atomicAdd(p.dot_acc + 0, g * wsym);
+          atomicAdd(p.dot_acc + 1, rr);
+          atomicAdd(p.dot_acc + 2, sv * wsym);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tacc, TN);
+}
+
+}  // namespace
+
+size_t tgemm_smem_bytes() { return sizeof(GSmem) + 1024; }
+
+cudaError_t launch_tgemm(TGemmParams& p, cudaStream_t stream) {
+  int base = 0;
+  for (int q = 0; q < p.nprob; ++q) {
+    TGemmProblem& pr = p.prob[q];
+    pr.mt = pr.M / TM;
+    pr.nt = pr.N / TN;
+    pr.tile_base = base;
+    base += pr.lower ? pr.mt * (pr.mt + 1) / 2 : pr.mt * pr.nt;
+  }
+  if (base == 0) return cudaSuccess;
+  const size_t smem = tgemm_smem_bytes();
+  cudaFuncSetAttribute(tgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  tgemm_kernel<<<base, kThreads, smem, stream>>>(p);
+  count_launches();
+  return cudaGetLastError();
+}
+
+}  // namespace ispa

@@ -1,0 +1,48 @@
+// Problem description of the 3xTF32 tensor-core GEMM (tgemm.cu).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace ispa {
+
+constexpr int kTriNone = 0;
+constexpr int kTriLowerA = 1;   // op(A) lower triangular: row block i reads K blocks 0..i
+constexpr int kTriUpperA = 2;   // op(A) upper triangular: row block i reads K blocks i..
+constexpr int kModeStore = 0;   // C = alpha * op(A) op(B) + beta * C
+constexpr int kModeDot3 = 1;    // accumulate <P, G>, <P, R>, <P, S> (P = op(A) op(B))
+
+// C[M x N] (+)= op(A)[M x K] op(B)[K x N]; M, N multiples of 128, K of 32.
+// op(A) is read from tensor map ta: K-major when a_mn == 0 (stored [M][K]),
+// MN-major when a_mn == 1 (stored [K][M]); op(B) from tb: MN-major when
+// b_mn == 1 (stored [K][N]), K-major when b_mn == 0 (stored [N][K]).
+// a_row0 / a_k0 / b_col0 / b_k0 offset the tiles inside the mapped tensors.
+struct TGemmProblem {
+  CUtensorMap ta;
+  CUtensorMap tb;
+  int a_mn, b_mn;
+  int M, N, K;
+  int a_row0, a_k0, b_col0, b_k0;
+  float* C;
+  int64_t ldc;
+  int c_row0, c_col0;
+  float alpha, beta;
+  int lower;     // only tiles (i, j) with j <= i
+  int tri;       // kTri*
+  int mode;      // kMode*
+  int mt, nt, tile_base;   // set by launch_tgemm
+};
+
+struct TGemmParams {
+  TGemmProblem prob[4];
+  int nprob;
+  const float* dot_M;   // kModeDot3: the [2d, 2d] Gram blocks
+  int dot_dim;
+  double* dot_acc;      // kModeDot3: 3 accumulators
+  int* status;
+};
+
+size_t tgemm_smem_bytes();
+cudaError_t launch_tgemm(TGemmParams& p, cudaStream_t stream);
+
+}  // namespace ispa
