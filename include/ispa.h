@@ -167,6 +167,30 @@ ISPA_API int ispa_absorb_solve(const float* M, const float* W, int dim, float la
                       float* lambda_out, void* workspace, size_t workspace_bytes, int* dev_status,
                       void* stream);
 
+/* ---- 3b. absorb solve without device allocation -------------------------
+ * The paper has no counterpart to this entry point: it is an interface
+ * variant of ispa_absorb_solve (same arithmetic, same kernels, same
+ * arguments and results) that needs no caller workspace. It exists for
+ * callers that cannot allocate device memory at the moment they need a
+ * solve, e.g. a host program that manages every device buffer itself and
+ * has no allocator to call, or a latency-critical loop that must never
+ * enter an allocator. The solve's scratch lives in a device array inside
+ * the library instead.
+ * Limits: dim must be a multiple of 128 and at most 512; larger dims return
+ * ISPA_ERR_UNSUPPORTED. The array (about 3.2 MB) is held by every GPU that
+ * loads the library until the process exits.
+ * Set-up: the first call on a device looks up the array's device address
+ * (once per device, with that device current); make that first call before
+ * any stream capture.
+ * Sharing: all calls use the same array, so calls that overlap on the GPU
+ * (other streams, other host threads) race; serialise them. The array keeps
+ * the last call's contents, which needs no clearing: each solve writes every
+ * scratch buffer before reading it.
+ */
+ISPA_API int ispa_absorb_solve_noalloc(const float* M, const float* W, int dim, float lambda,
+                                       float* dW, float* B, float* lambda_out, int* dev_status,
+                                       void* stream);
+
 /* ---- 4. reconstruction error and layer ranking -------------------------
  * Technical summary section 2, "Dynamic layer selection": every layer's
  * error after absorption, then an ascending ranking over layers; the K

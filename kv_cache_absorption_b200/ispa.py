@@ -32,6 +32,7 @@ EXPORTED = (
     "ispa_status_string", "ispa_version", "ispa_kernel_launches",
     "ispa_dual_attention_workspace_size", "ispa_dual_attention", "ispa_local_attention",
     "ispa_gram_accumulate", "ispa_absorb_workspace_size", "ispa_absorb_solve",
+    "ispa_absorb_solve_noalloc",
     "ispa_layer_error_workspace_size", "ispa_layer_error", "ispa_rank_layers",
 )
 
@@ -70,6 +71,7 @@ def _load():
         "ispa_gram_accumulate": (I, [P, P, I64, I, P, I, I, P]),
         "ispa_absorb_workspace_size": (SZ, [I]),
         "ispa_absorb_solve": (I, [P, P, I, F, P, P, P, P, SZ, P, P]),
+        "ispa_absorb_solve_noalloc": (I, [P, P, I, F, P, P, P, P, P]),
         "ispa_layer_error_workspace_size": (SZ, [I]),
         "ispa_layer_error": (I, [P, P, P, P, P, I, P, P, SZ, P]),
         "ispa_rank_layers": (I, [P, I, I, P, P, P]),
@@ -253,6 +255,27 @@ def ispa_absorb_solve(M, W, lam: float = 0.0, workspace=None, status=None, strea
                                    workspace.numel() * workspace.element_size(), _ptr(status),
                                    _stream(stream))
     _check(rc, "ispa_absorb_solve")
+    return {"dW": dW, "B": B, "lam": lam_out, "status": status}
+
+
+def ispa_absorb_solve_noalloc(M, W, lam: float = 0.0, status=None, stream=None) -> dict:
+    """ispa_absorb_solve without a workspace, for callers that cannot allocate
+    device memory when they solve: the scratch is an array inside the library
+    (dim <= 512; concurrent calls on one GPU race). The output buffers are
+    allocated here only because this binding returns new tensors."""
+    _dev_tensor(M, torch.float32, "M", 2)
+    _dev_tensor(W, torch.float32, "W", 2)
+    dim = W.shape[0]
+    if tuple(M.shape) != (2 * dim, 2 * dim) or W.shape[1] != dim:
+        raise ValueError("M must be [2d, 2d] and W [d, d]")
+    dev = W.device
+    dW = torch.empty(dim, dim, dtype=torch.float32, device=dev)
+    B = torch.empty(dim, dim, dtype=torch.float32, device=dev)
+    lam_out = torch.empty(1, dtype=torch.float32, device=dev)
+    status = new_status(dev) if status is None else status
+    rc = _load().ispa_absorb_solve_noalloc(_ptr(M), _ptr(W), dim, float(lam), _ptr(dW), _ptr(B),
+                                           _ptr(lam_out), _ptr(status), _stream(stream))
+    _check(rc, "ispa_absorb_solve_noalloc")
     return {"dW": dW, "B": B, "lam": lam_out, "status": status}
 
 
