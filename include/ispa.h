@@ -167,6 +167,26 @@ ISPA_API int ispa_absorb_solve(const float* M, const float* W, int dim, float la
                       float* lambda_out, void* workspace, size_t workspace_bytes, int* dev_status,
                       void* stream);
 
+/* ---- 3c. absorb solves of many layers in one call ---------------------
+ * Technical summary section 2, step 2: at the transition every layer gets
+ * its own Delta W, and the layers are independent; this call solves
+ * n_layers of them together so that each step of the factorisation is one
+ * launch for all layers (same arithmetic and results as ispa_absorb_solve
+ * per layer).
+ * Layer l reads M + l * m_layer_stride and W + l * w_layer_stride and writes
+ * dW + l * dw_layer_stride, B + l * b_layer_stride and lambda_out[l]
+ * (device float [n_layers], optional). Strides are in elements, multiples
+ * of 4 and at least one matrix (4 d^2 for M, d^2 for the others).
+ * workspace: >= n_layers * ispa_absorb_workspace_size(dim) bytes, 256-byte
+ * aligned. 1 <= n_layers <= 4096; other rules as ispa_absorb_solve.
+ */
+ISPA_API int ispa_absorb_solve_batched(int n_layers, const float* M, int64_t m_layer_stride,
+                                       const float* W, int64_t w_layer_stride, int dim,
+                                       float lambda, float* dW, int64_t dw_layer_stride,
+                                       float* B, int64_t b_layer_stride, float* lambda_out,
+                                       void* workspace, size_t workspace_bytes, int* dev_status,
+                                       void* stream);
+
 /* ---- 3b. absorb solve without device allocation -------------------------
  * The paper has no counterpart to this entry point: it is an interface
  * variant of ispa_absorb_solve (same arithmetic, same kernels, same
@@ -220,6 +240,16 @@ ISPA_API size_t ispa_layer_error_workspace_size(int dim);
 ISPA_API int ispa_layer_error(const float* M, const float* W, const float* dW, const float* B,
                      const float* lambda, int dim, double* err, void* workspace,
                      size_t workspace_bytes, void* stream);
+/* Many layers at once (same per-layer result as ispa_layer_error): layer l
+ * reads the buffers at the given element strides (as in
+ * ispa_absorb_solve_batched) and lambdas[l], and writes err[2 l], err[2 l + 1].
+ * workspace: >= n_layers * ispa_layer_error_workspace_size(dim) bytes. */
+ISPA_API int ispa_layer_error_batched(int n_layers, const float* M, int64_t m_layer_stride,
+                                      const float* W, int64_t w_layer_stride, const float* dW,
+                                      int64_t dw_layer_stride, const float* B,
+                                      int64_t b_layer_stride, const float* lambdas, int dim,
+                                      double* err, void* workspace, size_t workspace_bytes,
+                                      void* stream);
 ISPA_API int ispa_rank_layers(const double* err, int n_layers, int K, int* perm, uint8_t* selected,
                      void* stream);
 

@@ -19,6 +19,14 @@ cudaError_t absorb_solve(const float* M, const float* W, int dim, float lambda, 
                          cudaStream_t stream);
 cudaError_t layer_error(const float* M, const float* W, const float* dW, const float* B,
                         const float* lam, int dim, double* err, double* acc, cudaStream_t stream);
+cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const float* W,
+                                 int64_t w_stride, int dim, float lambda, float* dW,
+                                 int64_t dw_stride, float* B, int64_t b_stride, float* lambda_out,
+                                 void* workspace, int* status, cudaStream_t stream);
+cudaError_t layer_error_batched(int n, const float* M, int64_t m_stride, const float* W,
+                                int64_t w_stride, const float* dW, int64_t dw_stride,
+                                const float* B, int64_t b_stride, const float* lam, int dim,
+                                double* err, double* acc, cudaStream_t stream);
 cudaError_t rank_layers(const double* err, int n, int K, int* perm, uint8_t* selected,
                         cudaStream_t stream);
 }  // namespace ispa
@@ -237,6 +245,63 @@ int ispa_absorb_solve(const float* M, const float* W, int dim, float lambda, flo
   if (rc != ISPA_OK) return rc;
   return cuda_rc(ispa::absorb_solve(M, W, dim, lambda, dW, B, lambda_out, workspace, dev_status,
                                     static_cast<cudaStream_t>(stream)));
+}
+
+// Layer strides (elements) of batched calls: multiples of 4 (16-byte TMA
+// alignment) and at least one matrix apart.
+static bool stride_ok(int64_t stride, int64_t min_elems) {
+  return stride >= min_elems && stride % 4 == 0;
+}
+
+int ispa_absorb_solve_batched(int n_layers, const float* M, int64_t m_layer_stride,
+                              const float* W, int64_t w_layer_stride, int dim, float lambda,
+                              float* dW, int64_t dw_layer_stride, float* B,
+                              int64_t b_layer_stride, float* lambda_out, void* workspace,
+                              size_t workspace_bytes, int* dev_status, void* stream) {
+  if (n_layers < 1 || n_layers > 4096 || !M || !W || !dW || !B || !dev_status || dim <= 0 ||
+      lambda != lambda)
+    return ISPA_ERR_ARG;
+  if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
+  const int64_t dd = (int64_t)dim * dim;
+  if (!stride_ok(m_layer_stride, 4 * dd) || !stride_ok(w_layer_stride, dd) ||
+      !stride_ok(dw_layer_stride, dd) || !stride_ok(b_layer_stride, dd))
+    return ISPA_ERR_ARG;
+  if (!aligned16(M) || !aligned16(W) || !aligned16(dW) || !aligned16(B))
+    return ISPA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned256(workspace) ||
+      workspace_bytes / (size_t)n_layers < ispa::absorb_workspace_bytes(dim))
+    return ISPA_ERR_WORKSPACE;
+  int rc = check_device();
+  if (rc != ISPA_OK) return rc;
+  return cuda_rc(ispa::absorb_solve_batched(n_layers, M, m_layer_stride, W, w_layer_stride, dim,
+                                            lambda, dW, dw_layer_stride, B, b_layer_stride,
+                                            lambda_out, workspace, dev_status,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+int ispa_layer_error_batched(int n_layers, const float* M, int64_t m_layer_stride,
+                             const float* W, int64_t w_layer_stride, const float* dW,
+                             int64_t dw_layer_stride, const float* B, int64_t b_layer_stride,
+                             const float* lambdas, int dim, double* err, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  if (n_layers < 1 || n_layers > 4096 || !M || !W || !dW || !B || !lambdas || !err || dim <= 0)
+    return ISPA_ERR_ARG;
+  if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
+  const int64_t dd = (int64_t)dim * dim;
+  if (!stride_ok(m_layer_stride, 4 * dd) || !stride_ok(w_layer_stride, dd) ||
+      !stride_ok(dw_layer_stride, dd) || !stride_ok(b_layer_stride, dd))
+    return ISPA_ERR_ARG;
+  if (!aligned16(M) || !aligned16(W) || !aligned16(dW) || !aligned16(B))
+    return ISPA_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes / (size_t)n_layers < 256 ||
+      (reinterpret_cast<uintptr_t>(workspace) & 7u))
+    return ISPA_ERR_WORKSPACE;
+  int rc = check_device();
+  if (rc != ISPA_OK) return rc;
+  return cuda_rc(ispa::layer_error_batched(n_layers, M, m_layer_stride, W, w_layer_stride, dW,
+                                           dw_layer_stride, B, b_layer_stride, lambdas, dim, err,
+                                           static_cast<double*>(workspace),
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 size_t ispa_layer_error_workspace_size(int dim) { return dim > 0 ? 256 : 0; }

@@ -35,10 +35,14 @@ __device__ __forceinline__ double block_sum(double v, double* red) {
   return s;
 }
 
-// acc[3] += <dW, B>, acc[4] += ||dW||^2
-__global__ void dot_kernel(const float4* __restrict__ dW, const float4* __restrict__ B, size_t n4,
-                           double* __restrict__ acc) {
+// acc[3] += <dW, B>, acc[4] += ||dW||^2; layer blockIdx.y
+__global__ void dot_kernel(const float4* __restrict__ dW0, int64_t dw_stride4,
+                           const float4* __restrict__ B0, int64_t b_stride4, size_t n4,
+                           double* __restrict__ acc0) {
   __shared__ double red[8];
+  const float4* dW = dW0 + (int64_t)blockIdx.y * dw_stride4;
+  const float4* B = B0 + (int64_t)blockIdx.y * b_stride4;
+  double* acc = acc0 + 5 * (int64_t)blockIdx.y;
   double db = 0.0, dd = 0.0;
   for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n4;
        e += (size_t)gridDim.x * blockDim.x) {
@@ -54,13 +58,16 @@ __global__ void dot_kernel(const float4* __restrict__ dW, const float4* __restri
   }
 }
 
-__global__ void finalize_kernel(const double* __restrict__ acc, const float* __restrict__ lam,
-                                double* __restrict__ err) {
-  const double l = *lam;
-  const double e2 = acc[2] - acc[3] - l * acc[4];
+__global__ void finalize_kernel(int n, const double* __restrict__ acc0,
+                                const float* __restrict__ lam, double* __restrict__ err) {
+  const int l = blockIdx.x * blockDim.x + threadIdx.x;
+  if (l >= n) return;
+  const double* acc = acc0 + 5 * l;
+  const double lv = lam[l];
+  const double e2 = acc[2] - acc[3] - lv * acc[4];
   const double den = acc[0] + 2.0 * acc[1] + acc[2];
-  err[0] = e2;
-  err[1] = e2 / den;
+  err[2 * l] = e2;
+  err[2 * l + 1] = e2 / den;
 }
 
 // Stable ascending rank of the relative errors err[2 l + 1]: layer i lands at
@@ -81,35 +88,47 @@ __global__ void rank_kernel(const double* __restrict__ err, int n, int K, int* _
 
 }  // namespace
 
-cudaError_t layer_error(const float* M, const float* W, const float* dW, const float* B,
-                        const float* lam, int dim, double* err, double* acc,
-                        cudaStream_t stream) {
-  cudaMemsetAsync(acc, 0, 5 * sizeof(double), stream);
+cudaError_t layer_error_batched(int n, const float* M, int64_t m_stride, const float* W,
+                                int64_t w_stride, const float* dW, int64_t dw_stride,
+                                const float* B, int64_t b_stride, const float* lam, int dim,
+                                double* err, double* acc, cudaStream_t stream) {
+  cudaMemsetAsync(acc, 0, 5 * (size_t)n * sizeof(double), stream);
   {
     TGemmParams p{};
     p.nprob = 1;
     p.dot_M = M;
+    p.dot_m_stride = m_stride;
     p.dot_dim = dim;
     p.dot_acc = acc;
+    p.dot_acc_stride = 5;
     TGemmProblem& pr = p.prob[0];
     // P = W W^T: op(A) = W (K-major), op(B) = W^T, i.e. W read K-major
-    if (!encode_f32_operand(&pr.ta, W, dim, dim, dim, false) ||
-        !encode_f32_operand(&pr.tb, W, dim, dim, dim, false))
+    if (!encode_f32_operand_3d(&pr.ta, W, dim, dim, dim, n, w_stride, false) ||
+        !encode_f32_operand_3d(&pr.tb, W, dim, dim, dim, n, w_stride, false))
       return cudaErrorInvalidValue;
     pr.a_mn = 0;
     pr.b_mn = 0;
     pr.M = pr.N = pr.K = dim;
     pr.mode = kModeDot3;
     pr.alpha = 1.f;
+    pr.layers = n;
     cudaError_t e = launch_tgemm(p, stream);
     if (e != cudaSuccess) return e;
   }
   const size_t n4 = (size_t)dim * dim / 4;
-  dot_kernel<<<148 * 2, 256, 0, stream>>>(reinterpret_cast<const float4*>(dW),
-                                          reinterpret_cast<const float4*>(B), n4, acc);
-  finalize_kernel<<<1, 1, 0, stream>>>(acc, lam, err);
+  dot_kernel<<<dim3(n == 1 ? 148 * 2 : 148, n), 256, 0, stream>>>(
+      reinterpret_cast<const float4*>(dW), dw_stride / 4, reinterpret_cast<const float4*>(B),
+      b_stride / 4, n4, acc);
+  finalize_kernel<<<(n + 127) / 128, 128, 0, stream>>>(n, acc, lam, err);
   count_launches(2);
   return cudaGetLastError();
+}
+
+cudaError_t layer_error(const float* M, const float* W, const float* dW, const float* B,
+                        const float* lam, int dim, double* err, double* acc,
+                        cudaStream_t stream) {
+  const int64_t dd = (int64_t)dim * dim;
+  return layer_error_batched(1, M, 4 * dd, W, dd, dW, dd, B, dd, lam, dim, err, acc, stream);
 }
 
 cudaError_t rank_layers(const double* err, int n, int K, int* perm, uint8_t* selected,

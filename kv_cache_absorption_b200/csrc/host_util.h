@@ -18,4 +18,9 @@ bool encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esi
 bool encode_f32_operand(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols,
                         uint64_t ld, bool mn_major);
 
+// fp32 operand maps over `layers` matrices spaced `layer_stride` elements
+// apart (3-D: x = column, y = row, z = layer); same boxes as above.
+bool encode_f32_operand_3d(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols,
+                           uint64_t ld, uint64_t layers, uint64_t layer_stride, bool mn_major);
+
 }  // namespace ispa

@@ -29,10 +29,13 @@ namespace {
 
 constexpr int NB = 128;
 
-// lambda = value if value > 0, else 1e-2 * trace(G) / dim (G = M[0:d, 0:d]).
-__global__ void lambda_kernel(const float* __restrict__ M, int dim, float value, float* lam_ws,
-                              float* lam_out) {
+// lambda = value if value > 0, else 1e-2 * trace(G) / dim (G = M[0:d, 0:d]);
+// one block per layer.
+__global__ void lambda_kernel(const float* __restrict__ M0, int64_t m_stride, int dim, float value,
+                              float* lam_ws0, int64_t ws_stride, float* lam_out) {
   __shared__ double part[256];
+  const float* M = M0 + (int64_t)blockIdx.x * m_stride;
+  float* lam_ws = lam_ws0 + (int64_t)blockIdx.x * ws_stride;
   double s = 0.0;
   if (!(value > 0.f))
     for (int i = threadIdx.x; i < dim; i += blockDim.x) s += M[(size_t)i * 2 * dim + i];
@@ -45,16 +48,19 @@ __global__ void lambda_kernel(const float* __restrict__ M, int dim, float value,
   if (threadIdx.x == 0) {
     const float lam = value > 0.f ? value : (float)(1e-2 * part[0] / dim);
     *lam_ws = lam;
-    if (lam_out) *lam_out = lam;
+    if (lam_out) lam_out[blockIdx.x] = lam;
   }
 }
 
 // A = G + lambda I as a full symmetric matrix (G's 128 x 128 tiles are valid
-// on and above the tile diagonal; the rest is mirrored), Z = I.
-__global__ void build_kernel(const float* __restrict__ M, int dim, const float* lam,
-                             float* __restrict__ A, float* __restrict__ Z) {
+// on and above the tile diagonal; the rest is mirrored), Z = I; layer blockIdx.y.
+__global__ void build_kernel(const float* __restrict__ M0, int64_t m_stride, int dim,
+                             float* __restrict__ ws0, int64_t ws_stride, int64_t lam_off) {
   const size_t n = (size_t)dim * dim;
-  const float l = *lam;
+  const float* M = M0 + (int64_t)blockIdx.y * m_stride;
+  float* A = ws0 + (int64_t)blockIdx.y * ws_stride;
+  float* Z = A + n;
+  const float l = A[lam_off];
   for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n;
        e += (size_t)gridDim.x * blockDim.x) {
     const int i = (int)(e / dim), j = (int)(e % dim);
@@ -65,105 +71,142 @@ __global__ void build_kernel(const float* __restrict__ M, int dim, const float* 
 }
 
 // Factors the 128 x 128 diagonal block at A (lower triangle used) as L L^T
-// and writes Linv = L^-1 (lower, zero above) to `linv`, in fp32 shared
-// memory. Right-looking in 8-column panels, with the inverse carried along:
-//  * inside a panel, column j updates the later panel columns and the later
-//    panel rows of the inverse using UNSCALED values, a_ij a_cj / a_jj and
-//    a_ij z_jc / a_jj, so every column needs one barrier and no divide-then-
-//    use round trip;
-//  * the panel is then scaled by 1/sqrt(a_jj) (giving its L columns and its
-//    Linv rows) and copied to an aligned buffer;
-//  * one blocked update applies the whole panel to the trailing lower
-//    triangle of A and to the rows of the inverse below it.
-__global__ void __launch_bounds__(512) potrf_inv_kernel(const float* __restrict__ A, int lda,
-                                                        float* __restrict__ linv, int* status) {
+// and writes Linv = L^-1 (lower, zero above) to `linv`, in fp32, right-
+// looking in 8-column panels:
+//  * warp 0 factors the panel (all rows at or below it) in registers: lane l
+//    holds rows l, l+32, l+64, l+96 of the panel's 8 columns; pivots and
+//    panel rows travel by warp shuffles, so a column step needs no barrier;
+//  * one thread per column c then forms the panel's 8 rows of Linv by
+//    forward substitution with the 8 x 8 diagonal block of L;
+//  * all threads apply the panel to the trailing lower triangle of A and to
+//    the rows of Linv below the panel (4 threads per row).
+__global__ void __launch_bounds__(512) potrf_inv_kernel(const float* __restrict__ A0, int lda,
+                                                        float* __restrict__ linv0,
+                                                        int64_t ws_stride, int* status) {
   constexpr int W = 8;
+  const float* A = A0 + (int64_t)blockIdx.x * ws_stride;    // one block per layer
+  float* linv = linv0 + (int64_t)blockIdx.x * ws_stride;
   extern __shared__ float sh[];
   float (*a)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(sh);
   float (*z)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(sh + NB * (NB + 1));
-  float4 (*pan)[W / 4] = reinterpret_cast<float4 (*)[W / 4]>(sh + 2 * NB * (NB + 1));  // [NB][2]
-  __shared__ float dv[NB];
-  const int t = threadIdx.x;
+  float (*pan)[W] = reinterpret_cast<float (*)[W]>(sh + 2 * NB * (NB + 1));   // [NB][8], L of the panel
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   for (int e = t; e < NB * NB; e += blockDim.x) {
-    const int i = e / NB, c = e % NB;
+    const int i = e >> 7, c = e & (NB - 1);
     a[i][c] = A[(size_t)i * lda + c];
     z[i][c] = (i == c) ? 1.f : 0.f;
   }
   __syncthreads();
   for (int J = 0; J < NB; J += W) {
-    // ---- panel columns J .. J+W-1
-    for (int j = J; j < J + W; ++j) {
-      const float piv = a[j][j];
-      const float ip = 1.f / piv;
-      if (t == 0) {
-        if (!(piv > 0.f)) atomicOr(status, ISPA_STATUS_NOT_SPD);
-        dv[j] = rsqrtf(piv);   // NaN for a non-positive pivot: poisons what follows
-      }
-      const int cols = J + W - 1 - j;                  // later panel columns
-      const int rows = NB - 1 - j;                     // rows below j
-      for (int e = t; e < rows * cols; e += blockDim.x) {
-        const int i = j + 1 + e / cols, c = j + 1 + e % cols;
-        if (c <= i) a[i][c] -= a[i][j] * a[c][j] * ip;
-      }
-      const int zr = J + W - 1 - j;                    // later panel rows of the inverse
-      for (int e = t; e < zr * (j + 1); e += blockDim.x) {
-        const int i = j + 1 + e / (j + 1), c = e % (j + 1);
-        z[i][c] -= a[i][j] * z[j][c] * ip;
-      }
-      __syncthreads();
-    }
-    // ---- scale the panel: L columns and Linv rows; aligned copy of L rows
-    for (int e = t; e < (NB - J) * W; e += blockDim.x) {
-      const int i = J + e / W, m = e % W, j = J + m;
-      if (i >= j) a[i][j] *= dv[j];
-    }
-    for (int e = t; e < W * (J + W); e += blockDim.x) {
-      const int m = e / (J + W), c = e % (J + W), j = J + m;
-      if (c <= j) z[j][c] *= dv[j];
-    }
-    __syncthreads();
-    for (int i = J + W + t; i < NB; i += blockDim.x) {
-      pan[i][0] = make_float4(a[i][J], a[i][J + 1], a[i][J + 2], a[i][J + 3]);
-      pan[i][1] = make_float4(a[i][J + 4], a[i][J + 5], a[i][J + 6], a[i][J + 7]);
-    }
-    __syncthreads();
-    // ---- trailing: A_ic -= sum_m L_im L_cm (c <= i), Z_ic -= sum_m L_im Linv_mc
-    const int n = NB - J - W;
-    for (int e = t; e < n * NB; e += blockDim.x) {
-      const int i = J + W + e / NB, c = e % NB;
-      const float4 p0 = pan[i][0], p1 = pan[i][1];
-      if (c >= J + W) {
-        if (c <= i) {
-          const float4 q0 = pan[c][0], q1 = pan[c][1];
-          float acc = a[i][c];
-          acc -= p0.x * q0.x + p0.y * q0.y + p0.z * q0.z + p0.w * q0.w;
-          acc -= p1.x * q1.x + p1.y * q1.y + p1.z * q1.z + p1.w * q1.w;
-          a[i][c] = acc;
+    // ---- (1) warp 0: factor the panel columns J..J+7 for rows J..127
+    if (warp == 0) {
+      float r[4][W];
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+#pragma unroll
+        for (int m = 0; m < W; ++m) r[s][m] = a[lane + 32 * s][J + m];
+      const int ps = J >> 5;           // slot of the panel's rows (J..J+7 lie in one slot)
+#pragma unroll
+      for (int m = 0; m < W; ++m) {
+        const int j = J + m;
+        // pivot a_jj lives in lane j % 32, slot ps, column m
+        float own = r[0][m];
+        if (ps == 1) own = r[1][m];
+        if (ps == 2) own = r[2][m];
+        if (ps == 3) own = r[3][m];
+        const float piv = __shfl_sync(0xffffffffu, own, j & 31);
+        if (lane == 0 && !(piv > 0.f)) atomicOr(status, ISPA_STATUS_NOT_SPD);
+        const float sc = rsqrtf(piv);  // NaN for a non-positive pivot: poisons what follows
+        // scale column m of rows >= j: L_ij = a_ij / sqrt(a_jj)
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+          if (lane + 32 * s >= j) r[s][m] *= sc;
+        // update later panel columns: a_ic -= L_ij L_cj for rows i > j, c > j
+#pragma unroll
+        for (int cc = m + 1; cc < W; ++cc) {
+          float oc = r[0][m];
+          if (ps == 1) oc = r[1][m];
+          if (ps == 2) oc = r[2][m];
+          if (ps == 3) oc = r[3][m];
+          const float lcj = __shfl_sync(0xffffffffu, oc, (J + cc) & 31);   // L_{c j}, c = J + cc
+#pragma unroll
+          for (int s = 0; s < 4; ++s)
+            if (lane + 32 * s >= J + cc) r[s][cc] -= r[s][m] * lcj;
         }
-      } else {
-        float acc = z[i][c];
-        acc -= p0.x * z[J][c] + p0.y * z[J + 1][c] + p0.z * z[J + 2][c] + p0.w * z[J + 3][c];
-        acc -= p1.x * z[J + 4][c] + p1.y * z[J + 5][c] + p1.z * z[J + 6][c] + p1.w * z[J + 7][c];
-        z[i][c] = acc;
+      }
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const int i = lane + 32 * s;
+        if (i >= J)
+#pragma unroll
+          for (int m = 0; m < W; ++m) {
+            a[i][J + m] = r[s][m];
+            pan[i][m] = r[s][m];
+          }
+      }
+    }
+    __syncthreads();
+    // ---- (2) rows J..J+7 of Linv: forward substitution per column c <= J+7
+    if (t < J + W) {
+      const int c = t;
+      float zr[W];
+#pragma unroll
+      for (int m = 0; m < W; ++m) zr[m] = z[J + m][c];
+#pragma unroll
+      for (int m = 0; m < W; ++m) {
+#pragma unroll
+        for (int q = 0; q < m; ++q) zr[m] -= pan[J + m][q] * zr[q];
+        zr[m] /= pan[J + m][m];
+      }
+#pragma unroll
+      for (int m = 0; m < W; ++m) z[J + m][c] = zr[m];
+    }
+    __syncthreads();
+    // ---- (3) trailing: Z_ic -= sum_m L_im Linv_mc (c < J+8), A_ic -= sum_m L_im L_cm (J+8 <= c <= i)
+    const int ri = t >> 2, rq = t & 3;
+    if (ri >= J + W) {
+      float p[W];
+      {
+        const float4 v0 = *reinterpret_cast<const float4*>(&pan[ri][0]);
+        const float4 v1 = *reinterpret_cast<const float4*>(&pan[ri][4]);
+        p[0] = v0.x; p[1] = v0.y; p[2] = v0.z; p[3] = v0.w;
+        p[4] = v1.x; p[5] = v1.y; p[6] = v1.z; p[7] = v1.w;
+      }
+#pragma unroll 4
+      for (int c = rq; c < J + W; c += 4) {
+        float acc = z[ri][c];
+#pragma unroll
+        for (int m = 0; m < W; ++m) acc -= p[m] * z[J + m][c];
+        z[ri][c] = acc;
+      }
+#pragma unroll 4
+      for (int c = J + W + rq; c <= ri; c += 4) {
+        const float4 q0 = *reinterpret_cast<const float4*>(&pan[c][0]);
+        const float4 q1 = *reinterpret_cast<const float4*>(&pan[c][4]);
+        float acc = a[ri][c];
+        acc -= p[0] * q0.x + p[1] * q0.y + p[2] * q0.z + p[3] * q0.w;
+        acc -= p[4] * q1.x + p[5] * q1.y + p[6] * q1.z + p[7] * q1.w;
+        a[ri][c] = acc;
       }
     }
     __syncthreads();
   }
   for (int e = t; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e % NB;
+    const int r = e >> 7, c = e & (NB - 1);
     linv[e] = c <= r ? z[r][c] : 0.f;
   }
 }
 
 constexpr size_t kPotrfSmem = (2 * NB * (NB + 1) + NB * 8) * sizeof(float) + 16;
 
-void set_store(TGemmProblem& pr, int M, int N, int K, float* C, int64_t ldc, int c_row0,
-               int c_col0, float alpha, float beta) {
+void set_store(TGemmProblem& pr, int M, int N, int K, float* C, int64_t ldc, int64_t c_stride,
+               int c_row0, int c_col0, float alpha, float beta, int layers) {
   pr.M = M;
   pr.N = N;
   pr.K = K;
   pr.C = C;
   pr.ldc = ldc;
+  pr.c_layer_stride = c_stride;
   pr.c_row0 = c_row0;
   pr.c_col0 = c_col0;
   pr.alpha = alpha;
@@ -171,33 +214,46 @@ void set_store(TGemmProblem& pr, int M, int N, int K, float* C, int64_t ldc, int
   pr.lower = 0;
   pr.tri = kTriNone;
   pr.mode = kModeStore;
+  pr.layers = layers;
   pr.a_row0 = pr.a_k0 = pr.b_col0 = pr.b_k0 = 0;
+}
+
+// Operand map over `layers` matrices starting at `base`, `stride` elements apart.
+bool opmap(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols, uint64_t ld,
+           int layers, int64_t stride, bool mn_major) {
+  return encode_f32_operand_3d(m, base, rows, cols, ld, (uint64_t)layers, (uint64_t)stride,
+                               mn_major);
 }
 
 }  // namespace
 
 size_t absorb_workspace_bytes(int dim) {
   const size_t d = (size_t)dim;
-  // A (-> L), Z (-> L^-1), Y, one 128 x 128 inverse, lambda (+ padding)
-  return (3 * d * d + NB * NB) * sizeof(float) + 1024;
+  // A (-> L), Z (-> L^-1), Y, one 128 x 128 inverse, lambda (+ padding);
+  // a multiple of 256 bytes so that per-layer workspaces stack
+  return ((3 * d * d + NB * NB) * sizeof(float) + 1024 + 255) & ~size_t(255);
 }
 
-cudaError_t absorb_solve(const float* M, const float* W, int dim, float lambda, float* dW,
-                         float* B, float* lambda_out, void* workspace, int* status,
-                         cudaStream_t stream) {
+cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const float* W,
+                                 int64_t w_stride, int dim, float lambda, float* dW,
+                                 int64_t dw_stride, float* B, int64_t b_stride, float* lambda_out,
+                                 void* workspace, int* status, cudaStream_t stream) {
   const size_t d = (size_t)dim;
+  const int64_t ws = (int64_t)(absorb_workspace_bytes(dim) / sizeof(float));  // per-layer stride
   float* A = static_cast<float*>(workspace);
   float* Z = A + d * d;
   float* Y = Z + d * d;
   float* Linv = Y + d * d;
   float* lam = Linv + NB * NB;
+  const int64_t lam_off = (int64_t)(3 * d * d + NB * NB);
   const int nblk = dim / NB;
   cudaError_t e;
   cudaFuncSetAttribute(potrf_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)kPotrfSmem);
 
-  lambda_kernel<<<1, 256, 0, stream>>>(M, dim, lambda, lam, lambda_out);
-  build_kernel<<<148 * 8, 256, 0, stream>>>(M, dim, lam, A, Z);
+  lambda_kernel<<<n, 256, 0, stream>>>(M, m_stride, dim, lambda, lam, ws, lambda_out);
+  build_kernel<<<dim3(n == 1 ? 148 * 8 : 148, n), 256, 0, stream>>>(M, m_stride, dim, A, ws,
+                                                                     lam_off);
   count_launches(2);
 
   // B = R W (R = M[0:d, d:2d])
@@ -206,16 +262,16 @@ cudaError_t absorb_solve(const float* M, const float* W, int dim, float lambda, 
     p.nprob = 1;
     p.status = status;
     TGemmProblem& pr = p.prob[0];
-    if (!encode_f32_operand(&pr.ta, M + d, d, d, 2 * d, false) ||
-        !encode_f32_operand(&pr.tb, W, d, d, d, true))
+    if (!opmap(&pr.ta, M + d, d, d, 2 * d, n, m_stride, false) ||
+        !opmap(&pr.tb, W, d, d, d, n, w_stride, true))
       return cudaErrorInvalidValue;
-    set_store(pr, dim, dim, dim, B, dim, 0, 0, 1.f, 0.f);
+    set_store(pr, dim, dim, dim, B, dim, b_stride, 0, 0, 1.f, 0.f, n);
     pr.a_mn = 0;
     pr.b_mn = 1;
     if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
   }
 
-  potrf_inv_kernel<<<1, 512, kPotrfSmem, stream>>>(A, dim, Linv, status);
+  potrf_inv_kernel<<<n, 512, kPotrfSmem, stream>>>(A, dim, Linv, ws, status);
   count_launches();
   for (int k = 0; k < nblk; ++k) {
     const int kk = k * NB;
@@ -227,19 +283,19 @@ cudaError_t absorb_solve(const float* M, const float* W, int dim, float lambda, 
       int q = 0;
       if (m > 0) {
         TGemmProblem& pr = p.prob[q++];
-        if (!encode_f32_operand(&pr.ta, A + (size_t)(kk + NB) * d + kk, m, NB, d, false) ||
-            !encode_f32_operand(&pr.tb, Linv, NB, NB, NB, false))
+        if (!opmap(&pr.ta, A + (size_t)(kk + NB) * d + kk, m, NB, d, n, ws, false) ||
+            !opmap(&pr.tb, Linv, NB, NB, NB, n, ws, false))
           return cudaErrorInvalidValue;
-        set_store(pr, m, NB, NB, A, dim, kk + NB, kk, 1.f, 0.f);
+        set_store(pr, m, NB, NB, A, dim, ws, kk + NB, kk, 1.f, 0.f, n);
         pr.a_mn = 0;
         pr.b_mn = 0;
       }
       {
         TGemmProblem& pr = p.prob[q++];
-        if (!encode_f32_operand(&pr.ta, Linv, NB, NB, NB, false) ||
-            !encode_f32_operand(&pr.tb, Z + (size_t)kk * d, NB, kk + NB, d, true))
+        if (!opmap(&pr.ta, Linv, NB, NB, NB, n, ws, false) ||
+            !opmap(&pr.tb, Z + (size_t)kk * d, NB, kk + NB, d, n, ws, true))
           return cudaErrorInvalidValue;
-        set_store(pr, NB, kk + NB, NB, Z, dim, kk, 0, 1.f, 0.f);
+        set_store(pr, NB, kk + NB, NB, Z, dim, ws, kk, 0, 1.f, 0.f, n);
         pr.a_mn = 0;
         pr.b_mn = 1;
       }
@@ -254,24 +310,23 @@ cudaError_t absorb_solve(const float* M, const float* W, int dim, float lambda, 
       p.nprob = 2;
       const float* Lk = A + (size_t)(kk + NB) * d + kk;
       TGemmProblem& t1 = p.prob[0];
-      if (!encode_f32_operand(&t1.ta, Lk, m, NB, d, false) ||
-          !encode_f32_operand(&t1.tb, Lk, m, NB, d, false))
+      if (!opmap(&t1.ta, Lk, m, NB, d, n, ws, false) || !opmap(&t1.tb, Lk, m, NB, d, n, ws, false))
         return cudaErrorInvalidValue;
-      set_store(t1, m, m, NB, A, dim, kk + NB, kk + NB, -1.f, 1.f);
+      set_store(t1, m, m, NB, A, dim, ws, kk + NB, kk + NB, -1.f, 1.f, n);
       t1.a_mn = 0;
       t1.b_mn = 0;
       t1.lower = 1;
       TGemmProblem& t2 = p.prob[1];
-      if (!encode_f32_operand(&t2.ta, Lk, m, NB, d, false) ||
-          !encode_f32_operand(&t2.tb, Z + (size_t)kk * d, NB, kk + NB, d, true))
+      if (!opmap(&t2.ta, Lk, m, NB, d, n, ws, false) ||
+          !opmap(&t2.tb, Z + (size_t)kk * d, NB, kk + NB, d, n, ws, true))
         return cudaErrorInvalidValue;
-      set_store(t2, m, kk + NB, NB, Z, dim, kk + NB, 0, -1.f, 1.f);
+      set_store(t2, m, kk + NB, NB, Z, dim, ws, kk + NB, 0, -1.f, 1.f, n);
       t2.a_mn = 0;
       t2.b_mn = 1;
       if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
     }
-    potrf_inv_kernel<<<1, 512, kPotrfSmem, stream>>>(A + (size_t)(kk + NB) * d + kk + NB, dim,
-                                                     Linv, status);
+    potrf_inv_kernel<<<n, 512, kPotrfSmem, stream>>>(A + (size_t)(kk + NB) * d + kk + NB, dim,
+                                                     Linv, ws, status);
     count_launches();
   }
   // Y = Z B (Z lower triangular), Delta W = Z^T Y (Z^T upper triangular)
@@ -280,10 +335,9 @@ cudaError_t absorb_solve(const float* M, const float* W, int dim, float lambda, 
     p.nprob = 1;
     p.status = status;
     TGemmProblem& pr = p.prob[0];
-    if (!encode_f32_operand(&pr.ta, Z, d, d, d, false) ||
-        !encode_f32_operand(&pr.tb, B, d, d, d, true))
+    if (!opmap(&pr.ta, Z, d, d, d, n, ws, false) || !opmap(&pr.tb, B, d, d, d, n, b_stride, true))
       return cudaErrorInvalidValue;
-    set_store(pr, dim, dim, dim, Y, dim, 0, 0, 1.f, 0.f);
+    set_store(pr, dim, dim, dim, Y, dim, ws, 0, 0, 1.f, 0.f, n);
     pr.a_mn = 0;
     pr.b_mn = 1;
     pr.tri = kTriLowerA;
@@ -294,16 +348,23 @@ cudaError_t absorb_solve(const float* M, const float* W, int dim, float lambda, 
     p.nprob = 1;
     p.status = status;
     TGemmProblem& pr = p.prob[0];
-    if (!encode_f32_operand(&pr.ta, Z, d, d, d, true) ||
-        !encode_f32_operand(&pr.tb, Y, d, d, d, true))
+    if (!opmap(&pr.ta, Z, d, d, d, n, ws, true) || !opmap(&pr.tb, Y, d, d, d, n, ws, true))
       return cudaErrorInvalidValue;
-    set_store(pr, dim, dim, dim, dW, dim, 0, 0, 1.f, 0.f);
+    set_store(pr, dim, dim, dim, dW, dim, dw_stride, 0, 0, 1.f, 0.f, n);
     pr.a_mn = 1;
     pr.b_mn = 1;
     pr.tri = kTriUpperA;
     if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
   }
   return cudaGetLastError();
+}
+
+cudaError_t absorb_solve(const float* M, const float* W, int dim, float lambda, float* dW,
+                         float* B, float* lambda_out, void* workspace, int* status,
+                         cudaStream_t stream) {
+  const int64_t dd = (int64_t)dim * dim;
+  return absorb_solve_batched(1, M, 4 * dd, W, dd, dim, lambda, dW, dd, B, dd, lambda_out,
+                              workspace, status, stream);
 }
 
 }  // namespace ispa

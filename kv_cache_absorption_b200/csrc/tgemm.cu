@@ -55,12 +55,15 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Tile (i, j) of problem `q` from the launch-wide tile index.
-__device__ __forceinline__ void decode(const TGemmParams& p, int b, int& q, int& i, int& j) {
+// Layer and tile (i, j) of problem `q` from the launch-wide tile index.
+__device__ __forceinline__ void decode(const TGemmParams& p, int b, int& q, int& layer, int& i,
+                                       int& j) {
   q = 0;
   while (q + 1 < p.nprob && b >= p.prob[q + 1].tile_base) ++q;
   const TGemmProblem& pr = p.prob[q];
   int t = b - pr.tile_base;
+  layer = t / pr.tiles_per_layer;
+  t -= layer * pr.tiles_per_layer;
   if (pr.lower) {   // tiles with j <= i, row by row
     int r = (int)((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
     while ((r + 1) * (r + 2) / 2 <= t) ++r;
@@ -83,11 +86,11 @@ __device__ __forceinline__ void k_range(const TGemmProblem& pr, int i, int& kb, 
 // Loads one 32-deep slab of a 128-wide operand block (rows/cols starting at
 // `mn0`, K starting at `k0`) into `dst`.
 __device__ __forceinline__ void load_slab(uint8_t* dst, const CUtensorMap* m, bool mn_major,
-                                          int mn0, int k0, uint64_t* bar) {
+                                          int mn0, int k0, int layer, uint64_t* bar) {
   if (mn_major) {   // K rows x MN columns: four 32-wide boxes
-    for (int c = 0; c < 4; ++c) tma_load_2d(dst + c * (TK * 128), m, bar, mn0 + c * 32, k0);
+    for (int c = 0; c < 4; ++c) tma_load_3d(dst + c * (TK * 128), m, bar, mn0 + c * 32, k0, layer);
   } else {          // MN rows x K columns: one box of 128 rows x 32
-    tma_load_2d(dst, m, bar, k0, mn0);
+    tma_load_3d(dst, m, bar, k0, mn0, layer);
   }
 }
 
@@ -103,8 +106,8 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
   GSmem& s = *reinterpret_cast<GSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   volatile int* abort_flag = &s.abort_flag;
-  int q, ti, tj;
-  decode(p, blockIdx.x, q, ti, tj);
+  int q, layer, ti, tj;
+  decode(p, blockIdx.x, q, layer, ti, tj);
   const TGemmProblem& pr = p.prob[q];
   int kb, ke;
   k_range(pr, ti, kb, ke);
@@ -136,8 +139,10 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
         const int st = n % NSTAGE;
         if (n >= NSTAGE && !mbar_wait(&s.empty[st], ((n / NSTAGE) - 1) & 1, p.status, abort_flag)) break;
         mbar_expect_tx(&s.full[st], 2 * kSlab);
-        load_slab(s.a_hi[st], &pr.ta, pr.a_mn, pr.a_row0 + ti * TM, pr.a_k0 + k * TK, &s.full[st]);
-        load_slab(s.b_hi[st], &pr.tb, pr.b_mn, pr.b_col0 + tj * TN, pr.b_k0 + k * TK, &s.full[st]);
+        load_slab(s.a_hi[st], &pr.ta, pr.a_mn, pr.a_row0 + ti * TM, pr.a_k0 + k * TK, layer,
+                  &s.full[st]);
+        load_slab(s.b_hi[st], &pr.tb, pr.b_mn, pr.b_col0 + tj * TN, pr.b_k0 + k * TK, layer,
+                  &s.full[st]);
       }
       if (*abort_flag)
         for (int j = n - NSTAGE < 0 ? 0 : n - NSTAGE; j < n; ++j)
@@ -201,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
     if (ok && (nk == 0 || mbar_wait(&s.acc_full, 0, p.status, abort_flag))) {
       tc_fence_after();
       if (pr.mode == kModeStore) {
-        float* crow = pr.C + row * pr.ldc + col0;
+        float* crow = pr.C + (int64_t)layer * pr.c_layer_stride + row * pr.ldc + col0;
         const float alpha = pr.alpha, beta = pr.beta;
 #pragma unroll 1
         for (int c = 0; c < TN / 32; ++c) {
@@ -233,8 +238,9 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
         const int64_t ld = 2 * (int64_t)p.dot_dim;
         const double wsym = ti < tj ? 2.0 : (ti == tj ? 1.0 : 0.0);
         double g = 0.0, rr = 0.0, sv = 0.0;
-        const float* Mr = p.dot_M + row * ld;
-        const float* Sr = p.dot_M + (row + p.dot_dim) * ld + p.dot_dim;
+        const float* Ml = p.dot_M + (int64_t)layer * p.dot_m_stride;
+        const float* Mr = Ml + row * ld;
+        const float* Sr = Ml + (row + p.dot_dim) * ld + p.dot_dim;
 #pragma unroll 1
         for (int c = 0; c < TN / 32; ++c) {
           uint32_t v[32];
@@ -257,9 +263,10 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
           sv += __shfl_xor_sync(0xffffffffu, sv, o);
         }
         if (lane == 0) {
-          atomicAdd(p.dot_acc + 0, g * wsym);
-          atomicAdd(p.dot_acc + 1, rr);
-          atomicAdd(p.dot_acc + 2, sv * wsym);
+          double* acc = p.dot_acc + (int64_t)layer * p.dot_acc_stride;
+          atomicAdd(acc + 0, g * wsym);
+          atomicAdd(acc + 1, rr);
+          atomicAdd(acc + 2, sv * wsym);
         }
       }
     }
@@ -279,8 +286,10 @@ cudaError_t launch_tgemm(TGemmParams& p, cudaStream_t stream) {
     TGemmProblem& pr = p.prob[q];
     pr.mt = pr.M / TM;
     pr.nt = pr.N / TN;
+    if (pr.layers < 1) pr.layers = 1;
+    pr.tiles_per_layer = pr.lower ? pr.mt * (pr.mt + 1) / 2 : pr.mt * pr.nt;
     pr.tile_base = base;
-    base += pr.lower ? pr.mt * (pr.mt + 1) / 2 : pr.mt * pr.nt;
+    base += pr.tiles_per_layer * pr.layers;
   }
   if (base == 0) return cudaSuccess;
   const size_t smem = tgemm_smem_bytes();

@@ -12,11 +12,13 @@ constexpr int kTriUpperA = 2;   // op(A) upper triangular: row block i reads K b
 constexpr int kModeStore = 0;   // C = alpha * op(A) op(B) + beta * C
 constexpr int kModeDot3 = 1;    // accumulate <P, G>, <P, R>, <P, S> (P = op(A) op(B))
 
-// C[M x N] (+)= op(A)[M x K] op(B)[K x N]; M, N multiples of 128, K of 32.
-// op(A) is read from tensor map ta: K-major when a_mn == 0 (stored [M][K]),
-// MN-major when a_mn == 1 (stored [K][M]); op(B) from tb: MN-major when
-// b_mn == 1 (stored [K][N]), K-major when b_mn == 0 (stored [N][K]).
-// a_row0 / a_k0 / b_col0 / b_k0 offset the tiles inside the mapped tensors.
+// For each of `layers` independent layers l:
+// C_l[M x N] (+)= op(A_l)[M x K] op(B_l)[K x N]; M, N multiples of 128, K of 32.
+// op(A) is read from the 3-D tensor map ta (x = column, y = row, z = layer):
+// K-major when a_mn == 0 (stored [M][K]), MN-major when a_mn == 1 (stored
+// [K][M]); op(B) from tb: MN-major when b_mn == 1 (stored [K][N]), K-major
+// when b_mn == 0 (stored [N][K]). a_row0 / a_k0 / b_col0 / b_k0 offset the
+// tiles inside the mapped tensors; C_l = C + l * c_layer_stride.
 struct TGemmProblem {
   CUtensorMap ta;
   CUtensorMap tb;
@@ -25,20 +27,24 @@ struct TGemmProblem {
   int a_row0, a_k0, b_col0, b_k0;
   float* C;
   int64_t ldc;
+  int64_t c_layer_stride;
   int c_row0, c_col0;
   float alpha, beta;
   int lower;     // only tiles (i, j) with j <= i
   int tri;       // kTri*
   int mode;      // kMode*
-  int mt, nt, tile_base;   // set by launch_tgemm
+  int layers;    // >= 1
+  int mt, nt, tiles_per_layer, tile_base;   // set by launch_tgemm
 };
 
 struct TGemmParams {
   TGemmProblem prob[4];
   int nprob;
-  const float* dot_M;   // kModeDot3: the [2d, 2d] Gram blocks
+  const float* dot_M;      // kModeDot3: the [2d, 2d] Gram blocks of layer 0
+  int64_t dot_m_stride;    // elements between layers' M
   int dot_dim;
-  double* dot_acc;      // kModeDot3: 3 accumulators
+  double* dot_acc;         // kModeDot3: 3 accumulators of layer 0
+  int dot_acc_stride;      // doubles between layers' accumulators
   int* status;
 };
 

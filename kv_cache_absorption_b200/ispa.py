@@ -32,7 +32,7 @@ EXPORTED = (
     "ispa_status_string", "ispa_version", "ispa_kernel_launches",
     "ispa_dual_attention_workspace_size", "ispa_dual_attention", "ispa_local_attention",
     "ispa_gram_accumulate", "ispa_absorb_workspace_size", "ispa_absorb_solve",
-    "ispa_absorb_solve_noalloc",
+    "ispa_absorb_solve_noalloc", "ispa_absorb_solve_batched", "ispa_layer_error_batched",
     "ispa_layer_error_workspace_size", "ispa_layer_error", "ispa_rank_layers",
 )
 
@@ -72,6 +72,8 @@ def _load():
         "ispa_absorb_workspace_size": (SZ, [I]),
         "ispa_absorb_solve": (I, [P, P, I, F, P, P, P, P, SZ, P, P]),
         "ispa_absorb_solve_noalloc": (I, [P, P, I, F, P, P, P, P, P]),
+        "ispa_absorb_solve_batched": (I, [I, P, I64, P, I64, I, F, P, I64, P, I64, P, P, SZ, P, P]),
+        "ispa_layer_error_batched": (I, [I, P, I64, P, I64, P, I64, P, I64, P, I, P, P, SZ, P]),
         "ispa_layer_error_workspace_size": (SZ, [I]),
         "ispa_layer_error": (I, [P, P, P, P, P, I, P, P, SZ, P]),
         "ispa_rank_layers": (I, [P, I, I, P, P, P]),
@@ -277,6 +279,52 @@ def ispa_absorb_solve_noalloc(M, W, lam: float = 0.0, status=None, stream=None) 
                                            _ptr(lam_out), _ptr(status), _stream(stream))
     _check(rc, "ispa_absorb_solve_noalloc")
     return {"dW": dW, "B": B, "lam": lam_out, "status": status}
+
+
+def ispa_absorb_solve_batched(M, W, lam: float = 0.0, dW=None, B=None, lam_out=None,
+                              workspace=None, status=None, stream=None) -> dict:
+    """Delta W of L layers in one call. M: [L, 2d, 2d], W: [L, d, d] fp32
+    (contiguous, so layer strides are 4 d^2 and d^2 elements). Returns dW and
+    B ([L, d, d]), the lambdas ([L]) and the status word."""
+    _dev_tensor(M, torch.float32, "M", 3)
+    _dev_tensor(W, torch.float32, "W", 3)
+    L, dim = W.shape[0], W.shape[1]
+    if tuple(M.shape) != (L, 2 * dim, 2 * dim) or W.shape[2] != dim:
+        raise ValueError("M must be [L, 2d, 2d] and W [L, d, d]")
+    dev = W.device
+    dW = torch.empty(L, dim, dim, dtype=torch.float32, device=dev) if dW is None else dW
+    B = torch.empty(L, dim, dim, dtype=torch.float32, device=dev) if B is None else B
+    lam_out = torch.empty(L, dtype=torch.float32, device=dev) if lam_out is None else lam_out
+    if workspace is None:
+        workspace = torch.empty(L * ispa_absorb_workspace_size(dim), dtype=torch.uint8, device=dev)
+    status = new_status(dev) if status is None else status
+    dd = dim * dim
+    rc = _load().ispa_absorb_solve_batched(
+        L, _ptr(M), 4 * dd, _ptr(W), dd, dim, float(lam), _ptr(dW), dW.stride(0), _ptr(B),
+        B.stride(0), _ptr(lam_out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(status), _stream(stream))
+    _check(rc, "ispa_absorb_solve_batched")
+    return {"dW": dW, "B": B, "lam": lam_out, "status": status}
+
+
+def ispa_layer_error_batched(M, W, dW, B, lam, err=None, workspace=None, stream=None):
+    """Reconstruction errors of L layers: device double [L, 2]."""
+    for t, n in ((M, "M"), (W, "W"), (dW, "dW"), (B, "B")):
+        _dev_tensor(t, torch.float32, n, 3)
+    _dev_tensor(lam, torch.float32, "lam", 1)
+    L, dim = W.shape[0], W.shape[1]
+    dev = W.device
+    err = torch.empty(L, 2, dtype=torch.float64, device=dev) if err is None else err
+    if workspace is None:
+        workspace = torch.empty(L * ispa_layer_error_workspace_size(dim), dtype=torch.uint8,
+                                device=dev)
+    dd = dim * dim
+    rc = _load().ispa_layer_error_batched(
+        L, _ptr(M), 4 * dd, _ptr(W), dd, _ptr(dW), dW.stride(0), _ptr(B), B.stride(0), _ptr(lam),
+        dim, _ptr(err), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _check(rc, "ispa_layer_error_batched")
+    return err
 
 
 def ispa_layer_error_workspace_size(dim: int) -> int:

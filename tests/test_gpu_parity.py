@@ -311,3 +311,34 @@ def test_fp16_range_flag(lib):
     out = run_dual(lib, to_dev(ch))
     torch.cuda.synchronize()
     assert lib.read_status(out["status"]) & lib.ISPA_STATUS_FP16_RANGE
+
+
+def test_absorb_and_error_batched_over_layers(lib):
+    """Three layers solved and scored in single calls: each layer matches the
+    oracle and the single-layer entry points."""
+    dim, L = 256, 3
+    Ms, Ws, refs = [], [], []
+    for l in range(L):
+        a, f, W = synthetic_layer(3 * dim + 17 * l, dim, seed=40 + l)
+        G, R, S = oracle.gram(a, f - a)
+        M = pack_M(G, R, S)
+        G32, R32 = f64(M[:dim, :dim]), f64(M[:dim, dim:])
+        lam = oracle.default_lambda(G32)
+        dW, B = oracle.absorb(G32, R32, f64(W), lam)
+        refs.append((dW, oracle.reconstruction_error(a, f, f64(W), dW)))
+        Ms.append(M)
+        Ws.append(W)
+    M = torch.stack(Ms).cuda()
+    W = torch.stack(Ws).contiguous().cuda()
+    out = lib.ispa_absorb_solve_batched(M, W)
+    err = lib.ispa_layer_error_batched(M, W, out["dW"], out["B"], out["lam"])
+    torch.cuda.synchronize()
+    assert lib.read_status(out["status"]) == 0
+    for l in range(L):
+        dW_ref, (e2, eps) = refs[l]
+        assert rel_fro(f64(out["dW"][l]), dW_ref) <= DW_RELFRO
+        single = lib.ispa_absorb_solve(M[l].contiguous(), W[l].contiguous())
+        torch.cuda.synchronize()
+        assert torch.equal(single["dW"], out["dW"][l])
+        got = err[l].cpu().numpy()
+        assert abs(got[0] - e2) <= 2e-3 * e2 and abs(got[1] - eps) <= 2e-3 * eps
