@@ -251,14 +251,20 @@ def max_over_ranks(x: float, world: int) -> float:
 # ---------------------------------------------------------------- our arm
 
 def make_inputs(cfg, rank, device):
+    """Per layer: its Q/K/V frame streams and the chunk dicts (views into
+    them); the projections stacked as one [L, d, d] tensor."""
+    import torch
     from ispa_synth import layer_streams
-    layers = []
+    streams, chunks, Ws = [], [], []
     for l in range(cfg.layers):
         st = layer_streams(cfg, layer=l + 1000 * rank, seed=0, device=device)
-        chunks = [st.chunk(c) for c in range(cfg.n_chunks)]
-        layers.append((chunks, st.w))
-        del st
-    return layers
+        streams.append(st)
+        chunks.append([st.chunk(c) for c in range(cfg.n_chunks)])
+        Ws.append(st.w)
+    W_all = torch.stack(Ws)
+    for st in streams:
+        st.w = None
+    return streams, chunks, W_all
 
 
 def run_ours(args):
@@ -272,30 +278,28 @@ def run_ours(args):
     world, rank, local = dist_setup()
     dev = torch.device("cuda", torch.cuda.current_device())
     cfg = CONFIGS[args.config]
-    layers = make_inputs(cfg, rank, dev)
+    streams, chunks_per_layer, W_all = make_inputs(cfg, rank, dev)
     max_hist = max(len(cfg.history_frames_of(c)) for c in range(cfg.n_chunks)) * cfg.tokens_per_frame
-    runner = LayerWarmup(cfg.heads, cfg.head_dim, cfg.chunk_tokens, cfg.sink_tokens,
-                         cfg.chunk_tokens, max_hist, device=dev)
     L = cfg.layers
+    runner = LayerWarmup(cfg.heads, cfg.head_dim, cfg.chunk_tokens, cfg.sink_tokens,
+                         cfg.chunk_tokens, max_hist, n_layers=L, device=dev)
     K = cfg.select_k if cfg.select_k is not None else L // 2
     err = torch.empty(L, 2, dtype=torch.float64, device=dev)
     perm = torch.empty(L, dtype=torch.int32, device=dev)
     sel = torch.empty(L, dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
     E = lambda: torch.cuda.Event(enable_timing=True)
 
     def step(ev=None):
-        for li, (chunks, W) in enumerate(layers):
+        for li, chunks in enumerate(chunks_per_layer):
             for c, ch in enumerate(chunks):
                 if ev: ev["a0"].append(E()); ev["a0"][-1].record()
                 runner.attention(ch)
                 if ev: ev["a1"].append(E()); ev["a1"][-1].record()
-                runner.gram(first=(c == 0))
+                runner.gram(first=(c == 0), layer=li)
                 if ev: ev["g1"].append(E()); ev["g1"][-1].record()
-            runner.solve(W)
-            runner.error(W, err[li])
-            if ev: ev["s1"].append(E()); ev["s1"][-1].record()
+        runner.absorb_all(W_all, err)         # every layer's solve + error, batched
+        if ev: ev["s1"].append(E()); ev["s1"][-1].record()
         rank_layers(err, K, perm, sel)
 
     for _ in range(args.warmup):
@@ -329,12 +333,10 @@ def run_ours(args):
     step_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
     attn_ms = sum(a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"])) / args.steps
     gram_ms = sum(a.elapsed_time(b) for a, b in zip(ev["a1"], ev["g1"])) / args.steps
-    solve_ms = 0.0
-    n_chunks = cfg.n_chunks
-    for li in range(len(ev["s1"])):
-        # solve + error of a layer: from the end of its last Gram to s1
-        solve_ms += ev["g1"][(li + 1) * n_chunks - 1].elapsed_time(ev["s1"][li])
-    solve_ms /= args.steps
+    # batched solve + error of all layers: from the end of the last Gram to s1
+    per_step = L * cfg.n_chunks
+    solve_ms = sum(ev["g1"][(i + 1) * per_step - 1].elapsed_time(ev["s1"][i])
+                   for i in range(args.steps)) / args.steps
     step_ms_max = max_over_ranks(step_ms, world)
 
     work = step_work(cfg)
@@ -376,7 +378,8 @@ def run_ours(args):
         "clocks": clocks,
     }
     if not args.no_e2e:
-        out["e2e"] = run_e2e(args, cfg, layers, runner, err, perm, sel, K, world)
+        out["e2e"] = run_e2e(args, cfg, streams, chunks_per_layer, W_all, runner, err, perm,
+                             sel, K, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = oracle_throughput(cfg, args.cpu_budget)
     if rank == 0:
@@ -386,37 +389,37 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_e2e(args, cfg, layers, runner, err, perm, sel, K, world):
+def run_e2e(args, cfg, streams, chunks_per_layer, W_all, runner, err, perm, sel, K, world):
     """Same step through the public API with the inputs in pinned host
-    memory: host->device copies of every chunk's Q/K/V and each W, the step,
-    and device->host copies of every Delta W, the errors and the ranking, all
-    inside the timed region."""
+    memory: every step copies each layer's Q/K/V frame streams and the
+    stacked W host->device, runs the warmup, and copies every Delta W, the
+    errors and the ranking device->host, all inside the timed region."""
     import torch
     from kv_cache_absorption_b200.warmup import rank as rank_layers
-    host_layers = [([{k: v.cpu().pin_memory() for k, v in ch.items()} for ch in chunks],
-                    W.cpu().pin_memory()) for chunks, W in layers]
-    dev_layers = layers
-    L = cfg.layers
-    d = cfg.d
+    dev_tensors = [t for st in streams for t in (st.q, st.k, st.v)] + [W_all]
+    owners = {t.untyped_storage().data_ptr() for t in dev_tensors}
+    for chunks in chunks_per_layer:      # every chunk input is a view into an uploaded stream
+        for ch in chunks:
+            assert all(x.numel() == 0 or x.untyped_storage().data_ptr() in owners
+                       for x in ch.values())
+    host_tensors = [t.cpu().pin_memory() for t in dev_tensors]
+    L, d = cfg.layers, cfg.d
     dW_host = torch.empty(L, d, d, dtype=torch.float32).pin_memory()
     err_host = torch.empty(L, 2, dtype=torch.float64).pin_memory()
     perm_host = torch.empty(L, dtype=torch.int32).pin_memory()
-    h2d = sum(W.numel() * 4 + sum(x.numel() * x.element_size() for ch in chunks for x in ch.values())
-              for chunks, W in host_layers)
+    h2d = sum(t.numel() * t.element_size() for t in host_tensors)
     d2h = dW_host.numel() * 4 + err_host.numel() * 8 + perm_host.numel() * 4
 
     def step():
-        for li, ((hchunks, hW), (dchunks, dW_)) in enumerate(zip(host_layers, dev_layers)):
-            dW_.copy_(hW, non_blocking=True)
-            for c, (hc, dc) in enumerate(zip(hchunks, dchunks)):
-                for k in hc:
-                    dc[k].copy_(hc[k], non_blocking=True)
-                runner.attention(dc)
-                runner.gram(first=(c == 0))
-            runner.solve(dW_)
-            runner.error(dW_, err[li])
-            dW_host[li].copy_(runner.dW, non_blocking=True)
+        for h, dv in zip(host_tensors, dev_tensors):
+            dv.copy_(h, non_blocking=True)
+        for li, chunks in enumerate(chunks_per_layer):
+            for c, ch in enumerate(chunks):
+                runner.attention(ch)
+                runner.gram(first=(c == 0), layer=li)
+        runner.absorb_all(W_all, err)
         rank_layers(err, K, perm, sel)
+        dW_host.copy_(runner.dW, non_blocking=True)
         err_host.copy_(err, non_blocking=True)
         perm_host.copy_(perm, non_blocking=True)
 

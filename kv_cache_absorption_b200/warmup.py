@@ -7,6 +7,10 @@ and accumulates the statistics of the closed form; at the transition each
 layer's Delta W is solved, every layer's reconstruction error is formed and
 the layers are ranked; the K lowest-error layers become L-Layers.
 
+Every layer keeps its own statistics block M = [[G, R], [., S]], so the
+transition runs as two batched calls over all layers (solve, then error)
+instead of one pair of calls per layer.
+
 Orchestration only: buffers and workspaces are allocated once (through
 torch) and every step is a call into the C ABI, so a warmup issues no
 allocation and no host synchronisation.
@@ -19,12 +23,14 @@ from . import ispa
 
 
 class LayerWarmup:
-    """Buffers for one layer geometry, reused across chunks and layers."""
+    """Buffers for ``n_layers`` layers of one geometry; the attention
+    outputs are reused across chunks and layers."""
 
     def __init__(self, heads: int, head_dim: int, chunk_rows: int, max_sink: int,
-                 max_local: int, max_hist: int, device="cuda"):
+                 max_local: int, max_hist: int, n_layers: int = 1, device="cuda"):
         self.heads, self.head_dim = heads, head_dim
         self.d = d = heads * head_dim
+        self.n_layers = n_layers
         self.device = device
         f32 = dict(dtype=torch.float32, device=device)
         self.a_loc = torch.empty(chunk_rows, d, **f32)
@@ -34,15 +40,15 @@ class LayerWarmup:
         self.attn_ws = torch.empty(ispa.ispa_dual_attention_workspace_size(
             chunk_rows, max_sink, max_local, max_hist, heads, head_dim), dtype=torch.uint8,
             device=device)
-        self.M = torch.zeros(2 * d, 2 * d, **f32)
-        self.solve_ws = torch.empty(ispa.ispa_absorb_workspace_size(d), dtype=torch.uint8,
-                                    device=device)
-        self.err_ws = torch.empty(ispa.ispa_layer_error_workspace_size(d), dtype=torch.uint8,
-                                  device=device)
+        self.M = torch.zeros(n_layers, 2 * d, 2 * d, **f32)
+        self.solve_ws = torch.empty(n_layers * ispa.ispa_absorb_workspace_size(d),
+                                    dtype=torch.uint8, device=device)
+        self.err_ws = torch.empty(n_layers * ispa.ispa_layer_error_workspace_size(d),
+                                  dtype=torch.uint8, device=device)
         self.status = ispa.new_status(device)
-        self.dW = torch.empty(d, d, **f32)
-        self.B = torch.empty(d, d, **f32)
-        self.lam = torch.empty(1, **f32)
+        self.dW = torch.empty(n_layers, d, d, **f32)
+        self.B = torch.empty(n_layers, d, d, **f32)
+        self.lam = torch.empty(n_layers, **f32)
         self._rows = 0
 
     def attention(self, ch: dict, stream=None):
@@ -60,36 +66,67 @@ class LayerWarmup:
             ispa._ptr(self.status), ispa._stream(stream))
         ispa._check(rc, "ispa_dual_attention")
 
-    def gram(self, first: bool, stream=None):
-        """Fold the last chunk's rows into G, R, S (first chunk overwrites)."""
+    def gram(self, first: bool, layer: int = 0, stream=None):
+        """Fold the last chunk's rows into the layer's G, R, S (first chunk
+        overwrites)."""
         rc = ispa._load().ispa_gram_accumulate(
-            ispa._ptr(self.a_loc), ispa._ptr(self.d_out), self._rows, self.d, ispa._ptr(self.M),
-            0 if first else 1, 1, ispa._stream(stream))
+            ispa._ptr(self.a_loc), ispa._ptr(self.d_out), self._rows, self.d,
+            ispa._ptr(self.M[layer]), 0 if first else 1, 1, ispa._stream(stream))
         ispa._check(rc, "ispa_gram_accumulate")
 
-    def chunk(self, ch: dict, first: bool, stream=None):
+    def chunk(self, ch: dict, first: bool, layer: int = 0, stream=None):
         self.attention(ch, stream)
-        self.gram(first, stream)
+        self.gram(first, layer, stream)
 
-    def solve(self, W: torch.Tensor, lam: float = 0.0, stream=None):
-        """Delta W of the layer (and B = R W, lambda)."""
+    def solve(self, W: torch.Tensor, lam: float = 0.0, layer: int = 0, stream=None):
+        """Delta W (and B = R W, lambda) of one layer into its slot."""
         rc = ispa._load().ispa_absorb_solve(
-            ispa._ptr(self.M), ispa._ptr(W), self.d, float(lam), ispa._ptr(self.dW),
-            ispa._ptr(self.B), ispa._ptr(self.lam), ispa._ptr(self.solve_ws),
-            self.solve_ws.numel(), ispa._ptr(self.status), ispa._stream(stream))
+            ispa._ptr(self.M[layer]), ispa._ptr(W), self.d, float(lam),
+            ispa._ptr(self.dW[layer]), ispa._ptr(self.B[layer]), ispa._ptr(self.lam[layer:]),
+            ispa._ptr(self.solve_ws), self.solve_ws.numel(), ispa._ptr(self.status),
+            ispa._stream(stream))
         ispa._check(rc, "ispa_absorb_solve")
 
-    def error(self, W: torch.Tensor, err_slot: torch.Tensor, stream=None):
-        """The layer's {||E||^2, relative error} into err_slot (device double[2])."""
+    def error(self, W: torch.Tensor, err_slot: torch.Tensor, layer: int = 0, stream=None):
+        """One layer's {||E||^2, relative error} into err_slot (device double[2])."""
         rc = ispa._load().ispa_layer_error(
-            ispa._ptr(self.M), ispa._ptr(W), ispa._ptr(self.dW), ispa._ptr(self.B),
-            ispa._ptr(self.lam), self.d, ispa._ptr(err_slot), ispa._ptr(self.err_ws),
-            self.err_ws.numel(), ispa._stream(stream))
+            ispa._ptr(self.M[layer]), ispa._ptr(W), ispa._ptr(self.dW[layer]),
+            ispa._ptr(self.B[layer]), ispa._ptr(self.lam[layer:]), self.d, ispa._ptr(err_slot),
+            ispa._ptr(self.err_ws), self.err_ws.numel(), ispa._stream(stream))
         ispa._check(rc, "ispa_layer_error")
 
-    def absorb(self, W: torch.Tensor, err_slot: torch.Tensor, lam: float = 0.0, stream=None):
-        self.solve(W, lam, stream)
-        self.error(W, err_slot, stream)
+    def solve_all(self, W_all: torch.Tensor, lam: float = 0.0, stream=None):
+        """Delta W of every layer in one batched call; W_all is [n_layers, d, d]."""
+        n, d = self.n_layers, self.d
+        _check_stack(W_all, n, d)
+        rc = ispa._load().ispa_absorb_solve_batched(
+            n, ispa._ptr(self.M), 4 * d * d, ispa._ptr(W_all), W_all.stride(0), d, float(lam),
+            ispa._ptr(self.dW), d * d, ispa._ptr(self.B), d * d, ispa._ptr(self.lam),
+            ispa._ptr(self.solve_ws), self.solve_ws.numel(), ispa._ptr(self.status),
+            ispa._stream(stream))
+        ispa._check(rc, "ispa_absorb_solve_batched")
+
+    def error_all(self, W_all: torch.Tensor, err: torch.Tensor, stream=None):
+        """Every layer's {||E||^2, relative error} into err [n_layers, 2] fp64."""
+        n, d = self.n_layers, self.d
+        _check_stack(W_all, n, d)
+        if err.dtype != torch.float64 or err.shape != (n, 2) or not err.is_contiguous():
+            raise ValueError("err must be a contiguous float64 [n_layers, 2] tensor")
+        rc = ispa._load().ispa_layer_error_batched(
+            n, ispa._ptr(self.M), 4 * d * d, ispa._ptr(W_all), W_all.stride(0),
+            ispa._ptr(self.dW), d * d, ispa._ptr(self.B), d * d, ispa._ptr(self.lam), d,
+            ispa._ptr(err), ispa._ptr(self.err_ws), self.err_ws.numel(), ispa._stream(stream))
+        ispa._check(rc, "ispa_layer_error_batched")
+
+    def absorb_all(self, W_all: torch.Tensor, err: torch.Tensor, lam: float = 0.0, stream=None):
+        self.solve_all(W_all, lam, stream)
+        self.error_all(W_all, err, stream)
+
+
+def _check_stack(W_all: torch.Tensor, n: int, d: int):
+    if (W_all.dtype != torch.float32 or W_all.shape != (n, d, d) or W_all.stride(2) != 1
+            or W_all.stride(1) != d):
+        raise ValueError(f"W_all must be float32 [{n}, {d}, {d}] with contiguous rows")
 
 
 def rank(err: torch.Tensor, K: int, perm: torch.Tensor, selected: torch.Tensor, stream=None):
@@ -99,20 +136,22 @@ def rank(err: torch.Tensor, K: int, perm: torch.Tensor, selected: torch.Tensor, 
     ispa._check(rc, "ispa_rank_layers")
 
 
-def run_warmup(layers, K: int, runner: LayerWarmup, keep_dw: bool = False, stream=None):
-    """Whole warmup over ``layers``: a list of (chunks, W) per layer, chunks a
-    list of dicts of device tensors. Returns (err [L, 2] fp64, perm, selected,
-    list of Delta W if keep_dw)."""
-    n = len(layers)
+def run_warmup(chunks_per_layer, W_all: torch.Tensor, K: int, runner: LayerWarmup,
+               stream=None):
+    """Whole warmup: ``chunks_per_layer[l]`` is layer l's list of chunk dicts
+    (device tensors), ``W_all`` the [L, d, d] projections. Accumulates every
+    layer's statistics, solves and scores all layers in two batched calls and
+    ranks them. Returns (err [L, 2] fp64, perm, selected); Delta W of layer l
+    is ``runner.dW[l]``."""
+    n = len(chunks_per_layer)
+    if n != runner.n_layers:
+        raise ValueError(f"runner holds {runner.n_layers} layers, got {n}")
     err = torch.empty(n, 2, dtype=torch.float64, device=runner.device)
     perm = torch.empty(n, dtype=torch.int32, device=runner.device)
     sel = torch.empty(n, dtype=torch.uint8, device=runner.device)
-    dws = []
-    for li, (chunks, W) in enumerate(layers):
+    for li, chunks in enumerate(chunks_per_layer):
         for c, ch in enumerate(chunks):
-            runner.chunk(ch, first=(c == 0), stream=stream)
-        runner.absorb(W, err[li], stream=stream)
-        if keep_dw:
-            dws.append(runner.dW.clone())
+            runner.chunk(ch, first=(c == 0), layer=li, stream=stream)
+    runner.absorb_all(W_all, err, stream=stream)
     rank(err, K, perm, sel, stream)
-    return err, perm, sel, dws
+    return err, perm, sel

@@ -267,16 +267,15 @@ def test_warmup_tiny_end_to_end(lib):
     ref = oracle.warmup_layer(chunks, st.w)
     runner = LayerWarmup(C0.heads, C0.head_dim, C0.chunk_tokens, C0.sink_tokens,
                          C0.chunk_tokens, 256)
-    err, perm, sel, dws = run_warmup([([to_dev(c) for c in chunks], st.w.cuda())], 1, runner,
-                                     keep_dw=True)
+    err, perm, sel = run_warmup([[to_dev(c) for c in chunks]], st.w.cuda()[None], 1, runner)
     torch.cuda.synchronize()
     assert lib.read_status(runner.status) == 0
     d = C0.d
-    Mg = f64(runner.M)
+    Mg = f64(runner.M[0])
     up = upper_tile_mask(d)
     assert rel_fro(Mg[:d, :d][up], ref["G"][up]) <= GR_RELFRO
     assert rel_fro(Mg[:d, d:], ref["R"]) <= GR_RELFRO
-    assert rel_fro(f64(dws[0]), ref["dW"]) <= DW_RELFRO
+    assert rel_fro(f64(runner.dW[0]), ref["dW"]) <= DW_RELFRO
     assert abs(err[0, 1].item() - ref["eps"]) <= 5e-3 * ref["eps"]
 
 
@@ -286,16 +285,17 @@ def test_warmup_multilayer_ranking(lib):
     spread so that the errors separate."""
     from kv_cache_absorption_b200.warmup import LayerWarmup, run_warmup
     L = 6
-    layers_dev, eps_ref = [], []
+    chunks_dev, Ws, eps_ref = [], [], []
     for l in range(L):
         cfg = scaled(C0, tokens_per_frame=64, sink_tokens=64, chunk_frames=3, first_chunk_frame=1,
                      n_chunks=4, history_window=None, rho=0.5 + 0.08 * l)
         st = layer_streams(cfg, l, seed=1)
         chunks = [st.chunk(c) for c in range(4)]
         eps_ref.append(oracle.warmup_layer(chunks, st.w)["eps"])
-        layers_dev.append(([to_dev(c) for c in chunks], st.w.cuda()))
-    runner = LayerWarmup(2, 64, 192, 64, 192, 9 * 64)
-    err, perm, sel, _ = run_warmup(layers_dev, 3, runner)
+        chunks_dev.append([to_dev(c) for c in chunks])
+        Ws.append(st.w)
+    runner = LayerWarmup(2, 64, 192, 64, 192, 9 * 64, n_layers=L)
+    err, perm, sel = run_warmup(chunks_dev, torch.stack(Ws).cuda(), 3, runner)
     torch.cuda.synchronize()
     ref_perm, ref_sel = oracle.rank_layers(eps_ref, 3)
     got_eps = err[:, 1].cpu().numpy()
