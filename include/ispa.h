@@ -250,6 +250,29 @@ ISPA_API int ispa_layer_error_batched(int n_layers, const float* M, int64_t m_la
                                       int64_t b_layer_stride, const float* lambdas, int dim,
                                       double* err, void* workspace, size_t workspace_bytes,
                                       void* stream);
+/* Weight Gram, once per model: P_l = W_l W_l^T (full symmetric d x d,
+ * fp32-accurate 3xTF32 tensor-core product). The error identities above
+ * use W only through W W^T, which depends on the model weights and not on
+ * the instance, so a caller may form it when the weights are loaded and
+ * reuse it for every warmup.
+ * W: n_layers matrices [d, d] fp32 row-major, w_layer_stride elements
+ * apart; P: output, same layout with p_layer_stride. Strides >= d * d and
+ * multiples of 4; W and P 16-byte aligned; dim a multiple of 128.
+ * dev_status: device int, ISPA_STATUS_TIMEOUT on a stalled pipeline. */
+ISPA_API int ispa_weight_gram_batched(int n_layers, const float* W, int64_t w_layer_stride,
+                                      int dim, float* P, int64_t p_layer_stride, int* dev_status,
+                                      void* stream);
+/* Same per-layer result as ispa_layer_error_batched, with W W^T given as P
+ * (from ispa_weight_gram_batched): every sum is then one pass over G, R, S,
+ * P, dW and B with fp64 accumulation, no d^3 product.
+ * workspace: >= n_layers * ispa_layer_error_workspace_size(dim) bytes,
+ * 8-byte aligned. Other arguments as ispa_layer_error_batched. */
+ISPA_API int ispa_layer_error_wwt_batched(int n_layers, const float* M, int64_t m_layer_stride,
+                                          const float* P, int64_t p_layer_stride, const float* dW,
+                                          int64_t dw_layer_stride, const float* B,
+                                          int64_t b_layer_stride, const float* lambdas, int dim,
+                                          double* err, void* workspace, size_t workspace_bytes,
+                                          void* stream);
 ISPA_API int ispa_rank_layers(const double* err, int n_layers, int K, int* perm, uint8_t* selected,
                      void* stream);
 

@@ -27,6 +27,12 @@ cudaError_t layer_error_batched(int n, const float* M, int64_t m_stride, const f
                                 int64_t w_stride, const float* dW, int64_t dw_stride,
                                 const float* B, int64_t b_stride, const float* lam, int dim,
                                 double* err, double* acc, cudaStream_t stream);
+cudaError_t weight_gram_batched(int n, const float* W, int64_t w_stride, int dim, float* P,
+                                int64_t p_stride, int* status, cudaStream_t stream);
+cudaError_t layer_error_wwt_batched(int n, const float* M, int64_t m_stride, const float* P,
+                                    int64_t p_stride, const float* dW, int64_t dw_stride,
+                                    const float* B, int64_t b_stride, const float* lam, int dim,
+                                    double* err, double* acc, cudaStream_t stream);
 cudaError_t rank_layers(const double* err, int n, int K, int* perm, uint8_t* selected,
                         cudaStream_t stream);
 }  // namespace ispa
@@ -302,6 +308,44 @@ int ispa_layer_error_batched(int n_layers, const float* M, int64_t m_layer_strid
                                            dw_layer_stride, B, b_layer_stride, lambdas, dim, err,
                                            static_cast<double*>(workspace),
                                            static_cast<cudaStream_t>(stream)));
+}
+
+int ispa_weight_gram_batched(int n_layers, const float* W, int64_t w_layer_stride, int dim,
+                             float* P, int64_t p_layer_stride, int* dev_status, void* stream) {
+  if (n_layers < 1 || n_layers > 4096 || !W || !P || !dev_status || dim <= 0) return ISPA_ERR_ARG;
+  if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
+  const int64_t dd = (int64_t)dim * dim;
+  if (!stride_ok(w_layer_stride, dd) || !stride_ok(p_layer_stride, dd)) return ISPA_ERR_ARG;
+  if (!aligned16(W) || !aligned16(P)) return ISPA_ERR_UNSUPPORTED;
+  int rc = check_device();
+  if (rc != ISPA_OK) return rc;
+  return cuda_rc(ispa::weight_gram_batched(n_layers, W, w_layer_stride, dim, P, p_layer_stride,
+                                           dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+int ispa_layer_error_wwt_batched(int n_layers, const float* M, int64_t m_layer_stride,
+                                 const float* P, int64_t p_layer_stride, const float* dW,
+                                 int64_t dw_layer_stride, const float* B, int64_t b_layer_stride,
+                                 const float* lambdas, int dim, double* err, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (n_layers < 1 || n_layers > 4096 || !M || !P || !dW || !B || !lambdas || !err || dim <= 0)
+    return ISPA_ERR_ARG;
+  if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
+  const int64_t dd = (int64_t)dim * dim;
+  if (!stride_ok(m_layer_stride, 4 * dd) || !stride_ok(p_layer_stride, dd) ||
+      !stride_ok(dw_layer_stride, dd) || !stride_ok(b_layer_stride, dd))
+    return ISPA_ERR_ARG;
+  if (!aligned16(M) || !aligned16(P) || !aligned16(dW) || !aligned16(B))
+    return ISPA_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes / (size_t)n_layers < 256 ||
+      (reinterpret_cast<uintptr_t>(workspace) & 7u))
+    return ISPA_ERR_WORKSPACE;
+  int rc = check_device();
+  if (rc != ISPA_OK) return rc;
+  return cuda_rc(ispa::layer_error_wwt_batched(n_layers, M, m_layer_stride, P, p_layer_stride, dW,
+                                               dw_layer_stride, B, b_layer_stride, lambdas, dim,
+                                               err, static_cast<double*>(workspace),
+                                               static_cast<cudaStream_t>(stream)));
 }
 
 size_t ispa_layer_error_workspace_size(int dim) { return dim > 0 ? 256 : 0; }

@@ -9,15 +9,20 @@
 //
 // Organisation (block size 128, all products fp32-accurate 3xTF32 tensor-
 // core GEMMs, see tgemm.cu):
+//   * B = R W first (returned for the error computation);
 //   * one right-looking sweep over the 128-column panels factors A in place
-//     and, on the augmented block [A | Z] with Z = I, also yields
-//     Z = L^-1. Step k: factor and invert the diagonal block (one CTA,
-//     fp32, shared memory); panel L_{>k,k} = A_{>k,k} Linv_kk^T and row
-//     Z_k = Linv_kk Z_k (one grouped launch); trailing update of the lower
-//     tiles of A and of the rows of Z below k (one grouped launch).
-//   * then two triangular-aware GEMMs: Y = Z B and Delta W = Z^T Y, with
-//     B = R W formed first (and returned for the error computation).
-// Compared with two blocked triangular solves, this trades ~d^3/3 extra
+//     and, on the augmented block [A | Z | Y] with Z = I and Y = B, also
+//     yields Z = L^-1 and Y = L^-1 B (forward substitution). Step k: factor
+//     and invert the diagonal block (one CTA, fp32, shared memory); panel
+//     L_{>k,k} = A_{>k,k} Linv_kk^T and block rows Z_k = Linv_kk Z_k,
+//     Y_k = Linv_kk Y_k (one grouped launch); trailing update of the lower
+//     tiles of A and of the rows of Z and Y below k (one grouped launch);
+//   * then one triangular-aware GEMM: Delta W = Z^T Y.
+// Y is formed by substitution, not as the product Z B: entries of L^-1
+// alternate in sign and |L^-1| |B| can exceed |L^-1 B| by three orders of
+// magnitude, which a product at fp32 precision turns into a 1e-3 relative
+// error; substitution only forms products with L, with no such cancellation.
+// Compared with a backward substitution sweep, Z^T Y trades ~d^3/3 extra
 // flops for d/128 fewer dependent launches.
 #include "sm100.cuh"
 #include "attention.h"
@@ -70,134 +75,218 @@ __global__ void build_kernel(const float* __restrict__ M0, int64_t m_stride, int
   }
 }
 
-// Factors the 128 x 128 diagonal block at A (lower triangle used) as L L^T
-// and writes Linv = L^-1 (lower, zero above) to `linv`, in fp32, right-
-// looking in 8-column panels:
-//  * warp 0 factors the panel (all rows at or below it) in registers: lane l
-//    holds rows l, l+32, l+64, l+96 of the panel's 8 columns; pivots and
-//    panel rows travel by warp shuffles, so a column step needs no barrier;
-//  * one thread per column c then forms the panel's 8 rows of Linv by
-//    forward substitution with the 8 x 8 diagonal block of L;
-//  * all threads apply the panel to the trailing lower triangle of A and to
-//    the rows of Linv below the panel (4 threads per row).
-__global__ void __launch_bounds__(512) potrf_inv_kernel(const float* __restrict__ A0, int lda,
-                                                        float* __restrict__ linv0,
-                                                        int64_t ws_stride, int* status) {
-  constexpr int W = 8;
-  const float* A = A0 + (int64_t)blockIdx.x * ws_stride;    // one block per layer
-  float* linv = linv0 + (int64_t)blockIdx.x * ws_stride;
-  extern __shared__ float sh[];
-  float (*a)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(sh);
-  float (*z)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(sh + NB * (NB + 1));
-  float (*pan)[W] = reinterpret_cast<float (*)[W]>(sh + 2 * NB * (NB + 1));   // [NB][8], L of the panel
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  for (int e = t; e < NB * NB; e += blockDim.x) {
-    const int i = e >> 7, c = e & (NB - 1);
-    a[i][c] = A[(size_t)i * lda + c];
-    z[i][c] = (i == c) ? 1.f : 0.f;
-  }
-  __syncthreads();
-  for (int J = 0; J < NB; J += W) {
-    // ---- (1) warp 0: factor the panel columns J..J+7 for rows J..127
-    if (warp == 0) {
-      float r[4][W];
-#pragma unroll
-      for (int s = 0; s < 4; ++s)
-#pragma unroll
-        for (int m = 0; m < W; ++m) r[s][m] = a[lane + 32 * s][J + m];
-      const int ps = J >> 5;           // slot of the panel's rows (J..J+7 lie in one slot)
-#pragma unroll
-      for (int m = 0; m < W; ++m) {
-        const int j = J + m;
-        // pivot a_jj lives in lane j % 32, slot ps, column m
-        float own = r[0][m];
-        if (ps == 1) own = r[1][m];
-        if (ps == 2) own = r[2][m];
-        if (ps == 3) own = r[3][m];
-        const float piv = __shfl_sync(0xffffffffu, own, j & 31);
-        if (lane == 0 && !(piv > 0.f)) atomicOr(status, ISPA_STATUS_NOT_SPD);
-        const float sc = rsqrtf(piv);  // NaN for a non-positive pivot: poisons what follows
-        // scale column m of rows >= j: L_ij = a_ij / sqrt(a_jj)
-#pragma unroll
-        for (int s = 0; s < 4; ++s)
-          if (lane + 32 * s >= j) r[s][m] *= sc;
-        // update later panel columns: a_ic -= L_ij L_cj for rows i > j, c > j
-#pragma unroll
-        for (int cc = m + 1; cc < W; ++cc) {
-          float oc = r[0][m];
-          if (ps == 1) oc = r[1][m];
-          if (ps == 2) oc = r[2][m];
-          if (ps == 3) oc = r[3][m];
-          const float lcj = __shfl_sync(0xffffffffu, oc, (J + cc) & 31);   // L_{c j}, c = J + cc
-#pragma unroll
-          for (int s = 0; s < 4; ++s)
-            if (lane + 32 * s >= J + cc) r[s][cc] -= r[s][m] * lcj;
-        }
-      }
-#pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        const int i = lane + 32 * s;
-        if (i >= J)
-#pragma unroll
-          for (int m = 0; m < W; ++m) {
-            a[i][J + m] = r[s][m];
-            pan[i][m] = r[s][m];
-          }
-      }
-    }
-    __syncthreads();
-    // ---- (2) rows J..J+7 of Linv: forward substitution per column c <= J+7
-    if (t < J + W) {
-      const int c = t;
-      float zr[W];
-#pragma unroll
-      for (int m = 0; m < W; ++m) zr[m] = z[J + m][c];
-#pragma unroll
-      for (int m = 0; m < W; ++m) {
-#pragma unroll
-        for (int q = 0; q < m; ++q) zr[m] -= pan[J + m][q] * zr[q];
-        zr[m] /= pan[J + m][m];
-      }
-#pragma unroll
-      for (int m = 0; m < W; ++m) z[J + m][c] = zr[m];
-    }
-    __syncthreads();
-    // ---- (3) trailing: Z_ic -= sum_m L_im Linv_mc (c < J+8), A_ic -= sum_m L_im L_cm (J+8 <= c <= i)
-    const int ri = t >> 2, rq = t & 3;
-    if (ri >= J + W) {
-      float p[W];
-      {
-        const float4 v0 = *reinterpret_cast<const float4*>(&pan[ri][0]);
-        const float4 v1 = *reinterpret_cast<const float4*>(&pan[ri][4]);
-        p[0] = v0.x; p[1] = v0.y; p[2] = v0.z; p[3] = v0.w;
-        p[4] = v1.x; p[5] = v1.y; p[6] = v1.z; p[7] = v1.w;
-      }
-#pragma unroll 4
-      for (int c = rq; c < J + W; c += 4) {
-        float acc = z[ri][c];
-#pragma unroll
-        for (int m = 0; m < W; ++m) acc -= p[m] * z[J + m][c];
-        z[ri][c] = acc;
-      }
-#pragma unroll 4
-      for (int c = J + W + rq; c <= ri; c += 4) {
-        const float4 q0 = *reinterpret_cast<const float4*>(&pan[c][0]);
-        const float4 q1 = *reinterpret_cast<const float4*>(&pan[c][4]);
-        float acc = a[ri][c];
-        acc -= p[0] * q0.x + p[1] * q0.y + p[2] * q0.z + p[3] * q0.w;
-        acc -= p[4] * q1.x + p[5] * q1.y + p[6] * q1.z + p[7] * q1.w;
-        a[ri][c] = acc;
-      }
-    }
-    __syncthreads();
-  }
-  for (int e = t; e < NB * NB; e += blockDim.x) {
-    const int r = e >> 7, c = e & (NB - 1);
-    linv[e] = c <= r ? z[r][c] : 0.f;
-  }
+// dst[l] = src[l] for every layer l = blockIdx.y (float4 elements).
+__global__ void copy_layers_kernel(const float4* __restrict__ src, int64_t src_stride,
+                                   float4* __restrict__ dst, int64_t dst_stride, int64_t n4) {
+  const float4* s = src + (int64_t)blockIdx.y * src_stride;
+  float4* t = dst + (int64_t)blockIdx.y * dst_stride;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n4;
+       e += (int64_t)gridDim.x * blockDim.x)
+    t[e] = s[e];
 }
 
-constexpr size_t kPotrfSmem = (2 * NB * (NB + 1) + NB * 8) * sizeof(float) + 16;
+// Factors the 128 x 128 diagonal block at A (lower triangle used) as L L^T
+// and writes Linv = L^-1 (lower, zero above) to `linv`, in fp32. The sweep
+// over [A | Z], Z = I, runs in four 32-column steps J:
+//  (1) warp 0 factors the 32 x 32 diagonal sub-block and inverts it, in
+//      registers (lane l holds row l of L_JJ, then column l of L_JJ^-1);
+//      pivots and rows travel by warp shuffles, no barrier;
+//  (2) all 512 threads at once: the panel L_IJ = A_IJ L_JJ^-T for the m rows
+//      below (4 threads per row, 8 columns each) and the block row
+//      Z_J <- L_JJ^-1 Z_J (4 threads per column, 8 rows each);
+//      4 m + 4 (J + 32) = 512;
+//  (3) trailing update in 4 x 4 register tiles: A_II -= L_IJ L_IJ^T on the
+//      lower tiles and Z_I -= L_IJ Z_J.
+// Shared-memory row strides (132, 36, 100 floats) keep the float4 accesses
+// 16-byte aligned and free of bank conflicts.
+constexpr int kSA = 132;     // a, z: [128][kSA]
+constexpr int kSP = 36;      // panel, row-major [96][kSP]
+constexpr int kST = 100;     // panel, transposed [32][kST]
+constexpr int kSI = 36;      // L_JJ^-1, [32][kSI]
+constexpr size_t kPotrfSmem = (2 * NB * kSA + 96 * kSP + 32 * kST + 32 * kSI) * sizeof(float);
+
+__device__ __forceinline__ void ld4(float* d, const float* s) {
+  const float4 v = *reinterpret_cast<const float4*>(s);
+  d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+}
+__device__ __forceinline__ void st4(float* d, const float* s) {
+  *reinterpret_cast<float4*>(d) = make_float4(s[0], s[1], s[2], s[3]);
+}
+
+__global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restrict__ A0, int lda,
+                                                           float* __restrict__ linv0,
+                                                           int64_t ws_stride, int* status) {
+  const float* A = A0 + (int64_t)blockIdx.x * ws_stride;    // one block per layer
+  float* linv = linv0 + (int64_t)blockIdx.x * ws_stride;
+  extern __shared__ __align__(16) float sh[];
+  float* a = sh;
+  float* z = a + NB * kSA;
+  float* pl = z + NB * kSA;
+  float* plT = pl + 96 * kSP;
+  float* li = plT + 32 * kST;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  for (int e = t; e < NB * (NB / 4); e += blockDim.x) {
+    const int i = e >> 5, c = (e & 31) * 4;
+    *reinterpret_cast<float4*>(&a[i * kSA + c]) =
+        __ldg(reinterpret_cast<const float4*>(A + (size_t)i * lda + c));
+    *reinterpret_cast<float4*>(&z[i * kSA + c]) =
+        make_float4(i == c ? 1.f : 0.f, i == c + 1 ? 1.f : 0.f, i == c + 2 ? 1.f : 0.f,
+                    i == c + 3 ? 1.f : 0.f);
+  }
+  __syncthreads();
+  for (int J = 0; J < NB; J += 32) {
+    const int m = 96 - J;                       // rows below the diagonal sub-block
+    // ---- (1) L_JJ and L_JJ^-1
+    if (warp == 0) {
+      float r[32];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ld4(&r[4 * q], &a[(J + lane) * kSA + J + 4 * q]);
+#pragma unroll
+      for (int k = 0; k < 32; ++k) r[k] = (k <= lane) ? r[k] : 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float piv = __shfl_sync(0xffffffffu, r[j], j);
+        if (lane == 0 && !(piv > 0.f)) atomicOr(status, ISPA_STATUS_NOT_SPD);
+        const float inv = rsqrtf(piv);          // NaN for a non-positive pivot: poisons what follows
+        r[j] = lane > j ? r[j] * inv : (lane == j ? piv * inv : r[j]);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          if (c > j) {
+            const float lcj = __shfl_sync(0xffffffffu, r[j], c);
+            if (lane >= c) r[c] -= r[j] * lcj;
+          }
+        }
+      }
+      // column `lane` of L_JJ^-1 by forward substitution
+      float x[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) x[i] = (i == lane) ? 1.f : 0.f;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const float lkk = __shfl_sync(0xffffffffu, r[k], k);
+        x[k] = x[k] / lkk;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (i > k) x[i] -= __shfl_sync(0xffffffffu, r[k], i) * x[k];
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) li[i * kSI + lane] = x[i];
+    }
+    __syncthreads();
+    // ---- (2) panel rows and block row of Z, results held across the barrier
+    float o[8];
+    int p_row = 0, p_grp = 0;
+    const bool panel = t < 4 * m;
+    if (panel) {
+      p_row = t % m;                            // panel row J + 32 + p_row
+      p_grp = t / m;                            // columns 8 p_grp .. 8 p_grp + 7 (warp-uniform)
+      float ar[32];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ld4(&ar[4 * q], &a[(J + 32 + p_row) * kSA + J + 4 * q]);
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const float* lrow = &li[(8 * p_grp + c8) * kSI];
+        float acc = 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float l4[4];
+          ld4(l4, lrow + 4 * q);
+          acc = fmaf(ar[4 * q], l4[0], acc);
+          acc = fmaf(ar[4 * q + 1], l4[1], acc);
+          acc = fmaf(ar[4 * q + 2], l4[2], acc);
+          acc = fmaf(ar[4 * q + 3], l4[3], acc);
+        }
+        o[c8] = acc;
+      }
+    } else {
+      const int u = t - 4 * m, nc = J + 32;
+      p_row = u % nc;                           // column of Z
+      p_grp = u / nc;                           // rows J + 8 p_grp .. + 7 (warp-uniform)
+      float zc[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) zc[k] = z[(J + k) * kSA + p_row];
+#pragma unroll
+      for (int r8 = 0; r8 < 8; ++r8) {
+        const float* lrow = &li[(8 * p_grp + r8) * kSI];
+        float acc = 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float l4[4];
+          ld4(l4, lrow + 4 * q);
+          acc = fmaf(l4[0], zc[4 * q], acc);
+          acc = fmaf(l4[1], zc[4 * q + 1], acc);
+          acc = fmaf(l4[2], zc[4 * q + 2], acc);
+          acc = fmaf(l4[3], zc[4 * q + 3], acc);
+        }
+        o[r8] = acc;
+      }
+    }
+    __syncthreads();
+    if (panel) {
+      st4(&pl[p_row * kSP + 8 * p_grp], o);
+      st4(&pl[p_row * kSP + 8 * p_grp + 4], o + 4);
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) plT[(8 * p_grp + c8) * kST + p_row] = o[c8];
+    } else {
+#pragma unroll
+      for (int r8 = 0; r8 < 8; ++r8) z[(J + 8 * p_grp + r8) * kSA + p_row] = o[r8];
+    }
+    __syncthreads();
+    // ---- (3) trailing update, one 4 x 4 tile per thread (at most 492 tiles)
+    if (m > 0) {
+      const int mt = m / 4, n_tri = mt * (mt + 1) / 2, nzt = (J + 32) / 4;
+      if (t < n_tri + mt * nzt) {
+        int ti, tj;
+        const bool tri = t < n_tri;
+        if (tri) {
+          ti = (int)((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
+          while (ti * (ti + 1) / 2 > t) --ti;
+          while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
+          tj = t - ti * (ti + 1) / 2;
+        } else {
+          ti = (t - n_tri) / nzt;
+          tj = (t - n_tri) % nzt;
+        }
+        float acc[4][4] = {};
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float pa[4][4], pb[4][4];
+#pragma unroll
+          for (int r4 = 0; r4 < 4; ++r4) ld4(pa[r4], &pl[(4 * ti + r4) * kSP + 4 * q]);
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4)
+            ld4(pb[k4], tri ? &plT[(4 * q + k4) * kST + 4 * tj]
+                            : &z[(J + 4 * q + k4) * kSA + 4 * tj]);
+#pragma unroll
+          for (int r4 = 0; r4 < 4; ++r4)
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4)
+#pragma unroll
+              for (int c4 = 0; c4 < 4; ++c4) acc[r4][c4] = fmaf(pa[r4][k4], pb[k4][c4], acc[r4][c4]);
+        }
+        float* dst = tri ? &a[(J + 32 + 4 * ti) * kSA + J + 32 + 4 * tj]
+                         : &z[(J + 32 + 4 * ti) * kSA + 4 * tj];
+#pragma unroll
+        for (int r4 = 0; r4 < 4; ++r4) {
+          float v[4];
+          ld4(v, dst + r4 * kSA);
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) v[c4] -= acc[r4][c4];
+          st4(dst + r4 * kSA, v);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  for (int e = t; e < NB * (NB / 4); e += blockDim.x) {
+    const int i = e >> 5, c = (e & 31) * 4;
+    float v[4];
+    ld4(v, &z[i * kSA + c]);
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) v[c4] = (c + c4 <= i) ? v[c4] : 0.f;
+    st4(&linv[(size_t)i * NB + c], v);
+  }
+}
 
 void set_store(TGemmProblem& pr, int M, int N, int K, float* C, int64_t ldc, int64_t c_stride,
                int c_row0, int c_col0, float alpha, float beta, int layers) {
@@ -270,6 +359,11 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
     pr.b_mn = 1;
     if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
   }
+  // Y = B (every layer), the right-hand side of the forward substitution
+  copy_layers_kernel<<<dim3(n == 1 ? 148 * 4 : 148, n), 256, 0, stream>>>(
+      reinterpret_cast<const float4*>(B), b_stride / 4, reinterpret_cast<float4*>(Y), ws / 4,
+      (int64_t)(d * d / 4));
+  count_launches();
 
   potrf_inv_kernel<<<n, 512, kPotrfSmem, stream>>>(A, dim, Linv, ws, status);
   count_launches();
@@ -299,15 +393,25 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
         pr.a_mn = 0;
         pr.b_mn = 1;
       }
+      {
+        TGemmProblem& pr = p.prob[q++];
+        if (!opmap(&pr.ta, Linv, NB, NB, NB, n, ws, false) ||
+            !opmap(&pr.tb, Y + (size_t)kk * d, NB, d, d, n, ws, true))
+          return cudaErrorInvalidValue;
+        set_store(pr, NB, dim, NB, Y, dim, ws, kk, 0, 1.f, 0.f, n);
+        pr.a_mn = 0;
+        pr.b_mn = 1;
+      }
       p.nprob = q;
       if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
     }
     if (m <= 0) break;
-    // trailing: A_{>k,>k} -= L_{>k,k} L_{>k,k}^T (lower tiles); Z_{>k} -= L_{>k,k} Z_k
+    // trailing: A_{>k,>k} -= L_{>k,k} L_{>k,k}^T (lower tiles); Z_{>k} -= L_{>k,k} Z_k;
+    // Y_{>k} -= L_{>k,k} Y_k
     {
       TGemmParams p{};
       p.status = status;
-      p.nprob = 2;
+      p.nprob = 3;
       const float* Lk = A + (size_t)(kk + NB) * d + kk;
       TGemmProblem& t1 = p.prob[0];
       if (!opmap(&t1.ta, Lk, m, NB, d, n, ws, false) || !opmap(&t1.tb, Lk, m, NB, d, n, ws, false))
@@ -323,26 +427,20 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
       set_store(t2, m, kk + NB, NB, Z, dim, ws, kk + NB, 0, -1.f, 1.f, n);
       t2.a_mn = 0;
       t2.b_mn = 1;
+      TGemmProblem& t3 = p.prob[2];
+      if (!opmap(&t3.ta, Lk, m, NB, d, n, ws, false) ||
+          !opmap(&t3.tb, Y + (size_t)kk * d, NB, d, d, n, ws, true))
+        return cudaErrorInvalidValue;
+      set_store(t3, m, dim, NB, Y, dim, ws, kk + NB, 0, -1.f, 1.f, n);
+      t3.a_mn = 0;
+      t3.b_mn = 1;
       if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
     }
     potrf_inv_kernel<<<n, 512, kPotrfSmem, stream>>>(A + (size_t)(kk + NB) * d + kk + NB, dim,
                                                      Linv, ws, status);
     count_launches();
   }
-  // Y = Z B (Z lower triangular), Delta W = Z^T Y (Z^T upper triangular)
-  {
-    TGemmParams p{};
-    p.nprob = 1;
-    p.status = status;
-    TGemmProblem& pr = p.prob[0];
-    if (!opmap(&pr.ta, Z, d, d, d, n, ws, false) || !opmap(&pr.tb, B, d, d, d, n, b_stride, true))
-      return cudaErrorInvalidValue;
-    set_store(pr, dim, dim, dim, Y, dim, ws, 0, 0, 1.f, 0.f, n);
-    pr.a_mn = 0;
-    pr.b_mn = 1;
-    pr.tri = kTriLowerA;
-    if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
-  }
+  // Delta W = Z^T Y (Z^T upper triangular)
   {
     TGemmParams p{};
     p.nprob = 1;

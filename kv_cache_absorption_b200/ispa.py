@@ -34,6 +34,7 @@ EXPORTED = (
     "ispa_gram_accumulate", "ispa_absorb_workspace_size", "ispa_absorb_solve",
     "ispa_absorb_solve_noalloc", "ispa_absorb_solve_batched", "ispa_layer_error_batched",
     "ispa_layer_error_workspace_size", "ispa_layer_error", "ispa_rank_layers",
+    "ispa_weight_gram_batched", "ispa_layer_error_wwt_batched",
 )
 
 
@@ -77,6 +78,8 @@ def _load():
         "ispa_layer_error_workspace_size": (SZ, [I]),
         "ispa_layer_error": (I, [P, P, P, P, P, I, P, P, SZ, P]),
         "ispa_rank_layers": (I, [P, I, I, P, P, P]),
+        "ispa_weight_gram_batched": (I, [I, P, I64, I, P, I64, P, P]),
+        "ispa_layer_error_wwt_batched": (I, [I, P, I64, P, I64, P, I64, P, I64, P, I, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -324,6 +327,37 @@ def ispa_layer_error_batched(M, W, dW, B, lam, err=None, workspace=None, stream=
         dim, _ptr(err), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream))
     _check(rc, "ispa_layer_error_batched")
+    return err
+
+
+def ispa_weight_gram_batched(W, P=None, status=None, stream=None):
+    """P[l] = W[l] W[l]^T for W [L, d, d] fp32 (contiguous)."""
+    _dev_tensor(W, torch.float32, "W", 3)
+    L, dim = W.shape[0], W.shape[1]
+    P = torch.empty_like(W) if P is None else P
+    _dev_tensor(P, torch.float32, "P", 3)
+    status = new_status(W.device) if status is None else status
+    rc = _load().ispa_weight_gram_batched(L, _ptr(W), W.stride(0), dim, _ptr(P), P.stride(0),
+                                          _ptr(status), _stream(stream))
+    _check(rc, "ispa_weight_gram_batched")
+    return P
+
+
+def ispa_layer_error_wwt_batched(M, P, dW, B, lam, err=None, workspace=None, stream=None):
+    """Reconstruction errors of L layers from P = W W^T: device double [L, 2]."""
+    for t, n in ((M, "M"), (P, "P"), (dW, "dW"), (B, "B")):
+        _dev_tensor(t, torch.float32, n, 3)
+    _dev_tensor(lam, torch.float32, "lam", 1)
+    L, dim = P.shape[0], P.shape[1]
+    dev = P.device
+    err = torch.empty(L, 2, dtype=torch.float64, device=dev) if err is None else err
+    workspace = (torch.empty(L * ispa_layer_error_workspace_size(dim), dtype=torch.uint8,
+                             device=dev) if workspace is None else workspace)
+    rc = _load().ispa_layer_error_wwt_batched(
+        L, _ptr(M), M.stride(0), _ptr(P), P.stride(0), _ptr(dW), dW.stride(0), _ptr(B),
+        B.stride(0), _ptr(lam), dim, _ptr(err), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "ispa_layer_error_wwt_batched")
     return err
 
 

@@ -9,7 +9,10 @@ the layers are ranked; the K lowest-error layers become L-Layers.
 
 Every layer keeps its own statistics block M = [[G, R], [., S]], so the
 transition runs as two batched calls over all layers (solve, then error)
-instead of one pair of calls per layer.
+instead of one pair of calls per layer. The error uses W only through
+W W^T, a property of the model weights: ``weight_gram`` forms it once per
+layer when the weights are loaded, after which the error is one reduction
+pass per layer.
 
 Orchestration only: buffers and workspaces are allocated once (through
 torch) and every step is a call into the C ABI, so a warmup issues no
@@ -49,6 +52,7 @@ class LayerWarmup:
         self.dW = torch.empty(n_layers, d, d, **f32)
         self.B = torch.empty(n_layers, d, d, **f32)
         self.lam = torch.empty(n_layers, **f32)
+        self.P = None            # W W^T per layer, once weight_gram has run
         self._rows = 0
 
     def attention(self, ch: dict, stream=None):
@@ -106,12 +110,31 @@ class LayerWarmup:
             ispa._stream(stream))
         ispa._check(rc, "ispa_absorb_solve_batched")
 
+    def weight_gram(self, W_all: torch.Tensor, stream=None):
+        """P[l] = W[l] W[l]^T, formed once per set of weights."""
+        n, d = self.n_layers, self.d
+        _check_stack(W_all, n, d)
+        if self.P is None:
+            self.P = torch.empty(n, d, d, dtype=torch.float32, device=self.device)
+        rc = ispa._load().ispa_weight_gram_batched(
+            n, ispa._ptr(W_all), W_all.stride(0), d, ispa._ptr(self.P), d * d,
+            ispa._ptr(self.status), ispa._stream(stream))
+        ispa._check(rc, "ispa_weight_gram_batched")
+
     def error_all(self, W_all: torch.Tensor, err: torch.Tensor, stream=None):
-        """Every layer's {||E||^2, relative error} into err [n_layers, 2] fp64."""
+        """Every layer's {||E||^2, relative error} into err [n_layers, 2] fp64
+        (from W W^T when weight_gram has run, else from W)."""
         n, d = self.n_layers, self.d
         _check_stack(W_all, n, d)
         if err.dtype != torch.float64 or err.shape != (n, 2) or not err.is_contiguous():
             raise ValueError("err must be a contiguous float64 [n_layers, 2] tensor")
+        if self.P is not None:
+            rc = ispa._load().ispa_layer_error_wwt_batched(
+                n, ispa._ptr(self.M), 4 * d * d, ispa._ptr(self.P), d * d, ispa._ptr(self.dW),
+                d * d, ispa._ptr(self.B), d * d, ispa._ptr(self.lam), d, ispa._ptr(err),
+                ispa._ptr(self.err_ws), self.err_ws.numel(), ispa._stream(stream))
+            ispa._check(rc, "ispa_layer_error_wwt_batched")
+            return
         rc = ispa._load().ispa_layer_error_batched(
             n, ispa._ptr(self.M), 4 * d * d, ispa._ptr(W_all), W_all.stride(0),
             ispa._ptr(self.dW), d * d, ispa._ptr(self.B), d * d, ispa._ptr(self.lam), d,

@@ -35,7 +35,7 @@ def exported():
 
 def test_exports_match_header(ispa):
     names = declared()
-    assert len(names) == 15
+    assert len(names) == 17
     assert names == exported()
     assert names == set(ispa.EXPORTED)
     lib = ctypes.CDLL(ispa.LIB_PATH)
@@ -113,6 +113,18 @@ def test_other_entry_points_host_checks(ispa):
     assert lib.ispa_absorb_solve(P, P, 128, 0.0, P, P, None, P, 16, P, None) == ispa.ISPA_ERR_WORKSPACE
     assert lib.ispa_layer_error(P, P, P, P, None, 128, P, P, 256, None) == ispa.ISPA_ERR_ARG
     assert lib.ispa_layer_error(P, P, P, P, P, 128, P, P, 8, None) == ispa.ISPA_ERR_WORKSPACE
+    dd = 128 * 128
+    assert lib.ispa_weight_gram_batched(2, P, dd, 100, P, dd, P, None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert lib.ispa_weight_gram_batched(2, P, dd - 4, 128, P, dd, P, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_weight_gram_batched(2, P, dd, 128, P, dd + 2, P, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_weight_gram_batched(0, P, dd, 128, P, dd, P, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_weight_gram_batched(1, P + 4, dd, 128, P, dd, P, None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert lib.ispa_layer_error_wwt_batched(2, P, 4 * dd, P, dd, P, dd, P, dd, P, 128, P, P, 256,
+                                            None) == ispa.ISPA_ERR_WORKSPACE
+    assert lib.ispa_layer_error_wwt_batched(2, P, dd, P, dd, P, dd, P, dd, P, 128, P, P, 512,
+                                            None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_layer_error_wwt_batched(1, P, 4 * dd, None, dd, P, dd, P, dd, P, 128, P, P, 256,
+                                            None) == ispa.ISPA_ERR_ARG
     assert lib.ispa_rank_layers(P, 4, 5, P, None, None) == ispa.ISPA_ERR_ARG
     assert lib.ispa_rank_layers(P, 0, 0, P, None, None) == ispa.ISPA_ERR_ARG
 
