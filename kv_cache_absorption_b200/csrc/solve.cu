@@ -88,9 +88,10 @@ __global__ void copy_layers_kernel(const float4* __restrict__ src, int64_t src_s
 // Factors the 128 x 128 diagonal block at A (lower triangle used) as L L^T
 // and writes Linv = L^-1 (lower, zero above) to `linv`, in fp32. The sweep
 // over [A | Z], Z = I, runs in four 32-column steps J:
-//  (1) warp 0 factors the 32 x 32 diagonal sub-block and inverts it, in
-//      registers (lane l holds row l of L_JJ, then column l of L_JJ^-1);
-//      pivots and rows travel by warp shuffles, no barrier;
+//  (1) warp 0 factors the 32 x 32 diagonal sub-block in registers (lane l
+//      holds row l, a runtime loop over the columns keeps the code small
+//      enough for the instruction cache); all threads then invert L_JJ by
+//      recursive doubling over block sizes 1, 2, 4, 8, 16;
 //  (2) all 512 threads at once: the panel L_IJ = A_IJ L_JJ^-T for the m rows
 //      below (4 threads per row, 8 columns each) and the block row
 //      Z_J <- L_JJ^-1 Z_J (4 threads per column, 8 rows each);
@@ -103,7 +104,8 @@ constexpr int kSA = 132;     // a, z: [128][kSA]
 constexpr int kSP = 36;      // panel, row-major [96][kSP]
 constexpr int kST = 100;     // panel, transposed [32][kST]
 constexpr int kSI = 36;      // L_JJ^-1, [32][kSI]
-constexpr size_t kPotrfSmem = (2 * NB * kSA + 96 * kSP + 32 * kST + 32 * kSI) * sizeof(float);
+constexpr size_t kPotrfSmem =
+    (2 * NB * kSA + 96 * kSP + 32 * kST + 3 * 32 * kSI + 32) * sizeof(float);
 
 __device__ __forceinline__ void ld4(float* d, const float* s) {
   const float4 v = *reinterpret_cast<const float4*>(s);
@@ -123,7 +125,10 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
   float* z = a + NB * kSA;
   float* pl = z + NB * kSA;
   float* plT = pl + 96 * kSP;
-  float* li = plT + 32 * kST;
+  float* li = plT + 32 * kST;                  // L_JJ^-1
+  float* ljj = li + 32 * kSI;                   // L_JJ
+  float* ytmp = ljj + 32 * kSI;                 // C A^-1 blocks of the inversion
+  float* colv = ytmp + 32 * kSI;                // one rotated column of L_JJ
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   for (int e = t; e < NB * (NB / 4); e += blockDim.x) {
     const int i = e >> 5, c = (e & 31) * 4;
@@ -136,43 +141,63 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
   __syncthreads();
   for (int J = 0; J < NB; J += 32) {
     const int m = 96 - J;                       // rows below the diagonal sub-block
-    // ---- (1) L_JJ and L_JJ^-1
+    // ---- (1a) warp 0: L_JJ, a compact loop (lane l holds row l; r[0] is the
+    // current column, the row shifts left by one column per step)
     if (warp == 0) {
       float r[32];
 #pragma unroll
       for (int q = 0; q < 8; ++q) ld4(&r[4 * q], &a[(J + lane) * kSA + J + 4 * q]);
 #pragma unroll
       for (int k = 0; k < 32; ++k) r[k] = (k <= lane) ? r[k] : 0.f;
-#pragma unroll
+#pragma unroll 1
       for (int j = 0; j < 32; ++j) {
-        const float piv = __shfl_sync(0xffffffffu, r[j], j);
+        const float piv = __shfl_sync(0xffffffffu, r[0], j);
         if (lane == 0 && !(piv > 0.f)) atomicOr(status, ISPA_STATUS_NOT_SPD);
-        const float inv = rsqrtf(piv);          // NaN for a non-positive pivot: poisons what follows
-        r[j] = lane > j ? r[j] * inv : (lane == j ? piv * inv : r[j]);
+        const float inv = rsqrtf(piv);         // NaN for a non-positive pivot: poisons what follows
+        const float l0 = lane > j ? r[0] * inv : (lane == j ? piv * inv : 0.f);   // L[lane][j]
+        ljj[lane * kSI + j] = l0;
+        // column j rotated so that slot c holds L[j + c][j]; slots past row 31 hold 0
+        colv[lane >= j ? lane - j : lane - j + 32] = lane >= j ? l0 : 0.f;
+        __syncwarp();
+        float cv[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          if (c > j) {
-            const float lcj = __shfl_sync(0xffffffffu, r[j], c);
-            if (lane >= c) r[c] -= r[j] * lcj;
-          }
-        }
+        for (int q = 0; q < 8; ++q) ld4(&cv[4 * q], &colv[4 * q]);
+#pragma unroll
+        for (int c = 1; c < 32; ++c) r[c - 1] = fmaf(-l0, cv[c], r[c]);
+        r[31] = 0.f;
+        __syncwarp();
       }
-      // column `lane` of L_JJ^-1 by forward substitution
-      float x[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) x[i] = (i == lane) ? 1.f : 0.f;
-#pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const float lkk = __shfl_sync(0xffffffffu, r[k], k);
-        x[k] = x[k] / lkk;
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (i > k) x[i] -= __shfl_sync(0xffffffffu, r[k], i) * x[k];
-      }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) li[i * kSI + lane] = x[i];
     }
     __syncthreads();
+    // ---- (1b) L_JJ^-1 by recursive doubling: with A^-1 and B^-1 known for two
+    // diagonal blocks of size b, the block below them is -B^-1 C A^-1
+    for (int e = t; e < 32 * 32; e += blockDim.x) {
+      const int i = e >> 5, c = e & 31;
+      li[i * kSI + c] = i == c ? 1.f / ljj[i * kSI + i] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int b = 1; b < 32; b *= 2) {
+      const bool act = t < 16 * b;             // 16 / b block pairs, b^2 entries each
+      int row = 0, c0 = 0, p0 = 0;
+      if (act) {
+        const int pair = t / (b * b), e = t % (b * b);
+        p0 = pair * 2 * b;
+        row = p0 + b + e / b;
+        c0 = p0 + e % b;
+        float y = 0.f;
+        for (int k = 0; k < b; ++k) y = fmaf(ljj[row * kSI + p0 + k], li[(p0 + k) * kSI + c0], y);
+        ytmp[row * kSI + c0] = y;                // (C A^-1)
+      }
+      __syncthreads();
+      if (act) {
+        float x = 0.f;
+        for (int k = 0; k < b; ++k)
+          x = fmaf(li[row * kSI + p0 + b + k], ytmp[(p0 + b + k) * kSI + c0], x);
+        li[row * kSI + c0] = -x;                 // -B^-1 (C A^-1)
+      }
+      __syncthreads();
+    }
     // ---- (2) panel rows and block row of Z, results held across the barrier
     float o[8];
     int p_row = 0, p_grp = 0;
