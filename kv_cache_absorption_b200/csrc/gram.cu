@@ -36,8 +36,8 @@ struct alignas(1024) GramSmem {
   uint8_t b[NSTAGE][BN / 32][BK * 128];
   uint64_t full[NSTAGE];
   uint64_t empty[NSTAGE];
-  uint64_t acc_full;
-  uint64_t acc_empty;
+  uint64_t acc_full[2];     // segment accumulated in TMEM buffer b
+  uint64_t acc_empty[2];    // buffer b drained by the epilogue
   uint64_t drain;
   uint32_t taddr;
   int abort_flag;
@@ -90,13 +90,17 @@ __global__ void __launch_bounds__(kThreads, 1) gram_kernel(const __grid_constant
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NSTAGE; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
-    mbar_init(&s.acc_full, 1);
-    mbar_init(&s.acc_empty, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s.acc_full[b], 1);
+      mbar_init(&s.acc_empty[b], 128);
+    }
     mbar_init(&s.drain, 1);
     s.abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) { tmem_alloc(&s.taddr, BN); tmem_relinquish(); }
+  // two accumulators: segment seg uses buffer seg & 1, so the epilogue of one
+  // segment overlaps the MMAs of the next
+  if (warp == 1) { tmem_alloc(&s.taddr, 2 * BN); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -146,23 +150,28 @@ __global__ void __launch_bounds__(kThreads, 1) gram_kernel(const __grid_constant
       for (int64_t it = it_begin; ok && it < it_end; ++seg) {
         const int kb = (int)(it % p.k_iters);
         const int ke = (int)(kb + (it_end - it) < p.k_iters ? kb + (it_end - it) : p.k_iters);
-        // the epilogue must have drained the previous segment's accumulator
-        if (seg > 0 && !mbar_wait(&s.acc_empty, (seg - 1) & 1, p.status, abort_flag)) { ok = false; break; }
+        // the epilogue must have drained this buffer's previous segment (seg - 2)
+        if (seg >= 2 &&
+            !mbar_wait(&s.acc_empty[seg & 1], ((seg - 2) >> 1) & 1, p.status, abort_flag)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
+        const uint32_t acc = tacc + (uint32_t)((seg & 1) * BN);
         for (int k = kb; k < ke; ++k, ++n) {
           const int st = (int)(n % NSTAGE);
           if (!mbar_wait(&s.full[st], (n / NSTAGE) & 1, p.status, abort_flag)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < BK / 8; ++kk) {
-            mma_ss_tf32(tacc, smem_desc(smem_u32(s.a[st][0]) + kk * 1024, BK * 128, 512, 1),
+            mma_ss_tf32(acc, smem_desc(smem_u32(s.a[st][0]) + kk * 1024, BK * 128, 512, 1),
                         smem_desc(smem_u32(s.b[st][0]) + kk * 1024, BK * 128, 512, 1), idesc,
                         (k == kb && kk == 0) ? 0u : 1u);
           }
           tc_commit(&s.empty[st]);
         }
         if (!ok) break;
-        tc_commit(&s.acc_full);
+        tc_commit(&s.acc_full[seg & 1]);
         it += ke - kb;
       }
       if (!ok) {
@@ -183,15 +192,16 @@ __global__ void __launch_bounds__(kThreads, 1) gram_kernel(const __grid_constant
       const int kb = (int)(it % p.k_iters);
       const int ke = (int)(kb + (it_end - it) < p.k_iters ? kb + (it_end - it) : p.k_iters);
       const Tile t = decode_tile(tile, p.dim, BN);
-      if (!mbar_wait(&s.acc_full, seg & 1, p.status, abort_flag)) break;
+      if (!mbar_wait(&s.acc_full[seg & 1], (seg >> 1) & 1, p.status, abort_flag)) break;
       tc_fence_after();
+      const uint32_t acc = tacc + (uint32_t)((seg & 1) * BN);
       const int64_t row = (int64_t)t.I * BM + r + (t.type == 2 ? p.dim : 0);
       const int64_t col0 = (int64_t)t.J * BN + (t.type == 0 ? 0 : p.dim);
       float* dst_row = p.M + row * ld + col0;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t v[32];
-        tmem_ld32(tacc + lane_off + c * 32, v);
+        tmem_ld32(acc + lane_off + c * 32, v);
         tmem_ld_wait();
         // G and S: skip 128-column sub-blocks left of the diagonal block
         const int jblk = (t.J * BN + c * 32) / 128;
@@ -203,13 +213,13 @@ __global__ void __launch_bounds__(kThreads, 1) gram_kernel(const __grid_constant
                                         __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3])));
       }
       tc_fence_before();
-      mbar_arrive(&s.acc_empty);
+      mbar_arrive(&s.acc_empty[seg & 1]);
       it += ke - kb;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tacc, BN);
+  if (warp == 1) tmem_dealloc(tacc, 2 * BN);
 }
 
 }  // namespace

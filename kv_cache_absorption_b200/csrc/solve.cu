@@ -10,13 +10,22 @@
 // Organisation (block size 128, all products fp32-accurate 3xTF32 tensor-
 // core GEMMs, see tgemm.cu):
 //   * B = R W first (returned for the error computation);
-//   * one right-looking sweep over the 128-column panels factors A in place
-//     and, on the augmented block [A | Z | Y] with Z = I and Y = B, also
-//     yields Z = L^-1 and Y = L^-1 B (forward substitution). Step k: factor
-//     and invert the diagonal block (one CTA, fp32, shared memory); panel
-//     L_{>k,k} = A_{>k,k} Linv_kk^T and block rows Z_k = Linv_kk Z_k,
-//     Y_k = Linv_kk Y_k (one grouped launch); trailing update of the lower
-//     tiles of A and of the rows of Z and Y below k (one grouped launch);
+//   * one sweep over the 128-column blocks factors A in place and, on the
+//     augmented block [A | Z | Y] with Z = I and Y = B, also yields
+//     Z = L^-1 and Y = L^-1 B (forward substitution). Every step factors and
+//     inverts the diagonal block (one CTA per layer, fp32, shared memory) and
+//     forms the panel L_{>k,k} = A_{>k,k} Linv_kk^T and the block rows
+//     Z_k = Linv_kk Z_k, Y_k = Linv_kk Y_k (one grouped launch).
+//     Several layers: left-looking. Before step k, one grouped launch of
+//     long-K products brings block column k of A and block rows k of Z and Y
+//     up to date (A_{>=k,k} -= L_{>=k,<k} L_{k,<k}^T, Y_k -= L_{k,<k} Y_{<k},
+//     Z_k = -L_{k,<k} Z_{<k}); the finished part is read once per step and
+//     nothing below the block is rewritten, so HBM traffic stays low; these
+//     products sum K in 128-deep chunks (fp32) against accumulator drift.
+//     One layer: right-looking. After step k one grouped launch applies the
+//     rank-128 update to the lower tiles of A and to the rows of Z and Y
+//     below the block: more traffic, but (d/128)^2 tiles per launch where
+//     the left-looking step of a single layer would have ~2 d/128;
 //   * then one triangular-aware GEMM: Delta W = Z^T Y.
 // Y is formed by substitution, not as the product Z B: entries of L^-1
 // alternate in sign and |L^-1| |B| can exceed |L^-1 B| by three orders of
@@ -33,6 +42,9 @@ namespace ispa {
 namespace {
 
 constexpr int NB = 128;
+// Long-K products accumulate K = 128 per tensor-core accumulator and sum the
+// chunks in fp32 (see tgemm.cu).
+constexpr int kChunkSlabs = 4;
 
 // lambda = value if value > 0, else 1e-2 * trace(G) / dim (G = M[0:d, 0:d]);
 // one block per layer.
@@ -339,6 +351,45 @@ bool opmap(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols, uint
                                mn_major);
 }
 
+// Panel of step k (all in place): L_{>k,k} = A_{>k,k} Linv^T, Z_k = Linv Z_k,
+// Y_k = Linv Y_k, with Linv = L_kk^-1 from potrf_inv_kernel.
+cudaError_t panel_launch(int n, float* A, float* Z, float* Y, const float* Linv, size_t d, int kk,
+                         int m, int64_t ws, int* status, cudaStream_t stream) {
+  const int dim = (int)d;
+  TGemmParams p{};
+  p.status = status;
+  int q = 0;
+  if (m > 0) {
+    TGemmProblem& pr = p.prob[q++];
+    if (!opmap(&pr.ta, A + (size_t)(kk + NB) * d + kk, m, NB, d, n, ws, false) ||
+        !opmap(&pr.tb, Linv, NB, NB, NB, n, ws, false))
+      return cudaErrorInvalidValue;
+    set_store(pr, m, NB, NB, A, dim, ws, kk + NB, kk, 1.f, 0.f, n);
+    pr.a_mn = 0;
+    pr.b_mn = 0;
+  }
+  {
+    TGemmProblem& pr = p.prob[q++];
+    if (!opmap(&pr.ta, Linv, NB, NB, NB, n, ws, false) ||
+        !opmap(&pr.tb, Z + (size_t)kk * d, NB, kk + NB, d, n, ws, true))
+      return cudaErrorInvalidValue;
+    set_store(pr, NB, kk + NB, NB, Z, dim, ws, kk, 0, 1.f, 0.f, n);
+    pr.a_mn = 0;
+    pr.b_mn = 1;
+  }
+  {
+    TGemmProblem& pr = p.prob[q++];
+    if (!opmap(&pr.ta, Linv, NB, NB, NB, n, ws, false) ||
+        !opmap(&pr.tb, Y + (size_t)kk * d, NB, d, d, n, ws, true))
+      return cudaErrorInvalidValue;
+    set_store(pr, NB, dim, NB, Y, dim, ws, kk, 0, 1.f, 0.f, n);
+    pr.a_mn = 0;
+    pr.b_mn = 1;
+  }
+  p.nprob = q;
+  return launch_tgemm(p, stream);
+}
+
 }  // namespace
 
 size_t absorb_workspace_bytes(int dim) {
@@ -375,6 +426,7 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
     TGemmParams p{};
     p.nprob = 1;
     p.status = status;
+    p.kchunk = kChunkSlabs;
     TGemmProblem& pr = p.prob[0];
     if (!opmap(&pr.ta, M + d, d, d, 2 * d, n, m_stride, false) ||
         !opmap(&pr.tb, W, d, d, d, n, w_stride, true))
@@ -390,50 +442,23 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
       (int64_t)(d * d / 4));
   count_launches();
 
-  potrf_inv_kernel<<<n, 512, kPotrfSmem, stream>>>(A, dim, Linv, ws, status);
-  count_launches();
-  for (int k = 0; k < nblk; ++k) {
-    const int kk = k * NB;
-    const int m = dim - kk - NB;   // rows below the panel
-    // panel: L_{>k,k} = A_{>k,k} Linv^T (in place); Z_k = Linv Z_k (in place)
-    {
-      TGemmParams p{};
-      p.status = status;
-      int q = 0;
-      if (m > 0) {
-        TGemmProblem& pr = p.prob[q++];
-        if (!opmap(&pr.ta, A + (size_t)(kk + NB) * d + kk, m, NB, d, n, ws, false) ||
-            !opmap(&pr.tb, Linv, NB, NB, NB, n, ws, false))
-          return cudaErrorInvalidValue;
-        set_store(pr, m, NB, NB, A, dim, ws, kk + NB, kk, 1.f, 0.f, n);
-        pr.a_mn = 0;
-        pr.b_mn = 0;
-      }
-      {
-        TGemmProblem& pr = p.prob[q++];
-        if (!opmap(&pr.ta, Linv, NB, NB, NB, n, ws, false) ||
-            !opmap(&pr.tb, Z + (size_t)kk * d, NB, kk + NB, d, n, ws, true))
-          return cudaErrorInvalidValue;
-        set_store(pr, NB, kk + NB, NB, Z, dim, ws, kk, 0, 1.f, 0.f, n);
-        pr.a_mn = 0;
-        pr.b_mn = 1;
-      }
-      {
-        TGemmProblem& pr = p.prob[q++];
-        if (!opmap(&pr.ta, Linv, NB, NB, NB, n, ws, false) ||
-            !opmap(&pr.tb, Y + (size_t)kk * d, NB, d, d, n, ws, true))
-          return cudaErrorInvalidValue;
-        set_store(pr, NB, dim, NB, Y, dim, ws, kk, 0, 1.f, 0.f, n);
-        pr.a_mn = 0;
-        pr.b_mn = 1;
-      }
-      p.nprob = q;
-      if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
-    }
-    if (m <= 0) break;
-    // trailing: A_{>k,>k} -= L_{>k,k} L_{>k,k}^T (lower tiles); Z_{>k} -= L_{>k,k} Z_k;
-    // Y_{>k} -= L_{>k,k} Y_k
-    {
+  // One layer: right-looking (a rank-128 update of everything below the block
+  // after each step): up to (d/128)^2 tiles per launch keep the GPU busy.
+  // Several layers: left-looking (long-K products that read the finished
+  // part once): far less HBM traffic, and the layers supply the parallelism.
+  const bool left_looking = n > 1;
+  if (!left_looking) {
+    for (int k = 0; k < nblk; ++k) {
+      const int kk = k * NB;
+      const int m = dim - kk - NB;
+      potrf_inv_kernel<<<n, 512, kPotrfSmem, stream>>>(A + (size_t)kk * d + kk, dim, Linv, ws,
+                                                       status);
+      count_launches();
+      if ((e = panel_launch(n, A, Z, Y, Linv, d, kk, m, ws, status, stream)) != cudaSuccess)
+        return e;
+      if (m <= 0) break;
+      // A_{>k,>k} -= L_{>k,k} L_{>k,k}^T (lower tiles); Z_{>k} -= L_{>k,k} Z_k;
+      // Y_{>k} -= L_{>k,k} Y_k
       TGemmParams p{};
       p.status = status;
       p.nprob = 3;
@@ -461,15 +486,58 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
       t3.b_mn = 1;
       if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
     }
-    potrf_inv_kernel<<<n, 512, kPotrfSmem, stream>>>(A + (size_t)(kk + NB) * d + kk + NB, dim,
-                                                     Linv, ws, status);
+  }
+  for (int k = 0; left_looking && k < nblk; ++k) {
+    const int kk = k * NB;
+    const int m = dim - kk - NB;   // rows below the diagonal block
+    if (k > 0) {
+      // bring block column k of A and block rows k of Y and Z up to date with
+      // the finished blocks 0..k-1 (left-looking: long-K products that read
+      // the finished part once instead of rewriting the trailing matrix)
+      TGemmParams p{};
+      p.status = status;
+      p.nprob = 3;
+      p.kchunk = kChunkSlabs;
+      const float* Lrow = A + (size_t)kk * d;   // L_{k,<k}: rows kk.., columns 0..kk-1
+      // A_{>=k,k} -= L_{>=k,<k} L_{k,<k}^T
+      TGemmProblem& u1 = p.prob[0];
+      if (!opmap(&u1.ta, Lrow, d - kk, kk, d, n, ws, false) ||
+          !opmap(&u1.tb, Lrow, NB, kk, d, n, ws, false))
+        return cudaErrorInvalidValue;
+      set_store(u1, dim - kk, NB, kk, A, dim, ws, kk, kk, -1.f, 1.f, n);
+      u1.a_mn = 0;
+      u1.b_mn = 0;
+      // Y_k -= L_{k,<k} Y_{<k}
+      TGemmProblem& u2 = p.prob[1];
+      if (!opmap(&u2.ta, Lrow, NB, kk, d, n, ws, false) ||
+          !opmap(&u2.tb, Y, kk, d, d, n, ws, true))
+        return cudaErrorInvalidValue;
+      set_store(u2, NB, dim, kk, Y, dim, ws, kk, 0, -1.f, 1.f, n);
+      u2.a_mn = 0;
+      u2.b_mn = 1;
+      // Z_k[:, <kk] = -L_{k,<k} Z_{<k} (Z_{<k} lower triangular)
+      TGemmProblem& u3 = p.prob[2];
+      if (!opmap(&u3.ta, Lrow, NB, kk, d, n, ws, false) ||
+          !opmap(&u3.tb, Z, kk, kk, d, n, ws, true))
+        return cudaErrorInvalidValue;
+      set_store(u3, NB, kk, kk, Z, dim, ws, kk, 0, -1.f, 0.f, n);
+      u3.a_mn = 0;
+      u3.b_mn = 1;
+      u3.tri = kTriLowerB;
+      if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
+    }
+    potrf_inv_kernel<<<n, 512, kPotrfSmem, stream>>>(A + (size_t)kk * d + kk, dim, Linv, ws,
+                                                     status);
     count_launches();
+    if ((e = panel_launch(n, A, Z, Y, Linv, d, kk, m, ws, status, stream)) != cudaSuccess)
+      return e;
   }
   // Delta W = Z^T Y (Z^T upper triangular)
   {
     TGemmParams p{};
     p.nprob = 1;
     p.status = status;
+    p.kchunk = kChunkSlabs;
     TGemmProblem& pr = p.prob[0];
     if (!opmap(&pr.ta, Z, d, d, d, n, ws, true) || !opmap(&pr.tb, Y, d, d, d, n, ws, true))
       return cudaErrorInvalidValue;

@@ -14,11 +14,18 @@
 // (the K index contiguous) or MN-major (M or N contiguous), so transposes
 // cost nothing. A launch may hold up to 4 independent problems ("grouped");
 // a problem can be restricted to the tiles on or below its diagonal, and to
-// the K range a triangular A operand leaves non-zero.
+// the K range a triangular A or B operand leaves non-zero.
 //
 // Warp roles (192 threads): warp 0 TMA producer (3-stage ring of 32-deep K
 // slabs), warp 1 TMEM owner and MMA issuer, warps 2-5 split each slab into
 // hi/lo and then run the epilogue.
+//
+// Long K: the tensor core's accumulator does not round its additions to
+// nearest, and over thousands of terms with heavy cancellation (the Schur
+// complements of the Cholesky sweep) the drift reaches 1e-3 of the result.
+// With kchunk > 0 each chunk of kchunk slabs is accumulated in a fresh TMEM
+// buffer (two, in turn) and warps 2-5 add it to a running sum in TMEM with
+// fp32 round-to-nearest additions while the next chunk is in flight.
 #include "sm100.cuh"
 #include "attention.h"
 #include "tgemm.h"
@@ -40,6 +47,8 @@ struct alignas(1024) GSmem {
   uint64_t split[NSTAGE];   // hi/lo written
   uint64_t empty[NSTAGE];   // MMAs done reading
   uint64_t acc_full;
+  uint64_t chunk_full[2];   // chunk accumulated in buffer b
+  uint64_t chunk_empty[2];  // buffer b added to the running sum
   uint64_t drain;
   uint32_t taddr;
   int abort_flag;
@@ -76,11 +85,12 @@ __device__ __forceinline__ void decode(const TGemmParams& p, int b, int& q, int&
   }
 }
 
-__device__ __forceinline__ void k_range(const TGemmProblem& pr, int i, int& kb, int& ke) {
+__device__ __forceinline__ void k_range(const TGemmProblem& pr, int i, int j, int& kb, int& ke) {
   kb = 0;
   ke = pr.K / TK;
   if (pr.tri == kTriLowerA) ke = min(ke, (i + 1) * (TM / TK));
   if (pr.tri == kTriUpperA) kb = i * (TM / TK);
+  if (pr.tri == kTriLowerB) kb = min(ke, j * (TN / TK));
 }
 
 // Loads one 32-deep slab of a 128-wide operand block (rows/cols starting at
@@ -110,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
   decode(p, blockIdx.x, q, layer, ti, tj);
   const TGemmProblem& pr = p.prob[q];
   int kb, ke;
-  k_range(pr, ti, kb, ke);
+  k_range(pr, ti, tj, kb, ke);
   const int nk = ke - kb;
 
   if (threadIdx.x == 0) {
@@ -120,11 +130,19 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
       mbar_init(&s.empty[i], 1);
     }
     mbar_init(&s.acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s.chunk_full[b], 1);
+      mbar_init(&s.chunk_empty[b], 128);
+    }
     mbar_init(&s.drain, 1);
     s.abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) { tmem_alloc(&s.taddr, TN); tmem_relinquish(); }
+  // TMEM: running sum (columns 0..127) and, with chunking, two chunk buffers
+  const int kc = p.kchunk;
+  const int nchunks = kc > 0 ? (nk + kc - 1) / kc : 1;
+  constexpr int kTmemCols = 512;
+  if (warp == 1) { tmem_alloc(&s.taddr, kTmemCols); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -156,18 +174,28 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
       bool ok = true;
       for (int n = 0; n < nk; ++n) {
         const int st = n % NSTAGE;
+        const int c = kc > 0 ? n / kc : 0;               // chunk of this slab
+        const bool first = kc > 0 ? (n % kc == 0) : (n == 0);
+        // chunk c >= 1 goes to buffer (c - 1) & 1, free once chunk c - 2 was summed
+        if (first && c >= 3 &&
+            !mbar_wait(&s.chunk_empty[(c - 1) & 1], ((c - 3) >> 1) & 1, p.status, abort_flag)) {
+          ok = false;
+          break;
+        }
         if (!mbar_wait(&s.split[st], (n / NSTAGE) & 1, p.status, abort_flag)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t dst = c >= 1 ? tacc + (uint32_t)(TN * (1 + ((c - 1) & 1))) : tacc;
         const uint64_t ah = slab_desc(s.a_hi[st], pr.a_mn), al = slab_desc(s.a_lo[st], pr.a_mn);
         const uint64_t bh = slab_desc(s.b_hi[st], pr.b_mn), bl = slab_desc(s.b_lo[st], pr.b_mn);
 #pragma unroll
         for (int kk = 0; kk < TK / 8; ++kk) {
-          const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
-          mma_ss_tf32(tacc, ah + kk * a_step, bh + kk * b_step, idesc, acc);
-          mma_ss_tf32(tacc, ah + kk * a_step, bl + kk * b_step, idesc, 1u);
-          mma_ss_tf32(tacc, al + kk * a_step, bh + kk * b_step, idesc, 1u);
+          const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
+          mma_ss_tf32(dst, ah + kk * a_step, bh + kk * b_step, idesc, acc);
+          mma_ss_tf32(dst, ah + kk * a_step, bl + kk * b_step, idesc, 1u);
+          mma_ss_tf32(dst, al + kk * a_step, bh + kk * b_step, idesc, 1u);
         }
         tc_commit(&s.empty[st]);
+        if (c >= 1 && (n % kc == kc - 1 || n == nk - 1)) tc_commit(&s.chunk_full[(c - 1) & 1]);
       }
       if (ok) tc_commit(&s.acc_full);
       else { tc_commit(&s.drain); drain_wait(&s.drain, 0, p.status); }
@@ -176,9 +204,35 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
   } else {
     // ---------------------------------------------------- split, then epilogue
     const int et = threadIdx.x - 64;   // 0..127
+    const uint32_t row_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    // running sum += chunk c (c >= 1), then release its buffer
+    auto sum_chunk = [&](int c) -> bool {
+      const int b = (c - 1) & 1;
+      if (!mbar_wait(&s.chunk_full[b], ((c - 1) >> 1) & 1, p.status, abort_flag)) return false;
+      tc_fence_after();
+#pragma unroll 1
+      for (int q = 0; q < TN / 32; ++q) {
+        uint32_t v[32], w[32];
+        tmem_ld32(tacc + row_off + q * 32, v);
+        tmem_ld32(tacc + row_off + (uint32_t)(TN * (1 + b)) + q * 32, w);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(w[i]));
+        tmem_st32(tacc + row_off + q * 32, v);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&s.chunk_empty[b]);
+      return true;
+    };
     bool ok = true;
+    int summed = 0;                      // chunks 1..summed are in the running sum
     for (int n = 0; n < nk; ++n) {
       const int st = n % NSTAGE;
+      if (kc > 0 && n % kc == 0 && n / kc >= 3) {
+        if (!sum_chunk(n / kc - 2)) { ok = false; break; }
+        summed = n / kc - 2;
+      }
       if (!mbar_wait(&s.full[st], (n / NSTAGE) & 1, p.status, abort_flag)) { ok = false; break; }
 #pragma unroll 4
       for (int v = et; v < 2 * kSlab / 16; v += 128) {
@@ -198,9 +252,10 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
       fence_proxy_async_smem();   // generic-proxy writes -> visible to the MMA (async proxy)
       mbar_arrive(&s.split[st]);
     }
+    for (int c = summed + 1; ok && kc > 0 && c < nchunks; ++c) ok = sum_chunk(c);
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t lane_off = row_off;
     const int64_t row = (int64_t)pr.c_row0 + (int64_t)ti * TM + r;
     const int64_t col0 = (int64_t)pr.c_col0 + (int64_t)tj * TN;
     if (ok && (nk == 0 || mbar_wait(&s.acc_full, 0, p.status, abort_flag))) {
@@ -273,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tacc, TN);
+  if (warp == 1) tmem_dealloc(tacc, kTmemCols);
 }
 
 }  // namespace

@@ -9,6 +9,7 @@ namespace ispa {
 constexpr int kTriNone = 0;
 constexpr int kTriLowerA = 1;   // op(A) lower triangular: row block i reads K blocks 0..i
 constexpr int kTriUpperA = 2;   // op(A) upper triangular: row block i reads K blocks i..
+constexpr int kTriLowerB = 3;   // op(B) lower triangular: column block j reads K blocks j..
 constexpr int kModeStore = 0;   // C = alpha * op(A) op(B) + beta * C
 constexpr int kModeDot3 = 1;    // accumulate <P, G>, <P, R>, <P, S> (P = op(A) op(B))
 
@@ -45,6 +46,8 @@ struct TGemmParams {
   int dot_dim;
   double* dot_acc;         // kModeDot3: 3 accumulators of layer 0
   int dot_acc_stride;      // doubles between layers' accumulators
+  int kchunk;              // > 0: accumulate K in chunks of kchunk 32-deep slabs, each in a
+                           // fresh accumulator, and sum the chunks in fp32 (round to nearest)
   int* status;
 };
 
