@@ -198,11 +198,14 @@ class ClockSampler:
 _ORACLE_INPUTS = {}
 
 
-def oracle_timing(cfg, sample_rows: int, seed: int = 0):
-    """Times the float64 oracle on a bounded sample of one layer of ``cfg``:
-    dual attention of ``sample_rows`` query rows of the last chunk (all heads,
-    all keys), the Gram of those rows, the full-size closed-form solve and the
-    direct error on the sampled rows. Returns per-stage (flops, seconds)."""
+def oracle_timing(cfg, att_rows: int, gram_rows: int = 1024, seed: int = 0):
+    """Times the float64 oracle on a bounded sample of one layer of ``cfg``,
+    each stage at a size where its cost scales with the work: dual attention
+    of ``att_rows`` query rows of the last chunk (all heads, all keys); the
+    Gram and the direct error of ``gram_rows`` rows (the attention rows
+    repeated: their cost does not depend on the values); the full-size
+    closed-form solve. Returns per-stage (flops, seconds)."""
+    import numpy as np
     import oracle
     from ispa_synth import layer_streams
     key = (cfg.name, seed)
@@ -211,26 +214,31 @@ def oracle_timing(cfg, sample_rows: int, seed: int = 0):
         _ORACLE_INPUTS[key] = (st.chunk(cfg.n_chunks - 1), st.w)
     ch, w = _ORACLE_INPUTS[key]
     sub = dict(ch)
-    sub["q"] = ch["q"][:sample_rows]
+    sub["q"] = ch["q"][:att_rows]
     nk = ch["k_sink"].shape[0] + ch["k_loc"].shape[0] + ch["k_hist"].shape[0]
     d = cfg.d
     t0 = time.perf_counter()
     o = oracle.dual_attention(sub["q"], sub["k_sink"], sub["v_sink"], sub["k_loc"], sub["v_loc"],
                               sub["k_hist"], sub["v_hist"])
     t1 = time.perf_counter()
-    G, R, S = oracle.gram(o["a_loc"], o["d"])
+    reps = -(-gram_rows // att_rows)
+    a_loc = np.tile(o["a_loc"], (reps, 1))[:gram_rows]
+    a_full = np.tile(o["a_full"], (reps, 1))[:gram_rows]
+    d_rows = a_full - a_loc
     t2 = time.perf_counter()
-    W = oracle.as_f64(w)
+    G, R, S = oracle.gram(a_loc, d_rows)
     t3 = time.perf_counter()
-    dW, B = oracle.absorb(G, R, W, oracle.default_lambda(G))   # full d x d solve
+    W = oracle.as_f64(w)
     t4 = time.perf_counter()
-    oracle.reconstruction_error(o["a_loc"], o["a_full"], W, dW)
+    dW, B = oracle.absorb(G, R, W, oracle.default_lambda(G))   # full d x d solve
     t5 = time.perf_counter()
+    oracle.reconstruction_error(a_loc, a_full, W, dW)
+    t6 = time.perf_counter()
     return {
-        "attention": (4.0 * sample_rows * nk * d, t1 - t0),
-        "gram": (4.0 * sample_rows * d * d, t2 - t1),
-        "solve": ((1.0 / 3.0 + 4.0) * d ** 3, t4 - t3),
-        "error": (4.0 * sample_rows * d * d, t5 - t4),
+        "attention": (4.0 * att_rows * nk * d, t1 - t0),
+        "gram": (4.0 * gram_rows * d * d, t3 - t2),
+        "solve": ((1.0 / 3.0 + 4.0) * d ** 3, t5 - t4),
+        "error": (4.0 * gram_rows * d * d, t6 - t5),
     }
 
 
@@ -250,9 +258,10 @@ def cpu_cores():
 
 def oracle_throughput(cfg, budget_s: float):
     """Oracle throughput on this workload mix, extrapolated stage by stage
-    from bounded samples: t_full = sum_s F_s * (t_s / f_s)."""
+    from bounded samples: t_full = sum_s F_s * (t_s / f_s). The attention
+    sample doubles until the samples take about half the budget."""
     work = step_work(cfg)
-    rows = 4
+    rows = 8
     timing = oracle_timing(cfg, rows)
     spent = sum(t for _, t in timing.values())
     while spent < budget_s * 0.5 and rows < 256:
@@ -262,17 +271,13 @@ def oracle_throughput(cfg, budget_s: float):
     t_full = sum(work[s] * timing[s][1] / max(timing[s][0], 1.0) for s in work)
     total = sum(work.values())
     cores, blas = cpu_cores()
-    return {
-        "value": total / t_full / 1e12, "unit": "TFLOP/s", "cores": blas or cores,
-        "kind": "oracle",
-        "sample": (f"float64 oracle on {rows} query rows of one layer's last chunk (all heads, "
-                   f"all keys), their Gram and direct error, plus one full {cfg.d}x{cfg.d} "
-                   f"solve; per-stage rates extrapolated to the full step"),
-        "seconds": spent, "ms_per_full_step": t_full * 1e3,
-    }
+    return {"value": round(total / t_full / 1e12, 6), "unit": "TFLOP/s", "cores": blas or cores,
+            "kind": "oracle",
+            "sample": (f"float64 oracle on {rows} query rows of the last chunk (all heads, "
+                       f"all keys), the Gram and direct error of 1024 rows, one full "
+                       f"{cfg.d}x{cfg.d} solve; per-stage rates extrapolated to the full step"),
+            "seconds_per_full_step": round(t_full, 3)}
 
-
-# ---------------------------------------------------------------- distributed
 
 def dist_setup():
     import torch
@@ -308,6 +313,16 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # ---------------------------------------------------------------- our arm
 
+def workload(args):
+    from ispa_synth import CONFIGS, scaled
+    cfg = CONFIGS[args.config]
+    if args.layers is not None and args.layers != cfg.layers:
+        k = cfg.select_k if cfg.select_k is not None else cfg.layers // 2
+        cfg = scaled(cfg, name=f"{cfg.name}-{args.layers}layers", layers=args.layers,
+                     select_k=min(k, args.layers))
+    return cfg
+
+
 def make_inputs(cfg, rank, device):
     """Per layer: its Q/K/V frame streams and the chunk dicts (views into
     them); the projections stacked as one [L, d, d] tensor."""
@@ -335,7 +350,7 @@ def run_ours(args):
 
     world, rank, local = dist_setup()
     dev = torch.device("cuda", torch.cuda.current_device())
-    cfg = CONFIGS[args.config]
+    cfg = workload(args)
     streams, chunks_per_layer, W_all = make_inputs(cfg, rank, dev)
     max_hist = max(len(cfg.history_frames_of(c)) for c in range(cfg.n_chunks)) * cfg.tokens_per_frame
     L = cfg.layers
@@ -513,11 +528,10 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    from ispa_synth import CONFIGS
-    cfg = CONFIGS[args.config]
+    cfg = workload(args)
     work = step_work(cfg)
     total = sum(work.values())
-    rows = 2
+    rows = 8
     acc = {s: [0.0, 0.0] for s in work}
     for i in range(args.warmup + args.steps):
         timing = oracle_timing(cfg, rows)
@@ -530,8 +544,8 @@ def run_reference(args):
     value = total / t_full_step / 1e12
     cores, blas = cpu_cores()
     sample = (f"per step: float64 oracle on {rows} query rows of the last chunk (all heads, all "
-              f"keys), their Gram and direct error, one full {cfg.d}x{cfg.d} solve; rates "
-              f"extrapolated stage by stage to the full step")
+              f"keys), the Gram and direct error of 1024 rows, one full {cfg.d}x{cfg.d} solve; "
+              f"rates extrapolated stage by stage to the full step")
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": t_full_step * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -551,6 +565,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--config", choices=("c1", "c2", "c3"), default="c1")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the workload's layer count (smaller captures for ncu)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
