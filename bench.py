@@ -323,14 +323,18 @@ def workload(args):
     return cfg
 
 
-def make_inputs(cfg, rank, device):
+def make_inputs(cfg, rank, device, layers=None, replica=True):
     """Per layer: its Q/K/V frame streams and the chunk dicts (views into
-    them); the projections stacked as one [L, d, d] tensor."""
+    them); the projections stacked as one [L, d, d] tensor. ``layers`` lists
+    the global layer ids to build (default: all); replicas (one full copy of
+    the workload per rank) draw rank-specific seeds, layer shards the global
+    ones."""
     import torch
     from ispa_synth import layer_streams
+    layers = list(range(cfg.layers)) if layers is None else layers
     streams, chunks, Ws = [], [], []
-    for l in range(cfg.layers):
-        st = layer_streams(cfg, layer=l + 1000 * rank, seed=0, device=device)
+    for l in layers:
+        st = layer_streams(cfg, layer=l + (1000 * rank if replica else 0), seed=0, device=device)
         streams.append(st)
         chunks.append([st.chunk(c) for c in range(cfg.n_chunks)])
         Ws.append(st.w)
@@ -348,15 +352,22 @@ def run_ours(args):
     from kv_cache_absorption_b200.warmup import LayerWarmup, rank as rank_layers
     from ispa_synth import CONFIGS
 
+    from kv_cache_absorption_b200.sharding import gather_errors, owned_layers
     world, rank, local = dist_setup()
     dev = torch.device("cuda", torch.cuda.current_device())
     cfg = workload(args)
-    streams, chunks_per_layer, W_all = make_inputs(cfg, rank, dev)
+    # several GPUs: multi-layer warmups shard their layers (l on rank l mod N,
+    # errors all-gathered for the ranking); a one-layer step runs as replicas
+    sharded = world > 1 and cfg.layers >= world
+    my_layers = owned_layers(cfg.layers, world, rank) if sharded else list(range(cfg.layers))
+    streams, chunks_per_layer, W_all = make_inputs(cfg, rank, dev, my_layers, replica=not sharded)
     max_hist = max(len(cfg.history_frames_of(c)) for c in range(cfg.n_chunks)) * cfg.tokens_per_frame
     L = cfg.layers
+    L_mine = len(my_layers)
     runner = LayerWarmup(cfg.heads, cfg.head_dim, cfg.chunk_tokens, cfg.sink_tokens,
-                         cfg.chunk_tokens, max_hist, n_layers=L, device=dev)
+                         cfg.chunk_tokens, max_hist, n_layers=L_mine, device=dev)
     K = cfg.select_k if cfg.select_k is not None else L // 2
+    err_mine = torch.empty(L_mine, 2, dtype=torch.float64, device=dev)
     err = torch.empty(L, 2, dtype=torch.float64, device=dev)
     perm = torch.empty(L, dtype=torch.int32, device=dev)
     sel = torch.empty(L, dtype=torch.uint8, device=dev)
@@ -372,8 +383,9 @@ def run_ours(args):
                 if ev: ev["a1"].append(E()); ev["a1"][-1].record()
                 runner.gram(first=(c == 0), layer=li)
                 if ev: ev["g1"].append(E()); ev["g1"][-1].record()
-        runner.absorb_all(W_all, err)         # every layer's solve + error, batched
+        runner.absorb_all(W_all, err_mine)    # every layer's solve + error, batched
         if ev: ev["s1"].append(E()); ev["s1"][-1].record()
+        err.copy_(gather_errors(err_mine, L, world) if sharded else err_mine)
         rank_layers(err, K, perm, sel)
 
     for _ in range(args.warmup):
@@ -408,18 +420,19 @@ def run_ours(args):
     attn_ms = sum(a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"])) / args.steps
     gram_ms = sum(a.elapsed_time(b) for a, b in zip(ev["a1"], ev["g1"])) / args.steps
     # batched solve + error of all layers: from the end of the last Gram to s1
-    per_step = L * cfg.n_chunks
+    per_step = L_mine * cfg.n_chunks
     solve_ms = sum(ev["g1"][(i + 1) * per_step - 1].elapsed_time(ev["s1"][i])
                    for i in range(args.steps)) / args.steps
     step_ms_max = max_over_ranks(step_ms, world)
 
     work = step_work(cfg)
     total = sum(work.values())
-    value = total * world / (step_ms_max * 1e-3) / 1e12
-    attn_tflops = work["attention"] / (attn_ms * 1e-3) / 1e12
-    absorb_ms_layer = (gram_ms + solve_ms) / L
+    share = L_mine / L                 # this rank's part of the workload
+    value = total * (1 if sharded else world) / (step_ms_max * 1e-3) / 1e12
+    attn_tflops = work["attention"] * share / (attn_ms * 1e-3) / 1e12
+    absorb_ms_layer = (gram_ms + solve_ms) / L_mine
     bf16_peak, hbm_peak, peak_src = peaks()
-    attn_launches = L * cfg.n_chunks
+    attn_launches = L_mine * cfg.n_chunks
     roofline = {
         "bound": "tensor", "kernel": "dual-stream attention (V fp16 pre-pass + attention kernel)",
         "achieved": round(attn_tflops, 2), "peak": bf16_peak, "unit": "TFLOP/s",
@@ -428,11 +441,11 @@ def run_ours(args):
         "algorithmic_flops_per_launch": work["attention"] / attn_launches,
         "ms_per_launch": attn_ms / attn_launches,
     }
-    absorb_flops = work["gram"] + work["solve"] + work["error"]
+    absorb_flops = (work["gram"] + work["solve"] + work["error"]) * share
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": True, "scaling": "strong" if sharded else "weak", "vs_baseline": None,
         "dtype": "bf16 QK^T, fp16 PV, tf32 Gram, fp32 solve",
         "data": "synthetic AR(1) rho=0.9 bf16 Q/K/V, W ~ N(0,1/d), seeded",
         "config": {"workload": cfg.name, "layers": L, "heads": cfg.heads, "head_dim": cfg.head_dim,
@@ -442,20 +455,22 @@ def run_ours(args):
                                for c in range(cfg.n_chunks)],
                    "select_k": K, "l2": "flushed (512 MB write) before every timed step",
                    "weights": "W and W W^T per layer resident (W W^T formed once at load)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                   "parallelism": (f"layer-sharded x{world} (errors all-gathered)" if sharded else
+                                   f"replicas x{world}" if world > 1 else "single GPU")},
         "attention_tflops": round(attn_tflops, 2),
         "attention_ms_per_step": round(attn_ms, 4),
         "absorb_ms_per_layer": round(absorb_ms_layer, 4),
         "gram_ms_per_step": round(gram_ms, 4), "solve_error_ms_per_step": round(solve_ms, 4),
         "absorb_tflops": round(absorb_flops / ((gram_ms + solve_ms) * 1e-3) / 1e12, 2),
         "roofline": roofline,
-        "absorb_roofline": absorb_roofline(cfg, gram_ms, solve_ms, bf16_peak, hbm_peak),
+        "absorb_roofline": absorb_roofline(cfg, gram_ms * L / L_mine, solve_ms * L / L_mine,
+                                           bf16_peak, hbm_peak),
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
     if not args.no_e2e:
         out["e2e"] = run_e2e(args, cfg, streams, chunks_per_layer, W_all, runner, err, perm,
-                             sel, K, world)
+                             sel, K, world, err_mine if sharded else None)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = oracle_throughput(cfg, args.cpu_budget)
     if rank == 0:
@@ -465,7 +480,8 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_e2e(args, cfg, streams, chunks_per_layer, W_all, runner, err, perm, sel, K, world):
+def run_e2e(args, cfg, streams, chunks_per_layer, W_all, runner, err, perm, sel, K, world,
+            err_mine=None):
     """Same step through the public API with the instance's inputs in pinned
     host memory: every step copies each layer's Q/K/V frame streams
     host->device, runs the warmup, and copies every Delta W, the errors and
@@ -480,8 +496,9 @@ def run_e2e(args, cfg, streams, chunks_per_layer, W_all, runner, err, perm, sel,
             assert all(x.numel() == 0 or x.untyped_storage().data_ptr() in owners
                        for x in ch.values())
     host_tensors = [t.cpu().pin_memory() for t in dev_tensors]
+    from kv_cache_absorption_b200.sharding import gather_errors
     L, d = cfg.layers, cfg.d
-    dW_host = torch.empty(L, d, d, dtype=torch.float32).pin_memory()
+    dW_host = torch.empty(runner.n_layers, d, d, dtype=torch.float32).pin_memory()
     err_host = torch.empty(L, 2, dtype=torch.float64).pin_memory()
     perm_host = torch.empty(L, dtype=torch.int32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host_tensors)
@@ -494,7 +511,11 @@ def run_e2e(args, cfg, streams, chunks_per_layer, W_all, runner, err, perm, sel,
             for c, ch in enumerate(chunks):
                 runner.attention(ch)
                 runner.gram(first=(c == 0), layer=li)
-        runner.absorb_all(W_all, err)
+        if err_mine is not None:
+            runner.absorb_all(W_all, err_mine)
+            err.copy_(gather_errors(err_mine, L, world))
+        else:
+            runner.absorb_all(W_all, err)
         rank_layers(err, K, perm, sel)
         dW_host.copy_(runner.dW, non_blocking=True)
         err_host.copy_(err, non_blocking=True)
@@ -513,9 +534,133 @@ def run_e2e(args, cfg, streams, chunks_per_layer, W_all, runner, err, perm, sel,
     torch.cuda.synchronize()
     ms = max_over_ranks(s.elapsed_time(e) / n, world)
     total = sum(step_work(cfg).values())
-    return {"value": round(total * world / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+    reps = 1 if err_mine is not None else world
+    return {"value": round(total * reps / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
             "ms_per_step": round(ms, 4), "steps": n, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h)}
+
+
+# ---------------------------------------------------------------- streaming (after the transition)
+
+STREAM_METRIC = "post-transition streaming tokens/s (all layers) and KV bytes, ISPA vs all-F-Layer"
+
+
+def run_streaming(args):
+    """One step = one post-transition stream: every streaming chunk through
+    every layer (F-Layers: full attention over the growing history, then W;
+    L-Layers: sink + chunk attention, then W + Delta W). The warmup, the
+    batched absorb, the ranking and the transition run once, untimed. The
+    same stream with every layer kept full is timed alongside."""
+    import torch
+    from kv_cache_absorption_b200 import build
+    build.build()
+    from kv_cache_absorption_b200 import ispa
+    from kv_cache_absorption_b200.warmup import LayerWarmup, rank as rank_layers
+    from kv_cache_absorption_b200.streaming import StreamingLayers, kv_cache_bytes
+
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cfg = workload(args)
+    if cfg.stream_chunks < 1:
+        raise SystemExit("the streaming benchmark needs a workload with streaming chunks (c4)")
+    streams, warm_chunks, W_all = make_inputs(cfg, rank, dev)
+    L = cfg.layers
+    K = cfg.select_k if cfg.select_k is not None else L // 2
+    # warmup and transition
+    warm_hist = max(len(cfg.history_frames_of(c)) for c in range(cfg.n_chunks)) * cfg.tokens_per_frame
+    runner = LayerWarmup(cfg.heads, cfg.head_dim, cfg.chunk_tokens, cfg.sink_tokens,
+                         cfg.chunk_tokens, warm_hist, n_layers=L, device=dev)
+    runner.weight_gram(W_all)
+    for li, chunks in enumerate(warm_chunks):
+        for c, ch in enumerate(chunks):
+            runner.chunk(ch, first=(c == 0), layer=li)
+    err = torch.empty(L, 2, dtype=torch.float64, device=dev)
+    perm = torch.empty(L, dtype=torch.int32, device=dev)
+    sel = torch.empty(L, dtype=torch.uint8, device=dev)
+    runner.absorb_all(W_all, err)
+    rank_layers(err, K, perm, sel)
+    c_first, c_last = cfg.n_chunks, cfg.n_chunks + cfg.stream_chunks - 1
+    hist_last = len(cfg.history_frames_of(c_last)) * cfg.tokens_per_frame
+    sl = StreamingLayers(cfg.heads, cfg.head_dim, cfg.chunk_tokens, cfg.sink_tokens,
+                         cfg.chunk_tokens, hist_last, n_layers=L, device=dev)
+    sl.transition(W_all, runner.dW, sel.cpu().bool())
+    torch.cuda.synchronize()
+    status = ispa.read_status(runner.status)
+    del runner, warm_chunks
+    torch.cuda.empty_cache()
+    schunks = [[st.chunk(c) for c in range(c_first, c_last + 1)] for st in streams]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def one_pass(all_full):
+        for j in range(cfg.stream_chunks):
+            for l in range(L):
+                sl.layer(l, schunks[l][j], local=False if all_full else None)
+
+    def timed(all_full):
+        for _ in range(args.warmup):
+            one_pass(all_full)
+        torch.cuda.synchronize()
+        barrier(world)
+        ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record()
+            one_pass(all_full)
+            s1.record()
+            torch.cuda.synchronize()
+            ms.append(s0.elapsed_time(s1))
+        return max_over_ranks(sum(ms) / len(ms), world)
+
+    bus = torch.cuda.get_device_properties(dev)
+    bus_id = f"{getattr(bus, 'pci_domain_id', 0):08x}:{getattr(bus, 'pci_bus_id', 0):02x}:" \
+             f"{getattr(bus, 'pci_device_id', 0):02x}.0"
+    sampler = ClockSampler(bus_id)
+    time.sleep(0.15)
+    launches0 = ispa.ispa_kernel_launches()
+    ms_ispa = timed(False)
+    launches = (ispa.ispa_kernel_launches() - launches0) // (args.warmup + args.steps)
+    ms_full = timed(True)
+    clocks = sampler.stop()
+    status |= ispa.read_status(sl.status)
+    n_local = int(sel.sum().item())
+    tokens = cfg.stream_chunks * cfg.chunk_tokens
+    d = cfg.d
+    f_flops = 0.0
+    for c in range(c_first, c_last + 1):
+        nk = cfg.sink_tokens + cfg.chunk_tokens + len(cfg.history_frames_of(c)) * cfg.tokens_per_frame
+        f_flops += 4.0 * cfg.chunk_tokens * nk * d
+    kv_all = kv_cache_bytes(L, 0, cfg.sink_tokens, hist_last, cfg.chunk_tokens, d)
+    kv_ispa = kv_cache_bytes(L - n_local, n_local, cfg.sink_tokens, hist_last, cfg.chunk_tokens, d)
+    bf16_peak, _, peak_src = peaks()
+    out = {
+        "metric": STREAM_METRIC, "value": round(tokens * world / (ms_ispa * 1e-3), 1),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_ispa, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 QK^T, fp16 PV, bf16 projection",
+        "data": "synthetic AR(1) rho=0.9 bf16 Q/K/V, W ~ N(0,1/d), seeded",
+        "config": {"workload": cfg.name, "layers": L, "local_layers": n_local, "heads": cfg.heads,
+                   "head_dim": cfg.head_dim, "d": d, "stream_chunks": cfg.stream_chunks,
+                   "chunk_rows": cfg.chunk_tokens, "sink": cfg.sink_tokens,
+                   "history": [len(cfg.history_frames_of(c_first)) * cfg.tokens_per_frame,
+                               hist_last],
+                   "l2": "flushed (512 MB write) before every timed step",
+                   "selection": "K lowest-error layers of this instance's warmup"},
+        "all_f_tokens_per_s": round(tokens * world / (ms_full * 1e-3), 1),
+        "all_f_ms_per_step": round(ms_full, 3),
+        "speedup_vs_all_f": round(ms_full / ms_ispa, 3),
+        "kv_bytes_last_chunk": {"ispa": kv_ispa, "all_f": kv_all,
+                                "saved_frac": round(1 - kv_ispa / kv_all, 4)},
+        "f_layer_attention_tflops_all_f": round(f_flops * L / (ms_full * 1e-3) / 1e12, 2),
+        "attention_frac_of_bf16_peak_all_f": round(f_flops * L / (ms_full * 1e-3) / 1e12 / bf16_peak, 4),
+        "peak_source": f"{peak_src} bf16 dense (burst)",
+        "gpu_launches": int(launches), "device_status": status, "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
 
 
 # ---------------------------------------------------------------- reference arm
@@ -564,7 +709,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--config", choices=("c1", "c2", "c3"), default="c1")
+    ap.add_argument("--config", choices=("c1", "c2", "c3", "c4"), default="c1")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the workload's layer count (smaller captures for ncu)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -580,6 +725,8 @@ def main():
         return
     if args.impl == "reference":
         run_reference(args)
+    elif args.config == "c4":
+        run_streaming(args)
     else:
         run_ours(args)
 

@@ -125,6 +125,43 @@ ISPA_API int ispa_local_attention(const void* q, int64_t nq, int heads, int head
                          ispa_kv local, float scale, float* out_f32, void* out_bf16, float* lse,
                          void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
 
+/* ---- 1c. full attention (F-Layer after the transition) ----------------
+ * Technical summary section 2, step 3: a full-attention layer keeps its
+ * whole KV cache and attends over sink, current chunk and every earlier
+ * frame. Computed with the decomposition of 1a (the pages' LSE states):
+ * the local branch and the history branch, the history cut into equal key
+ * ranges when it is long (split-KV: each range is its own unit of work),
+ * merged by their log-sum-exps. out_bf16 [nq, d] bf16 (required); lse
+ * [heads, nq] fp32 natural log of the full softmax denominator, optional.
+ * workspace: >= ispa_full_attention_workspace_size() bytes, 256-byte
+ * aligned (fp16 V copies, one fp32 [nq, d] output and LSE block per history
+ * range, the local branch's output). Other arguments, alignment, status
+ * and errors as ispa_dual_attention.
+ */
+ISPA_API size_t ispa_full_attention_workspace_size(int64_t nq, int64_t sink_len, int64_t local_len,
+                                                   int64_t hist_len, int heads, int head_dim);
+ISPA_API int ispa_full_attention(const void* q, int64_t nq, int heads, int head_dim, ispa_kv sink,
+                                 ispa_kv local, ispa_kv hist, float scale, void* out_bf16,
+                                 float* lse, void* workspace, size_t workspace_bytes,
+                                 int* dev_status, void* stream);
+
+/* ---- 1d. output projection of the streaming layers --------------------
+ * Technical summary section 2, step 3: after the transition an L-Layer's
+ * local-attention output is projected with the absorbed weight W + Delta W,
+ * an F-Layer's full-attention output with W.
+ * ispa_absorbed_weight: w_bf16 [d, d] bf16 = bf16(W + dW) (dW NULL: bf16(W)),
+ * once per layer at the transition. W, dW fp32 [d, d] row-major.
+ * ispa_project: out [rows, d] = a [rows, d] (bf16, row-major) x w [d, d]
+ * (bf16, row-major), fp32 accumulation on the tensor cores; out bf16
+ * (out_fp32 = 0) or fp32. rows >= 0 arbitrary (rows = 0: nothing is read
+ * or written, a and out may be NULL); d a multiple of 128; pointers 16-byte
+ * aligned. dev_status: ISPA_STATUS_TIMEOUT on a stalled
+ * pipeline. */
+ISPA_API int ispa_absorbed_weight(const float* W, const float* dW, int dim, void* w_bf16,
+                                  void* stream);
+ISPA_API int ispa_project(const void* a_bf16, int64_t rows, int dim, const void* w_bf16, void* out,
+                          int out_fp32, int* dev_status, void* stream);
+
 /* ---- 2. Gram accumulation --------------------------------------------
  * Technical summary section 2, step 2: the closed form needs
  * G = A_loc^T A_loc and R = A_loc^T (A_full - A_loc) over all warmup rows;

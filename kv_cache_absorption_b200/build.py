@@ -18,7 +18,8 @@ CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libispa.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
-SOURCES = ["api.cu", "host_util.cu", "attention.cu", "gram.cu", "tgemm.cu", "solve.cu", "error.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "host_util.cu", "attention.cu", "gram.cu", "tgemm.cu", "solve.cu", "error.cu",
+           "noalloc.cu", "proj.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I" + INCLUDE]

@@ -71,10 +71,29 @@ bool kv_ok(const ispa_kv& b) {
 
 size_t v_half_bytes(int64_t len, int d) { return round256((size_t)len * d * 2); }
 
+// Workspace of one attention call: fp16 V of every branch, per history split
+// an fp32 output and an LSE row block, the local LSEs and, when A_loc is not
+// an output (full attention with history), the local branch's output.
+size_t attention_workspace(int64_t nq, int64_t sink_len, int64_t local_len, int64_t hist_len,
+                           int heads, int head_dim, bool local_out_in_ws) {
+  if (nq < 0 || sink_len < 0 || local_len < 0 || hist_len < 0 || heads < 1 || head_dim < 1) return 0;
+  const int d = heads * head_dim;
+  const int n_split = ispa::history_splits(sink_len, local_len, hist_len);
+  const size_t lse = round256((size_t)heads * nq * 4);
+  const size_t out = round256((size_t)nq * d * 4);
+  // local LSEs, then per history split an LSE block and an output (without
+  // a history, one spare LSE block keeps the layout of a single split)
+  const size_t hist = hist_len > 0 ? (size_t)n_split * (out + lse) : lse;
+  const size_t loc = (local_out_in_ws && hist_len > 0) ? out : 0;
+  return v_half_bytes(sink_len, d) + v_half_bytes(local_len, d) + v_half_bytes(hist_len, d) +
+         hist + loc + lse + 256;
+}
+
 int attention_common(const void* q, int64_t nq, int heads, int head_dim, const ispa_kv (&br)[3],
                      float scale, int round_tf32, float* a_loc, float* d_out, void* a_full,
                      float* lse_loc, float* lse_hist, float* lse_full, void* workspace,
-                     size_t workspace_bytes, int* dev_status, void* stream) {
+                     size_t workspace_bytes, int* dev_status, void* stream,
+                     bool full_only = false) {
   if (!q || !dev_status || nq < 0 || nq > (int64_t)1 << 30 || heads < 1 || heads > 65535)
     return ISPA_ERR_ARG;
   if (head_dim != 64 && head_dim != 128) return ISPA_ERR_UNSUPPORTED;
@@ -86,8 +105,8 @@ int attention_common(const void* q, int64_t nq, int heads, int head_dim, const i
       (a_full && !aligned16(a_full)))
     return ISPA_ERR_UNSUPPORTED;
   const int d = heads * head_dim;
-  const size_t need = ispa_dual_attention_workspace_size(nq, br[0].len, br[1].len, br[2].len, heads,
-                                                         head_dim);
+  const size_t need = attention_workspace(nq, br[0].len, br[1].len, br[2].len, heads, head_dim,
+                                          full_only);
   if (!workspace || workspace_bytes < need || !aligned256(workspace)) return ISPA_ERR_WORKSPACE;
   int rc = check_device();
   if (rc != ISPA_OK) return rc;
@@ -117,18 +136,29 @@ int attention_common(const void* q, int64_t nq, int heads, int head_dim, const i
                    CU_TENSOR_MAP_SWIZZLE_128B))
       return ISPA_ERR_CUDA;
   }
+  p.n_split = ispa::history_splits(br[0].len, br[1].len, br[2].len);
+  p.split_tiles = ispa::history_split_tiles(br[2].len, p.n_split);
+  const size_t out_bytes = round256((size_t)nq * d * 4);
+  const size_t lse_bytes = round256((size_t)heads * nq * 4);
+  p.hist_stride = (int64_t)(out_bytes / 4);
+  p.lse_stride = (int64_t)(lse_bytes / 4);
+  p.loc_out = a_loc;
   if (br[2].len > 0) {
     p.hist_out = reinterpret_cast<float*>(ws);
-    ws += round256((size_t)nq * d * 4);
+    ws += (size_t)p.n_split * out_bytes;
+    if (full_only) {
+      p.loc_out = reinterpret_cast<float*>(ws);
+      ws += out_bytes;
+    }
   }
   p.lse_loc_ws = reinterpret_cast<float*>(ws);
-  ws += round256((size_t)heads * nq * 4);
+  ws += lse_bytes;
   p.lse_hist_ws = reinterpret_cast<float*>(ws);
   p.nq = (int)nq;
   p.heads = heads;
   p.n_pairs = ispa::attention_pairs(nq);
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.round_tf32 = round_tf32;
+  p.round_tf32 = full_only ? 0 : round_tf32;
   p.a_loc = a_loc;
   p.d_out = d_out;
   p.a_full = static_cast<__nv_bfloat16*>(a_full);
@@ -165,12 +195,22 @@ uint64_t ispa_kernel_launches(void) { return ispa::g_launches.load(std::memory_o
 
 size_t ispa_dual_attention_workspace_size(int64_t nq, int64_t sink_len, int64_t local_len,
                                           int64_t hist_len, int heads, int head_dim) {
-  if (nq < 0 || sink_len < 0 || local_len < 0 || hist_len < 0 || heads < 1 || head_dim < 1) return 0;
-  const int d = heads * head_dim;
-  const size_t lse = round256((size_t)heads * nq * 4);
-  const size_t hist_out = hist_len > 0 ? round256((size_t)nq * d * 4) : 0;
-  return v_half_bytes(sink_len, d) + v_half_bytes(local_len, d) + v_half_bytes(hist_len, d) +
-         hist_out + 2 * lse + 256;
+  return attention_workspace(nq, sink_len, local_len, hist_len, heads, head_dim, false);
+}
+
+size_t ispa_full_attention_workspace_size(int64_t nq, int64_t sink_len, int64_t local_len,
+                                          int64_t hist_len, int heads, int head_dim) {
+  return attention_workspace(nq, sink_len, local_len, hist_len, heads, head_dim, true);
+}
+
+int ispa_full_attention(const void* q, int64_t nq, int heads, int head_dim, ispa_kv sink,
+                        ispa_kv local, ispa_kv hist, float scale, void* out_bf16, float* lse,
+                        void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+  if (!out_bf16) return ISPA_ERR_ARG;
+  const ispa_kv br[3] = {sink, local, hist};
+  return attention_common(q, nq, heads, head_dim, br, scale, 0, nullptr, nullptr, out_bf16,
+                          nullptr, nullptr, lse, workspace, workspace_bytes, dev_status, stream,
+                          true);
 }
 
 int ispa_dual_attention(const void* q, int64_t nq, int heads, int head_dim, ispa_kv sink,
@@ -346,6 +386,42 @@ int ispa_layer_error_wwt_batched(int n_layers, const float* M, int64_t m_layer_s
                                                dw_layer_stride, B, b_layer_stride, lambdas, dim,
                                                err, static_cast<double*>(workspace),
                                                static_cast<cudaStream_t>(stream)));
+}
+
+int ispa_absorbed_weight(const float* W, const float* dW, int dim, void* w_bf16, void* stream) {
+  if (!W || !w_bf16 || dim <= 0) return ISPA_ERR_ARG;
+  if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
+  if (!aligned16(W) || (dW && !aligned16(dW)) || !aligned16(w_bf16)) return ISPA_ERR_UNSUPPORTED;
+  int rc = check_device();
+  if (rc != ISPA_OK) return rc;
+  return cuda_rc(ispa::launch_absorbed_weight(W, dW, (int64_t)dim * dim, w_bf16,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+int ispa_project(const void* a_bf16, int64_t rows, int dim, const void* w_bf16, void* out,
+                 int out_fp32, int* dev_status, void* stream) {
+  if (!w_bf16 || !dev_status || rows < 0 || rows > ((int64_t)1 << 31) - 128 || dim <= 0)
+    return ISPA_ERR_ARG;
+  if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
+  if (rows == 0) return ISPA_OK;        // nothing to read or write: a and out may be NULL
+  if (!a_bf16 || !out) return ISPA_ERR_ARG;
+  if (!aligned16(a_bf16) || !aligned16(w_bf16) || !aligned16(out)) return ISPA_ERR_UNSUPPORTED;
+  int rc = check_device();
+  if (rc != ISPA_OK) return rc;
+  ispa::ProjParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!encode_2d(&p.ta, a_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dim, rows, dim, 64, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&p.tb, w_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dim, dim, dim, 64, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return ISPA_ERR_CUDA;
+  p.M = rows;
+  p.N = dim;
+  p.K = dim;
+  p.out = out;
+  p.out_fp32 = out_fp32 ? 1 : 0;
+  p.status = dev_status;
+  return cuda_rc(ispa::launch_proj(p, static_cast<cudaStream_t>(stream)));
 }
 
 size_t ispa_layer_error_workspace_size(int dim) { return dim > 0 ? 256 : 0; }

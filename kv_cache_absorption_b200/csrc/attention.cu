@@ -70,20 +70,37 @@ struct Unit {
   int q0;          // first query row of the pair
   int n_qt;        // query tiles with rows in range (1 or 2)
   int hist;        // 1 = history branch, 0 = local branch (sink then local)
+  int split;       // history split (key range) of a history unit
+  int t0;          // first history key tile of the split
   int n_tiles;
 };
 
+// Units: every history split of every (head, query pair) first, then the
+// local units.
 __device__ __forceinline__ Unit unit_of(const AttnParams& p) {
   Unit u;
   int b = blockIdx.x;
   const int per = p.heads * p.n_pairs;
-  u.hist = (p.len[2] > 0 && b < per) ? 1 : 0;
-  if (p.len[2] > 0 && b >= per) b -= per;
+  const int n_hist_units = p.len[2] > 0 ? per * p.n_split : 0;
+  u.hist = b < n_hist_units ? 1 : 0;
+  if (u.hist) {
+    u.split = b / per;
+    b -= u.split * per;
+  } else {
+    u.split = 0;
+    b -= n_hist_units;
+  }
   u.head = b / p.n_pairs;
   u.q0 = (b % p.n_pairs) * (BM * NQT);
   u.n_qt = (p.nq - u.q0 > BM) ? 2 : 1;
-  u.n_tiles = u.hist ? (int)((p.len[2] + BN - 1) / BN)
-                     : (int)((p.len[0] + BN - 1) / BN) + (int)((p.len[1] + BN - 1) / BN);
+  if (u.hist) {
+    const int total = (int)((p.len[2] + BN - 1) / BN);
+    u.t0 = u.split * p.split_tiles;
+    u.n_tiles = total - u.t0 < p.split_tiles ? total - u.t0 : p.split_tiles;
+  } else {
+    u.t0 = 0;
+    u.n_tiles = (int)((p.len[0] + BN - 1) / BN) + (int)((p.len[1] + BN - 1) / BN);
+  }
   return u;
 }
 
@@ -186,7 +203,7 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
           tma_load_2d(s.q[t][b], &p.tm_q, &s.q_full, u.head * HD + b * 64, u.q0 + t * BM);
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
-        const TileInfo ti = tile_of(j, u.hist, p);
+        const TileInfo ti = tile_of(u.t0 + j, u.hist, p);
         const int sk = j % NK, sv = j % NV;
         if (j >= NK && !mbar_wait(&s.k_empty[sk], ((j / NK) - 1) & 1, p.status, abort_flag)) break;
         mbar_expect_tx(&s.k_full[sk], (HD / 64) * BN * 128);
@@ -279,7 +296,7 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
     float m = -INFINITY, l = 0.f;                 // running max (log2 units), sum
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      const TileInfo ti = tile_of(j, u.hist, p);
+      const TileInfo ti = tile_of(u.t0 + j, u.hist, p);
       if (!mbar_wait(&s.s_full[t], j & 1, p.status, abort_flag)) { ok = false; break; }
       tc_fence_after();
       float sv[BN];
@@ -367,9 +384,9 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(raw[i]) * inv;
         if (u.hist) {
-          store_f32x32(p.hist_out + base + c * 32, a, false);
+          store_f32x32(p.hist_out + u.split * p.hist_stride + base + c * 32, a, false);
         } else {
-          if (p.a_loc) store_f32x32(p.a_loc + base + c * 32, a, p.round_tf32 != 0);
+          if (p.loc_out) store_f32x32(p.loc_out + base + c * 32, a, p.round_tf32 != 0);
           if (direct && p.a_full) store_bf16x32(p.a_full + base + c * 32, a);
           if (direct && p.d_out) {
             float z[32];
@@ -382,7 +399,7 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
       if (row_ok) {
         const int64_t li = (int64_t)u.head * p.nq + row;
         if (u.hist) {
-          p.lse_hist_ws[li] = lse;
+          p.lse_hist_ws[u.split * p.lse_stride + li] = lse;
         } else {
           p.lse_loc_ws[li] = lse;
           if (direct) {
@@ -399,7 +416,14 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
   if (warp == 1) tmem_dealloc(tbase, kTmemCols);
 }
 
-// Post-hoc LSE merge of the two branches (element-wise, 4 columns a thread).
+// Post-hoc LSE merge of the local branch and the history splits (element-
+// wise, 4 columns a thread): with w_b = exp(LSE_b - LSE_full), A_full =
+// sum_b w_b O_b and D = A_full - A_loc = sum_s w_s (O_s - A_loc).
+__device__ __forceinline__ float log_add_exp(float x, float y) {
+  const float hi = fmaxf(x, y), lo = fminf(x, y);
+  return hi == -INFINITY ? hi : hi + log1pf(expf(lo - hi));
+}
+
 __global__ void lse_merge_kernel(const AttnParams p, int hd) {
   const int64_t d = (int64_t)p.heads * hd;
   const int64_t n4 = (int64_t)p.nq * d / 4;
@@ -408,13 +432,20 @@ __global__ void lse_merge_kernel(const AttnParams p, int hd) {
     const int64_t row = (e * 4) / d;
     const int head = (int)(((e * 4) % d) / hd);
     const int64_t li = (int64_t)head * p.nq + row;
-    const float ll = p.lse_loc_ws[li], lh = p.lse_hist_ws[li];
-    const float hi = fmaxf(ll, lh), lo = fminf(ll, lh);
-    const float lf = hi + log1pf(expf(lo - hi));
-    const float w = expf(lh - lf);
-    const float4 a = reinterpret_cast<const float4*>(p.a_loc)[e];
-    const float4 h = reinterpret_cast<const float4*>(p.hist_out)[e];
-    const float4 dd = make_float4(w * (h.x - a.x), w * (h.y - a.y), w * (h.z - a.z), w * (h.w - a.w));
+    const float ll = p.lse_loc_ws[li];
+    float lh = -INFINITY;
+    for (int sp = 0; sp < p.n_split; ++sp) lh = log_add_exp(lh, p.lse_hist_ws[sp * p.lse_stride + li]);
+    const float lf = log_add_exp(ll, lh);
+    const float4 a = reinterpret_cast<const float4*>(p.loc_out)[e];
+    float4 dd = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sp = 0; sp < p.n_split; ++sp) {
+      const float w = expf(p.lse_hist_ws[sp * p.lse_stride + li] - lf);
+      const float4 h = reinterpret_cast<const float4*>(p.hist_out + sp * p.hist_stride)[e];
+      dd.x += w * (h.x - a.x);
+      dd.y += w * (h.y - a.y);
+      dd.z += w * (h.z - a.z);
+      dd.w += w * (h.w - a.w);
+    }
     if (p.d_out)
       reinterpret_cast<float4*>(p.d_out)[e] =
           make_float4(to_tf32(dd.x), to_tf32(dd.y), to_tf32(dd.z), to_tf32(dd.w));
@@ -476,8 +507,25 @@ cudaError_t launch_v_to_half(const void* src, void* dst, int64_t n_elems, int* s
 
 int attention_pairs(int64_t nq) { return (int)((nq + BM * NQT - 1) / (BM * NQT)); }
 
+int history_splits(int64_t sink_len, int64_t local_len, int64_t hist_len) {
+  if (hist_len <= 0) return 1;
+  const int64_t loc_tiles = (sink_len + BN - 1) / BN + (local_len + BN - 1) / BN;
+  const int64_t hist_tiles = (hist_len + BN - 1) / BN;
+  if (hist_tiles <= 3 * loc_tiles) return 1;
+  int64_t n = (hist_tiles + 2 * loc_tiles - 1) / (2 * loc_tiles);
+  if (n > 64) n = 64;
+  // equal splits of ceil(T / n) tiles; recount so that no split is empty
+  const int64_t per = (hist_tiles + n - 1) / n;
+  return (int)((hist_tiles + per - 1) / per);
+}
+
+int history_split_tiles(int64_t hist_len, int n_split) {
+  const int64_t hist_tiles = (hist_len + BN - 1) / BN;
+  return (int)((hist_tiles + n_split - 1) / n_split);
+}
+
 cudaError_t launch_dual_attention(const AttnParams& p, int head_dim, cudaStream_t stream) {
-  const int units = p.heads * p.n_pairs * (p.len[2] > 0 ? 2 : 1);
+  const int units = p.heads * p.n_pairs * (p.len[2] > 0 ? p.n_split + 1 : 1);
   const size_t smem = attention_smem_bytes(head_dim);
   if (head_dim == 64) {
     cudaFuncSetAttribute(branch_attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -30,11 +30,23 @@ struct AttnParams {
   float* lse_loc;         // [heads, nq] or nullptr
   float* lse_hist;
   float* lse_full;
-  float* hist_out;        // workspace: history-branch output [nq, d] fp32
+  float* loc_out;         // local-branch output: a_loc, or workspace when A_loc is not wanted
+  float* hist_out;        // workspace: per history split, output [nq, d] fp32
   float* lse_loc_ws;      // workspace: [heads, nq]
-  float* lse_hist_ws;     // workspace: [heads, nq]
+  float* lse_hist_ws;     // workspace: per history split, [heads, nq]
+  int n_split;            // history key ranges (split-KV), >= 1
+  int split_tiles;        // 128-key tiles per history split
+  int64_t hist_stride;    // elements between the splits' hist_out (nq * d)
+  int64_t lse_stride;     // elements between the splits' lse_hist_ws (heads * nq)
   int* status;
 };
+
+// Number of history splits for these branch lengths: one while the history
+// is at most three times the local branch, else about two local branches of
+// keys per split (balances long histories over the SMs).
+int history_splits(int64_t sink_len, int64_t local_len, int64_t hist_len);
+// Key tiles per history split.
+int history_split_tiles(int64_t hist_len, int n_split);
 
 size_t attention_smem_bytes(int head_dim);
 int attention_pairs(int64_t nq);
@@ -56,6 +68,20 @@ struct GramParams {
   int* status;
 };
 cudaError_t launch_gram(const GramParams& p, int bn, int grid, cudaStream_t stream);
+
+// Output projection of the streaming layers: see proj.cu.
+struct ProjParams {
+  CUtensorMap ta;         // A [M, K] bf16 row-major, 64-column x 128-row boxes, 128-byte swizzle
+  CUtensorMap tb;         // W' [K, N] bf16 row-major, 64-column x 64-row boxes, 128-byte swizzle
+  int64_t M;
+  int N, K;               // multiples of 128 and 64
+  void* out;              // [M, N] bf16 or fp32
+  int out_fp32;
+  int* status;
+};
+cudaError_t launch_proj(const ProjParams& p, cudaStream_t stream);
+cudaError_t launch_absorbed_weight(const float* W, const float* dW, int64_t n, void* out,
+                                   cudaStream_t stream);
 int gram_tile_count(int dim, int bn, int want_s);
 
 

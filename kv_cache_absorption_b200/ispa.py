@@ -35,6 +35,8 @@ EXPORTED = (
     "ispa_absorb_solve_noalloc", "ispa_absorb_solve_batched", "ispa_layer_error_batched",
     "ispa_layer_error_workspace_size", "ispa_layer_error", "ispa_rank_layers",
     "ispa_weight_gram_batched", "ispa_layer_error_wwt_batched",
+    "ispa_full_attention_workspace_size", "ispa_full_attention", "ispa_absorbed_weight",
+    "ispa_project",
 )
 
 
@@ -69,6 +71,10 @@ def _load():
         "ispa_dual_attention": (I, [P, I64, I, I, IspaKV, IspaKV, IspaKV, F, P, P, P, P, P, P,
                                     P, SZ, P, P]),
         "ispa_local_attention": (I, [P, I64, I, I, IspaKV, IspaKV, F, P, P, P, P, SZ, P, P]),
+        "ispa_full_attention_workspace_size": (SZ, [I64, I64, I64, I64, I, I]),
+        "ispa_full_attention": (I, [P, I64, I, I, IspaKV, IspaKV, IspaKV, F, P, P, P, SZ, P, P]),
+        "ispa_absorbed_weight": (I, [P, P, I, P, P]),
+        "ispa_project": (I, [P, I64, I, P, P, I, P, P]),
         "ispa_gram_accumulate": (I, [P, P, I64, I, P, I, I, P]),
         "ispa_absorb_workspace_size": (SZ, [I]),
         "ispa_absorb_solve": (I, [P, P, I, F, P, P, P, P, SZ, P, P]),
@@ -216,6 +222,65 @@ def ispa_local_attention(q, k_sink, v_sink, k_loc, v_loc, scale=None, out_dtype=
         _stream(stream))
     _check(rc, "ispa_local_attention")
     return {"out": out, "lse": lse, "status": status}
+
+
+def ispa_full_attention_workspace_size(nq, sink_len, local_len, hist_len, heads, head_dim) -> int:
+    return _load().ispa_full_attention_workspace_size(nq, sink_len, local_len, hist_len, heads,
+                                                      head_dim)
+
+
+def ispa_full_attention(q, k_sink, v_sink, k_loc, v_loc, k_hist=None, v_hist=None, scale=None,
+                        want_lse=False, out=None, workspace=None, status=None, stream=None) -> dict:
+    """Full attention of an F-Layer over sink, current chunk and history.
+    Returns a dict with out ([nq, d] bf16), lse and the status word."""
+    _dev_tensor(q, torch.bfloat16, "q", 3)
+    nq, heads, hd = q.shape
+    sink = _kv(k_sink, v_sink, heads, hd, "sink")
+    loc = _kv(k_loc, v_loc, heads, hd, "local")
+    hist = _kv(k_hist, v_hist, heads, hd, "history")
+    dev = q.device
+    if scale is None:
+        scale = hd ** -0.5
+    out = torch.empty(nq, heads * hd, dtype=torch.bfloat16, device=dev) if out is None else out
+    lse = torch.empty(heads, nq, dtype=torch.float32, device=dev) if want_lse else None
+    need = ispa_full_attention_workspace_size(nq, sink.len, loc.len, hist.len, heads, hd)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    status = new_status(dev) if status is None else status
+    rc = _load().ispa_full_attention(
+        _ptr(q), nq, heads, hd, sink, loc, hist, float(scale), _ptr(out), _ptr(lse),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream(stream))
+    _check(rc, "ispa_full_attention")
+    return {"out": out, "lse": lse, "status": status}
+
+
+def ispa_absorbed_weight(W, dW=None, out=None, stream=None):
+    """bf16(W + dW) (or bf16(W)) for the streaming projection: [d, d] bf16."""
+    _dev_tensor(W, torch.float32, "W", 2)
+    if dW is not None:
+        _dev_tensor(dW, torch.float32, "dW", 2)
+    dim = W.shape[0]
+    out = torch.empty(dim, dim, dtype=torch.bfloat16, device=W.device) if out is None else out
+    rc = _load().ispa_absorbed_weight(_ptr(W), _ptr(dW), dim, _ptr(out), _stream(stream))
+    _check(rc, "ispa_absorbed_weight")
+    return out
+
+
+def ispa_project(a, w, out=None, out_dtype=torch.bfloat16, status=None, stream=None):
+    """out [rows, d] = a [rows, d] (bf16) x w [d, d] (bf16), fp32 accumulation."""
+    _dev_tensor(a, torch.bfloat16, "a", 2)
+    _dev_tensor(w, torch.bfloat16, "w", 2)
+    rows, dim = a.shape
+    if out is None:
+        out = torch.empty(rows, dim, dtype=out_dtype, device=a.device)
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out must be bf16 or fp32")
+    status = new_status(a.device) if status is None else status
+    rc = _load().ispa_project(_ptr(a), rows, dim, _ptr(w), _ptr(out),
+                              1 if out.dtype == torch.float32 else 0, _ptr(status), _stream(stream))
+    _check(rc, "ispa_project")
+    return out
 
 
 def ispa_gram_accumulate(a_loc, d, M=None, accumulate=False, want_s=True, stream=None):

@@ -1,0 +1,91 @@
+"""Post-transition streaming on one GPU: F-Layers and L-Layers.
+
+"Towards Memory-Efficient Autoregressive Video Generation via
+Instance-Specific Parametric Absorption", technical summary section 2,
+step 3: after the warmup's transition the K lowest-error layers become
+L-Layers. They keep only the sink and the current chunk in their KV cache,
+attend locally and project with the absorbed weight W + Delta W. The other
+layers (F-Layers) keep their whole cache, attend over every earlier frame and
+project with W. The memory saving is the dropped history of the L-Layers.
+
+Orchestration only: every step is a call into the C ABI (full or local
+attention, then the projection); buffers and workspaces are allocated once.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import ispa
+
+
+def kv_cache_bytes(n_full: int, n_local: int, sink: int, history: int, chunk: int, d: int,
+                   bytes_per_elem: int = 2) -> int:
+    """KV-cache bytes of one model at a chunk: an F-Layer holds keys and values
+    of the sink, the history and the current chunk; an L-Layer only of the
+    sink and the current chunk."""
+    per_token = 2 * d * bytes_per_elem            # K and V
+    return n_full * (sink + history + chunk) * per_token + n_local * (sink + chunk) * per_token
+
+
+class StreamingLayers:
+    """Layer weights after the transition and the buffers of one chunk."""
+
+    def __init__(self, heads: int, head_dim: int, chunk_rows: int, max_sink: int, max_local: int,
+                 max_hist: int, n_layers: int, device="cuda"):
+        self.heads, self.head_dim = heads, head_dim
+        self.d = d = heads * head_dim
+        self.n_layers = n_layers
+        self.device = device
+        bf16 = dict(dtype=torch.bfloat16, device=device)
+        self.att = torch.empty(chunk_rows, d, **bf16)
+        self.out = torch.empty(chunk_rows, d, **bf16)
+        full_ws = ispa.ispa_full_attention_workspace_size(chunk_rows, max_sink, max_local, max_hist,
+                                                          heads, head_dim)
+        local_ws = ispa.ispa_dual_attention_workspace_size(chunk_rows, max_sink, max_local, 0,
+                                                           heads, head_dim)
+        self.ws = torch.empty(max(full_ws, local_ws), dtype=torch.uint8, device=device)
+        self.status = ispa.new_status(device)
+        self.Wp = torch.empty(n_layers, d, d, **bf16)
+        self.local = torch.zeros(n_layers, dtype=torch.bool)
+
+    def transition(self, W_all: torch.Tensor, dW_all: torch.Tensor, selected, stream=None):
+        """Weights for streaming: bf16(W + Delta W) for the selected layers
+        (L-Layers), bf16(W) for the others (F-Layers)."""
+        sel = torch.as_tensor(selected).to("cpu", torch.bool)
+        if sel.numel() != self.n_layers:
+            raise ValueError(f"selected must have {self.n_layers} entries")
+        self.local = sel.clone()
+        for l in range(self.n_layers):
+            ispa.ispa_absorbed_weight(W_all[l], dW_all[l] if bool(sel[l]) else None,
+                                      out=self.Wp[l], stream=stream)
+
+    def layer(self, l: int, ch: dict, local=None, stream=None) -> torch.Tensor:
+        """One chunk through layer l (its kind from the transition unless
+        ``local`` overrides it). Returns the projected rows (bf16, reused)."""
+        is_local = bool(self.local[l]) if local is None else bool(local)
+        q = ch["q"]
+        nq = q.shape[0]
+        kv_sink = ispa._kv(ch["k_sink"], ch["v_sink"], self.heads, self.head_dim, "sink")
+        kv_loc = ispa._kv(ch["k_loc"], ch["v_loc"], self.heads, self.head_dim, "local")
+        att = self.att[:nq]
+        lib = ispa._load()
+        scale = float(self.head_dim ** -0.5)
+        if is_local:
+            rc = lib.ispa_local_attention(
+                ispa._ptr(q), nq, self.heads, self.head_dim, kv_sink, kv_loc, scale, None,
+                ispa._ptr(att), None, ispa._ptr(self.ws), self.ws.numel(), ispa._ptr(self.status),
+                ispa._stream(stream))
+            ispa._check(rc, "ispa_local_attention")
+        else:
+            kv_hist = ispa._kv(ch.get("k_hist"), ch.get("v_hist"), self.heads, self.head_dim,
+                               "history")
+            rc = lib.ispa_full_attention(
+                ispa._ptr(q), nq, self.heads, self.head_dim, kv_sink, kv_loc, kv_hist, scale,
+                ispa._ptr(att), None, ispa._ptr(self.ws), self.ws.numel(), ispa._ptr(self.status),
+                ispa._stream(stream))
+            ispa._check(rc, "ispa_full_attention")
+        out = self.out[:nq]
+        rc = lib.ispa_project(ispa._ptr(att), nq, self.d, ispa._ptr(self.Wp[l]), ispa._ptr(out), 0,
+                              ispa._ptr(self.status), ispa._stream(stream))
+        ispa._check(rc, "ispa_project")
+        return out

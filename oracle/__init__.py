@@ -18,6 +18,7 @@ from .ispa_oracle import (  # noqa: F401
     default_lambda,
     absorb,
     reconstruction_error,
+    streaming_layer,
     rank_layers,
     warmup_layer,
     as_f64,

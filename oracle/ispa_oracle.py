@@ -6,8 +6,9 @@ benchmark's CPU-baseline leg; never by the library.
 Source: "Towards Memory-Efficient Autoregressive Video Generation via
 Instance-Specific Parametric Absorption" -- the technical summary (Dutch
 page, section 2 "Methodologie", steps 1-3 and "Dynamische Laagselectie";
-the Portuguese page repeats it). Notation follows the pages: A_loc, A_full,
-W, Delta W, lambda, epsilon, K layers.
+the Portuguese page repeats it). Step 3 also defines the post-transition
+streaming layers (streaming_layer). Notation follows the pages: A_loc,
+A_full, W, Delta W, lambda, epsilon, K layers.
 
 Readings where the pages are silent (each also listed in the design notes):
 * attention outputs are the per-head softmax(q k^T / sqrt(hd)) v,
@@ -165,3 +166,18 @@ def warmup_layer(chunks, W, lam=None):
     e2, eps = reconstruction_error(a_loc, a_full, W, dW)
     return {"chunks": outs, "a_loc": a_loc, "a_full": a_full, "G": G, "R": R, "S": S,
             "lam": lam, "dW": dW, "B": B, "err2": e2, "eps": eps}
+
+
+def streaming_layer(q, k_sink, v_sink, k_loc, v_loc, k_hist, v_hist, W, dW=None, local=False,
+                    scale=None):
+    """One layer's output for a chunk after the transition (technical
+    summary, section 2, step 3). An L-Layer (``local=True``) keeps only the
+    sink and the current chunk and projects with the absorbed weight
+    W + Delta W; an F-Layer attends over sink, chunk and history and projects
+    with W. Returns the projected rows [nq, d] in float64."""
+    W = as_f64(W)
+    if local:
+        a, _ = local_attention(q, k_sink, v_sink, k_loc, v_loc, scale)
+        return a @ (W + (as_f64(dW) if dW is not None else 0.0))
+    a = dual_attention(q, k_sink, v_sink, k_loc, v_loc, k_hist, v_hist, scale)["a_full"]
+    return a @ W

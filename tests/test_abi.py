@@ -35,7 +35,7 @@ def exported():
 
 def test_exports_match_header(ispa):
     names = declared()
-    assert len(names) == 17
+    assert len(names) == 21
     assert names == exported()
     assert names == set(ispa.EXPORTED)
     lib = ctypes.CDLL(ispa.LIB_PATH)
@@ -65,6 +65,17 @@ def test_workspace_sizes(ispa):
     assert ispa.ispa_absorb_workspace_size(n) >= 2 * n * n * 4
     assert ispa.ispa_absorb_workspace_size(0) == 0
     assert ispa.ispa_layer_error_workspace_size(128) >= 40
+    # a history longer than three local branches is cut into key ranges, each
+    # with its own fp32 output and LSE block; full attention also keeps the
+    # local branch's output
+    nq, H, hd = 4680, 12, 128
+    out = r256(nq * H * hd * 4)
+    lse = r256(H * nq * 4)
+    v = lambda n: r256(n * H * hd * 2)
+    assert ispa.ispa_dual_attention_workspace_size(nq, 1560, 4680, 93600, H, hd) == \
+        v(1560) + v(4680) + v(93600) + 8 * (out + lse) + lse + 256   # 732 tiles: 8 ranges
+    assert ispa.ispa_full_attention_workspace_size(nq, 1560, 4680, 93600, H, hd) == \
+        ispa.ispa_dual_attention_workspace_size(nq, 1560, 4680, 93600, H, hd) + out
 
 
 def _kv(ispa, n, addr=0x10000):
@@ -125,6 +136,17 @@ def test_other_entry_points_host_checks(ispa):
                                             None) == ispa.ISPA_ERR_ARG
     assert lib.ispa_layer_error_wwt_batched(1, P, 4 * dd, None, dd, P, dd, P, dd, P, 128, P, P, 256,
                                             None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_project(P, 10, 100, P, P, 0, P, None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert lib.ispa_project(P, -1, 128, P, P, 0, P, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_project(None, 10, 128, P, P, 0, P, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_project(P + 8, 10, 128, P, P, 0, P, None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert lib.ispa_absorbed_weight(P, None, 96, P, None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert lib.ispa_absorbed_weight(None, None, 128, P, None) == ispa.ISPA_ERR_ARG
+    kv = ispa.IspaKV(0x10000, 0x10000, 64)
+    assert lib.ispa_full_attention(P, 64, 2, 64, kv, kv, kv, 0.125, None, None, P, 1 << 30, P,
+                                   None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_full_attention(P, 64, 2, 96, kv, kv, kv, 0.125, P, None, P, 1 << 30, P,
+                                   None) == ispa.ISPA_ERR_UNSUPPORTED
     assert lib.ispa_rank_layers(P, 4, 5, P, None, None) == ispa.ISPA_ERR_ARG
     assert lib.ispa_rank_layers(P, 0, 0, P, None, None) == ispa.ISPA_ERR_ARG
 

@@ -444,3 +444,116 @@ def test_weight_gram_and_error_from_wwt(lib):
         assert abs(got[0] - e2) <= 2e-3 * e2 and abs(got[1] - eps) <= 2e-3 * eps
         # both paths reduce the same fp32 W W^T entries in fp64
         assert np.allclose(got, err_w[l].cpu().numpy(), rtol=1e-9, atol=0)
+
+
+# ---------------------------------------------------------------- split history, streaming layers
+
+@pytest.mark.parametrize("nq,sink,loc,hist,H,hd", [
+    (300, 16, 100, 2000, 2, 128),    # 2 local tiles, 16 history tiles: 4 key ranges
+    (129, 0, 64, 3100, 3, 64),       # 1 local tile, 25 history tiles: 13 ranges, ragged
+])
+def test_dual_attention_split_history(lib, nq, sink, loc, hist, H, hd):
+    """Histories longer than three local branches are cut into key ranges
+    (split-KV) and merged by their log-sum-exps: same results as the oracle's
+    undecomposed pass."""
+    ch = random_chunk(nq, sink, loc, hist, H, hd, seed=hist)
+    out = run_dual(lib, to_dev(ch))
+    torch.cuda.synchronize()
+    assert lib.read_status(out["status"]) == 0
+    check_attention(out, ref_dual(ch), "split history")
+
+
+@pytest.mark.parametrize("hist", [0, 700, 2000])
+def test_full_attention_vs_oracle(lib, hist):
+    """F-Layer attention (A_full and its LSE only), with and without split
+    history."""
+    ch = random_chunk(260, 16, 100, hist, 2, 128, seed=7 + hist)
+    d = to_dev(ch)
+    out = lib.ispa_full_attention(d["q"], d["k_sink"], d["v_sink"], d["k_loc"], d["v_loc"],
+                                  d["k_hist"], d["v_hist"], want_lse=True)
+    torch.cuda.synchronize()
+    assert lib.read_status(out["status"]) == 0
+    ref = ref_dual(ch)
+    got = f64(out["out"])
+    assert np.max(np.abs(got - ref["a_full"])) <= ATT_MAXABS
+    assert rel_fro(got, ref["a_full"]) <= ATT_RELFRO
+    assert np.max(np.abs(f64(out["lse"]) - ref["lse_full"])) <= LSE_ABS
+
+
+def test_project_and_absorbed_weight(lib):
+    """out = A W' on the bf16 tensor cores (ragged rows): fp32 output within
+    fp32 accumulation of the exact bf16 products, bf16 output within its own
+    rounding; W' = bf16(W + Delta W) bit-exact against torch's rounding."""
+    rows, dim = 333, 256
+    a = gaussian((rows, dim), 3, 0, "X").to(torch.bfloat16)
+    W = gaussian((dim, dim), 4, 0, "W") / math.sqrt(dim)
+    dW = 0.1 * gaussian((dim, dim), 5, 0, "W") / math.sqrt(dim)
+    w_bf = lib.ispa_absorbed_weight(W.cuda(), dW.cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(w_bf.cpu(), (W + dW).to(torch.bfloat16))
+    ref = f64(a) @ f64(w_bf)
+    out32 = lib.ispa_project(a.cuda(), w_bf, out_dtype=torch.float32)
+    out16 = lib.ispa_project(a.cuda(), w_bf)
+    torch.cuda.synchronize()
+    assert rel_fro(f64(out32), ref) <= product_tol(f64(a), f64(w_bf), ref)
+    assert rel_fro(f64(out16), ref) <= 2.0 ** -8
+    assert lib.ispa_project(a[:0].cuda(), w_bf).shape == (0, dim)
+
+
+@pytest.mark.parametrize("local", [False, True])
+def test_streaming_layer_vs_oracle(lib, local):
+    """A post-transition chunk through one layer: F-Layer = full attention
+    (split history) then W; L-Layer = local attention then W + Delta W. Both
+    operands of the projection are bf16, so the tolerance is two bf16
+    roundings (2 x 2^-9 relative) on top of the attention's."""
+    ch = random_chunk(200, 16, 100, 1800, 2, 128, seed=11)
+    dim = 256
+    W = gaussian((dim, dim), 12, 0, "W") / math.sqrt(dim)
+    dW = 0.2 * gaussian((dim, dim), 13, 0, "W") / math.sqrt(dim)
+    d = to_dev(ch)
+    if local:
+        att = lib.ispa_local_attention(d["q"], d["k_sink"], d["v_sink"], d["k_loc"], d["v_loc"])
+        w_bf = lib.ispa_absorbed_weight(W.cuda(), dW.cuda())
+    else:
+        att = lib.ispa_full_attention(d["q"], d["k_sink"], d["v_sink"], d["k_loc"], d["v_loc"],
+                                      d["k_hist"], d["v_hist"])
+        w_bf = lib.ispa_absorbed_weight(W.cuda())
+    out = lib.ispa_project(att["out"], w_bf)
+    torch.cuda.synchronize()
+    assert lib.read_status(att["status"]) == 0
+    ref = oracle.streaming_layer(ch["q"], ch["k_sink"], ch["v_sink"], ch["k_loc"], ch["v_loc"],
+                                 ch["k_hist"], ch["v_hist"], f64(W), f64(dW) if local else None,
+                                 local=local)
+    assert rel_fro(f64(out), ref) <= ATT_RELFRO + 2 * 2.0 ** -9
+
+
+@pytest.mark.parametrize("c", [4, 20])
+def test_streaming_full_size_sampled_rows(lib, c):
+    """1.3B streaming at full size: the first (history 12 frames) and last
+    (history 60 frames = 93600 tokens, split into key ranges) post-transition
+    chunks through an F-Layer and an L-Layer, the launches the streaming
+    benchmark times, on 8 sampled rows against the oracle."""
+    from ispa_synth import C4
+    from kv_cache_absorption_b200.streaming import StreamingLayers
+    st = layer_streams(C4, 0, seed=0)
+    ch = st.chunk(c)
+    dim = C4.d
+    dW = 0.05 * gaussian((dim, dim), 21, 0, "W") / math.sqrt(dim)
+    max_hist = len(C4.history_frames_of(C4.n_chunks + C4.stream_chunks - 1)) * C4.tokens_per_frame
+    s = StreamingLayers(C4.heads, C4.head_dim, C4.chunk_tokens, C4.sink_tokens, C4.chunk_tokens,
+                        max_hist, n_layers=2)
+    W2 = torch.stack([st.w, st.w]).cuda()
+    s.transition(W2, torch.stack([dW, dW]).cuda(), [False, True])
+    d = to_dev(ch)
+    rows = np.linspace(0, C4.chunk_tokens - 1, 8).astype(int)
+    sub = dict(ch)
+    sub["q"] = ch["q"][rows]
+    for layer, local in ((0, False), (1, True)):
+        out = f64(s.layer(layer, d))[rows]
+        torch.cuda.synchronize()
+        assert lib.read_status(s.status) == 0
+        ref = oracle.streaming_layer(sub["q"], ch["k_sink"], ch["v_sink"], ch["k_loc"], ch["v_loc"],
+                                     ch["k_hist"], ch["v_hist"], f64(st.w),
+                                     f64(dW) if local else None, local=local)
+        assert rel_fro(out, ref) <= ATT_RELFRO + 2 * 2.0 ** -9, (c, local, rel_fro(out, ref))
+

@@ -348,3 +348,48 @@ def test_attention_pins_catch_planted_mistakes():
     bad3, _ = branch_attention(q, k, v[::-1], 0.37)
     for bad in (bad1, bad2, bad3):
         assert not np.allclose(bad, ref, atol=1e-12)
+
+
+# ---------------------------------------------------------------- streaming layers
+
+def test_streaming_f_layer_is_library_attention_times_w():
+    """An F-Layer's output is softmax attention over every key (here torch's
+    own attention on the concatenated keys) projected with W."""
+    q = rand(6, 2, 8)
+    ks, vs, kl, vl, kh, vh = (rand(n, 2, 8) for n in (3, 3, 5, 5, 9, 9))
+    W, dW = rand(16, 16), rand(16, 16)
+    got = oracle.streaming_layer(q, ks, vs, kl, vl, kh, vh, W, dW, local=False)
+    ref = sdpa(q, np.concatenate([ks, kl, kh]), np.concatenate([vs, vl, vh]), 8 ** -0.5)
+    np.testing.assert_allclose(got, ref.reshape(6, 16) @ W, rtol=0, atol=1e-12)
+
+
+def test_streaming_l_layer_drops_history_and_uses_absorbed_weight():
+    q = rand(6, 2, 8)
+    ks, vs, kl, vl, kh, vh = (rand(n, 2, 8) for n in (3, 3, 5, 5, 9, 9))
+    W, dW = rand(16, 16), rand(16, 16)
+    got = oracle.streaming_layer(q, ks, vs, kl, vl, kh, vh, W, dW, local=True)
+    ref = sdpa(q, np.concatenate([ks, kl]), np.concatenate([vs, vl]), 8 ** -0.5)
+    np.testing.assert_allclose(got, ref.reshape(6, 16) @ (W + dW), rtol=0, atol=1e-12)
+    # the history does not enter an L-Layer
+    got2 = oracle.streaming_layer(q, ks, vs, kl, vl, 3 * kh, vh + 1, W, dW, local=True)
+    np.testing.assert_array_equal(got, got2)
+    # with no history and no absorption both layer kinds coincide
+    f = oracle.streaming_layer(q, ks, vs, kl, vl, kh[:0], vh[:0], W, None, local=False)
+    l0 = oracle.streaming_layer(q, ks, vs, kl, vl, kh[:0], vh[:0], W, None, local=True)
+    np.testing.assert_allclose(f, l0, rtol=0, atol=1e-13)
+
+
+def test_streaming_l_layer_with_absorbed_weight_tracks_full_layer():
+    """Delta W absorbed on a chunk's own rows brings the L-Layer's output on
+    that chunk closer to the F-Layer's than Delta W = 0 does (the ridge
+    objective includes Delta W = 0)."""
+    q = rand(40, 2, 8)
+    ks, vs, kl, vl, kh, vh = (rand(n, 2, 8) for n in (3, 3, 6, 6, 30, 30))
+    W = rand(16, 16, scale=0.25)
+    o = dual_attention(q, ks, vs, kl, vl, kh, vh)
+    G, R, _ = gram(o["a_loc"], o["d"])
+    dW, _ = absorb(G, R, W, default_lambda(G))
+    full = oracle.streaming_layer(q, ks, vs, kl, vl, kh, vh, W, local=False)
+    l_abs = oracle.streaming_layer(q, ks, vs, kl, vl, kh, vh, W, dW, local=True)
+    l_raw = oracle.streaming_layer(q, ks, vs, kl, vl, kh, vh, W, None, local=True)
+    assert np.sum((l_abs - full) ** 2) < np.sum((l_raw - full) ** 2)
