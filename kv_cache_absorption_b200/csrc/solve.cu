@@ -102,12 +102,11 @@ __global__ void copy_layers_kernel(const float4* __restrict__ src, int64_t src_s
 // over [A | Z], Z = I, runs in four 32-column steps J:
 //  (1) warp 0 factors the 32 x 32 diagonal sub-block in registers (lane l
 //      holds row l, a runtime loop over the columns keeps the code small
-//      enough for the instruction cache); all threads then invert L_JJ by
-//      recursive doubling over block sizes 1, 2, 4, 8, 16;
-//  (2) all 512 threads at once: the panel L_IJ = A_IJ L_JJ^-T for the m rows
-//      below (4 threads per row, 8 columns each) and the block row
-//      Z_J <- L_JJ^-1 Z_J (4 threads per column, 8 rows each);
-//      4 m + 4 (J + 32) = 512;
+//      enough for the instruction cache) and stores L_JJ column by column
+//      with the reciprocals of its diagonal;
+//  (2) forward substitution with L_JJ, one thread per 32-vector: the panel
+//      rows L_IJ = A_IJ L_JJ^-T (m rows) and the columns of the block row
+//      Z_J <- L_JJ^-1 Z_J (J + 32 columns), m + J + 32 = 128 threads;
 //  (3) trailing update in 4 x 4 register tiles: A_II -= L_IJ L_IJ^T on the
 //      lower tiles and Z_I -= L_IJ Z_J.
 // Shared-memory row strides (132, 36, 100 floats) keep the float4 accesses
@@ -115,9 +114,8 @@ __global__ void copy_layers_kernel(const float4* __restrict__ src, int64_t src_s
 constexpr int kSA = 132;     // a, z: [128][kSA]
 constexpr int kSP = 36;      // panel, row-major [96][kSP]
 constexpr int kST = 100;     // panel, transposed [32][kST]
-constexpr int kSI = 36;      // L_JJ^-1, [32][kSI]
-constexpr size_t kPotrfSmem =
-    (2 * NB * kSA + 96 * kSP + 32 * kST + 3 * 32 * kSI + 32) * sizeof(float);
+constexpr int kSI = 36;      // L_JJ column-major, [32][kSI]
+constexpr size_t kPotrfSmem = (2 * NB * kSA + 96 * kSP + 32 * kST + 32 * kSI + 64) * sizeof(float);
 
 __device__ __forceinline__ void ld4(float* d, const float* s) {
   const float4 v = *reinterpret_cast<const float4*>(s);
@@ -137,10 +135,9 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
   float* z = a + NB * kSA;
   float* pl = z + NB * kSA;
   float* plT = pl + 96 * kSP;
-  float* li = plT + 32 * kST;                  // L_JJ^-1
-  float* ljj = li + 32 * kSI;                   // L_JJ
-  float* ytmp = ljj + 32 * kSI;                 // C A^-1 blocks of the inversion
-  float* colv = ytmp + 32 * kSI;                // one rotated column of L_JJ
+  float* ljt = plT + 32 * kST;                 // L_JJ, column-major (row c = column c)
+  float* rinv = ljt + 32 * kSI;                 // 1 / diagonal of L_JJ
+  float* colv = rinv + 32;                      // one rotated column of L_JJ
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   for (int e = t; e < NB * (NB / 4); e += blockDim.x) {
     const int i = e >> 5, c = (e & 31) * 4;
@@ -167,7 +164,8 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
         if (lane == 0 && !(piv > 0.f)) atomicOr(status, ISPA_STATUS_NOT_SPD);
         const float inv = rsqrtf(piv);         // NaN for a non-positive pivot: poisons what follows
         const float l0 = lane > j ? r[0] * inv : (lane == j ? piv * inv : 0.f);   // L[lane][j]
-        ljj[lane * kSI + j] = l0;
+        ljt[j * kSI + lane] = l0;                // column j of L_JJ
+        if (lane == j) rinv[j] = inv;            // 1 / L_jj
         // column j rotated so that slot c holds L[j + c][j]; slots past row 31 hold 0
         colv[lane >= j ? lane - j : lane - j + 32] = lane >= j ? l0 : 0.f;
         __syncwarp();
@@ -181,92 +179,39 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
       }
     }
     __syncthreads();
-    // ---- (1b) L_JJ^-1 by recursive doubling: with A^-1 and B^-1 known for two
-    // diagonal blocks of size b, the block below them is -B^-1 C A^-1
-    for (int e = t; e < 32 * 32; e += blockDim.x) {
-      const int i = e >> 5, c = e & 31;
-      li[i * kSI + c] = i == c ? 1.f / ljj[i * kSI + i] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int b = 1; b < 32; b *= 2) {
-      const bool act = t < 16 * b;             // 16 / b block pairs, b^2 entries each
-      int row = 0, c0 = 0, p0 = 0;
-      if (act) {
-        const int pair = t / (b * b), e = t % (b * b);
-        p0 = pair * 2 * b;
-        row = p0 + b + e / b;
-        c0 = p0 + e % b;
-        float y = 0.f;
-        for (int k = 0; k < b; ++k) y = fmaf(ljj[row * kSI + p0 + k], li[(p0 + k) * kSI + c0], y);
-        ytmp[row * kSI + c0] = y;                // (C A^-1)
+    // ---- (2) forward substitution with L_JJ, one 32-vector per thread: the
+    // panel rows (x L_JJ^T = a, i.e. L_JJ x^T = a^T) and the columns of the
+    // block row of Z (L_JJ y = z); m + (J + 32) = 128 threads
+    if (t < NB) {
+      const bool prow = t < m;                 // warp-uniform: m is a multiple of 32
+      const int zc = t - m;                    // Z column
+      float acc[32];
+      if (prow) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) ld4(&acc[4 * q], &a[(J + 32 + t) * kSA + J + 4 * q]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) acc[k] = z[(J + k) * kSA + zc];
       }
-      __syncthreads();
-      if (act) {
-        float x = 0.f;
-        for (int k = 0; k < b; ++k)
-          x = fmaf(li[row * kSI + p0 + b + k], ytmp[(p0 + b + k) * kSI + c0], x);
-        li[row * kSI + c0] = -x;                 // -B^-1 (C A^-1)
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const float y = acc[k] * rinv[k];
+        acc[k] = y;
+        float lc[32];
+#pragma unroll
+        for (int q = k / 4; q < 8; ++q) ld4(&lc[4 * q], &ljt[k * kSI + 4 * q]);
+#pragma unroll
+        for (int r2 = k + 1; r2 < 32; ++r2) acc[r2] = fmaf(-y, lc[r2], acc[r2]);
       }
-      __syncthreads();
-    }
-    // ---- (2) panel rows and block row of Z, results held across the barrier
-    float o[8];
-    int p_row = 0, p_grp = 0;
-    const bool panel = t < 4 * m;
-    if (panel) {
-      p_row = t % m;                            // panel row J + 32 + p_row
-      p_grp = t / m;                            // columns 8 p_grp .. 8 p_grp + 7 (warp-uniform)
-      float ar[32];
+      if (prow) {
 #pragma unroll
-      for (int q = 0; q < 8; ++q) ld4(&ar[4 * q], &a[(J + 32 + p_row) * kSA + J + 4 * q]);
+        for (int q = 0; q < 8; ++q) st4(&pl[t * kSP + 4 * q], &acc[4 * q]);
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const float* lrow = &li[(8 * p_grp + c8) * kSI];
-        float acc = 0.f;
+        for (int c = 0; c < 32; ++c) plT[c * kST + t] = acc[c];
+      } else {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float l4[4];
-          ld4(l4, lrow + 4 * q);
-          acc = fmaf(ar[4 * q], l4[0], acc);
-          acc = fmaf(ar[4 * q + 1], l4[1], acc);
-          acc = fmaf(ar[4 * q + 2], l4[2], acc);
-          acc = fmaf(ar[4 * q + 3], l4[3], acc);
-        }
-        o[c8] = acc;
+        for (int k = 0; k < 32; ++k) z[(J + k) * kSA + zc] = acc[k];
       }
-    } else {
-      const int u = t - 4 * m, nc = J + 32;
-      p_row = u % nc;                           // column of Z
-      p_grp = u / nc;                           // rows J + 8 p_grp .. + 7 (warp-uniform)
-      float zc[32];
-#pragma unroll
-      for (int k = 0; k < 32; ++k) zc[k] = z[(J + k) * kSA + p_row];
-#pragma unroll
-      for (int r8 = 0; r8 < 8; ++r8) {
-        const float* lrow = &li[(8 * p_grp + r8) * kSI];
-        float acc = 0.f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float l4[4];
-          ld4(l4, lrow + 4 * q);
-          acc = fmaf(l4[0], zc[4 * q], acc);
-          acc = fmaf(l4[1], zc[4 * q + 1], acc);
-          acc = fmaf(l4[2], zc[4 * q + 2], acc);
-          acc = fmaf(l4[3], zc[4 * q + 3], acc);
-        }
-        o[r8] = acc;
-      }
-    }
-    __syncthreads();
-    if (panel) {
-      st4(&pl[p_row * kSP + 8 * p_grp], o);
-      st4(&pl[p_row * kSP + 8 * p_grp + 4], o + 4);
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) plT[(8 * p_grp + c8) * kST + p_row] = o[c8];
-    } else {
-#pragma unroll
-      for (int r8 = 0; r8 < 8; ++r8) z[(J + 8 * p_grp + r8) * kSA + p_row] = o[r8];
     }
     __syncthreads();
     // ---- (3) trailing update, one 4 x 4 tile per thread (at most 492 tiles)
@@ -351,38 +296,92 @@ bool opmap(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols, uint
                                mn_major);
 }
 
-// Panel of step k (all in place): L_{>k,k} = A_{>k,k} Linv^T, Z_k = Linv Z_k,
-// Y_k = Linv Y_k, with Linv = L_kk^-1 from potrf_inv_kernel.
-cudaError_t panel_launch(int n, float* A, float* Z, float* Y, const float* Linv, size_t d, int kk,
-                         int m, int64_t ws, int* status, cudaStream_t stream) {
+// Per-layer workspace, in floats (d = dim): A, Z, Y (fp32), then the hi and
+// lo planes of A, Z and Y (each plane d^2, lo = hi + d^2), one 128 x 128
+// inverse and lambda. Finished blocks of L (in A's planes), of L^-1 and of
+// L^-1 B are kept only as planes: every product that reads them again takes
+// them pre-split.
+struct SolveWs {
+  float *A, *Z, *Y, *Ah, *Zh, *Yh, *Linv, *lam;
+  int64_t plane;        // lo = hi + plane
+  int64_t stride;       // floats between layers' workspaces
+};
+
+SolveWs solve_ws(void* workspace, size_t d, int64_t stride) {
+  SolveWs w;
+  const size_t dd = d * d;
+  w.A = static_cast<float*>(workspace);
+  w.Z = w.A + dd;
+  w.Y = w.Z + dd;
+  w.Ah = w.Y + dd;
+  w.Zh = w.Ah + 2 * dd;
+  w.Yh = w.Zh + 2 * dd;
+  w.Linv = w.Yh + 2 * dd;
+  w.lam = w.Linv + NB * NB;
+  w.plane = (int64_t)dd;
+  w.stride = stride;
+  return w;
+}
+
+// A pre-split operand: maps of its hi plane (at `hi`) and lo plane.
+bool opmap_split(TGemmProblem& pr, bool is_a, const float* hi, int64_t plane, uint64_t rows,
+                 uint64_t cols, uint64_t ld, int layers, int64_t stride, bool mn_major) {
+  if (is_a) {
+    pr.a_split = 1;
+    pr.a_mn = mn_major;
+    return opmap(&pr.ta, hi, rows, cols, ld, layers, stride, mn_major) &&
+           opmap(&pr.ta_lo, hi + plane, rows, cols, ld, layers, stride, mn_major);
+  }
+  pr.b_split = 1;
+  pr.b_mn = mn_major;
+  return opmap(&pr.tb, hi, rows, cols, ld, layers, stride, mn_major) &&
+         opmap(&pr.tb_lo, hi + plane, rows, cols, ld, layers, stride, mn_major);
+}
+
+// Store the problem's output only as hi / lo planes starting at `hi`.
+void to_planes(TGemmProblem& pr, float* hi, int64_t plane) {
+  pr.C_hi = hi;
+  pr.C_lo = hi + plane;
+  pr.C = nullptr;
+}
+
+// Panel of step k: L_{>k,k} = A_{>k,k} Linv^T, Z_k = Linv Z_k, Y_k = Linv Y_k,
+// with Linv = L_kk^-1 from potrf_inv_kernel. Inputs are fp32 (split in the
+// kernel, K = 128); outputs go to the planes, where later products read them.
+cudaError_t panel_launch(int n, const SolveWs& w, size_t d, int kk, int m, int* status,
+                         cudaStream_t stream) {
   const int dim = (int)d;
+  const int64_t ws = w.stride;
   TGemmParams p{};
   p.status = status;
   int q = 0;
   if (m > 0) {
     TGemmProblem& pr = p.prob[q++];
-    if (!opmap(&pr.ta, A + (size_t)(kk + NB) * d + kk, m, NB, d, n, ws, false) ||
-        !opmap(&pr.tb, Linv, NB, NB, NB, n, ws, false))
+    if (!opmap(&pr.ta, w.A + (size_t)(kk + NB) * d + kk, m, NB, d, n, ws, false) ||
+        !opmap(&pr.tb, w.Linv, NB, NB, NB, n, ws, false))
       return cudaErrorInvalidValue;
-    set_store(pr, m, NB, NB, A, dim, ws, kk + NB, kk, 1.f, 0.f, n);
+    set_store(pr, m, NB, NB, nullptr, dim, ws, kk + NB, kk, 1.f, 0.f, n);
+    to_planes(pr, w.Ah, w.plane);
     pr.a_mn = 0;
     pr.b_mn = 0;
   }
   {
     TGemmProblem& pr = p.prob[q++];
-    if (!opmap(&pr.ta, Linv, NB, NB, NB, n, ws, false) ||
-        !opmap(&pr.tb, Z + (size_t)kk * d, NB, kk + NB, d, n, ws, true))
+    if (!opmap(&pr.ta, w.Linv, NB, NB, NB, n, ws, false) ||
+        !opmap(&pr.tb, w.Z + (size_t)kk * d, NB, kk + NB, d, n, ws, true))
       return cudaErrorInvalidValue;
-    set_store(pr, NB, kk + NB, NB, Z, dim, ws, kk, 0, 1.f, 0.f, n);
+    set_store(pr, NB, kk + NB, NB, nullptr, dim, ws, kk, 0, 1.f, 0.f, n);
+    to_planes(pr, w.Zh, w.plane);
     pr.a_mn = 0;
     pr.b_mn = 1;
   }
   {
     TGemmProblem& pr = p.prob[q++];
-    if (!opmap(&pr.ta, Linv, NB, NB, NB, n, ws, false) ||
-        !opmap(&pr.tb, Y + (size_t)kk * d, NB, d, d, n, ws, true))
+    if (!opmap(&pr.ta, w.Linv, NB, NB, NB, n, ws, false) ||
+        !opmap(&pr.tb, w.Y + (size_t)kk * d, NB, d, d, n, ws, true))
       return cudaErrorInvalidValue;
-    set_store(pr, NB, dim, NB, Y, dim, ws, kk, 0, 1.f, 0.f, n);
+    set_store(pr, NB, dim, NB, nullptr, dim, ws, kk, 0, 1.f, 0.f, n);
+    to_planes(pr, w.Yh, w.plane);
     pr.a_mn = 0;
     pr.b_mn = 1;
   }
@@ -394,9 +393,9 @@ cudaError_t panel_launch(int n, float* A, float* Z, float* Y, const float* Linv,
 
 size_t absorb_workspace_bytes(int dim) {
   const size_t d = (size_t)dim;
-  // A (-> L), Z (-> L^-1), Y, one 128 x 128 inverse, lambda (+ padding);
+  // A, Z, Y; hi/lo planes of each; one 128 x 128 inverse; lambda (+ padding);
   // a multiple of 256 bytes so that per-layer workspaces stack
-  return ((3 * d * d + NB * NB) * sizeof(float) + 1024 + 255) & ~size_t(255);
+  return ((9 * d * d + NB * NB) * sizeof(float) + 1024 + 255) & ~size_t(255);
 }
 
 cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const float* W,
@@ -405,145 +404,120 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
                                  void* workspace, int* status, cudaStream_t stream) {
   const size_t d = (size_t)dim;
   const int64_t ws = (int64_t)(absorb_workspace_bytes(dim) / sizeof(float));  // per-layer stride
-  float* A = static_cast<float*>(workspace);
-  float* Z = A + d * d;
-  float* Y = Z + d * d;
-  float* Linv = Y + d * d;
-  float* lam = Linv + NB * NB;
-  const int64_t lam_off = (int64_t)(3 * d * d + NB * NB);
+  const SolveWs w = solve_ws(workspace, d, ws);
+  const int64_t lam_off = w.lam - w.A;
   const int nblk = dim / NB;
   cudaError_t e;
   cudaFuncSetAttribute(potrf_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)kPotrfSmem);
 
-  lambda_kernel<<<n, 256, 0, stream>>>(M, m_stride, dim, lambda, lam, ws, lambda_out);
-  build_kernel<<<dim3(n == 1 ? 148 * 8 : 148, n), 256, 0, stream>>>(M, m_stride, dim, A, ws,
-                                                                     lam_off);
-  count_launches(2);
+  lambda_kernel<<<n, 256, 0, stream>>>(M, m_stride, dim, lambda, w.lam, ws, lambda_out);
+  count_launches();
 
-  // B = R W (R = M[0:d, d:2d])
+  // B = R W (R = M[0:d, d:2d]): both split once into the Z and Y planes (free
+  // until the sweep), then one pre-split product
+  if ((e = launch_split_planes(n, M + d, 2 * d, m_stride, w.Zh, w.Zh + w.plane, d, ws, dim, dim,
+                               stream)) != cudaSuccess ||
+      (e = launch_split_planes(n, W, d, w_stride, w.Yh, w.Yh + w.plane, d, ws, dim, dim,
+                               stream)) != cudaSuccess)
+    return e;
   {
     TGemmParams p{};
     p.nprob = 1;
     p.status = status;
     p.kchunk = kChunkSlabs;
     TGemmProblem& pr = p.prob[0];
-    if (!opmap(&pr.ta, M + d, d, d, 2 * d, n, m_stride, false) ||
-        !opmap(&pr.tb, W, d, d, d, n, w_stride, true))
+    if (!opmap_split(pr, true, w.Zh, w.plane, d, d, d, n, ws, false) ||
+        !opmap_split(pr, false, w.Yh, w.plane, d, d, d, n, ws, true))
       return cudaErrorInvalidValue;
     set_store(pr, dim, dim, dim, B, dim, b_stride, 0, 0, 1.f, 0.f, n);
-    pr.a_mn = 0;
-    pr.b_mn = 1;
     if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
   }
-  // Y = B (every layer), the right-hand side of the forward substitution
+  // A = G + lambda I, Z = I; Y = B (the right-hand side of the substitution)
+  build_kernel<<<dim3(n == 1 ? 148 * 8 : 148, n), 256, 0, stream>>>(M, m_stride, dim, w.A, ws,
+                                                                     lam_off);
   copy_layers_kernel<<<dim3(n == 1 ? 148 * 4 : 148, n), 256, 0, stream>>>(
-      reinterpret_cast<const float4*>(B), b_stride / 4, reinterpret_cast<float4*>(Y), ws / 4,
+      reinterpret_cast<const float4*>(B), b_stride / 4, reinterpret_cast<float4*>(w.Y), ws / 4,
       (int64_t)(d * d / 4));
-  count_launches();
+  count_launches(2);
 
   // One layer: right-looking (a rank-128 update of everything below the block
   // after each step): up to (d/128)^2 tiles per launch keep the GPU busy.
   // Several layers: left-looking (long-K products that read the finished
   // part once): far less HBM traffic, and the layers supply the parallelism.
   const bool left_looking = n > 1;
-  if (!left_looking) {
-    for (int k = 0; k < nblk; ++k) {
-      const int kk = k * NB;
-      const int m = dim - kk - NB;
-      potrf_inv_kernel<<<n, 512, kPotrfSmem, stream>>>(A + (size_t)kk * d + kk, dim, Linv, ws,
-                                                       status);
-      count_launches();
-      if ((e = panel_launch(n, A, Z, Y, Linv, d, kk, m, ws, status, stream)) != cudaSuccess)
-        return e;
-      if (m <= 0) break;
-      // A_{>k,>k} -= L_{>k,k} L_{>k,k}^T (lower tiles); Z_{>k} -= L_{>k,k} Z_k;
-      // Y_{>k} -= L_{>k,k} Y_k
-      TGemmParams p{};
-      p.status = status;
-      p.nprob = 3;
-      const float* Lk = A + (size_t)(kk + NB) * d + kk;
-      TGemmProblem& t1 = p.prob[0];
-      if (!opmap(&t1.ta, Lk, m, NB, d, n, ws, false) || !opmap(&t1.tb, Lk, m, NB, d, n, ws, false))
-        return cudaErrorInvalidValue;
-      set_store(t1, m, m, NB, A, dim, ws, kk + NB, kk + NB, -1.f, 1.f, n);
-      t1.a_mn = 0;
-      t1.b_mn = 0;
-      t1.lower = 1;
-      TGemmProblem& t2 = p.prob[1];
-      if (!opmap(&t2.ta, Lk, m, NB, d, n, ws, false) ||
-          !opmap(&t2.tb, Z + (size_t)kk * d, NB, kk + NB, d, n, ws, true))
-        return cudaErrorInvalidValue;
-      set_store(t2, m, kk + NB, NB, Z, dim, ws, kk + NB, 0, -1.f, 1.f, n);
-      t2.a_mn = 0;
-      t2.b_mn = 1;
-      TGemmProblem& t3 = p.prob[2];
-      if (!opmap(&t3.ta, Lk, m, NB, d, n, ws, false) ||
-          !opmap(&t3.tb, Y + (size_t)kk * d, NB, d, d, n, ws, true))
-        return cudaErrorInvalidValue;
-      set_store(t3, m, dim, NB, Y, dim, ws, kk + NB, 0, -1.f, 1.f, n);
-      t3.a_mn = 0;
-      t3.b_mn = 1;
-      if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
-    }
-  }
-  for (int k = 0; left_looking && k < nblk; ++k) {
+  for (int k = 0; k < nblk; ++k) {
     const int kk = k * NB;
     const int m = dim - kk - NB;   // rows below the diagonal block
-    if (k > 0) {
+    if (left_looking && k > 0) {
       // bring block column k of A and block rows k of Y and Z up to date with
-      // the finished blocks 0..k-1 (left-looking: long-K products that read
-      // the finished part once instead of rewriting the trailing matrix)
+      // the finished blocks 0..k-1, read pre-split from the planes
       TGemmParams p{};
       p.status = status;
       p.nprob = 3;
       p.kchunk = kChunkSlabs;
-      const float* Lrow = A + (size_t)kk * d;   // L_{k,<k}: rows kk.., columns 0..kk-1
+      const float* Lrow_h = w.Ah + (size_t)kk * d;   // L_{k,<k} and below: rows kk.., columns 0..kk-1
       // A_{>=k,k} -= L_{>=k,<k} L_{k,<k}^T
       TGemmProblem& u1 = p.prob[0];
-      if (!opmap(&u1.ta, Lrow, d - kk, kk, d, n, ws, false) ||
-          !opmap(&u1.tb, Lrow, NB, kk, d, n, ws, false))
+      if (!opmap_split(u1, true, Lrow_h, w.plane, d - kk, kk, d, n, ws, false) ||
+          !opmap_split(u1, false, Lrow_h, w.plane, NB, kk, d, n, ws, false))
         return cudaErrorInvalidValue;
-      set_store(u1, dim - kk, NB, kk, A, dim, ws, kk, kk, -1.f, 1.f, n);
-      u1.a_mn = 0;
-      u1.b_mn = 0;
+      set_store(u1, dim - kk, NB, kk, w.A, dim, ws, kk, kk, -1.f, 1.f, n);
       // Y_k -= L_{k,<k} Y_{<k}
       TGemmProblem& u2 = p.prob[1];
-      if (!opmap(&u2.ta, Lrow, NB, kk, d, n, ws, false) ||
-          !opmap(&u2.tb, Y, kk, d, d, n, ws, true))
+      if (!opmap_split(u2, true, Lrow_h, w.plane, NB, kk, d, n, ws, false) ||
+          !opmap_split(u2, false, w.Yh, w.plane, kk, d, d, n, ws, true))
         return cudaErrorInvalidValue;
-      set_store(u2, NB, dim, kk, Y, dim, ws, kk, 0, -1.f, 1.f, n);
-      u2.a_mn = 0;
-      u2.b_mn = 1;
+      set_store(u2, NB, dim, kk, w.Y, dim, ws, kk, 0, -1.f, 1.f, n);
       // Z_k[:, <kk] = -L_{k,<k} Z_{<k} (Z_{<k} lower triangular)
       TGemmProblem& u3 = p.prob[2];
-      if (!opmap(&u3.ta, Lrow, NB, kk, d, n, ws, false) ||
-          !opmap(&u3.tb, Z, kk, kk, d, n, ws, true))
+      if (!opmap_split(u3, true, Lrow_h, w.plane, NB, kk, d, n, ws, false) ||
+          !opmap_split(u3, false, w.Zh, w.plane, kk, kk, d, n, ws, true))
         return cudaErrorInvalidValue;
-      set_store(u3, NB, kk, kk, Z, dim, ws, kk, 0, -1.f, 0.f, n);
-      u3.a_mn = 0;
-      u3.b_mn = 1;
+      set_store(u3, NB, kk, kk, w.Z, dim, ws, kk, 0, -1.f, 0.f, n);
       u3.tri = kTriLowerB;
       if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
     }
-    potrf_inv_kernel<<<n, 512, kPotrfSmem, stream>>>(A + (size_t)kk * d + kk, dim, Linv, ws,
+    potrf_inv_kernel<<<n, 512, kPotrfSmem, stream>>>(w.A + (size_t)kk * d + kk, dim, w.Linv, ws,
                                                      status);
     count_launches();
-    if ((e = panel_launch(n, A, Z, Y, Linv, d, kk, m, ws, status, stream)) != cudaSuccess)
-      return e;
+    if ((e = panel_launch(n, w, d, kk, m, status, stream)) != cudaSuccess) return e;
+    if (left_looking || m <= 0) continue;
+    // right-looking: A_{>k,>k} -= L_{>k,k} L_{>k,k}^T (lower tiles);
+    // Z_{>k} -= L_{>k,k} Z_k; Y_{>k} -= L_{>k,k} Y_k (panel outputs pre-split)
+    TGemmParams p{};
+    p.status = status;
+    p.nprob = 3;
+    const float* Lk_h = w.Ah + (size_t)(kk + NB) * d + kk;
+    TGemmProblem& t1 = p.prob[0];
+    if (!opmap_split(t1, true, Lk_h, w.plane, m, NB, d, n, ws, false) ||
+        !opmap_split(t1, false, Lk_h, w.plane, m, NB, d, n, ws, false))
+      return cudaErrorInvalidValue;
+    set_store(t1, m, m, NB, w.A, dim, ws, kk + NB, kk + NB, -1.f, 1.f, n);
+    t1.lower = 1;
+    TGemmProblem& t2 = p.prob[1];
+    if (!opmap_split(t2, true, Lk_h, w.plane, m, NB, d, n, ws, false) ||
+        !opmap_split(t2, false, w.Zh + (size_t)kk * d, w.plane, NB, kk + NB, d, n, ws, true))
+      return cudaErrorInvalidValue;
+    set_store(t2, m, kk + NB, NB, w.Z, dim, ws, kk + NB, 0, -1.f, 1.f, n);
+    TGemmProblem& t3 = p.prob[2];
+    if (!opmap_split(t3, true, Lk_h, w.plane, m, NB, d, n, ws, false) ||
+        !opmap_split(t3, false, w.Yh + (size_t)kk * d, w.plane, NB, d, d, n, ws, true))
+      return cudaErrorInvalidValue;
+    set_store(t3, m, dim, NB, w.Y, dim, ws, kk + NB, 0, -1.f, 1.f, n);
+    if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
   }
-  // Delta W = Z^T Y (Z^T upper triangular)
+  // Delta W = Z^T Y (Z^T upper triangular), both from the planes
   {
     TGemmParams p{};
     p.nprob = 1;
     p.status = status;
     p.kchunk = kChunkSlabs;
     TGemmProblem& pr = p.prob[0];
-    if (!opmap(&pr.ta, Z, d, d, d, n, ws, true) || !opmap(&pr.tb, Y, d, d, d, n, ws, true))
+    if (!opmap_split(pr, true, w.Zh, w.plane, d, d, d, n, ws, true) ||
+        !opmap_split(pr, false, w.Yh, w.plane, d, d, d, n, ws, true))
       return cudaErrorInvalidValue;
     set_store(pr, dim, dim, dim, dW, dim, dw_stride, 0, 0, 1.f, 0.f, n);
-    pr.a_mn = 1;
-    pr.b_mn = 1;
     pr.tri = kTriUpperA;
     if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
   }

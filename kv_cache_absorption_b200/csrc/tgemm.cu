@@ -20,6 +20,12 @@
 // slabs), warp 1 TMEM owner and MMA issuer, warps 2-5 split each slab into
 // hi/lo and then run the epilogue.
 //
+// The split in shared memory costs as much as the MMAs themselves (it halves
+// the kernel's rate). Operands that later products read again are therefore
+// kept pre-split in global memory as two planes, hi and lo, rounded exactly
+// as the in-kernel split rounds them: the epilogue can write such planes
+// (C_hi, C_lo) and TMA then loads them straight into the hi and lo buffers.
+//
 // Long K: the tensor core's accumulator does not round its additions to
 // nearest, and over thousands of terms with heavy cancellation (the Schur
 // complements of the Cholesky sweep) the drift reaches 1e-3 of the result.
@@ -152,15 +158,23 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
     if (lane == 0 && nk > 0) {
       tma_prefetch(&pr.ta);
       tma_prefetch(&pr.tb);
+      if (pr.a_split) tma_prefetch(&pr.ta_lo);
+      if (pr.b_split) tma_prefetch(&pr.tb_lo);
       int n = 0;
       for (int k = kb; k < ke; ++k, ++n) {
         const int st = n % NSTAGE;
         if (n >= NSTAGE && !mbar_wait(&s.empty[st], ((n / NSTAGE) - 1) & 1, p.status, abort_flag)) break;
-        mbar_expect_tx(&s.full[st], 2 * kSlab);
+        mbar_expect_tx(&s.full[st], (2 + pr.a_split + pr.b_split) * kSlab);
         load_slab(s.a_hi[st], &pr.ta, pr.a_mn, pr.a_row0 + ti * TM, pr.a_k0 + k * TK, layer,
                   &s.full[st]);
         load_slab(s.b_hi[st], &pr.tb, pr.b_mn, pr.b_col0 + tj * TN, pr.b_k0 + k * TK, layer,
                   &s.full[st]);
+        if (pr.a_split)
+          load_slab(s.a_lo[st], &pr.ta_lo, pr.a_mn, pr.a_row0 + ti * TM, pr.a_k0 + k * TK, layer,
+                    &s.full[st]);
+        if (pr.b_split)
+          load_slab(s.b_lo[st], &pr.tb_lo, pr.b_mn, pr.b_col0 + tj * TN, pr.b_k0 + k * TK, layer,
+                    &s.full[st]);
       }
       if (*abort_flag)
         for (int j = n - NSTAGE < 0 ? 0 : n - NSTAGE; j < n; ++j)
@@ -234,8 +248,11 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
         summed = n / kc - 2;
       }
       if (!mbar_wait(&s.full[st], (n / NSTAGE) & 1, p.status, abort_flag)) { ok = false; break; }
+      // operands given pre-split need no work; the others are split in place
+      const int v_begin = pr.a_split ? kSlab / 16 : 0;
+      const int v_end = pr.b_split ? kSlab / 16 : 2 * kSlab / 16;
 #pragma unroll 4
-      for (int v = et; v < 2 * kSlab / 16; v += 128) {
+      for (int v = v_begin + et; v < v_end; v += 128) {
         const bool is_b = v >= kSlab / 16;
         const int off = (is_b ? v - kSlab / 16 : v) * 16;
         float4* hi = reinterpret_cast<float4*>((is_b ? s.b_hi[st] : s.a_hi[st]) + off);
@@ -261,14 +278,16 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
     if (ok && (nk == 0 || mbar_wait(&s.acc_full, 0, p.status, abort_flag))) {
       tc_fence_after();
       if (pr.mode == kModeStore) {
-        float* crow = pr.C + (int64_t)layer * pr.c_layer_stride + row * pr.ldc + col0;
+        const int64_t off = (int64_t)layer * pr.c_layer_stride + row * pr.ldc + col0;
+        float* crow = pr.C ? pr.C + off : nullptr;            // beta != 0 needs C
+        float* hrow = pr.C_hi ? pr.C_hi + off : nullptr;
+        float* lrow = pr.C_lo ? pr.C_lo + off : nullptr;
         const float alpha = pr.alpha, beta = pr.beta;
 #pragma unroll 1
         for (int c = 0; c < TN / 32; ++c) {
           uint32_t v[32];
           tmem_ld32(tacc + lane_off + c * 32, v);
           tmem_ld_wait();
-          float4* dst = reinterpret_cast<float4*>(crow + c * 32);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             float4 o;
@@ -277,13 +296,22 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
             o.z = nk > 0 ? alpha * __uint_as_float(v[4 * i + 2]) : 0.f;
             o.w = nk > 0 ? alpha * __uint_as_float(v[4 * i + 3]) : 0.f;
             if (beta != 0.f) {
-              const float4 old = dst[i];
+              const float4 old = reinterpret_cast<const float4*>(crow + c * 32)[i];
               o.x = fmaf(beta, old.x, o.x);
               o.y = fmaf(beta, old.y, o.y);
               o.z = fmaf(beta, old.z, o.z);
               o.w = fmaf(beta, old.w, o.w);
             }
-            dst[i] = o;
+            if (crow) reinterpret_cast<float4*>(crow + c * 32)[i] = o;
+            if (hrow) {
+              float4 h, l;
+              h.x = to_tf32(o.x); l.x = to_tf32(o.x - h.x);
+              h.y = to_tf32(o.y); l.y = to_tf32(o.y - h.y);
+              h.z = to_tf32(o.z); l.z = to_tf32(o.z - h.z);
+              h.w = to_tf32(o.w); l.w = to_tf32(o.w - h.w);
+              reinterpret_cast<float4*>(hrow + c * 32)[i] = h;
+              reinterpret_cast<float4*>(lrow + c * 32)[i] = l;
+            }
           }
         }
       } else {
@@ -331,7 +359,46 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
   if (warp == 1) tmem_dealloc(tacc, kTmemCols);
 }
 
+// hi = tf32(x), lo = tf32(x - hi) (both rounded to nearest) for a rows x cols
+// block of each layer (blockIdx.y): the split tgemm_kernel applies to a
+// shared-memory slab, done once in global memory.
+__global__ void split_planes_kernel(const float* __restrict__ src0, int64_t ld_src,
+                                    int64_t src_stride, float* __restrict__ hi0,
+                                    float* __restrict__ lo0, int64_t ld_dst, int64_t dst_stride,
+                                    int rows, int cols) {
+  const float* src = src0 + (int64_t)blockIdx.y * src_stride;
+  float* hi = hi0 + (int64_t)blockIdx.y * dst_stride;
+  float* lo = lo0 + (int64_t)blockIdx.y * dst_stride;
+  const int q = cols / 4;
+  const int64_t n4 = (int64_t)rows * q;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n4;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / q, c = (e % q) * 4;
+    const float4 x = *reinterpret_cast<const float4*>(src + r * ld_src + c);
+    float4 h, l;
+    h.x = to_tf32(x.x); l.x = to_tf32(x.x - h.x);
+    h.y = to_tf32(x.y); l.y = to_tf32(x.y - h.y);
+    h.z = to_tf32(x.z); l.z = to_tf32(x.z - h.z);
+    h.w = to_tf32(x.w); l.w = to_tf32(x.w - h.w);
+    *reinterpret_cast<float4*>(hi + r * ld_dst + c) = h;
+    *reinterpret_cast<float4*>(lo + r * ld_dst + c) = l;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_split_planes(int layers, const float* src, int64_t ld_src, int64_t src_stride,
+                                float* hi, float* lo, int64_t ld_dst, int64_t dst_stride, int rows,
+                                int cols, cudaStream_t stream) {
+  const int64_t n4 = (int64_t)rows * (cols / 4);
+  int blocks = (int)((n4 + 255) / 256);
+  const int cap = layers == 1 ? 148 * 8 : 148;
+  if (blocks > cap) blocks = cap;
+  split_planes_kernel<<<dim3(blocks, layers), 256, 0, stream>>>(src, ld_src, src_stride, hi, lo,
+                                                                ld_dst, dst_stride, rows, cols);
+  count_launches();
+  return cudaGetLastError();
+}
 
 size_t tgemm_smem_bytes() { return sizeof(GSmem) + 1024; }
 

@@ -21,12 +21,17 @@ constexpr int kModeDot3 = 1;    // accumulate <P, G>, <P, R>, <P, S> (P = op(A) 
 // when b_mn == 0 (stored [N][K]). a_row0 / a_k0 / b_col0 / b_k0 offset the
 // tiles inside the mapped tensors; C_l = C + l * c_layer_stride.
 struct TGemmProblem {
-  CUtensorMap ta;
+  CUtensorMap ta;         // op(A): fp32 values, or the hi plane when a_split
   CUtensorMap tb;
+  CUtensorMap ta_lo;      // the lo plane of a pre-split operand (a_split / b_split)
+  CUtensorMap tb_lo;
+  int a_split, b_split;   // operand given as tf32 hi/lo planes: no split in the kernel
   int a_mn, b_mn;
   int M, N, K;
   int a_row0, a_k0, b_col0, b_k0;
-  float* C;
+  float* C;              // fp32 output (nullable when only the split planes are wanted)
+  float* C_hi;           // optional split copy of the output (same indexing as C):
+  float* C_lo;           // hi = tf32(v), lo = tf32(v - hi), both rounded to nearest
   int64_t ldc;
   int64_t c_layer_stride;
   int c_row0, c_col0;
@@ -52,6 +57,11 @@ struct TGemmParams {
 };
 
 size_t tgemm_smem_bytes();
+// hi / lo planes (tf32, rounded to nearest) of a rows x cols fp32 block of
+// `layers` matrices (src_stride / dst_stride elements apart).
+cudaError_t launch_split_planes(int layers, const float* src, int64_t ld_src, int64_t src_stride,
+                                float* hi, float* lo, int64_t ld_dst, int64_t dst_stride, int rows,
+                                int cols, cudaStream_t stream);
 cudaError_t launch_tgemm(TGemmParams& p, cudaStream_t stream);
 
 }  // namespace ispa
