@@ -584,6 +584,7 @@ def run_streaming(args):
     sl = StreamingLayers(cfg.heads, cfg.head_dim, cfg.chunk_tokens, cfg.sink_tokens,
                          cfg.chunk_tokens, hist_last, n_layers=L, device=dev)
     sl.transition(W_all, runner.dW, sel.cpu().bool())
+    sl.quantize_weights(W_all, runner.dW)
     torch.cuda.synchronize()
     status = ispa.read_status(runner.status)
     del runner, warm_chunks
@@ -591,14 +592,14 @@ def run_streaming(args):
     schunks = [[st.chunk(c) for c in range(c_first, c_last + 1)] for st in streams]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def one_pass(all_full):
+    def one_pass(all_full, w8a8=False):
         for j in range(cfg.stream_chunks):
             for l in range(L):
-                sl.layer(l, schunks[l][j], local=False if all_full else None)
+                sl.layer(l, schunks[l][j], local=False if all_full else None, w8a8=w8a8)
 
-    def timed(all_full):
+    def timed(all_full, w8a8=False):
         for _ in range(args.warmup):
-            one_pass(all_full)
+            one_pass(all_full, w8a8)
         torch.cuda.synchronize()
         barrier(world)
         ms = []
@@ -606,7 +607,7 @@ def run_streaming(args):
             flush.zero_()
             s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s0.record()
-            one_pass(all_full)
+            one_pass(all_full, w8a8)
             s1.record()
             torch.cuda.synchronize()
             ms.append(s0.elapsed_time(s1))
@@ -621,6 +622,7 @@ def run_streaming(args):
     ms_ispa = timed(False)
     launches = (ispa.ispa_kernel_launches() - launches0) // (args.warmup + args.steps)
     ms_full = timed(True)
+    ms_w8a8 = timed(False, True)
     clocks = sampler.stop()
     status |= ispa.read_status(sl.status)
     n_local = int(sel.sum().item())
@@ -649,6 +651,8 @@ def run_streaming(args):
         "all_f_tokens_per_s": round(tokens * world / (ms_full * 1e-3), 1),
         "all_f_ms_per_step": round(ms_full, 3),
         "speedup_vs_all_f": round(ms_full / ms_ispa, 3),
+        "ispa_w8a8_tokens_per_s": round(tokens * world / (ms_w8a8 * 1e-3), 1),
+        "ispa_w8a8_speedup_vs_all_f": round(ms_full / ms_w8a8, 3),
         "kv_bytes_last_chunk": {"ispa": kv_ispa, "all_f": kv_all,
                                 "saved_frac": round(1 - kv_ispa / kv_all, 4)},
         "f_layer_attention_tflops_all_f": round(f_flops * L / (ms_full * 1e-3) / 1e12, 2),

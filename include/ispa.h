@@ -162,6 +162,28 @@ ISPA_API int ispa_absorbed_weight(const float* W, const float* dW, int dim, void
 ISPA_API int ispa_project(const void* a_bf16, int64_t rows, int dim, const void* w_bf16, void* out,
                           int out_fp32, int* dev_status, void* stream);
 
+/* ---- 1e. W8A8 output projection (8-bit weights and activations) --------
+ * Technical summary, results: ISPA combined with post-training quantisation
+ * of weights and activations to 8 bits (W8A8). The pages fix no scheme; this
+ * is the plainest: symmetric int8, per output column for the weights, per row
+ * (token) for the activations, int32 accumulation on the tensor cores.
+ * ispa_quantize_weight_int8: W' = W + dW (dW NULL: W), both fp32 [d, d]
+ * row-major, summed in fp32; w_scale[n] = max_k |W'[k][n]| / 127 (1 for an
+ * all-zero column); wq_t[n][k] = round-half-even(W'[k][n] / w_scale[n]) in
+ * fp32, clamped to +-127: the codes transposed, [d, d] int8 row-major.
+ * ispa_project_w8a8: out [rows, d] (bf16 if out_fp32 = 0, else fp32) =
+ * s_a[m] w_scale[n] sum_k q_a[m][k] wq_t[n][k], with s_a and q_a the
+ * per-row scales and codes of a [rows, d] bf16 (same rule), formed in the
+ * workspace (>= ispa_project_w8a8_workspace_size(rows, dim) bytes, 256-byte
+ * aligned). rows >= 0 (0: nothing read or written); d a multiple of 128;
+ * a, wq_t, out 16-byte aligned. */
+ISPA_API int ispa_quantize_weight_int8(const float* W, const float* dW, int dim, int8_t* wq_t,
+                                       float* w_scale, void* stream);
+ISPA_API size_t ispa_project_w8a8_workspace_size(int64_t rows, int dim);
+ISPA_API int ispa_project_w8a8(const void* a_bf16, int64_t rows, int dim, const int8_t* wq_t,
+                               const float* w_scale, void* out, int out_fp32, void* workspace,
+                               size_t workspace_bytes, int* dev_status, void* stream);
+
 /* ---- 2. Gram accumulation --------------------------------------------
  * Technical summary section 2, step 2: the closed form needs
  * G = A_loc^T A_loc and R = A_loc^T (A_full - A_loc) over all warmup rows;

@@ -8,6 +8,7 @@
 
 #include "sm100.cuh"
 #include "attention.h"
+#include "w8a8.h"
 #include "host_util.h"
 
 namespace ispa {
@@ -422,6 +423,60 @@ int ispa_project(const void* a_bf16, int64_t rows, int dim, const void* w_bf16, 
   p.out_fp32 = out_fp32 ? 1 : 0;
   p.status = dev_status;
   return cuda_rc(ispa::launch_proj(p, static_cast<cudaStream_t>(stream)));
+}
+
+int ispa_quantize_weight_int8(const float* W, const float* dW, int dim, int8_t* wq_t,
+                              float* w_scale, void* stream) {
+  if (!W || !wq_t || !w_scale || dim <= 0) return ISPA_ERR_ARG;
+  if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
+  if (!aligned16(W) || (dW && !aligned16(dW)) || !aligned16(wq_t)) return ISPA_ERR_UNSUPPORTED;
+  int rc = check_device();
+  if (rc != ISPA_OK) return rc;
+  return cuda_rc(ispa::launch_quant_weight(W, dW, dim, wq_t, w_scale,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+size_t ispa_project_w8a8_workspace_size(int64_t rows, int dim) {
+  if (rows < 0 || dim <= 0) return 0;
+  return round256((size_t)rows * dim) + round256((size_t)rows * 4) + 256;
+}
+
+int ispa_project_w8a8(const void* a_bf16, int64_t rows, int dim, const int8_t* wq_t,
+                      const float* w_scale, void* out, int out_fp32, void* workspace,
+                      size_t workspace_bytes, int* dev_status, void* stream) {
+  if (!wq_t || !w_scale || !dev_status || rows < 0 || rows > ((int64_t)1 << 31) - 128 || dim <= 0)
+    return ISPA_ERR_ARG;
+  if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
+  if (rows == 0) return ISPA_OK;        // nothing to read or write
+  if (!a_bf16 || !out) return ISPA_ERR_ARG;
+  if (!aligned16(a_bf16) || !aligned16(wq_t) || !aligned16(out)) return ISPA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned256(workspace) ||
+      workspace_bytes < ispa_project_w8a8_workspace_size(rows, dim))
+    return ISPA_ERR_WORKSPACE;
+  int rc = check_device();
+  if (rc != ISPA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int8_t* aq = static_cast<int8_t*>(workspace);
+  float* a_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                            round256((size_t)rows * dim));
+  cudaError_t e = ispa::launch_quant_rows(a_bf16, rows, dim, aq, a_scale, s);
+  if (e != cudaSuccess) return cuda_rc(e);
+  ispa::Q8Params p;
+  std::memset(&p, 0, sizeof(p));
+  if (!encode_2d(&p.ta, aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, dim, rows, dim, 128, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&p.tb, wq_t, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, dim, dim, dim, 128, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return ISPA_ERR_CUDA;
+  p.a_scale = a_scale;
+  p.w_scale = w_scale;
+  p.M = rows;
+  p.N = dim;
+  p.K = dim;
+  p.out = out;
+  p.out_fp32 = out_fp32 ? 1 : 0;
+  p.status = dev_status;
+  return cuda_rc(ispa::launch_gemm_i8(p, s));
 }
 
 size_t ispa_layer_error_workspace_size(int dim) { return dim > 0 ? 256 : 0; }

@@ -36,7 +36,8 @@ EXPORTED = (
     "ispa_layer_error_workspace_size", "ispa_layer_error", "ispa_rank_layers",
     "ispa_weight_gram_batched", "ispa_layer_error_wwt_batched",
     "ispa_full_attention_workspace_size", "ispa_full_attention", "ispa_absorbed_weight",
-    "ispa_project",
+    "ispa_project", "ispa_quantize_weight_int8", "ispa_project_w8a8_workspace_size",
+    "ispa_project_w8a8",
 )
 
 
@@ -75,6 +76,9 @@ def _load():
         "ispa_full_attention": (I, [P, I64, I, I, IspaKV, IspaKV, IspaKV, F, P, P, P, SZ, P, P]),
         "ispa_absorbed_weight": (I, [P, P, I, P, P]),
         "ispa_project": (I, [P, I64, I, P, P, I, P, P]),
+        "ispa_quantize_weight_int8": (I, [P, P, I, P, P, P]),
+        "ispa_project_w8a8_workspace_size": (SZ, [I64, I]),
+        "ispa_project_w8a8": (I, [P, I64, I, P, P, P, I, P, SZ, P, P]),
         "ispa_gram_accumulate": (I, [P, P, I64, I, P, I, I, P]),
         "ispa_absorb_workspace_size": (SZ, [I]),
         "ispa_absorb_solve": (I, [P, P, I, F, P, P, P, P, SZ, P, P]),
@@ -280,6 +284,46 @@ def ispa_project(a, w, out=None, out_dtype=torch.bfloat16, status=None, stream=N
     rc = _load().ispa_project(_ptr(a), rows, dim, _ptr(w), _ptr(out),
                               1 if out.dtype == torch.float32 else 0, _ptr(status), _stream(stream))
     _check(rc, "ispa_project")
+    return out
+
+
+def ispa_quantize_weight_int8(W, dW=None, wq_t=None, w_scale=None, stream=None):
+    """8-bit codes of W' = W (+ dW) per output column, transposed ([d, d] int8,
+    row n = column n of W'), and the column scales ([d] fp32)."""
+    _dev_tensor(W, torch.float32, "W", 2)
+    if dW is not None:
+        _dev_tensor(dW, torch.float32, "dW", 2)
+    dim = W.shape[0]
+    wq_t = torch.empty(dim, dim, dtype=torch.int8, device=W.device) if wq_t is None else wq_t
+    w_scale = torch.empty(dim, dtype=torch.float32, device=W.device) if w_scale is None else w_scale
+    rc = _load().ispa_quantize_weight_int8(_ptr(W), _ptr(dW), dim, _ptr(wq_t), _ptr(w_scale),
+                                           _stream(stream))
+    _check(rc, "ispa_quantize_weight_int8")
+    return wq_t, w_scale
+
+
+def ispa_project_w8a8_workspace_size(rows: int, dim: int) -> int:
+    return _load().ispa_project_w8a8_workspace_size(rows, dim)
+
+
+def ispa_project_w8a8(a, wq_t, w_scale, out=None, out_dtype=torch.bfloat16, workspace=None,
+                      status=None, stream=None):
+    """out [rows, d] = W8A8 product of a [rows, d] (bf16, quantised per row
+    on the fly) and the weight codes from ispa_quantize_weight_int8."""
+    _dev_tensor(a, torch.bfloat16, "a", 2)
+    _dev_tensor(wq_t, torch.int8, "wq_t", 2)
+    _dev_tensor(w_scale, torch.float32, "w_scale", 1)
+    rows, dim = a.shape
+    if out is None:
+        out = torch.empty(rows, dim, dtype=out_dtype, device=a.device)
+    if workspace is None:
+        workspace = torch.empty(max(ispa_project_w8a8_workspace_size(rows, dim), 256),
+                                dtype=torch.uint8, device=a.device)
+    status = new_status(a.device) if status is None else status
+    rc = _load().ispa_project_w8a8(_ptr(a), rows, dim, _ptr(wq_t), _ptr(w_scale), _ptr(out),
+                                   1 if out.dtype == torch.float32 else 0, _ptr(workspace),
+                                   workspace.numel(), _ptr(status), _stream(stream))
+    _check(rc, "ispa_project_w8a8")
     return out
 
 

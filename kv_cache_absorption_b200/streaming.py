@@ -47,6 +47,10 @@ class StreamingLayers:
         self.status = ispa.new_status(device)
         self.Wp = torch.empty(n_layers, d, d, **bf16)
         self.local = torch.zeros(n_layers, dtype=torch.bool)
+        self.wq = None           # int8 codes and scales of W' once quantize_weights has run
+        self.wq_scale = None
+        self.q_ws = torch.empty(ispa.ispa_project_w8a8_workspace_size(chunk_rows, d),
+                                dtype=torch.uint8, device=device)
 
     def transition(self, W_all: torch.Tensor, dW_all: torch.Tensor, selected, stream=None):
         """Weights for streaming: bf16(W + Delta W) for the selected layers
@@ -59,9 +63,20 @@ class StreamingLayers:
             ispa.ispa_absorbed_weight(W_all[l], dW_all[l] if bool(sel[l]) else None,
                                       out=self.Wp[l], stream=stream)
 
-    def layer(self, l: int, ch: dict, local=None, stream=None) -> torch.Tensor:
+    def quantize_weights(self, W_all: torch.Tensor, dW_all: torch.Tensor, stream=None):
+        """W8A8: 8-bit codes of every layer's projection weight (W + Delta W for
+        the L-Layers, W for the F-Layers), per output column."""
+        n, d = self.n_layers, self.d
+        self.wq = torch.empty(n, d, d, dtype=torch.int8, device=self.device)
+        self.wq_scale = torch.empty(n, d, dtype=torch.float32, device=self.device)
+        for l in range(n):
+            ispa.ispa_quantize_weight_int8(W_all[l], dW_all[l] if bool(self.local[l]) else None,
+                                           wq_t=self.wq[l], w_scale=self.wq_scale[l], stream=stream)
+
+    def layer(self, l: int, ch: dict, local=None, w8a8: bool = False, stream=None) -> torch.Tensor:
         """One chunk through layer l (its kind from the transition unless
-        ``local`` overrides it). Returns the projected rows (bf16, reused)."""
+        ``local`` overrides it; with ``w8a8`` the projection runs on 8-bit
+        weights and activations). Returns the projected rows (bf16, reused)."""
         is_local = bool(self.local[l]) if local is None else bool(local)
         q = ch["q"]
         nq = q.shape[0]
@@ -85,6 +100,13 @@ class StreamingLayers:
                 ispa._stream(stream))
             ispa._check(rc, "ispa_full_attention")
         out = self.out[:nq]
+        if w8a8:
+            rc = lib.ispa_project_w8a8(ispa._ptr(att), nq, self.d, ispa._ptr(self.wq[l]),
+                                       ispa._ptr(self.wq_scale[l]), ispa._ptr(out), 0,
+                                       ispa._ptr(self.q_ws), self.q_ws.numel(),
+                                       ispa._ptr(self.status), ispa._stream(stream))
+            ispa._check(rc, "ispa_project_w8a8")
+            return out
         rc = lib.ispa_project(ispa._ptr(att), nq, self.d, ispa._ptr(self.Wp[l]), ispa._ptr(out), 0,
                               ispa._ptr(self.status), ispa._stream(stream))
         ispa._check(rc, "ispa_project")

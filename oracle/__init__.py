@@ -19,6 +19,8 @@ from .ispa_oracle import (  # noqa: F401
     absorb,
     reconstruction_error,
     streaming_layer,
+    quantize_rows_int8,
+    project_w8a8,
     rank_layers,
     warmup_layer,
     as_f64,

@@ -181,3 +181,31 @@ def streaming_layer(q, k_sink, v_sink, k_loc, v_loc, k_hist, v_hist, W, dW=None,
         return a @ (W + (as_f64(dW) if dW is not None else 0.0))
     a = dual_attention(q, k_sink, v_sink, k_loc, v_loc, k_hist, v_hist, scale)["a_full"]
     return a @ W
+
+
+def quantize_rows_int8(X):
+    """Symmetric 8-bit codes per row of a float32 matrix (the W8A8 reading:
+    technical summary, results, post-training quantisation): s = max|x| / 127
+    (fp32 division; an all-zero row gets s = 1), q = round-half-even(x / s)
+    in fp32, clamped to [-127, 127]. Returns (codes int8, scales float32)."""
+    X = np.asarray(X, dtype=np.float32)
+    mx = np.max(np.abs(X), axis=1)
+    s = np.where(mx > 0, mx / np.float32(127.0), np.float32(1.0)).astype(np.float32)
+    q = np.rint(X / s[:, None]).clip(-127, 127).astype(np.int8)
+    return q, s
+
+
+def project_w8a8(a, W, dW=None):
+    """W8A8 projection of a streaming layer: activations a [rows, d] (bf16
+    values) quantised per row, W' = W (+ Delta W, summed in fp32) quantised
+    per output column; out = s_a s_w sum_k q_a q_w, in float64. Returns
+    (out, q_a, s_a, q_w^T, s_w)."""
+    A32 = as_f64(a).astype(np.float32)
+    Wp = np.asarray(as_f64(W), dtype=np.float32)
+    if dW is not None:
+        Wp = Wp + np.asarray(as_f64(dW), dtype=np.float32)
+    qa, sa = quantize_rows_int8(A32)
+    qwt, sw = quantize_rows_int8(Wp.T)          # columns of W' = rows of its transpose
+    acc = qa.astype(np.int64) @ qwt.astype(np.int64).T
+    out = acc.astype(np.float64) * sa.astype(np.float64)[:, None] * sw.astype(np.float64)[None, :]
+    return out, qa, sa, qwt, sw

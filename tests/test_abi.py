@@ -35,7 +35,7 @@ def exported():
 
 def test_exports_match_header(ispa):
     names = declared()
-    assert len(names) == 21
+    assert len(names) == 24
     assert names == exported()
     assert names == set(ispa.EXPORTED)
     lib = ctypes.CDLL(ispa.LIB_PATH)
@@ -141,6 +141,13 @@ def test_other_entry_points_host_checks(ispa):
     assert lib.ispa_project(None, 10, 128, P, P, 0, P, None) == ispa.ISPA_ERR_ARG
     assert lib.ispa_project(P + 8, 10, 128, P, P, 0, P, None) == ispa.ISPA_ERR_UNSUPPORTED
     assert lib.ispa_absorbed_weight(P, None, 96, P, None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert lib.ispa_quantize_weight_int8(P, None, 96, P, P, None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert lib.ispa_quantize_weight_int8(None, None, 128, P, P, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_project_w8a8(P, 10, 128, P, P, P, 0, P, 16, P, None) == ispa.ISPA_ERR_WORKSPACE
+    assert lib.ispa_project_w8a8(P, 10, 100, P, P, P, 0, P, 1 << 20, P, None) == \
+        ispa.ISPA_ERR_UNSUPPORTED
+    assert lib.ispa_project_w8a8(P, -1, 128, P, P, P, 0, P, 1 << 20, P, None) == ispa.ISPA_ERR_ARG
+    assert ispa.ispa_project_w8a8_workspace_size(4680, 1536) >= 4680 * 1536 + 4680 * 4
     assert lib.ispa_absorbed_weight(None, None, 128, P, None) == ispa.ISPA_ERR_ARG
     kv = ispa.IspaKV(0x10000, 0x10000, 64)
     assert lib.ispa_full_attention(P, 64, 2, 64, kv, kv, kv, 0.125, None, None, P, 1 << 30, P,

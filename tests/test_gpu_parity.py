@@ -557,3 +557,47 @@ def test_streaming_full_size_sampled_rows(lib, c):
                                      f64(dW) if local else None, local=local)
         assert rel_fro(out, ref) <= ATT_RELFRO + 2 * 2.0 ** -9, (c, local, rel_fro(out, ref))
 
+
+
+def test_w8a8_projection_vs_oracle(lib):
+    """W8A8 projection: the integer codes and scales bit-exact against the
+    oracle's (the same fp32 divisions and rounding decide them), the output
+    within fp32 scaling of the exact int32 sums; ragged rows."""
+    rows, dim = 333, 256
+    a = gaussian((rows, dim), 31, 0, "X").to(torch.bfloat16)
+    a[5] = 0                                        # an all-zero row: scale 1, codes 0
+    W = gaussian((dim, dim), 32, 0, "W") / math.sqrt(dim)
+    dW = 0.1 * gaussian((dim, dim), 33, 0, "W") / math.sqrt(dim)
+    wq_t, w_scale = lib.ispa_quantize_weight_int8(W.cuda(), dW.cuda())
+    ws = torch.empty(lib.ispa_project_w8a8_workspace_size(rows, dim), dtype=torch.uint8,
+                     device="cuda")
+    out32 = lib.ispa_project_w8a8(a.cuda(), wq_t, w_scale, out_dtype=torch.float32, workspace=ws)
+    out16 = lib.ispa_project_w8a8(a.cuda(), wq_t, w_scale)
+    torch.cuda.synchronize()
+    ref, qa, sa, qwt, sw = oracle.project_w8a8(a, W.numpy(), dW.numpy())
+    assert np.array_equal(wq_t.cpu().numpy(), qwt)
+    assert np.array_equal(w_scale.cpu().numpy(), sw)
+    aq = ws[:rows * dim].view(torch.int8).view(rows, dim).cpu().numpy()
+    assert np.array_equal(aq, qa)
+    assert rel_fro(f64(out32), ref) <= 1e-6
+    assert rel_fro(f64(out16), ref) <= 2.0 ** -8
+    assert lib.ispa_project_w8a8(a[:0].cuda(), wq_t, w_scale).shape == (0, dim)
+
+
+def test_w8a8_full_size_streaming_chunk(lib):
+    """The 1.3B chunk shape (4680 rows, d = 1536) on an L-Layer's absorbed
+    weight: against the oracle's W8A8 definition on sampled rows, and within
+    the quantisation error of the bf16 projection."""
+    rows, dim = 4680, 1536
+    a = (0.1 * gaussian((rows, dim), 41, 0, "X")).to(torch.bfloat16)
+    W = gaussian((dim, dim), 42, 0, "W") / math.sqrt(dim)
+    dW = 0.05 * gaussian((dim, dim), 43, 0, "W") / math.sqrt(dim)
+    wq_t, w_scale = lib.ispa_quantize_weight_int8(W.cuda(), dW.cuda())
+    out = lib.ispa_project_w8a8(a.cuda(), wq_t, w_scale, out_dtype=torch.float32)
+    full = lib.ispa_project(a.cuda(), lib.ispa_absorbed_weight(W.cuda(), dW.cuda()),
+                            out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    sel = np.linspace(0, rows - 1, 16).astype(int)
+    ref = oracle.project_w8a8(a[sel], W.numpy(), dW.numpy())[0]
+    assert rel_fro(f64(out)[sel], ref) <= 1e-6
+    assert rel_fro(f64(out), f64(full)) <= 2e-2

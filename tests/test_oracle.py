@@ -393,3 +393,47 @@ def test_streaming_l_layer_with_absorbed_weight_tracks_full_layer():
     l_abs = oracle.streaming_layer(q, ks, vs, kl, vl, kh, vh, W, dW, local=True)
     l_raw = oracle.streaming_layer(q, ks, vs, kl, vl, kh, vh, W, None, local=True)
     assert np.sum((l_abs - full) ** 2) < np.sum((l_raw - full) ** 2)
+
+
+# ---------------------------------------------------------------- W8A8 projection
+
+def test_int8_codes_scale_and_rounding():
+    X = np.array([[0.0, 0.0, 0.0], [1.0, -2.0, 0.5], [127.0, 0.5, 1.5]], dtype=np.float32)
+    q, s = oracle.quantize_rows_int8(X)
+    assert s[0] == 1.0 and not q[0].any()                       # zero row
+    assert s[1] == np.float32(2.0) / np.float32(127.0)
+    assert list(q[1]) == [64, -127, 32]                            # 63.5 -> 64 (half to even), 31.75 -> 32
+    assert s[2] == 1.0 and list(q[2]) == [127, 0, 2]              # 0.5 -> 0 and 1.5 -> 2: half to even
+    r = np.random.default_rng(3).standard_normal((50, 64)).astype(np.float32)
+    q, s = oracle.quantize_rows_int8(r)
+    assert np.all(np.abs(q) <= 127) and np.all(np.abs(q).max(axis=1) == 127)
+    # dequantisation error at most half a step per element
+    assert np.all(np.abs(q * s[:, None] - r) <= 0.5 * s[:, None] * (1 + 1e-6))
+
+
+def test_w8a8_exact_on_integer_grids():
+    """Rows whose largest magnitude is 127 and whose entries are integers get
+    scale 1 and exact codes: the W8A8 product is then the exact product."""
+    r = np.random.default_rng(5)
+    a = r.integers(-127, 128, size=(20, 32)).astype(np.float32)
+    a[:, 0] = 127
+    W = r.integers(-127, 128, size=(32, 16)).astype(np.float32)
+    W[0, :] = -127
+    out, qa, sa, qwt, sw = oracle.project_w8a8(a, W)
+    assert np.all(sa == 1) and np.all(sw == 1)
+    np.testing.assert_array_equal(out, a.astype(np.float64) @ W.astype(np.float64))
+
+
+def test_w8a8_close_to_full_precision_product():
+    r = np.random.default_rng(6)
+    a = r.standard_normal((200, 256)).astype(np.float32)
+    W = (r.standard_normal((256, 256)) / 16).astype(np.float32)
+    dW = (0.1 * r.standard_normal((256, 256)) / 16).astype(np.float32)
+    out = oracle.project_w8a8(a, W, dW)[0]
+    ref = a.astype(np.float64) @ (W + dW).astype(np.float64)
+    err = np.linalg.norm(out - ref) / np.linalg.norm(ref)
+    # per-element rounding of both operands: about (max/127)/sqrt(12) each
+    assert 1e-4 < err < 2e-2
+    # the sum of W and Delta W is taken before quantising
+    out_w = oracle.project_w8a8(a, W + dW)[0]
+    np.testing.assert_array_equal(out, out_w)
