@@ -33,6 +33,8 @@
 // error; substitution only forms products with L, with no such cancellation.
 // Compared with a backward substitution sweep, Z^T Y trades ~d^3/3 extra
 // flops for d/128 fewer dependent launches.
+#include <mutex>
+
 #include "sm100.cuh"
 #include "attention.h"
 #include "host_util.h"
@@ -345,6 +347,33 @@ void to_planes(TGemmProblem& pr, float* hi, int64_t plane) {
   pr.C = nullptr;
 }
 
+// A second stream and two events per device for the one-layer sweep's
+// lookahead (created on first use, kept for the process). The mutex is held
+// while a solve enqueues its work, so that concurrent callers do not re-record
+// each other's events.
+struct Lookahead {
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_look_mutex;
+Lookahead g_look[64];
+
+cudaError_t lookahead_for_device(Lookahead** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  Lookahead& l = g_look[dev];
+  if (!l.side) {
+    if ((e = cudaStreamCreateWithFlags(&l.side, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&l.fork, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&l.join, cudaEventDisableTiming)) != cudaSuccess)
+      return e;
+  }
+  *out = &l;
+  return cudaSuccess;
+}
+
 // Panel of step k: L_{>k,k} = A_{>k,k} Linv^T, Z_k = Linv Z_k, Y_k = Linv Y_k,
 // with Linv = L_kk^-1 from potrf_inv_kernel. Inputs are fp32 (split in the
 // kernel, K = 128); outputs go to the planes, where later products read them.
@@ -446,6 +475,13 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
   // Several layers: left-looking (long-K products that read the finished
   // part once): far less HBM traffic, and the layers supply the parallelism.
   const bool left_looking = n > 1;
+  Lookahead* look = nullptr;
+  std::unique_lock<std::mutex> look_lock;
+  if (!left_looking && nblk > 2) {
+    look_lock = std::unique_lock<std::mutex>(g_look_mutex);
+    if ((e = lookahead_for_device(&look)) != cudaSuccess) return e;
+  }
+  bool side_pending = false;
   for (int k = 0; k < nblk; ++k) {
     const int kk = k * NB;
     const int m = dim - kk - NB;   // rows below the diagonal block
@@ -483,30 +519,59 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
     count_launches();
     if ((e = panel_launch(n, w, d, kk, m, status, stream)) != cudaSuccess) return e;
     if (left_looking || m <= 0) continue;
-    // right-looking: A_{>k,>k} -= L_{>k,k} L_{>k,k}^T (lower tiles);
-    // Z_{>k} -= L_{>k,k} Z_k; Y_{>k} -= L_{>k,k} Y_k (panel outputs pre-split)
-    TGemmParams p{};
-    p.status = status;
-    p.nprob = 3;
-    const float* Lk_h = w.Ah + (size_t)(kk + NB) * d + kk;
-    TGemmProblem& t1 = p.prob[0];
-    if (!opmap_split(t1, true, Lk_h, w.plane, m, NB, d, n, ws, false) ||
-        !opmap_split(t1, false, Lk_h, w.plane, m, NB, d, n, ws, false))
-      return cudaErrorInvalidValue;
-    set_store(t1, m, m, NB, w.A, dim, ws, kk + NB, kk + NB, -1.f, 1.f, n);
-    t1.lower = 1;
-    TGemmProblem& t2 = p.prob[1];
-    if (!opmap_split(t2, true, Lk_h, w.plane, m, NB, d, n, ws, false) ||
-        !opmap_split(t2, false, w.Zh + (size_t)kk * d, w.plane, NB, kk + NB, d, n, ws, true))
-      return cudaErrorInvalidValue;
-    set_store(t2, m, kk + NB, NB, w.Z, dim, ws, kk + NB, 0, -1.f, 1.f, n);
-    TGemmProblem& t3 = p.prob[2];
-    if (!opmap_split(t3, true, Lk_h, w.plane, m, NB, d, n, ws, false) ||
-        !opmap_split(t3, false, w.Yh + (size_t)kk * d, w.plane, NB, d, d, n, ws, true))
-      return cudaErrorInvalidValue;
-    set_store(t3, m, dim, NB, w.Y, dim, ws, kk + NB, 0, -1.f, 1.f, n);
-    if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
+    // right-looking, with lookahead: the rank-128 update of step k
+    // (A_{>k,>k} -= L_{>k,k} L_{>k,k}^T on the lower tiles, Z_{>k} -= L_{>k,k} Z_k,
+    // Y_{>k} -= L_{>k,k} Y_k; panel outputs pre-split) is cut in two. The part
+    // step k+1 needs first -- block column k+1 of A, block rows k+1 of Z and Y
+    // -- runs on `stream`; the rest (rows and columns from k+2 on) runs on a
+    // side stream while step k+1 factors its block and forms its panel. The
+    // side stream's previous update must be done before this step's first part
+    // (it wrote block k+1), and the final one before Delta W.
+    const float* Lk_h = w.Ah + (size_t)(kk + NB) * d + kk;   // L_{>k,k}
+    if (k > 0 && look && (e = cudaStreamWaitEvent(stream, look->join, 0)) != cudaSuccess) return e;
+    for (int part = 0; part < 2; ++part) {
+      const int r0 = part == 0 ? 0 : NB;            // first row (within the rows below) updated
+      const int rows = part == 0 ? (look ? NB : m) : m - NB;
+      if (rows <= 0) break;
+      TGemmParams p{};
+      p.status = status;
+      int q = 0;
+      // A: part 0 = block column k+1 (all rows below), part 1 = lower tiles of the rest
+      {
+        TGemmProblem& t1 = p.prob[q++];
+        const int a_rows = part == 0 ? m : m - NB;
+        const int a_cols = part == 0 ? (look ? NB : m) : m - NB;
+        if (!opmap_split(t1, true, Lk_h + (size_t)r0 * d, w.plane, a_rows, NB, d, n, ws, false) ||
+            !opmap_split(t1, false, Lk_h + (size_t)r0 * d, w.plane, a_cols, NB, d, n, ws, false))
+          return cudaErrorInvalidValue;
+        set_store(t1, a_rows, a_cols, NB, w.A, dim, ws, kk + NB + r0, kk + NB + r0, -1.f, 1.f, n);
+        t1.lower = (part == 1 || !look) ? 1 : 0;
+      }
+      TGemmProblem& t2 = p.prob[q++];
+      if (!opmap_split(t2, true, Lk_h + (size_t)r0 * d, w.plane, rows, NB, d, n, ws, false) ||
+          !opmap_split(t2, false, w.Zh + (size_t)kk * d, w.plane, NB, kk + NB, d, n, ws, true))
+        return cudaErrorInvalidValue;
+      set_store(t2, rows, kk + NB, NB, w.Z, dim, ws, kk + NB + r0, 0, -1.f, 1.f, n);
+      TGemmProblem& t3 = p.prob[q++];
+      if (!opmap_split(t3, true, Lk_h + (size_t)r0 * d, w.plane, rows, NB, d, n, ws, false) ||
+          !opmap_split(t3, false, w.Yh + (size_t)kk * d, w.plane, NB, d, d, n, ws, true))
+        return cudaErrorInvalidValue;
+      set_store(t3, rows, dim, NB, w.Y, dim, ws, kk + NB + r0, 0, -1.f, 1.f, n);
+      p.nprob = q;
+      if (part == 0) {
+        if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
+        if (!look) break;
+      } else {
+        if ((e = cudaEventRecord(look->fork, stream)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(look->side, look->fork, 0)) != cudaSuccess ||
+            (e = launch_tgemm(p, look->side)) != cudaSuccess ||
+            (e = cudaEventRecord(look->join, look->side)) != cudaSuccess)
+          return e;
+        side_pending = true;
+      }
+    }
   }
+  if (side_pending && (e = cudaStreamWaitEvent(stream, look->join, 0)) != cudaSuccess) return e;
   // Delta W = Z^T Y (Z^T upper triangular), both from the planes
   {
     TGemmParams p{};
