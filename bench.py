@@ -363,12 +363,16 @@ def run_ours(args):
     # errors all-gathered for the ranking); a one-layer step runs as replicas
     sharded = world > 1 and cfg.layers >= world
     my_layers = owned_layers(cfg.layers, world, rank) if sharded else list(range(cfg.layers))
-    streams, chunks_per_layer, W_all = make_inputs(cfg, rank, dev, my_layers, replica=not sharded)
+    layer_streams_, chunks_per_layer, W_all = make_inputs(cfg, rank, dev, my_layers,
+                                                          replica=not sharded)
     max_hist = max(len(cfg.history_frames_of(c)) for c in range(cfg.n_chunks)) * cfg.tokens_per_frame
     L = cfg.layers
     L_mine = len(my_layers)
+    # two layers in flight on two streams when there are several (their
+    # launches fill each other's tail SMs)
     runner = LayerWarmup(cfg.heads, cfg.head_dim, cfg.chunk_tokens, cfg.sink_tokens,
-                         cfg.chunk_tokens, max_hist, n_layers=L_mine, device=dev)
+                         cfg.chunk_tokens, max_hist, n_layers=L_mine, device=dev,
+                         n_slots=2 if L_mine >= 2 else 1)
     K = cfg.select_k if cfg.select_k is not None else L // 2
     err_mine = torch.empty(L_mine, 2, dtype=torch.float64, device=dev)
     err = torch.empty(L, 2, dtype=torch.float64, device=dev)
@@ -377,17 +381,26 @@ def run_ours(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     E = lambda: torch.cuda.Event(enable_timing=True)
     runner.weight_gram(W_all)     # W W^T per layer: model weights only, formed once at load
+    streams = [torch.cuda.current_stream()] + ([torch.cuda.Stream()] if runner.n_slots > 1 else [])
 
-    def step(ev=None):
+    def step():
+        runner.layers_chunks(chunks_per_layer, streams)
+        runner.absorb_all(W_all, err_mine)    # every layer's solve + error, batched
+        err.copy_(gather_errors(err_mine, L, world) if sharded else err_mine)
+        rank_layers(err, K, perm, sel)
+
+    def step_instrumented(ev):
+        """The same work on one stream with events around every stage (the
+        per-stage breakdown; not the timed steps)."""
         for li, chunks in enumerate(chunks_per_layer):
             for c, ch in enumerate(chunks):
-                if ev: ev["a0"].append(E()); ev["a0"][-1].record()
+                ev["a0"].append(E()); ev["a0"][-1].record()
                 runner.attention(ch)
-                if ev: ev["a1"].append(E()); ev["a1"][-1].record()
+                ev["a1"].append(E()); ev["a1"][-1].record()
                 runner.gram(first=(c == 0), layer=li)
-                if ev: ev["g1"].append(E()); ev["g1"][-1].record()
-        runner.absorb_all(W_all, err_mine)    # every layer's solve + error, batched
-        if ev: ev["s1"].append(E()); ev["s1"][-1].record()
+                ev["g1"].append(E()); ev["g1"][-1].record()
+        runner.absorb_all(W_all, err_mine)
+        ev["s1"].append(E()); ev["s1"][-1].record()
         err.copy_(gather_errors(err_mine, L, world) if sharded else err_mine)
         rank_layers(err, K, perm, sel)
 
@@ -400,7 +413,6 @@ def run_ours(args):
     bus = torch.cuda.get_device_properties(dev)
     bus_id = f"{getattr(bus, 'pci_domain_id', 0):08x}:{getattr(bus, 'pci_bus_id', 0):02x}:" \
              f"{getattr(bus, 'pci_device_id', 0):02x}.0"
-    ev = {"a0": [], "a1": [], "g1": [], "s1": []}
     starts, ends = [], []
     barrier(world)
     torch.cuda.synchronize()
@@ -409,23 +421,30 @@ def run_ours(args):
     launches0 = ispa.ispa_kernel_launches()
     for _ in range(args.steps):
         flush.zero_()                       # L2 flush between timed steps, outside the events
-        s, e = E(), E()
-        s.record()
-        step(ev)
-        e.record()
-        starts.append(s), ends.append(e)
+        s0, e0 = E(), E()
+        s0.record()
+        step()
+        e0.record()
+        starts.append(s0), ends.append(e0)
     torch.cuda.synchronize()
     launches = ispa.ispa_kernel_launches() - launches0
     clocks = sampler.stop()
     barrier(world)
-
     step_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
-    attn_ms = sum(a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"])) / args.steps
-    gram_ms = sum(a.elapsed_time(b) for a, b in zip(ev["a1"], ev["g1"])) / args.steps
+
+    # per-stage breakdown: a few more steps on one stream, events around every stage
+    n_inst = max(1, min(args.steps, 5))
+    ev = {"a0": [], "a1": [], "g1": [], "s1": []}
+    for _ in range(n_inst):
+        flush.zero_()
+        step_instrumented(ev)
+    torch.cuda.synchronize()
+    attn_ms = sum(a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"])) / n_inst
+    gram_ms = sum(a.elapsed_time(b) for a, b in zip(ev["a1"], ev["g1"])) / n_inst
     # batched solve + error of all layers: from the end of the last Gram to s1
     per_step = L_mine * cfg.n_chunks
     solve_ms = sum(ev["g1"][(i + 1) * per_step - 1].elapsed_time(ev["s1"][i])
-                   for i in range(args.steps)) / args.steps
+                   for i in range(n_inst)) / n_inst
     step_ms_max = max_over_ranks(step_ms, world)
 
     work = step_work(cfg)
@@ -472,8 +491,8 @@ def run_ours(args):
         "clocks": clocks,
     }
     if not args.no_e2e:
-        out["e2e"] = run_e2e(args, cfg, streams, chunks_per_layer, W_all, runner, err, perm,
-                             sel, K, world, err_mine if sharded else None)
+        out["e2e"] = run_e2e(args, cfg, layer_streams_, chunks_per_layer, W_all, runner, err,
+                             perm, sel, K, world, err_mine if sharded else None, streams)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = oracle_throughput(cfg, args.cpu_budget)
     if rank == 0:
@@ -484,7 +503,7 @@ def run_ours(args):
 
 
 def run_e2e(args, cfg, streams, chunks_per_layer, W_all, runner, err, perm, sel, K, world,
-            err_mine=None):
+            err_mine=None, cuda_streams=None):
     """Same step through the public API with the instance's inputs in pinned
     host memory: every step copies each layer's Q/K/V frame streams
     host->device, runs the warmup, and copies every Delta W, the errors and
@@ -510,10 +529,7 @@ def run_e2e(args, cfg, streams, chunks_per_layer, W_all, runner, err, perm, sel,
     def step():
         for h, dv in zip(host_tensors, dev_tensors):
             dv.copy_(h, non_blocking=True)
-        for li, chunks in enumerate(chunks_per_layer):
-            for c, ch in enumerate(chunks):
-                runner.attention(ch)
-                runner.gram(first=(c == 0), layer=li)
+        runner.layers_chunks(chunks_per_layer, cuda_streams)
         if err_mine is not None:
             runner.absorb_all(W_all, err_mine)
             err.copy_(gather_errors(err_mine, L, world))

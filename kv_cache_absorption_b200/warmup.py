@@ -25,24 +25,41 @@ import torch
 from . import ispa
 
 
-class LayerWarmup:
-    """Buffers for ``n_layers`` layers of one geometry; the attention
-    outputs are reused across chunks and layers."""
+class _Slot:
+    """Attention outputs and workspace of one chunk in flight."""
 
-    def __init__(self, heads: int, head_dim: int, chunk_rows: int, max_sink: int,
-                 max_local: int, max_hist: int, n_layers: int = 1, device="cuda"):
-        self.heads, self.head_dim = heads, head_dim
-        self.d = d = heads * head_dim
-        self.n_layers = n_layers
-        self.device = device
+    def __init__(self, heads, head_dim, chunk_rows, max_sink, max_local, max_hist, device):
+        d = heads * head_dim
         f32 = dict(dtype=torch.float32, device=device)
         self.a_loc = torch.empty(chunk_rows, d, **f32)
         self.d_out = torch.empty(chunk_rows, d, **f32)
         self.a_full = torch.empty(chunk_rows, d, dtype=torch.bfloat16, device=device)
         self.lse = [torch.empty(heads, chunk_rows, **f32) for _ in range(3)]
-        self.attn_ws = torch.empty(ispa.ispa_dual_attention_workspace_size(
+        self.ws = torch.empty(ispa.ispa_dual_attention_workspace_size(
             chunk_rows, max_sink, max_local, max_hist, heads, head_dim), dtype=torch.uint8,
             device=device)
+        self.rows = 0
+
+
+class LayerWarmup:
+    """Buffers for ``n_layers`` layers of one geometry. The attention outputs
+    are reused across chunks and layers; ``n_slots`` sets of them let that
+    many layers run their chunks at once on separate streams (layers are
+    independent until the transition), which fills the SMs the tail of one
+    layer's launches leaves idle."""
+
+    def __init__(self, heads: int, head_dim: int, chunk_rows: int, max_sink: int,
+                 max_local: int, max_hist: int, n_layers: int = 1, device="cuda",
+                 n_slots: int = 1):
+        self.heads, self.head_dim = heads, head_dim
+        self.d = d = heads * head_dim
+        self.n_layers = n_layers
+        self.device = device
+        f32 = dict(dtype=torch.float32, device=device)
+        self.slots = [_Slot(heads, head_dim, chunk_rows, max_sink, max_local, max_hist, device)
+                      for _ in range(max(1, n_slots))]
+        s0 = self.slots[0]
+        self.a_loc, self.d_out, self.a_full, self.lse = s0.a_loc, s0.d_out, s0.a_full, s0.lse
         self.M = torch.zeros(n_layers, 2 * d, 2 * d, **f32)
         self.solve_ws = torch.empty(n_layers * ispa.ispa_absorb_workspace_size(d),
                                     dtype=torch.uint8, device=device)
@@ -53,34 +70,65 @@ class LayerWarmup:
         self.B = torch.empty(n_layers, d, d, **f32)
         self.lam = torch.empty(n_layers, **f32)
         self.P = None            # W W^T per layer, once weight_gram has run
-        self._rows = 0
 
-    def attention(self, ch: dict, stream=None):
-        """Dual-stream attention of one chunk into a_loc, d_out, a_full, LSEs."""
+    @property
+    def n_slots(self) -> int:
+        return len(self.slots)
+
+    def attention(self, ch: dict, stream=None, slot: int = 0):
+        """Dual-stream attention of one chunk into the slot's a_loc, d_out,
+        a_full and LSEs."""
+        sl = self.slots[slot]
         q = ch["q"]
-        self._rows = nq = q.shape[0]
+        sl.rows = nq = q.shape[0]
         kv = [ispa._kv(ch["k_sink"], ch["v_sink"], self.heads, self.head_dim, "sink"),
               ispa._kv(ch["k_loc"], ch["v_loc"], self.heads, self.head_dim, "local"),
               ispa._kv(ch.get("k_hist"), ch.get("v_hist"), self.heads, self.head_dim, "history")]
         rc = ispa._load().ispa_dual_attention(
             ispa._ptr(q), nq, self.heads, self.head_dim, kv[0], kv[1], kv[2],
-            float(self.head_dim ** -0.5), ispa._ptr(self.a_loc), ispa._ptr(self.d_out),
-            ispa._ptr(self.a_full), ispa._ptr(self.lse[0]), ispa._ptr(self.lse[1]),
-            ispa._ptr(self.lse[2]), ispa._ptr(self.attn_ws), self.attn_ws.numel(),
+            float(self.head_dim ** -0.5), ispa._ptr(sl.a_loc), ispa._ptr(sl.d_out),
+            ispa._ptr(sl.a_full), ispa._ptr(sl.lse[0]), ispa._ptr(sl.lse[1]),
+            ispa._ptr(sl.lse[2]), ispa._ptr(sl.ws), sl.ws.numel(),
             ispa._ptr(self.status), ispa._stream(stream))
         ispa._check(rc, "ispa_dual_attention")
 
-    def gram(self, first: bool, layer: int = 0, stream=None):
-        """Fold the last chunk's rows into the layer's G, R, S (first chunk
+    def gram(self, first: bool, layer: int = 0, stream=None, slot: int = 0):
+        """Fold the slot's last chunk into the layer's G, R, S (first chunk
         overwrites)."""
+        sl = self.slots[slot]
         rc = ispa._load().ispa_gram_accumulate(
-            ispa._ptr(self.a_loc), ispa._ptr(self.d_out), self._rows, self.d,
+            ispa._ptr(sl.a_loc), ispa._ptr(sl.d_out), sl.rows, self.d,
             ispa._ptr(self.M[layer]), 0 if first else 1, 1, ispa._stream(stream))
         ispa._check(rc, "ispa_gram_accumulate")
 
-    def chunk(self, ch: dict, first: bool, layer: int = 0, stream=None):
-        self.attention(ch, stream)
-        self.gram(first, layer, stream)
+    def chunk(self, ch: dict, first: bool, layer: int = 0, stream=None, slot: int = 0):
+        self.attention(ch, stream, slot)
+        self.gram(first, layer, stream, slot)
+
+    def layers_chunks(self, chunks_per_layer, streams=None):
+        """Every chunk of every layer into the layers' statistics. With
+        ``streams`` (one per slot, the first the caller's current stream),
+        layer l runs on streams[l mod n_slots]; the others fork from and join
+        back into the first."""
+        if not streams or len(streams) == 1 or self.n_slots == 1:
+            s = streams[0] if streams else None
+            for li, chunks in enumerate(chunks_per_layer):
+                for c, ch in enumerate(chunks):
+                    self.chunk(ch, first=(c == 0), layer=li, stream=s)
+            return
+        n = min(len(streams), self.n_slots)
+        fork = torch.cuda.Event()
+        fork.record(streams[0])
+        for s in streams[1:n]:
+            s.wait_event(fork)
+        for li, chunks in enumerate(chunks_per_layer):
+            slot = li % n
+            for c, ch in enumerate(chunks):
+                self.chunk(ch, first=(c == 0), layer=li, stream=streams[slot], slot=slot)
+        for s in streams[1:n]:
+            join = torch.cuda.Event()
+            join.record(s)
+            streams[0].wait_event(join)
 
     def solve(self, W: torch.Tensor, lam: float = 0.0, layer: int = 0, stream=None):
         """Delta W (and B = R W, lambda) of one layer into its slot."""
@@ -160,21 +208,19 @@ def rank(err: torch.Tensor, K: int, perm: torch.Tensor, selected: torch.Tensor, 
 
 
 def run_warmup(chunks_per_layer, W_all: torch.Tensor, K: int, runner: LayerWarmup,
-               stream=None):
+               stream=None, streams=None):
     """Whole warmup: ``chunks_per_layer[l]`` is layer l's list of chunk dicts
     (device tensors), ``W_all`` the [L, d, d] projections. Accumulates every
-    layer's statistics, solves and scores all layers in two batched calls and
-    ranks them. Returns (err [L, 2] fp64, perm, selected); Delta W of layer l
-    is ``runner.dW[l]``."""
+    layer's statistics (layers spread over ``streams`` when given), solves and
+    scores all layers in two batched calls and ranks them. Returns (err
+    [L, 2] fp64, perm, selected); Delta W of layer l is ``runner.dW[l]``."""
     n = len(chunks_per_layer)
     if n != runner.n_layers:
         raise ValueError(f"runner holds {runner.n_layers} layers, got {n}")
     err = torch.empty(n, 2, dtype=torch.float64, device=runner.device)
     perm = torch.empty(n, dtype=torch.int32, device=runner.device)
     sel = torch.empty(n, dtype=torch.uint8, device=runner.device)
-    for li, chunks in enumerate(chunks_per_layer):
-        for c, ch in enumerate(chunks):
-            runner.chunk(ch, first=(c == 0), layer=li, stream=stream)
+    runner.layers_chunks(chunks_per_layer, streams if streams else ([stream] if stream else None))
     runner.absorb_all(W_all, err, stream=stream)
     rank(err, K, perm, sel, stream)
     return err, perm, sel

@@ -362,14 +362,18 @@ def test_warmup_multilayer_ranking(lib):
         eps_ref.append(oracle.warmup_layer(chunks, st.w)["eps"])
         chunks_dev.append([to_dev(c) for c in chunks])
         Ws.append(st.w)
-    runner = LayerWarmup(2, 64, 192, 64, 192, 9 * 64, n_layers=L)
-    err, perm, sel = run_warmup(chunks_dev, torch.stack(Ws).cuda(), 3, runner)
-    torch.cuda.synchronize()
     ref_perm, ref_sel = oracle.rank_layers(eps_ref, 3)
-    got_eps = err[:, 1].cpu().numpy()
-    assert np.max(np.abs(got_eps - eps_ref) / np.asarray(eps_ref)) <= 5e-3
-    assert perm.cpu().numpy().tolist() == ref_perm.tolist()
-    assert sel.cpu().numpy().astype(bool).tolist() == ref_sel.tolist()
+    # one stream, then layers alternating over two streams (two buffer slots)
+    for n_slots in (1, 2):
+        runner = LayerWarmup(2, 64, 192, 64, 192, 9 * 64, n_layers=L, n_slots=n_slots)
+        streams = [torch.cuda.current_stream()] + [torch.cuda.Stream()] * (n_slots - 1)
+        err, perm, sel = run_warmup(chunks_dev, torch.stack(Ws).cuda(), 3, runner,
+                                    streams=streams)
+        torch.cuda.synchronize()
+        got_eps = err[:, 1].cpu().numpy()
+        assert np.max(np.abs(got_eps - eps_ref) / np.asarray(eps_ref)) <= 5e-3, n_slots
+        assert perm.cpu().numpy().tolist() == ref_perm.tolist(), n_slots
+        assert sel.cpu().numpy().astype(bool).tolist() == ref_sel.tolist(), n_slots
 
 
 def test_fp16_range_flag(lib):
