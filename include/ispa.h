@@ -208,8 +208,13 @@ ISPA_API int ispa_gram_accumulate(const float* a_loc, const float* d_in, int64_t
  * Technical summary section 2, step 2 (closed form): solves
  *     (G + lambda I) Delta W = R W
  * with G, R read from M (layout of ispa_gram_accumulate) by a blocked
- * Cholesky factorisation of G + lambda I in fp32 followed by two triangular
- * solves.
+ * Cholesky factorisation of G + lambda I carrying L^-1 and L^-1 R W along
+ * (forward substitution), then Delta W = L^-T (L^-1 R W); every product is
+ * fp32-accurate (3xTF32 on the tensor cores).
+ * Streams: the work is ordered on `stream`. A single-layer solve of more than
+ * two 128-blocks also runs part of each update on a side stream owned by the
+ * library (created on first use per device, joined back with events before
+ * the call's last kernel), so stream capture sees a fork and a join.
  * W        [dim, dim] fp32 row-major, the layer's output projection.
  * lambda   > 0: used as given. <= 0: lambda = 1e-2 * trace(G) / dim,
  *          computed on the device.
@@ -264,7 +269,8 @@ ISPA_API int ispa_absorb_solve_batched(int n_layers, const float* M, int64_t m_l
  * Sharing: all calls use the same array, so calls that overlap on the GPU
  * (other streams, other host threads) race; serialise them. The array keeps
  * the last call's contents, which needs no clearing: each solve writes every
- * scratch buffer before reading it.
+ * scratch buffer before reading it. Everything runs on `stream` (no side
+ * stream, unlike ispa_absorb_solve).
  */
 ISPA_API int ispa_absorb_solve_noalloc(const float* M, const float* W, int dim, float lambda,
                                        float* dW, float* B, float* lambda_out, int* dev_status,

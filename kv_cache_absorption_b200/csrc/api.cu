@@ -17,13 +17,14 @@ void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_rela
 size_t absorb_workspace_bytes(int dim);
 cudaError_t absorb_solve(const float* M, const float* W, int dim, float lambda, float* dW,
                          float* B, float* lambda_out, void* workspace, int* status,
-                         cudaStream_t stream);
+                         cudaStream_t stream, bool side_stream = true);
 cudaError_t layer_error(const float* M, const float* W, const float* dW, const float* B,
                         const float* lam, int dim, double* err, double* acc, cudaStream_t stream);
 cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const float* W,
                                  int64_t w_stride, int dim, float lambda, float* dW,
                                  int64_t dw_stride, float* B, int64_t b_stride, float* lambda_out,
-                                 void* workspace, int* status, cudaStream_t stream);
+                                 void* workspace, int* status, cudaStream_t stream,
+                                 bool side_stream = true);
 cudaError_t layer_error_batched(int n, const float* M, int64_t m_stride, const float* W,
                                 int64_t w_stride, const float* dW, int64_t dw_stride,
                                 const float* B, int64_t b_stride, const float* lam, int dim,

@@ -23,7 +23,7 @@ namespace ispa {
 size_t absorb_workspace_bytes(int dim);
 cudaError_t absorb_solve(const float* M, const float* W, int dim, float lambda, float* dW,
                          float* B, float* lambda_out, void* workspace, int* status,
-                         cudaStream_t stream);
+                         cudaStream_t stream, bool side_stream = true);
 }  // namespace ispa
 
 namespace {
@@ -77,8 +77,9 @@ int ispa_absorb_solve_noalloc(const float* M, const float* W, int dim, float lam
   void* scratch = nullptr;
   const int rc = scratch_for_current_device(&scratch);
   if (rc != ISPA_OK) return rc;
+  // no side stream either: everything runs on the caller's stream
   cudaError_t e = ispa::absorb_solve(M, W, dim, lambda, dW, B, lambda_out, scratch, dev_status,
-                                     static_cast<cudaStream_t>(stream));
+                                     static_cast<cudaStream_t>(stream), false);
   return e == cudaSuccess ? ISPA_OK : ISPA_ERR_CUDA;
 }
 

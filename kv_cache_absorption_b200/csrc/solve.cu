@@ -430,7 +430,8 @@ size_t absorb_workspace_bytes(int dim) {
 cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const float* W,
                                  int64_t w_stride, int dim, float lambda, float* dW,
                                  int64_t dw_stride, float* B, int64_t b_stride, float* lambda_out,
-                                 void* workspace, int* status, cudaStream_t stream) {
+                                 void* workspace, int* status, cudaStream_t stream,
+                                 bool side_stream) {
   const size_t d = (size_t)dim;
   const int64_t ws = (int64_t)(absorb_workspace_bytes(dim) / sizeof(float));  // per-layer stride
   const SolveWs w = solve_ws(workspace, d, ws);
@@ -477,7 +478,7 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
   const bool left_looking = n > 1;
   Lookahead* look = nullptr;
   std::unique_lock<std::mutex> look_lock;
-  if (!left_looking && nblk > 2) {
+  if (!left_looking && nblk > 2 && side_stream) {
     look_lock = std::unique_lock<std::mutex>(g_look_mutex);
     if ((e = lookahead_for_device(&look)) != cudaSuccess) return e;
   }
@@ -591,10 +592,10 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
 
 cudaError_t absorb_solve(const float* M, const float* W, int dim, float lambda, float* dW,
                          float* B, float* lambda_out, void* workspace, int* status,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, bool side_stream) {
   const int64_t dd = (int64_t)dim * dim;
   return absorb_solve_batched(1, M, 4 * dd, W, dd, dim, lambda, dW, dd, B, dd, lambda_out,
-                              workspace, status, stream);
+                              workspace, status, stream, side_stream);
 }
 
 }  // namespace ispa
