@@ -142,6 +142,57 @@ def test_dual_attention_full_size_sampled_rows(lib):
     check_attention(got, ref, "full-size sample")
 
 
+def _full_size_sample(lib, cfg, chunk, n_rows, seed):
+    st = layer_streams(cfg, 0, seed=0)
+    ch = st.chunk(chunk)
+    out = run_dual(lib, to_dev(ch))
+    torch.cuda.synchronize()
+    assert lib.read_status(out["status"]) == 0
+    rows = np.sort(np.random.default_rng(seed).choice(cfg.chunk_tokens, n_rows, replace=False))
+    rows = np.concatenate([rows, [0, cfg.chunk_tokens - 1]])
+    sub = dict(ch)
+    sub["q"] = ch["q"][torch.from_numpy(rows)]
+    ref = ref_dual(sub)
+    idx = torch.from_numpy(rows).cuda()
+    got = {k: (v[idx] if k in ("a_loc", "d", "a_full") else v[:, idx]) for k, v in out.items()
+           if k != "status"}
+    check_attention(got, ref, f"{cfg.name} chunk {chunk}")
+
+
+def test_dual_attention_full_size_14B_sampled_rows(lib):
+    """14B width at full size (40 heads x 128, Nq 4680, keys 1560 + 4680 +
+    14040: the last warmup chunk), 30 sampled rows against the oracle."""
+    from ispa_synth import C3
+    _full_size_sample(lib, C3, C3.n_chunks - 1, 30, seed=3)
+
+
+def test_dual_attention_full_size_first_warmup_chunk(lib):
+    """1.3B warmup chunk 0 at full size: no history (the local units write
+    the final outputs directly, D = 0, LSE_hist = -inf)."""
+    from ispa_synth import C2
+    _full_size_sample(lib, C2, 0, 48, seed=4)
+
+
+def test_gram_full_size_14B_sampled_tiles(lib):
+    """The Gram of 4680 rows at the 14B width (d = 5120, stream-K over 1640
+    output tiles): 8 sampled 128 x 128 tiles of G, R and S against float64."""
+    rows, dim = 4680, 5120
+    a = attention_like(rows, dim, seed=51)
+    dm = 0.3 * attention_like(rows, dim, seed=52)
+    M = lib.ispa_gram_accumulate(a.cuda(), dm.cuda())
+    torch.cuda.synchronize()
+    a64, d64 = f64(a), f64(dm)
+    r = np.random.default_rng(5)
+    for _ in range(8):
+        I, J = sorted(r.integers(0, dim // 128, size=2))
+        i, j = I * 128, J * 128
+        for name, X, Y, oi, oj in (("G", a64, a64, 0, 0), ("R", a64, d64, 0, dim),
+                                   ("S", d64, d64, dim, dim)):
+            ref = X[:, i:i + 128].T @ Y[:, j:j + 128]
+            got = f64(M[oi + i:oi + i + 128, oj + j:oj + j + 128])
+            assert rel_fro(got, ref) <= GR_RELFRO, (name, I, J)
+
+
 # ---------------------------------------------------------------- Gram
 
 def upper_tile_mask(dim):
