@@ -606,7 +606,7 @@ def run_streaming(args):
     build.build()
     from kv_cache_absorption_b200 import ispa
     from kv_cache_absorption_b200.warmup import LayerWarmup, rank as rank_layers
-    from kv_cache_absorption_b200.streaming import StreamingLayers, kv_cache_bytes
+    from kv_cache_absorption_b200.streaming import KVCache, StreamingLayers, kv_cache_bytes
 
     world, rank, local = dist_setup()
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -639,17 +639,50 @@ def run_streaming(args):
     status = ispa.read_status(runner.status)
     del runner, warm_chunks
     torch.cuda.empty_cache()
-    schunks = [[st.chunk(c) for c in range(c_first, c_last + 1)] for st in streams]
+    # per layer and streaming chunk: the new query rows and the chunk's keys
+    # and values, which each step appends to the layer's KV cache
+    new_rows = []
+    for st in streams:
+        rows = []
+        for c in range(c_first, c_last + 1):
+            ch = st.chunk(c)
+            rows.append((ch["q"], ch["k_loc"], ch["v_loc"]))
+        new_rows.append(rows)
+    local_sel = sel.cpu().bool()
+
+    def caches(all_full):
+        """The layers' KV caches at the transition: an F-Layer's holds the
+        sink and the history so far, with room for the rest of the stream; an
+        L-Layer's only the sink and one chunk."""
+        out = []
+        for l, st in enumerate(streams):
+            full = all_full or not bool(local_sel[l])
+            kc = KVCache(cfg.heads, cfg.head_dim, cfg.sink_tokens, cfg.chunk_tokens,
+                         hist_last, full, device=dev)
+            ch = st.chunk(c_first)
+            kc.set_sink(ch["k_sink"], ch["v_sink"])
+            if full:
+                kc.set_history(ch["k_hist"], ch["v_hist"])
+            out.append(kc)
+        return out
+
+    kv_ispa_c, kv_full_c = caches(False), caches(True)
+    torch.cuda.synchronize()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def one_pass(all_full, w8a8=False):
+    def one_pass(kv, all_full, w8a8=False):
+        for kc in kv:
+            kc.rewind()
         for j in range(cfg.stream_chunks):
             for l in range(L):
-                sl.layer(l, schunks[l][j], local=False if all_full else None, w8a8=w8a8)
+                q, k, v = new_rows[l][j]
+                kv[l].append(k, v)
+                sl.layer(l, kv[l].chunk_inputs(q), local=False if all_full else None, w8a8=w8a8)
 
     def timed(all_full, w8a8=False):
+        kv = kv_full_c if all_full else kv_ispa_c
         for _ in range(args.warmup):
-            one_pass(all_full, w8a8)
+            one_pass(kv, all_full, w8a8)
         torch.cuda.synchronize()
         barrier(world)
         ms = []
@@ -657,7 +690,7 @@ def run_streaming(args):
             flush.zero_()
             s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s0.record()
-            one_pass(all_full, w8a8)
+            one_pass(kv, all_full, w8a8)
             s1.record()
             torch.cuda.synchronize()
             ms.append(s0.elapsed_time(s1))
@@ -684,6 +717,7 @@ def run_streaming(args):
         f_flops += 4.0 * cfg.chunk_tokens * nk * d
     kv_all = kv_cache_bytes(L, 0, cfg.sink_tokens, hist_last, cfg.chunk_tokens, d)
     kv_ispa = kv_cache_bytes(L - n_local, n_local, cfg.sink_tokens, hist_last, cfg.chunk_tokens, d)
+    kv_alloc = {"ispa": sum(kc.nbytes for kc in kv_ispa_c), "all_f": sum(kc.nbytes for kc in kv_full_c)}
     bf16_peak, _, peak_src = peaks()
     out = {
         "metric": STREAM_METRIC, "value": round(tokens * world / (ms_ispa * 1e-3), 1),
@@ -705,6 +739,7 @@ def run_streaming(args):
         "ispa_w8a8_speedup_vs_all_f": round(ms_full / ms_w8a8, 3),
         "kv_bytes_last_chunk": {"ispa": kv_ispa, "all_f": kv_all,
                                 "saved_frac": round(1 - kv_ispa / kv_all, 4)},
+        "kv_cache_bytes_allocated": kv_alloc,
         "f_layer_attention_tflops_all_f": round(f_flops * L / (ms_full * 1e-3) / 1e12, 2),
         "attention_frac_of_bf16_peak_all_f": round(f_flops * L / (ms_full * 1e-3) / 1e12 / bf16_peak, 4),
         "peak_source": f"{peak_src} bf16 dense (burst)",

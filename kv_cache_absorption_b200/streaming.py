@@ -27,6 +27,68 @@ def kv_cache_bytes(n_full: int, n_local: int, sink: int, history: int, chunk: in
     return n_full * (sink + history + chunk) * per_token + n_local * (sink + chunk) * per_token
 
 
+class KVCache:
+    """One layer's KV cache after the transition, laid out [sink | history |
+    current chunk] along the token axis. An F-Layer's cache has room for the
+    whole stream and keeps every chunk (the current chunk becomes history
+    when the next one arrives); an L-Layer's holds the sink and one chunk,
+    which each new chunk overwrites."""
+
+    def __init__(self, heads: int, head_dim: int, sink: int, chunk: int, max_hist: int,
+                 full: bool, device="cuda"):
+        cap = sink + chunk + (max_hist if full else 0)
+        self.k = torch.empty(cap, heads, head_dim, dtype=torch.bfloat16, device=device)
+        self.v = torch.empty_like(self.k)
+        self.sink, self.chunk, self.full = sink, chunk, full
+        self.hist = 0            # history tokens held
+        self.cur = 0             # tokens of the current chunk
+        self.hist0 = 0           # history preloaded at the transition
+
+    @property
+    def nbytes(self) -> int:
+        return self.k.numel() * self.k.element_size() + self.v.numel() * self.v.element_size()
+
+    def set_sink(self, k: torch.Tensor, v: torch.Tensor):
+        self.k[:self.sink].copy_(k)
+        self.v[:self.sink].copy_(v)
+
+    def set_history(self, k: torch.Tensor, v: torch.Tensor):
+        """Preload the history an F-Layer holds at the transition."""
+        if not self.full:
+            raise ValueError("an L-Layer keeps no history")
+        n = k.shape[0]
+        if self.sink + n + self.chunk > self.k.shape[0]:
+            raise ValueError("history exceeds the cache")
+        self.k[self.sink:self.sink + n].copy_(k)
+        self.v[self.sink:self.sink + n].copy_(v)
+        self.hist, self.cur, self.hist0 = n, 0, n
+
+    def rewind(self):
+        """Back to the state right after the transition (the preloaded history,
+        no current chunk); the stored tokens are not touched."""
+        self.hist, self.cur = self.hist0, 0
+
+    def append(self, k: torch.Tensor, v: torch.Tensor):
+        """A new chunk's keys and values: an F-Layer moves its previous chunk
+        into the history, an L-Layer drops it."""
+        n = k.shape[0]
+        if self.full:
+            self.hist += self.cur
+        base = self.sink + self.hist
+        if base + n > self.k.shape[0]:
+            raise ValueError("the cache is full")
+        self.k[base:base + n].copy_(k)
+        self.v[base:base + n].copy_(v)
+        self.cur = n
+
+    def chunk_inputs(self, q: torch.Tensor) -> dict:
+        """Attention inputs for the current chunk: views into the cache."""
+        s, h, c = self.sink, self.hist, self.cur
+        return {"q": q, "k_sink": self.k[:s], "v_sink": self.v[:s],
+                "k_loc": self.k[s + h:s + h + c], "v_loc": self.v[s + h:s + h + c],
+                "k_hist": self.k[s:s + h], "v_hist": self.v[s:s + h]}
+
+
 class StreamingLayers:
     """Layer weights after the transition and the buffers of one chunk."""
 
@@ -74,6 +136,8 @@ class StreamingLayers:
                                            wq_t=self.wq[l], w_scale=self.wq_scale[l], stream=stream)
 
     def layer(self, l: int, ch: dict, local=None, w8a8: bool = False, stream=None) -> torch.Tensor:
+        # ``ch`` holds the chunk's query rows and the layer's keys/values (e.g.
+        # KVCache.chunk_inputs); an L-Layer reads only the sink and the chunk.
         """One chunk through layer l (its kind from the transition unless
         ``local`` overrides it; with ``w8a8`` the projection runs on 8-bit
         weights and activations). Returns the projected rows (bf16, reused)."""

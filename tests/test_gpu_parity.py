@@ -614,6 +614,52 @@ def test_streaming_full_size_sampled_rows(lib, c):
 
 
 
+def test_streaming_through_kv_caches(lib):
+    """A stream of post-transition chunks through an F-Layer and an L-Layer
+    whose keys and values come from KV caches the chunks are appended to
+    (the F-Layer's growing over the stream, the L-Layer's holding the sink and
+    one chunk): every chunk's output against the oracle, which takes each
+    chunk's keys straight from the synthetic frame streams. Ragged sizes: 200
+    tokens per frame, a 72-token sink, histories of 600 to 1200 tokens."""
+    from ispa_synth import Config
+    from kv_cache_absorption_b200.streaming import KVCache, StreamingLayers
+    cfg = Config("kv-cache-stream", layers=1, heads=2, head_dim=128, tokens_per_frame=200,
+                 sink_tokens=72, chunk_frames=1, first_chunk_frame=1, n_chunks=3,
+                 history_window=None, stream_chunks=4)
+    st = layer_streams(cfg, 0, seed=5)
+    dim = cfg.d
+    dW = 0.1 * gaussian((dim, dim), 22, 0, "W") / math.sqrt(dim)
+    c_first, c_last = cfg.n_chunks, cfg.n_chunks + cfg.stream_chunks - 1
+    hist_last = len(cfg.history_frames_of(c_last)) * cfg.tokens_per_frame
+    s = StreamingLayers(cfg.heads, cfg.head_dim, cfg.chunk_tokens, cfg.sink_tokens,
+                        cfg.chunk_tokens, hist_last, n_layers=2)
+    s.transition(torch.stack([st.w, st.w]).cuda(), torch.stack([dW, dW]).cuda(), [False, True])
+    first = to_dev(st.chunk(c_first))
+    caches = []
+    for full in (True, False):
+        kc = KVCache(cfg.heads, cfg.head_dim, cfg.sink_tokens, cfg.chunk_tokens, hist_last, full)
+        kc.set_sink(first["k_sink"], first["v_sink"])
+        if full:
+            kc.set_history(first["k_hist"], first["v_hist"])
+        caches.append(kc)
+    for c in range(c_first, c_last + 1):
+        ch = st.chunk(c)
+        d = to_dev(ch)
+        for layer, kc in enumerate(caches):
+            kc.append(d["k_loc"], d["v_loc"])
+            out = f64(s.layer(layer, kc.chunk_inputs(d["q"])))
+            torch.cuda.synchronize()
+            assert lib.read_status(s.status) == 0
+            local = layer == 1
+            ref = oracle.streaming_layer(ch["q"], ch["k_sink"], ch["v_sink"], ch["k_loc"],
+                                         ch["v_loc"], ch["k_hist"], ch["v_hist"], f64(st.w),
+                                         f64(dW) if local else None, local=local)
+            assert rel_fro(out, ref) <= ATT_RELFRO + 2 * 2.0 ** -9, (c, local, rel_fro(out, ref))
+    # at the last chunk the F-Layer's cache holds its whole history, the L-Layer's none
+    assert (caches[0].hist, caches[0].cur) == (hist_last, cfg.chunk_tokens)
+    assert (caches[1].hist, caches[1].cur) == (0, cfg.chunk_tokens)
+
+
 def test_w8a8_projection_vs_oracle(lib):
     """W8A8 projection: the integer codes and scales bit-exact against the
     oracle's (the same fp32 divisions and rounding decide them), the output
