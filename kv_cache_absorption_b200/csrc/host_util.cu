@@ -65,4 +65,18 @@ bool encode_f32_operand_3d(CUtensorMap* m, const float* base, uint64_t rows, uin
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_f32_output_3d(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols,
+                          uint64_t ld, uint64_t layers, uint64_t layer_stride) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  if (layers < 1) layers = 1;
+  cuuint64_t dims[3] = {cols, rows, layers};
+  cuuint64_t strides[2] = {ld * 4, layer_stride * 4};
+  cuuint32_t box[3] = {32u, 32u, 1u};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace ispa

@@ -23,4 +23,10 @@ bool encode_f32_operand(CUtensorMap* m, const float* base, uint64_t rows, uint64
 bool encode_f32_operand_3d(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols,
                            uint64_t ld, uint64_t layers, uint64_t layer_stride, bool mn_major);
 
+// fp32 output maps for tgemm's TMA epilogue: 32 x 32 boxes (one warp's rows
+// x 32 columns), 128-byte swizzle, over `layers` matrices (x = column,
+// y = row, z = layer).
+bool encode_f32_output_3d(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols,
+                          uint64_t ld, uint64_t layers, uint64_t layer_stride);
+
 }  // namespace ispa

@@ -103,9 +103,13 @@ __global__ void copy_layers_kernel(const float4* __restrict__ src, int64_t src_s
 // and writes Linv = L^-1 (lower, zero above) to `linv`, in fp32. The sweep
 // over [A | Z], Z = I, runs in four 32-column steps J:
 //  (1) warp 0 factors the 32 x 32 diagonal sub-block in registers (lane l
-//      holds row l, a runtime loop over the columns keeps the code small
-//      enough for the instruction cache) and stores L_JJ column by column
-//      with the reciprocals of its diagonal;
+//      holds row l) four columns at a time: within a group each pivot comes
+//      from the pivot lane's own entries (one shuffle away from the previous
+//      column), the group's other columns are updated through shuffles, and
+//      the rest of the sub-block gets one rank-4 update from the group's rows
+//      of L broadcast through shared memory (a runtime loop over the groups
+//      keeps the code small); L_JJ is stored column by column with the
+//      reciprocals of its diagonal;
 //  (2) forward substitution with L_JJ, one thread per 32-vector: the panel
 //      rows L_IJ = A_IJ L_JJ^-T (m rows) and the columns of the block row
 //      Z_J <- L_JJ^-1 Z_J (J + 32 columns), m + J + 32 = 128 threads;
@@ -117,7 +121,7 @@ constexpr int kSA = 132;     // a, z: [128][kSA]
 constexpr int kSP = 36;      // panel, row-major [96][kSP]
 constexpr int kST = 100;     // panel, transposed [32][kST]
 constexpr int kSI = 36;      // L_JJ column-major, [32][kSI]
-constexpr size_t kPotrfSmem = (2 * NB * kSA + 96 * kSP + 32 * kST + 32 * kSI + 64) * sizeof(float);
+constexpr size_t kPotrfSmem = (2 * NB * kSA + 96 * kSP + 32 * kST + 32 * kSI + 32 + 4 * 64) * sizeof(float);
 
 __device__ __forceinline__ void ld4(float* d, const float* s) {
   const float4 v = *reinterpret_cast<const float4*>(s);
@@ -139,8 +143,10 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
   float* plT = pl + 96 * kSP;
   float* ljt = plT + 32 * kST;                 // L_JJ, column-major (row c = column c)
   float* rinv = ljt + 32 * kSI;                 // 1 / diagonal of L_JJ
-  float* colv = rinv + 32;                      // one rotated column of L_JJ
+  // rows of L_JJ in one column group (row i: L[i][j0 .. j0+3]); rows 32..63 stay zero
+  float4* grp = reinterpret_cast<float4*>(rinv + 32);
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  if (t < 64) grp[t] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int e = t; e < NB * (NB / 4); e += blockDim.x) {
     const int i = e >> 5, c = (e & 31) * 4;
     *reinterpret_cast<float4*>(&a[i * kSA + c]) =
@@ -152,8 +158,10 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
   __syncthreads();
   for (int J = 0; J < NB; J += 32) {
     const int m = 96 - J;                       // rows below the diagonal sub-block
-    // ---- (1a) warp 0: L_JJ, a compact loop (lane l holds row l; r[0] is the
-    // current column, the row shifts left by one column per step)
+    // ---- (1) warp 0: L_JJ in groups of four columns. r[c] holds row `lane`,
+    // column j0 + c of the sub-block, updated with every column before j0
+    // (zero above the diagonal of the stored factor; the row shifts left by
+    // four columns per group).
     if (warp == 0) {
       float r[32];
 #pragma unroll
@@ -161,22 +169,38 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
 #pragma unroll
       for (int k = 0; k < 32; ++k) r[k] = (k <= lane) ? r[k] : 0.f;
 #pragma unroll 1
-      for (int j = 0; j < 32; ++j) {
-        const float piv = __shfl_sync(0xffffffffu, r[0], j);
-        if (lane == 0 && !(piv > 0.f)) atomicOr(status, ISPA_STATUS_NOT_SPD);
-        const float inv = rsqrtf(piv);         // NaN for a non-positive pivot: poisons what follows
-        const float l0 = lane > j ? r[0] * inv : (lane == j ? piv * inv : 0.f);   // L[lane][j]
-        ljt[j * kSI + lane] = l0;                // column j of L_JJ
-        if (lane == j) rinv[j] = inv;            // 1 / L_jj
-        // column j rotated so that slot c holds L[j + c][j]; slots past row 31 hold 0
-        colv[lane >= j ? lane - j : lane - j + 32] = lane >= j ? l0 : 0.f;
+      for (int j0 = 0; j0 < 32; j0 += 4) {
+        float tp = r[0];                          // on lane j0: the group's first pivot
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int j = j0 + m;
+          const float piv = __shfl_sync(0xffffffffu, tp, j);
+          if (lane == 0 && !(piv > 0.f)) atomicOr(status, ISPA_STATUS_NOT_SPD);
+          const float inv = rsqrtf(piv);         // NaN for a non-positive pivot: poisons what follows
+          const float lv = lane > j ? r[m] * inv : (lane == j ? piv * inv : 0.f);   // L[lane][j]
+          r[m] = lv;
+          ljt[j * kSI + lane] = lv;              // column j of L_JJ
+          if (lane == j) rinv[j] = inv;          // 1 / L_jj
+          // lane j + 1 forms its next pivot from its own entries (the same
+          // arithmetic as the shuffled update below gives it)
+          if (m < 3) tp = fmaf(-lv, lv, r[m + 1]);
+#pragma unroll
+          for (int m2 = m + 1; m2 < 4; ++m2)
+            r[m2] = fmaf(-lv, __shfl_sync(0xffffffffu, lv, j0 + m2), r[m2]);
+        }
+        const float l0 = r[0], l1 = r[1], l2 = r[2], l3 = r[3];
+        grp[lane] = make_float4(l0, l1, l2, l3);
         __syncwarp();
-        float cv[32];
+        // rank-4 update of the later columns, shifted left by the group
 #pragma unroll
-        for (int q = 0; q < 8; ++q) ld4(&cv[4 * q], &colv[4 * q]);
-#pragma unroll
-        for (int c = 1; c < 32; ++c) r[c - 1] = fmaf(-l0, cv[c], r[c]);
-        r[31] = 0.f;
+        for (int c = 4; c < 32; ++c) {
+          const float4 x = grp[j0 + c];          // L[j0 + c][j0 .. j0+3]; zero past row 31
+          float v = fmaf(-l0, x.x, r[c]);
+          v = fmaf(-l1, x.y, v);
+          v = fmaf(-l2, x.z, v);
+          r[c - 4] = fmaf(-l3, x.w, v);
+        }
+        r[28] = r[29] = r[30] = r[31] = 0.f;
         __syncwarp();
       }
     }
@@ -347,13 +371,17 @@ void to_planes(TGemmProblem& pr, float* hi, int64_t plane) {
   pr.C = nullptr;
 }
 
-// A second stream and two events per device for the one-layer sweep's
-// lookahead (created on first use, kept for the process). The mutex is held
-// while a solve enqueues its work, so that concurrent callers do not re-record
-// each other's events.
+// Streams and events per device for the one-layer sweep (created on first
+// use, kept for the process): the sweep's critical path -- factor, panel and
+// the part of each update the next step needs -- runs on `crit`, created at the
+// device's greatest stream priority; the rest of each update runs on `side`, at
+// the least, so that the block scheduler dispatches critical-path CTAs ahead of
+// the bulk update's pending ones. Both are forked from the caller's stream and
+// joined back to it. The mutex is held while a solve enqueues its work, so that
+// concurrent callers do not re-record each other's events.
 struct Lookahead {
-  cudaStream_t side = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaStream_t crit = nullptr, side = nullptr;
+  cudaEvent_t start = nullptr, fork = nullptr, join = nullptr, done = nullptr;
 };
 std::mutex g_look_mutex;
 Lookahead g_look[64];
@@ -365,14 +393,34 @@ cudaError_t lookahead_for_device(Lookahead** out) {
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   Lookahead& l = g_look[dev];
   if (!l.side) {
-    if ((e = cudaStreamCreateWithFlags(&l.side, cudaStreamNonBlocking)) != cudaSuccess ||
+    int least = 0, greatest = 0;
+    if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess ||
+        (e = cudaStreamCreateWithPriority(&l.crit, cudaStreamNonBlocking, greatest)) != cudaSuccess ||
+        (e = cudaStreamCreateWithPriority(&l.side, cudaStreamNonBlocking, least)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&l.start, cudaEventDisableTiming)) != cudaSuccess ||
         (e = cudaEventCreateWithFlags(&l.fork, cudaEventDisableTiming)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&l.join, cudaEventDisableTiming)) != cudaSuccess)
+        (e = cudaEventCreateWithFlags(&l.join, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&l.done, cudaEventDisableTiming)) != cudaSuccess)
       return e;
   }
   *out = &l;
   return cudaSuccess;
 }
+
+// Joins the sweep's streams back into the caller's stream when the solve
+// returns, on its error paths too: `crit` waits for the side stream's last
+// update, then the caller's stream waits for `crit`.
+struct SweepJoin {
+  Lookahead* look = nullptr;
+  cudaStream_t caller = nullptr;
+  bool side_pending = false;
+  ~SweepJoin() {
+    if (!look) return;
+    if (side_pending) cudaStreamWaitEvent(look->crit, look->join, 0);
+    cudaEventRecord(look->done, look->crit);
+    cudaStreamWaitEvent(caller, look->done, 0);
+  }
+};
 
 // Panel of step k: L_{>k,k} = A_{>k,k} Linv^T, Z_k = Linv Z_k, Y_k = Linv Y_k,
 // with Linv = L_kk^-1 from potrf_inv_kernel. Inputs are fp32 (split in the
@@ -441,6 +489,25 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
   cudaFuncSetAttribute(potrf_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)kPotrfSmem);
 
+  // One layer: right-looking (a rank-128 update of everything below the block
+  // after each step): up to (d/128)^2 tiles per launch keep the GPU busy.
+  // Several layers: left-looking (long-K products that read the finished
+  // part once): far less HBM traffic, and the layers supply the parallelism.
+  const bool left_looking = n > 1;
+  std::unique_lock<std::mutex> look_lock;
+  SweepJoin join;
+  join.caller = stream;
+  Lookahead* look = nullptr;
+  if (!left_looking && nblk > 2 && side_stream) {
+    look_lock = std::unique_lock<std::mutex>(g_look_mutex);
+    if ((e = lookahead_for_device(&look)) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(look->start, stream)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(look->crit, look->start, 0)) != cudaSuccess)
+      return e;
+    join.look = look;
+    stream = look->crit;            // everything below runs on the critical-path stream
+  }
+
   lambda_kernel<<<n, 256, 0, stream>>>(M, m_stride, dim, lambda, w.lam, ws, lambda_out);
   count_launches();
 
@@ -471,18 +538,6 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
       (int64_t)(d * d / 4));
   count_launches(2);
 
-  // One layer: right-looking (a rank-128 update of everything below the block
-  // after each step): up to (d/128)^2 tiles per launch keep the GPU busy.
-  // Several layers: left-looking (long-K products that read the finished
-  // part once): far less HBM traffic, and the layers supply the parallelism.
-  const bool left_looking = n > 1;
-  Lookahead* look = nullptr;
-  std::unique_lock<std::mutex> look_lock;
-  if (!left_looking && nblk > 2 && side_stream) {
-    look_lock = std::unique_lock<std::mutex>(g_look_mutex);
-    if ((e = lookahead_for_device(&look)) != cudaSuccess) return e;
-  }
-  bool side_pending = false;
   for (int k = 0; k < nblk; ++k) {
     const int kk = k * NB;
     const int m = dim - kk - NB;   // rows below the diagonal block
@@ -568,11 +623,14 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
             (e = launch_tgemm(p, look->side)) != cudaSuccess ||
             (e = cudaEventRecord(look->join, look->side)) != cudaSuccess)
           return e;
-        side_pending = true;
+        join.side_pending = true;
       }
     }
   }
-  if (side_pending && (e = cudaStreamWaitEvent(stream, look->join, 0)) != cudaSuccess) return e;
+  if (join.side_pending) {
+    if ((e = cudaStreamWaitEvent(stream, look->join, 0)) != cudaSuccess) return e;
+    join.side_pending = false;
+  }
   // Delta W = Z^T Y (Z^T upper triangular), both from the planes
   {
     TGemmParams p{};

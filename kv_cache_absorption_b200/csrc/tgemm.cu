@@ -20,6 +20,15 @@
 // slabs), warp 1 TMEM owner and MMA issuer, warps 2-5 split each slab into
 // hi/lo and then run the epilogue.
 //
+// Epilogue: each epilogue warp owns 32 accumulator rows (its TMEM lane
+// quarter). Where the output allows it (beta 0 or 1, 16-byte aligned rows),
+// the warp stages its rows 32 columns at a time in the operand ring, free once
+// the accumulator is ready, and hands each 32 x 32 box to TMA: a store for
+// beta = 0, an fp32 reduce-add into C for beta = 1 (C + alpha op(A) op(B),
+// rounded once, as a read-modify-write would round it). Neither waits on
+// global memory, and each box moves as whole 128-byte rows. Otherwise each
+// thread reads and writes its own row directly.
+//
 // The split in shared memory costs as much as the MMAs themselves (it halves
 // the kernel's rate). Operands that later products read again are therefore
 // kept pre-split in global memory as two planes, hi and lo, rounded exactly
@@ -34,6 +43,7 @@
 // fp32 round-to-nearest additions while the next chunk is in flight.
 #include "sm100.cuh"
 #include "attention.h"
+#include "host_util.h"
 #include "tgemm.h"
 
 namespace ispa {
@@ -43,6 +53,26 @@ constexpr int TM = 128, TN = 128, TK = 32;
 constexpr int NSTAGE = 3;
 constexpr int kThreads = 192;
 constexpr int kSlab = TM * TK * 4;   // 16 KB: one operand slab, fp32
+
+// TMA epilogue helpers (shared -> global tile copies, bulk-group completion)
+__device__ __forceinline__ void tma_store_box(const CUtensorMap* m, const void* src, int x, int y,
+                                              int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void tma_add_box(const CUtensorMap* m, const void* src, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], [%1];"
+      ::"l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+constexpr int kBox = 32 * 32 * 4;   // one 32 x 32 fp32 output box
 
 struct alignas(1024) GSmem {
   uint8_t a_hi[NSTAGE][kSlab];
@@ -277,7 +307,62 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
     const int64_t col0 = (int64_t)pr.c_col0 + (int64_t)tj * TN;
     if (ok && (nk == 0 || mbar_wait(&s.acc_full, 0, p.status, abort_flag))) {
       tc_fence_after();
-      if (pr.mode == kModeStore) {
+      if (pr.mode == kModeStore && pr.out_tma) {
+        // boxes of this warp: per 32-column chunk, C and/or the hi and lo
+        // planes; at most 4 x 3 boxes (48 KB) a warp, 192 KB = the whole ring
+        const float alpha = pr.alpha;
+        const bool add = pr.beta != 0.f;
+        const int nbox = (pr.C ? 1 : 0) + (pr.C_hi ? 2 : 0);
+        uint8_t* wbox = s.a_hi[0] + (size_t)quarter * (TN / 32) * nbox * kBox;
+        const int x0 = pr.c_col0 + tj * TN;
+        const int y0 = pr.c_row0 + ti * TM + quarter * 32;
+#pragma unroll 1
+        for (int c = 0; c < TN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tacc + lane_off + c * 32, v);
+          tmem_ld_wait();
+          uint8_t* bx = wbox + (size_t)c * nbox * kBox;
+          uint8_t* rowp = bx + lane * 128;   // this thread's row of each box
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float4 o;
+            o.x = nk > 0 ? alpha * __uint_as_float(v[4 * j]) : 0.f;
+            o.y = nk > 0 ? alpha * __uint_as_float(v[4 * j + 1]) : 0.f;
+            o.z = nk > 0 ? alpha * __uint_as_float(v[4 * j + 2]) : 0.f;
+            o.w = nk > 0 ? alpha * __uint_as_float(v[4 * j + 3]) : 0.f;
+            const int sw = (j ^ (lane & 7)) << 4;   // 128-byte swizzle of 16-byte chunks
+            int b = 0;
+            if (pr.C) { *reinterpret_cast<float4*>(rowp + sw) = o; b = 1; }
+            if (pr.C_hi) {
+              float4 h, l;
+              h.x = to_tf32(o.x); l.x = to_tf32(o.x - h.x);
+              h.y = to_tf32(o.y); l.y = to_tf32(o.y - h.y);
+              h.z = to_tf32(o.z); l.z = to_tf32(o.z - h.z);
+              h.w = to_tf32(o.w); l.w = to_tf32(o.w - h.w);
+              *reinterpret_cast<float4*>(rowp + b * kBox + sw) = h;
+              *reinterpret_cast<float4*>(rowp + (b + 1) * kBox + sw) = l;
+            }
+          }
+          fence_proxy_async_smem();   // generic-proxy writes -> visible to TMA (async proxy)
+          __syncwarp();
+          if (lane == 0) {
+            const int x = x0 + c * 32;
+            int b = 0;
+            if (pr.C) {
+              if (add) tma_add_box(&pr.tc, bx, x, y0, layer);
+              else tma_store_box(&pr.tc, bx, x, y0, layer);
+              b = 1;
+            }
+            if (pr.C_hi) {
+              tma_store_box(&pr.tc_hi, bx + b * kBox, x, y0, layer);
+              tma_store_box(&pr.tc_lo, bx + (b + 1) * kBox, x, y0, layer);
+            }
+            bulk_commit();
+          }
+        }
+        if (lane == 0) bulk_wait_read_all();   // the boxes are read before the CTA exits
+        __syncwarp();
+      } else if (pr.mode == kModeStore) {
         const int64_t off = (int64_t)layer * pr.c_layer_stride + row * pr.ldc + col0;
         float* crow = pr.C ? pr.C + off : nullptr;            // beta != 0 needs C
         float* hrow = pr.C_hi ? pr.C_hi + off : nullptr;
@@ -402,10 +487,35 @@ cudaError_t launch_split_planes(int layers, const float* src, int64_t ld_src, in
 
 size_t tgemm_smem_bytes() { return sizeof(GSmem) + 1024; }
 
+// Output map of one destination of a store problem: the rows and columns the
+// problem can reach, over its layers.
+static bool output_map(CUtensorMap* m, const float* base, const TGemmProblem& pr) {
+  if (!base || (reinterpret_cast<uintptr_t>(base) & 15)) return false;
+  const uint64_t rows = (uint64_t)pr.c_row0 + (uint64_t)pr.M;
+  const uint64_t cols = (uint64_t)pr.c_col0 + (uint64_t)pr.N;
+  const uint64_t ls = pr.layers > 1 ? (uint64_t)pr.c_layer_stride : rows * (uint64_t)pr.ldc;
+  return encode_f32_output_3d(m, base, rows, cols, (uint64_t)pr.ldc, (uint64_t)pr.layers, ls);
+}
+
+// The TMA epilogue takes beta = 0 (any destinations) or beta = 1 into C alone,
+// 16-byte aligned rows and column offsets; other problems keep the per-thread
+// epilogue.
+static void plan_output(TGemmProblem& pr) {
+  pr.out_tma = 0;
+  if (pr.mode != kModeStore || !(pr.C || pr.C_hi)) return;
+  if (!(pr.beta == 0.f || (pr.beta == 1.f && !pr.C_hi))) return;
+  if (pr.ldc % 4 != 0 || pr.c_col0 % 4 != 0 || pr.c_row0 < 0 || pr.c_col0 < 0) return;
+  if (pr.layers > 1 && pr.c_layer_stride % 4 != 0) return;
+  if (pr.C && !output_map(&pr.tc, pr.C, pr)) return;
+  if (pr.C_hi && !(output_map(&pr.tc_hi, pr.C_hi, pr) && output_map(&pr.tc_lo, pr.C_lo, pr))) return;
+  pr.out_tma = 1;
+}
+
 cudaError_t launch_tgemm(TGemmParams& p, cudaStream_t stream) {
   int base = 0;
   for (int q = 0; q < p.nprob; ++q) {
     TGemmProblem& pr = p.prob[q];
+    plan_output(pr);
     pr.mt = pr.M / TM;
     pr.nt = pr.N / TN;
     if (pr.layers < 1) pr.layers = 1;

@@ -25,6 +25,7 @@ struct TGemmProblem {
   CUtensorMap tb;
   CUtensorMap ta_lo;      // the lo plane of a pre-split operand (a_split / b_split)
   CUtensorMap tb_lo;
+  CUtensorMap tc, tc_hi, tc_lo;   // output maps of the TMA epilogue (set by launch_tgemm)
   int a_split, b_split;   // operand given as tf32 hi/lo planes: no split in the kernel
   int a_mn, b_mn;
   int M, N, K;
@@ -41,6 +42,7 @@ struct TGemmProblem {
   int mode;      // kMode*
   int layers;    // >= 1
   int mt, nt, tiles_per_layer, tile_base;   // set by launch_tgemm
+  int out_tma;   // set by launch_tgemm: the epilogue stores (beta = 0) or reduce-adds (beta = 1) by TMA
 };
 
 struct TGemmParams {
