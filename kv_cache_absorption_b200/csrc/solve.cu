@@ -38,6 +38,7 @@
 #include "sm100.cuh"
 #include "attention.h"
 #include "host_util.h"
+#include "pdl.h"
 #include "tgemm.h"
 
 namespace ispa {
@@ -147,6 +148,8 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
   float4* grp = reinterpret_cast<float4*>(rinv + 32);
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   if (t < 64) grp[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+  pdl_wait();       // the update that wrote this block has completed
+  pdl_trigger();
   for (int e = t; e < NB * (NB / 4); e += blockDim.x) {
     const int i = e >> 5, c = (e & 31) * 4;
     *reinterpret_cast<float4*>(&a[i * kSA + c]) =
@@ -570,8 +573,10 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
       u3.tri = kTriLowerB;
       if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
     }
-    potrf_inv_kernel<<<n, 512, kPotrfSmem, stream>>>(w.A + (size_t)kk * d + kk, dim, w.Linv, ws,
-                                                     status);
+    if ((e = launch_pdl(potrf_inv_kernel, dim3(n), dim3(512), kPotrfSmem, stream,
+                        (const float*)(w.A + (size_t)kk * d + kk), dim, w.Linv, ws, status)) !=
+        cudaSuccess)
+      return e;
     count_launches();
     if ((e = panel_launch(n, w, d, kk, m, status, stream)) != cudaSuccess) return e;
     if (left_looking || m <= 0) continue;

@@ -44,6 +44,7 @@
 #include "sm100.cuh"
 #include "attention.h"
 #include "host_util.h"
+#include "pdl.h"
 #include "tgemm.h"
 
 namespace ispa {
@@ -183,6 +184,10 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tacc = s.taddr;
+  // launched after the previous kernel of the stream may have started: its
+  // outputs are complete from here on; the next kernel may start its prologue
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0 && nk > 0) {
@@ -526,9 +531,9 @@ cudaError_t launch_tgemm(TGemmParams& p, cudaStream_t stream) {
   if (base == 0) return cudaSuccess;
   const size_t smem = tgemm_smem_bytes();
   cudaFuncSetAttribute(tgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  tgemm_kernel<<<base, kThreads, smem, stream>>>(p);
+  const cudaError_t e = launch_pdl(tgemm_kernel, dim3(base), dim3(kThreads), smem, stream, p);
   count_launches();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace ispa
