@@ -384,7 +384,7 @@ void to_planes(TGemmProblem& pr, float* hi, int64_t plane) {
 // concurrent callers do not re-record each other's events.
 struct Lookahead {
   cudaStream_t crit = nullptr, side = nullptr;
-  cudaEvent_t start = nullptr, fork = nullptr, join = nullptr, done = nullptr;
+  cudaEvent_t start = nullptr, fork = nullptr, join = nullptr, done = nullptr, rw = nullptr;
 };
 std::mutex g_look_mutex;
 Lookahead g_look[64];
@@ -403,7 +403,8 @@ cudaError_t lookahead_for_device(Lookahead** out) {
         (e = cudaEventCreateWithFlags(&l.start, cudaEventDisableTiming)) != cudaSuccess ||
         (e = cudaEventCreateWithFlags(&l.fork, cudaEventDisableTiming)) != cudaSuccess ||
         (e = cudaEventCreateWithFlags(&l.join, cudaEventDisableTiming)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&l.done, cudaEventDisableTiming)) != cudaSuccess)
+        (e = cudaEventCreateWithFlags(&l.done, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&l.rw, cudaEventDisableTiming)) != cudaSuccess)
       return e;
   }
   *out = &l;
@@ -515,11 +516,18 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
   count_launches();
 
   // B = R W (R = M[0:d, d:2d]): both split once into the Z and Y planes (free
-  // until the sweep), then one pre-split product
+  // until the sweep's first panel), then one pre-split product; Y = B is the
+  // right-hand side of the substitution. With the side stream this runs there,
+  // beside the build and the first block factor, which touch neither.
+  cudaStream_t rw_stream = stream;
+  if (look) {
+    if ((e = cudaStreamWaitEvent(look->side, look->start, 0)) != cudaSuccess) return e;
+    rw_stream = look->side;
+  }
   if ((e = launch_split_planes(n, M + d, 2 * d, m_stride, w.Zh, w.Zh + w.plane, d, ws, dim, dim,
-                               stream)) != cudaSuccess ||
+                               rw_stream)) != cudaSuccess ||
       (e = launch_split_planes(n, W, d, w_stride, w.Yh, w.Yh + w.plane, d, ws, dim, dim,
-                               stream)) != cudaSuccess)
+                               rw_stream)) != cudaSuccess)
     return e;
   {
     TGemmParams p{};
@@ -531,15 +539,22 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
         !opmap_split(pr, false, w.Yh, w.plane, d, d, d, n, ws, true))
       return cudaErrorInvalidValue;
     set_store(pr, dim, dim, dim, B, dim, b_stride, 0, 0, 1.f, 0.f, n);
-    if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
+    if ((e = launch_tgemm(p, rw_stream)) != cudaSuccess) return e;
   }
-  // A = G + lambda I, Z = I; Y = B (the right-hand side of the substitution)
-  build_kernel<<<dim3(n == 1 ? 148 * 8 : 148, n), 256, 0, stream>>>(M, m_stride, dim, w.A, ws,
-                                                                     lam_off);
-  copy_layers_kernel<<<dim3(n == 1 ? 148 * 4 : 148, n), 256, 0, stream>>>(
+  copy_layers_kernel<<<dim3(n == 1 ? 148 * 4 : 148, n), 256, 0, rw_stream>>>(
       reinterpret_cast<const float4*>(B), b_stride / 4, reinterpret_cast<float4*>(w.Y), ws / 4,
       (int64_t)(d * d / 4));
-  count_launches(2);
+  count_launches();
+  if (look) {
+    if ((e = cudaEventRecord(look->rw, look->side)) != cudaSuccess ||
+        (e = cudaEventRecord(look->join, look->side)) != cudaSuccess)
+      return e;
+    join.side_pending = true;
+  }
+  // A = G + lambda I, Z = I
+  build_kernel<<<dim3(n == 1 ? 148 * 8 : 148, n), 256, 0, stream>>>(M, m_stride, dim, w.A, ws,
+                                                                     lam_off);
+  count_launches();
 
   for (int k = 0; k < nblk; ++k) {
     const int kk = k * NB;
@@ -578,6 +593,7 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
         cudaSuccess)
       return e;
     count_launches();
+    if (k == 0 && look && (e = cudaStreamWaitEvent(stream, look->rw, 0)) != cudaSuccess) return e;
     if ((e = panel_launch(n, w, d, kk, m, status, stream)) != cudaSuccess) return e;
     if (left_looking || m <= 0) continue;
     // right-looking, with lookahead: the rank-128 update of step k
@@ -648,6 +664,14 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
       return cudaErrorInvalidValue;
     set_store(pr, dim, dim, dim, dW, dim, dw_stride, 0, 0, 1.f, 0.f, n);
     pr.tri = kTriUpperA;
+    if (n == 1) {
+      // one layer: the first tile rows read up to d/32 slabs and the last 4;
+      // two CTAs per tile, each over half of its slabs, reduce-add into a
+      // zeroed Delta W (as many CTAs as SMs twice over, the longest half as long)
+      if ((e = cudaMemsetAsync(dW, 0, d * d * sizeof(float), stream)) != cudaSuccess) return e;
+      pr.beta = 1.f;
+      pr.ksplit = 2;
+    }
     if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
   }
   return cudaGetLastError();

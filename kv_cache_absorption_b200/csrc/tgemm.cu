@@ -103,13 +103,16 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 // Layer and tile (i, j) of problem `q` from the launch-wide tile index.
 __device__ __forceinline__ void decode(const TGemmParams& p, int b, int& q, int& layer, int& i,
-                                       int& j) {
+                                       int& j, int& part) {
   q = 0;
   while (q + 1 < p.nprob && b >= p.prob[q + 1].tile_base) ++q;
   const TGemmProblem& pr = p.prob[q];
   int t = b - pr.tile_base;
   layer = t / pr.tiles_per_layer;
   t -= layer * pr.tiles_per_layer;
+  const int ks = pr.ksplit > 1 ? pr.ksplit : 1;
+  part = t % ks;
+  t /= ks;
   if (pr.lower) {   // tiles with j <= i, row by row
     int r = (int)((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
     while ((r + 1) * (r + 2) / 2 <= t) ++r;
@@ -122,12 +125,19 @@ __device__ __forceinline__ void decode(const TGemmParams& p, int b, int& q, int&
   }
 }
 
-__device__ __forceinline__ void k_range(const TGemmProblem& pr, int i, int j, int& kb, int& ke) {
+__device__ __forceinline__ void k_range(const TGemmProblem& pr, int i, int j, int part, int& kb,
+                                        int& ke) {
   kb = 0;
   ke = pr.K / TK;
   if (pr.tri == kTriLowerA) ke = min(ke, (i + 1) * (TM / TK));
   if (pr.tri == kTriUpperA) kb = i * (TM / TK);
   if (pr.tri == kTriLowerB) kb = min(ke, j * (TN / TK));
+  if (pr.ksplit > 1) {   // this CTA's share of the tile's slabs
+    const int len = ke - kb, ks = pr.ksplit;
+    const int b0 = kb + (len * part) / ks, b1 = kb + (len * (part + 1)) / ks;
+    kb = b0;
+    ke = b1;
+  }
 }
 
 // Loads one 32-deep slab of a 128-wide operand block (rows/cols starting at
@@ -153,11 +163,11 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
   GSmem& s = *reinterpret_cast<GSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   volatile int* abort_flag = &s.abort_flag;
-  int q, layer, ti, tj;
-  decode(p, blockIdx.x, q, layer, ti, tj);
+  int q, layer, ti, tj, part;
+  decode(p, blockIdx.x, q, layer, ti, tj, part);
   const TGemmProblem& pr = p.prob[q];
   int kb, ke;
-  k_range(pr, ti, tj, kb, ke);
+  k_range(pr, ti, tj, part, kb, ke);
   const int nk = ke - kb;
 
   if (threadIdx.x == 0) {
@@ -507,6 +517,7 @@ static bool output_map(CUtensorMap* m, const float* base, const TGemmProblem& pr
 // epilogue.
 static void plan_output(TGemmProblem& pr) {
   pr.out_tma = 0;
+  if (pr.ksplit > 1 && (pr.beta != 1.f || pr.C_hi)) return;   // split K accumulates into C
   if (pr.mode != kModeStore || !(pr.C || pr.C_hi)) return;
   if (!(pr.beta == 0.f || (pr.beta == 1.f && !pr.C_hi))) return;
   if (pr.ldc % 4 != 0 || pr.c_col0 % 4 != 0 || pr.c_row0 < 0 || pr.c_col0 < 0) return;
@@ -524,7 +535,9 @@ cudaError_t launch_tgemm(TGemmParams& p, cudaStream_t stream) {
     pr.mt = pr.M / TM;
     pr.nt = pr.N / TN;
     if (pr.layers < 1) pr.layers = 1;
-    pr.tiles_per_layer = pr.lower ? pr.mt * (pr.mt + 1) / 2 : pr.mt * pr.nt;
+    if (pr.ksplit > 2) return cudaErrorInvalidValue;
+    if (pr.ksplit == 2 && !pr.out_tma) return cudaErrorInvalidValue;   // needs the reduce-add epilogue
+    pr.tiles_per_layer = (pr.lower ? pr.mt * (pr.mt + 1) / 2 : pr.mt * pr.nt) * (pr.ksplit > 1 ? pr.ksplit : 1);
     pr.tile_base = base;
     base += pr.tiles_per_layer * pr.layers;
   }

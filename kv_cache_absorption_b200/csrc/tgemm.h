@@ -43,6 +43,10 @@ struct TGemmProblem {
   int layers;    // >= 1
   int mt, nt, tiles_per_layer, tile_base;   // set by launch_tgemm
   int out_tma;   // set by launch_tgemm: the epilogue stores (beta = 0) or reduce-adds (beta = 1) by TMA
+  int ksplit;    // 0/1: one CTA per tile; 2: two CTAs per tile, each over half of the tile's K
+                 // slabs, both reduce-adding into C (beta = 1, C zeroed by the caller; the two
+                 // fp32 partial sums meet in one commutative addition, so the result does not
+                 // depend on their order)
 };
 
 struct TGemmParams {
