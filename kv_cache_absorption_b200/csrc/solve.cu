@@ -115,7 +115,9 @@ __global__ void copy_layers_kernel(const float4* __restrict__ src, int64_t src_s
 //      rows L_IJ = A_IJ L_JJ^-T (m rows) and the columns of the block row
 //      Z_J <- L_JJ^-1 Z_J (J + 32 columns), m + J + 32 = 128 threads;
 //  (3) trailing update in 4 x 4 register tiles: A_II -= L_IJ L_IJ^T on the
-//      lower tiles and Z_I -= L_IJ Z_J.
+//      lower tiles and Z_I -= L_IJ Z_J. With lookahead: the next diagonal
+//      sub-block is updated by warp 0, which factors it at once, while warps
+//      1-15 apply the rest of the update.
 // Shared-memory row strides (132, 36, 100 floats) keep the float4 accesses
 // 16-byte aligned and free of bank conflicts.
 constexpr int kSA = 132;     // a, z: [128][kSA]
@@ -159,14 +161,11 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
                     i == c + 3 ? 1.f : 0.f);
   }
   __syncthreads();
-  for (int J = 0; J < NB; J += 32) {
-    const int m = 96 - J;                       // rows below the diagonal sub-block
-    // ---- (1) warp 0: L_JJ in groups of four columns. r[c] holds row `lane`,
-    // column j0 + c of the sub-block, updated with every column before j0
-    // (zero above the diagonal of the stored factor; the row shifts left by
-    // four columns per group).
-    if (warp == 0) {
+  // warp 0: L_JJ of the 32 x 32 diagonal sub-block at J (see step (1) above)
+  auto factor32 = [&](int J) {
+    {
       float r[32];
+      bool bad = false;
 #pragma unroll
       for (int q = 0; q < 8; ++q) ld4(&r[4 * q], &a[(J + lane) * kSA + J + 4 * q]);
 #pragma unroll
@@ -178,7 +177,7 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
         for (int m = 0; m < 4; ++m) {
           const int j = j0 + m;
           const float piv = __shfl_sync(0xffffffffu, tp, j);
-          if (lane == 0 && !(piv > 0.f)) atomicOr(status, ISPA_STATUS_NOT_SPD);
+          bad |= !(piv > 0.f);
           const float inv = rsqrtf(piv);         // NaN for a non-positive pivot: poisons what follows
           const float lv = lane > j ? r[m] * inv : (lane == j ? piv * inv : 0.f);   // L[lane][j]
           r[m] = lv;
@@ -205,6 +204,87 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
         }
         r[28] = r[29] = r[30] = r[31] = 0.f;
         __syncwarp();
+      }
+      if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, ISPA_STATUS_NOT_SPD);
+    }
+  };
+  for (int J = 0; J < NB; J += 32) {
+    const int m = 96 - J;                       // rows below the diagonal sub-block
+    // ---- (1) with lookahead: warp 0 brings the diagonal sub-block J up to
+    // date with the previous step's panel (its lower triangle) and factors it,
+    // while warps 1-15 apply the rest of the previous step's trailing update
+    if (warp == 0) {
+      if (J > 0) {
+        float li[32];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) ld4(&li[4 * q], &pl[lane * kSP + 4 * q]);
+        float* arow = &a[(J + lane) * kSA + J];
+#pragma unroll 1
+        for (int c0 = 0; c0 < 32; c0 += 4) {
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            float lc[4][4];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) ld4(lc[cc], &pl[(c0 + cc) * kSP + 4 * q4]);
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+              for (int cc = 0; cc < 4; ++cc) acc[cc] = fmaf(li[4 * q4 + qq], lc[cc][qq], acc[cc]);
+          }
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+            if (c0 + cc <= lane) arow[c0 + cc] -= acc[cc];
+        }
+        __syncwarp();
+      }
+      factor32(J);
+    } else if (J > 0) {
+      // ---- (3) trailing update of the previous step, one 4 x 4 tile per thread
+      const int Jp = J - 32, mp = 96 - Jp;
+      const int mt = mp / 4, n_tri = mt * (mt + 1) / 2, nzt = (Jp + 32) / 4;
+      // triangle tiles are numbered row by row: the first 36 (rows 0..7) are
+      // the next diagonal sub-block, which warp 0 has updated itself
+      const int tt = t - 32 + 36;
+      if (tt < n_tri + mt * nzt) {
+        int ti, tj;
+        const bool tri = tt < n_tri;
+        if (tri) {
+          ti = (int)((sqrtf(8.f * tt + 1.f) - 1.f) * 0.5f);
+          while (ti * (ti + 1) / 2 > tt) --ti;
+          while ((ti + 1) * (ti + 2) / 2 <= tt) ++ti;
+          tj = tt - ti * (ti + 1) / 2;
+        } else {
+          ti = (tt - n_tri) / nzt;
+          tj = (tt - n_tri) % nzt;
+        }
+        float acc[4][4] = {};
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float pa[4][4], pb[4][4];
+#pragma unroll
+          for (int r4 = 0; r4 < 4; ++r4) ld4(pa[r4], &pl[(4 * ti + r4) * kSP + 4 * q]);
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4)
+            ld4(pb[k4], tri ? &plT[(4 * q + k4) * kST + 4 * tj]
+                            : &z[(Jp + 4 * q + k4) * kSA + 4 * tj]);
+#pragma unroll
+          for (int r4 = 0; r4 < 4; ++r4)
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4)
+#pragma unroll
+              for (int c4 = 0; c4 < 4; ++c4) acc[r4][c4] = fmaf(pa[r4][k4], pb[k4][c4], acc[r4][c4]);
+        }
+        float* dst = tri ? &a[(J + 4 * ti) * kSA + J + 4 * tj]
+                         : &z[(J + 4 * ti) * kSA + 4 * tj];
+#pragma unroll
+        for (int r4 = 0; r4 < 4; ++r4) {
+          float v[4];
+          ld4(v, dst + r4 * kSA);
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) v[c4] -= acc[r4][c4];
+          st4(dst + r4 * kSA, v);
+        }
       }
     }
     __syncthreads();
@@ -240,51 +320,6 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
       } else {
 #pragma unroll
         for (int k = 0; k < 32; ++k) z[(J + k) * kSA + zc] = acc[k];
-      }
-    }
-    __syncthreads();
-    // ---- (3) trailing update, one 4 x 4 tile per thread (at most 492 tiles)
-    if (m > 0) {
-      const int mt = m / 4, n_tri = mt * (mt + 1) / 2, nzt = (J + 32) / 4;
-      if (t < n_tri + mt * nzt) {
-        int ti, tj;
-        const bool tri = t < n_tri;
-        if (tri) {
-          ti = (int)((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
-          while (ti * (ti + 1) / 2 > t) --ti;
-          while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
-          tj = t - ti * (ti + 1) / 2;
-        } else {
-          ti = (t - n_tri) / nzt;
-          tj = (t - n_tri) % nzt;
-        }
-        float acc[4][4] = {};
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float pa[4][4], pb[4][4];
-#pragma unroll
-          for (int r4 = 0; r4 < 4; ++r4) ld4(pa[r4], &pl[(4 * ti + r4) * kSP + 4 * q]);
-#pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4)
-            ld4(pb[k4], tri ? &plT[(4 * q + k4) * kST + 4 * tj]
-                            : &z[(J + 4 * q + k4) * kSA + 4 * tj]);
-#pragma unroll
-          for (int r4 = 0; r4 < 4; ++r4)
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4)
-#pragma unroll
-              for (int c4 = 0; c4 < 4; ++c4) acc[r4][c4] = fmaf(pa[r4][k4], pb[k4][c4], acc[r4][c4]);
-        }
-        float* dst = tri ? &a[(J + 32 + 4 * ti) * kSA + J + 32 + 4 * tj]
-                         : &z[(J + 32 + 4 * ti) * kSA + 4 * tj];
-#pragma unroll
-        for (int r4 = 0; r4 < 4; ++r4) {
-          float v[4];
-          ld4(v, dst + r4 * kSA);
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) v[c4] -= acc[r4][c4];
-          st4(dst + r4 * kSA, v);
-        }
       }
     }
     __syncthreads();
