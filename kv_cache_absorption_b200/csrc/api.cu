@@ -253,15 +253,15 @@ int ispa_gram_accumulate(const float* a_loc, const float* d_in, int64_t rows, in
   if (rows == 0) return ISPA_OK;
   ispa::GramParams p;
   std::memset(&p, 0, sizeof(p));
-  if (!encode_2d(&p.tm_a, a_loc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dim, rows, dim, 32, 32,
+  if (!encode_2d(&p.tm_a, a_loc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dim, rows, dim, 32, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) ||
-      !encode_2d(&p.tm_d, d_in, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dim, rows, dim, 32, 32,
+      !encode_2d(&p.tm_d, d_in, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dim, rows, dim, 32, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B))
     return ISPA_ERR_CUDA;
   const int bn = (dim % 256 == 0) ? 256 : 128;
   p.M = M;
   p.dim = dim;
-  p.k_iters = (int)((rows + 31) / 32);
+  p.k_iters = (int)((rows + 63) / 64);   // 64-row k-blocks (the kernel's BK)
   p.want_s = want_s ? 1 : 0;
   p.n_tiles = ispa::gram_tile_count(dim, bn, p.want_s);
   p.total_iters = (int64_t)p.n_tiles * p.k_iters;

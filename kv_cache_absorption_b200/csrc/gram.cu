@@ -14,7 +14,7 @@
 // operands require. The inputs are used as tf32 (the attention epilogue
 // already rounds them to nearest), accumulation is fp32 in TMEM.
 //
-// Work split: persistent stream-K. The (tile, 32-row k-block) iteration
+// Work split: persistent stream-K. The (tile, 64-row k-block) iteration
 // space is cut into equal contiguous ranges, one per CTA, so every SM does
 // the same number of MMAs whatever the tile count; each range's partial tile
 // is added into M with fp32 vector atomics (M is zeroed first when the call
@@ -26,8 +26,8 @@ namespace ispa {
 namespace {
 
 constexpr int BM = 128;
-constexpr int BK = 32;          // rows per stage
-constexpr int NSTAGE = 4;
+constexpr int BK = 64;          // rows per stage (64-row TMA boxes: half the boxes of 32)
+constexpr int NSTAGE = 2;
 constexpr int kThreads = 192;
 
 template <int BN>
