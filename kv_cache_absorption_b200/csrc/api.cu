@@ -270,7 +270,9 @@ int ispa_gram_accumulate(const float* a_loc, const float* d_in, int64_t rows, in
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t grid = p.total_iters < sms ? p.total_iters : sms;
-  p.iters_per_cta = (p.total_iters + grid - 1) / grid;
+  // whole tiles in waves of `grid`, then the rest split evenly (see gram.cu)
+  const int64_t tail = p.total_iters - (int64_t)(p.n_tiles / grid) * grid * p.k_iters;
+  p.iters_per_cta = (tail + grid - 1) / grid;
   p.status = nullptr;
   return cuda_rc(ispa::launch_gram(p, bn, (int)grid, s));
 }

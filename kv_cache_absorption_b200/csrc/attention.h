@@ -56,15 +56,15 @@ cudaError_t launch_dual_attention(const AttnParams& p, int head_dim, cudaStream_
 
 // Gram accumulation: see gram.cu.
 struct GramParams {
-  CUtensorMap tm_a;       // A_loc [rows, dim] fp32, 32-column x 32-row boxes
+  CUtensorMap tm_a;       // A_loc [rows, dim] fp32, 32-column x 64-row boxes
   CUtensorMap tm_d;       // D
   float* M;               // [2 dim, 2 dim]
   int dim;
-  int k_iters;            // ceil(rows / 32)
+  int k_iters;            // ceil(rows / 64)
   int want_s;
   int n_tiles;
   int64_t total_iters;
-  int64_t iters_per_cta;
+  int64_t iters_per_cta;  // of the iterations left after the whole-tile waves
   int* status;
 };
 cudaError_t launch_gram(const GramParams& p, int bn, int grid, cudaStream_t stream);
