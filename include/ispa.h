@@ -211,10 +211,13 @@ ISPA_API int ispa_gram_accumulate(const float* a_loc, const float* d_in, int64_t
  * Cholesky factorisation of G + lambda I carrying L^-1 and L^-1 R W along
  * (forward substitution), then Delta W = L^-T (L^-1 R W); every product is
  * fp32-accurate (3xTF32 on the tensor cores).
- * Streams: the work is ordered on `stream`. A single-layer solve of more than
- * two 128-blocks also runs part of each update on a side stream owned by the
- * library (created on first use per device, joined back with events before
- * the call's last kernel), so stream capture sees a fork and a join.
+ * Streams: the work is ordered after `stream`'s earlier work, and `stream`
+ * waits for all of it before its next work. A single-layer solve of more than
+ * two 128-blocks runs on two streams owned by the library (created on first
+ * use per device): the factorisation's critical path on one at the device's
+ * greatest priority, R W and the bulk of each update on the other at the
+ * least; both fork from `stream` with an event and join back into it with
+ * events, on error returns too, so stream capture sees a fork and a join.
  * W        [dim, dim] fp32 row-major, the layer's output projection.
  * lambda   > 0: used as given. <= 0: lambda = 1e-2 * trace(G) / dim,
  *          computed on the device.
