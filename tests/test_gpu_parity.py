@@ -201,8 +201,11 @@ def upper_tile_mask(dim):
     return I <= J
 
 
-@pytest.mark.parametrize("rows,dim", [(1000, 256), (777, 384), (64, 128)])
+@pytest.mark.parametrize("rows,dim", [(1000, 256), (777, 384), (64, 128), (700, 1536)])
 def test_gram_accumulate_two_calls(lib, rows, dim):
+    """Every output tile against float64; at d = 1536 there are 156 tiles, so
+    the kernel runs one wave of whole tiles and splits the remaining tiles'
+    row blocks over all CTAs (stream-K)."""
     a1 = attention_like(rows, dim, seed=1)
     d1 = 0.3 * attention_like(rows, dim, seed=2)
     a2 = attention_like(rows + 40, dim, seed=3)
@@ -268,6 +271,23 @@ def test_absorb_solve_isolated(lib, dim):
     dW, B = oracle.absorb(Gf, Rf, f64(W), lam)
     assert rel_fro(f64(out["B"]), B) <= product_tol(Rf, f64(W), B)
     assert rel_fro(f64(out["dW"]), dW) <= DW_RELFRO
+
+
+def test_absorb_solve_deterministic(lib):
+    """Two solves of the same layer give bit-identical B and Delta W: the
+    single-layer sweep runs on two streams and Delta W sums two K halves
+    into a zeroed output, whose fp32 addition does not depend on the order."""
+    dim = 512
+    a, f, W = synthetic_layer(4 * dim + 100, dim, seed=77)
+    G, R, S = oracle.gram(a, f - a)
+    M = pack_M(G, R, S).cuda()
+    Wd = W.cuda()
+    first = lib.ispa_absorb_solve(M, Wd)
+    second = lib.ispa_absorb_solve(M, Wd)
+    torch.cuda.synchronize()
+    assert lib.read_status(first["status"]) == 0 and lib.read_status(second["status"]) == 0
+    assert torch.equal(first["dW"], second["dW"])
+    assert torch.equal(first["B"], second["B"])
 
 
 # Full-size solve inputs: rows = iid N(0, 1) plus one common mean mode m. The
