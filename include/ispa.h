@@ -264,7 +264,7 @@ ISPA_API int ispa_absorb_solve_batched(int n_layers, const float* M, int64_t m_l
  * enter an allocator. The solve's scratch lives in a device array inside
  * the library instead.
  * Limits: dim must be a multiple of 128 and at most 512; larger dims return
- * ISPA_ERR_UNSUPPORTED. The array (about 9.5 MB) is held by every GPU that
+ * ISPA_ERR_UNSUPPORTED. The array (about 9.6 MB) is held by every GPU that
  * loads the library until the process exits.
  * Set-up: the first call on a device looks up the array's device address
  * (once per device, with that device current); make that first call before

@@ -8,7 +8,7 @@
 // caller still provides M, W and every output.
 //
 // The array holds the scratch of one solve of dimension up to
-// kNoAllocMaxDim (about 9.5 MB); every GPU that loads this library holds it
+// kNoAllocMaxDim (about 9.6 MB); every GPU that loads this library holds it
 // until the process exits. All calls share it, so calls that overlap on the
 // GPU (different streams, or different host threads on one device) race and
 // corrupt each other's results; serialise them. Each solve writes every
@@ -30,7 +30,7 @@ namespace {
 
 constexpr int kNoAllocMaxDim = 512;
 // (9 d^2 + 128^2) floats + 1 KB for d = 512, the layout ispa::absorb_solve uses.
-constexpr size_t kNoAllocBytes = (9ull * 512 * 512 + 128 * 128) * sizeof(float) + 1024;
+constexpr size_t kNoAllocBytes = (9ull * 512 * 512 + 3 * 128 * 128) * sizeof(float) + 1024;
 
 __device__ __align__(256) unsigned char g_absorb_scratch[kNoAllocBytes];
 

@@ -331,6 +331,13 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
 #pragma unroll
     for (int c4 = 0; c4 < 4; ++c4) v[c4] = (c + c4 <= i) ? v[c4] : 0.f;
     st4(&linv[(size_t)i * NB + c], v);
+    // the planes the panel products read: hi = tf32(v), lo = tf32(v - hi),
+    // rounded as the GEMM's in-kernel split rounds them
+    float h[4], l[4];
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) { h[c4] = to_tf32(v[c4]); l[c4] = to_tf32(v[c4] - h[c4]); }
+    st4(&linv[NB * NB + (size_t)i * NB + c], h);
+    st4(&linv[2 * NB * NB + (size_t)i * NB + c], l);
   }
 }
 
@@ -362,11 +369,11 @@ bool opmap(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols, uint
 
 // Per-layer workspace, in floats (d = dim): A, Z, Y (fp32), then the hi and
 // lo planes of A, Z and Y (each plane d^2, lo = hi + d^2), one 128 x 128
-// inverse and lambda. Finished blocks of L (in A's planes), of L^-1 and of
-// L^-1 B are kept only as planes: every product that reads them again takes
-// them pre-split.
+// inverse (fp32, then its hi and lo planes) and lambda. Finished blocks of L
+// (in A's planes), of L^-1 and of L^-1 B are kept only as planes: every
+// product that reads them again takes them pre-split.
 struct SolveWs {
-  float *A, *Z, *Y, *Ah, *Zh, *Yh, *Linv, *lam;
+  float *A, *Z, *Y, *Ah, *Zh, *Yh, *Linv, *Lh, *lam;
   int64_t plane;        // lo = hi + plane
   int64_t stride;       // floats between layers' workspaces
 };
@@ -381,7 +388,8 @@ SolveWs solve_ws(void* workspace, size_t d, int64_t stride) {
   w.Zh = w.Ah + 2 * dd;
   w.Yh = w.Zh + 2 * dd;
   w.Linv = w.Yh + 2 * dd;
-  w.lam = w.Linv + NB * NB;
+  w.Lh = w.Linv + NB * NB;          // hi / lo planes of Linv (lo = hi + NB * NB)
+  w.lam = w.Lh + 2 * NB * NB;
   w.plane = (int64_t)dd;
   w.stride = stride;
   return w;
@@ -462,8 +470,9 @@ struct SweepJoin {
 };
 
 // Panel of step k: L_{>k,k} = A_{>k,k} Linv^T, Z_k = Linv Z_k, Y_k = Linv Y_k,
-// with Linv = L_kk^-1 from potrf_inv_kernel. Inputs are fp32 (split in the
-// kernel, K = 128); outputs go to the planes, where later products read them.
+// with Linv = L_kk^-1 from potrf_inv_kernel, read from its pre-split planes;
+// A_{>k,k}, Z_k and Y_k are fp32 (split in the kernel, K = 128); outputs go to
+// the planes, where later products read them.
 cudaError_t panel_launch(int n, const SolveWs& w, size_t d, int kk, int m, int* status,
                          cudaStream_t stream) {
   const int dim = (int)d;
@@ -474,31 +483,28 @@ cudaError_t panel_launch(int n, const SolveWs& w, size_t d, int kk, int m, int* 
   if (m > 0) {
     TGemmProblem& pr = p.prob[q++];
     if (!opmap(&pr.ta, w.A + (size_t)(kk + NB) * d + kk, m, NB, d, n, ws, false) ||
-        !opmap(&pr.tb, w.Linv, NB, NB, NB, n, ws, false))
+        !opmap_split(pr, false, w.Lh, NB * NB, NB, NB, NB, n, ws, false))
       return cudaErrorInvalidValue;
     set_store(pr, m, NB, NB, nullptr, dim, ws, kk + NB, kk, 1.f, 0.f, n);
     to_planes(pr, w.Ah, w.plane);
     pr.a_mn = 0;
-    pr.b_mn = 0;
   }
   {
     TGemmProblem& pr = p.prob[q++];
-    if (!opmap(&pr.ta, w.Linv, NB, NB, NB, n, ws, false) ||
+    if (!opmap_split(pr, true, w.Lh, NB * NB, NB, NB, NB, n, ws, false) ||
         !opmap(&pr.tb, w.Z + (size_t)kk * d, NB, kk + NB, d, n, ws, true))
       return cudaErrorInvalidValue;
     set_store(pr, NB, kk + NB, NB, nullptr, dim, ws, kk, 0, 1.f, 0.f, n);
     to_planes(pr, w.Zh, w.plane);
-    pr.a_mn = 0;
     pr.b_mn = 1;
   }
   {
     TGemmProblem& pr = p.prob[q++];
-    if (!opmap(&pr.ta, w.Linv, NB, NB, NB, n, ws, false) ||
+    if (!opmap_split(pr, true, w.Lh, NB * NB, NB, NB, NB, n, ws, false) ||
         !opmap(&pr.tb, w.Y + (size_t)kk * d, NB, d, d, n, ws, true))
       return cudaErrorInvalidValue;
     set_store(pr, NB, dim, NB, nullptr, dim, ws, kk, 0, 1.f, 0.f, n);
     to_planes(pr, w.Yh, w.plane);
-    pr.a_mn = 0;
     pr.b_mn = 1;
   }
   p.nprob = q;
@@ -509,9 +515,10 @@ cudaError_t panel_launch(int n, const SolveWs& w, size_t d, int kk, int m, int* 
 
 size_t absorb_workspace_bytes(int dim) {
   const size_t d = (size_t)dim;
-  // A, Z, Y; hi/lo planes of each; one 128 x 128 inverse; lambda (+ padding);
+  // A, Z, Y; hi/lo planes of each; one 128 x 128 inverse and its hi/lo
+  // planes; lambda (+ padding);
   // a multiple of 256 bytes so that per-layer workspaces stack
-  return ((9 * d * d + NB * NB) * sizeof(float) + 1024 + 255) & ~size_t(255);
+  return ((9 * d * d + 3 * NB * NB) * sizeof(float) + 1024 + 255) & ~size_t(255);
 }
 
 cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const float* W,
