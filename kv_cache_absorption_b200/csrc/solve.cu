@@ -50,10 +50,13 @@ constexpr int NB = 128;
 constexpr int kChunkSlabs = 4;
 
 // lambda = value if value > 0, else 1e-2 * trace(G) / dim (G = M[0:d, 0:d]);
-// one block per layer.
+// one block of kLambdaThreads per layer (the diagonal entries are 2d floats
+// apart: one or two loads a thread keep the read latency off the critical
+// path of a one-layer solve).
+constexpr int kLambdaThreads = 1024;
 __global__ void lambda_kernel(const float* __restrict__ M0, int64_t m_stride, int dim, float value,
                               float* lam_ws0, int64_t ws_stride, float* lam_out) {
-  __shared__ double part[256];
+  __shared__ double part[kLambdaThreads];
   const float* M = M0 + (int64_t)blockIdx.x * m_stride;
   float* lam_ws = lam_ws0 + (int64_t)blockIdx.x * ws_stride;
   double s = 0.0;
@@ -554,7 +557,7 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
     stream = look->crit;            // everything below runs on the critical-path stream
   }
 
-  lambda_kernel<<<n, 256, 0, stream>>>(M, m_stride, dim, lambda, w.lam, ws, lambda_out);
+  lambda_kernel<<<n, kLambdaThreads, 0, stream>>>(M, m_stride, dim, lambda, w.lam, ws, lambda_out);
   count_launches();
 
   // B = R W (R = M[0:d, d:2d]): both split once into the Z and Y planes (free
