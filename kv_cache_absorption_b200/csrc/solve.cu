@@ -25,8 +25,12 @@
 //     One layer: right-looking. After step k one grouped launch applies the
 //     rank-128 update to the lower tiles of A and to the rows of Z and Y
 //     below the block: more traffic, but (d/128)^2 tiles per launch where
-//     the left-looking step of a single layer would have ~2 d/128;
-//   * then one triangular-aware GEMM: Delta W = Z^T Y.
+//     the left-looking step of a single layer would have ~2 d/128. The
+//     sweep's critical path (factor, panel, the part of each update the
+//     next step needs) runs on a high-priority stream; B = R W and the rest
+//     of each update run on a second stream beside it;
+//   * then one triangular-aware GEMM: Delta W = Z^T Y (for one layer in two
+//     K halves per tile that reduce-add into a zeroed Delta W).
 // Y is formed by substitution, not as the product Z B: entries of L^-1
 // alternate in sign and |L^-1| |B| can exceed |L^-1 B| by three orders of
 // magnitude, which a product at fp32 precision turns into a 1e-3 relative

@@ -14,7 +14,10 @@
 // (the K index contiguous) or MN-major (M or N contiguous), so transposes
 // cost nothing. A launch may hold up to 4 independent problems ("grouped");
 // a problem can be restricted to the tiles on or below its diagonal, and to
-// the K range a triangular A or B operand leaves non-zero.
+// the K range a triangular A or B operand leaves non-zero. A problem may also
+// give each tile to two CTAs, each over half of its K slabs, both
+// reduce-adding into C (for a triangular product of one layer, whose
+// longest tiles would otherwise set the time).
 //
 // Warp roles (192 threads): warp 0 TMA producer (3-stage ring of 32-deep K
 // slabs), warp 1 TMEM owner and MMA issuer, warps 2-5 split each slab into
