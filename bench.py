@@ -368,11 +368,11 @@ def run_ours(args):
     max_hist = max(len(cfg.history_frames_of(c)) for c in range(cfg.n_chunks)) * cfg.tokens_per_frame
     L = cfg.layers
     L_mine = len(my_layers)
-    # two layers in flight on two streams when there are several (their
-    # launches fill each other's tail SMs)
+    # several layers in flight on as many streams (their launches fill each
+    # other's tail SMs); three by default
     runner = LayerWarmup(cfg.heads, cfg.head_dim, cfg.chunk_tokens, cfg.sink_tokens,
                          cfg.chunk_tokens, max_hist, n_layers=L_mine, device=dev,
-                         n_slots=2 if L_mine >= 2 else 1)
+                         n_slots=max(1, min(args.slots, L_mine)))
     K = cfg.select_k if cfg.select_k is not None else L // 2
     err_mine = torch.empty(L_mine, 2, dtype=torch.float64, device=dev)
     err = torch.empty(L, 2, dtype=torch.float64, device=dev)
@@ -381,7 +381,7 @@ def run_ours(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     E = lambda: torch.cuda.Event(enable_timing=True)
     runner.weight_gram(W_all)     # W W^T per layer: model weights only, formed once at load
-    streams = [torch.cuda.current_stream()] + ([torch.cuda.Stream()] if runner.n_slots > 1 else [])
+    streams = [torch.cuda.current_stream()] + [torch.cuda.Stream() for _ in range(runner.n_slots - 1)]
 
     def step():
         runner.layers_chunks(chunks_per_layer, streams)
@@ -870,6 +870,8 @@ def main():
     ap.add_argument("--config", choices=("c1", "c2", "c3", "c4"), default="c1")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the workload's layer count (smaller captures for ncu)")
+    ap.add_argument("--slots", type=int, default=3,
+                    help="layers in flight on separate streams in a multi-layer warmup")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
