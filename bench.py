@@ -369,7 +369,7 @@ def run_ours(args):
     L = cfg.layers
     L_mine = len(my_layers)
     # several layers in flight on as many streams (their launches fill each
-    # other's tail SMs); three by default
+    # other's tail SMs); two by default
     runner = LayerWarmup(cfg.heads, cfg.head_dim, cfg.chunk_tokens, cfg.sink_tokens,
                          cfg.chunk_tokens, max_hist, n_layers=L_mine, device=dev,
                          n_slots=max(1, min(args.slots, L_mine)))
@@ -870,7 +870,7 @@ def main():
     ap.add_argument("--config", choices=("c1", "c2", "c3", "c4"), default="c1")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the workload's layer count (smaller captures for ncu)")
-    ap.add_argument("--slots", type=int, default=3,
+    ap.add_argument("--slots", type=int, default=2,
                     help="layers in flight on separate streams in a multi-layer warmup")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
