@@ -1,0 +1,59 @@
+"""The benchmark's work model and roofline arithmetic (no GPU): the counts
+behind every TFLOP/s and % of roofline that bench.py reports."""
+import argparse
+import math
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from ispa_synth import C1, C2, C3  # noqa: E402
+
+
+def test_chunk_step_work_matches_the_stated_counts():
+    """1.3B chunk: attention 4 Nq Nk d over sink + local + history keys (the
+    number the attention roofline divides by), Gram 4 N d^2, solve
+    (1/3 + 4) d^3, error d^3."""
+    w = bench.step_work(C1)
+    nq, nk, d = 4680, 1560 + 4680 + 14040, 1536
+    assert w["attention"] == 4.0 * nq * nk * d == 583129497600.0
+    assert w["gram"] == 4.0 * 4680 * d * d
+    assert math.isclose(w["solve"], (1.0 / 3.0 + 4.0) * d ** 3)
+    assert w["error"] == float(d) ** 3
+
+
+def test_warmup_step_work_sums_every_chunk_and_layer():
+    """1.3B warmup: four chunks with 0, 3, 6, 9 frames of history, 30 layers;
+    the Gram counts every warmup row once (4 x 4680 = 18720)."""
+    w = bench.step_work(C2)
+    d, tpf = 1536, 1560
+    attn = sum(4.0 * 4680 * (1560 + 4680 + 3 * c * tpf) * d for c in range(4))
+    assert w["attention"] == pytest.approx(attn * 30)
+    assert w["gram"] == pytest.approx(4.0 * 18720 * d * d * 30)
+    assert w["solve"] == pytest.approx((1.0 / 3.0 + 4.0) * d ** 3 * 30)
+
+
+def test_absorb_roofline_is_the_sum_of_its_parts():
+    """T* per layer = Gram at the tf32 rate + solve at a third of it + error
+    reads at the HBM rate; frac = T* / measured."""
+    tf32, _ = bench.tf32_peak(1600.0)
+    d, n = C3.d, C3.warmup_rows
+    r = bench.absorb_roofline(C3, gram_ms=40 * 3.5, solve_ms=40 * 5.0, bf16_peak=1600.0,
+                              hbm_peak=6500.0)
+    t_gram = 4.0 * n * d * d / (tf32 * 1e12) * 1e3
+    t_solve = (1.0 / 3.0 + 4.0) * d ** 3 / (tf32 / 3.0 * 1e12) * 1e3
+    t_err = 6.0 * d * d * 4 / (6500.0 * 1e9) * 1e3
+    assert r["t_star_ms_per_layer"] == pytest.approx(t_gram + t_solve + t_err, abs=1e-4)
+    assert r["achieved_ms_per_layer"] == pytest.approx(8.5)
+    assert r["frac"] == pytest.approx((t_gram + t_solve + t_err) / 8.5, abs=1e-4)
+
+
+@pytest.mark.parametrize("config,layers,k", [("c2", 4, 2), ("c3", 2, 1), ("c2", 30, 15)])
+def test_layer_override_keeps_the_fraction_of_l_layers(config, layers, k):
+    args = argparse.Namespace(config=config, layers=layers)
+    cfg = bench.workload(args)
+    assert cfg.layers == layers and cfg.select_k == k
