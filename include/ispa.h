@@ -53,9 +53,11 @@ extern "C" {
 
 /* ---- device status bits (OR-ed into *dev_status) --------------------- */
 #define ISPA_STATUS_TIMEOUT 1      /* a bounded wait in a kernel gave up */
-#define ISPA_STATUS_FP16_RANGE 2   /* a V value fell outside fp16 range (|v| > 65504) */
+#define ISPA_STATUS_FP16_RANGE 2   /* a V value is not finite or beyond fp16 range (|v| > 65504) */
 #define ISPA_STATUS_NOT_SPD 4      /* G + lambda I was not positive definite */
-#define ISPA_STATUS_NONFINITE 8    /* a non-finite value reached an output */
+#define ISPA_STATUS_NONFINITE 8    /* a non-finite value reached a result: an attention row's
+                                      softmax normaliser (non-finite Q or K), or a Cholesky pivot
+                                      (non-finite G, R or lambda) */
 
 /* One branch of the KV cache: keys and values [len, heads, head_dim] bf16.
  * len may be 0 (then k and v are ignored and may be NULL). */
@@ -70,6 +72,17 @@ ISPA_API const char* ispa_status_string(int code);
 
 /* Library version as major*10000 + minor*100 + patch. */
 ISPA_API int ispa_version(void);
+
+/* Limit of every pipeline wait in the kernels launched after this call, in
+ * nanoseconds (process-wide; 0 restores the default of 2 s, larger values
+ * are clamped to it). A wait that runs past the limit gives up: the kernel
+ * sets ISPA_STATUS_TIMEOUT in the call's status word, lets the copies and
+ * tensor-core operations it already issued finish, frees its tensor memory
+ * and returns; the outputs of that call are then undefined, and the next
+ * call with the default limit runs normally. Waits normally last
+ * microseconds, so a short limit exists to exercise that path in tests.
+ * Returns ISPA_OK. */
+ISPA_API int ispa_set_wait_limit_ns(uint64_t ns);
 
 /* Number of CUDA kernels this library has launched in this process so far
  * (all devices and threads; memsets and copies not included). For
@@ -99,16 +112,37 @@ ISPA_API uint64_t ispa_kernel_launches(void);
  * a_full   out [nq, d] bf16, optional (NULL: not written).
  * lse_loc, lse_hist, lse_full: out [heads, nq] fp32, natural log, optional.
  * workspace: device scratch of >= ispa_dual_attention_workspace_size()
- *          bytes, 256-byte aligned; holds V converted to fp16 (the P.V
- *          product runs with fp16 P and fp16 V), the history branch's
- *          output and both branches' LSEs. Its contents are overwritten; it
+ *          bytes, 256-byte aligned; holds every key range's normalised
+ *          output and LSE and the per-(head, pair) completion counters (see
+ *          ispa_attention_units). The size does not depend on the split
+ *          counts chosen and never decreases as nq or hist_len grows, so a
+ *          workspace sized for the longest history serves every chunk with
+ *          the same sink and local lengths. Its contents are overwritten; it
  *          must not be used by another call in flight.
- * dev_status: device int; ISPA_STATUS_FP16_RANGE if a V value overflowed
- *          fp16, ISPA_STATUS_TIMEOUT if a kernel wait gave up.
+ * dev_status: device int; ISPA_STATUS_FP16_RANGE if a V value is not finite
+ *          or beyond fp16 range (the P.V product runs with fp16 P and V, V
+ *          converted from bf16 inside the kernel), ISPA_STATUS_NONFINITE if a
+ *          row's log-sum-exp is not finite (a non-finite q or k),
+ *          ISPA_STATUS_TIMEOUT if a kernel wait gave up.
  * Returns ISPA_OK or an ISPA_ERR_* code (nothing is launched on error).
  */
 ISPA_API size_t ispa_dual_attention_workspace_size(int64_t nq, int64_t sink_len, int64_t local_len,
                                                    int64_t hist_len, int heads, int head_dim);
+/* The unit decomposition ispa_dual_attention (and the local / full variants)
+ * use for these branch lengths: the local branch (sink, then local keys) is
+ * cut into *local_splits key ranges and the history into *hist_splits (0
+ * without a history); each range of each head and 256-row query-tile pair is
+ * one unit of work, and the last unit of a (head, pair) to finish applies the
+ * LSE merge. The counts are chosen per shape so that the units fill whole
+ * waves of the GPU's SMs. Host only, needs no device. Returns the number of
+ * units (0 on invalid sizes); either output pointer may be NULL. */
+ISPA_API int64_t ispa_attention_units(int64_t nq, int64_t sink_len, int64_t local_len,
+                                      int64_t hist_len, int heads, int* local_splits,
+                                      int* hist_splits);
+/* Forces the split counts of later attention calls (0 = automatic, the
+ * default), for measurement. Applies process-wide; query workspace sizes
+ * after changing it. Returns ISPA_OK, or ISPA_ERR_ARG for a negative count. */
+ISPA_API int ispa_attention_set_splits(int local_splits, int hist_splits);
 ISPA_API int ispa_dual_attention(const void* q, int64_t nq, int heads, int head_dim, ispa_kv sink,
                         ispa_kv local, ispa_kv hist, float scale, float* a_loc, float* d_out,
                         void* a_full, float* lse_loc, float* lse_hist, float* lse_full,
@@ -134,9 +168,9 @@ ISPA_API int ispa_local_attention(const void* q, int64_t nq, int heads, int head
  * merged by their log-sum-exps. out_bf16 [nq, d] bf16 (required); lse
  * [heads, nq] fp32 natural log of the full softmax denominator, optional.
  * workspace: >= ispa_full_attention_workspace_size() bytes, 256-byte
- * aligned (fp16 V copies, one fp32 [nq, d] output and LSE block per history
- * range, the local branch's output). Other arguments, alignment, status
- * and errors as ispa_dual_attention.
+ * aligned (one fp32 [nq, d] output and LSE block per key range, the
+ * completion counters). Other arguments, alignment, status and errors as
+ * ispa_dual_attention.
  */
 ISPA_API size_t ispa_full_attention_workspace_size(int64_t nq, int64_t sink_len, int64_t local_len,
                                                    int64_t hist_len, int heads, int head_dim);
@@ -200,9 +234,11 @@ ISPA_API int ispa_project_w8a8(const void* a_bf16, int64_t rows, int dim, const 
  * cores in tf32 (inputs are used as tf32, accumulation in fp32).
  * dim must be a multiple of 128; rows >= 0 (rows = 0 with accumulate = 0
  * zeroes the written tiles).
+ * dev_status: device int (required); ISPA_STATUS_TIMEOUT if a pipeline wait
+ * gave up (M is then incomplete).
  */
 ISPA_API int ispa_gram_accumulate(const float* a_loc, const float* d_in, int64_t rows, int dim, float* M,
-                         int accumulate, int want_s, void* stream);
+                         int accumulate, int want_s, int* dev_status, void* stream);
 
 /* ---- 3. absorb solve ---------------------------------------------------
  * Technical summary section 2, step 2 (closed form): solves
@@ -225,8 +261,10 @@ ISPA_API int ispa_gram_accumulate(const float* a_loc, const float* d_in, int64_t
  * B        out [dim, dim] fp32: R W (kept for ispa_layer_error).
  * lambda_out out, device float, optional: the lambda used.
  * workspace: >= ispa_absorb_workspace_size(dim) bytes, 256-byte aligned.
- * dev_status: ISPA_STATUS_NOT_SPD if a Cholesky pivot was not positive
- *          (dW is then undefined).
+ * dev_status: ISPA_STATUS_NOT_SPD if a Cholesky pivot was not positive,
+ *          ISPA_STATUS_NONFINITE if one was NaN or infinite (a non-finite G,
+ *          R or lambda; a non-positive pivot also makes the later ones NaN,
+ *          so NOT_SPD usually comes with NONFINITE). dW is then undefined.
  * dim must be a multiple of 128.
  */
 ISPA_API size_t ispa_absorb_workspace_size(int dim);
@@ -268,7 +306,8 @@ ISPA_API int ispa_absorb_solve_batched(int n_layers, const float* M, int64_t m_l
  * loads the library until the process exits.
  * Set-up: the first call on a device looks up the array's device address
  * (once per device, with that device current); make that first call before
- * any stream capture.
+ * any stream capture. The address is kept for the life of the process:
+ * calls after a cudaDeviceReset() are not supported.
  * Sharing: all calls use the same array, so calls that overlap on the GPU
  * (other streams, other host threads) race; serialise them. The array keeps
  * the last call's contents, which needs no clearing: each solve writes every

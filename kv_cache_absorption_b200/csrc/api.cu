@@ -42,6 +42,7 @@ cudaError_t rank_layers(const double* err, int n, int K, int* perm, uint8_t* sel
 namespace {
 
 using ispa::AttnParams;
+using ispa::cuda_rc;
 using ispa::encode_2d;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -59,36 +60,28 @@ int check_device() {
   return (major == 10 && minor == 0) ? ISPA_OK : ISPA_ERR_NO_DEVICE;
 }
 
-int cuda_rc(cudaError_t e) {
-  if (e == cudaSuccess) return ISPA_OK;
-  std::fprintf(stderr, "ispa: CUDA error %s\n", cudaGetErrorString(e));
-  return ISPA_ERR_CUDA;
-}
-
 bool kv_ok(const ispa_kv& b) {
   if (b.len < 0 || b.len > (int64_t)1 << 31) return false;
   if (b.len == 0) return true;
   return b.k && b.v && aligned16(b.k) && aligned16(b.v);
 }
 
-size_t v_half_bytes(int64_t len, int d) { return round256((size_t)len * d * 2); }
-
-// Workspace of one attention call: fp16 V of every branch, per history split
-// an fp32 output and an LSE row block, the local LSEs and, when A_loc is not
-// an output (full attention with history), the local branch's output.
+// Workspace of one attention call (see attention.cu): the per-(head, pair)
+// completion counters, an LSE block per key-range slot and an fp32 [nq, d]
+// output per slot (a call whose plan has a single local slot stores it in
+// A_loc, one with a single slot writes its outputs directly). Sized for the
+// most slots any candidate plan of these lengths may use, so that it does
+// not depend on the plan chosen and grows with nq and hist_len.
 size_t attention_workspace(int64_t nq, int64_t sink_len, int64_t local_len, int64_t hist_len,
-                           int heads, int head_dim, bool local_out_in_ws) {
+                           int heads, int head_dim) {
   if (nq < 0 || sink_len < 0 || local_len < 0 || hist_len < 0 || heads < 1 || head_dim < 1) return 0;
   const int d = heads * head_dim;
-  const int n_split = ispa::history_splits(sink_len, local_len, hist_len);
+  const size_t counters = round256((size_t)heads * ispa::attention_pairs(nq) * 4);
   const size_t lse = round256((size_t)heads * nq * 4);
   const size_t out = round256((size_t)nq * d * 4);
-  // local LSEs, then per history split an LSE block and an output (without
-  // a history, one spare LSE block keeps the layout of a single split)
-  const size_t hist = hist_len > 0 ? (size_t)n_split * (out + lse) : lse;
-  const size_t loc = (local_out_in_ws && hist_len > 0) ? out : 0;
-  return v_half_bytes(sink_len, d) + v_half_bytes(local_len, d) + v_half_bytes(hist_len, d) +
-         hist + loc + lse + 256;
+  const int slots = ispa::attention_slot_bound(sink_len, local_len, hist_len);
+  if (slots <= 1) return 256;
+  return counters + (size_t)slots * (lse + out) + 256;
 }
 
 int attention_common(const void* q, int64_t nq, int heads, int head_dim, const ispa_kv (&br)[3],
@@ -107,8 +100,9 @@ int attention_common(const void* q, int64_t nq, int heads, int head_dim, const i
       (a_full && !aligned16(a_full)))
     return ISPA_ERR_UNSUPPORTED;
   const int d = heads * head_dim;
-  const size_t need = attention_workspace(nq, br[0].len, br[1].len, br[2].len, heads, head_dim,
-                                          full_only);
+  // the local slot lives in the workspace when A_loc is not an output
+  const bool local_in_ws = full_only || a_loc == nullptr;
+  const size_t need = attention_workspace(nq, br[0].len, br[1].len, br[2].len, heads, head_dim);
   if (!workspace || workspace_bytes < need || !aligned256(workspace)) return ISPA_ERR_WORKSPACE;
   int rc = check_device();
   if (rc != ISPA_OK) return rc;
@@ -120,7 +114,6 @@ int attention_common(const void* q, int64_t nq, int heads, int head_dim, const i
   if (!encode_2d(&p.tm_q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, nq, d, 64, 128,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return ISPA_ERR_CUDA;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
   for (int b = 0; b < 3; ++b) {
     p.len[b] = br[b].len;
     if (br[b].len == 0) {  // never read: no tiles of this branch
@@ -128,40 +121,35 @@ int attention_common(const void* q, int64_t nq, int heads, int head_dim, const i
       p.tm_v[b] = p.tm_q;
       continue;
     }
-    void* vh = ws;
-    ws += v_half_bytes(br[b].len, d);
-    cudaError_t e = ispa::launch_v_to_half(br[b].v, vh, br[b].len * d, dev_status, s);
-    if (e != cudaSuccess) return cuda_rc(e);
     if (!encode_2d(&p.tm_k[b], br[b].k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, br[b].len, d, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&p.tm_v[b], vh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, br[b].len, d, 64, 128,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+        !encode_2d(&p.tm_v[b], br[b].v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, br[b].len, d, 64,
+                   128, CU_TENSOR_MAP_SWIZZLE_128B))
       return ISPA_ERR_CUDA;
   }
-  p.n_split = ispa::history_splits(br[0].len, br[1].len, br[2].len);
-  p.split_tiles = ispa::history_split_tiles(br[2].len, p.n_split);
-  const size_t out_bytes = round256((size_t)nq * d * 4);
-  const size_t lse_bytes = round256((size_t)heads * nq * 4);
-  p.hist_stride = (int64_t)(out_bytes / 4);
-  p.lse_stride = (int64_t)(lse_bytes / 4);
-  p.loc_out = a_loc;
-  if (br[2].len > 0) {
-    p.hist_out = reinterpret_cast<float*>(ws);
-    ws += (size_t)p.n_split * out_bytes;
-    if (full_only) {
-      p.loc_out = reinterpret_cast<float*>(ws);
-      ws += out_bytes;
-    }
-  }
-  p.lse_loc_ws = reinterpret_cast<float*>(ws);
-  ws += lse_bytes;
-  p.lse_hist_ws = reinterpret_cast<float*>(ws);
+  p.plan = ispa::attention_plan(nq, br[0].len, br[1].len, br[2].len, heads);
+  ispa::attention_slot_order(p.plan,
+                             ispa::attention_key_tiles(br[0].len) + ispa::attention_key_tiles(br[1].len),
+                             ispa::attention_key_tiles(br[2].len), p.order);
   p.nq = (int)nq;
   p.heads = heads;
   p.n_pairs = ispa::attention_pairs(nq);
+  const size_t out_bytes = round256((size_t)nq * d * 4);
+  const size_t lse_bytes = round256((size_t)heads * nq * 4);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (p.plan.n_slots() > 1) {
+    p.counters = reinterpret_cast<int*>(ws);
+    ws += round256((size_t)heads * p.n_pairs * 4);
+    p.part_lse = reinterpret_cast<float*>(ws);
+    ws += (size_t)p.plan.n_slots() * lse_bytes;
+    p.part = reinterpret_cast<float*>(ws);
+    p.part_first = (p.plan.n_ls == 1 && !local_in_ws) ? 1 : 0;
+    p.part_stride = (int64_t)(out_bytes / 4);
+    p.lse_stride = (int64_t)(lse_bytes / 4);
+  }
   p.scale_log2 = scale * 1.4426950408889634f;
   p.round_tf32 = full_only ? 0 : round_tf32;
-  p.a_loc = a_loc;
+  p.a_loc = full_only ? nullptr : a_loc;
   p.d_out = d_out;
   p.a_full = static_cast<__nv_bfloat16*>(a_full);
   p.lse_loc = lse_loc;
@@ -195,19 +183,42 @@ int ispa_version(void) { return 100; }
 
 uint64_t ispa_kernel_launches(void) { return ispa::g_launches.load(std::memory_order_relaxed); }
 
+int ispa_set_wait_limit_ns(uint64_t ns) {
+  ispa::set_wait_limit_ns(ns);
+  return ISPA_OK;
+}
+
+int64_t ispa_attention_units(int64_t nq, int64_t sink_len, int64_t local_len, int64_t hist_len,
+                             int heads, int* local_splits, int* hist_splits) {
+  if (nq < 0 || sink_len < 0 || local_len < 0 || hist_len < 0 || heads < 1 ||
+      sink_len + local_len < 1)
+    return 0;
+  const ispa::AttnPlan pl = ispa::attention_plan(nq, sink_len, local_len, hist_len, heads);
+  if (local_splits) *local_splits = pl.n_ls;
+  if (hist_splits) *hist_splits = pl.n_hs;
+  return (int64_t)heads * ispa::attention_pairs(nq) * pl.n_slots();
+}
+
+int ispa_attention_set_splits(int local_splits, int hist_splits) {
+  if (local_splits < 0 || hist_splits < 0) return ISPA_ERR_ARG;
+  ispa::attention_force_splits(local_splits, hist_splits);
+  return ISPA_OK;
+}
+
 size_t ispa_dual_attention_workspace_size(int64_t nq, int64_t sink_len, int64_t local_len,
                                           int64_t hist_len, int heads, int head_dim) {
-  return attention_workspace(nq, sink_len, local_len, hist_len, heads, head_dim, false);
+  return attention_workspace(nq, sink_len, local_len, hist_len, heads, head_dim);
 }
 
 size_t ispa_full_attention_workspace_size(int64_t nq, int64_t sink_len, int64_t local_len,
                                           int64_t hist_len, int heads, int head_dim) {
-  return attention_workspace(nq, sink_len, local_len, hist_len, heads, head_dim, true);
+  return attention_workspace(nq, sink_len, local_len, hist_len, heads, head_dim);
 }
 
 int ispa_full_attention(const void* q, int64_t nq, int heads, int head_dim, ispa_kv sink,
                         ispa_kv local, ispa_kv hist, float scale, void* out_bf16, float* lse,
                         void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+  ISPA_NVTX_RANGE();
   if (!out_bf16) return ISPA_ERR_ARG;
   const ispa_kv br[3] = {sink, local, hist};
   return attention_common(q, nq, heads, head_dim, br, scale, 0, nullptr, nullptr, out_bf16,
@@ -219,6 +230,7 @@ int ispa_dual_attention(const void* q, int64_t nq, int heads, int head_dim, ispa
                         ispa_kv local, ispa_kv hist, float scale, float* a_loc, float* d_out,
                         void* a_full, float* lse_loc, float* lse_hist, float* lse_full,
                         void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+  ISPA_NVTX_RANGE();
   if (!a_loc || !d_out) return ISPA_ERR_ARG;
   const ispa_kv br[3] = {sink, local, hist};
   return attention_common(q, nq, heads, head_dim, br, scale, 1, a_loc, d_out, a_full, lse_loc,
@@ -228,6 +240,7 @@ int ispa_dual_attention(const void* q, int64_t nq, int heads, int head_dim, ispa
 int ispa_local_attention(const void* q, int64_t nq, int heads, int head_dim, ispa_kv sink,
                          ispa_kv local, float scale, float* out_f32, void* out_bf16, float* lse,
                          void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+  ISPA_NVTX_RANGE();
   if (!out_f32 && !out_bf16) return ISPA_ERR_ARG;
   const ispa_kv br[3] = {sink, local, ispa_kv{nullptr, nullptr, 0}};
   return attention_common(q, nq, heads, head_dim, br, scale, 0, out_f32, nullptr, out_bf16, lse,
@@ -235,8 +248,10 @@ int ispa_local_attention(const void* q, int64_t nq, int heads, int head_dim, isp
 }
 
 int ispa_gram_accumulate(const float* a_loc, const float* d_in, int64_t rows, int dim, float* M,
-                         int accumulate, int want_s, void* stream) {
-  if (!M || rows < 0 || rows > ((int64_t)1 << 31) - 64 || dim <= 0) return ISPA_ERR_ARG;
+                         int accumulate, int want_s, int* dev_status, void* stream) {
+  ISPA_NVTX_RANGE();
+  if (!M || !dev_status || rows < 0 || rows > ((int64_t)1 << 31) - 64 || dim <= 0)
+    return ISPA_ERR_ARG;
   if (dim % 128 != 0 || dim > 32768 || !aligned16(M)) return ISPA_ERR_UNSUPPORTED;
   if (rows > 0 && (!a_loc || !d_in)) return ISPA_ERR_ARG;
   if (rows > 0 && (!aligned16(a_loc) || !aligned16(d_in))) return ISPA_ERR_UNSUPPORTED;
@@ -273,7 +288,7 @@ int ispa_gram_accumulate(const float* a_loc, const float* d_in, int64_t rows, in
   // whole tiles in waves of `grid`, then the rest split evenly (see gram.cu)
   const int64_t tail = p.total_iters - (int64_t)(p.n_tiles / grid) * grid * p.k_iters;
   p.iters_per_cta = (tail + grid - 1) / grid;
-  p.status = nullptr;
+  p.status = dev_status;
   return cuda_rc(ispa::launch_gram(p, bn, (int)grid, s));
 }
 
@@ -285,6 +300,7 @@ size_t ispa_absorb_workspace_size(int dim) {
 int ispa_absorb_solve(const float* M, const float* W, int dim, float lambda, float* dW, float* B,
                       float* lambda_out, void* workspace, size_t workspace_bytes, int* dev_status,
                       void* stream) {
+  ISPA_NVTX_RANGE();
   if (!M || !W || !dW || !B || !dev_status || dim <= 0 || lambda != lambda) return ISPA_ERR_ARG;
   if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
   if (!aligned16(M) || !aligned16(W) || !aligned16(dW) || !aligned16(B))
@@ -308,6 +324,7 @@ int ispa_absorb_solve_batched(int n_layers, const float* M, int64_t m_layer_stri
                               float* dW, int64_t dw_layer_stride, float* B,
                               int64_t b_layer_stride, float* lambda_out, void* workspace,
                               size_t workspace_bytes, int* dev_status, void* stream) {
+  ISPA_NVTX_RANGE();
   if (n_layers < 1 || n_layers > 4096 || !M || !W || !dW || !B || !dev_status || dim <= 0 ||
       lambda != lambda)
     return ISPA_ERR_ARG;
@@ -334,6 +351,7 @@ int ispa_layer_error_batched(int n_layers, const float* M, int64_t m_layer_strid
                              int64_t dw_layer_stride, const float* B, int64_t b_layer_stride,
                              const float* lambdas, int dim, double* err, void* workspace,
                              size_t workspace_bytes, void* stream) {
+  ISPA_NVTX_RANGE();
   if (n_layers < 1 || n_layers > 4096 || !M || !W || !dW || !B || !lambdas || !err || dim <= 0)
     return ISPA_ERR_ARG;
   if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
@@ -356,6 +374,7 @@ int ispa_layer_error_batched(int n_layers, const float* M, int64_t m_layer_strid
 
 int ispa_weight_gram_batched(int n_layers, const float* W, int64_t w_layer_stride, int dim,
                              float* P, int64_t p_layer_stride, int* dev_status, void* stream) {
+  ISPA_NVTX_RANGE();
   if (n_layers < 1 || n_layers > 4096 || !W || !P || !dev_status || dim <= 0) return ISPA_ERR_ARG;
   if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
   const int64_t dd = (int64_t)dim * dim;
@@ -372,6 +391,7 @@ int ispa_layer_error_wwt_batched(int n_layers, const float* M, int64_t m_layer_s
                                  int64_t dw_layer_stride, const float* B, int64_t b_layer_stride,
                                  const float* lambdas, int dim, double* err, void* workspace,
                                  size_t workspace_bytes, void* stream) {
+  ISPA_NVTX_RANGE();
   if (n_layers < 1 || n_layers > 4096 || !M || !P || !dW || !B || !lambdas || !err || dim <= 0)
     return ISPA_ERR_ARG;
   if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
@@ -393,6 +413,7 @@ int ispa_layer_error_wwt_batched(int n_layers, const float* M, int64_t m_layer_s
 }
 
 int ispa_absorbed_weight(const float* W, const float* dW, int dim, void* w_bf16, void* stream) {
+  ISPA_NVTX_RANGE();
   if (!W || !w_bf16 || dim <= 0) return ISPA_ERR_ARG;
   if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
   if (!aligned16(W) || (dW && !aligned16(dW)) || !aligned16(w_bf16)) return ISPA_ERR_UNSUPPORTED;
@@ -404,6 +425,7 @@ int ispa_absorbed_weight(const float* W, const float* dW, int dim, void* w_bf16,
 
 int ispa_project(const void* a_bf16, int64_t rows, int dim, const void* w_bf16, void* out,
                  int out_fp32, int* dev_status, void* stream) {
+  ISPA_NVTX_RANGE();
   if (!w_bf16 || !dev_status || rows < 0 || rows > ((int64_t)1 << 31) - 128 || dim <= 0)
     return ISPA_ERR_ARG;
   if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
@@ -430,6 +452,7 @@ int ispa_project(const void* a_bf16, int64_t rows, int dim, const void* w_bf16, 
 
 int ispa_quantize_weight_int8(const float* W, const float* dW, int dim, int8_t* wq_t,
                               float* w_scale, void* stream) {
+  ISPA_NVTX_RANGE();
   if (!W || !wq_t || !w_scale || dim <= 0) return ISPA_ERR_ARG;
   if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
   if (!aligned16(W) || (dW && !aligned16(dW)) || !aligned16(wq_t)) return ISPA_ERR_UNSUPPORTED;
@@ -447,6 +470,7 @@ size_t ispa_project_w8a8_workspace_size(int64_t rows, int dim) {
 int ispa_project_w8a8(const void* a_bf16, int64_t rows, int dim, const int8_t* wq_t,
                       const float* w_scale, void* out, int out_fp32, void* workspace,
                       size_t workspace_bytes, int* dev_status, void* stream) {
+  ISPA_NVTX_RANGE();
   if (!wq_t || !w_scale || !dev_status || rows < 0 || rows > ((int64_t)1 << 31) - 128 || dim <= 0)
     return ISPA_ERR_ARG;
   if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
@@ -487,6 +511,7 @@ size_t ispa_layer_error_workspace_size(int dim) { return dim > 0 ? 256 : 0; }
 int ispa_layer_error(const float* M, const float* W, const float* dW, const float* B,
                      const float* lambda, int dim, double* err, void* workspace,
                      size_t workspace_bytes, void* stream) {
+  ISPA_NVTX_RANGE();
   if (!M || !W || !dW || !B || !lambda || !err || dim <= 0) return ISPA_ERR_ARG;
   if (dim % 128 != 0 || dim > 32768) return ISPA_ERR_UNSUPPORTED;
   if (!aligned16(M) || !aligned16(W) || !aligned16(dW) || !aligned16(B))
@@ -501,6 +526,7 @@ int ispa_layer_error(const float* M, const float* W, const float* dW, const floa
 
 int ispa_rank_layers(const double* err, int n_layers, int K, int* perm, uint8_t* selected,
                      void* stream) {
+  ISPA_NVTX_RANGE();
   if (!err || !perm || n_layers < 1 || n_layers > 4096 || K < 0 || K > n_layers)
     return ISPA_ERR_ARG;
   int rc = check_device();

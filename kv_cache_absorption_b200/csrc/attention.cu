@@ -7,17 +7,28 @@
 // by splitting the keys into a local and a history branch, each run as an
 // online softmax that keeps its log-sum-exp, and merging the branches post hoc.
 //
-// That decomposition is also the work split here. A unit is one branch of
-// one head for a pair of 128-row query tiles; history units (the longer ones)
-// are scheduled first, local units fill in behind them, and a separate
-// element-wise kernel applies the LSE merge:
-//   LSE_full = log(e^LSE_loc + e^LSE_hist), w = e^(LSE_hist - LSE_full),
-//   D = w (A_hist - A_loc), A_full = A_loc + D.
+// That decomposition is also the work split here. A unit is one key range
+// (slot) of one head for a pair of 128-row query tiles: the local branch
+// (sink tiles, then the chunk's) is cut into one or more ranges, a long
+// history into several (split-KV). The host picks the split counts per shape
+// by simulating the block scheduler (longest units first, each SM taking the
+// next unit as it frees) over the candidates and keeping the shortest
+// makespan, so that warmup chunks of every history length fill whole waves.
+// Every unit writes its normalised output and LSE to its slot and bumps a
+// per-(head, pair) completion counter; the unit that finishes last reads the
+// others' slots and applies the post-hoc LSE merge in its own epilogue:
+//   LSE_loc = logsumexp over the local slots, LSE_full = logsumexp over all,
+//   A_loc = sum_local e^(LSE_s - LSE_loc) O_s,
+//   D = sum_hist e^(LSE_s - LSE_full) (O_s - A_loc), A_full = A_loc + D.
+// No unit waits for another: whichever finishes last does the merge.
 //
 // Unit CTA (384 threads), both query tiles t = 0, 1 share every K/V tile:
 //   warp 0      TMA producer: the two Q tiles, then 128-key tiles into a
-//               3-stage K ring (bf16) and a 2-stage V ring (fp16 copies).
+//               3-stage K ring and a 2-stage V ring (bf16 as stored).
 //               K(j) is released after both QK(j), V(j) after both PV(j).
+//   warps 2-3   convert each V tile in shared memory from bf16 to fp16 in
+//               place (same swizzled layout: both are 2-byte types) and flag
+//               values beyond fp16 range.
 //   warp 1      owns TMEM; one lane issues every tcgen05.mma in the order
 //               PV_0(j-1), QK_0(j), PV_1(j-1), QK_1(j): S_t = Q_t K^T (bf16,
 //               SS form) and O_t += P_t V (fp16, TS form, P_t read from TMEM
@@ -26,11 +37,22 @@
 //   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: one thread
 //               per query row; base-2 online softmax with a lazily rescaled
 //               running max; paired fp32 arithmetic (f32x2) where it applies.
+//               They also run the epilogue (slot write, counter, merge).
 // Because PV_t(j-1) is issued before QK_t(j), S_t(j) being ready means O_t is
 // quiescent, so the softmax may rescale it without another wait.
 // TMEM: S_0 [0,128), O_0 [128,128+HD), S_1 [256,384), O_1 [384,384+HD).
+#include <algorithm>
+#include <atomic>
+#include <functional>
+#include <map>
+#include <mutex>
+#include <queue>
+#include <tuple>
+#include <vector>
+
 #include "sm100.cuh"
 #include "attention.h"
+#include "host_util.h"
 
 namespace ispa {
 namespace {
@@ -55,7 +77,8 @@ struct alignas(1024) Smem {
   uint64_t q_full;
   uint64_t k_full[NK];
   uint64_t k_empty[NK];
-  uint64_t v_full[NV];
+  uint64_t v_full[NV];       // bf16 tile landed
+  uint64_t v_conv[NV];       // converted to fp16 (two converter warps arrive)
   uint64_t v_empty[NV];
   uint64_t s_full[NQT];
   uint64_t p_full[NQT][2];   // P_t keys [0,64) and [64,128) written
@@ -63,44 +86,44 @@ struct alignas(1024) Smem {
   uint64_t drain;
   uint32_t taddr;
   int abort_flag;
+  int merge;                 // this unit finished last: it merges the slots
 };
 
 struct Unit {
   int head;
+  int pair;
   int q0;          // first query row of the pair
   int n_qt;        // query tiles with rows in range (1 or 2)
+  int slot;        // key range: local range slot (< n_ls) or history range
   int hist;        // 1 = history branch, 0 = local branch (sink then local)
-  int split;       // history split (key range) of a history unit
-  int t0;          // first history key tile of the split
+  int t0;          // first key tile of the range within its branch
   int n_tiles;
 };
 
-// Units: every history split of every (head, query pair) first, then the
-// local units.
+// Grid order: for each slot in p.order (longest key range first), every
+// (head, query pair).
 __device__ __forceinline__ Unit unit_of(const AttnParams& p) {
   Unit u;
-  int b = blockIdx.x;
   const int per = p.heads * p.n_pairs;
-  const int n_hist_units = p.len[2] > 0 ? per * p.n_split : 0;
-  u.hist = b < n_hist_units ? 1 : 0;
-  if (u.hist) {
-    u.split = b / per;
-    b -= u.split * per;
-  } else {
-    u.split = 0;
-    b -= n_hist_units;
-  }
+  const int b = blockIdx.x % per;
+  u.slot = p.order[blockIdx.x / per];
   u.head = b / p.n_pairs;
-  u.q0 = (b % p.n_pairs) * (BM * NQT);
+  u.pair = b % p.n_pairs;
+  u.q0 = u.pair * (BM * NQT);
   u.n_qt = (p.nq - u.q0 > BM) ? 2 : 1;
+  u.hist = u.slot >= p.plan.n_ls ? 1 : 0;
+  int total, per_range, k;
   if (u.hist) {
-    const int total = (int)((p.len[2] + BN - 1) / BN);
-    u.t0 = u.split * p.split_tiles;
-    u.n_tiles = total - u.t0 < p.split_tiles ? total - u.t0 : p.split_tiles;
+    total = (int)((p.len[2] + BN - 1) / BN);
+    per_range = p.plan.hs_tiles;
+    k = u.slot - p.plan.n_ls;
   } else {
-    u.t0 = 0;
-    u.n_tiles = (int)((p.len[0] + BN - 1) / BN) + (int)((p.len[1] + BN - 1) / BN);
+    total = (int)((p.len[0] + BN - 1) / BN) + (int)((p.len[1] + BN - 1) / BN);
+    per_range = p.plan.ls_tiles;
+    k = u.slot;
   }
+  u.t0 = k * per_range;
+  u.n_tiles = total - u.t0 < per_range ? total - u.t0 : per_range;
   return u;
 }
 
@@ -131,10 +154,44 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* 
   mbar_wait(bar, parity, status, &dummy);
 }
 
-__device__ __forceinline__ void store_f32x32(float* dst, const float (&v)[32], bool tf32) {
+// Named barrier over the epilogue threads; returns whether every thread
+// passed `pred` true.
+__device__ __forceinline__ bool epi_barrier_and(int nthreads, bool pred) {
+  uint32_t in = pred ? 1u : 0u, out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.and.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out) : "r"(in), "r"(nthreads) : "memory");
+  return out != 0;
+}
+__device__ __forceinline__ void epi_barrier(int nthreads) {
+  asm volatile("barrier.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+// Generic-proxy shared-memory writes become visible to the async proxy
+// (the tensor core reading the converted V tile).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// 16 consecutive fp32 values: stores (optionally rounded to tf32), loads
+// that bypass L1 (slots written by other SMs in this launch).
+__device__ __forceinline__ void store_f32x16(float* dst, const float (&v)[16], bool tf32) {
   float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < 4; ++i) {
     float4 x;
     x.x = tf32 ? to_tf32(v[4 * i]) : v[4 * i];
     x.y = tf32 ? to_tf32(v[4 * i + 1]) : v[4 * i + 1];
@@ -143,11 +200,18 @@ __device__ __forceinline__ void store_f32x32(float* dst, const float (&v)[32], b
     d4[i] = x;
   }
 }
-
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
+__device__ __forceinline__ void load_f32x16(const float* src, float (&v)[16]) {
+  const float4* s4 = reinterpret_cast<const float4*>(src);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
+    const float4 x = __ldcg(s4 + i);
+    v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
+  }
+}
+__device__ __forceinline__ void store_bf16x16(__nv_bfloat16* dst, const float (&v)[16]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
     uint32_t w[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -156,6 +220,35 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&
     }
     d4[i] = make_uint4(w[0], w[1], w[2], w[3]);
   }
+}
+
+__device__ __forceinline__ bool finite_f(float x) { return fabsf(x) <= 3.402823466e38f; }
+
+__device__ __forceinline__ float log_add_exp(float x, float y) {
+  const float hi = fmaxf(x, y), lo = fminf(x, y);
+  return hi == -INFINITY ? hi : hi + log1pf(expf(lo - hi));
+}
+
+// Where slot k's normalised output lives: slot 0 in a_loc itself when the
+// plan says so (stored rounded like the final A_loc), else the workspace.
+__device__ __forceinline__ float* slot_out(const AttnParams& p, int k) {
+  return k < p.part_first ? p.a_loc : p.part + (int64_t)(k - p.part_first) * p.part_stride;
+}
+
+// bf16 -> fp16 of one 16-byte chunk (8 values); `big` collects |v| >= 2^16
+// (the bf16 values that overflow fp16) as a per-half maximum.
+__device__ __forceinline__ uint4 bf16x8_to_half(uint4 x, uint32_t& big) {
+  uint32_t in[4] = {x.x, x.y, x.z, x.w}, out[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float lo = __uint_as_float(in[k] << 16);
+    const float hi = __uint_as_float(in[k] & 0xFFFF0000u);
+    out[k] = pack_half2(lo, hi);
+    uint32_t m;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(m) : "r"(big), "r"(in[k] & 0x7FFF7FFFu));
+    big = m;
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 template <int HD>
@@ -173,7 +266,11 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
   if (threadIdx.x == 0) {
     mbar_init(&s.q_full, 1);
     for (int i = 0; i < NK; ++i) { mbar_init(&s.k_full[i], 1); mbar_init(&s.k_empty[i], 1); }
-    for (int i = 0; i < NV; ++i) { mbar_init(&s.v_full[i], 1); mbar_init(&s.v_empty[i], 1); }
+    for (int i = 0; i < NV; ++i) {
+      mbar_init(&s.v_full[i], 1);
+      mbar_init(&s.v_conv[i], 2);
+      mbar_init(&s.v_empty[i], 1);
+    }
     for (int i = 0; i < NQT; ++i) {
       mbar_init(&s.s_full[i], 1);
       mbar_init(&s.p_full[i][0], 128);
@@ -182,6 +279,7 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
     mbar_init(&s.o_final, 1);
     mbar_init(&s.drain, 1);
     s.abort_flag = 0;
+    s.merge = 0;
     fence_mbar_init();
   }
   if (warp == 1) { tmem_alloc(&s.taddr, kTmemCols); tmem_relinquish(); }
@@ -205,25 +303,46 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
       for (int j = 0; j < n_tiles; ++j) {
         const TileInfo ti = tile_of(u.t0 + j, u.hist, p);
         const int sk = j % NK, sv = j % NV;
-        if (j >= NK && !mbar_wait(&s.k_empty[sk], ((j / NK) - 1) & 1, p.status, abort_flag)) break;
+        if (j >= NK && !mbar_wait(&s.k_empty[sk], ((j / NK) - 1) & 1, p.status, abort_flag, p.wait_ns)) break;
         mbar_expect_tx(&s.k_full[sk], (HD / 64) * BN * 128);
         for (int b = 0; b < HD / 64; ++b)
           tma_load_2d(s.k[sk][b], &p.tm_k[ti.branch], &s.k_full[sk], u.head * HD + b * 64, ti.row0);
         k_issued = j + 1;
-        if (j >= NV && !mbar_wait(&s.v_empty[sv], ((j / NV) - 1) & 1, p.status, abort_flag)) break;
+        if (j >= NV && !mbar_wait(&s.v_empty[sv], ((j / NV) - 1) & 1, p.status, abort_flag, p.wait_ns)) break;
         mbar_expect_tx(&s.v_full[sv], (HD / 64) * BN * 128);
         for (int b = 0; b < HD / 64; ++b)
           tma_load_2d(s.v[sv][b], &p.tm_v[ti.branch], &s.v_full[sv], u.head * HD + b * 64, ti.row0);
         v_issued = j + 1;
       }
-      if (*abort_flag) {  // let copies still in flight land before the CTA exits
-        drain_wait(&s.q_full, 0, p.status);
-        for (int j = k_issued - NK < 0 ? 0 : k_issued - NK; j < k_issued; ++j)
-          drain_wait(&s.k_full[j % NK], (j / NK) & 1, p.status);
-        for (int j = v_issued - NV < 0 ? 0 : v_issued - NV; j < v_issued; ++j)
-          drain_wait(&s.v_full[j % NV], (j / NV) & 1, p.status);
-      }
+      // Every copy issued has landed before the CTA exits, whether or not a
+      // consumer gave up (the latest phase of each stage; at once when none did).
+      drain_wait(&s.q_full, 0, p.status);
+      for (int j = k_issued - NK < 0 ? 0 : k_issued - NK; j < k_issued; ++j)
+        drain_wait(&s.k_full[j % NK], (j / NK) & 1, p.status);
+      for (int j = v_issued - NV < 0 ? 0 : v_issued - NV; j < v_issued; ++j)
+        drain_wait(&s.v_full[j % NV], (j / NV) & 1, p.status);
     }
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ V converters
+    // Tile j is converted after it lands and before its P.V; the slot is not
+    // reloaded until that P.V has retired (v_empty), so conversion and the
+    // next copy into the slot never overlap.
+    const int ct = threadIdx.x - 64;
+    constexpr int kChunks = (HD / 64) * BN * 128 / 16;
+    uint32_t big = 0;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int sv = j % NV;
+      if (!mbar_wait_warp(&s.v_full[sv], (j / NV) & 1, p.status, abort_flag, p.wait_ns)) break;
+      uint4* buf = reinterpret_cast<uint4*>(&s.v[sv][0][0]);
+#pragma unroll 4
+      for (int i = ct; i < kChunks; i += 64) buf[i] = bf16x8_to_half(buf[i], big);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.v_conv[sv]);
+    }
+    // bf16 magnitudes >= 2^16 (0x4780) do not fit fp16 (largest finite 65504)
+    const bool bad = (big & 0xFFFFu) >= 0x4780u || (big >> 16) >= 0x4780u;
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.status, ISPA_STATUS_FP16_RANGE);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -235,12 +354,12 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
       for (int t = 0; t < NQT; ++t) dq[t] = smem_desc(smem_u32(s.q[t][0]), 16, 1024);
       for (int i = 0; i < NK; ++i) dk[i] = smem_desc(smem_u32(s.k[i][0]), 16, 1024);
       for (int i = 0; i < NV; ++i) dv[i] = smem_desc(smem_u32(s.v[i][0]), BN * 128, 1024);
-      bool ok = mbar_wait(&s.q_full, 0, p.status, abort_flag);
+      bool ok = mbar_wait(&s.q_full, 0, p.status, abort_flag, p.wait_ns);
       for (int j = 0; ok && j <= n_tiles; ++j) {
         for (int t = 0; ok && t < u.n_qt; ++t) {
           if (j > 0) {   // O_t += P_t(j-1) V(j-1), one 64-key half at a time
             const int sv = (j - 1) % NV;
-            if (t == 0 && !mbar_wait(&s.v_full[sv], ((j - 1) / NV) & 1, p.status, abort_flag)) {
+            if (t == 0 && !mbar_wait(&s.v_conv[sv], ((j - 1) / NV) & 1, p.status, abort_flag, p.wait_ns)) {
               ok = false;
               break;
             }
@@ -248,7 +367,7 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
             const uint32_t ao = t_s(t), oo = t_o(t);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              if (!mbar_wait(&s.p_full[t][h], (j - 1) & 1, p.status, abort_flag)) { ok = false; break; }
+              if (!mbar_wait(&s.p_full[t][h], (j - 1) & 1, p.status, abort_flag, p.wait_ns)) { ok = false; break; }
               tc_fence_after();
 #pragma unroll
               for (int kk = h * 4; kk < h * 4 + 4; ++kk)
@@ -260,7 +379,7 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
           }
           if (j < n_tiles) {   // S_t = Q_t K(j)^T
             const int sk = j % NK;
-            if (t == 0 && !mbar_wait(&s.k_full[sk], (j / NK) & 1, p.status, abort_flag)) {
+            if (t == 0 && !mbar_wait(&s.k_full[sk], (j / NK) & 1, p.status, abort_flag, p.wait_ns)) {
               ok = false;
               break;
             }
@@ -279,10 +398,10 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
         }
       }
       if (ok) tc_commit(&s.o_final);
-      if (!ok) {  // let issued MMAs finish before TMEM is freed
-        tc_commit(&s.drain);
-        drain_wait(&s.drain, 0, p.status);
-      }
+      // every MMA issued has finished before TMEM is freed, also when a
+      // softmax warp gave up on o_final while the last ones still ran
+      tc_commit(&s.drain);
+      drain_wait(&s.drain, 0, p.status);
     }
     __syncwarp();
   } else if (warp >= 4 && (warp - 4) / 4 < u.n_qt) {
@@ -297,7 +416,7 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       const TileInfo ti = tile_of(u.t0 + j, u.hist, p);
-      if (!mbar_wait(&s.s_full[t], j & 1, p.status, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(&s.s_full[t], j & 1, p.status, abort_flag, p.wait_ns)) { ok = false; break; }
       tc_fence_after();
       float sv[BN];
 #pragma unroll
@@ -365,123 +484,160 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
       l += (rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y);
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && mbar_wait(&s.o_final, 0, p.status, abort_flag)) {
+    const int n_epi = 128 * u.n_qt;
+    ok = ok && mbar_wait(&s.o_final, 0, p.status, abort_flag, p.wait_ns);   // per thread: agreed below
+    if (epi_barrier_and(n_epi, ok)) {
       tc_fence_after();
       const int row = u.q0 + t * BM + r;
       const bool row_ok = row < p.nq;
       const int64_t d = (int64_t)p.heads * HD;
       const int64_t base = (int64_t)row * d + (int64_t)u.head * HD;
+      const int64_t li = (int64_t)u.head * p.nq + row;
       const float lse = (m + log2f(l)) * kLn2;
       const float inv = 1.f / l;
-      const bool direct = !u.hist && p.len[2] == 0;   // no history: write the final outputs
+      const int n_slots = p.plan.n_slots();
+      bool nonfinite = false;
+      if (n_slots == 1) {
+        // one local range and no history: write the final outputs directly
 #pragma unroll 1
-      for (int c = 0; c < HD / 32; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(to + c * 32, raw);
-        tmem_ld_wait();
-        if (!row_ok) continue;
-        float a[32];
+        for (int c = 0; c < HD / 16; ++c) {
+          uint32_t raw[16];
+          tmem_ld16(to + c * 16, raw);
+          tmem_ld_wait();
+          if (!row_ok) continue;
+          float a[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(raw[i]) * inv;
-        if (u.hist) {
-          store_f32x32(p.hist_out + u.split * p.hist_stride + base + c * 32, a, false);
-        } else {
-          if (p.loc_out) store_f32x32(p.loc_out + base + c * 32, a, p.round_tf32 != 0);
-          if (direct && p.a_full) store_bf16x32(p.a_full + base + c * 32, a);
-          if (direct && p.d_out) {
-            float z[32];
+          for (int i = 0; i < 16; ++i) a[i] = __uint_as_float(raw[i]) * inv;
+          if (p.a_loc) store_f32x16(p.a_loc + base + c * 16, a, p.round_tf32 != 0);
+          if (p.a_full) store_bf16x16(p.a_full + base + c * 16, a);
+          if (p.d_out) {
+            float z[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) z[i] = 0.f;
-            store_f32x32(p.d_out + base + c * 32, z, false);
+            for (int i = 0; i < 16; ++i) z[i] = 0.f;
+            store_f32x16(p.d_out + base + c * 16, z, false);
           }
         }
-      }
-      if (row_ok) {
-        const int64_t li = (int64_t)u.head * p.nq + row;
-        if (u.hist) {
-          p.lse_hist_ws[u.split * p.lse_stride + li] = lse;
-        } else {
-          p.lse_loc_ws[li] = lse;
-          if (direct) {
-            if (p.lse_loc) p.lse_loc[li] = lse;
-            if (p.lse_hist) p.lse_hist[li] = -INFINITY;
-            if (p.lse_full) p.lse_full[li] = lse;
+        if (row_ok) {
+          if (p.lse_loc) p.lse_loc[li] = lse;
+          if (p.lse_hist) p.lse_hist[li] = -INFINITY;
+          if (p.lse_full) p.lse_full[li] = lse;
+        }
+        // a finite LSE bounds every output of the row (softmax averages of V)
+        nonfinite = row_ok && !finite_f(lse);
+      } else {
+        // 1. this unit's slot: normalised output and LSE
+        const bool own_rnd = u.slot < p.part_first && p.round_tf32 != 0;
+        float* own = slot_out(p, u.slot);
+#pragma unroll 1
+        for (int c = 0; c < HD / 16; ++c) {
+          uint32_t raw[16];
+          tmem_ld16(to + c * 16, raw);
+          tmem_ld_wait();
+          if (!row_ok) continue;
+          float a[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) a[i] = __uint_as_float(raw[i]) * inv;
+          store_f32x16(own + base + c * 16, a, own_rnd);
+        }
+        if (row_ok) p.part_lse[u.slot * p.lse_stride + li] = lse;
+        // 2. count this unit finished; the last of the (head, pair) merges
+        __threadfence();
+        epi_barrier(n_epi);
+        if (threadIdx.x == 128) {
+          const int done = atomicAdd(&p.counters[u.head * p.n_pairs + u.pair], 1);
+          s.merge = (done == n_slots - 1) ? 1 : 0;
+          __threadfence();
+        }
+        epi_barrier(n_epi);
+        if (s.merge) {
+          __threadfence();
+          const int n_ls = p.plan.n_ls;
+          float lse_loc = -INFINITY, lse_hist = -INFINITY;
+          if (row_ok) {
+            for (int k = 0; k < n_slots; ++k) {
+              const float v = __ldcg(p.part_lse + k * p.lse_stride + li);
+              if (k < n_ls) lse_loc = log_add_exp(lse_loc, v);
+              else lse_hist = log_add_exp(lse_hist, v);
+            }
           }
+          const float lse_full = log_add_exp(lse_loc, lse_hist);
+          const bool rnd = p.round_tf32 != 0;
+#pragma unroll 1
+          for (int c = 0; c < HD / 16; ++c) {
+            uint32_t raw[16];
+            tmem_ld16(to + c * 16, raw);
+            tmem_ld_wait();
+            if (!row_ok) continue;
+            float mine[16], al[16], dd[16], x[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              mine[i] = __uint_as_float(raw[i]) * inv;
+              if (own_rnd) mine[i] = to_tf32(mine[i]);   // exactly what the slot holds
+            }
+            const int64_t off = base + c * 16;
+            // A_loc: the local slots merged (a single local slot as stored)
+            if (n_ls == 1) {
+              if (u.slot == 0) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) al[i] = mine[i];
+              } else {
+                load_f32x16(slot_out(p, 0) + off, al);
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) al[i] = 0.f;
+              for (int k = 0; k < n_ls; ++k) {
+                const float w = expf(__ldcg(p.part_lse + k * p.lse_stride + li) - lse_loc);
+                if (k == u.slot) {
+#pragma unroll
+                  for (int i = 0; i < 16; ++i) x[i] = mine[i];
+                } else {
+                  load_f32x16(slot_out(p, k) + off, x);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) al[i] = fmaf(w, x[i], al[i]);
+              }
+              if (rnd) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) al[i] = to_tf32(al[i]);
+              }
+              if (p.a_loc) store_f32x16(p.a_loc + off, al, false);
+            }
+            // D = A_full - A_loc = sum over history slots of w (O - A_loc)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) dd[i] = 0.f;
+            for (int k = n_ls; k < n_slots; ++k) {
+              const float w = expf(__ldcg(p.part_lse + k * p.lse_stride + li) - lse_full);
+              if (k == u.slot) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) x[i] = mine[i];
+              } else {
+                load_f32x16(slot_out(p, k) + off, x);
+              }
+#pragma unroll
+              for (int i = 0; i < 16; ++i) dd[i] = fmaf(w, x[i] - al[i], dd[i]);
+            }
+            if (p.d_out) store_f32x16(p.d_out + off, dd, rnd);
+            if (p.a_full) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) x[i] = al[i] + dd[i];
+              store_bf16x16(p.a_full + off, x);
+            }
+          }
+          if (row_ok) {
+            if (p.lse_loc) p.lse_loc[li] = lse_loc;
+            if (p.lse_hist) p.lse_hist[li] = lse_hist;
+            if (p.lse_full) p.lse_full[li] = lse_full;
+          }
+          nonfinite = row_ok && !finite_f(lse_full);
         }
       }
+      if (__any_sync(0xffffffffu, nonfinite) && lane == 0) atomicOr(p.status, ISPA_STATUS_NONFINITE);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tbase, kTmemCols);
-}
-
-// Post-hoc LSE merge of the local branch and the history splits (element-
-// wise, 4 columns a thread): with w_b = exp(LSE_b - LSE_full), A_full =
-// sum_b w_b O_b and D = A_full - A_loc = sum_s w_s (O_s - A_loc).
-__device__ __forceinline__ float log_add_exp(float x, float y) {
-  const float hi = fmaxf(x, y), lo = fminf(x, y);
-  return hi == -INFINITY ? hi : hi + log1pf(expf(lo - hi));
-}
-
-__global__ void lse_merge_kernel(const AttnParams p, int hd) {
-  const int64_t d = (int64_t)p.heads * hd;
-  const int64_t n4 = (int64_t)p.nq * d / 4;
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n4;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = (e * 4) / d;
-    const int head = (int)(((e * 4) % d) / hd);
-    const int64_t li = (int64_t)head * p.nq + row;
-    const float ll = p.lse_loc_ws[li];
-    float lh = -INFINITY;
-    for (int sp = 0; sp < p.n_split; ++sp) lh = log_add_exp(lh, p.lse_hist_ws[sp * p.lse_stride + li]);
-    const float lf = log_add_exp(ll, lh);
-    const float4 a = reinterpret_cast<const float4*>(p.loc_out)[e];
-    float4 dd = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sp = 0; sp < p.n_split; ++sp) {
-      const float w = expf(p.lse_hist_ws[sp * p.lse_stride + li] - lf);
-      const float4 h = reinterpret_cast<const float4*>(p.hist_out + sp * p.hist_stride)[e];
-      dd.x += w * (h.x - a.x);
-      dd.y += w * (h.y - a.y);
-      dd.z += w * (h.z - a.z);
-      dd.w += w * (h.w - a.w);
-    }
-    if (p.d_out)
-      reinterpret_cast<float4*>(p.d_out)[e] =
-          make_float4(to_tf32(dd.x), to_tf32(dd.y), to_tf32(dd.z), to_tf32(dd.w));
-    if (p.a_full) {
-      __nv_bfloat162 b0 = __floats2bfloat162_rn(a.x + dd.x, a.y + dd.y);
-      __nv_bfloat162 b1 = __floats2bfloat162_rn(a.z + dd.z, a.w + dd.w);
-      reinterpret_cast<uint2*>(p.a_full)[e] =
-          make_uint2(*reinterpret_cast<uint32_t*>(&b0), *reinterpret_cast<uint32_t*>(&b1));
-    }
-    if (((e * 4) % hd) == 0) {   // one thread per (row, head) writes the LSEs
-      if (p.lse_loc) p.lse_loc[li] = ll;
-      if (p.lse_hist) p.lse_hist[li] = lh;
-      if (p.lse_full) p.lse_full[li] = lf;
-    }
-  }
-}
-
-// bf16 -> fp16 copy of the value tensors (the P.V product runs in fp16);
-// flags values outside fp16 range.
-__global__ void v_to_half_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int64_t n8,
-                                 int* status) {
-  int bad = 0;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    uint4 x = src[i];
-    uint32_t in[4] = {x.x, x.y, x.z, x.w}, out[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float lo = __uint_as_float(in[k] << 16);
-      const float hi = __uint_as_float(in[k] & 0xFFFF0000u);
-      bad |= (fabsf(lo) > 65504.f) | (fabsf(hi) > 65504.f);
-      out[k] = pack_half2(lo, hi);
-    }
-    dst[i] = make_uint4(out[0], out[1], out[2], out[3]);
-  }
-  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, ISPA_STATUS_FP16_RANGE);
 }
 
 }  // namespace
@@ -493,40 +649,170 @@ size_t attention_smem_bytes(int head_dim) {
   return need < 120 * 1024 ? 120 * 1024 : need;
 }
 
-cudaError_t launch_v_to_half(const void* src, void* dst, int64_t n_elems, int* status,
-                             cudaStream_t stream) {
-  if (n_elems == 0) return cudaSuccess;
-  const int64_t n8 = n_elems / 8;
-  int blocks = (int)((n8 + 255) / 256);
-  if (blocks > 148 * 8) blocks = 148 * 8;
-  v_to_half_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4*>(src),
-                                               static_cast<uint4*>(dst), n8, status);
-  count_launches();
-  return cudaGetLastError();
-}
-
 int attention_pairs(int64_t nq) { return (int)((nq + BM * NQT - 1) / (BM * NQT)); }
 
-int history_splits(int64_t sink_len, int64_t local_len, int64_t hist_len) {
-  if (hist_len <= 0) return 1;
-  const int64_t loc_tiles = (sink_len + BN - 1) / BN + (local_len + BN - 1) / BN;
-  const int64_t hist_tiles = (hist_len + BN - 1) / BN;
+int64_t attention_key_tiles(int64_t len) { return (len + BN - 1) / BN; }
+
+// ---------------------------------------------------------------- planning
+//
+// Split counts are chosen per shape by simulating the hardware block
+// scheduler on the units: blocks start in grid order (longest key range
+// first), each on the SM that frees first; a unit costs its key tiles plus a
+// fixed per-unit cost (prologue, epilogue, merge). Candidates: the local
+// branch in 1..4 ranges; the history (when present) in n0, n0 + 1, n0 + 2
+// ranges, n0 being about two local branches of keys per range (at most 64).
+// The fewest units win unless more splits shorten the makespan by > 1%.
+
+namespace {
+
+constexpr double kUnitCost = 2.0;   // key-tile steps
+constexpr int kPlanSms = 148;
+
+std::atomic<int> g_force_ls{0}, g_force_hs{0};
+
+int ranges_of(int64_t tiles, int n, int* per) {
+  if (tiles <= 0) { *per = 0; return 0; }
+  if (n > tiles) n = (int)tiles;
+  if (n < 1) n = 1;
+  *per = (int)((tiles + n - 1) / n);
+  return (int)((tiles + *per - 1) / *per);   // recount: no empty range
+}
+
+void slot_lengths(const AttnPlan& pl, int64_t loc_tiles, int64_t hist_tiles, int* len) {
+  for (int k = 0; k < pl.n_ls; ++k) {
+    const int64_t rem = loc_tiles - (int64_t)k * pl.ls_tiles;
+    len[k] = (int)(rem < pl.ls_tiles ? rem : pl.ls_tiles);
+  }
+  for (int k = 0; k < pl.n_hs; ++k) {
+    const int64_t rem = hist_tiles - (int64_t)k * pl.hs_tiles;
+    len[pl.n_ls + k] = (int)(rem < pl.hs_tiles ? rem : pl.hs_tiles);
+  }
+}
+
+double simulate(const AttnPlan& pl, int64_t loc_tiles, int64_t hist_tiles, int per) {
+  int len[kMaxSlots];
+  uint8_t order[kMaxSlots];
+  slot_lengths(pl, loc_tiles, hist_tiles, len);
+  attention_slot_order(pl, loc_tiles, hist_tiles, order);
+  std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
+  for (int i = 0; i < kPlanSms; ++i) free_at.push(0.0);
+  double end = 0.0;
+  for (int o = 0; o < pl.n_slots(); ++o) {
+    const double cost = len[order[o]] + kUnitCost;
+    for (int b = 0; b < per; ++b) {
+      const double t = free_at.top() + cost;
+      free_at.pop();
+      free_at.push(t);
+      if (t > end) end = t;
+    }
+  }
+  return end;
+}
+
+struct PlanKey {
+  int64_t pairs, loc_tiles, hist_tiles;
+  int heads, fls, fhs;
+  bool operator<(const PlanKey& o) const {
+    return std::tie(pairs, loc_tiles, hist_tiles, heads, fls, fhs) <
+           std::tie(o.pairs, o.loc_tiles, o.hist_tiles, o.heads, o.fls, o.fhs);
+  }
+};
+
+}  // namespace
+
+void attention_force_splits(int local_splits, int hist_splits) {
+  g_force_ls.store(local_splits < 0 ? 0 : local_splits);
+  g_force_hs.store(hist_splits < 0 ? 0 : hist_splits);
+}
+
+void attention_slot_order(const AttnPlan& pl, int64_t loc_tiles, int64_t hist_tiles,
+                          uint8_t* order) {
+  int len[kMaxSlots];
+  slot_lengths(pl, loc_tiles, hist_tiles, len);
+  const int n = pl.n_slots();
+  for (int k = 0; k < n; ++k) order[k] = (uint8_t)k;
+  // longest first; equal lengths keep slot order (local ranges first)
+  std::stable_sort(order, order + n, [&](uint8_t a, uint8_t b) { return len[a] > len[b]; });
+}
+
+namespace {
+// History ranges of about two local branches each (at most 64).
+int base_hist_ranges(int64_t loc_tiles, int64_t hist_tiles) {
+  if (hist_tiles <= 0) return 0;
   if (hist_tiles <= 3 * loc_tiles) return 1;
-  int64_t n = (hist_tiles + 2 * loc_tiles - 1) / (2 * loc_tiles);
-  if (n > 64) n = 64;
-  // equal splits of ceil(T / n) tiles; recount so that no split is empty
-  const int64_t per = (hist_tiles + n - 1) / n;
-  return (int)((hist_tiles + per - 1) / per);
+  const int64_t n = (hist_tiles + 2 * loc_tiles - 1) / (2 * loc_tiles);
+  return (int)(n > 64 ? 64 : n);
+}
+constexpr int kMaxLocalRanges = 4;
+constexpr int kExtraHistRanges = 2;
+}  // namespace
+
+int attention_slot_bound(int64_t sink_len, int64_t local_len, int64_t hist_len) {
+  const int64_t loc_tiles = attention_key_tiles(sink_len) + attention_key_tiles(local_len);
+  const int64_t hist_tiles = attention_key_tiles(hist_len);
+  const int fls = g_force_ls.load(), fhs = g_force_hs.load();
+  int64_t ls = fls > kMaxLocalRanges ? fls : kMaxLocalRanges;
+  if (ls > loc_tiles) ls = loc_tiles;
+  int64_t hs = 0;
+  if (hist_tiles > 0) {
+    hs = base_hist_ranges(loc_tiles, hist_tiles) + kExtraHistRanges;
+    if (fhs > hs) hs = fhs;
+    if (hs > hist_tiles) hs = hist_tiles;
+  }
+  const int64_t n = ls + hs;
+  return (int)(n > kMaxSlots ? kMaxSlots : n);
 }
 
-int history_split_tiles(int64_t hist_len, int n_split) {
-  const int64_t hist_tiles = (hist_len + BN - 1) / BN;
-  return (int)((hist_tiles + n_split - 1) / n_split);
+AttnPlan attention_plan(int64_t nq, int64_t sink_len, int64_t local_len, int64_t hist_len,
+                        int heads) {
+  const int64_t loc_tiles = attention_key_tiles(sink_len) + attention_key_tiles(local_len);
+  const int64_t hist_tiles = attention_key_tiles(hist_len);
+  const int pairs = attention_pairs(nq);
+  const PlanKey key{pairs, loc_tiles, hist_tiles, heads, g_force_ls.load(), g_force_hs.load()};
+  static std::mutex mu;
+  static std::map<PlanKey, AttnPlan> cache;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  const int hs0 = base_hist_ranges(loc_tiles, hist_tiles);
+  const int per = heads * pairs;
+  AttnPlan best{};
+  double best_t = 0.0;
+  bool have = false;
+  const int ls_lo = key.fls ? key.fls : 1, ls_hi = key.fls ? key.fls : kMaxLocalRanges;
+  const int hs_lo = hist_tiles == 0 ? 0 : (key.fhs ? key.fhs : hs0);
+  const int hs_hi = hist_tiles == 0 ? 0 : (key.fhs ? key.fhs : hs0 + kExtraHistRanges);
+  for (int hs = hs_lo; hs <= hs_hi; ++hs) {
+    for (int ls = ls_lo; ls <= ls_hi; ++ls) {
+      AttnPlan pl{};
+      pl.n_ls = ranges_of(loc_tiles, ls, &pl.ls_tiles);
+      pl.n_hs = ranges_of(hist_tiles, hs, &pl.hs_tiles);
+      if (pl.n_slots() > kMaxSlots) continue;   // also bounds the workspace query
+      const double t = simulate(pl, loc_tiles, hist_tiles, per);
+      const bool fewer = have && pl.n_slots() < best.n_slots();
+      if (!have || (fewer ? t <= best_t * 1.01 : t < best_t * 0.99)) {
+        best = pl;
+        best_t = t;
+        have = true;
+      }
+    }
+  }
+  std::lock_guard<std::mutex> g(mu);
+  cache[key] = best;
+  return best;
 }
 
-cudaError_t launch_dual_attention(const AttnParams& p, int head_dim, cudaStream_t stream) {
-  const int units = p.heads * p.n_pairs * (p.len[2] > 0 ? p.n_split + 1 : 1);
+cudaError_t launch_dual_attention(const AttnParams& p0, int head_dim, cudaStream_t stream) {
+  AttnParams p = p0;
+  p.wait_ns = wait_limit_ns();
+  const int units = p.heads * p.n_pairs * p.plan.n_slots();
   const size_t smem = attention_smem_bytes(head_dim);
+  if (p.plan.n_slots() > 1) {
+    cudaError_t e = cudaMemsetAsync(p.counters, 0, sizeof(int) * p.heads * p.n_pairs, stream);
+    if (e != cudaSuccess) return e;
+  }
   if (head_dim == 64) {
     cudaFuncSetAttribute(branch_attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
@@ -536,13 +822,6 @@ cudaError_t launch_dual_attention(const AttnParams& p, int head_dim, cudaStream_
                          (int)smem);
     branch_attention_kernel<128><<<units, kThreads, smem, stream>>>(p);
   }
-  count_launches();
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || p.len[2] == 0) return e;
-  const int64_t n4 = (int64_t)p.nq * p.heads * head_dim / 4;
-  int blocks = (int)((n4 + 255) / 256);
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  lse_merge_kernel<<<blocks, 256, 0, stream>>>(p, head_dim);
   count_launches();
   return cudaGetLastError();
 }

@@ -11,9 +11,23 @@ namespace ispa {
 // Kernel launches made by the library (read by ispa_kernel_launches).
 void count_launches(unsigned n = 1);
 
+// Most key-range units (slots) one query-tile pair of one head is cut into.
+constexpr int kMaxSlots = 72;
+
+// How one attention call is cut into units of work. A unit is one key range
+// (slot) of one head for a pair of 128-row query tiles: the local branch
+// (sink tiles, then the current chunk's) is cut into n_ls ranges of ls_tiles
+// 128-key tiles, the history into n_hs ranges of hs_tiles (n_hs = 0 without
+// a history). Slot k < n_ls is local range k, slot n_ls + k history range k.
+struct AttnPlan {
+  int n_ls, ls_tiles;
+  int n_hs, hs_tiles;
+  __host__ __device__ int n_slots() const { return n_ls + n_hs; }
+};
+
 // Parameters of one dual-stream attention launch. Tensor maps address
-// [len, heads * head_dim] row-major matrices in 64-column x 128-row boxes
-// with 128-byte swizzle: Q and K in bf16, V in fp16 (converted copies).
+// [len, heads * head_dim] bf16 row-major matrices in 64-column x 128-row
+// boxes with 128-byte swizzle.
 struct AttnParams {
   CUtensorMap tm_q;
   CUtensorMap tm_k[3];    // sink, local, history
@@ -24,34 +38,43 @@ struct AttnParams {
   int n_pairs;            // ceil(nq / 256): query-tile pairs per head
   float scale_log2;       // softmax scale * log2(e)
   int round_tf32;         // round A_loc / D stores to tf32 (nearest, ties away)
-  float* a_loc;           // [nq, d] fp32 or nullptr (required with history)
+  float* a_loc;           // [nq, d] fp32 or nullptr
   float* d_out;           // [nq, d] fp32 or nullptr
   __nv_bfloat16* a_full;  // [nq, d] bf16 or nullptr
   float* lse_loc;         // [heads, nq] or nullptr
   float* lse_hist;
   float* lse_full;
-  float* loc_out;         // local-branch output: a_loc, or workspace when A_loc is not wanted
-  float* hist_out;        // workspace: per history split, output [nq, d] fp32
-  float* lse_loc_ws;      // workspace: [heads, nq]
-  float* lse_hist_ws;     // workspace: per history split, [heads, nq]
-  int n_split;            // history key ranges (split-KV), >= 1
-  int split_tiles;        // 128-key tiles per history split
-  int64_t hist_stride;    // elements between the splits' hist_out (nq * d)
-  int64_t lse_stride;     // elements between the splits' lse_hist_ws (heads * nq)
+  AttnPlan plan;
+  uint8_t order[kMaxSlots];  // slots, longest key range first (grid order)
+  // Workspace. Every unit of a multi-unit (head, pair) leaves its normalised
+  // output and LSE in its slot; the last unit to finish merges them.
+  float* part;            // [slots - part_first][nq, d] fp32 partial outputs
+  int part_first;         // 1: slot 0's output is a_loc itself (stored rounded)
+  int64_t part_stride;    // elements between slots in `part`
+  float* part_lse;        // [slots][heads, nq]
+  int64_t lse_stride;     // elements between slots in `part_lse`
+  int* counters;          // [heads * n_pairs] units finished, zero at launch
   int* status;
+  uint64_t wait_ns;       // limit of a pipeline wait (set at launch)
 };
 
-// Number of history splits for these branch lengths: one while the history
-// is at most three times the local branch, else about two local branches of
-// keys per split (balances long histories over the SMs).
-int history_splits(int64_t sink_len, int64_t local_len, int64_t hist_len);
-// Key tiles per history split.
-int history_split_tiles(int64_t hist_len, int n_split);
+// The unit decomposition of a call with these branch lengths (see
+// attention.cu for the rule). Cached per shape.
+AttnPlan attention_plan(int64_t nq, int64_t sink_len, int64_t local_len, int64_t hist_len,
+                        int heads);
+// Most slots any plan for these branch lengths may use (the candidates'
+// maximum): non-decreasing in hist_len, so a workspace sized for the longest
+// history serves every shorter one with the same sink and local lengths.
+int attention_slot_bound(int64_t sink_len, int64_t local_len, int64_t hist_len);
+// Forces the split counts of later plans (0 = automatic). For measurement.
+void attention_force_splits(int local_splits, int hist_splits);
+// Longest-first order of the plan's slots (grid order of the units).
+void attention_slot_order(const AttnPlan& plan, int64_t loc_tiles, int64_t hist_tiles,
+                          uint8_t* order);
 
 size_t attention_smem_bytes(int head_dim);
 int attention_pairs(int64_t nq);
-cudaError_t launch_v_to_half(const void* src, void* dst, int64_t n_elems, int* status,
-                             cudaStream_t stream);
+int64_t attention_key_tiles(int64_t len);
 cudaError_t launch_dual_attention(const AttnParams& p, int head_dim, cudaStream_t stream);
 
 // Gram accumulation: see gram.cu.
@@ -66,6 +89,7 @@ struct GramParams {
   int64_t total_iters;
   int64_t iters_per_cta;  // of the iterations left after the whole-tile waves
   int* status;
+  uint64_t wait_ns;       // limit of a pipeline wait (set at launch)
 };
 cudaError_t launch_gram(const GramParams& p, int bn, int grid, cudaStream_t stream);
 
@@ -78,6 +102,7 @@ struct ProjParams {
   void* out;              // [M, N] bf16 or fp32
   int out_fp32;
   int* status;
+  uint64_t wait_ns;       // limit of a pipeline wait (set at launch)
 };
 cudaError_t launch_proj(const ProjParams& p, cudaStream_t stream);
 cudaError_t launch_absorbed_weight(const float* W, const float* dW, int64_t n, void* out,

@@ -25,6 +25,7 @@
 // (M is zeroed first when the call does not accumulate).
 #include "sm100.cuh"
 #include "attention.h"
+#include "host_util.h"
 
 namespace ispa {
 namespace {
@@ -154,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1) gram_kernel(const __grid_constant
         bool ok = true;
         for (int k = kb; k < ke; ++k, ++n) {
           const int st = (int)(n % NSTAGE);
-          if (n >= NSTAGE && !mbar_wait(&s.empty[st], ((n / NSTAGE) - 1) & 1, p.status, abort_flag)) {
+          if (n >= NSTAGE && !mbar_wait(&s.empty[st], ((n / NSTAGE) - 1) & 1, p.status, abort_flag, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -166,10 +167,10 @@ __global__ void __launch_bounds__(kThreads, 1) gram_kernel(const __grid_constant
         }
         if (!ok) break;
       }
-      if (*abort_flag) {
-        for (int64_t j = n - NSTAGE < 0 ? 0 : n - NSTAGE; j < n; ++j)
-          drain_wait(&s.full[j % NSTAGE], (j / NSTAGE) & 1, p.status);
-      }
+      // every copy issued has landed before the CTA exits (at once unless a
+      // consumer gave up)
+      for (int64_t j = n - NSTAGE < 0 ? 0 : n - NSTAGE; j < n; ++j)
+        drain_wait(&s.full[j % NSTAGE], (j / NSTAGE) & 1, p.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -183,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1) gram_kernel(const __grid_constant
       for (; ok && seg_next(p, si, tile, kb, ke); ++seg) {
         // the epilogue must have drained this buffer's previous segment (seg - 2)
         if (seg >= 2 &&
-            !mbar_wait(&s.acc_empty[seg & 1], ((seg - 2) >> 1) & 1, p.status, abort_flag)) {
+            !mbar_wait(&s.acc_empty[seg & 1], ((seg - 2) >> 1) & 1, p.status, abort_flag, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -191,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1) gram_kernel(const __grid_constant
         const uint32_t acc = tacc + (uint32_t)((seg & 1) * BN);
         for (int k = kb; k < ke; ++k, ++n) {
           const int st = (int)(n % NSTAGE);
-          if (!mbar_wait(&s.full[st], (n / NSTAGE) & 1, p.status, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&s.full[st], (n / NSTAGE) & 1, p.status, abort_flag, p.wait_ns)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < BK / 8; ++kk) {
@@ -204,10 +205,9 @@ __global__ void __launch_bounds__(kThreads, 1) gram_kernel(const __grid_constant
         if (!ok) break;
         tc_commit(&s.acc_full[seg & 1]);
       }
-      if (!ok) {
-        tc_commit(&s.drain);
-        drain_wait(&s.drain, 0, p.status);
-      }
+      // every MMA issued has finished before TMEM is freed
+      tc_commit(&s.drain);
+      drain_wait(&s.drain, 0, p.status);
     }
     __syncwarp();
   } else {
@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) gram_kernel(const __grid_constant
     int tile, kb, ke;
     for (; seg_next(p, si, tile, kb, ke); ++seg) {
       const Tile t = decode_tile(tile, p.dim, BN);
-      if (!mbar_wait(&s.acc_full[seg & 1], (seg >> 1) & 1, p.status, abort_flag)) break;
+      if (!mbar_wait_warp(&s.acc_full[seg & 1], (seg >> 1) & 1, p.status, abort_flag, p.wait_ns)) break;
       tc_fence_after();
       const uint32_t acc = tacc + (uint32_t)((seg & 1) * BN);
       const int64_t row = (int64_t)t.I * BM + r + (t.type == 2 ? p.dim : 0);
@@ -259,7 +259,9 @@ int gram_tile_count(int dim, int bn, int want_s) {
   return upper + nI * nJ + (want_s ? upper : 0);
 }
 
-cudaError_t launch_gram(const GramParams& p, int bn, int grid, cudaStream_t stream) {
+cudaError_t launch_gram(const GramParams& p0, int bn, int grid, cudaStream_t stream) {
+  GramParams p = p0;
+  p.wait_ns = wait_limit_ns();
   if (bn == 256) {
     const size_t smem = sizeof(GramSmem<256>) + 1024;
     cudaFuncSetAttribute(gram_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -1,4 +1,6 @@
-// TMA descriptor encoding (host side).
+// Host-side helpers: CUDA error reporting, TMA descriptor encoding.
+#include <atomic>
+#include <cstdio>
 #include <mutex>
 
 #include "host_util.h"
@@ -26,6 +28,22 @@ EncodeTiledFn encode_fn() {
 }
 
 }  // namespace
+
+namespace {
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;   // the kernels' kWaitLimitNs
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+}  // namespace
+
+uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
+void set_wait_limit_ns(uint64_t ns) {
+  g_wait_ns.store(ns == 0 || ns > kDefaultWaitNs ? kDefaultWaitNs : ns, std::memory_order_relaxed);
+}
+
+int cuda_rc(cudaError_t e) {
+  if (e == cudaSuccess) return ISPA_OK;
+  std::fprintf(stderr, "ispa: CUDA error %s\n", cudaGetErrorString(e));
+  return ISPA_ERR_CUDA;
+}
 
 bool encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t cols,
                uint64_t rows, uint64_t ld, uint32_t box_cols, uint32_t box_rows,

@@ -5,7 +5,38 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <nvtx3/nvToolsExt.h>
+
+#include "../../include/ispa.h"
+
 namespace ispa {
+
+// ISPA_OK for cudaSuccess; otherwise prints the CUDA error on stderr and
+// returns ISPA_ERR_CUDA.
+int cuda_rc(cudaError_t e);
+
+// An NVTX range named after the C-ABI entry point for the rest of the scope
+// (what a profiler's timeline shows around the call's launches). Without a
+// tool attached the push and pop are empty calls.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define ISPA_NVTX_RANGE() ::ispa::NvtxRange ispa_nvtx_range_(__func__)
+
+// Limit of a kernel's pipeline waits, in ns, for the launches that follow
+// (process-wide; 2 s unless set_wait_limit_ns changed it; 0 restores 2 s).
+uint64_t wait_limit_ns();
+void set_wait_limit_ns(uint64_t ns);
+
+// Bytes of one absorb solve's scratch at dimension d: A, Z, Y; the tf32
+// hi/lo planes of each; one 128 x 128 inverse with its hi/lo planes; lambda
+// and padding; a multiple of 256 bytes so that per-layer workspaces stack.
+constexpr size_t absorb_scratch_bytes(size_t d) {
+  return ((9 * d * d + 3 * 128 * 128) * sizeof(float) + 1024 + 255) & ~size_t(255);
+}
 
 // Row-major [rows, cols] matrix with leading dimension ld (elements), tiles
 // of box_cols x box_rows. Returns false if the driver rejects the map.

@@ -16,6 +16,7 @@
 // not stored.
 #include "sm100.cuh"
 #include "attention.h"
+#include "host_util.h"
 
 namespace ispa {
 namespace {
@@ -69,15 +70,15 @@ __global__ void __launch_bounds__(kPThreads, 1) proj_kernel(const __grid_constan
       int n = 0;
       for (; n < nk; ++n) {
         const int st = n % PSTAGE;
-        if (n >= PSTAGE && !mbar_wait(&s.empty[st], ((n / PSTAGE) - 1) & 1, p.status, abort_flag))
+        if (n >= PSTAGE && !mbar_wait(&s.empty[st], ((n / PSTAGE) - 1) & 1, p.status, abort_flag, p.wait_ns))
           break;
         mbar_expect_tx(&s.full[st], (PM + PN) * PK * 2);
         tma_load_2d(s.a[st], &p.ta, &s.full[st], n * PK, row0);
         for (int c = 0; c < PN / 64; ++c) tma_load_2d(s.b[st][c], &p.tb, &s.full[st], col0 + c * 64, n * PK);
       }
-      if (*abort_flag)
-        for (int j = n - PSTAGE < 0 ? 0 : n - PSTAGE; j < n; ++j)
-          proj_drain_wait(&s.full[j % PSTAGE], (j / PSTAGE) & 1, p.status);
+      // every copy issued has landed before the CTA exits
+      for (int j = n - PSTAGE < 0 ? 0 : n - PSTAGE; j < n; ++j)
+        proj_drain_wait(&s.full[j % PSTAGE], (j / PSTAGE) & 1, p.status);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(kPThreads, 1) proj_kernel(const __grid_constan
       bool ok = true;
       for (int n = 0; n < nk; ++n) {
         const int st = n % PSTAGE;
-        if (!mbar_wait(&s.full[st], (n / PSTAGE) & 1, p.status, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&s.full[st], (n / PSTAGE) & 1, p.status, abort_flag, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
         // A: 128-byte rows, 8-row groups 1024 B apart, 16 K = 32 B per step.
         // B: 64-column blocks 8 KB apart, 8-row groups 1024 B apart, 16 K rows = 2 KB per step.
@@ -98,7 +99,8 @@ __global__ void __launch_bounds__(kPThreads, 1) proj_kernel(const __grid_constan
         tc_commit(&s.empty[st]);
       }
       if (ok) tc_commit(&s.acc_full);
-      else { tc_commit(&s.drain); proj_drain_wait(&s.drain, 0, p.status); }
+      tc_commit(&s.drain);                 // every MMA issued has finished before TMEM is freed
+      proj_drain_wait(&s.drain, 0, p.status);
     }
     __syncwarp();
   } else {
@@ -106,7 +108,7 @@ __global__ void __launch_bounds__(kPThreads, 1) proj_kernel(const __grid_constan
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int64_t row = (int64_t)row0 + r;
-    if (mbar_wait(&s.acc_full, 0, p.status, abort_flag)) {
+    if (mbar_wait_warp(&s.acc_full, 0, p.status, abort_flag, p.wait_ns)) {
       tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < PN / 32; ++c) {
@@ -161,7 +163,9 @@ __global__ void absorbed_weight_kernel(const float4* __restrict__ W, const float
 
 }  // namespace
 
-cudaError_t launch_proj(const ProjParams& p, cudaStream_t stream) {
+cudaError_t launch_proj(const ProjParams& p0, cudaStream_t stream) {
+  ProjParams p = p0;
+  p.wait_ns = wait_limit_ns();
   if (p.M == 0) return cudaSuccess;
   const size_t smem = sizeof(ProjSmem) + 1024;
   cudaFuncSetAttribute(proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

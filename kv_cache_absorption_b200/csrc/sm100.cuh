@@ -73,24 +73,39 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed. Gives up after
-// kWaitLimitNs, flags ISPA_STATUS_TIMEOUT in *status (and *abort_flag, a
-// CTA-wide shared flag) and returns false. Also returns false at once when
-// another thread of the CTA has already given up.
+// limit_ns, flags ISPA_STATUS_TIMEOUT in *status (and *abort_flag, a CTA-wide
+// shared flag) and returns false. Also returns false at once when another
+// thread of the CTA has already given up. Pipeline waits take the launch's
+// limit (kWaitLimitNs unless a caller shortened it to exercise this path);
+// the waits that let in-flight copies and MMAs land while unwinding always
+// keep kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
-                                          volatile int* abort_flag) {
+                                          volatile int* abort_flag,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try(bar, parity)) return true;
-  uint64_t t0 = global_ns();
-  for (uint32_t it = 1;; ++it) {
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 0;; ++it) {
     if (mbar_try(bar, parity)) return true;
-    if ((it & 255u) == 0) {
+    if ((it & 255u) == 0) {   // at the first retry, then every 256
       if (*abort_flag) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         if (status) atomicOr(status, ISPA_STATUS_TIMEOUT);
         return false;
       }
     }
   }
+}
+
+// mbar_wait for code that continues with warp-collective instructions
+// (tcgen05.ld/st .sync.aligned, __syncwarp, votes): every lane of the warp
+// calls it and all get the same answer, false if any lane's wait gave up, so
+// the warp never splits between the work and the unwind path.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* status,
+                                               volatile int* abort_flag,
+                                               uint64_t limit_ns = kWaitLimitNs) {
+  const bool ok = mbar_wait(bar, parity, status, abort_flag, limit_ns);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // Warpgroup-wide register budget changes. Every warp of a warpgroup must run

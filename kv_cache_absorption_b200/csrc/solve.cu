@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
   auto factor32 = [&](int J) {
     {
       float r[32];
-      bool bad = false;
+      bool bad = false, nonfinite = false;
 #pragma unroll
       for (int q = 0; q < 8; ++q) ld4(&r[4 * q], &a[(J + lane) * kSA + J + 4 * q]);
 #pragma unroll
@@ -184,7 +184,8 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
         for (int m = 0; m < 4; ++m) {
           const int j = j0 + m;
           const float piv = __shfl_sync(0xffffffffu, tp, j);
-          bad |= !(piv > 0.f);
+          nonfinite |= !(fabsf(piv) <= 3.402823466e38f);   // NaN or infinite: bad input
+          bad |= piv <= 0.f;
           const float inv = rsqrtf(piv);         // NaN for a non-positive pivot: poisons what follows
           const float lv = lane > j ? r[m] * inv : (lane == j ? piv * inv : 0.f);   // L[lane][j]
           r[m] = lv;
@@ -213,6 +214,7 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
         __syncwarp();
       }
       if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, ISPA_STATUS_NOT_SPD);
+      if (__any_sync(0xffffffffu, nonfinite) && lane == 0) atomicOr(status, ISPA_STATUS_NONFINITE);
     }
   };
   for (int J = 0; J < NB; J += 32) {
@@ -521,11 +523,8 @@ cudaError_t panel_launch(int n, const SolveWs& w, size_t d, int kk, int m, int* 
 }  // namespace
 
 size_t absorb_workspace_bytes(int dim) {
-  const size_t d = (size_t)dim;
-  // A, Z, Y; hi/lo planes of each; one 128 x 128 inverse and its hi/lo
-  // planes; lambda (+ padding);
-  // a multiple of 256 bytes so that per-layer workspaces stack
-  return ((9 * d * d + 3 * NB * NB) * sizeof(float) + 1024 + 255) & ~size_t(255);
+  static_assert(NB == 128, "absorb_scratch_bytes assumes 128-wide blocks");
+  return absorb_scratch_bytes((size_t)dim);
 }
 
 cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const float* W,

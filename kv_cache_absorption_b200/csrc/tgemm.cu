@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
       int n = 0;
       for (int k = kb; k < ke; ++k, ++n) {
         const int st = n % NSTAGE;
-        if (n >= NSTAGE && !mbar_wait(&s.empty[st], ((n / NSTAGE) - 1) & 1, p.status, abort_flag)) break;
+        if (n >= NSTAGE && !mbar_wait(&s.empty[st], ((n / NSTAGE) - 1) & 1, p.status, abort_flag, p.wait_ns)) break;
         mbar_expect_tx(&s.full[st], (2 + pr.a_split + pr.b_split) * kSlab);
         load_slab(s.a_hi[st], &pr.ta, pr.a_mn, pr.a_row0 + ti * TM, pr.a_k0 + k * TK, layer,
                   &s.full[st]);
@@ -224,9 +224,9 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
           load_slab(s.b_lo[st], &pr.tb_lo, pr.b_mn, pr.b_col0 + tj * TN, pr.b_k0 + k * TK, layer,
                     &s.full[st]);
       }
-      if (*abort_flag)
-        for (int j = n - NSTAGE < 0 ? 0 : n - NSTAGE; j < n; ++j)
-          drain_wait(&s.full[j % NSTAGE], (j / NSTAGE) & 1, p.status);
+      // every copy issued has landed before the CTA exits
+      for (int j = n - NSTAGE < 0 ? 0 : n - NSTAGE; j < n; ++j)
+        drain_wait(&s.full[j % NSTAGE], (j / NSTAGE) & 1, p.status);
     }
   } else if (warp == 1) {
     if (lane == 0 && nk > 0) {
@@ -240,11 +240,11 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
         const bool first = kc > 0 ? (n % kc == 0) : (n == 0);
         // chunk c >= 1 goes to buffer (c - 1) & 1, free once chunk c - 2 was summed
         if (first && c >= 3 &&
-            !mbar_wait(&s.chunk_empty[(c - 1) & 1], ((c - 3) >> 1) & 1, p.status, abort_flag)) {
+            !mbar_wait(&s.chunk_empty[(c - 1) & 1], ((c - 3) >> 1) & 1, p.status, abort_flag, p.wait_ns)) {
           ok = false;
           break;
         }
-        if (!mbar_wait(&s.split[st], (n / NSTAGE) & 1, p.status, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&s.split[st], (n / NSTAGE) & 1, p.status, abort_flag, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t dst = c >= 1 ? tacc + (uint32_t)(TN * (1 + ((c - 1) & 1))) : tacc;
         const uint64_t ah = slab_desc(s.a_hi[st], pr.a_mn), al = slab_desc(s.a_lo[st], pr.a_mn);
@@ -260,7 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
         if (c >= 1 && (n % kc == kc - 1 || n == nk - 1)) tc_commit(&s.chunk_full[(c - 1) & 1]);
       }
       if (ok) tc_commit(&s.acc_full);
-      else { tc_commit(&s.drain); drain_wait(&s.drain, 0, p.status); }
+      tc_commit(&s.drain);                 // every MMA issued has finished before TMEM is freed
+      drain_wait(&s.drain, 0, p.status);
     }
     __syncwarp();
   } else {
@@ -270,7 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
     // running sum += chunk c (c >= 1), then release its buffer
     auto sum_chunk = [&](int c) -> bool {
       const int b = (c - 1) & 1;
-      if (!mbar_wait(&s.chunk_full[b], ((c - 1) >> 1) & 1, p.status, abort_flag)) return false;
+      if (!mbar_wait_warp(&s.chunk_full[b], ((c - 1) >> 1) & 1, p.status, abort_flag, p.wait_ns))
+        return false;
       tc_fence_after();
 #pragma unroll 1
       for (int q = 0; q < TN / 32; ++q) {
@@ -295,7 +297,10 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
         if (!sum_chunk(n / kc - 2)) { ok = false; break; }
         summed = n / kc - 2;
       }
-      if (!mbar_wait(&s.full[st], (n / NSTAGE) & 1, p.status, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(&s.full[st], (n / NSTAGE) & 1, p.status, abort_flag, p.wait_ns)) {
+        ok = false;
+        break;
+      }
       // operands given pre-split need no work; the others are split in place
       const int v_begin = pr.a_split ? kSlab / 16 : 0;
       const int v_end = pr.b_split ? kSlab / 16 : 2 * kSlab / 16;
@@ -323,7 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1) tgemm_kernel(const __grid_constan
     const uint32_t lane_off = row_off;
     const int64_t row = (int64_t)pr.c_row0 + (int64_t)ti * TM + r;
     const int64_t col0 = (int64_t)pr.c_col0 + (int64_t)tj * TN;
-    if (ok && (nk == 0 || mbar_wait(&s.acc_full, 0, p.status, abort_flag))) {
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && (nk == 0 || mbar_wait_warp(&s.acc_full, 0, p.status, abort_flag, p.wait_ns))) {
       tc_fence_after();
       if (pr.mode == kModeStore && pr.out_tma) {
         // boxes of this warp: per 32-column chunk, C and/or the hi and lo
@@ -531,6 +537,7 @@ static void plan_output(TGemmProblem& pr) {
 }
 
 cudaError_t launch_tgemm(TGemmParams& p, cudaStream_t stream) {
+  p.wait_ns = wait_limit_ns();
   int base = 0;
   for (int q = 0; q < p.nprob; ++q) {
     TGemmProblem& pr = p.prob[q];

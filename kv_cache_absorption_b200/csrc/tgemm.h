@@ -60,6 +60,7 @@ struct TGemmParams {
   int kchunk;              // > 0: accumulate K in chunks of kchunk 32-deep slabs, each in a
                            // fresh accumulator, and sum the chunks in fp32 (round to nearest)
   int* status;
+  uint64_t wait_ns;         // limit of a pipeline wait (set at launch)
 };
 
 size_t tgemm_smem_bytes();

@@ -21,6 +21,7 @@
 // MMA issuer (K = 32 per instruction), warps 2-5 epilogue.
 #include "sm100.cuh"
 #include "attention.h"
+#include "host_util.h"
 #include "w8a8.h"
 
 namespace ispa {
@@ -97,15 +98,15 @@ __global__ void __launch_bounds__(kQThreads, 1) gemm_i8_kernel(const __grid_cons
       int n = 0;
       for (; n < nk; ++n) {
         const int st = n % QSTAGE;
-        if (n >= QSTAGE && !mbar_wait(&s.empty[st], ((n / QSTAGE) - 1) & 1, p.status, abort_flag))
+        if (n >= QSTAGE && !mbar_wait(&s.empty[st], ((n / QSTAGE) - 1) & 1, p.status, abort_flag, p.wait_ns))
           break;
         mbar_expect_tx(&s.full[st], (QM + QN) * QK);
         tma_load_2d(s.a[st], &p.ta, &s.full[st], n * QK, row0);
         tma_load_2d(s.b[st], &p.tb, &s.full[st], n * QK, col0);
       }
-      if (*abort_flag)
-        for (int j = n - QSTAGE < 0 ? 0 : n - QSTAGE; j < n; ++j)
-          q8_drain_wait(&s.full[j % QSTAGE], (j / QSTAGE) & 1, p.status);
+      // every copy issued has landed before the CTA exits
+      for (int j = n - QSTAGE < 0 ? 0 : n - QSTAGE; j < n; ++j)
+        q8_drain_wait(&s.full[j % QSTAGE], (j / QSTAGE) & 1, p.status);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -113,7 +114,7 @@ __global__ void __launch_bounds__(kQThreads, 1) gemm_i8_kernel(const __grid_cons
       bool ok = true;
       for (int n = 0; n < nk; ++n) {
         const int st = n % QSTAGE;
-        if (!mbar_wait(&s.full[st], (n / QSTAGE) & 1, p.status, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&s.full[st], (n / QSTAGE) & 1, p.status, abort_flag, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
         // 128-byte rows, 8-row groups 1024 B apart; K = 32 bytes per MMA
         const uint64_t ad = smem_desc(smem_u32(s.a[st]), 16, 1024);
@@ -125,7 +126,8 @@ __global__ void __launch_bounds__(kQThreads, 1) gemm_i8_kernel(const __grid_cons
         tc_commit(&s.empty[st]);
       }
       if (ok) tc_commit(&s.acc_full);
-      else { tc_commit(&s.drain); q8_drain_wait(&s.drain, 0, p.status); }
+      tc_commit(&s.drain);                 // every MMA issued has finished before TMEM is freed
+      q8_drain_wait(&s.drain, 0, p.status);
     }
     __syncwarp();
   } else {
@@ -133,7 +135,7 @@ __global__ void __launch_bounds__(kQThreads, 1) gemm_i8_kernel(const __grid_cons
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int64_t row = (int64_t)row0 + r;
-    if (mbar_wait(&s.acc_full, 0, p.status, abort_flag)) {
+    if (mbar_wait_warp(&s.acc_full, 0, p.status, abort_flag, p.wait_ns)) {
       tc_fence_after();
       const float sa = row < p.M ? p.a_scale[row] : 0.f;
 #pragma unroll 1
@@ -240,7 +242,9 @@ __global__ void weight_quant_t_kernel(const float* __restrict__ W, const float* 
 
 }  // namespace
 
-cudaError_t launch_gemm_i8(const Q8Params& p, cudaStream_t stream) {
+cudaError_t launch_gemm_i8(const Q8Params& p0, cudaStream_t stream) {
+  Q8Params p = p0;
+  p.wait_ns = wait_limit_ns();
   if (p.M == 0) return cudaSuccess;
   const size_t smem = sizeof(Q8Smem) + 1024;
   cudaFuncSetAttribute(gemm_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

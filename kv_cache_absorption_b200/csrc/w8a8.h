@@ -17,6 +17,7 @@ struct Q8Params {
   void* out;              // [M, N] bf16 or fp32
   int out_fp32;
   int* status;
+  uint64_t wait_ns;       // limit of a pipeline wait (set at launch)
 };
 
 cudaError_t launch_gemm_i8(const Q8Params& p, cudaStream_t stream);

@@ -37,7 +37,8 @@ EXPORTED = (
     "ispa_weight_gram_batched", "ispa_layer_error_wwt_batched",
     "ispa_full_attention_workspace_size", "ispa_full_attention", "ispa_absorbed_weight",
     "ispa_project", "ispa_quantize_weight_int8", "ispa_project_w8a8_workspace_size",
-    "ispa_project_w8a8",
+    "ispa_project_w8a8", "ispa_attention_units", "ispa_attention_set_splits",
+    "ispa_set_wait_limit_ns",
 )
 
 
@@ -69,6 +70,9 @@ def _load():
         "ispa_version": (I, []),
         "ispa_kernel_launches": (ctypes.c_uint64, []),
         "ispa_dual_attention_workspace_size": (SZ, [I64, I64, I64, I64, I, I]),
+        "ispa_attention_units": (I64, [I64, I64, I64, I64, I, P, P]),
+        "ispa_attention_set_splits": (I, [I, I]),
+        "ispa_set_wait_limit_ns": (I, [ctypes.c_uint64]),
         "ispa_dual_attention": (I, [P, I64, I, I, IspaKV, IspaKV, IspaKV, F, P, P, P, P, P, P,
                                     P, SZ, P, P]),
         "ispa_local_attention": (I, [P, I64, I, I, IspaKV, IspaKV, F, P, P, P, P, SZ, P, P]),
@@ -79,7 +83,7 @@ def _load():
         "ispa_quantize_weight_int8": (I, [P, P, I, P, P, P]),
         "ispa_project_w8a8_workspace_size": (SZ, [I64, I]),
         "ispa_project_w8a8": (I, [P, I64, I, P, P, P, I, P, SZ, P, P]),
-        "ispa_gram_accumulate": (I, [P, P, I64, I, P, I, I, P]),
+        "ispa_gram_accumulate": (I, [P, P, I64, I, P, I, I, P, P]),
         "ispa_absorb_workspace_size": (SZ, [I]),
         "ispa_absorb_solve": (I, [P, P, I, F, P, P, P, P, SZ, P, P]),
         "ispa_absorb_solve_noalloc": (I, [P, P, I, F, P, P, P, P, P]),
@@ -228,6 +232,28 @@ def ispa_local_attention(q, k_sink, v_sink, k_loc, v_loc, scale=None, out_dtype=
     return {"out": out, "lse": lse, "status": status}
 
 
+def ispa_attention_units(nq: int, sink_len: int, local_len: int, hist_len: int,
+                         heads: int) -> tuple:
+    """(units, local key ranges, history key ranges) of an attention call of
+    this shape. Host only."""
+    ls, hs = ctypes.c_int(0), ctypes.c_int(0)
+    n = _load().ispa_attention_units(nq, sink_len, local_len, hist_len, heads, ctypes.byref(ls),
+                                     ctypes.byref(hs))
+    return int(n), ls.value, hs.value
+
+
+def ispa_set_wait_limit_ns(ns: int = 0) -> None:
+    """Limit of the kernels' pipeline waits for later launches (0 = default
+    2 s); a wait past it ends the kernel with ISPA_STATUS_TIMEOUT."""
+    _check(_load().ispa_set_wait_limit_ns(int(ns)), "ispa_set_wait_limit_ns")
+
+
+def ispa_attention_set_splits(local_splits: int = 0, hist_splits: int = 0) -> None:
+    """Force the key-range split counts of later attention calls (0 = automatic)."""
+    _check(_load().ispa_attention_set_splits(int(local_splits), int(hist_splits)),
+           "ispa_attention_set_splits")
+
+
 def ispa_full_attention_workspace_size(nq, sink_len, local_len, hist_len, heads, head_dim) -> int:
     return _load().ispa_full_attention_workspace_size(nq, sink_len, local_len, hist_len, heads,
                                                       head_dim)
@@ -327,9 +353,12 @@ def ispa_project_w8a8(a, wq_t, w_scale, out=None, out_dtype=torch.bfloat16, work
     return out
 
 
-def ispa_gram_accumulate(a_loc, d, M=None, accumulate=False, want_s=True, stream=None):
+def ispa_gram_accumulate(a_loc, d, M=None, accumulate=False, want_s=True, status=None,
+                         stream=None):
     """M[0:d,0:d] (G) (+)= A_loc^T A_loc, M[0:d,d:2d] (R) (+)= A_loc^T D,
-    M[d:2d,d:2d] (S) (+)= D^T D; M is [2d, 2d] fp32. Returns M."""
+    M[d:2d,d:2d] (S) (+)= D^T D; M is [2d, 2d] fp32. ``status``: a device
+    status word (``new_status``) that receives ISPA_STATUS_* bits; one is made
+    when not given. Returns M."""
     _dev_tensor(a_loc, torch.float32, "a_loc", 2)
     _dev_tensor(d, torch.float32, "d", 2)
     rows, dim = a_loc.shape
@@ -339,8 +368,9 @@ def ispa_gram_accumulate(a_loc, d, M=None, accumulate=False, want_s=True, stream
         M = torch.empty(2 * dim, 2 * dim, dtype=torch.float32, device=a_loc.device)
         accumulate = False
     _dev_tensor(M, torch.float32, "M", 2)
+    status = new_status(a_loc.device) if status is None else status
     rc = _load().ispa_gram_accumulate(_ptr(a_loc), _ptr(d), rows, dim, _ptr(M), int(bool(accumulate)),
-                                      int(bool(want_s)), _stream(stream))
+                                      int(bool(want_s)), _ptr(status), _stream(stream))
     _check(rc, "ispa_gram_accumulate")
     return M
 

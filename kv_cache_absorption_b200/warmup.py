@@ -98,7 +98,8 @@ class LayerWarmup:
         sl = self.slots[slot]
         rc = ispa._load().ispa_gram_accumulate(
             ispa._ptr(sl.a_loc), ispa._ptr(sl.d_out), sl.rows, self.d,
-            ispa._ptr(self.M[layer]), 0 if first else 1, 1, ispa._stream(stream))
+            ispa._ptr(self.M[layer]), 0 if first else 1, 1, ispa._ptr(self.status),
+            ispa._stream(stream))
         ispa._check(rc, "ispa_gram_accumulate")
 
     def chunk(self, ch: dict, first: bool, layer: int = 0, stream=None, slot: int = 0):

@@ -35,7 +35,7 @@ def exported():
 
 def test_exports_match_header(ispa):
     names = declared()
-    assert len(names) == 24
+    assert len(names) == 27
     assert names == exported()
     assert names == set(ispa.EXPORTED)
     lib = ctypes.CDLL(ispa.LIB_PATH)
@@ -54,28 +54,65 @@ def test_version_and_status_strings(ispa):
 def test_workspace_sizes(ispa):
     def r256(x):
         return (x + 255) // 256 * 256
-    d = 12 * 128
-    assert ispa.ispa_dual_attention_workspace_size(4680, 1560, 4680, 14040, 12, 128) == \
-        r256(1560 * d * 2) + r256(4680 * d * 2) + r256(14040 * d * 2) + r256(4680 * d * 4) + \
-        2 * r256(12 * 4680 * 4) + 256
-    assert ispa.ispa_dual_attention_workspace_size(10, 1, 1, 0, 1, 64) == \
-        r256(64 * 2) * 2 + 2 * r256(40) + 256
+    nq, H, hd = 4680, 12, 128
+    out = r256(nq * H * hd * 4)
+    lse = r256(H * nq * 4)
+    cnt = r256(H * 19 * 4)                    # 19 query-tile pairs per head
+    loc_tiles = 13 + 37                       # 1560 sink + 4680 local keys
+
+    def bound(hist):                          # most key ranges any candidate plan uses
+        t = -(-hist // 128)
+        if t == 0:
+            return 4
+        base = 1 if t <= 3 * loc_tiles else min(64, -(-t // (2 * loc_tiles)))
+        return 4 + min(base + 2, t)
+    # one completion counter per (head, pair), an LSE block and an fp32
+    # output per key range, for the most ranges any candidate plan may use
+    sizes = []
+    for hist in (0, 4680, 9360, 14040, 18720, 93600):
+        want = cnt + bound(hist) * (lse + out) + 256
+        assert ispa.ispa_dual_attention_workspace_size(nq, 1560, 4680, hist, H, hd) == want
+        assert ispa.ispa_full_attention_workspace_size(nq, 1560, 4680, hist, H, hd) == want
+        units, ls, hs = ispa.ispa_attention_units(nq, 1560, 4680, hist, H)
+        assert ls + hs <= bound(hist)
+        sizes.append(want)
+    # non-decreasing in the history length: sized for the longest, fits all
+    assert sizes == sorted(sizes)
+    # one key tile and no history: one unit per (head, pair), no scratch
+    assert ispa.ispa_attention_units(10, 1, 0, 0, 1) == (1, 1, 0)
+    assert ispa.ispa_dual_attention_workspace_size(10, 1, 0, 0, 1, 64) == 256
     assert ispa.ispa_dual_attention_workspace_size(1, -1, 1, 1, 1, 64) == 0
     n = 1536
     assert ispa.ispa_absorb_workspace_size(n) >= 2 * n * n * 4
     assert ispa.ispa_absorb_workspace_size(0) == 0
     assert ispa.ispa_layer_error_workspace_size(128) >= 40
-    # a history longer than three local branches is cut into key ranges, each
-    # with its own fp32 output and LSE block; full attention also keeps the
-    # local branch's output
-    nq, H, hd = 4680, 12, 128
-    out = r256(nq * H * hd * 4)
-    lse = r256(H * nq * 4)
-    v = lambda n: r256(n * H * hd * 2)
-    assert ispa.ispa_dual_attention_workspace_size(nq, 1560, 4680, 93600, H, hd) == \
-        v(1560) + v(4680) + v(93600) + 8 * (out + lse) + lse + 256   # 732 tiles: 8 ranges
-    assert ispa.ispa_full_attention_workspace_size(nq, 1560, 4680, 93600, H, hd) == \
-        ispa.ispa_dual_attention_workspace_size(nq, 1560, 4680, 93600, H, hd) + out
+
+
+def test_attention_plan(ispa):
+    """The unit decomposition: key ranges cover each branch without empty
+    ranges, long histories are cut (split-KV), the counts can be forced, and
+    the plan follows the shape (host only)."""
+    nq, H = 4680, 12
+    per = H * 19
+    for hist in (0, 4680, 9360, 14040, 93600):
+        units, ls, hs = ispa.ispa_attention_units(nq, 1560, 4680, hist, H)
+        assert units == per * (ls + hs)
+        assert 1 <= ls <= 4 and ls <= 50           # 13 sink + 37 local key tiles
+        assert (hs == 0) == (hist == 0)
+    assert ispa.ispa_attention_units(nq, 1560, 4680, 93600, H)[2] >= 8   # 732 history tiles
+    # a branch of one key tile cannot be cut
+    assert ispa.ispa_attention_units(64, 0, 64, 0, 2)[1:] == (1, 0)
+    assert ispa.ispa_attention_units(1, 0, 0, 0, 1)[0] == 0               # no keys: invalid
+    try:
+        ispa.ispa_attention_set_splits(2, 3)
+        assert ispa.ispa_attention_units(nq, 1560, 4680, 14040, H) == (per * 5, 2, 3)
+        assert ispa.ispa_attention_units(nq, 1560, 4680, 0, H) == (per * 2, 2, 0)
+        # more ranges than tiles: one range per tile
+        assert ispa.ispa_attention_units(64, 16, 64, 128, 2)[1:] == (2, 1)
+    finally:
+        ispa.ispa_attention_set_splits(0, 0)
+    with pytest.raises(ispa.IspaError):
+        ispa.ispa_attention_set_splits(-1, 0)
 
 
 def _kv(ispa, n, addr=0x10000):
@@ -115,10 +152,11 @@ def test_dual_attention_host_checks(ispa):
 def test_other_entry_points_host_checks(ispa):
     lib = ispa._load()
     P = 0x1000
-    assert lib.ispa_gram_accumulate(P, P, 100, 100, P, 0, 1, None) == ispa.ISPA_ERR_UNSUPPORTED
-    assert lib.ispa_gram_accumulate(P, P, -1, 128, P, 0, 1, None) == ispa.ISPA_ERR_ARG
-    assert lib.ispa_gram_accumulate(None, P, 10, 128, P, 0, 1, None) == ispa.ISPA_ERR_ARG
-    assert lib.ispa_gram_accumulate(P, P, 10, 128, None, 0, 1, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_gram_accumulate(P, P, 100, 100, P, 0, 1, P, None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert lib.ispa_gram_accumulate(P, P, -1, 128, P, 0, 1, P, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_gram_accumulate(None, P, 10, 128, P, 0, 1, P, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_gram_accumulate(P, P, 10, 128, None, 0, 1, P, None) == ispa.ISPA_ERR_ARG
+    assert lib.ispa_gram_accumulate(P, P, 10, 128, P, 0, 1, None, None) == ispa.ISPA_ERR_ARG
     assert lib.ispa_absorb_solve(P, P, 128, float("nan"), P, P, None, P, 1 << 30, P, None) == ispa.ISPA_ERR_ARG
     assert lib.ispa_absorb_solve(P, P, 100, 0.0, P, P, None, P, 1 << 30, P, None) == ispa.ISPA_ERR_UNSUPPORTED
     assert lib.ispa_absorb_solve(P, P, 128, 0.0, P, P, None, P, 16, P, None) == ispa.ISPA_ERR_WORKSPACE

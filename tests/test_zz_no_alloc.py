@@ -5,9 +5,11 @@ host program that owns every device buffer and has no allocator at hand, or
 a loop that must never enter an allocator), the library keeps this solve's
 scratch in a device array of its own. This checks, through the C ABI, that
 two calls in a row -- the second one smaller, over the first one's leftover
-scratch contents -- give the workspace-based solve's results within the
-Delta W tolerance of the other tests, and that sizes beyond the array are
-refused. It runs last so that a failure here leaves every other test run.
+scratch contents, then a larger one again -- give the workspace-based
+solve's results within the Delta W tolerance of the other tests; that a call
+after the first one's set-up leaves the device's allocated and free memory
+unchanged; and that sizes beyond the array are refused. It runs last so that
+a failure here leaves every other test run.
 """
 import ctypes
 import math
@@ -38,11 +40,15 @@ def rel_fro(a, b):
     return (torch.linalg.norm((a - b).double()) / torch.linalg.norm(b.double())).item()
 
 
-def noalloc_call(lib, M, W, dim):
-    dW = torch.empty(dim, dim, dtype=torch.float32, device="cuda")
-    B = torch.empty(dim, dim, dtype=torch.float32, device="cuda")
-    lam = torch.empty(1, dtype=torch.float32, device="cuda")
-    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+def outputs(dim):
+    return (torch.empty(dim, dim, dtype=torch.float32, device="cuda"),
+            torch.empty(dim, dim, dtype=torch.float32, device="cuda"),
+            torch.empty(1, dtype=torch.float32, device="cuda"),
+            torch.zeros(1, dtype=torch.int32, device="cuda"))
+
+
+def noalloc_call(lib, M, W, dim, out=None):
+    dW, B, lam, status = outputs(dim) if out is None else out
     rc = lib._load().ispa_absorb_solve_noalloc(
         ctypes.c_void_p(M.data_ptr()), ctypes.c_void_p(W.data_ptr()), dim, 0.0,
         ctypes.c_void_p(dW.data_ptr()), ctypes.c_void_p(B.data_ptr()),
@@ -53,7 +59,9 @@ def noalloc_call(lib, M, W, dim):
 
 
 def test_noalloc_solve_matches_workspace_solve_on_two_calls(lib):
-    for dim, seed in ((512, 3), (256, 4)):          # second call is smaller: stale scratch above it
+    # the second call is smaller (stale scratch above it), the third larger
+    # again (over the second call's leftovers)
+    for dim, seed in ((512, 3), (256, 4), (512, 5)):
         M, W = make_problem(3 * dim, dim, seed)
         dW, B, lam, status = noalloc_call(lib, M, W, dim)
         ref = lib.ispa_absorb_solve(M, W)            # the workspace-based entry point
@@ -75,3 +83,24 @@ def test_noalloc_solve_refuses_sizes_beyond_its_array(lib):
         ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(out.data_ptr()), None,
         ctypes.c_void_p(st.data_ptr()), None)
     assert rc == lib.ISPA_ERR_UNSUPPORTED
+
+
+def test_noalloc_solve_allocates_nothing(lib):
+    """After the first call on the device has looked up the array's address,
+    a call changes neither torch's allocated bytes nor the device's free
+    memory: every byte it touches is the caller's or the library's array."""
+    dim = 384
+    M, W = make_problem(3 * dim, dim, 7)
+    noalloc_call(lib, M, W, dim)                      # set-up on this device
+    torch.cuda.synchronize()
+    out = outputs(dim)
+    torch.cuda.synchronize()
+    alloc0, free0 = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
+    dW, _, _, status = noalloc_call(lib, M, W, dim, out)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert int(status.item()) == 0
+    ref = lib.ispa_absorb_solve(M, W)
+    torch.cuda.synchronize()
+    assert rel_fro(dW, ref["dW"]) <= DW_RELFRO
