@@ -4,16 +4,22 @@
 One step = the whole hot path over one batch of synthetic input: dual-stream
 attention of every chunk, Gram accumulation of its rows, the closed-form
 Delta W solve, the reconstruction error of every layer and the layer ranking.
-Default workload: the 1.3B-class single-layer chunk (12 heads x 128, 4680
-queries, 1560 sink + 4680 local + 14040 history keys). ``--config c2`` /
-``c3`` run the 1.3B / 14B full warmups (30 / 40 layers, 4 chunks each).
+Default workload: the 1.3B-class full warmup (30 layers of 12 heads x 128,
+4 chunks of 4680 queries over 1560 sink + 4680 local + 0..14040 history
+keys). The same invocation also measures the 14B-class warmup (40 layers,
+40 heads) and the 1.3B single chunk (the last warmup chunk of one layer) and
+reports them as the sub-objects ``14B-warmup`` and ``1.3B-chunk``.
+``--config c1|c3`` makes one of those the main line (no sub-objects);
+``--config c4`` runs the post-transition streaming benchmark.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 Prints one JSON line (rank 0). ``value`` is the step's algorithmic TFLOP
-(attention 4*Nq*Nk*d counted once, Gram 4*N*d^2, solve (1/3+4)*d^3, error
-d^3) divided by the device time of the step, summed over all ranks' work;
-attention TFLOP/s and absorb ms per layer are reported alongside.
+(attention 4*Nq*Nk*d counted once, Gram 4*N*d^2, solve (1/3+4)*d^3; the
+error pass is an HBM-bound reduction credited with no flops) divided by the
+device time of the step, summed over all ranks' work; the attention TFLOP/s
+and the absorb ms per layer, each against its roofline, are the per-stage
+figures.
 """
 from __future__ import annotations
 
@@ -32,7 +38,6 @@ sys.path.insert(0, ROOT)
 
 METRIC = "dual-stream attention TFLOP/s and absorb ms/layer at 1.3B/14B shapes, % roofline"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dual_attention_1.3B_chunk_traffic.txt")
 TF32_FILE = os.path.join(ROOT, "profiles", "tf32_peak_cublas_gemm_8192.txt")
 L2_FLUSH_BYTES = 512 << 20
 
@@ -48,9 +53,10 @@ def step_work(cfg):
         attn += 4.0 * cfg.chunk_tokens * nk * d
     gram = 4.0 * cfg.warmup_rows * d * d
     solve = (1.0 / 3.0 + 4.0) * d ** 3
-    err = float(d) ** 3
     L = cfg.layers
-    return {"attention": attn * L, "gram": gram * L, "solve": solve * L, "error": err * L}
+    # the error stage reads G, R, S, W W^T, Delta W and B once (W W^T is
+    # formed when the weights load, outside the step): no flops credited
+    return {"attention": attn * L, "gram": gram * L, "solve": solve * L, "error": 0.0}
 
 
 def peaks():
@@ -127,11 +133,16 @@ def source_hash():
     return h.hexdigest()[:16]
 
 
-def traffic_per_launch():
-    """DRAM bytes per attention launch from the committed ncu summary, or None
-    when the kernel source changed since the counters were taken."""
+def traffic_file(workload_name):
+    return os.path.join(ROOT, "profiles", f"dual_attention_{workload_name}_traffic.txt")
+
+
+def traffic_per_launch(workload_name):
+    """DRAM bytes per attention launch of this workload from the committed ncu
+    summary, or None when there is none or the kernel source changed since
+    the counters were taken."""
     try:
-        with open(TRAFFIC_FILE) as f:
+        with open(traffic_file(workload_name)) as f:
             kv = dict(line.strip().split("=", 1) for line in f if "=" in line and not line.startswith("#"))
         if kv.get("source_hash") != source_hash():
             return None
@@ -270,7 +281,7 @@ def oracle_throughput(cfg, budget_s: float):
             acc[s][1] += timing[s][1]
         spent += sum(t for _, t in timing.values())
         n += 1
-    t_full = sum(work[s] * acc[s][1] / max(acc[s][0], 1.0) for s in work)
+    t_full = sum(work[s] * acc[s][1] / max(acc[s][0], 1.0) for s in work if work[s] > 0)
     total = sum(work.values())
     cores, blas = cpu_cores()
     return {"value": round(total / t_full / 1e12, 6), "unit": "TFLOP/s", "cores": blas or cores,
@@ -347,18 +358,33 @@ def make_inputs(cfg, rank, device, layers=None, replica=True):
     return streams, chunks, W_all
 
 
-def run_ours(args):
+def config_of(cfg, world, sharded, K):
+    """The ``config`` object of a bench line (both arms print the same one)."""
+    return {"workload": cfg.name, "layers": cfg.layers, "heads": cfg.heads,
+            "head_dim": cfg.head_dim, "d": cfg.d, "chunks": cfg.n_chunks,
+            "chunk_rows": cfg.chunk_tokens, "sink": cfg.sink_tokens,
+            "history": [len(cfg.history_frames_of(c)) * cfg.tokens_per_frame
+                        for c in range(cfg.n_chunks)],
+            "select_k": K, "l2": "flushed (512 MB write) before every timed step",
+            "weights": "W and W W^T per layer resident (W W^T formed once at load)",
+            "parallelism": (f"layer-sharded x{world} (errors all-gathered)" if sharded else
+                            f"replicas x{world}" if world > 1 else "single GPU")}
+
+
+def bus_id_of(dev):
     import torch
-    from kv_cache_absorption_b200 import build
-    build.build()
+    pr = torch.cuda.get_device_properties(dev)
+    return f"{getattr(pr, 'pci_domain_id', 0):08x}:{getattr(pr, 'pci_bus_id', 0):02x}:" \
+           f"{getattr(pr, 'pci_device_id', 0):02x}.0"
+
+
+def measure_warmup(args, cfg, world, rank, steps, warmup, with_e2e, with_cpu):
+    """Times the whole warmup step of ``cfg`` and returns its bench fields."""
+    import torch
     from kv_cache_absorption_b200 import ispa
     from kv_cache_absorption_b200.warmup import LayerWarmup, rank as rank_layers
-    from ispa_synth import CONFIGS
-
     from kv_cache_absorption_b200.sharding import gather_errors, owned_layers
-    world, rank, local = dist_setup()
     dev = torch.device("cuda", torch.cuda.current_device())
-    cfg = workload(args)
     # several GPUs: multi-layer warmups shard their layers (l on rank l mod N,
     # errors all-gathered for the ranking); a one-layer step runs as replicas
     sharded = world > 1 and cfg.layers >= world
@@ -404,22 +430,19 @@ def run_ours(args):
         err.copy_(gather_errors(err_mine, L, world) if sharded else err_mine)
         rank_layers(err, K, perm, sel)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     if ispa.read_status(runner.status) != 0:
         raise RuntimeError(f"device status {ispa.read_status(runner.status)} after warmup")
 
-    bus = torch.cuda.get_device_properties(dev)
-    bus_id = f"{getattr(bus, 'pci_domain_id', 0):08x}:{getattr(bus, 'pci_bus_id', 0):02x}:" \
-             f"{getattr(bus, 'pci_device_id', 0):02x}.0"
     starts, ends = [], []
     barrier(world)
     torch.cuda.synchronize()
-    sampler = ClockSampler(bus_id)
+    sampler = ClockSampler(bus_id_of(dev))
     time.sleep(0.15)
     launches0 = ispa.ispa_kernel_launches()
-    for _ in range(args.steps):
+    for _ in range(steps):
         flush.zero_()                       # L2 flush between timed steps, outside the events
         s0, e0 = E(), E()
         s0.record()
@@ -430,10 +453,10 @@ def run_ours(args):
     launches = ispa.ispa_kernel_launches() - launches0
     clocks = sampler.stop()
     barrier(world)
-    step_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    step_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / steps
 
     # per-stage breakdown: a few more steps on one stream, events around every stage
-    n_inst = max(1, min(args.steps, 5))
+    n_inst = max(1, min(steps, 5))
     ev = {"a0": [], "a1": [], "g1": [], "s1": []}
     for _ in range(n_inst):
         flush.zero_()
@@ -445,6 +468,7 @@ def run_ours(args):
     per_step = L_mine * cfg.n_chunks
     solve_ms = sum(ev["g1"][(i + 1) * per_step - 1].elapsed_time(ev["s1"][i])
                    for i in range(n_inst)) / n_inst
+    status = ispa.read_status(runner.status)
     step_ms_max = max_over_ranks(step_ms, world)
 
     work = step_work(cfg)
@@ -455,31 +479,29 @@ def run_ours(args):
     absorb_ms_layer = (gram_ms + solve_ms) / L_mine
     bf16_peak, hbm_peak, peak_src = peaks()
     attn_launches = L_mine * cfg.n_chunks
+    sm_mhz = clocks.get("sm_mhz") if clocks else None
     roofline = {
-        "bound": "tensor", "kernel": "dual-stream attention (V fp16 pre-pass + attention kernel)",
+        "bound": "tensor", "kernel": "dual-stream attention (branch_attention_kernel, merge fused)",
         "achieved": round(attn_tflops, 2), "peak": bf16_peak, "unit": "TFLOP/s",
         "frac": round(attn_tflops / bf16_peak, 4), "peak_source": f"{peak_src} bf16 dense (burst)",
-        "traffic": traffic_per_launch(),
-        "algorithmic_flops_per_launch": work["attention"] / attn_launches,
+        "traffic": traffic_per_launch(cfg.name),
+        "algorithmic_flops_per_launch": work["attention"] * share / attn_launches,
+        "algorithmic_bytes_per_launch": attention_bytes(cfg) / cfg.n_chunks,
         "ms_per_launch": attn_ms / attn_launches,
+        "launches_per_step": attn_launches,
+        # box-to-box comparable: the attention time in SM clock cycles
+        "sm_mcycles_per_step": round(attn_ms * sm_mhz * 1e-3, 3) if sm_mhz else None,
     }
-    absorb_flops = (work["gram"] + work["solve"] + work["error"]) * share
+    absorb_flops = (work["gram"] + work["solve"]) * share
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 4),
+        "steps": steps, "warmup": warmup, "ms_per_step": round(step_ms_max, 4),
         "higher_is_better": True, "scaling": "strong" if sharded else "weak", "vs_baseline": None,
         "dtype": "bf16 QK^T, fp16 PV, tf32 Gram, fp32 solve",
         "data": "synthetic AR(1) rho=0.9 bf16 Q/K/V, W ~ N(0,1/d), seeded",
-        "config": {"workload": cfg.name, "layers": L, "heads": cfg.heads, "head_dim": cfg.head_dim,
-                   "d": cfg.d, "chunks": cfg.n_chunks, "chunk_rows": cfg.chunk_tokens,
-                   "sink": cfg.sink_tokens,
-                   "history": [len(cfg.history_frames_of(c)) * cfg.tokens_per_frame
-                               for c in range(cfg.n_chunks)],
-                   "select_k": K, "l2": "flushed (512 MB write) before every timed step",
-                   "weights": "W and W W^T per layer resident (W W^T formed once at load)",
-                   "parallelism": (f"layer-sharded x{world} (errors all-gathered)" if sharded else
-                                   f"replicas x{world}" if world > 1 else "single GPU")},
+        "config": config_of(cfg, world, sharded, K),
         "attention_tflops": round(attn_tflops, 2),
+        "attention_frac_of_bf16_peak": round(attn_tflops / bf16_peak, 4),
         "attention_ms_per_step": round(attn_ms, 4),
         "absorb_ms_per_layer": round(absorb_ms_layer, 4),
         "gram_ms_per_step": round(gram_ms, 4), "solve_error_ms_per_step": round(solve_ms, 4),
@@ -488,13 +510,54 @@ def run_ours(args):
         "absorb_roofline": absorb_roofline(cfg, gram_ms * L / L_mine, solve_ms * L / L_mine,
                                            bf16_peak, hbm_peak),
         "gpu_launches": int(launches),
+        "device_status": status,
         "clocks": clocks,
     }
-    if not args.no_e2e:
+    if with_e2e:
         out["e2e"] = run_e2e(args, cfg, layer_streams_, chunks_per_layer, W_all, runner, err,
                              perm, sel, K, world, err_mine if sharded else None, streams)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if with_cpu and rank == 0 and world == 1:
         out["cpu_baseline"] = oracle_throughput(cfg, args.cpu_budget)
+    return out
+
+
+def attention_bytes(cfg):
+    """Algorithmic DRAM bytes of one layer's attention over all its chunks:
+    Q, K and V read once (bf16), A_loc and D written (fp32), A_full written
+    (bf16), three LSE rows per head written (fp32)."""
+    d = cfg.d
+    total = 0.0
+    for c in range(cfg.n_chunks):
+        keys = cfg.sink_tokens + cfg.chunk_tokens + len(cfg.history_frames_of(c)) * cfg.tokens_per_frame
+        total += (cfg.chunk_tokens + 2 * keys) * d * 2 + cfg.chunk_tokens * d * (4 + 4 + 2) \
+            + 3 * cfg.heads * cfg.chunk_tokens * 4
+    return total
+
+
+SUB_WORKLOADS = (("14B-warmup", "c3"), ("1.3B-chunk", "c1"))
+SUB_KEYS = ("value", "unit", "ms_per_step", "steps", "warmup", "config", "attention_tflops",
+            "attention_frac_of_bf16_peak", "attention_ms_per_step", "absorb_ms_per_layer",
+            "gram_ms_per_step", "solve_error_ms_per_step", "absorb_tflops", "roofline",
+            "absorb_roofline", "gpu_launches", "device_status", "clocks", "cpu_baseline")
+
+
+def run_ours(args):
+    import torch
+    from kv_cache_absorption_b200 import build
+    build.build()
+    from ispa_synth import CONFIGS
+    world, rank, local = dist_setup()
+    cfg = workload(args)
+    out = measure_warmup(args, cfg, world, rank, args.steps, args.warmup,
+                         with_e2e=not args.no_e2e, with_cpu=not args.no_cpu_baseline)
+    # the other shapes the metric is quoted on, in the same invocation
+    if args.config == "c2" and args.layers is None and not args.no_sub:
+        for key, name in SUB_WORKLOADS:
+            torch.cuda.empty_cache()
+            sub_steps = max(3, min(args.steps, 5 if name == "c3" else 50))
+            sub = measure_warmup(args, CONFIGS[name], world, rank, sub_steps, args.warmup,
+                                 with_e2e=False, with_cpu=not args.no_cpu_baseline)
+            out[key] = {k: sub[k] for k in SUB_KEYS if k in sub}
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
@@ -822,9 +885,10 @@ def run_reference_streaming(args, cfg, world):
 
 
 def run_reference(args):
-    """The float64 oracle on the host cores: each step times one bounded
-    sample of the workload; the reported rate is the stage-weighted
-    extrapolation to the full step."""
+    """The float64 oracle on the host cores. Each step times one bounded
+    sample of the workload (``ms_per_step`` is that sample's wall time); the
+    reported rate is the stage-weighted extrapolation of the sampled rates to
+    the full step (its duration in ``full_step_s_extrapolated``)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -836,24 +900,29 @@ def run_reference(args):
     work = step_work(cfg)
     total = sum(work.values())
     acc = {s: [0.0, 0.0] for s in work}
+    wall = []
     for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
         timing = oracle_timing(cfg)
         if i >= args.warmup:
+            wall.append(time.perf_counter() - t0)
             for s in acc:
                 acc[s][0] += timing[s][0]
                 acc[s][1] += timing[s][1]
-    t_full = sum(work[s] * acc[s][1] / acc[s][0] for s in work) / 1.0
-    t_full_step = t_full  # seconds per full step at the sampled rates
-    value = total / t_full_step / 1e12
+    t_full = sum(work[s] * acc[s][1] / acc[s][0] for s in work if acc[s][0] > 0)
+    value = total / t_full / 1e12
     cores, blas = cpu_cores()
     sample = (f"per step: float64 oracle on 256 query rows of the last chunk for one head (all "
               f"keys), the Gram and direct error of 1024 rows, one full {cfg.d}x{cfg.d} solve; "
               f"rates extrapolated stage by stage to the full step")
+    K = cfg.select_k if cfg.select_k is not None else cfg.layers // 2
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-           "ms_per_step": t_full_step * 1e3, "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": cfg.name, "d": cfg.d, "layers": cfg.layers},
+           "ms_per_step": sum(wall) / len(wall) * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": config_of(cfg, 1, False, K),
+           "step_is": "a bounded sample of the workload (see cpu_baseline.sample)",
+           "full_step_s_extrapolated": round(t_full, 3),
            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas or cores,
                             "kind": "oracle", "sample": sample},
            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -864,15 +933,17 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--config", choices=("c1", "c2", "c3", "c4"), default="c1")
+    ap.add_argument("--config", choices=("c1", "c2", "c3", "c4"), default="c2")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the workload's layer count (smaller captures for ncu)")
     ap.add_argument("--slots", type=int, default=2,
                     help="layers in flight on separate streams in a multi-layer warmup")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sub", action="store_true",
+                    help="measure only the main workload (no 14B / single-chunk sub-objects)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--measure-tf32-peak", action="store_true",
