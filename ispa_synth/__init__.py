@@ -34,7 +34,7 @@ from __future__ import annotations
 
 import dataclasses
 import math
-from typing import List, Optional
+from typing import List, Optional, Tuple
 
 import torch
 
@@ -60,6 +60,16 @@ class Config:
     rho: float = 0.9
     select_k: Optional[int] = None  # layers turned local (lowest error)
     stream_chunks: int = 0    # post-transition chunks (streaming workload)
+    # Ranking-stress variant: layer l draws with its own correlation, spread
+    # evenly over [lo, hi] in the scrambled order (7 l mod L), so that the
+    # layers' errors separate and the ranking is not the layer order.
+    rho_spread: Optional[Tuple[float, float]] = None
+
+    def rho_of(self, layer: int) -> float:
+        if self.rho_spread is None or self.layers < 2:
+            return self.rho
+        lo, hi = self.rho_spread
+        return lo + (hi - lo) * ((7 * layer) % self.layers) / (self.layers - 1)
 
     @property
     def d(self) -> int:
@@ -102,7 +112,12 @@ C3 = Config("14B-warmup", layers=40, heads=40, head_dim=128, tokens_per_frame=15
 C4 = Config("1.3B-stream", layers=30, heads=12, head_dim=128, tokens_per_frame=1560,
             sink_tokens=1560, chunk_frames=3, first_chunk_frame=1, n_chunks=4,
             history_window=None, select_k=15, stream_chunks=17)
-CONFIGS = {"c0": C0, "c1": C1, "c2": C2, "c3": C3, "c4": C4}
+# Addition to the five: the 1.3B warmup with per-layer correlations spread
+# over [0.5, 0.95] (ranking-stress variant; not one of the five workloads).
+C2R = Config("1.3B-warmup-rho-spread", layers=30, heads=12, head_dim=128, tokens_per_frame=1560,
+             sink_tokens=1560, chunk_frames=3, first_chunk_frame=1, n_chunks=4,
+             history_window=None, select_k=15, rho_spread=(0.5, 0.95))
+CONFIGS = {"c0": C0, "c1": C1, "c2": C2, "c3": C3, "c4": C4, "c2r": C2R}
 
 
 def scaled(cfg: Config, **kw) -> Config:
@@ -171,7 +186,8 @@ def layer_streams(cfg: Config, layer: int, seed: int = 0, device="cpu",
                   n_frames: Optional[int] = None) -> LayerStreams:
     nf = cfg.n_frames if n_frames is None else n_frames
     shape = (nf, cfg.tokens_per_frame, cfg.heads, cfg.head_dim)
-    mk = lambda t: ar1_stream(nf, cfg.tokens_per_frame, cfg.d, cfg.rho, seed, layer, t,
+    rho = cfg.rho_of(layer)
+    mk = lambda t: ar1_stream(nf, cfg.tokens_per_frame, cfg.d, rho, seed, layer, t,
                               device).reshape(shape)
     return LayerStreams(cfg, mk("Q"), mk("K"), mk("V"), projection(cfg.d, seed, layer, device))
 
@@ -207,3 +223,16 @@ def attention_like(rows: int, dim: int, seed: int, rho: float = 0.9, common: flo
         for i in range(1, rows):
             out[i] = rho * out[i - 1] + innov * z[i]
     return (out * 0.1 + mean).contiguous()
+
+
+SKETCH_SEED = 977
+
+
+def sketch_matrices(n_rows: int, dim: int, k: int = 16):
+    """Fixed Gaussian test matrices for comparing large results through small
+    two-sided sketches X -> L^T X R (E ||L^T X R||_F^2 = k^2 ||X||_F^2 for
+    N(0, 1) entries). Returns (rows [n_rows, k], left [dim, k], right [dim, k])
+    in float32, identical on every machine (CPU generator)."""
+    return (gaussian((n_rows, k), SKETCH_SEED, 0, "X"),
+            gaussian((dim, k), SKETCH_SEED, 1, "X"),
+            gaussian((dim, k), SKETCH_SEED, 2, "X"))
