@@ -251,6 +251,166 @@ __device__ __forceinline__ uint4 bf16x8_to_half(uint4 x, uint32_t& big) {
   return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
+// VEC consecutive fp32 values (VEC = 2 or 4) through L2 (slots written by
+// other SMs in this launch).
+template <int VEC>
+__device__ __forceinline__ void ld_vec(const float* src, float (&v)[VEC]) {
+  if constexpr (VEC == 4) {
+    const float4 x = __ldcg(reinterpret_cast<const float4*>(src));
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else {
+    const float2 x = __ldcg(reinterpret_cast<const float2*>(src));
+    v[0] = x.x; v[1] = x.y;
+  }
+}
+template <int VEC>
+__device__ __forceinline__ void st_vec(float* dst, const float (&v)[VEC], bool tf32) {
+  if constexpr (VEC == 4) {
+    *reinterpret_cast<float4*>(dst) = tf32 ? make_float4(to_tf32(v[0]), to_tf32(v[1]),
+                                                         to_tf32(v[2]), to_tf32(v[3]))
+                                           : make_float4(v[0], v[1], v[2], v[3]);
+  } else {
+    *reinterpret_cast<float2*>(dst) = tf32 ? make_float2(to_tf32(v[0]), to_tf32(v[1]))
+                                           : make_float2(v[0], v[1]);
+  }
+}
+template <int VEC>
+__device__ __forceinline__ void st_vec_bf16(__nv_bfloat16* dst, const float (&v)[VEC]) {
+  __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]);
+  if constexpr (VEC == 4) {
+    __nv_bfloat162 b1 = __floats2bfloat162_rn(v[2], v[3]);
+    *reinterpret_cast<uint2*>(dst) =
+        make_uint2(*reinterpret_cast<uint32_t*>(&b0), *reinterpret_cast<uint32_t*>(&b1));
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = *reinterpret_cast<uint32_t*>(&b0);
+  }
+}
+
+// The LSE merge of one (head, query pair) by the unit that finished last.
+// Row rr of the pair is merged by epilogue warp rr / G mod (warps), each lane
+// holding VEC consecutive columns; the unit's own slot comes from `stage`
+// (what its slot holds, row stride HD + 4), the others from L2, G rows per
+// warp at a time so that their loads are in flight together. With w_s =
+// e^(LSE_s - LSE_loc) over the local slots and e^(LSE_s - LSE_full) over the
+// history slots: A_loc = sum_local w_s O_s (a single local slot as stored),
+// D = sum_hist w_s (O_s - A_loc), A_full = A_loc + D. Slots are summed in
+// slot order, so the result does not depend on which unit came last.
+template <int HD>
+__device__ __forceinline__ void merge_rows(const AttnParams& p, const Unit& u, const float* stage,
+                                           const float* stats, int n_epi) {
+  constexpr int VEC = HD / 32;
+  constexpr int G = 8;
+  constexpr int kLd = HD + 4;
+  const int n_warps = n_epi / 32;
+  const int ew = (int)(threadIdx.x - 128) / 32;
+  const int lane = threadIdx.x % 32;
+  const int n_ls = p.plan.n_ls, ns = p.plan.n_slots();
+  const int64_t d = (int64_t)p.heads * HD;
+  const bool rnd = p.round_tf32 != 0;
+  const int rows = p.nq - u.q0 < u.n_qt * BM ? p.nq - u.q0 : u.n_qt * BM;
+  for (int r0 = ew * G; r0 < rows; r0 += n_warps * G) {
+    float al[G][VEC], acc[G][VEC], x[G][VEC];
+    int64_t off[G], li[G];
+    bool ok[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const int rr = r0 + g;
+      ok[g] = rr < rows;
+      const int row = u.q0 + (ok[g] ? rr : 0);
+      off[g] = (int64_t)row * d + (int64_t)u.head * HD + lane * VEC;
+      li[g] = (int64_t)u.head * p.nq + row;
+    }
+    // A_loc
+    if (n_ls == 1 && u.slot == 0) {
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) al[g][i] = stage[(r0 + g) * kLd + lane * VEC + i];
+    } else if (n_ls == 1) {
+      const float* src = slot_out(p, 0);
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+        if (ok[g]) ld_vec<VEC>(src + off[g], al[g]);
+    } else {
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) al[g][i] = 0.f;
+      for (int k = 0; k < n_ls; ++k) {
+        float w[G];
+        if (k == u.slot) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            w[g] = ok[g] ? __ldcg(p.part_lse + k * p.lse_stride + li[g]) : 0.f;
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) x[g][i] = stage[(r0 + g) * kLd + lane * VEC + i];
+          }
+        } else {
+          const float* src = slot_out(p, k);
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            w[g] = ok[g] ? __ldcg(p.part_lse + k * p.lse_stride + li[g]) : 0.f;
+            if (ok[g]) ld_vec<VEC>(src + off[g], x[g]);
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float wg = ok[g] ? expf(w[g] - stats[2 * (r0 + g)]) : 0.f;
+#pragma unroll
+          for (int i = 0; i < VEC; ++i) al[g][i] = fmaf(wg, ok[g] ? x[g][i] : 0.f, al[g][i]);
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        if (rnd) {
+#pragma unroll
+          for (int i = 0; i < VEC; ++i) al[g][i] = to_tf32(al[g][i]);
+        }
+        if (ok[g] && p.a_loc) st_vec<VEC>(p.a_loc + off[g], al[g], false);
+      }
+    }
+    // D = A_full - A_loc
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) acc[g][i] = 0.f;
+    for (int k = n_ls; k < ns; ++k) {
+      float w[G];
+      if (k == u.slot) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          w[g] = ok[g] ? __ldcg(p.part_lse + k * p.lse_stride + li[g]) : 0.f;
+#pragma unroll
+          for (int i = 0; i < VEC; ++i) x[g][i] = stage[(r0 + g) * kLd + lane * VEC + i];
+        }
+      } else {
+        const float* src = slot_out(p, k);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          w[g] = ok[g] ? __ldcg(p.part_lse + k * p.lse_stride + li[g]) : 0.f;
+          if (ok[g]) ld_vec<VEC>(src + off[g], x[g]);
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float wg = ok[g] ? expf(w[g] - stats[2 * (r0 + g) + 1]) : 0.f;
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) acc[g][i] = fmaf(wg, (ok[g] ? x[g][i] : 0.f) - al[g][i], acc[g][i]);
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      if (!ok[g]) continue;
+      if (p.d_out) st_vec<VEC>(p.d_out + off[g], acc[g], rnd);
+      if (p.a_full) {
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) x[g][i] = al[g][i] + acc[g][i];
+        st_vec_bf16<VEC>(p.a_full + off[g], x[g]);
+      }
+    }
+  }
+}
+
 template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
 branch_attention_kernel(const __grid_constant__ AttnParams p) {
@@ -551,9 +711,33 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
         epi_barrier(n_epi);
         if (s.merge) {
           __threadfence();
+          // (a) each row thread stages its own normalised output exactly as
+          // its slot holds it (the operand rings are idle once o_final has
+          // completed), merges the row's LSEs and writes them
+          constexpr int kLd = HD + 4;                 // padded: conflict-free float4 rows
+          float* stage = reinterpret_cast<float*>(&s.q[0][0][0]);
+          float* stats = stage + NQT * BM * kLd;       // per row: LSE_loc, LSE_full
+          const int rr = t * BM + r;
+#pragma unroll 1
+          for (int c = 0; c < HD / 16; ++c) {
+            uint32_t raw[16];
+            tmem_ld16(to + c * 16, raw);
+            tmem_ld_wait();
+            float4* s4 = reinterpret_cast<float4*>(stage + rr * kLd + c * 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              float4 x = make_float4(__uint_as_float(raw[4 * i]) * inv,
+                                     __uint_as_float(raw[4 * i + 1]) * inv,
+                                     __uint_as_float(raw[4 * i + 2]) * inv,
+                                     __uint_as_float(raw[4 * i + 3]) * inv);
+              if (own_rnd) x = make_float4(to_tf32(x.x), to_tf32(x.y), to_tf32(x.z), to_tf32(x.w));
+              s4[i] = x;
+            }
+          }
           const int n_ls = p.plan.n_ls;
           float lse_loc = -INFINITY, lse_hist = -INFINITY;
           if (row_ok) {
+#pragma unroll 4
             for (int k = 0; k < n_slots; ++k) {
               const float v = __ldcg(p.part_lse + k * p.lse_stride + li);
               if (k < n_ls) lse_loc = log_add_exp(lse_loc, v);
@@ -561,75 +745,18 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
             }
           }
           const float lse_full = log_add_exp(lse_loc, lse_hist);
-          const bool rnd = p.round_tf32 != 0;
-#pragma unroll 1
-          for (int c = 0; c < HD / 16; ++c) {
-            uint32_t raw[16];
-            tmem_ld16(to + c * 16, raw);
-            tmem_ld_wait();
-            if (!row_ok) continue;
-            float mine[16], al[16], dd[16], x[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              mine[i] = __uint_as_float(raw[i]) * inv;
-              if (own_rnd) mine[i] = to_tf32(mine[i]);   // exactly what the slot holds
-            }
-            const int64_t off = base + c * 16;
-            // A_loc: the local slots merged (a single local slot as stored)
-            if (n_ls == 1) {
-              if (u.slot == 0) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) al[i] = mine[i];
-              } else {
-                load_f32x16(slot_out(p, 0) + off, al);
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) al[i] = 0.f;
-              for (int k = 0; k < n_ls; ++k) {
-                const float w = expf(__ldcg(p.part_lse + k * p.lse_stride + li) - lse_loc);
-                if (k == u.slot) {
-#pragma unroll
-                  for (int i = 0; i < 16; ++i) x[i] = mine[i];
-                } else {
-                  load_f32x16(slot_out(p, k) + off, x);
-                }
-#pragma unroll
-                for (int i = 0; i < 16; ++i) al[i] = fmaf(w, x[i], al[i]);
-              }
-              if (rnd) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) al[i] = to_tf32(al[i]);
-              }
-              if (p.a_loc) store_f32x16(p.a_loc + off, al, false);
-            }
-            // D = A_full - A_loc = sum over history slots of w (O - A_loc)
-#pragma unroll
-            for (int i = 0; i < 16; ++i) dd[i] = 0.f;
-            for (int k = n_ls; k < n_slots; ++k) {
-              const float w = expf(__ldcg(p.part_lse + k * p.lse_stride + li) - lse_full);
-              if (k == u.slot) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) x[i] = mine[i];
-              } else {
-                load_f32x16(slot_out(p, k) + off, x);
-              }
-#pragma unroll
-              for (int i = 0; i < 16; ++i) dd[i] = fmaf(w, x[i] - al[i], dd[i]);
-            }
-            if (p.d_out) store_f32x16(p.d_out + off, dd, rnd);
-            if (p.a_full) {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) x[i] = al[i] + dd[i];
-              store_bf16x16(p.a_full + off, x);
-            }
-          }
+          stats[2 * rr] = lse_loc;
+          stats[2 * rr + 1] = lse_full;
           if (row_ok) {
             if (p.lse_loc) p.lse_loc[li] = lse_loc;
             if (p.lse_hist) p.lse_hist[li] = lse_hist;
             if (p.lse_full) p.lse_full[li] = lse_full;
           }
           nonfinite = row_ok && !finite_f(lse_full);
+          epi_barrier(n_epi);
+          // (b) every epilogue warp merges whole rows of the pair: coalesced
+          // loads of the other slots, several rows in flight a warp
+          merge_rows<HD>(p, u, stage, stats, n_epi);
         }
       }
       if (__any_sync(0xffffffffu, nonfinite) && lane == 0) atomicOr(p.status, ISPA_STATUS_NONFINITE);
@@ -665,7 +792,11 @@ int64_t attention_key_tiles(int64_t len) { return (len + BN - 1) / BN; }
 
 namespace {
 
-constexpr double kUnitCost = 2.0;   // key-tile steps
+// Fitted to measured calls of the 1.3B and 14B chunk shapes under forced
+// split counts (one unit costs about ten key-tile steps beyond its tiles:
+// prologue, epilogue, slot write and merge); it picks the fastest measured
+// plan of every shape to within 1%.
+constexpr double kUnitCost = 10.0;   // key-tile steps
 constexpr int kPlanSms = 148;
 
 std::atomic<int> g_force_ls{0}, g_force_hs{0};
