@@ -468,6 +468,32 @@ def measure_warmup(args, cfg, world, rank, steps, warmup, with_e2e, with_cpu):
     per_step = L_mine * cfg.n_chunks
     solve_ms = sum(ev["g1"][(i + 1) * per_step - 1].elapsed_time(ev["s1"][i])
                    for i in range(n_inst)) / n_inst
+    # the attention calls alone, with the layers in flight on the step's streams
+    # (the concurrency the timed step runs them at; no Gram, solve or error)
+    def attention_pass():
+        n_s = len(streams)
+        fork = torch.cuda.Event()
+        fork.record(streams[0])
+        for s_ in streams[1:]:
+            s_.wait_event(fork)
+        for li, chunks in enumerate(chunks_per_layer):
+            for ch in chunks:
+                runner.attention(ch, stream=streams[li % n_s], slot=li % n_s)
+        for s_ in streams[1:]:
+            join = torch.cuda.Event()
+            join.record(s_)
+            streams[0].wait_event(join)
+
+    attention_pass()
+    torch.cuda.synchronize()
+    a0, a1 = E(), E()
+    flush.zero_()
+    a0.record(streams[0])
+    for _ in range(n_inst):
+        attention_pass()
+    a1.record(streams[0])
+    torch.cuda.synchronize()
+    attn_streams_ms = a0.elapsed_time(a1) / n_inst
     status = ispa.read_status(runner.status)
     step_ms_max = max_over_ranks(step_ms, world)
 
@@ -503,6 +529,12 @@ def measure_warmup(args, cfg, world, rank, steps, warmup, with_e2e, with_cpu):
         "attention_tflops": round(attn_tflops, 2),
         "attention_frac_of_bf16_peak": round(attn_tflops / bf16_peak, 4),
         "attention_ms_per_step": round(attn_ms, 4),
+        # as the step runs them: layers in flight on the step's streams
+        "attention_tflops_layers_in_flight": round(work["attention"] * share
+                                                   / (attn_streams_ms * 1e-3) / 1e12, 2),
+        "attention_frac_layers_in_flight": round(work["attention"] * share
+                                                 / (attn_streams_ms * 1e-3) / 1e12 / bf16_peak, 4),
+        "attention_streams": len(streams),
         "absorb_ms_per_layer": round(absorb_ms_layer, 4),
         "gram_ms_per_step": round(gram_ms, 4), "solve_error_ms_per_step": round(solve_ms, 4),
         "absorb_tflops": round(absorb_flops / ((gram_ms + solve_ms) * 1e-3) / 1e12, 2),
@@ -536,7 +568,8 @@ def attention_bytes(cfg):
 
 SUB_WORKLOADS = (("14B-warmup", "c3"), ("1.3B-chunk", "c1"))
 SUB_KEYS = ("value", "unit", "ms_per_step", "steps", "warmup", "config", "attention_tflops",
-            "attention_frac_of_bf16_peak", "attention_ms_per_step", "absorb_ms_per_layer",
+            "attention_frac_of_bf16_peak", "attention_ms_per_step",
+            "attention_tflops_layers_in_flight", "attention_frac_layers_in_flight", "absorb_ms_per_layer",
             "gram_ms_per_step", "solve_error_ms_per_step", "absorb_tflops", "roofline",
             "absorb_roofline", "gpu_launches", "device_status", "clocks", "cpu_baseline")
 
