@@ -286,6 +286,35 @@ __device__ __forceinline__ void st_vec_bf16(__nv_bfloat16* dst, const float (&v)
   }
 }
 
+// Coalesced stores of a warp's rows. Each thread holds 32 consecutive values
+// of its row (row0 + lane); they are staged in shared memory (32 rows x 36
+// floats a warp: the padding makes the float4 writes of 32 rows and the row
+// reads conflict-free) and written back row by row, each row with one
+// 128-byte warp store. Destinations point at this block's first row and
+// column in row-major [nq, d] matrices (row stride d elements); any may be
+// null. The fp32 copy is optionally rounded to tf32; the bf16 copy is
+// rounded from the unrounded value; `zero` receives zeros. Rows >= nq are
+// skipped.
+__device__ __forceinline__ void rows_out(float* st, const float (&v)[32], int row0, int nq,
+                                         int64_t d, float* f32, bool f32_round,
+                                         __nv_bfloat16* bf16, float* zero) {
+  const int lane = threadIdx.x % 32;
+  float4* w = reinterpret_cast<float4*>(st + lane * 36);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  __syncwarp();
+  const int n = nq - row0 < 32 ? nq - row0 : 32;
+#pragma unroll 4
+  for (int i = 0; i < n; ++i) {
+    const float x = st[i * 36 + lane];
+    const int64_t o = (int64_t)i * d + lane;
+    if (f32) f32[o] = f32_round ? to_tf32(x) : x;
+    if (bf16) bf16[o] = __float2bfloat16_rn(x);
+    if (zero) zero[o] = 0.f;
+  }
+  __syncwarp();   // the block is read before the next one overwrites it
+}
+
 // The LSE merge of one (head, query pair) by the unit that finished last.
 // Row rr of the pair is merged by epilogue warp rr / G mod (warps), each lane
 // holding VEC consecutive columns; the unit's own slot comes from `stage`
@@ -657,25 +686,24 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
       const float inv = 1.f / l;
       const int n_slots = p.plan.n_slots();
       bool nonfinite = false;
+      // per-warp staging block for the coalesced stores (the operand rings are
+      // idle once o_final has completed)
+      float* wst = reinterpret_cast<float*>(&s.q[0][0][0]) + (warp - 4) * 32 * 36;
+      const int wrow0 = u.q0 + t * BM + quarter * 32;       // first row of this warp
+      const int64_t wbase = (int64_t)wrow0 * d + (int64_t)u.head * HD;
       if (n_slots == 1) {
         // one local range and no history: write the final outputs directly
 #pragma unroll 1
-        for (int c = 0; c < HD / 16; ++c) {
-          uint32_t raw[16];
-          tmem_ld16(to + c * 16, raw);
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t raw[32];
+          tmem_ld32(to + c * 32, raw);
           tmem_ld_wait();
-          if (!row_ok) continue;
-          float a[16];
+          float a[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) a[i] = __uint_as_float(raw[i]) * inv;
-          if (p.a_loc) store_f32x16(p.a_loc + base + c * 16, a, p.round_tf32 != 0);
-          if (p.a_full) store_bf16x16(p.a_full + base + c * 16, a);
-          if (p.d_out) {
-            float z[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) z[i] = 0.f;
-            store_f32x16(p.d_out + base + c * 16, z, false);
-          }
+          for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(raw[i]) * inv;
+          rows_out(wst, a, wrow0, p.nq, d, p.a_loc ? p.a_loc + wbase + c * 32 : nullptr,
+                   p.round_tf32 != 0, p.a_full ? p.a_full + wbase + c * 32 : nullptr,
+                   p.d_out ? p.d_out + wbase + c * 32 : nullptr);
         }
         if (row_ok) {
           if (p.lse_loc) p.lse_loc[li] = lse;
@@ -689,15 +717,14 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
         const bool own_rnd = u.slot < p.part_first && p.round_tf32 != 0;
         float* own = slot_out(p, u.slot);
 #pragma unroll 1
-        for (int c = 0; c < HD / 16; ++c) {
-          uint32_t raw[16];
-          tmem_ld16(to + c * 16, raw);
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t raw[32];
+          tmem_ld32(to + c * 32, raw);
           tmem_ld_wait();
-          if (!row_ok) continue;
-          float a[16];
+          float a[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) a[i] = __uint_as_float(raw[i]) * inv;
-          store_f32x16(own + base + c * 16, a, own_rnd);
+          for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(raw[i]) * inv;
+          rows_out(wst, a, wrow0, p.nq, d, own + wbase + c * 32, own_rnd, nullptr, nullptr);
         }
         if (row_ok) p.part_lse[u.slot * p.lse_stride + li] = lse;
         // 2. count this unit finished; the last of the (head, pair) merges
