@@ -49,6 +49,13 @@ namespace ispa {
 namespace {
 
 constexpr int NB = 128;
+
+// Waits with the full limit and no abort flag: the waits that let issued
+// copies and tensor-core operations land before their memory is reused.
+__device__ __forceinline__ void drain_wait_step(uint64_t* bar, uint32_t parity, int* status) {
+  int dummy = 0;
+  mbar_wait(bar, parity, status, &dummy);
+}
 // Long-K products accumulate K = 128 per tensor-core accumulator and sum the
 // chunks in fp32 (see tgemm.cu).
 constexpr int kChunkSlabs = 4;
@@ -80,20 +87,36 @@ __global__ void lambda_kernel(const float* __restrict__ M0, int64_t m_stride, in
 }
 
 // A = G + lambda I as a full symmetric matrix (G's 128 x 128 tiles are valid
-// on and above the tile diagonal; the rest is mirrored), Z = I; layer blockIdx.y.
-__global__ void build_kernel(const float* __restrict__ M0, int64_t m_stride, int dim,
-                             float* __restrict__ ws0, int64_t ws_stride, int64_t lam_off) {
-  const size_t n = (size_t)dim * dim;
+// on and above the tile diagonal; the rest is mirrored), Z = I; layer
+// blockIdx.y. Tiles of 32 x 32: a mirrored tile is read row by row and
+// transposed through shared memory, so that reads and writes stay coalesced.
+__global__ void __launch_bounds__(256) build_kernel(const float* __restrict__ M0, int64_t m_stride,
+                                                    int dim, float* __restrict__ ws0,
+                                                    int64_t ws_stride, int64_t lam_off) {
+  __shared__ float tile[32][33];
   const float* M = M0 + (int64_t)blockIdx.y * m_stride;
   float* A = ws0 + (int64_t)blockIdx.y * ws_stride;
-  float* Z = A + n;
+  float* Z = A + (size_t)dim * dim;
   const float l = A[lam_off];
-  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n;
-       e += (size_t)gridDim.x * blockDim.x) {
-    const int i = (int)(e / dim), j = (int)(e % dim);
-    const float g = (i / 128 <= j / 128) ? M[(size_t)i * 2 * dim + j] : M[(size_t)j * 2 * dim + i];
-    A[e] = (i == j) ? g + l : g;
-    Z[e] = (i == j) ? 1.f : 0.f;
+  const int nt = dim / 32, tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 8 rows of 32
+  for (int b = blockIdx.x; b < nt * nt; b += gridDim.x) {
+    const int bi = b / nt, bj = b % nt, i0 = 32 * bi, j0 = 32 * bj;
+    const bool direct = (i0 / 128) <= (j0 / 128);
+    __syncthreads();   // the previous tile's reads of `tile` are done
+#pragma unroll
+    for (int r = ty; r < 32; r += 8) {
+      // direct: row i0 + r of the tile; mirrored: row j0 + r of G's tile (j, i)
+      tile[r][tx] = direct ? M[(size_t)(i0 + r) * 2 * dim + j0 + tx]
+                           : M[(size_t)(j0 + r) * 2 * dim + i0 + tx];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = ty; r < 32; r += 8) {
+      const int i = i0 + r, j = j0 + tx;
+      const float g = direct ? tile[r][tx] : tile[tx][r];
+      A[(size_t)i * dim + j] = (i == j) ? g + l : g;
+      Z[(size_t)i * dim + j] = (i == j) ? 1.f : 0.f;
+    }
   }
 }
 
@@ -141,33 +164,18 @@ __device__ __forceinline__ void st4(float* d, const float* s) {
   *reinterpret_cast<float4*>(d) = make_float4(s[0], s[1], s[2], s[3]);
 }
 
-__global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restrict__ A0, int lda,
-                                                           float* __restrict__ linv0,
-                                                           int64_t ws_stride, int* status) {
-  const float* A = A0 + (int64_t)blockIdx.x * ws_stride;    // one block per layer
-  float* linv = linv0 + (int64_t)blockIdx.x * ws_stride;
-  extern __shared__ __align__(16) float sh[];
-  float* a = sh;
-  float* z = a + NB * kSA;
-  float* pl = z + NB * kSA;
-  float* plT = pl + 96 * kSP;
-  float* ljt = plT + 32 * kST;                 // L_JJ, column-major (row c = column c)
-  float* rinv = ljt + 32 * kSI;                 // 1 / diagonal of L_JJ
-  // rows of L_JJ in one column group (row i: L[i][j0 .. j0+3]); rows 32..63 stay zero
-  float4* grp = reinterpret_cast<float4*>(rinv + 32);
+// The factor and inverse of steps (1)-(3) above on the block in shared
+// memory: a (lower triangle) is factored in place and z (= I on entry)
+// becomes L^-1, zero above the diagonal. on_idle(J) runs on warps 1-15 once
+// their part of step J's trailing update is done, while warp 0 brings up and
+// factors sub-block J: a hook for the caller's own work, which must leave
+// alone what step J reads (for J = 0: rows and columns 0-31 of a, ljt,
+// rinv, grp). Ends with a barrier.
+template <class Idle>
+__device__ __forceinline__ void factor_invert(float* a, float* z, float* pl, float* plT,
+                                              float* ljt, float* rinv, float4* grp, int* status,
+                                              Idle&& on_idle) {
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  if (t < 64) grp[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-  pdl_wait();       // the update that wrote this block has completed
-  pdl_trigger();
-  for (int e = t; e < NB * (NB / 4); e += blockDim.x) {
-    const int i = e >> 5, c = (e & 31) * 4;
-    *reinterpret_cast<float4*>(&a[i * kSA + c]) =
-        __ldg(reinterpret_cast<const float4*>(A + (size_t)i * lda + c));
-    *reinterpret_cast<float4*>(&z[i * kSA + c]) =
-        make_float4(i == c ? 1.f : 0.f, i == c + 1 ? 1.f : 0.f, i == c + 2 ? 1.f : 0.f,
-                    i == c + 3 ? 1.f : 0.f);
-  }
-  __syncthreads();
   // warp 0: L_JJ of the 32 x 32 diagonal sub-block at J (see step (1) above)
   auto factor32 = [&](int J) {
     {
@@ -296,6 +304,7 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
         }
       }
     }
+    if (warp != 0) on_idle(J);                 // warps 1-15, their part of (3) done
     __syncthreads();
     // ---- (2) forward substitution with L_JJ, one 32-vector per thread: the
     // panel rows (x L_JJ^T = a, i.e. L_JJ x^T = a^T) and the columns of the
@@ -333,21 +342,289 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
     }
     __syncthreads();
   }
-  for (int e = t; e < NB * (NB / 4); e += blockDim.x) {
+}
+
+// Writes rows [i0, i1) of L^-1 (z) to linv in fp32, zero above the diagonal,
+// then its tf32 planes: hi = tf32(v), lo = tf32(v - hi), rounded as the
+// GEMM's in-kernel split rounds them.
+__device__ __forceinline__ void store_linv(const float* z, float* linv, int i0 = 0, int i1 = NB) {
+  const int t = threadIdx.x;
+  for (int e = i0 * (NB / 4) + t; e < i1 * (NB / 4); e += blockDim.x) {
     const int i = e >> 5, c = (e & 31) * 4;
     float v[4];
     ld4(v, &z[i * kSA + c]);
 #pragma unroll
     for (int c4 = 0; c4 < 4; ++c4) v[c4] = (c + c4 <= i) ? v[c4] : 0.f;
     st4(&linv[(size_t)i * NB + c], v);
-    // the planes the panel products read: hi = tf32(v), lo = tf32(v - hi),
-    // rounded as the GEMM's in-kernel split rounds them
     float h[4], l[4];
 #pragma unroll
     for (int c4 = 0; c4 < 4; ++c4) { h[c4] = to_tf32(v[c4]); l[c4] = to_tf32(v[c4] - h[c4]); }
     st4(&linv[NB * NB + (size_t)i * NB + c], h);
     st4(&linv[2 * NB * NB + (size_t)i * NB + c], l);
   }
+}
+
+__global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restrict__ A0, int lda,
+                                                           float* __restrict__ linv0,
+                                                           int64_t ws_stride, int* status) {
+  const float* A = A0 + (int64_t)blockIdx.x * ws_stride;    // one block per layer
+  float* linv = linv0 + (int64_t)blockIdx.x * ws_stride;
+  extern __shared__ __align__(16) float sh[];
+  float* a = sh;
+  float* z = a + NB * kSA;
+  float* pl = z + NB * kSA;
+  float* plT = pl + 96 * kSP;
+  float* ljt = plT + 32 * kST;                 // L_JJ, column-major (row c = column c)
+  float* rinv = ljt + 32 * kSI;                 // 1 / diagonal of L_JJ
+  // rows of L_JJ in one column group (row i: L[i][j0 .. j0+3]); rows 32..63 stay zero
+  float4* grp = reinterpret_cast<float4*>(rinv + 32);
+  const int t = threadIdx.x;
+  if (t < 64) grp[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+  pdl_wait();       // the update that wrote this block has completed
+  pdl_trigger();
+  for (int e = t; e < NB * (NB / 4); e += blockDim.x) {
+    const int i = e >> 5, c = (e & 31) * 4;
+    *reinterpret_cast<float4*>(&a[i * kSA + c]) =
+        __ldg(reinterpret_cast<const float4*>(A + (size_t)i * lda + c));
+    *reinterpret_cast<float4*>(&z[i * kSA + c]) =
+        make_float4(i == c ? 1.f : 0.f, i == c + 1 ? 1.f : 0.f, i == c + 2 ? 1.f : 0.f,
+                    i == c + 3 ? 1.f : 0.f);
+  }
+  __syncthreads();
+  factor_invert(a, z, pl, plT, ljt, rinv, grp, status, [](int) {});
+  store_linv(z, linv);
+}
+
+constexpr int kSlice = 32;                   // rows of the block column a step CTA finishes
+// shared memory of the step kernel: the factor's, then S [32][kSA], then the
+// barriers and the tensor-memory address
+constexpr size_t kStepSlice = kPotrfSmem;
+constexpr size_t kStepBars = kStepSlice + kSlice * kSA * sizeof(float);
+constexpr size_t kStepSmem = kStepBars + 64;
+// the previous step's panel, staged for the tensor cores while z, pl and plT
+// are still free: per 32-deep slab of K, the hi plane then the lo plane, each
+// L_{k,k-1} (128 rows) followed by L_{S,k-1} (32 rows), 128-byte rows in
+// 128-byte swizzle (the TMA boxes' layout); two slabs in flight
+constexpr uint32_t kBoxLp = 128 * 32 * 4, kBoxLs = kSlice * 32 * 4;
+constexpr uint32_t kStagePlane = kBoxLp + kBoxLs, kStageBytes = 2 * kStagePlane;
+constexpr size_t kOffZ = NB * kSA * sizeof(float);
+constexpr size_t kOffLjt = 2 * NB * kSA * sizeof(float) + (96 * kSP + 32 * kST) * sizeof(float);
+static_assert(kOffZ + 1023 + 2 * kStageBytes <= kOffLjt,
+              "the staging area (z aligned up to 1 KB) must end before L_JJ");
+
+struct StepParams {
+  CUtensorMap lp_hi, lp_lo;   // A's tf32 hi / lo planes, 32 x 128 boxes
+  CUtensorMap ls_hi, ls_lo;   // the same planes, 32 x 32 boxes
+  float* A;                   // fp32 working matrix, row stride d
+  float* Ah;                  // hi plane (lo = Ah + plane)
+  int64_t plane;
+  int d, kk;
+  float* linv;                // this step's slot: Linv, then its hi / lo planes
+  int* status;
+  uint64_t wait_ns;
+};
+
+// Step k of the one-layer sweep, the part on its critical path (diagonal
+// block at kk = 128 k, m = d - kk - 128 rows below it). CTA b owns the rows
+// r0 = kk + 128 + 32 b .. r0 + 31 of block column k (one CTA when m = 0):
+//  (1) it applies the previous step's update to the diagonal block A_kk and
+//      to its slice S = A[r0.., kk..]:
+//          [A_kk | S^T] -= L_{k,k-1} [L_{k,k-1} ; L_{S,k-1}]^T,
+//      a 128 x 160 x 128 product on the tensor cores (3xTF32 from the hi/lo
+//      planes the previous step wrote, fp32 accumulation in tensor memory),
+//      while the CTA's threads load A_kk and S (fp32);
+//  (2) it factors A_kk and forms Linv = L_kk^-1 (factor_invert): every CTA
+//      does the same arithmetic on the same data, so all hold the same Linv;
+//  (3) it forms its slice of the panel, L_{S,k} = S Linv^T (fp32), and
+//      stores it as tf32 hi/lo planes in Ah, where this step's products and
+//      the next step's update read it;
+// The CTAs also write Linv with its planes to this step's slot, each a share
+// of its rows, where the products forming block rows k of Z and Y read it. No CTA waits for another:
+// the block factor is repeated instead of shared. Updates of block column k
+// by steps before k - 1 are applied beforehand by the trailing products.
+__global__ void __launch_bounds__(512, 1) sweep_step_kernel(const __grid_constant__ StepParams p) {
+  extern __shared__ __align__(16) float sh[];
+  uint8_t* shb = reinterpret_cast<uint8_t*>(sh);
+  float* a = sh;
+  float* z = a + NB * kSA;
+  float* pl = z + NB * kSA;
+  float* plT = pl + 96 * kSP;
+  float* ljt = plT + 32 * kST;
+  float* rinv = ljt + 32 * kSI;
+  float4* grp = reinterpret_cast<float4*>(rinv + 32);
+  float* sl = reinterpret_cast<float*>(shb + kStepSlice);   // S, [32][kSA]
+  uint64_t* full = reinterpret_cast<uint64_t*>(shb + kStepBars);   // [2] a slab landed
+  uint64_t* freed = full + 2;                                     // [2] its MMAs are done
+  uint64_t* done = full + 4;                                      // every MMA is done
+  uint32_t* taddr_s = reinterpret_cast<uint32_t*>(full + 5);
+  volatile int* abort_flag = reinterpret_cast<int*>(full + 5) + 1;
+  uint8_t* stage0 = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(z) + 1023) & ~uintptr_t(1023));
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int d = p.d, kk = p.kk;
+  float* A = p.A;
+  const bool slice = d - kk - NB > 0;
+  const int r0 = kk + NB + kSlice * blockIdx.x;
+  const bool upd = kk > 0;
+  const uint32_t nrows = slice ? NB + kSlice : NB;   // N of the update product
+  if (t < 64) grp[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (t == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&freed[i], 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (upd && warp == 1) {
+    tmem_alloc(taddr_s, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tacc = *taddr_s;
+  pdl_wait();       // the previous step's panel is complete
+  // ---- (1) the update product: thread 0 loads slabs and issues the MMAs
+  auto load_slab = [&](int sl_k, uint8_t* st, uint64_t* bar) {
+    const int x = kk - NB + 32 * sl_k;
+    mbar_expect_tx(bar, slice ? kStageBytes : 2 * kBoxLp);
+    tma_load_2d(st, &p.lp_hi, bar, x, kk);
+    tma_load_2d(st + kStagePlane, &p.lp_lo, bar, x, kk);
+    if (slice) {
+      tma_load_2d(st + kBoxLp, &p.ls_hi, bar, x, r0);
+      tma_load_2d(st + kStagePlane + kBoxLp, &p.ls_lo, bar, x, r0);
+    }
+  };
+  if (upd && t == 0) {
+    tma_prefetch(&p.lp_hi);
+    tma_prefetch(&p.lp_lo);
+    if (slice) {
+      tma_prefetch(&p.ls_hi);
+      tma_prefetch(&p.ls_lo);
+    }
+    load_slab(0, stage0, &full[0]);
+    load_slab(1, stage0 + kStageBytes, &full[1]);
+  }
+  // meanwhile: A_kk and S (fp32); z = I when there is no update
+  for (int e = t; e < NB * (NB / 4); e += blockDim.x) {
+    const int i = e >> 5, c = (e & 31) * 4;
+    *reinterpret_cast<float4*>(&a[i * kSA + c]) =
+        *reinterpret_cast<const float4*>(A + (size_t)(kk + i) * d + kk + c);
+    if (!upd)
+      *reinterpret_cast<float4*>(&z[i * kSA + c]) =
+          make_float4(i == c ? 1.f : 0.f, i == c + 1 ? 1.f : 0.f, i == c + 2 ? 1.f : 0.f,
+                      i == c + 3 ? 1.f : 0.f);
+  }
+  if (slice)
+    for (int e = t; e < kSlice * (NB / 4); e += blockDim.x) {
+      const int i = e >> 5, c = (e & 31) * 4;
+      *reinterpret_cast<float4*>(&sl[i * kSA + c]) =
+          *reinterpret_cast<const float4*>(A + (size_t)(r0 + i) * d + kk + c);
+    }
+  if (upd) {
+    if (t == 0) {
+      const uint32_t idesc = instr_desc(2, 2, 0, 0, NB, nrows);
+      int issued = 2;
+      for (int s = 0; s < 4; ++s) {
+        const int b = s & 1;
+        uint8_t* st = stage0 + b * kStageBytes;
+        if (!mbar_wait(&full[b], (s >> 1) & 1, p.status, abort_flag, p.wait_ns)) break;
+        tc_fence_after();
+        const uint64_t hi = smem_desc(smem_u32(st), 16, 1024, 2);
+        const uint64_t lo = smem_desc(smem_u32(st + kStagePlane), 16, 1024, 2);
+#pragma unroll
+        for (int k8 = 0; k8 < 4; ++k8) {   // 8-deep steps: 32 bytes along the swizzled rows
+          const uint64_t o = (uint64_t)(k8 * 2);
+          mma_ss_tf32(tacc, hi + o, hi + o, idesc, (s > 0 || k8 > 0) ? 1u : 0u);
+          mma_ss_tf32(tacc, hi + o, lo + o, idesc, 1u);
+          mma_ss_tf32(tacc, lo + o, hi + o, idesc, 1u);
+        }
+        tc_commit(&freed[b]);
+        if (s + 2 < 4) {
+          if (!mbar_wait(&freed[b], 0, p.status, abort_flag, p.wait_ns)) break;
+          load_slab(s + 2, st, &full[b]);
+          ++issued;
+        }
+      }
+      tc_commit(done);   // arrives once every MMA issued has completed
+      // every copy issued has landed before the staging area is reused
+      for (int j = issued - 2; j < issued; ++j) drain_wait_step(&full[j & 1], (j >> 1) & 1, p.status);
+    }
+    drain_wait_step(done, 0, p.status);
+    tc_fence_after();
+    // A_kk[i][j] -= D[i][j] (j < 128) and S[s][i] -= D[i][128 + s]; warp w
+    // reads the accumulator rows of its lane quarter, 32 columns at a time
+    if (__all_sync(0xffffffffu, *abort_flag == 0)) {
+      const int q = warp & 3, row = 32 * q + lane;
+      const int nchunk = (int)nrows / 32;
+      for (int c = warp >> 2; c < nchunk; c += 4) {
+        uint32_t v[32];
+        tmem_ld32(tacc + ((uint32_t)(32 * q) << 16) + 32 * c, v);
+        tmem_ld_wait();
+        if (c < 4) {
+#pragma unroll
+          for (int m4 = 0; m4 < 8; ++m4) {
+            float* dst = &a[row * kSA + 32 * c + 4 * m4];
+            float4 x = *reinterpret_cast<float4*>(dst);
+            x.x -= __uint_as_float(v[4 * m4]);
+            x.y -= __uint_as_float(v[4 * m4 + 1]);
+            x.z -= __uint_as_float(v[4 * m4 + 2]);
+            x.w -= __uint_as_float(v[4 * m4 + 3]);
+            *reinterpret_cast<float4*>(dst) = x;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sl[i * kSA + row] -= __uint_as_float(v[i]);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tacc, 256);
+    }
+    // z = I for the inverse (the staging area is free)
+    for (int e = t; e < NB * (NB / 4); e += blockDim.x) {
+      const int i = e >> 5, c = (e & 31) * 4;
+      *reinterpret_cast<float4*>(&z[i * kSA + c]) =
+          make_float4(i == c ? 1.f : 0.f, i == c + 1 ? 1.f : 0.f, i == c + 2 ? 1.f : 0.f,
+                      i == c + 3 ? 1.f : 0.f);
+    }
+  }
+  __syncthreads();
+  // ---- (2)
+  factor_invert(a, z, pl, plT, ljt, rinv, grp, p.status, [](int) {});
+  pdl_trigger();
+  // ---- (3) L_{S,k}[i][j] = sum_{c <= j} S[i][c] Linv[j][c]: thread = column
+  // j and 8 rows; the warp's columns bound c (Linv is zero above the diagonal)
+  if (slice) {
+    const int j = t & (NB - 1), i0 = (t >> 7) * 8, cend = (j | 31) + 1;
+    float acc[8] = {};
+    for (int c = 0; c < cend; c += 4) {
+      float zv[4];
+      ld4(zv, z + j * kSA + c);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) zv[q] = (c + q <= j) ? zv[q] : 0.f;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        float xv[4];
+        ld4(xv, sl + (i0 + r) * kSA + c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[r] = fmaf(xv[q], zv[q], acc[r]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const size_t o = (size_t)(r0 + i0 + r) * d + kk + j;
+      const float v = acc[r], h = to_tf32(v);
+      p.Ah[o] = h;
+      p.Ah[p.plane + o] = to_tf32(v - h);
+    }
+  }
+  store_linv(z, p.linv, blockIdx.x * NB / gridDim.x, (blockIdx.x + 1) * NB / gridDim.x);
 }
 
 void set_store(TGemmProblem& pr, int M, int N, int K, float* C, int64_t ldc, int64_t c_stride,
@@ -377,9 +654,10 @@ bool opmap(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols, uint
 }
 
 // Per-layer workspace, in floats (d = dim): A, Z, Y (fp32), then the hi and
-// lo planes of A, Z and Y (each plane d^2, lo = hi + d^2), one 128 x 128
-// inverse (fp32, then its hi and lo planes) and lambda. Finished blocks of L
-// (in A's planes), of L^-1 and of L^-1 B are kept only as planes: every
+// lo planes of A, Z and Y (each plane d^2, lo = hi + d^2), one slot per block
+// column for its 128 x 128 inverse (fp32, then its hi and lo planes; the
+// several-layer sweep uses the first slot only) and lambda. Finished blocks
+// of L (in A's planes), of L^-1 and of L^-1 B are kept as planes: every
 // product that reads them again takes them pre-split.
 struct SolveWs {
   float *A, *Z, *Y, *Ah, *Zh, *Yh, *Linv, *Lh, *lam;
@@ -398,7 +676,7 @@ SolveWs solve_ws(void* workspace, size_t d, int64_t stride) {
   w.Yh = w.Zh + 2 * dd;
   w.Linv = w.Yh + 2 * dd;
   w.Lh = w.Linv + NB * NB;          // hi / lo planes of Linv (lo = hi + NB * NB)
-  w.lam = w.Lh + 2 * NB * NB;
+  w.lam = w.Linv + 3 * NB * d;      // d / NB slots of 3 NB^2
   w.plane = (int64_t)dd;
   w.stride = stride;
   return w;
@@ -427,16 +705,18 @@ void to_planes(TGemmProblem& pr, float* hi, int64_t plane) {
 }
 
 // Streams and events per device for the one-layer sweep (created on first
-// use, kept for the process): the sweep's critical path -- factor, panel and
-// the part of each update the next step needs -- runs on `crit`, created at the
-// device's greatest stream priority; the rest of each update runs on `side`, at
-// the least, so that the block scheduler dispatches critical-path CTAs ahead of
-// the bulk update's pending ones. Both are forked from the caller's stream and
-// joined back to it. The mutex is held while a solve enqueues its work, so that
+// use, kept for the process): the sweep's critical path -- one step kernel
+// per block column -- runs on `crit`, created at the device's greatest stream
+// priority; the trailing update of A runs on `sa`, the Z and Y block rows on
+// `sz` and the accumulation of Delta W on `sw`, all at the least, so that the
+// block scheduler dispatches critical-path CTAs ahead of the bulk products'
+// pending ones. All four are forked from the caller's stream and joined back
+// to it. The mutex is held while a solve enqueues its work, so that
 // concurrent callers do not re-record each other's events.
 struct Lookahead {
-  cudaStream_t crit = nullptr, side = nullptr;
-  cudaEvent_t start = nullptr, fork = nullptr, join = nullptr, done = nullptr, rw = nullptr;
+  cudaStream_t crit = nullptr, sa = nullptr, sz = nullptr, sw = nullptr;
+  cudaEvent_t start = nullptr, built = nullptr, step = nullptr, a[2] = {nullptr, nullptr},
+              zrow = nullptr, ja = nullptr, jz = nullptr, jw = nullptr, done = nullptr;
 };
 std::mutex g_look_mutex;
 Lookahead g_look[64];
@@ -447,43 +727,49 @@ cudaError_t lookahead_for_device(Lookahead** out) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   Lookahead& l = g_look[dev];
-  if (!l.side) {
+  if (!l.done) {
     int least = 0, greatest = 0;
+    cudaStream_t* low[] = {&l.sa, &l.sz, &l.sw};
+    cudaEvent_t* evs[] = {&l.start, &l.built, &l.step, &l.a[0], &l.a[1], &l.zrow, &l.ja, &l.jz, &l.jw};
     if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess ||
-        (e = cudaStreamCreateWithPriority(&l.crit, cudaStreamNonBlocking, greatest)) != cudaSuccess ||
-        (e = cudaStreamCreateWithPriority(&l.side, cudaStreamNonBlocking, least)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&l.start, cudaEventDisableTiming)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&l.fork, cudaEventDisableTiming)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&l.join, cudaEventDisableTiming)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&l.done, cudaEventDisableTiming)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&l.rw, cudaEventDisableTiming)) != cudaSuccess)
+        (e = cudaStreamCreateWithPriority(&l.crit, cudaStreamNonBlocking, greatest)) != cudaSuccess)
       return e;
+    for (cudaStream_t* st : low)
+      if ((e = cudaStreamCreateWithPriority(st, cudaStreamNonBlocking, least)) != cudaSuccess) return e;
+    for (cudaEvent_t* ev : evs)
+      if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+    // created last: marks the set complete
+    if ((e = cudaEventCreateWithFlags(&l.done, cudaEventDisableTiming)) != cudaSuccess) return e;
   }
   *out = &l;
   return cudaSuccess;
 }
 
 // Joins the sweep's streams back into the caller's stream when the solve
-// returns, on its error paths too: `crit` waits for the side stream's last
-// update, then the caller's stream waits for `crit`.
+// returns, on its error paths too: `crit` waits for the last work of `sa`,
+// `sz` and `sw`, then the caller's stream waits for `crit`.
 struct SweepJoin {
   Lookahead* look = nullptr;
   cudaStream_t caller = nullptr;
-  bool side_pending = false;
   ~SweepJoin() {
     if (!look) return;
-    if (side_pending) cudaStreamWaitEvent(look->crit, look->join, 0);
+    cudaEventRecord(look->ja, look->sa);
+    cudaStreamWaitEvent(look->crit, look->ja, 0);
+    cudaEventRecord(look->jz, look->sz);
+    cudaStreamWaitEvent(look->crit, look->jz, 0);
+    cudaEventRecord(look->jw, look->sw);
+    cudaStreamWaitEvent(look->crit, look->jw, 0);
     cudaEventRecord(look->done, look->crit);
     cudaStreamWaitEvent(caller, look->done, 0);
   }
 };
 
 // Panel of step k: L_{>k,k} = A_{>k,k} Linv^T, Z_k = Linv Z_k, Y_k = Linv Y_k,
-// with Linv = L_kk^-1 from potrf_inv_kernel, read from its pre-split planes;
+// with Linv = L_kk^-1 read from its pre-split planes at lh (lo = lh + 128^2);
 // A_{>k,k}, Z_k and Y_k are fp32 (split in the kernel, K = 128); outputs go to
 // the planes, where later products read them.
-cudaError_t panel_launch(int n, const SolveWs& w, size_t d, int kk, int m, int* status,
-                         cudaStream_t stream) {
+cudaError_t panel_launch(int n, const SolveWs& w, const float* lh, size_t d, int kk, int m,
+                         int* status, cudaStream_t stream) {
   const int dim = (int)d;
   const int64_t ws = w.stride;
   TGemmParams p{};
@@ -492,7 +778,7 @@ cudaError_t panel_launch(int n, const SolveWs& w, size_t d, int kk, int m, int* 
   if (m > 0) {
     TGemmProblem& pr = p.prob[q++];
     if (!opmap(&pr.ta, w.A + (size_t)(kk + NB) * d + kk, m, NB, d, n, ws, false) ||
-        !opmap_split(pr, false, w.Lh, NB * NB, NB, NB, NB, n, ws, false))
+        !opmap_split(pr, false, lh, NB * NB, NB, NB, NB, n, ws, false))
       return cudaErrorInvalidValue;
     set_store(pr, m, NB, NB, nullptr, dim, ws, kk + NB, kk, 1.f, 0.f, n);
     to_planes(pr, w.Ah, w.plane);
@@ -500,7 +786,7 @@ cudaError_t panel_launch(int n, const SolveWs& w, size_t d, int kk, int m, int* 
   }
   {
     TGemmProblem& pr = p.prob[q++];
-    if (!opmap_split(pr, true, w.Lh, NB * NB, NB, NB, NB, n, ws, false) ||
+    if (!opmap_split(pr, true, lh, NB * NB, NB, NB, NB, n, ws, false) ||
         !opmap(&pr.tb, w.Z + (size_t)kk * d, NB, kk + NB, d, n, ws, true))
       return cudaErrorInvalidValue;
     set_store(pr, NB, kk + NB, NB, nullptr, dim, ws, kk, 0, 1.f, 0.f, n);
@@ -509,7 +795,7 @@ cudaError_t panel_launch(int n, const SolveWs& w, size_t d, int kk, int m, int* 
   }
   {
     TGemmProblem& pr = p.prob[q++];
-    if (!opmap_split(pr, true, w.Lh, NB * NB, NB, NB, NB, n, ws, false) ||
+    if (!opmap_split(pr, true, lh, NB * NB, NB, NB, NB, n, ws, false) ||
         !opmap(&pr.tb, w.Y + (size_t)kk * d, NB, d, d, n, ws, true))
       return cudaErrorInvalidValue;
     set_store(pr, NB, dim, NB, nullptr, dim, ws, kk, 0, 1.f, 0.f, n);
@@ -527,6 +813,200 @@ size_t absorb_workspace_bytes(int dim) {
   return absorb_scratch_bytes((size_t)dim);
 }
 
+namespace {
+
+// B = R W (R = M[0:d, d:2d]) for n layers: both split once into the Z and Y
+// planes (free until the sweep's first block rows of Z and Y), one pre-split
+// product, then Y = B, the right-hand side of the substitution.
+cudaError_t rw_launch(int n, const float* M, int64_t m_stride, const float* W, int64_t w_stride,
+                      int dim, float* B, int64_t b_stride, const SolveWs& w, int* status,
+                      cudaStream_t stream) {
+  const size_t d = (size_t)dim;
+  const int64_t ws = w.stride;
+  cudaError_t e;
+  if ((e = launch_split_planes(n, M + d, 2 * d, m_stride, w.Zh, w.Zh + w.plane, d, ws, dim, dim,
+                               stream)) != cudaSuccess ||
+      (e = launch_split_planes(n, W, d, w_stride, w.Yh, w.Yh + w.plane, d, ws, dim, dim,
+                               stream)) != cudaSuccess)
+    return e;
+  TGemmParams p{};
+  p.nprob = 1;
+  p.status = status;
+  p.kchunk = kChunkSlabs;
+  TGemmProblem& pr = p.prob[0];
+  if (!opmap_split(pr, true, w.Zh, w.plane, d, d, d, n, ws, false) ||
+      !opmap_split(pr, false, w.Yh, w.plane, d, d, d, n, ws, true))
+    return cudaErrorInvalidValue;
+  set_store(pr, dim, dim, dim, B, dim, b_stride, 0, 0, 1.f, 0.f, n);
+  if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
+  copy_layers_kernel<<<dim3(n == 1 ? 148 * 4 : 148, n), 256, 0, stream>>>(
+      reinterpret_cast<const float4*>(B), b_stride / 4, reinterpret_cast<float4*>(w.Y), ws / 4,
+      (int64_t)(d * d / 4));
+  count_launches();
+  return cudaGetLastError();
+}
+
+// Delta W = Z^T Y (Z^T upper triangular), both from the planes, for n layers.
+cudaError_t ztw_launch(int n, const SolveWs& w, int dim, float* dW, int64_t dw_stride, int* status,
+                       cudaStream_t stream) {
+  const size_t d = (size_t)dim;
+  TGemmParams p{};
+  p.nprob = 1;
+  p.status = status;
+  p.kchunk = kChunkSlabs;
+  TGemmProblem& pr = p.prob[0];
+  if (!opmap_split(pr, true, w.Zh, w.plane, d, d, d, n, w.stride, true) ||
+      !opmap_split(pr, false, w.Yh, w.plane, d, d, d, n, w.stride, true))
+    return cudaErrorInvalidValue;
+  set_store(pr, dim, dim, dim, dW, dim, dw_stride, 0, 0, 1.f, 0.f, n);
+  pr.tri = kTriUpperA;
+  return launch_tgemm(p, stream);
+}
+
+// One layer, right-looking. Per block column k, one step kernel on the
+// critical path (sweep_step_kernel: the previous step's update of this block
+// column, the block factor and inverse, the panel L_{>k,k}); after it, on
+// `sa`, the rank-128 update of A's lower tiles from block column k + 2 on
+// (block column k + 1 is updated by the next step kernel itself); on `sz` the
+// block rows Z_k = Linv Z_k, Y_k = Linv Y_k followed by
+// Z_{>k} -= L_{>k,k} Z_k, Y_{>k} -= L_{>k,k} Y_k; and on `sw`, once Z_k and
+// Y_k are final, Delta W += Z_k^T Y_k (Delta W = Z^T Y = sum_k Z_k^T Y_k,
+// accumulated in fp32 into a zeroed Delta W). The step kernel of k + 2 waits
+// for the update of A from step k, nothing else. B = R W (the right-hand
+// side Y starts from) runs on `sz` once A is built. Without side streams
+// every launch runs in this order on `stream`.
+cudaError_t sweep_one_layer(const float* M, int64_t m_stride, const float* W, int64_t w_stride,
+                            int dim, float lambda, float* dW, int64_t dw_stride, float* B,
+                            int64_t b_stride, float* lambda_out, const SolveWs& w, int* status,
+                            cudaStream_t stream, bool side_stream) {
+  const size_t d = (size_t)dim;
+  const int64_t ws = w.stride;
+  const int64_t lam_off = w.lam - w.A;
+  const int nblk = dim / NB;
+  cudaError_t e;
+  cudaFuncSetAttribute(sweep_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)kStepSmem);
+  StepParams sp{};
+  if (!encode_2d(&sp.lp_hi, w.Ah, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, d, d, 32, NB,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&sp.lp_lo, w.Ah + w.plane, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, d, d, 32, NB,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&sp.ls_hi, w.Ah, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, d, d, 32, kSlice,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&sp.ls_lo, w.Ah + w.plane, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, d, d, 32, kSlice,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  sp.A = w.A;
+  sp.Ah = w.Ah;
+  sp.plane = w.plane;
+  sp.d = dim;
+  sp.status = status;
+  sp.wait_ns = wait_limit_ns();
+  std::unique_lock<std::mutex> look_lock;
+  SweepJoin join;
+  join.caller = stream;
+  Lookahead* look = nullptr;
+  cudaStream_t crit = stream, sa = stream, sz = stream, sw = stream;
+  if (side_stream && nblk > 1) {
+    look_lock = std::unique_lock<std::mutex>(g_look_mutex);
+    if ((e = lookahead_for_device(&look)) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(look->start, stream)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(look->crit, look->start, 0)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(look->sa, look->start, 0)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(look->sz, look->start, 0)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(look->sw, look->start, 0)) != cudaSuccess)
+      return e;
+    join.look = look;
+    crit = look->crit;
+    sa = look->sa;
+    sz = look->sz;
+    sw = look->sw;
+  }
+  if ((e = cudaMemsetAsync(dW, 0, d * d * sizeof(float), sw)) != cudaSuccess) return e;
+  lambda_kernel<<<1, kLambdaThreads, 0, crit>>>(M, m_stride, dim, lambda, w.lam, ws, lambda_out);
+  count_launches();
+  // A = G + lambda I, Z = I
+  build_kernel<<<dim3(148 * 8, 1), 256, 0, crit>>>(M, m_stride, dim, w.A, ws, lam_off);
+  count_launches();
+  // B = R W and Y = B on sz, once the build has the SMs no more
+  if (look && ((e = cudaEventRecord(look->built, crit)) != cudaSuccess ||
+               (e = cudaStreamWaitEvent(sz, look->built, 0)) != cudaSuccess))
+    return e;
+  if ((e = rw_launch(1, M, m_stride, W, w_stride, dim, B, b_stride, w, status, sz)) != cudaSuccess)
+    return e;
+  for (int k = 0; k < nblk; ++k) {
+    const int kk = k * NB;
+    const int m = dim - kk - NB;   // rows below the diagonal block
+    float* linv = w.Linv + (size_t)k * 3 * NB * NB;
+    // block column k has the updates of steps 0 .. k - 2 (sa, in order)
+    if (look && k >= 2 && (e = cudaStreamWaitEvent(crit, look->a[k & 1], 0)) != cudaSuccess)
+      return e;
+    sp.kk = kk;
+    sp.linv = linv;
+    if ((e = launch_pdl(sweep_step_kernel, dim3(m > 0 ? m / kSlice : 1), dim3(512), kStepSmem,
+                        crit, sp)) != cudaSuccess)
+      return e;
+    count_launches();
+    if (look && ((e = cudaEventRecord(look->step, crit)) != cudaSuccess ||
+                 (e = cudaStreamWaitEvent(sa, look->step, 0)) != cudaSuccess ||
+                 (e = cudaStreamWaitEvent(sz, look->step, 0)) != cudaSuccess))
+      return e;
+    const float* Lk_h = w.Ah + (size_t)(kk + NB) * d + kk;   // L_{>k,k}, planes
+    if (m > NB) {
+      // A_{>k+1,>k+1} -= L_{>k+1,k} L_{>k+1,k}^T on the lower tiles
+      TGemmParams p{};
+      p.status = status;
+      p.nprob = 1;
+      TGemmProblem& t1 = p.prob[0];
+      const int r = m - NB;
+      if (!opmap_split(t1, true, Lk_h + (size_t)NB * d, w.plane, r, NB, d, 1, ws, false) ||
+          !opmap_split(t1, false, Lk_h + (size_t)NB * d, w.plane, r, NB, d, 1, ws, false))
+        return cudaErrorInvalidValue;
+      set_store(t1, r, r, NB, w.A, dim, ws, kk + 2 * NB, kk + 2 * NB, -1.f, 1.f, 1);
+      t1.lower = 1;
+      if ((e = launch_tgemm(p, sa)) != cudaSuccess) return e;
+      if (look && (e = cudaEventRecord(look->a[k & 1], sa)) != cudaSuccess) return e;
+    }
+    // Z_k = Linv Z_k, Y_k = Linv Y_k (to the planes): final from here on
+    if ((e = panel_launch(1, w, linv + NB * NB, d, kk, 0, status, sz)) != cudaSuccess) return e;
+    if (look && ((e = cudaEventRecord(look->zrow, sz)) != cudaSuccess ||
+                 (e = cudaStreamWaitEvent(sw, look->zrow, 0)) != cudaSuccess))
+      return e;
+    {
+      // Delta W[0 : kk + 128, :] += Z_k^T Y_k (Z_k is zero right of column kk + 127)
+      TGemmParams p{};
+      p.status = status;
+      p.nprob = 1;
+      TGemmProblem& pr = p.prob[0];
+      if (!opmap_split(pr, true, w.Zh + (size_t)kk * d, w.plane, NB, kk + NB, d, 1, ws, true) ||
+          !opmap_split(pr, false, w.Yh + (size_t)kk * d, w.plane, NB, d, d, 1, ws, true))
+        return cudaErrorInvalidValue;
+      set_store(pr, kk + NB, dim, NB, dW, dim, dw_stride, 0, 0, 1.f, 1.f, 1);
+      if ((e = launch_tgemm(p, sw)) != cudaSuccess) return e;
+    }
+    if (m > 0) {
+      // Z_{>k} -= L_{>k,k} Z_k, Y_{>k} -= L_{>k,k} Y_k
+      TGemmParams p{};
+      p.status = status;
+      p.nprob = 2;
+      TGemmProblem& t2 = p.prob[0];
+      if (!opmap_split(t2, true, Lk_h, w.plane, m, NB, d, 1, ws, false) ||
+          !opmap_split(t2, false, w.Zh + (size_t)kk * d, w.plane, NB, kk + NB, d, 1, ws, true))
+        return cudaErrorInvalidValue;
+      set_store(t2, m, kk + NB, NB, w.Z, dim, ws, kk + NB, 0, -1.f, 1.f, 1);
+      TGemmProblem& t3 = p.prob[1];
+      if (!opmap_split(t3, true, Lk_h, w.plane, m, NB, d, 1, ws, false) ||
+          !opmap_split(t3, false, w.Yh + (size_t)kk * d, w.plane, NB, d, d, 1, ws, true))
+        return cudaErrorInvalidValue;
+      set_store(t3, m, dim, NB, w.Y, dim, ws, kk + NB, 0, -1.f, 1.f, 1);
+      if ((e = launch_tgemm(p, sz)) != cudaSuccess) return e;
+    }
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const float* W,
                                  int64_t w_stride, int dim, float lambda, float* dW,
                                  int64_t dw_stride, float* B, int64_t b_stride, float* lambda_out,
@@ -535,79 +1015,29 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
   const size_t d = (size_t)dim;
   const int64_t ws = (int64_t)(absorb_workspace_bytes(dim) / sizeof(float));  // per-layer stride
   const SolveWs w = solve_ws(workspace, d, ws);
+  if (n == 1)
+    return sweep_one_layer(M, m_stride, W, w_stride, dim, lambda, dW, dw_stride, B, b_stride,
+                           lambda_out, w, status, stream, side_stream);
+  // Several layers: left-looking (long-K products that read the finished
+  // part once): far less HBM traffic than right-looking updates, and the
+  // layers supply the parallelism.
   const int64_t lam_off = w.lam - w.A;
   const int nblk = dim / NB;
   cudaError_t e;
   cudaFuncSetAttribute(potrf_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)kPotrfSmem);
-
-  // One layer: right-looking (a rank-128 update of everything below the block
-  // after each step): up to (d/128)^2 tiles per launch keep the GPU busy.
-  // Several layers: left-looking (long-K products that read the finished
-  // part once): far less HBM traffic, and the layers supply the parallelism.
-  const bool left_looking = n > 1;
-  std::unique_lock<std::mutex> look_lock;
-  SweepJoin join;
-  join.caller = stream;
-  Lookahead* look = nullptr;
-  if (!left_looking && nblk > 2 && side_stream) {
-    look_lock = std::unique_lock<std::mutex>(g_look_mutex);
-    if ((e = lookahead_for_device(&look)) != cudaSuccess) return e;
-    if ((e = cudaEventRecord(look->start, stream)) != cudaSuccess ||
-        (e = cudaStreamWaitEvent(look->crit, look->start, 0)) != cudaSuccess)
-      return e;
-    join.look = look;
-    stream = look->crit;            // everything below runs on the critical-path stream
-  }
-
   lambda_kernel<<<n, kLambdaThreads, 0, stream>>>(M, m_stride, dim, lambda, w.lam, ws, lambda_out);
   count_launches();
-
-  // B = R W (R = M[0:d, d:2d]): both split once into the Z and Y planes (free
-  // until the sweep's first panel), then one pre-split product; Y = B is the
-  // right-hand side of the substitution. With the side stream this runs there,
-  // beside the build and the first block factor, which touch neither.
-  cudaStream_t rw_stream = stream;
-  if (look) {
-    if ((e = cudaStreamWaitEvent(look->side, look->start, 0)) != cudaSuccess) return e;
-    rw_stream = look->side;
-  }
-  if ((e = launch_split_planes(n, M + d, 2 * d, m_stride, w.Zh, w.Zh + w.plane, d, ws, dim, dim,
-                               rw_stream)) != cudaSuccess ||
-      (e = launch_split_planes(n, W, d, w_stride, w.Yh, w.Yh + w.plane, d, ws, dim, dim,
-                               rw_stream)) != cudaSuccess)
+  if ((e = rw_launch(n, M, m_stride, W, w_stride, dim, B, b_stride, w, status, stream)) !=
+      cudaSuccess)
     return e;
-  {
-    TGemmParams p{};
-    p.nprob = 1;
-    p.status = status;
-    p.kchunk = kChunkSlabs;
-    TGemmProblem& pr = p.prob[0];
-    if (!opmap_split(pr, true, w.Zh, w.plane, d, d, d, n, ws, false) ||
-        !opmap_split(pr, false, w.Yh, w.plane, d, d, d, n, ws, true))
-      return cudaErrorInvalidValue;
-    set_store(pr, dim, dim, dim, B, dim, b_stride, 0, 0, 1.f, 0.f, n);
-    if ((e = launch_tgemm(p, rw_stream)) != cudaSuccess) return e;
-  }
-  copy_layers_kernel<<<dim3(n == 1 ? 148 * 4 : 148, n), 256, 0, rw_stream>>>(
-      reinterpret_cast<const float4*>(B), b_stride / 4, reinterpret_cast<float4*>(w.Y), ws / 4,
-      (int64_t)(d * d / 4));
-  count_launches();
-  if (look) {
-    if ((e = cudaEventRecord(look->rw, look->side)) != cudaSuccess ||
-        (e = cudaEventRecord(look->join, look->side)) != cudaSuccess)
-      return e;
-    join.side_pending = true;
-  }
   // A = G + lambda I, Z = I
-  build_kernel<<<dim3(n == 1 ? 148 * 8 : 148, n), 256, 0, stream>>>(M, m_stride, dim, w.A, ws,
-                                                                     lam_off);
+  build_kernel<<<dim3(148, n), 256, 0, stream>>>(M, m_stride, dim, w.A, ws, lam_off);
   count_launches();
-
   for (int k = 0; k < nblk; ++k) {
     const int kk = k * NB;
     const int m = dim - kk - NB;   // rows below the diagonal block
-    if (left_looking && k > 0) {
+    if (k > 0) {
       // bring block column k of A and block rows k of Y and Z up to date with
       // the finished blocks 0..k-1, read pre-split from the planes
       TGemmParams p{};
@@ -641,87 +1071,9 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
         cudaSuccess)
       return e;
     count_launches();
-    if (k == 0 && look && (e = cudaStreamWaitEvent(stream, look->rw, 0)) != cudaSuccess) return e;
-    if ((e = panel_launch(n, w, d, kk, m, status, stream)) != cudaSuccess) return e;
-    if (left_looking || m <= 0) continue;
-    // right-looking, with lookahead: the rank-128 update of step k
-    // (A_{>k,>k} -= L_{>k,k} L_{>k,k}^T on the lower tiles, Z_{>k} -= L_{>k,k} Z_k,
-    // Y_{>k} -= L_{>k,k} Y_k; panel outputs pre-split) is cut in two. The part
-    // step k+1 needs first -- block column k+1 of A, block rows k+1 of Z and Y
-    // -- runs on `stream`; the rest (rows and columns from k+2 on) runs on a
-    // side stream while step k+1 factors its block and forms its panel. The
-    // side stream's previous update must be done before this step's first part
-    // (it wrote block k+1), and the final one before Delta W.
-    const float* Lk_h = w.Ah + (size_t)(kk + NB) * d + kk;   // L_{>k,k}
-    if (k > 0 && look && (e = cudaStreamWaitEvent(stream, look->join, 0)) != cudaSuccess) return e;
-    for (int part = 0; part < 2; ++part) {
-      const int r0 = part == 0 ? 0 : NB;            // first row (within the rows below) updated
-      const int rows = part == 0 ? (look ? NB : m) : m - NB;
-      if (rows <= 0) break;
-      TGemmParams p{};
-      p.status = status;
-      int q = 0;
-      // A: part 0 = block column k+1 (all rows below), part 1 = lower tiles of the rest
-      {
-        TGemmProblem& t1 = p.prob[q++];
-        const int a_rows = part == 0 ? m : m - NB;
-        const int a_cols = part == 0 ? (look ? NB : m) : m - NB;
-        if (!opmap_split(t1, true, Lk_h + (size_t)r0 * d, w.plane, a_rows, NB, d, n, ws, false) ||
-            !opmap_split(t1, false, Lk_h + (size_t)r0 * d, w.plane, a_cols, NB, d, n, ws, false))
-          return cudaErrorInvalidValue;
-        set_store(t1, a_rows, a_cols, NB, w.A, dim, ws, kk + NB + r0, kk + NB + r0, -1.f, 1.f, n);
-        t1.lower = (part == 1 || !look) ? 1 : 0;
-      }
-      TGemmProblem& t2 = p.prob[q++];
-      if (!opmap_split(t2, true, Lk_h + (size_t)r0 * d, w.plane, rows, NB, d, n, ws, false) ||
-          !opmap_split(t2, false, w.Zh + (size_t)kk * d, w.plane, NB, kk + NB, d, n, ws, true))
-        return cudaErrorInvalidValue;
-      set_store(t2, rows, kk + NB, NB, w.Z, dim, ws, kk + NB + r0, 0, -1.f, 1.f, n);
-      TGemmProblem& t3 = p.prob[q++];
-      if (!opmap_split(t3, true, Lk_h + (size_t)r0 * d, w.plane, rows, NB, d, n, ws, false) ||
-          !opmap_split(t3, false, w.Yh + (size_t)kk * d, w.plane, NB, d, d, n, ws, true))
-        return cudaErrorInvalidValue;
-      set_store(t3, rows, dim, NB, w.Y, dim, ws, kk + NB + r0, 0, -1.f, 1.f, n);
-      p.nprob = q;
-      if (part == 0) {
-        if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
-        if (!look) break;
-      } else {
-        if ((e = cudaEventRecord(look->fork, stream)) != cudaSuccess ||
-            (e = cudaStreamWaitEvent(look->side, look->fork, 0)) != cudaSuccess ||
-            (e = launch_tgemm(p, look->side)) != cudaSuccess ||
-            (e = cudaEventRecord(look->join, look->side)) != cudaSuccess)
-          return e;
-        join.side_pending = true;
-      }
-    }
+    if ((e = panel_launch(n, w, w.Lh, d, kk, m, status, stream)) != cudaSuccess) return e;
   }
-  if (join.side_pending) {
-    if ((e = cudaStreamWaitEvent(stream, look->join, 0)) != cudaSuccess) return e;
-    join.side_pending = false;
-  }
-  // Delta W = Z^T Y (Z^T upper triangular), both from the planes
-  {
-    TGemmParams p{};
-    p.nprob = 1;
-    p.status = status;
-    p.kchunk = kChunkSlabs;
-    TGemmProblem& pr = p.prob[0];
-    if (!opmap_split(pr, true, w.Zh, w.plane, d, d, d, n, ws, true) ||
-        !opmap_split(pr, false, w.Yh, w.plane, d, d, d, n, ws, true))
-      return cudaErrorInvalidValue;
-    set_store(pr, dim, dim, dim, dW, dim, dw_stride, 0, 0, 1.f, 0.f, n);
-    pr.tri = kTriUpperA;
-    if (n == 1) {
-      // one layer: the first tile rows read up to d/32 slabs and the last 4;
-      // two CTAs per tile, each over half of its slabs, reduce-add into a
-      // zeroed Delta W (as many CTAs as SMs twice over, the longest half as long)
-      if ((e = cudaMemsetAsync(dW, 0, d * d * sizeof(float), stream)) != cudaSuccess) return e;
-      pr.beta = 1.f;
-      pr.ksplit = 2;
-    }
-    if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
-  }
+  if ((e = ztw_launch(n, w, dim, dW, dw_stride, status, stream)) != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
