@@ -146,8 +146,8 @@ __global__ void copy_layers_kernel(const float4* __restrict__ src, int64_t src_s
 //      Z_J <- L_JJ^-1 Z_J (J + 32 columns), m + J + 32 = 128 threads;
 //  (3) trailing update in 4 x 4 register tiles: A_II -= L_IJ L_IJ^T on the
 //      lower tiles and Z_I -= L_IJ Z_J. With lookahead: the next diagonal
-//      sub-block is updated by warp 0, which factors it at once, while warps
-//      1-15 apply the rest of the update.
+//      sub-block is updated by warp 0, which factors it at once, while the
+//      warps that do not share its scheduler apply the rest of the update.
 // Shared-memory row strides (132, 36, 100 floats) keep the float4 accesses
 // 16-byte aligned and free of bank conflicts.
 constexpr int kSA = 132;     // a, z: [128][kSA]
@@ -261,9 +261,11 @@ __device__ __forceinline__ void factor_invert(float* a, float* z, float* pl, flo
       const int Jp = J - 32, mp = 96 - Jp;
       const int mt = mp / 4, n_tri = mt * (mt + 1) / 2, nzt = (Jp + 32) / 4;
       // triangle tiles are numbered row by row: the first 36 (rows 0..7) are
-      // the next diagonal sub-block, which warp 0 has updated itself
-      const int tt = t - 32 + 36;
-      if (tt < n_tri + mt * nzt) {
+      // the next diagonal sub-block, which warp 0 has updated itself. Warps
+      // 4, 8 and 12 share warp 0's scheduler and stay out, so that the factor
+      // loop keeps its issue slots; the other 12 warps take the tiles
+      for (int tt = (warp & 3) ? (warp - 1 - (warp >> 2)) * 32 + lane + 36 : (1 << 30);
+           tt < n_tri + mt * nzt; tt += 384) {
         int ti, tj;
         const bool tri = tt < n_tri;
         if (tri) {
