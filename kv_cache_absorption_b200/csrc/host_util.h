@@ -32,11 +32,11 @@ uint64_t wait_limit_ns();
 void set_wait_limit_ns(uint64_t ns);
 
 // Bytes of one absorb solve's scratch at dimension d: A, Z, Y; the tf32
-// hi/lo planes of each; a 128 x 128 inverse with its hi/lo planes per block
+// hi/lo planes of each; the hi/lo planes of a 128 x 128 inverse per block
 // column (d / 128 of them); lambda and padding; a multiple of 256 bytes so
 // that per-layer workspaces stack.
 constexpr size_t absorb_scratch_bytes(size_t d) {
-  return ((9 * d * d + 3 * 128 * d) * sizeof(float) + 1024 + 255) & ~size_t(255);
+  return ((9 * d * d + 2 * 128 * d) * sizeof(float) + 1024 + 255) & ~size_t(255);
 }
 
 // Row-major [rows, cols] matrix with leading dimension ld (elements), tiles

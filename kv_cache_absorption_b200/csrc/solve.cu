@@ -346,9 +346,9 @@ __device__ __forceinline__ void factor_invert(float* a, float* z, float* pl, flo
   }
 }
 
-// Writes rows [i0, i1) of L^-1 (z) to linv in fp32, zero above the diagonal,
-// then its tf32 planes: hi = tf32(v), lo = tf32(v - hi), rounded as the
-// GEMM's in-kernel split rounds them.
+// Writes rows [i0, i1) of L^-1 (z, zero above the diagonal) to linv as tf32
+// planes, hi = tf32(v) then lo = tf32(v - hi) NB^2 floats later, rounded as
+// the GEMM's in-kernel split rounds them: the products read only the planes.
 __device__ __forceinline__ void store_linv(const float* z, float* linv, int i0 = 0, int i1 = NB) {
   const int t = threadIdx.x;
   for (int e = i0 * (NB / 4) + t; e < i1 * (NB / 4); e += blockDim.x) {
@@ -357,12 +357,11 @@ __device__ __forceinline__ void store_linv(const float* z, float* linv, int i0 =
     ld4(v, &z[i * kSA + c]);
 #pragma unroll
     for (int c4 = 0; c4 < 4; ++c4) v[c4] = (c + c4 <= i) ? v[c4] : 0.f;
-    st4(&linv[(size_t)i * NB + c], v);
     float h[4], l[4];
 #pragma unroll
     for (int c4 = 0; c4 < 4; ++c4) { h[c4] = to_tf32(v[c4]); l[c4] = to_tf32(v[c4] - h[c4]); }
-    st4(&linv[NB * NB + (size_t)i * NB + c], h);
-    st4(&linv[2 * NB * NB + (size_t)i * NB + c], l);
+    st4(&linv[(size_t)i * NB + c], h);
+    st4(&linv[NB * NB + (size_t)i * NB + c], l);
   }
 }
 
@@ -421,7 +420,7 @@ struct StepParams {
   float* Ah;                  // hi plane (lo = Ah + plane)
   int64_t plane;
   int d, kk;
-  float* linv;                // this step's slot: Linv, then its hi / lo planes
+  float* linv;                // this step's slot: the hi / lo planes of Linv
   int* status;
   uint64_t wait_ns;
 };
@@ -605,6 +604,7 @@ __global__ void __launch_bounds__(512, 1) sweep_step_kernel(const __grid_constan
   if (slice) {
     const int j = t & (NB - 1), i0 = (t >> 7) * 8, cend = (j | 31) + 1;
     float acc[8] = {};
+#pragma unroll 2
     for (int c = 0; c < cend; c += 4) {
       float zv[4];
       ld4(zv, z + j * kSA + c);
@@ -657,12 +657,12 @@ bool opmap(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols, uint
 
 // Per-layer workspace, in floats (d = dim): A, Z, Y (fp32), then the hi and
 // lo planes of A, Z and Y (each plane d^2, lo = hi + d^2), one slot per block
-// column for its 128 x 128 inverse (fp32, then its hi and lo planes; the
-// several-layer sweep uses the first slot only) and lambda. Finished blocks
+// column for the hi and lo planes of its 128 x 128 inverse (the several-layer
+// sweep uses the first slot only) and lambda. Finished blocks
 // of L (in A's planes), of L^-1 and of L^-1 B are kept as planes: every
 // product that reads them again takes them pre-split.
 struct SolveWs {
-  float *A, *Z, *Y, *Ah, *Zh, *Yh, *Linv, *Lh, *lam;
+  float *A, *Z, *Y, *Ah, *Zh, *Yh, *Lh, *lam;
   int64_t plane;        // lo = hi + plane
   int64_t stride;       // floats between layers' workspaces
 };
@@ -676,9 +676,8 @@ SolveWs solve_ws(void* workspace, size_t d, int64_t stride) {
   w.Ah = w.Y + dd;
   w.Zh = w.Ah + 2 * dd;
   w.Yh = w.Zh + 2 * dd;
-  w.Linv = w.Yh + 2 * dd;
-  w.Lh = w.Linv + NB * NB;          // hi / lo planes of Linv (lo = hi + NB * NB)
-  w.lam = w.Linv + 3 * NB * d;      // d / NB slots of 3 NB^2
+  w.Lh = w.Yh + 2 * dd;             // hi / lo planes of Linv (lo = hi + NB * NB)
+  w.lam = w.Lh + 2 * NB * d;        // d / NB slots of 2 NB^2
   w.plane = (int64_t)dd;
   w.stride = stride;
   return w;
@@ -939,7 +938,7 @@ cudaError_t sweep_one_layer(const float* M, int64_t m_stride, const float* W, in
   for (int k = 0; k < nblk; ++k) {
     const int kk = k * NB;
     const int m = dim - kk - NB;   // rows below the diagonal block
-    float* linv = w.Linv + (size_t)k * 3 * NB * NB;
+    float* linv = w.Lh + (size_t)k * 2 * NB * NB;
     // block column k has the updates of steps 0 .. k - 2 (sa, in order)
     if (look && k >= 2 && (e = cudaStreamWaitEvent(crit, look->a[k & 1], 0)) != cudaSuccess)
       return e;
@@ -970,7 +969,7 @@ cudaError_t sweep_one_layer(const float* M, int64_t m_stride, const float* W, in
       if (look && (e = cudaEventRecord(look->a[k & 1], sa)) != cudaSuccess) return e;
     }
     // Z_k = Linv Z_k, Y_k = Linv Y_k (to the planes): final from here on
-    if ((e = panel_launch(1, w, linv + NB * NB, d, kk, 0, status, sz)) != cudaSuccess) return e;
+    if ((e = panel_launch(1, w, linv, d, kk, 0, status, sz)) != cudaSuccess) return e;
     if (look && ((e = cudaEventRecord(look->zrow, sz)) != cudaSuccess ||
                  (e = cudaStreamWaitEvent(sw, look->zrow, 0)) != cudaSuccess))
       return e;
@@ -1069,7 +1068,7 @@ cudaError_t absorb_solve_batched(int n, const float* M, int64_t m_stride, const 
       if ((e = launch_tgemm(p, stream)) != cudaSuccess) return e;
     }
     if ((e = launch_pdl(potrf_inv_kernel, dim3(n), dim3(512), kPotrfSmem, stream,
-                        (const float*)(w.A + (size_t)kk * d + kk), dim, w.Linv, ws, status)) !=
+                        (const float*)(w.A + (size_t)kk * d + kk), dim, w.Lh, ws, status)) !=
         cudaSuccess)
       return e;
     count_launches();
