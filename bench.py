@@ -137,14 +137,17 @@ def traffic_file(workload_name):
     return os.path.join(ROOT, "profiles", f"dual_attention_{workload_name}_traffic.txt")
 
 
-def traffic_per_launch(workload_name):
+def traffic_per_launch(workload_name, layers_per_launch=1):
     """DRAM bytes per attention launch of this workload from the committed ncu
-    summary, or None when there is none or the kernel source changed since
-    the counters were taken."""
+    summary, or None when there is none, the kernel source changed since the
+    counters were taken, or they were taken on launches of another number of
+    layers."""
     try:
         with open(traffic_file(workload_name)) as f:
             kv = dict(line.strip().split("=", 1) for line in f if "=" in line and not line.startswith("#"))
         if kv.get("source_hash") != source_hash():
+            return None
+        if int(kv.get("layers_per_launch", "1")) != layers_per_launch:
             return None
         return float(kv["dram_bytes_per_launch"])
     except Exception:
@@ -339,23 +342,22 @@ def workload(args):
 
 def make_inputs(cfg, rank, device, layers=None, replica=True):
     """Per layer: its Q/K/V frame streams and the chunk dicts (views into
-    them); the projections stacked as one [L, d, d] tensor. ``layers`` lists
-    the global layer ids to build (default: all); replicas (one full copy of
-    the workload per rank) draw rank-specific seeds, layer shards the global
+    them); the projections stacked as one [L, d, d] tensor; the streams'
+    storage, one [L, frames, tokens, heads, head_dim] tensor per Q, K, V (a
+    chunk of every layer is one strided view of it). ``layers`` lists the
+    global layer ids to build (default: all); replicas (one full copy of the
+    workload per rank) draw rank-specific seeds, layer shards the global
     ones."""
     import torch
-    from ispa_synth import layer_streams
+    from ispa_synth import stacked_layer_streams
     layers = list(range(cfg.layers)) if layers is None else layers
-    streams, chunks, Ws = [], [], []
-    for l in layers:
-        st = layer_streams(cfg, layer=l + (1000 * rank if replica else 0), seed=0, device=device)
-        streams.append(st)
-        chunks.append([st.chunk(c) for c in range(cfg.n_chunks)])
-        Ws.append(st.w)
-    W_all = torch.stack(Ws)
+    ids = [l + (1000 * rank if replica else 0) for l in layers]
+    streams, qkv = stacked_layer_streams(cfg, ids, seed=0, device=device)
+    chunks = [[st.chunk(c) for c in range(cfg.n_chunks)] for st in streams]
+    W_all = torch.stack([st.w for st in streams])
     for st in streams:
         st.w = None
-    return streams, chunks, W_all
+    return streams, chunks, W_all, qkv
 
 
 def config_of(cfg, world, sharded, K):
@@ -384,21 +386,28 @@ def measure_warmup(args, cfg, world, rank, steps, warmup, with_e2e, with_cpu):
     from kv_cache_absorption_b200 import ispa
     from kv_cache_absorption_b200.warmup import LayerWarmup, rank as rank_layers
     from kv_cache_absorption_b200.sharding import gather_errors, owned_layers
+    from ispa_synth import stacked_chunk
     dev = torch.device("cuda", torch.cuda.current_device())
     # several GPUs: multi-layer warmups shard their layers (l on rank l mod N,
     # errors all-gathered for the ranking); a one-layer step runs as replicas
     sharded = world > 1 and cfg.layers >= world
     my_layers = owned_layers(cfg.layers, world, rank) if sharded else list(range(cfg.layers))
-    layer_streams_, chunks_per_layer, W_all = make_inputs(cfg, rank, dev, my_layers,
-                                                          replica=not sharded)
+    layer_streams_, chunks_per_layer, W_all, qkv = make_inputs(cfg, rank, dev, my_layers,
+                                                               replica=not sharded)
     max_hist = max(len(cfg.history_frames_of(c)) for c in range(cfg.n_chunks)) * cfg.tokens_per_frame
     L = cfg.layers
     L_mine = len(my_layers)
-    # several layers in flight on as many streams (their launches fill each
-    # other's tail SMs); two by default
+    # the same chunk of `group` layers in one attention launch (one grid over
+    # all their units: whole waves of the SMs), groups in flight on as many
+    # streams as slots (their launches fill each other's tails); 10 layers a
+    # launch and two streams by default
+    group = max(1, min(args.group, L_mine))
+    stacked_chunks = ([stacked_chunk(cfg, qkv, c) for c in range(cfg.n_chunks)]
+                      if group > 1 else None)
     runner = LayerWarmup(cfg.heads, cfg.head_dim, cfg.chunk_tokens, cfg.sink_tokens,
                          cfg.chunk_tokens, max_hist, n_layers=L_mine, device=dev,
-                         n_slots=max(1, min(args.slots, L_mine)))
+                         n_slots=max(1, min(args.slots, L_mine)), group=group)
+    groups = runner.layer_groups() if group > 1 else [(l, 1) for l in range(L_mine)]
     K = cfg.select_k if cfg.select_k is not None else L // 2
     err_mine = torch.empty(L_mine, 2, dtype=torch.float64, device=dev)
     err = torch.empty(L, 2, dtype=torch.float64, device=dev)
@@ -409,8 +418,14 @@ def measure_warmup(args, cfg, world, rank, steps, warmup, with_e2e, with_cpu):
     runner.weight_gram(W_all)     # W W^T per layer: model weights only, formed once at load
     streams = [torch.cuda.current_stream()] + [torch.cuda.Stream() for _ in range(runner.n_slots - 1)]
 
+    def chunks_in(sets_stacked, sets_per_layer, strms):
+        if sets_stacked is not None:
+            runner.layers_chunks_stacked(sets_stacked, strms)
+        else:
+            runner.layers_chunks(sets_per_layer, strms)
+
     def step():
-        runner.layers_chunks(chunks_per_layer, streams)
+        chunks_in(stacked_chunks, chunks_per_layer, streams)
         runner.absorb_all(W_all, err_mine)    # every layer's solve + error, batched
         err.copy_(gather_errors(err_mine, L, world) if sharded else err_mine)
         rank_layers(err, K, perm, sel)
@@ -418,12 +433,19 @@ def measure_warmup(args, cfg, world, rank, steps, warmup, with_e2e, with_cpu):
     def step_instrumented(ev):
         """The same work on one stream with events around every stage (the
         per-stage breakdown; not the timed steps)."""
-        for li, chunks in enumerate(chunks_per_layer):
-            for c, ch in enumerate(chunks):
+        for l0, n in groups:
+            for c in range(cfg.n_chunks):
                 ev["a0"].append(E()); ev["a0"][-1].record()
-                runner.attention(ch)
+                if stacked_chunks is not None:
+                    runner.attention_layers(stacked_chunks[c], l0, n)
+                else:
+                    runner.attention(chunks_per_layer[l0][c])
                 ev["a1"].append(E()); ev["a1"][-1].record()
-                runner.gram(first=(c == 0), layer=li)
+                for j in range(n):
+                    if stacked_chunks is not None:
+                        runner.gram_group(c == 0, j, l0 + j)
+                    else:
+                        runner.gram(first=(c == 0), layer=l0 + j)
                 ev["g1"].append(E()); ev["g1"][-1].record()
         runner.absorb_all(W_all, err_mine)
         ev["s1"].append(E()); ev["s1"][-1].record()
@@ -465,7 +487,7 @@ def measure_warmup(args, cfg, world, rank, steps, warmup, with_e2e, with_cpu):
     attn_ms = sum(a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"])) / n_inst
     gram_ms = sum(a.elapsed_time(b) for a, b in zip(ev["a1"], ev["g1"])) / n_inst
     # batched solve + error of all layers: from the end of the last Gram to s1
-    per_step = L_mine * cfg.n_chunks
+    per_step = len(groups) * cfg.n_chunks
     solve_ms = sum(ev["g1"][(i + 1) * per_step - 1].elapsed_time(ev["s1"][i])
                    for i in range(n_inst)) / n_inst
     # the attention calls alone, with the layers in flight on the step's streams
@@ -476,9 +498,14 @@ def measure_warmup(args, cfg, world, rank, steps, warmup, with_e2e, with_cpu):
         fork.record(streams[0])
         for s_ in streams[1:]:
             s_.wait_event(fork)
-        for li, chunks in enumerate(chunks_per_layer):
-            for ch in chunks:
-                runner.attention(ch, stream=streams[li % n_s], slot=li % n_s)
+        for g, (l0, n) in enumerate(groups):
+            for c in range(cfg.n_chunks):
+                if stacked_chunks is not None:
+                    runner.attention_layers(stacked_chunks[c], l0, n, stream=streams[g % n_s],
+                                            slot=g % n_s)
+                else:
+                    runner.attention(chunks_per_layer[l0][c], stream=streams[g % n_s],
+                                     slot=g % n_s)
         for s_ in streams[1:]:
             join = torch.cuda.Event()
             join.record(s_)
@@ -504,15 +531,15 @@ def measure_warmup(args, cfg, world, rank, steps, warmup, with_e2e, with_cpu):
     attn_tflops = work["attention"] * share / (attn_ms * 1e-3) / 1e12
     absorb_ms_layer = (gram_ms + solve_ms) / L_mine
     bf16_peak, hbm_peak, peak_src = peaks()
-    attn_launches = L_mine * cfg.n_chunks
+    attn_launches = len(groups) * cfg.n_chunks
     sm_mhz = clocks.get("sm_mhz") if clocks else None
     roofline = {
         "bound": "tensor", "kernel": "dual-stream attention (branch_attention_kernel, merge fused)",
         "achieved": round(attn_tflops, 2), "peak": bf16_peak, "unit": "TFLOP/s",
         "frac": round(attn_tflops / bf16_peak, 4), "peak_source": f"{peak_src} bf16 dense (burst)",
-        "traffic": traffic_per_launch(cfg.name),
+        "traffic": traffic_per_launch(cfg.name, group),
         "algorithmic_flops_per_launch": work["attention"] * share / attn_launches,
-        "algorithmic_bytes_per_launch": attention_bytes(cfg) / cfg.n_chunks,
+        "algorithmic_bytes_per_launch": attention_bytes(cfg) * L_mine / attn_launches,
         "ms_per_launch": attn_ms / attn_launches,
         "launches_per_step": attn_launches,
         # box-to-box comparable: the attention time in SM clock cycles
@@ -535,6 +562,7 @@ def measure_warmup(args, cfg, world, rank, steps, warmup, with_e2e, with_cpu):
         "attention_frac_layers_in_flight": round(work["attention"] * share
                                                  / (attn_streams_ms * 1e-3) / 1e12 / bf16_peak, 4),
         "attention_streams": len(streams),
+        "attention_layers_per_launch": group,
         "absorb_ms_per_layer": round(absorb_ms_layer, 4),
         "gram_ms_per_step": round(gram_ms, 4), "solve_error_ms_per_step": round(solve_ms, 4),
         "absorb_tflops": round(absorb_flops / ((gram_ms + solve_ms) * 1e-3) / 1e12, 2),
@@ -546,8 +574,9 @@ def measure_warmup(args, cfg, world, rank, steps, warmup, with_e2e, with_cpu):
         "clocks": clocks,
     }
     if with_e2e:
-        out["e2e"] = run_e2e(args, cfg, layer_streams_, chunks_per_layer, W_all, runner, err,
-                             perm, sel, K, world, err_mine if sharded else None, streams)
+        out["e2e"] = run_e2e(args, cfg, layer_streams_, chunks_per_layer, qkv, W_all, runner,
+                             err, perm, sel, K, world, err_mine if sharded else None, streams,
+                             grouped=stacked_chunks is not None)
     if with_cpu and rank == 0 and world == 1:
         out["cpu_baseline"] = oracle_throughput(cfg, args.cpu_budget)
     return out
@@ -598,8 +627,8 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_e2e(args, cfg, streams, chunks_per_layer, W_all, runner, err, perm, sel, K, world,
-            err_mine=None, cuda_streams=None):
+def run_e2e(args, cfg, streams, chunks_per_layer, qkv, W_all, runner, err, perm, sel, K, world,
+            err_mine=None, cuda_streams=None, grouped=False):
     """Same step through the public API with the instance's inputs in pinned
     host memory: every step copies each layer's Q/K/V frame streams
     host->device, runs the warmup, and copies every Delta W, the errors and
@@ -610,19 +639,25 @@ def run_e2e(args, cfg, streams, chunks_per_layer, W_all, runner, err, perm, sel,
     copy to the last result read back."""
     import dataclasses
     import torch
+    from ispa_synth import stacked_chunk
     from kv_cache_absorption_b200.warmup import rank as rank_layers
     from kv_cache_absorption_b200.sharding import gather_errors
-    sets = [(streams, chunks_per_layer)]
-    clones = [dataclasses.replace(st, q=torch.empty_like(st.q), k=torch.empty_like(st.k),
-                                  v=torch.empty_like(st.v)) for st in streams]
-    sets.append((clones, [[st.chunk(c) for c in range(cfg.n_chunks)] for st in clones]))
-    dev_sets = [[t for st in ss for t in (st.q, st.k, st.v)] for ss, _ in sets]
-    for ss, chunks in sets:           # every chunk input is a view into an uploaded stream
-        owners = {t.untyped_storage().data_ptr() for st in ss for t in (st.q, st.k, st.v)}
-        for layer_chunks in chunks:
-            for ch in layer_chunks:
-                assert all(x.numel() == 0 or x.untyped_storage().data_ptr() in owners
-                           for x in ch.values())
+    # two device input sets, each the three [L, frames, ...] stream tensors;
+    # the per-layer and stacked chunks are views into them
+    qkv2 = tuple(torch.empty_like(x) for x in qkv)
+    clones = [dataclasses.replace(st, q=qkv2[0][i], k=qkv2[1][i], v=qkv2[2][i])
+              for i, st in enumerate(streams)]
+    sets = []
+    for ss, store in ((streams, qkv), (clones, qkv2)):
+        per_layer = [[st.chunk(c) for c in range(cfg.n_chunks)] for st in ss]
+        stacked = [stacked_chunk(cfg, store, c) for c in range(cfg.n_chunks)] if grouped else None
+        sets.append((per_layer, stacked, store))
+    dev_sets = [list(store) for _, _, store in sets]
+    for per_layer, stacked, store in sets:   # every chunk input is a view into an uploaded set
+        owners = {t.untyped_storage().data_ptr() for t in store}
+        views = [x for layer_chunks in per_layer for ch in layer_chunks for x in ch.values()]
+        views += [x for sch in (stacked or []) for x in sch.values()]
+        assert all(x.numel() == 0 or x.untyped_storage().data_ptr() in owners for x in views)
     host_tensors = [t.cpu().pin_memory() for t in dev_sets[0]]
     L, d = cfg.layers, cfg.d
     dW_host = torch.empty(runner.n_layers, d, d, dtype=torch.float32).pin_memory()
@@ -647,7 +682,10 @@ def run_e2e(args, cfg, streams, chunks_per_layer, W_all, runner, err, perm, sel,
     def compute_step(i):
         b = i % 2
         compute.wait_event(copied[b])
-        runner.layers_chunks(sets[b][1], cuda_streams)
+        if grouped:
+            runner.layers_chunks_stacked(sets[b][1], cuda_streams)
+        else:
+            runner.layers_chunks(sets[b][0], cuda_streams)
         if err_mine is not None:
             runner.absorb_all(W_all, err_mine)
             err.copy_(gather_errors(err_mine, L, world))
@@ -709,7 +747,7 @@ def run_streaming(args):
     cfg = workload(args)
     if cfg.stream_chunks < 1:
         raise SystemExit("the streaming benchmark needs a workload with streaming chunks (c4)")
-    streams, warm_chunks, W_all = make_inputs(cfg, rank, dev)
+    streams, warm_chunks, W_all, _ = make_inputs(cfg, rank, dev)
     L = cfg.layers
     K = cfg.select_k if cfg.select_k is not None else L // 2
     # warmup and transition
@@ -974,6 +1012,8 @@ def main():
                     help="override the workload's layer count (smaller captures for ncu)")
     ap.add_argument("--slots", type=int, default=2,
                     help="layers in flight on separate streams in a multi-layer warmup")
+    ap.add_argument("--group", type=int, default=10,
+                    help="layers per attention launch in the warmups (1: one launch per layer)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sub", action="store_true",
                     help="measure only the main workload (no 14B / single-chunk sub-objects)")

@@ -67,6 +67,17 @@ typedef struct {
   int64_t len;
 } ispa_kv;
 
+/* One branch of the KV cache of several layers: layer l's keys and values
+ * [len, heads, head_dim] bf16 start l * layer_stride elements after k and v
+ * (layer_stride a multiple of 8, >= len * heads * head_dim when there are
+ * several layers). len may be 0 (then k and v are ignored and may be NULL). */
+typedef struct {
+  const void* k;
+  const void* v;
+  int64_t len;
+  int64_t layer_stride;
+} ispa_kv_layers;
+
 /* Text for a return code or a status bit. Never NULL. Host only. */
 ISPA_API const char* ispa_status_string(int code);
 
@@ -147,6 +158,32 @@ ISPA_API int ispa_dual_attention(const void* q, int64_t nq, int heads, int head_
                         ispa_kv local, ispa_kv hist, float scale, float* a_loc, float* d_out,
                         void* a_full, float* lse_loc, float* lse_hist, float* lse_full,
                         void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
+
+/* ispa_dual_attention for n_layers layers of one shape in one launch (the
+ * same chunk of every layer: layers are independent until the transition,
+ * and one grid over all of them fills whole waves where one layer's units
+ * would leave a tail). Layer l's q starts l * q_layer_stride elements after
+ * q, its keys and values as ispa_kv_layers says, its a_loc, d_out and a_full
+ * l * out_layer_stride elements after layer 0's, its LSEs l *
+ * lse_layer_stride after. With several layers the strides are at least one
+ * layer's extent (nq * d, heads * nq), q_layer_stride and out_layer_stride
+ * multiples of 8. workspace: >= ispa_dual_attention_layers_workspace_size()
+ * bytes (n_layers single-layer workspaces, 256-byte aligned). Each layer's
+ * results equal those of ispa_dual_attention on that layer alone, bit for
+ * bit. Other arguments, status and errors as ispa_dual_attention.
+ */
+ISPA_API size_t ispa_dual_attention_layers_workspace_size(int n_layers, int64_t nq,
+                                                          int64_t sink_len, int64_t local_len,
+                                                          int64_t hist_len, int heads,
+                                                          int head_dim);
+ISPA_API int ispa_dual_attention_layers(int n_layers, const void* q, int64_t q_layer_stride,
+                                        int64_t nq, int heads, int head_dim, ispa_kv_layers sink,
+                                        ispa_kv_layers local, ispa_kv_layers hist, float scale,
+                                        float* a_loc, float* d_out, void* a_full,
+                                        int64_t out_layer_stride, float* lse_loc, float* lse_hist,
+                                        float* lse_full, int64_t lse_layer_stride,
+                                        void* workspace, size_t workspace_bytes, int* dev_status,
+                                        void* stream);
 
 /* ---- 1b. local attention (L-Layer after the transition) --------------
  * Technical summary section 2, step 3: a local-attention layer keeps only

@@ -192,6 +192,48 @@ def layer_streams(cfg: Config, layer: int, seed: int = 0, device="cpu",
     return LayerStreams(cfg, mk("Q"), mk("K"), mk("V"), projection(cfg.d, seed, layer, device))
 
 
+def stacked_layer_streams(cfg: Config, layers: List[int], seed: int = 0, device="cpu",
+                          n_frames: Optional[int] = None, gen_device=None):
+    """layer_streams of several layers with their Q, K and V each in one
+    [L, n_frames, tokens_per_frame, heads, head_dim] tensor on ``device``:
+    stream i's q, k and v are views of entry i (layer ``layers[i]``), so
+    that one chunk of every layer is one strided tensor (``stacked_chunk``).
+    Each layer is drawn on ``gen_device`` (default: ``device``; the draws
+    depend on the device the generator runs on) and copied in. Returns the
+    streams and the (Q, K, V) storage."""
+    gen_device = device if gen_device is None else gen_device
+    nf = cfg.n_frames if n_frames is None else n_frames
+    shape = (len(layers), nf, cfg.tokens_per_frame, cfg.heads, cfg.head_dim)
+    Q, K, V = (torch.empty(shape, dtype=torch.bfloat16, device=device) for _ in range(3))
+    streams = []
+    for i, l in enumerate(layers):
+        st = layer_streams(cfg, l, seed, gen_device, n_frames=nf)
+        Q[i].copy_(st.q)
+        K[i].copy_(st.k)
+        V[i].copy_(st.v)
+        streams.append(LayerStreams(cfg, Q[i], K[i], V[i], st.w.to(device)))
+        del st
+    return streams, (Q, K, V)
+
+
+def stacked_chunk(cfg: Config, qkv, c: int) -> dict:
+    """Chunk c of every layer of a ``stacked_layer_streams`` storage: the
+    inputs of LayerStreams.chunk(c) as [L, tokens, heads, head_dim] views
+    (each layer's rows contiguous, the layers one stream apart)."""
+    Q, K, V = qkv
+    L, H, hd = Q.shape[0], cfg.heads, cfg.head_dim
+
+    def rows(x, frames):
+        if not frames:
+            return x.new_zeros(L, 0, H, hd)
+        return x[:, frames[0]:frames[-1] + 1].reshape(L, -1, H, hd)
+
+    cur, hist = cfg.chunk_frames_of(c), cfg.history_frames_of(c)
+    return {"q": rows(Q, cur), "k_sink": K[:, 0, :cfg.sink_tokens], "v_sink": V[:, 0, :cfg.sink_tokens],
+            "k_loc": rows(K, cur), "v_loc": rows(V, cur),
+            "k_hist": rows(K, hist), "v_hist": rows(V, hist)}
+
+
 def gaussian(shape, seed: int, layer: int = 0, tensor: str = "X", device="cpu",
              dtype=torch.float32) -> torch.Tensor:
     """Plain seeded N(0, 1) draws for kernel-level tests that feed a stage

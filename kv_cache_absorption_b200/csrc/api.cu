@@ -44,6 +44,7 @@ namespace {
 using ispa::AttnParams;
 using ispa::cuda_rc;
 using ispa::encode_2d;
+using ispa::encode_3d;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
@@ -84,11 +85,19 @@ size_t attention_workspace(int64_t nq, int64_t sink_len, int64_t local_len, int6
   return counters + (size_t)slots * (lse + out) + 256;
 }
 
+// Layers of one call: layer l's Q, keys and values, outputs and LSEs start
+// l times these strides (elements) after layer 0's; its workspace l times the
+// single-layer workspace after.
+struct LayerStrides {
+  int n = 1;
+  int64_t q = 0, kv[3] = {0, 0, 0}, out = 0, lse = 0;
+};
+
 int attention_common(const void* q, int64_t nq, int heads, int head_dim, const ispa_kv (&br)[3],
                      float scale, int round_tf32, float* a_loc, float* d_out, void* a_full,
                      float* lse_loc, float* lse_hist, float* lse_full, void* workspace,
                      size_t workspace_bytes, int* dev_status, void* stream,
-                     bool full_only = false) {
+                     bool full_only = false, const LayerStrides& ls = LayerStrides()) {
   if (!q || !dev_status || nq < 0 || nq > (int64_t)1 << 30 || heads < 1 || heads > 65535)
     return ISPA_ERR_ARG;
   if (head_dim != 64 && head_dim != 128) return ISPA_ERR_UNSUPPORTED;
@@ -100,9 +109,20 @@ int attention_common(const void* q, int64_t nq, int heads, int head_dim, const i
       (a_full && !aligned16(a_full)))
     return ISPA_ERR_UNSUPPORTED;
   const int d = heads * head_dim;
+  if (ls.n < 1 || ls.n > 65535) return ISPA_ERR_ARG;
+  if (ls.n > 1) {
+    // layers may not overlap; every layer's rows stay 16-byte aligned
+    if (ls.q < nq * d || ls.out < nq * d || ls.lse < heads * nq) return ISPA_ERR_ARG;
+    for (int b = 0; b < 3; ++b)
+      if (br[b].len > 0 && ls.kv[b] < br[b].len * d) return ISPA_ERR_ARG;
+    if (ls.q % 8 || ls.out % 8 || ls.kv[0] % 8 || ls.kv[1] % 8 || ls.kv[2] % 8)
+      return ISPA_ERR_UNSUPPORTED;
+  }
   // the local slot lives in the workspace when A_loc is not an output
   const bool local_in_ws = full_only || a_loc == nullptr;
-  const size_t need = attention_workspace(nq, br[0].len, br[1].len, br[2].len, heads, head_dim);
+  const size_t per_layer =
+      attention_workspace(nq, br[0].len, br[1].len, br[2].len, heads, head_dim);
+  const size_t need = per_layer * (size_t)ls.n;
   if (!workspace || workspace_bytes < need || !aligned256(workspace)) return ISPA_ERR_WORKSPACE;
   int rc = check_device();
   if (rc != ISPA_OK) return rc;
@@ -111,7 +131,7 @@ int attention_common(const void* q, int64_t nq, int heads, int head_dim, const i
 
   AttnParams p;
   std::memset(&p, 0, sizeof(p));
-  if (!encode_2d(&p.tm_q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, nq, d, 64, 128,
+  if (!encode_3d(&p.tm_q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, nq, d, ls.n, ls.q, 64, 128,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return ISPA_ERR_CUDA;
   for (int b = 0; b < 3; ++b) {
@@ -121,10 +141,10 @@ int attention_common(const void* q, int64_t nq, int heads, int head_dim, const i
       p.tm_v[b] = p.tm_q;
       continue;
     }
-    if (!encode_2d(&p.tm_k[b], br[b].k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, br[b].len, d, 64, 128,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&p.tm_v[b], br[b].v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, br[b].len, d, 64,
-                   128, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!encode_3d(&p.tm_k[b], br[b].k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, br[b].len, d,
+                   ls.n, ls.kv[b], 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_3d(&p.tm_v[b], br[b].v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, br[b].len, d,
+                   ls.n, ls.kv[b], 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
       return ISPA_ERR_CUDA;
   }
   p.plan = ispa::attention_plan(nq, br[0].len, br[1].len, br[2].len, heads);
@@ -155,6 +175,10 @@ int attention_common(const void* q, int64_t nq, int heads, int head_dim, const i
   p.lse_loc = lse_loc;
   p.lse_hist = lse_hist;
   p.lse_full = lse_full;
+  p.n_layers = ls.n;
+  p.out_lstride = ls.out;
+  p.lse_lstride = ls.lse;
+  p.ws_lstride = (int64_t)per_layer;
   p.status = dev_status;
   return cuda_rc(ispa::launch_dual_attention(p, head_dim, s));
 }
@@ -235,6 +259,37 @@ int ispa_dual_attention(const void* q, int64_t nq, int heads, int head_dim, ispa
   const ispa_kv br[3] = {sink, local, hist};
   return attention_common(q, nq, heads, head_dim, br, scale, 1, a_loc, d_out, a_full, lse_loc,
                           lse_hist, lse_full, workspace, workspace_bytes, dev_status, stream);
+}
+
+size_t ispa_dual_attention_layers_workspace_size(int n_layers, int64_t nq, int64_t sink_len,
+                                                 int64_t local_len, int64_t hist_len, int heads,
+                                                 int head_dim) {
+  if (n_layers < 1 || n_layers > 65535) return 0;
+  return attention_workspace(nq, sink_len, local_len, hist_len, heads, head_dim) * (size_t)n_layers;
+}
+
+int ispa_dual_attention_layers(int n_layers, const void* q, int64_t q_layer_stride, int64_t nq,
+                               int heads, int head_dim, ispa_kv_layers sink, ispa_kv_layers local,
+                               ispa_kv_layers hist, float scale, float* a_loc, float* d_out,
+                               void* a_full, int64_t out_layer_stride, float* lse_loc,
+                               float* lse_hist, float* lse_full, int64_t lse_layer_stride,
+                               void* workspace, size_t workspace_bytes, int* dev_status,
+                               void* stream) {
+  ISPA_NVTX_RANGE();
+  if (!a_loc || !d_out || n_layers < 1) return ISPA_ERR_ARG;
+  const ispa_kv br[3] = {{sink.k, sink.v, sink.len}, {local.k, local.v, local.len},
+                         {hist.k, hist.v, hist.len}};
+  LayerStrides ls;
+  ls.n = n_layers;
+  ls.q = q_layer_stride;
+  ls.kv[0] = sink.layer_stride;
+  ls.kv[1] = local.layer_stride;
+  ls.kv[2] = hist.layer_stride;
+  ls.out = out_layer_stride;
+  ls.lse = lse_layer_stride;
+  return attention_common(q, nq, heads, head_dim, br, scale, 1, a_loc, d_out, a_full, lse_loc,
+                          lse_hist, lse_full, workspace, workspace_bytes, dev_status, stream,
+                          false, ls);
 }
 
 int ispa_local_attention(const void* q, int64_t nq, int heads, int head_dim, ispa_kv sink,

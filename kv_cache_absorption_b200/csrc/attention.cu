@@ -90,6 +90,7 @@ struct alignas(1024) Smem {
 };
 
 struct Unit {
+  int layer;
   int head;
   int pair;
   int q0;          // first query row of the pair
@@ -101,12 +102,15 @@ struct Unit {
 };
 
 // Grid order: for each slot in p.order (longest key range first), every
-// (head, query pair).
+// (layer, head, query pair).
 __device__ __forceinline__ Unit unit_of(const AttnParams& p) {
   Unit u;
   const int per = p.heads * p.n_pairs;
-  const int b = blockIdx.x % per;
-  u.slot = p.order[blockIdx.x / per];
+  const int per_slot = per * p.n_layers;
+  const int lb = blockIdx.x % per_slot;
+  u.slot = p.order[blockIdx.x / per_slot];
+  u.layer = lb / per;
+  const int b = lb % per;
   u.head = b / p.n_pairs;
   u.pair = b % p.n_pairs;
   u.q0 = u.pair * (BM * NQT);
@@ -229,10 +233,48 @@ __device__ __forceinline__ float log_add_exp(float x, float y) {
   return hi == -INFINITY ? hi : hi + log1pf(expf(lo - hi));
 }
 
+// One layer's outputs and workspace (the launch's layer-0 pointers moved by
+// the layer strides; null outputs stay null).
+struct LayerIO {
+  float* a_loc;
+  float* d_out;
+  __nv_bfloat16* a_full;
+  float* lse_loc;
+  float* lse_hist;
+  float* lse_full;
+  float* part;
+  float* part_lse;
+  int* counters;
+};
+
+template <typename T>
+__device__ __forceinline__ T* moved(T* ptr, int64_t elems) {
+  return ptr ? ptr + elems : nullptr;
+}
+template <typename T>
+__device__ __forceinline__ T* moved_bytes(T* ptr, int64_t bytes) {
+  return ptr ? reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(ptr) + bytes) : nullptr;
+}
+
+__device__ __forceinline__ LayerIO layer_io(const AttnParams& p, int layer) {
+  const int64_t o = layer * p.out_lstride, l = layer * p.lse_lstride, w = layer * p.ws_lstride;
+  LayerIO io;
+  io.a_loc = moved(p.a_loc, o);
+  io.d_out = moved(p.d_out, o);
+  io.a_full = moved(p.a_full, o);
+  io.lse_loc = moved(p.lse_loc, l);
+  io.lse_hist = moved(p.lse_hist, l);
+  io.lse_full = moved(p.lse_full, l);
+  io.part = moved_bytes(p.part, w);
+  io.part_lse = moved_bytes(p.part_lse, w);
+  io.counters = moved_bytes(p.counters, w);
+  return io;
+}
+
 // Where slot k's normalised output lives: slot 0 in a_loc itself when the
 // plan says so (stored rounded like the final A_loc), else the workspace.
-__device__ __forceinline__ float* slot_out(const AttnParams& p, int k) {
-  return k < p.part_first ? p.a_loc : p.part + (int64_t)(k - p.part_first) * p.part_stride;
+__device__ __forceinline__ float* slot_out(const AttnParams& p, const LayerIO& io, int k) {
+  return k < p.part_first ? io.a_loc : io.part + (int64_t)(k - p.part_first) * p.part_stride;
 }
 
 // bf16 -> fp16 of one 16-byte chunk (8 values); `big` collects |v| >= 2^16
@@ -325,8 +367,8 @@ __device__ __forceinline__ void rows_out(float* st, const float (&v)[32], int ro
 // D = sum_hist w_s (O_s - A_loc), A_full = A_loc + D. Slots are summed in
 // slot order, so the result does not depend on which unit came last.
 template <int HD>
-__device__ __forceinline__ void merge_rows(const AttnParams& p, const Unit& u, const float* stage,
-                                           const float* stats, int n_epi) {
+__device__ __forceinline__ void merge_rows(const AttnParams& p, const LayerIO& io, const Unit& u,
+                                           const float* stage, const float* stats, int n_epi) {
   constexpr int VEC = HD / 32;
   constexpr int G = 8;
   constexpr int kLd = HD + 4;
@@ -356,7 +398,7 @@ __device__ __forceinline__ void merge_rows(const AttnParams& p, const Unit& u, c
 #pragma unroll
         for (int i = 0; i < VEC; ++i) al[g][i] = stage[(r0 + g) * kLd + lane * VEC + i];
     } else if (n_ls == 1) {
-      const float* src = slot_out(p, 0);
+      const float* src = slot_out(p, io, 0);
 #pragma unroll
       for (int g = 0; g < G; ++g)
         if (ok[g]) ld_vec<VEC>(src + off[g], al[g]);
@@ -370,15 +412,15 @@ __device__ __forceinline__ void merge_rows(const AttnParams& p, const Unit& u, c
         if (k == u.slot) {
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            w[g] = ok[g] ? __ldcg(p.part_lse + k * p.lse_stride + li[g]) : 0.f;
+            w[g] = ok[g] ? __ldcg(io.part_lse + k * p.lse_stride + li[g]) : 0.f;
 #pragma unroll
             for (int i = 0; i < VEC; ++i) x[g][i] = stage[(r0 + g) * kLd + lane * VEC + i];
           }
         } else {
-          const float* src = slot_out(p, k);
+          const float* src = slot_out(p, io, k);
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            w[g] = ok[g] ? __ldcg(p.part_lse + k * p.lse_stride + li[g]) : 0.f;
+            w[g] = ok[g] ? __ldcg(io.part_lse + k * p.lse_stride + li[g]) : 0.f;
             if (ok[g]) ld_vec<VEC>(src + off[g], x[g]);
           }
         }
@@ -395,7 +437,7 @@ __device__ __forceinline__ void merge_rows(const AttnParams& p, const Unit& u, c
 #pragma unroll
           for (int i = 0; i < VEC; ++i) al[g][i] = to_tf32(al[g][i]);
         }
-        if (ok[g] && p.a_loc) st_vec<VEC>(p.a_loc + off[g], al[g], false);
+        if (ok[g] && io.a_loc) st_vec<VEC>(io.a_loc + off[g], al[g], false);
       }
     }
     // D = A_full - A_loc
@@ -408,15 +450,15 @@ __device__ __forceinline__ void merge_rows(const AttnParams& p, const Unit& u, c
       if (k == u.slot) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          w[g] = ok[g] ? __ldcg(p.part_lse + k * p.lse_stride + li[g]) : 0.f;
+          w[g] = ok[g] ? __ldcg(io.part_lse + k * p.lse_stride + li[g]) : 0.f;
 #pragma unroll
           for (int i = 0; i < VEC; ++i) x[g][i] = stage[(r0 + g) * kLd + lane * VEC + i];
         }
       } else {
-        const float* src = slot_out(p, k);
+        const float* src = slot_out(p, io, k);
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          w[g] = ok[g] ? __ldcg(p.part_lse + k * p.lse_stride + li[g]) : 0.f;
+          w[g] = ok[g] ? __ldcg(io.part_lse + k * p.lse_stride + li[g]) : 0.f;
           if (ok[g]) ld_vec<VEC>(src + off[g], x[g]);
         }
       }
@@ -430,11 +472,11 @@ __device__ __forceinline__ void merge_rows(const AttnParams& p, const Unit& u, c
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       if (!ok[g]) continue;
-      if (p.d_out) st_vec<VEC>(p.d_out + off[g], acc[g], rnd);
-      if (p.a_full) {
+      if (io.d_out) st_vec<VEC>(io.d_out + off[g], acc[g], rnd);
+      if (io.a_full) {
 #pragma unroll
         for (int i = 0; i < VEC; ++i) x[g][i] = al[g][i] + acc[g][i];
-        st_vec_bf16<VEC>(p.a_full + off[g], x[g]);
+        st_vec_bf16<VEC>(io.a_full + off[g], x[g]);
       }
     }
   }
@@ -449,6 +491,7 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const Unit u = unit_of(p);
+  const LayerIO io = layer_io(p, u.layer);
   const int n_tiles = u.n_tiles;
   volatile int* abort_flag = &s.abort_flag;
 
@@ -487,7 +530,7 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
       mbar_expect_tx(&s.q_full, u.n_qt * (HD / 64) * BM * 128);
       for (int t = 0; t < u.n_qt; ++t)
         for (int b = 0; b < HD / 64; ++b)
-          tma_load_2d(s.q[t][b], &p.tm_q, &s.q_full, u.head * HD + b * 64, u.q0 + t * BM);
+          tma_load_3d(s.q[t][b], &p.tm_q, &s.q_full, u.head * HD + b * 64, u.q0 + t * BM, u.layer);
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
         const TileInfo ti = tile_of(u.t0 + j, u.hist, p);
@@ -495,12 +538,14 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
         if (j >= NK && !mbar_wait(&s.k_empty[sk], ((j / NK) - 1) & 1, p.status, abort_flag, p.wait_ns)) break;
         mbar_expect_tx(&s.k_full[sk], (HD / 64) * BN * 128);
         for (int b = 0; b < HD / 64; ++b)
-          tma_load_2d(s.k[sk][b], &p.tm_k[ti.branch], &s.k_full[sk], u.head * HD + b * 64, ti.row0);
+          tma_load_3d(s.k[sk][b], &p.tm_k[ti.branch], &s.k_full[sk], u.head * HD + b * 64, ti.row0,
+                      u.layer);
         k_issued = j + 1;
         if (j >= NV && !mbar_wait(&s.v_empty[sv], ((j / NV) - 1) & 1, p.status, abort_flag, p.wait_ns)) break;
         mbar_expect_tx(&s.v_full[sv], (HD / 64) * BN * 128);
         for (int b = 0; b < HD / 64; ++b)
-          tma_load_2d(s.v[sv][b], &p.tm_v[ti.branch], &s.v_full[sv], u.head * HD + b * 64, ti.row0);
+          tma_load_3d(s.v[sv][b], &p.tm_v[ti.branch], &s.v_full[sv], u.head * HD + b * 64, ti.row0,
+                      u.layer);
         v_issued = j + 1;
       }
       // Every copy issued has landed before the CTA exits, whether or not a
@@ -701,21 +746,21 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
           float a[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(raw[i]) * inv;
-          rows_out(wst, a, wrow0, p.nq, d, p.a_loc ? p.a_loc + wbase + c * 32 : nullptr,
-                   p.round_tf32 != 0, p.a_full ? p.a_full + wbase + c * 32 : nullptr,
-                   p.d_out ? p.d_out + wbase + c * 32 : nullptr);
+          rows_out(wst, a, wrow0, p.nq, d, io.a_loc ? io.a_loc + wbase + c * 32 : nullptr,
+                   p.round_tf32 != 0, io.a_full ? io.a_full + wbase + c * 32 : nullptr,
+                   io.d_out ? io.d_out + wbase + c * 32 : nullptr);
         }
         if (row_ok) {
-          if (p.lse_loc) p.lse_loc[li] = lse;
-          if (p.lse_hist) p.lse_hist[li] = -INFINITY;
-          if (p.lse_full) p.lse_full[li] = lse;
+          if (io.lse_loc) io.lse_loc[li] = lse;
+          if (io.lse_hist) io.lse_hist[li] = -INFINITY;
+          if (io.lse_full) io.lse_full[li] = lse;
         }
         // a finite LSE bounds every output of the row (softmax averages of V)
         nonfinite = row_ok && !finite_f(lse);
       } else {
         // 1. this unit's slot: normalised output and LSE
         const bool own_rnd = u.slot < p.part_first && p.round_tf32 != 0;
-        float* own = slot_out(p, u.slot);
+        float* own = slot_out(p, io, u.slot);
 #pragma unroll 1
         for (int c = 0; c < HD / 32; ++c) {
           uint32_t raw[32];
@@ -726,12 +771,12 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
           for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(raw[i]) * inv;
           rows_out(wst, a, wrow0, p.nq, d, own + wbase + c * 32, own_rnd, nullptr, nullptr);
         }
-        if (row_ok) p.part_lse[u.slot * p.lse_stride + li] = lse;
+        if (row_ok) io.part_lse[u.slot * p.lse_stride + li] = lse;
         // 2. count this unit finished; the last of the (head, pair) merges
         __threadfence();
         epi_barrier(n_epi);
         if (threadIdx.x == 128) {
-          const int done = atomicAdd(&p.counters[u.head * p.n_pairs + u.pair], 1);
+          const int done = atomicAdd(&io.counters[u.head * p.n_pairs + u.pair], 1);
           s.merge = (done == n_slots - 1) ? 1 : 0;
           __threadfence();
         }
@@ -766,7 +811,7 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
           if (row_ok) {
 #pragma unroll 4
             for (int k = 0; k < n_slots; ++k) {
-              const float v = __ldcg(p.part_lse + k * p.lse_stride + li);
+              const float v = __ldcg(io.part_lse + k * p.lse_stride + li);
               if (k < n_ls) lse_loc = log_add_exp(lse_loc, v);
               else lse_hist = log_add_exp(lse_hist, v);
             }
@@ -775,15 +820,15 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
           stats[2 * rr] = lse_loc;
           stats[2 * rr + 1] = lse_full;
           if (row_ok) {
-            if (p.lse_loc) p.lse_loc[li] = lse_loc;
-            if (p.lse_hist) p.lse_hist[li] = lse_hist;
-            if (p.lse_full) p.lse_full[li] = lse_full;
+            if (io.lse_loc) io.lse_loc[li] = lse_loc;
+            if (io.lse_hist) io.lse_hist[li] = lse_hist;
+            if (io.lse_full) io.lse_full[li] = lse_full;
           }
           nonfinite = row_ok && !finite_f(lse_full);
           epi_barrier(n_epi);
           // (b) every epilogue warp merges whole rows of the pair: coalesced
           // loads of the other slots, several rows in flight a warp
-          merge_rows<HD>(p, u, stage, stats, n_epi);
+          merge_rows<HD>(p, io, u, stage, stats, n_epi);
         }
       }
       if (__any_sync(0xffffffffu, nonfinite) && lane == 0) atomicOr(p.status, ISPA_STATUS_NONFINITE);
@@ -965,10 +1010,16 @@ AttnPlan attention_plan(int64_t nq, int64_t sink_len, int64_t local_len, int64_t
 cudaError_t launch_dual_attention(const AttnParams& p0, int head_dim, cudaStream_t stream) {
   AttnParams p = p0;
   p.wait_ns = wait_limit_ns();
-  const int units = p.heads * p.n_pairs * p.plan.n_slots();
+  if (p.n_layers < 1) return cudaErrorInvalidValue;
+  const int units = p.heads * p.n_pairs * p.plan.n_slots() * p.n_layers;
   const size_t smem = attention_smem_bytes(head_dim);
   if (p.plan.n_slots() > 1) {
-    cudaError_t e = cudaMemsetAsync(p.counters, 0, sizeof(int) * p.heads * p.n_pairs, stream);
+    // every layer's completion counters (ws_lstride bytes apart) to zero
+    const size_t width = sizeof(int) * p.heads * p.n_pairs;
+    cudaError_t e = p.n_layers == 1
+                        ? cudaMemsetAsync(p.counters, 0, width, stream)
+                        : cudaMemset2DAsync(p.counters, (size_t)p.ws_lstride, 0, width,
+                                            (size_t)p.n_layers, stream);
     if (e != cudaSuccess) return e;
   }
   if (head_dim == 64) {

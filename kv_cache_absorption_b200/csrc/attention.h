@@ -25,9 +25,12 @@ struct AttnPlan {
   __host__ __device__ int n_slots() const { return n_ls + n_hs; }
 };
 
-// Parameters of one dual-stream attention launch. Tensor maps address
-// [len, heads * head_dim] bf16 row-major matrices in 64-column x 128-row
-// boxes with 128-byte swizzle.
+// Parameters of one dual-stream attention launch over n_layers layers of the
+// same shape. Tensor maps address [n_layers][len, heads * head_dim] bf16
+// row-major matrices (x = column, y = row, z = layer) in 64-column x 128-row
+// boxes with 128-byte swizzle. Layer l's outputs start out_lstride (A_loc,
+// D, A_full) or lse_lstride (LSEs) elements after layer 0's, its workspace
+// ws_lstride bytes after (part, part_lse and counters below are layer 0's).
 struct AttnParams {
   CUtensorMap tm_q;
   CUtensorMap tm_k[3];    // sink, local, history
@@ -54,6 +57,10 @@ struct AttnParams {
   float* part_lse;        // [slots][heads, nq]
   int64_t lse_stride;     // elements between slots in `part_lse`
   int* counters;          // [heads * n_pairs] units finished, zero at launch
+  int n_layers;
+  int64_t out_lstride;
+  int64_t lse_lstride;
+  int64_t ws_lstride;
   int* status;
   uint64_t wait_ns;       // limit of a pipeline wait (set at launch)
 };

@@ -59,6 +59,22 @@ bool encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esi
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t cols,
+               uint64_t rows, uint64_t ld, uint64_t layers, uint64_t layer_stride,
+               uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  if (layers < 1) layers = 1;
+  if (layers == 1) layer_stride = rows * ld;   // unused: any valid stride
+  cuuint64_t dims[3] = {cols, rows, layers};
+  cuuint64_t strides[2] = {ld * (uint64_t)esize, layer_stride * (uint64_t)esize};
+  cuuint32_t box[3] = {box_cols, box_rows, 1u};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_f32_operand(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols,
                         uint64_t ld, bool mn_major) {
   return mn_major ? encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, cols, rows, ld, 32, 32,

@@ -45,6 +45,13 @@ bool encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esi
                uint64_t rows, uint64_t ld, uint32_t box_cols, uint32_t box_rows,
                CUtensorMapSwizzle sw);
 
+// [layers][rows, cols] matrices, row stride ld and layer stride layer_stride
+// (elements), tiles of box_cols x box_rows x 1 (x = column, y = row,
+// z = layer). Returns false if the driver rejects the map.
+bool encode_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t cols,
+               uint64_t rows, uint64_t ld, uint64_t layers, uint64_t layer_stride,
+               uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw);
+
 // fp32 operand maps for tgemm: K-major (32 x 128 boxes, 128-byte swizzle) or
 // MN-major (32 x 32 boxes, 128-byte swizzle of 32-byte atoms).
 bool encode_f32_operand(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols,

@@ -38,12 +38,18 @@ EXPORTED = (
     "ispa_full_attention_workspace_size", "ispa_full_attention", "ispa_absorbed_weight",
     "ispa_project", "ispa_quantize_weight_int8", "ispa_project_w8a8_workspace_size",
     "ispa_project_w8a8", "ispa_attention_units", "ispa_attention_set_splits",
-    "ispa_set_wait_limit_ns",
+    "ispa_set_wait_limit_ns", "ispa_dual_attention_layers_workspace_size",
+    "ispa_dual_attention_layers",
 )
 
 
 class IspaKV(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("len", ctypes.c_int64)]
+
+
+class IspaKVLayers(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("len", ctypes.c_int64),
+                ("layer_stride", ctypes.c_int64)]
 
 
 class IspaError(RuntimeError):
@@ -76,6 +82,10 @@ def _load():
         "ispa_dual_attention": (I, [P, I64, I, I, IspaKV, IspaKV, IspaKV, F, P, P, P, P, P, P,
                                     P, SZ, P, P]),
         "ispa_local_attention": (I, [P, I64, I, I, IspaKV, IspaKV, F, P, P, P, P, SZ, P, P]),
+        "ispa_dual_attention_layers_workspace_size": (SZ, [I, I64, I64, I64, I64, I, I]),
+        "ispa_dual_attention_layers": (I, [I, P, I64, I64, I, I, IspaKVLayers, IspaKVLayers,
+                                           IspaKVLayers, F, P, P, P, I64, P, P, P, I64, P, SZ,
+                                           P, P]),
         "ispa_full_attention_workspace_size": (SZ, [I64, I64, I64, I64, I, I]),
         "ispa_full_attention": (I, [P, I64, I, I, IspaKV, IspaKV, IspaKV, F, P, P, P, SZ, P, P]),
         "ispa_absorbed_weight": (I, [P, P, I, P, P]),
@@ -199,6 +209,75 @@ def ispa_dual_attention(q, k_sink, v_sink, k_loc, v_loc, k_hist=None, v_hist=Non
         _ptr(a_full), _ptr(lse[0]), _ptr(lse[1]), _ptr(lse[2]), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream))
     _check(rc, "ispa_dual_attention")
+    return {"a_loc": a_loc, "d": d_out, "a_full": a_full, "lse_loc": lse[0], "lse_hist": lse[1],
+            "lse_full": lse[2], "status": status}
+
+
+def ispa_dual_attention_layers_workspace_size(n_layers, nq, sink_len, local_len, hist_len, heads,
+                                              head_dim) -> int:
+    return int(_load().ispa_dual_attention_layers_workspace_size(
+        n_layers, nq, sink_len, local_len, hist_len, heads, head_dim))
+
+
+def _kv_layers(k: Optional[torch.Tensor], v: Optional[torch.Tensor], L: int, heads: int, hd: int,
+               name: str):
+    """[L, len, heads, head_dim] keys and values (each layer contiguous, the
+    layers at a common stride) as an ispa_kv_layers."""
+    if k is None or k.shape[1] == 0:
+        return IspaKVLayers(None, None, 0, 0)
+    for t, what in ((k, "keys"), (v, "values")):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} {what}: expected a CUDA bf16 tensor")
+        if t.dim() != 4 or tuple(t.shape) != (L, k.shape[1], heads, hd) or not t[0].is_contiguous():
+            raise ValueError(f"{name} {what}: expected [{L}, len, {heads}, {hd}] with contiguous layers")
+    if k.stride(0) != v.stride(0):
+        raise ValueError(f"{name}: keys and values must share their layer stride")
+    return IspaKVLayers(k.data_ptr(), v.data_ptr(), k.shape[1], k.stride(0) if L > 1 else 0)
+
+
+def ispa_dual_attention_layers(q, k_sink, v_sink, k_loc, v_loc, k_hist=None, v_hist=None,
+                               scale=None, a_loc=None, d_out=None, a_full=None, lse=None,
+                               workspace=None, status=None, stream=None) -> dict:
+    """Dual-stream attention of the same chunk of L layers in one launch.
+    q: [L, nq, heads, head_dim]; k_*, v_*: [L, len, heads, head_dim] bf16
+    (each layer contiguous, any common layer stride). Outputs a_loc, d
+    ([L, nq, d] fp32), a_full ([L, nq, d] bf16) and, with ``lse`` a list of
+    three [L, heads, nq] fp32 tensors (or True to allocate them), the LSEs."""
+    if not isinstance(q, torch.Tensor) or q.dim() != 4 or not q[0].is_contiguous():
+        raise ValueError("q: expected [L, nq, heads, head_dim] with contiguous layers")
+    L, nq, heads, hd = q.shape
+    d = heads * hd
+    sink = _kv_layers(k_sink, v_sink, L, heads, hd, "sink")
+    loc = _kv_layers(k_loc, v_loc, L, heads, hd, "local")
+    hist = _kv_layers(k_hist, v_hist, L, heads, hd, "history")
+    dev = q.device
+    if scale is None:
+        scale = hd ** -0.5
+    f32 = dict(dtype=torch.float32, device=dev)
+    a_loc = torch.empty(L, nq, d, **f32) if a_loc is None else a_loc
+    d_out = torch.empty(L, nq, d, **f32) if d_out is None else d_out
+    a_full = torch.empty(L, nq, d, dtype=torch.bfloat16, device=dev) if a_full is None else a_full
+    for t in (a_loc, d_out, a_full):
+        if t.shape != (L, nq, d) or not t[0].is_contiguous() or t.stride(0) != a_loc.stride(0):
+            raise ValueError("outputs: expected [L, nq, d] with contiguous layers and one stride")
+    if lse is True:
+        lse = [torch.empty(L, heads, nq, **f32) for _ in range(3)]
+    lse = lse or [None, None, None]
+    lse_stride = next((t.stride(0) for t in lse if t is not None), 0)
+    for t in lse:
+        if t is not None and (t.shape != (L, heads, nq) or not t[0].is_contiguous()
+                              or t.stride(0) != lse_stride):
+            raise ValueError("lse: expected [L, heads, nq] with contiguous layers and one stride")
+    need = ispa_dual_attention_layers_workspace_size(L, nq, sink.len, loc.len, hist.len, heads, hd)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    status = new_status(dev) if status is None else status
+    rc = _load().ispa_dual_attention_layers(
+        L, _ptr(q), q.stride(0) if L > 1 else 0, nq, heads, hd, sink, loc, hist, float(scale),
+        _ptr(a_loc), _ptr(d_out), _ptr(a_full), a_loc.stride(0) if L > 1 else 0, _ptr(lse[0]),
+        _ptr(lse[1]), _ptr(lse[2]), lse_stride if L > 1 else 0, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream))
+    _check(rc, "ispa_dual_attention_layers")
     return {"a_loc": a_loc, "d": d_out, "a_full": a_full, "lse_loc": lse[0], "lse_hist": lse[1],
             "lse_full": lse[2], "status": status}
 

@@ -41,16 +41,37 @@ class _Slot:
         self.rows = 0
 
 
+class _GroupSlot:
+    """Attention outputs and workspace of one chunk of up to ``group`` layers
+    in flight ([group, rows, d] outputs, one launch over the layers)."""
+
+    def __init__(self, group, heads, head_dim, chunk_rows, max_sink, max_local, max_hist, device):
+        d = heads * head_dim
+        f32 = dict(dtype=torch.float32, device=device)
+        self.a_loc = torch.empty(group, chunk_rows, d, **f32)
+        self.d_out = torch.empty(group, chunk_rows, d, **f32)
+        self.a_full = torch.empty(group, chunk_rows, d, dtype=torch.bfloat16, device=device)
+        self.lse = [torch.empty(group, heads * chunk_rows, **f32) for _ in range(3)]
+        self.heads = heads
+        self.ws = torch.empty(ispa.ispa_dual_attention_layers_workspace_size(
+            group, chunk_rows, max_sink, max_local, max_hist, heads, head_dim), dtype=torch.uint8,
+            device=device)
+        self.rows = 0
+
+
 class LayerWarmup:
     """Buffers for ``n_layers`` layers of one geometry. The attention outputs
     are reused across chunks and layers; ``n_slots`` sets of them let that
     many layers run their chunks at once on separate streams (layers are
     independent until the transition), which fills the SMs the tail of one
-    layer's launches leaves idle."""
+    layer's launches leaves idle. With ``group`` > 1 there are also
+    ``n_slots`` sets of outputs for ``group`` layers each, for
+    ``layers_chunks_stacked``: the same chunk of ``group`` layers in one
+    attention launch, whose units fill whole waves of the SMs."""
 
     def __init__(self, heads: int, head_dim: int, chunk_rows: int, max_sink: int,
                  max_local: int, max_hist: int, n_layers: int = 1, device="cuda",
-                 n_slots: int = 1):
+                 n_slots: int = 1, group: int = 1):
         self.heads, self.head_dim = heads, head_dim
         self.d = d = heads * head_dim
         self.n_layers = n_layers
@@ -58,6 +79,10 @@ class LayerWarmup:
         f32 = dict(dtype=torch.float32, device=device)
         self.slots = [_Slot(heads, head_dim, chunk_rows, max_sink, max_local, max_hist, device)
                       for _ in range(max(1, n_slots))]
+        self.group = max(1, min(group, n_layers))
+        self.group_slots = [] if self.group == 1 else [
+            _GroupSlot(self.group, heads, head_dim, chunk_rows, max_sink, max_local, max_hist,
+                       device) for _ in range(max(1, n_slots))]
         s0 = self.slots[0]
         self.a_loc, self.d_out, self.a_full, self.lse = s0.a_loc, s0.d_out, s0.a_full, s0.lse
         self.M = torch.zeros(n_layers, 2 * d, 2 * d, **f32)
@@ -130,6 +155,68 @@ class LayerWarmup:
             join = torch.cuda.Event()
             join.record(s)
             streams[0].wait_event(join)
+
+    def attention_layers(self, sch: dict, l0: int, n: int, stream=None, slot: int = 0):
+        """Dual-stream attention of one chunk of layers l0 .. l0 + n - 1 in
+        one launch, into the group slot. ``sch``: the chunk's inputs as
+        [L, rows, heads, head_dim] tensors (``ispa_synth.stacked_chunk``)."""
+        gs = self.group_slots[slot]
+        if n > self.group:
+            raise ValueError(f"{n} layers exceed the group size {self.group}")
+        take = lambda key: None if sch.get(key) is None else sch[key][l0:l0 + n]
+        q = take("q")
+        gs.rows = nq = q.shape[1]
+        if nq > gs.a_loc.shape[1]:
+            raise ValueError(f"{nq} query rows exceed the slot's {gs.a_loc.shape[1]}")
+        ispa.ispa_dual_attention_layers(
+            q, take("k_sink"), take("v_sink"), take("k_loc"), take("v_loc"), take("k_hist"),
+            take("v_hist"), a_loc=gs.a_loc[:n, :nq], d_out=gs.d_out[:n, :nq],
+            a_full=gs.a_full[:n, :nq],
+            lse=[x[:n, :gs.heads * nq].view(n, gs.heads, nq) for x in gs.lse], workspace=gs.ws,
+            status=self.status, stream=stream)
+
+    def gram_group(self, first: bool, j: int, layer: int, stream=None, slot: int = 0):
+        """Fold layer j of the group slot's last chunk into the statistics of
+        ``layer`` (first chunk overwrites)."""
+        gs = self.group_slots[slot]
+        rc = ispa._load().ispa_gram_accumulate(
+            ispa._ptr(gs.a_loc[j]), ispa._ptr(gs.d_out[j]), gs.rows, self.d,
+            ispa._ptr(self.M[layer]), 0 if first else 1, 1, ispa._ptr(self.status),
+            ispa._stream(stream))
+        ispa._check(rc, "ispa_gram_accumulate")
+
+    def layer_groups(self):
+        """(first layer, layers) of each group, in order."""
+        return [(l0, min(self.group, self.n_layers - l0))
+                for l0 in range(0, self.n_layers, self.group)]
+
+    def layers_chunks_stacked(self, stacked_chunks, streams=None):
+        """Every chunk of every layer into the layers' statistics, ``group``
+        layers per attention launch: ``stacked_chunks[c]`` holds chunk c of
+        all layers (``ispa_synth.stacked_chunk``). Group g runs on
+        streams[g mod n_slots]; the others fork from and join back into the
+        first."""
+        if not self.group_slots:
+            raise ValueError("this runner was built with group = 1")
+        streams = streams or [None]
+        n = min(len(streams), len(self.group_slots))
+        if n > 1:
+            fork = torch.cuda.Event()
+            fork.record(streams[0])
+            for s in streams[1:n]:
+                s.wait_event(fork)
+        for g, (l0, cnt) in enumerate(self.layer_groups()):
+            slot = g % n
+            s = streams[slot]
+            for c, sch in enumerate(stacked_chunks):
+                self.attention_layers(sch, l0, cnt, stream=s, slot=slot)
+                for j in range(cnt):
+                    self.gram_group(c == 0, j, l0 + j, stream=s, slot=slot)
+        if n > 1:
+            for s in streams[1:n]:
+                join = torch.cuda.Event()
+                join.record(s)
+                streams[0].wait_event(join)
 
     def solve(self, W: torch.Tensor, lam: float = 0.0, layer: int = 0, stream=None):
         """Delta W (and B = R W, lambda) of one layer into its slot."""
@@ -209,19 +296,25 @@ def rank(err: torch.Tensor, K: int, perm: torch.Tensor, selected: torch.Tensor, 
 
 
 def run_warmup(chunks_per_layer, W_all: torch.Tensor, K: int, runner: LayerWarmup,
-               stream=None, streams=None):
+               stream=None, streams=None, stacked_chunks=None):
     """Whole warmup: ``chunks_per_layer[l]`` is layer l's list of chunk dicts
     (device tensors), ``W_all`` the [L, d, d] projections. Accumulates every
-    layer's statistics (layers spread over ``streams`` when given), solves and
-    scores all layers in two batched calls and ranks them. Returns (err
-    [L, 2] fp64, perm, selected); Delta W of layer l is ``runner.dW[l]``."""
-    n = len(chunks_per_layer)
+    layer's statistics (layers spread over ``streams`` when given; with
+    ``stacked_chunks``, chunk c of all layers as [L, ...] tensors, and a
+    runner built with group > 1, that many layers per attention launch),
+    solves and scores all layers in two batched calls and ranks them. Returns
+    (err [L, 2] fp64, perm, selected); Delta W of layer l is ``runner.dW[l]``."""
+    n = len(chunks_per_layer) if stacked_chunks is None else stacked_chunks[0]["q"].shape[0]
     if n != runner.n_layers:
         raise ValueError(f"runner holds {runner.n_layers} layers, got {n}")
     err = torch.empty(n, 2, dtype=torch.float64, device=runner.device)
     perm = torch.empty(n, dtype=torch.int32, device=runner.device)
     sel = torch.empty(n, dtype=torch.uint8, device=runner.device)
-    runner.layers_chunks(chunks_per_layer, streams if streams else ([stream] if stream else None))
+    sts = streams if streams else ([stream] if stream else None)
+    if stacked_chunks is not None:
+        runner.layers_chunks_stacked(stacked_chunks, sts)
+    else:
+        runner.layers_chunks(chunks_per_layer, sts)
     runner.absorb_all(W_all, err, stream=stream)
     rank(err, K, perm, sel, stream)
     return err, perm, sel

@@ -35,7 +35,7 @@ def exported():
 
 def test_exports_match_header(ispa):
     names = declared()
-    assert len(names) == 27
+    assert len(names) == 29
     assert names == exported()
     assert names == set(ispa.EXPORTED)
     lib = ctypes.CDLL(ispa.LIB_PATH)
@@ -145,6 +145,45 @@ def test_dual_attention_host_checks(ispa):
     # arguments that pass every host check then need an sm_100 device
     import torch
     rc = _dual(ispa)
+    if not torch.cuda.is_available():
+        assert rc in (ispa.ISPA_ERR_CUDA, ispa.ISPA_ERR_NO_DEVICE)
+
+
+def _dual_layers(ispa, L=3, q=0x1000, qs=64 * 128, nq=64, heads=2, hd=64, sink=16, loc=64,
+                 hist=256, kvs=None, outs=64 * 128, lses=2 * 64, a_loc=0x2000, d_out=0x3000,
+                 ws=0x100000, ws_bytes=1 << 30, status=0x4000):
+    lib = ispa._load()
+    d = heads * hd
+    kvs = kvs or {"sink": sink * d, "loc": loc * d, "hist": hist * d}
+    kv = lambda n, s: ispa.IspaKVLayers(0x10000, 0x20000, n, s) if n else \
+        ispa.IspaKVLayers(None, None, 0, 0)
+    return lib.ispa_dual_attention_layers(
+        L, q, qs, nq, heads, hd, kv(sink, kvs["sink"]), kv(loc, kvs["loc"]),
+        kv(hist, kvs["hist"]), 0.125, a_loc, d_out, None, outs, None, None, None, lses, ws,
+        ws_bytes, status, None)
+
+
+def test_dual_attention_layers_host_checks(ispa):
+    """The batched entry: layer counts and strides are checked before any
+    device work (layers may not overlap, rows stay 16-byte aligned), and the
+    workspace is one single-layer workspace per layer."""
+    one = ispa.ispa_dual_attention_workspace_size(4680, 1560, 4680, 14040, 12, 128)
+    assert ispa.ispa_dual_attention_layers_workspace_size(30, 4680, 1560, 4680, 14040, 12,
+                                                          128) == 30 * one
+    assert ispa.ispa_dual_attention_layers_workspace_size(0, 4680, 1560, 4680, 0, 12, 128) == 0
+    assert _dual_layers(ispa, L=0) == ispa.ISPA_ERR_ARG
+    assert _dual_layers(ispa, qs=64 * 128 - 8) == ispa.ISPA_ERR_ARG          # layers overlap
+    assert _dual_layers(ispa, outs=64 * 128 - 8) == ispa.ISPA_ERR_ARG
+    assert _dual_layers(ispa, lses=2 * 64 - 1) == ispa.ISPA_ERR_ARG
+    assert _dual_layers(ispa, kvs={"sink": 16 * 128, "loc": 64 * 128 - 8,
+                                   "hist": 256 * 128}) == ispa.ISPA_ERR_ARG
+    assert _dual_layers(ispa, qs=64 * 128 + 4) == ispa.ISPA_ERR_UNSUPPORTED  # 16-byte rows
+    assert _dual_layers(ispa, outs=64 * 128 + 4) == ispa.ISPA_ERR_UNSUPPORTED
+    assert _dual_layers(ispa, ws_bytes=1000) == ispa.ISPA_ERR_WORKSPACE
+    # one layer: strides are not used
+    assert _dual_layers(ispa, L=1, qs=0, outs=0, lses=0, ws_bytes=100) == ispa.ISPA_ERR_WORKSPACE
+    import torch
+    rc = _dual_layers(ispa)
     if not torch.cuda.is_available():
         assert rc in (ispa.ISPA_ERR_CUDA, ispa.ISPA_ERR_NO_DEVICE)
 

@@ -14,7 +14,8 @@ import pytest
 import torch
 
 import oracle
-from ispa_synth import C0, C1, attention_like, gaussian, layer_streams, scaled
+from ispa_synth import (C0, C1, attention_like, gaussian, layer_streams, scaled,
+                        stacked_chunk, stacked_layer_streams)
 
 pytestmark = pytest.mark.gpu
 
@@ -72,6 +73,46 @@ def random_chunk(nq, sink, loc, hist, H, hd, seed):
 
 
 # ---------------------------------------------------------------- attention
+
+def _stack_layers(chunks, key, pad_rows=0):
+    """[L, len + pad_rows, H, hd] bf16 on the device, layer l's rows first:
+    the layers at a stride wider than one layer's rows."""
+    t = torch.stack([ch[key] for ch in chunks]).cuda()
+    if pad_rows:
+        pad = torch.zeros(t.shape[0], pad_rows, *t.shape[2:], dtype=t.dtype, device=t.device)
+        t = torch.cat([t, pad], dim=1)
+    return t
+
+
+@pytest.mark.parametrize("hist", [0, 2000])
+def test_dual_attention_layers_equals_single_layer_calls(lib, hist):
+    """One launch over three layers (ragged query pairs; with a history the
+    plan has several key ranges, so the merge runs per layer) equals three
+    single-layer calls bit for bit; inputs and outputs at strides wider than
+    a layer."""
+    L, nq, H, hd = 3, 700, 4, 128
+    chunks = [random_chunk(nq, 300, 600, hist, H, hd, seed=40 + 7 * l) for l in range(L)]
+    st = lambda key, n: _stack_layers(chunks, key, pad_rows=n)[:, :chunks[0][key].shape[0]]
+    q = st("q", 8)
+    ks, vs, kl, vl = st("k_sink", 16), st("v_sink", 16), st("k_loc", 0), st("v_loc", 0)
+    kh, vh = (st("k_hist", 24), st("v_hist", 24)) if hist else (None, None)
+    d = H * hd
+    outs = [torch.empty(L, nq + 4, d, dtype=dt, device="cuda")[:, :nq]
+            for dt in (torch.float32, torch.float32, torch.bfloat16)]
+    lse = [torch.empty(L, H * nq + 16, device="cuda")[:, :H * nq].view(L, H, nq) for _ in range(3)]
+    got = lib.ispa_dual_attention_layers(q, ks, vs, kl, vl, kh, vh, a_loc=outs[0], d_out=outs[1],
+                                         a_full=outs[2], lse=lse)
+    torch.cuda.synchronize()
+    assert lib.read_status(got["status"]) == 0
+    for l in range(L):
+        one = run_dual(lib, to_dev(chunks[l]))
+        torch.cuda.synchronize()
+        for key in ("a_loc", "d", "a_full", "lse_loc", "lse_hist", "lse_full"):
+            assert torch.equal(got[key][l], one[key]), (l, key)
+    # and layer 1 against the oracle
+    check_attention({k: v[1] for k, v in got.items() if k != "status"}, ref_dual(chunks[1]),
+                    "layer 1 of 3")
+
 
 def test_dual_attention_tiny_workload_all_chunks(lib):
     st = layer_streams(C0, 0, seed=0)
@@ -463,6 +504,39 @@ def test_warmup_tiny_end_to_end(lib):
     assert rel_fro(Mg[:d, d:], ref["R"]) <= GR_RELFRO
     assert rel_fro(f64(runner.dW[0]), ref["dW"]) <= DW_RELFRO
     assert abs(err[0, 1].item() - ref["eps"]) <= 5e-3 * ref["eps"]
+
+
+def test_warmup_grouped_layers_equal_per_layer_path(lib):
+    """The warmup driver's grouped path (the same chunk of two layers per
+    attention launch, groups of 2, 2 and 1 layers on two streams) gives the
+    per-layer path's statistics and Delta W bit for bit, and its errors and
+    ranking."""
+    import dataclasses
+    from kv_cache_absorption_b200.warmup import LayerWarmup, run_warmup
+    cfg = dataclasses.replace(C0, layers=5)
+    sts, qkv = stacked_layer_streams(cfg, list(range(cfg.layers)), seed=3, device="cuda")
+    per_layer = [[st.chunk(c) for c in range(cfg.n_chunks)] for st in sts]
+    stacked = [stacked_chunk(cfg, qkv, c) for c in range(cfg.n_chunks)]
+    W_all = torch.stack([st.w for st in sts]).cuda()
+    max_hist = max(len(cfg.history_frames_of(c)) for c in range(cfg.n_chunks)) * cfg.tokens_per_frame
+    streams = [torch.cuda.current_stream(), torch.cuda.Stream()]
+    res = []
+    for group in (1, 2):
+        r = LayerWarmup(cfg.heads, cfg.head_dim, cfg.chunk_tokens, cfg.sink_tokens,
+                        cfg.chunk_tokens, max_hist, n_layers=cfg.layers, n_slots=2, group=group)
+        out = run_warmup(per_layer if group == 1 else None, W_all, 2, r, streams=streams,
+                         stacked_chunks=stacked if group > 1 else None)
+        torch.cuda.synchronize()
+        assert lib.read_status(r.status) == 0
+        res.append((r, out))
+    (r1, (e1, p1, s1)), (r2, (e2, p2, s2)) = res
+    assert r2.layer_groups() == [(0, 2), (2, 2), (4, 1)]
+    assert torch.equal(r1.M, r2.M)
+    assert torch.equal(r1.dW, r2.dW)
+    # epsilon's fp64 sums are added across CTAs by atomics: equal up to the
+    # order of those additions
+    assert torch.allclose(e1, e2, rtol=1e-12, atol=0.0)
+    assert torch.equal(p1, p2) and torch.equal(s1, s2)
 
 
 def test_warmup_multilayer_ranking(lib):

@@ -3,10 +3,10 @@
 spread over [0.5, 0.95]) and the 14B warmup (40 layers, d = 5120), four
 chunks of 4680 query rows each.
 
-The GPU runs its own chain through the warmup driver exactly as a caller
-would (dual attention of every chunk, Gram accumulation, one batched solve,
-one batched error pass, the ranking; two layers in flight) on the same
-seeded inputs the oracle saw. The oracle's results are stored in
+The GPU runs its own chain through the warmup driver exactly as the
+benchmark does (dual attention of each chunk for ten layers per launch, Gram
+accumulation, one batched solve, one batched error pass, the ranking; two
+groups of layers in flight) on the same seeded inputs the oracle saw. The oracle's results are stored in
 ``tests/golden/<workload>_warmup_oracle.npz`` (written by
 ``tests/golden/make_warmup_golden.py``, which calls only the oracle and the
 input generator). A d x d Delta W per layer is too large to store, so the
@@ -39,7 +39,7 @@ import pytest
 import torch
 
 import oracle
-from ispa_synth import CONFIGS, layer_streams, sketch_matrices
+from ispa_synth import CONFIGS, sketch_matrices, stacked_chunk, stacked_layer_streams
 
 pytestmark = pytest.mark.gpu
 
@@ -48,6 +48,7 @@ ATT_RELFRO, GR_RELFRO, DW_RELFRO = 5e-3, 1e-3, 2e-3
 EPS_REL = 5e-3          # end-to-end relative error of epsilon
 LAM_REL = 1e-3          # lambda = 1e-2 tr(G) / d inherits G's tolerance
 SEED = 0
+GROUP = 10              # layers per attention launch (the benchmark's default)
 
 
 def golden(name):
@@ -83,18 +84,21 @@ def run_warmup_on_gpu(cfg, dense_layers):
     from kv_cache_absorption_b200.warmup import LayerWarmup, run_warmup
     L, d, N = cfg.layers, cfg.d, cfg.warmup_rows
     max_hist = max(len(cfg.history_frames_of(c)) for c in range(cfg.n_chunks)) * cfg.tokens_per_frame
-    chunks, Ws = [], []
-    for l in range(L):
-        st = layer_streams(cfg, l, seed=SEED)
-        chunks.append([{k: v.cuda() for k, v in st.chunk(c).items()} for c in range(cfg.n_chunks)])
-        Ws.append(st.w)
-        del st
-    W_all = torch.stack(Ws).cuda()
+    # the oracle's inputs (drawn on the CPU), held on the GPU as one tensor
+    # per Q, K, V over all layers: per-layer chunks and stacked chunks view it
+    sts, qkv = stacked_layer_streams(cfg, list(range(L)), seed=SEED, device="cuda",
+                                     gen_device="cpu")
+    chunks = [[st.chunk(c) for c in range(cfg.n_chunks)] for st in sts]
+    stacked = [stacked_chunk(cfg, qkv, c) for c in range(cfg.n_chunks)]
+    W_all = torch.stack([st.w for st in sts])
     runner = LayerWarmup(cfg.heads, cfg.head_dim, cfg.chunk_tokens, cfg.sink_tokens,
-                         cfg.chunk_tokens, max_hist, n_layers=L, n_slots=2)
+                         cfg.chunk_tokens, max_hist, n_layers=L, n_slots=2, group=GROUP)
     runner.weight_gram(W_all)
     streams = [torch.cuda.current_stream(), torch.cuda.Stream()]
-    err, perm, sel = run_warmup(chunks, W_all, cfg.select_k, runner, streams=streams)
+    # as the benchmark runs it: GROUP layers per attention launch, two
+    # groups in flight
+    err, perm, sel = run_warmup(None, W_all, cfg.select_k, runner, streams=streams,
+                                stacked_chunks=stacked)
     torch.cuda.synchronize()
     out = {"status": int(runner.status.item()), "err": err.cpu().numpy(),
            "perm": perm.cpu().numpy(), "sel": sel.cpu().numpy().astype(bool),
