@@ -168,9 +168,12 @@ ISPA_API int ispa_dual_attention(const void* q, int64_t nq, int heads, int head_
  * lse_layer_stride after. With several layers the strides are at least one
  * layer's extent (nq * d, heads * nq), q_layer_stride and out_layer_stride
  * multiples of 8. workspace: >= ispa_dual_attention_layers_workspace_size()
- * bytes (n_layers single-layer workspaces, 256-byte aligned). Each layer's
- * results equal those of ispa_dual_attention on that layer alone, bit for
- * bit. Other arguments, status and errors as ispa_dual_attention.
+ * bytes (n_layers single-layer workspaces, 256-byte aligned). The key-range
+ * split (ispa_attention_units) is chosen for the whole launch: with many
+ * layers the units fill the waves without cutting the branches further.
+ * With the same split (ispa_attention_set_splits) each layer's results equal
+ * those of ispa_dual_attention on that layer alone, bit for bit. Other
+ * arguments, status and errors as ispa_dual_attention.
  */
 ISPA_API size_t ispa_dual_attention_layers_workspace_size(int n_layers, int64_t nq,
                                                           int64_t sink_len, int64_t local_len,

@@ -147,7 +147,7 @@ int attention_common(const void* q, int64_t nq, int heads, int head_dim, const i
                    ls.n, ls.kv[b], 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
       return ISPA_ERR_CUDA;
   }
-  p.plan = ispa::attention_plan(nq, br[0].len, br[1].len, br[2].len, heads);
+  p.plan = ispa::attention_plan(nq, br[0].len, br[1].len, br[2].len, heads, ls.n);
   ispa::attention_slot_order(p.plan,
                              ispa::attention_key_tiles(br[0].len) + ispa::attention_key_tiles(br[1].len),
                              ispa::attention_key_tiles(br[2].len), p.order);

@@ -914,10 +914,10 @@ double simulate(const AttnPlan& pl, int64_t loc_tiles, int64_t hist_tiles, int p
 
 struct PlanKey {
   int64_t pairs, loc_tiles, hist_tiles;
-  int heads, fls, fhs;
+  int heads, layers, fls, fhs;
   bool operator<(const PlanKey& o) const {
-    return std::tie(pairs, loc_tiles, hist_tiles, heads, fls, fhs) <
-           std::tie(o.pairs, o.loc_tiles, o.hist_tiles, o.heads, o.fls, o.fhs);
+    return std::tie(pairs, loc_tiles, hist_tiles, heads, layers, fls, fhs) <
+           std::tie(o.pairs, o.loc_tiles, o.hist_tiles, o.heads, o.layers, o.fls, o.fhs);
   }
 };
 
@@ -967,11 +967,13 @@ int attention_slot_bound(int64_t sink_len, int64_t local_len, int64_t hist_len) 
 }
 
 AttnPlan attention_plan(int64_t nq, int64_t sink_len, int64_t local_len, int64_t hist_len,
-                        int heads) {
+                        int heads, int layers) {
   const int64_t loc_tiles = attention_key_tiles(sink_len) + attention_key_tiles(local_len);
   const int64_t hist_tiles = attention_key_tiles(hist_len);
   const int pairs = attention_pairs(nq);
-  const PlanKey key{pairs, loc_tiles, hist_tiles, heads, g_force_ls.load(), g_force_hs.load()};
+  if (layers < 1) layers = 1;
+  const PlanKey key{pairs, loc_tiles, hist_tiles, heads, layers, g_force_ls.load(),
+                    g_force_hs.load()};
   static std::mutex mu;
   static std::map<PlanKey, AttnPlan> cache;
   {
@@ -980,7 +982,7 @@ AttnPlan attention_plan(int64_t nq, int64_t sink_len, int64_t local_len, int64_t
     if (it != cache.end()) return it->second;
   }
   const int hs0 = base_hist_ranges(loc_tiles, hist_tiles);
-  const int per = heads * pairs;
+  const int per = heads * pairs * layers;   // units per slot over the launch
   AttnPlan best{};
   double best_t = 0.0;
   bool have = false;

@@ -65,10 +65,10 @@ struct AttnParams {
   uint64_t wait_ns;       // limit of a pipeline wait (set at launch)
 };
 
-// The unit decomposition of a call with these branch lengths (see
-// attention.cu for the rule). Cached per shape.
+// The unit decomposition of a call with these branch lengths over `layers`
+// layers in one launch (see attention.cu for the rule). Cached per shape.
 AttnPlan attention_plan(int64_t nq, int64_t sink_len, int64_t local_len, int64_t hist_len,
-                        int heads);
+                        int heads, int layers = 1);
 // Most slots any plan for these branch lengths may use (the candidates'
 // maximum): non-decreasing in hist_len, so a workspace sized for the longest
 // history serves every shorter one with the same sink and local lengths.

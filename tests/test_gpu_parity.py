@@ -87,9 +87,10 @@ def _stack_layers(chunks, key, pad_rows=0):
 @pytest.mark.parametrize("hist", [0, 2000])
 def test_dual_attention_layers_equals_single_layer_calls(lib, hist):
     """One launch over three layers (ragged query pairs; with a history the
-    plan has several key ranges, so the merge runs per layer) equals three
-    single-layer calls bit for bit; inputs and outputs at strides wider than
-    a layer."""
+    key ranges are forced to a split with several ranges, so the merge runs
+    per layer) equals three single-layer calls with the same split bit for
+    bit; inputs and outputs at strides wider than a layer. Without forcing,
+    the launch's own split matches the oracle."""
     L, nq, H, hd = 3, 700, 4, 128
     chunks = [random_chunk(nq, 300, 600, hist, H, hd, seed=40 + 7 * l) for l in range(L)]
     st = lambda key, n: _stack_layers(chunks, key, pad_rows=n)[:, :chunks[0][key].shape[0]]
@@ -100,18 +101,26 @@ def test_dual_attention_layers_equals_single_layer_calls(lib, hist):
     outs = [torch.empty(L, nq + 4, d, dtype=dt, device="cuda")[:, :nq]
             for dt in (torch.float32, torch.float32, torch.bfloat16)]
     lse = [torch.empty(L, H * nq + 16, device="cuda")[:, :H * nq].view(L, H, nq) for _ in range(3)]
-    got = lib.ispa_dual_attention_layers(q, ks, vs, kl, vl, kh, vh, a_loc=outs[0], d_out=outs[1],
-                                         a_full=outs[2], lse=lse)
+    lib.ispa_attention_set_splits(2, 2 if hist else 0)
+    try:
+        got = lib.ispa_dual_attention_layers(q, ks, vs, kl, vl, kh, vh, a_loc=outs[0],
+                                             d_out=outs[1], a_full=outs[2], lse=lse)
+        torch.cuda.synchronize()
+        assert lib.read_status(got["status"]) == 0
+        for l in range(L):
+            one = run_dual(lib, to_dev(chunks[l]))
+            torch.cuda.synchronize()
+            for key in ("a_loc", "d", "a_full", "lse_loc", "lse_hist", "lse_full"):
+                assert torch.equal(got[key][l], one[key]), (l, key)
+    finally:
+        lib.ispa_attention_set_splits(0, 0)
+    # the launch's own split, every layer against the oracle
+    got = lib.ispa_dual_attention_layers(q, ks, vs, kl, vl, kh, vh, lse=True)
     torch.cuda.synchronize()
     assert lib.read_status(got["status"]) == 0
     for l in range(L):
-        one = run_dual(lib, to_dev(chunks[l]))
-        torch.cuda.synchronize()
-        for key in ("a_loc", "d", "a_full", "lse_loc", "lse_hist", "lse_full"):
-            assert torch.equal(got[key][l], one[key]), (l, key)
-    # and layer 1 against the oracle
-    check_attention({k: v[1] for k, v in got.items() if k != "status"}, ref_dual(chunks[1]),
-                    "layer 1 of 3")
+        check_attention({k: v[l] for k, v in got.items() if k != "status"}, ref_dual(chunks[l]),
+                        f"layer {l} of {L}")
 
 
 def test_dual_attention_tiny_workload_all_chunks(lib):
@@ -509,8 +518,9 @@ def test_warmup_tiny_end_to_end(lib):
 def test_warmup_grouped_layers_equal_per_layer_path(lib):
     """The warmup driver's grouped path (the same chunk of two layers per
     attention launch, groups of 2, 2 and 1 layers on two streams) gives the
-    per-layer path's statistics and Delta W bit for bit, and its errors and
-    ranking."""
+    per-layer path's statistics, Delta W, errors and ranking. With the
+    per-layer key-range split forced on both, M and Delta W agree bit for
+    bit; with each launch's own split, to the fp32 rounding of the merge."""
     import dataclasses
     from kv_cache_absorption_b200.warmup import LayerWarmup, run_warmup
     cfg = dataclasses.replace(C0, layers=5)
@@ -520,22 +530,34 @@ def test_warmup_grouped_layers_equal_per_layer_path(lib):
     W_all = torch.stack([st.w for st in sts]).cuda()
     max_hist = max(len(cfg.history_frames_of(c)) for c in range(cfg.n_chunks)) * cfg.tokens_per_frame
     streams = [torch.cuda.current_stream(), torch.cuda.Stream()]
-    res = []
-    for group in (1, 2):
+
+    def run(group):
         r = LayerWarmup(cfg.heads, cfg.head_dim, cfg.chunk_tokens, cfg.sink_tokens,
                         cfg.chunk_tokens, max_hist, n_layers=cfg.layers, n_slots=2, group=group)
         out = run_warmup(per_layer if group == 1 else None, W_all, 2, r, streams=streams,
                          stacked_chunks=stacked if group > 1 else None)
         torch.cuda.synchronize()
         assert lib.read_status(r.status) == 0
-        res.append((r, out))
-    (r1, (e1, p1, s1)), (r2, (e2, p2, s2)) = res
+        return r, out
+
+    rel = lambda a, b: float((a - b).norm() / b.norm())
+    # the per-layer split forced on both paths: bit for bit (epsilon's fp64
+    # sums are added across CTAs by atomics: equal up to their order)
+    lib.ispa_attention_set_splits(1, 1)
+    try:
+        (r1, (e1, p1, s1)), (r2, (e2, p2, s2)) = run(1), run(2)
+    finally:
+        lib.ispa_attention_set_splits(0, 0)
     assert r2.layer_groups() == [(0, 2), (2, 2), (4, 1)]
     assert torch.equal(r1.M, r2.M)
     assert torch.equal(r1.dW, r2.dW)
-    # epsilon's fp64 sums are added across CTAs by atomics: equal up to the
-    # order of those additions
     assert torch.allclose(e1, e2, rtol=1e-12, atol=0.0)
+    assert torch.equal(p1, p2) and torch.equal(s1, s2)
+    # each launch's own split
+    (r1, (e1, p1, s1)), (r2, (e2, p2, s2)) = run(1), run(2)
+    assert rel(r2.M, r1.M) <= 1e-6
+    assert rel(r2.dW, r1.dW) <= 1e-4
+    assert torch.allclose(e1, e2, rtol=1e-5, atol=0.0)
     assert torch.equal(p1, p2) and torch.equal(s1, s2)
 
 
