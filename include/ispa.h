@@ -151,8 +151,13 @@ ISPA_API int64_t ispa_attention_units(int64_t nq, int64_t sink_len, int64_t loca
                                       int64_t hist_len, int heads, int* local_splits,
                                       int* hist_splits);
 /* Forces the split counts of later attention calls (0 = automatic, the
- * default), for measurement. Applies process-wide; query workspace sizes
- * after changing it. Returns ISPA_OK, or ISPA_ERR_ARG for a negative count. */
+ * default), for measurement. hist_splits = -1 asks for joint units where a
+ * call has a history and returns A_loc: one unit per head and query-tile pair
+ * runs the local keys, stores A_loc, then runs the history and merges in its
+ * epilogue (the automatic choice may pick it for calls over several layers).
+ * Applies process-wide; query workspace sizes after changing it. Returns
+ * ISPA_OK, or ISPA_ERR_ARG for a negative local count or a history count
+ * below -1. */
 ISPA_API int ispa_attention_set_splits(int local_splits, int hist_splits);
 ISPA_API int ispa_dual_attention(const void* q, int64_t nq, int heads, int head_dim, ispa_kv sink,
                         ispa_kv local, ispa_kv hist, float scale, float* a_loc, float* d_out,

@@ -147,7 +147,7 @@ int attention_common(const void* q, int64_t nq, int heads, int head_dim, const i
                    ls.n, ls.kv[b], 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
       return ISPA_ERR_CUDA;
   }
-  p.plan = ispa::attention_plan(nq, br[0].len, br[1].len, br[2].len, heads, ls.n);
+  p.plan = ispa::attention_plan(nq, br[0].len, br[1].len, br[2].len, heads, ls.n, !local_in_ws);
   ispa::attention_slot_order(p.plan,
                              ispa::attention_key_tiles(br[0].len) + ispa::attention_key_tiles(br[1].len),
                              ispa::attention_key_tiles(br[2].len), p.order);
@@ -224,7 +224,7 @@ int64_t ispa_attention_units(int64_t nq, int64_t sink_len, int64_t local_len, in
 }
 
 int ispa_attention_set_splits(int local_splits, int hist_splits) {
-  if (local_splits < 0 || hist_splits < 0) return ISPA_ERR_ARG;
+  if (local_splits < 0 || hist_splits < -1) return ISPA_ERR_ARG;
   ispa::attention_force_splits(local_splits, hist_splits);
   return ISPA_OK;
 }

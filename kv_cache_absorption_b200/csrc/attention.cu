@@ -99,10 +99,13 @@ struct Unit {
   int hist;        // 1 = history branch, 0 = local branch (sink then local)
   int t0;          // first key tile of the range within its branch
   int n_tiles;
+  int joint;       // 1: local tiles, then history tiles (a joint plan)
+  int n_loc;       // joint: local tiles before the history starts
 };
 
 // Grid order: for each slot in p.order (longest key range first), every
 // (layer, head, query pair).
+template <bool JOINT>
 __device__ __forceinline__ Unit unit_of(const AttnParams& p) {
   Unit u;
   const int per = p.heads * p.n_pairs;
@@ -128,6 +131,14 @@ __device__ __forceinline__ Unit unit_of(const AttnParams& p) {
   }
   u.t0 = k * per_range;
   u.n_tiles = total - u.t0 < per_range ? total - u.t0 : per_range;
+  u.joint = JOINT ? 1 : 0;
+  u.n_loc = 0;
+  if constexpr (JOINT) {   // the whole local branch, then the whole history
+    u.hist = 0;
+    u.t0 = 0;
+    u.n_loc = (int)((p.len[0] + BN - 1) / BN) + (int)((p.len[1] + BN - 1) / BN);
+    u.n_tiles = u.n_loc + (int)((p.len[2] + BN - 1) / BN);
+  }
   return u;
 }
 
@@ -150,6 +161,13 @@ __device__ __forceinline__ TileInfo tile_of(int j, bool hist, const AttnParams& 
   const int64_t rem = p.len[t.branch] - t.row0;
   t.valid = rem < BN ? (int)rem : BN;
   return t;
+}
+
+// Key tile j of unit u (a joint unit crosses into the history at n_loc).
+template <bool JOINT>
+__device__ __forceinline__ TileInfo tile_of_unit(const Unit& u, int j, const AttnParams& p) {
+  if (JOINT && j >= u.n_loc) return tile_of(j - u.n_loc, true, p);
+  return tile_of(u.t0 + j, u.hist, p);
 }
 
 // Bounded wait used while unwinding: ignores the abort flag.
@@ -482,7 +500,9 @@ __device__ __forceinline__ void merge_rows(const AttnParams& p, const LayerIO& i
   }
 }
 
-template <int HD>
+// JOINT: the plan's joint units (a separate instantiation, so that the other
+// plans' kernel keeps its register allocation).
+template <int HD, bool JOINT>
 __global__ void __launch_bounds__(kThreads, 1)
 branch_attention_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -490,7 +510,7 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const Unit u = unit_of(p);
+  const Unit u = unit_of<JOINT>(p);
   const LayerIO io = layer_io(p, u.layer);
   const int n_tiles = u.n_tiles;
   volatile int* abort_flag = &s.abort_flag;
@@ -533,7 +553,7 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
           tma_load_3d(s.q[t][b], &p.tm_q, &s.q_full, u.head * HD + b * 64, u.q0 + t * BM, u.layer);
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
-        const TileInfo ti = tile_of(u.t0 + j, u.hist, p);
+        const TileInfo ti = tile_of_unit<JOINT>(u, j, p);
         const int sk = j % NK, sv = j % NV;
         if (j >= NK && !mbar_wait(&s.k_empty[sk], ((j / NK) - 1) & 1, p.status, abort_flag, p.wait_ns)) break;
         mbar_expect_tx(&s.k_full[sk], (HD / 64) * BN * 128);
@@ -606,7 +626,7 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
 #pragma unroll
               for (int kk = h * 4; kk < h * 4 + 4; ++kk)
                 mma_ts(oo, ao + kk * 8, bv + (uint64_t)((kk * 2048) >> 4), idesc_pv,
-                       (j == 1 && kk == 0) ? 0u : 1u);
+                       ((j == 1 || (JOINT && j == u.n_loc + 1)) && kk == 0) ? 0u : 1u);
             }
             if (!ok) break;
             if (t == u.n_qt - 1) tc_commit(&s.v_empty[sv]);
@@ -647,11 +667,44 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
     const uint32_t ts = t_s(t) + lane_off, to = t_o(t) + lane_off;
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;                 // running max (log2 units), sum
+    float lse_loc_joint = -INFINITY;              // joint unit: the local branch's LSE
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      const TileInfo ti = tile_of(u.t0 + j, u.hist, p);
+      const TileInfo ti = tile_of_unit<JOINT>(u, j, p);
       if (!mbar_wait_warp(&s.s_full[t], j & 1, p.status, abort_flag, p.wait_ns)) { ok = false; break; }
       tc_fence_after();
+      const bool fresh = j == 0 || (JOINT && j == u.n_loc);
+      if (JOINT && j == u.n_loc) {
+        // the local branch is complete (PV_t(j-1) preceded S_t(j)): A_loc and
+        // LSE_loc from O_t; the history starts from a fresh state, and its
+        // first PV overwrites O_t
+        const float inv = 1.f / l;
+        lse_loc_joint = (m + log2f(l)) * kLn2;
+        const int row = u.q0 + t * BM + r;
+        const bool row_ok = row < p.nq;
+        float* dst = io.a_loc + (int64_t)row * p.heads * HD + (int64_t)u.head * HD;
+        const bool rnd = p.round_tf32 != 0;
+#pragma unroll 1
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t raw[32];
+          tmem_ld32(to + c * 32, raw);
+          tmem_ld_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float4 x = make_float4(__uint_as_float(raw[4 * i]) * inv,
+                                     __uint_as_float(raw[4 * i + 1]) * inv,
+                                     __uint_as_float(raw[4 * i + 2]) * inv,
+                                     __uint_as_float(raw[4 * i + 3]) * inv);
+              if (rnd) x = make_float4(to_tf32(x.x), to_tf32(x.y), to_tf32(x.z), to_tf32(x.w));
+              reinterpret_cast<float4*>(dst + c * 32)[i] = x;
+            }
+          }
+        }
+        if (row_ok && io.lse_loc) io.lse_loc[(int64_t)u.head * p.nq + row] = lse_loc_joint;
+        m = -INFINITY;
+        l = 0.f;
+      }
       float sv[BN];
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
@@ -676,7 +729,7 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
       const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
                              fmaxf(mx8[6], mx8[7]));
       const float m_new = fmaxf(m, mx * sl2);
-      if (j == 0) {
+      if (fresh) {
         m = m_new;
       } else {
         const bool need = m_new > m + kRescaleThreshold;
@@ -736,7 +789,48 @@ branch_attention_kernel(const __grid_constant__ AttnParams p) {
       float* wst = reinterpret_cast<float*>(&s.q[0][0][0]) + (warp - 4) * 32 * 36;
       const int wrow0 = u.q0 + t * BM + quarter * 32;       // first row of this warp
       const int64_t wbase = (int64_t)wrow0 * d + (int64_t)u.head * HD;
-      if (n_slots == 1) {
+      if constexpr (JOINT) {
+        // joint unit: O_t holds the history branch; with the A_loc stored
+        // where the history started (re-read as stored), the merge of a
+        // local and a history range: w = e^(LSE_hist - LSE_full),
+        // D = w (A_hist - A_loc), A_full = A_loc + D
+        const float lse_full = log_add_exp(lse_loc_joint, lse);
+        const float w = expf(lse - lse_full);
+        const bool rnd = p.round_tf32 != 0;
+        const float* src = io.a_loc + base;
+#pragma unroll 1
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t raw[32];
+          tmem_ld32(to + c * 32, raw);
+          tmem_ld_wait();
+          float al[32], dv[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 x = row_ok ? reinterpret_cast<const float4*>(src + c * 32)[i]
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            al[4 * i] = x.x;
+            al[4 * i + 1] = x.y;
+            al[4 * i + 2] = x.z;
+            al[4 * i + 3] = x.w;
+          }
+#pragma unroll
+          // A_hist rounded as a stored range output is (no contraction into
+          // the difference), then the merge's arithmetic
+          for (int i = 0; i < 32; ++i)
+            dv[i] = fmaf(w, __fmul_rn(__uint_as_float(raw[i]), inv) - al[i], 0.f);
+          rows_out(wst, dv, wrow0, p.nq, d, io.d_out ? io.d_out + wbase + c * 32 : nullptr, rnd,
+                   nullptr, nullptr);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) dv[i] = al[i] + dv[i];
+          rows_out(wst, dv, wrow0, p.nq, d, nullptr, false,
+                   io.a_full ? io.a_full + wbase + c * 32 : nullptr, nullptr);
+        }
+        if (row_ok) {
+          if (io.lse_hist) io.lse_hist[li] = lse;
+          if (io.lse_full) io.lse_full[li] = lse_full;
+        }
+        nonfinite = row_ok && !finite_f(lse_full);
+      } else if (n_slots == 1) {
         // one local range and no history: write the final outputs directly
 #pragma unroll 1
         for (int c = 0; c < HD / 32; ++c) {
@@ -869,6 +963,9 @@ namespace {
 // prologue, epilogue, slot write and merge); it picks the fastest measured
 // plan of every shape to within 1%.
 constexpr double kUnitCost = 10.0;   // key-tile steps
+// A joint unit's extra cost: A_loc stored where the history starts, and its
+// epilogue reads it back.
+constexpr double kJointCost = 2.0;
 constexpr int kPlanSms = 148;
 
 std::atomic<int> g_force_ls{0}, g_force_hs{0};
@@ -882,6 +979,10 @@ int ranges_of(int64_t tiles, int n, int* per) {
 }
 
 void slot_lengths(const AttnPlan& pl, int64_t loc_tiles, int64_t hist_tiles, int* len) {
+  if (pl.joint) {
+    len[0] = (int)(loc_tiles + hist_tiles);
+    return;
+  }
   for (int k = 0; k < pl.n_ls; ++k) {
     const int64_t rem = loc_tiles - (int64_t)k * pl.ls_tiles;
     len[k] = (int)(rem < pl.ls_tiles ? rem : pl.ls_tiles);
@@ -901,7 +1002,7 @@ double simulate(const AttnPlan& pl, int64_t loc_tiles, int64_t hist_tiles, int p
   for (int i = 0; i < kPlanSms; ++i) free_at.push(0.0);
   double end = 0.0;
   for (int o = 0; o < pl.n_slots(); ++o) {
-    const double cost = len[order[o]] + kUnitCost;
+    const double cost = len[order[o]] + kUnitCost + (pl.joint ? kJointCost : 0.0);
     for (int b = 0; b < per; ++b) {
       const double t = free_at.top() + cost;
       free_at.pop();
@@ -914,10 +1015,11 @@ double simulate(const AttnPlan& pl, int64_t loc_tiles, int64_t hist_tiles, int p
 
 struct PlanKey {
   int64_t pairs, loc_tiles, hist_tiles;
-  int heads, layers, fls, fhs;
+  int heads, layers, joint_ok, fls, fhs;
   bool operator<(const PlanKey& o) const {
-    return std::tie(pairs, loc_tiles, hist_tiles, heads, layers, fls, fhs) <
-           std::tie(o.pairs, o.loc_tiles, o.hist_tiles, o.heads, o.layers, o.fls, o.fhs);
+    return std::tie(pairs, loc_tiles, hist_tiles, heads, layers, joint_ok, fls, fhs) <
+           std::tie(o.pairs, o.loc_tiles, o.hist_tiles, o.heads, o.layers, o.joint_ok, o.fls,
+                    o.fhs);
   }
 };
 
@@ -925,7 +1027,7 @@ struct PlanKey {
 
 void attention_force_splits(int local_splits, int hist_splits) {
   g_force_ls.store(local_splits < 0 ? 0 : local_splits);
-  g_force_hs.store(hist_splits < 0 ? 0 : hist_splits);
+  g_force_hs.store(hist_splits < -1 ? 0 : hist_splits);
 }
 
 void attention_slot_order(const AttnPlan& pl, int64_t loc_tiles, int64_t hist_tiles,
@@ -953,7 +1055,7 @@ constexpr int kExtraHistRanges = 2;
 int attention_slot_bound(int64_t sink_len, int64_t local_len, int64_t hist_len) {
   const int64_t loc_tiles = attention_key_tiles(sink_len) + attention_key_tiles(local_len);
   const int64_t hist_tiles = attention_key_tiles(hist_len);
-  const int fls = g_force_ls.load(), fhs = g_force_hs.load();
+  const int fls = g_force_ls.load(), fhs = g_force_hs.load() > 0 ? g_force_hs.load() : 0;
   int64_t ls = fls > kMaxLocalRanges ? fls : kMaxLocalRanges;
   if (ls > loc_tiles) ls = loc_tiles;
   int64_t hs = 0;
@@ -967,13 +1069,14 @@ int attention_slot_bound(int64_t sink_len, int64_t local_len, int64_t hist_len) 
 }
 
 AttnPlan attention_plan(int64_t nq, int64_t sink_len, int64_t local_len, int64_t hist_len,
-                        int heads, int layers) {
+                        int heads, int layers, bool allow_joint) {
   const int64_t loc_tiles = attention_key_tiles(sink_len) + attention_key_tiles(local_len);
   const int64_t hist_tiles = attention_key_tiles(hist_len);
   const int pairs = attention_pairs(nq);
   if (layers < 1) layers = 1;
-  const PlanKey key{pairs, loc_tiles, hist_tiles, heads, layers, g_force_ls.load(),
-                    g_force_hs.load()};
+  const bool joint_ok = allow_joint && hist_tiles > 0;
+  const PlanKey key{pairs, loc_tiles, hist_tiles, heads, layers, joint_ok ? 1 : 0,
+                    g_force_ls.load(), g_force_hs.load()};
   static std::mutex mu;
   static std::map<PlanKey, AttnPlan> cache;
   {
@@ -986,10 +1089,23 @@ AttnPlan attention_plan(int64_t nq, int64_t sink_len, int64_t local_len, int64_t
   AttnPlan best{};
   double best_t = 0.0;
   bool have = false;
+  // a joint unit per (head, pair): forced (hist_splits -1), or a candidate when
+  // the launch spans several layers (enough units to fill the waves without
+  // cutting the branches)
+  if (joint_ok && (key.fhs == -1 || (key.fhs == 0 && key.fls == 0 && layers > 1))) {
+    AttnPlan pl{};
+    pl.joint = 1;
+    pl.n_ls = ranges_of(loc_tiles, 1, &pl.ls_tiles);
+    pl.n_hs = ranges_of(hist_tiles, 1, &pl.hs_tiles);
+    best = pl;
+    best_t = simulate(pl, loc_tiles, hist_tiles, per);
+    have = true;
+  }
+  const int fhs = key.fhs > 0 ? key.fhs : 0;
   const int ls_lo = key.fls ? key.fls : 1, ls_hi = key.fls ? key.fls : kMaxLocalRanges;
-  const int hs_lo = hist_tiles == 0 ? 0 : (key.fhs ? key.fhs : hs0);
-  const int hs_hi = hist_tiles == 0 ? 0 : (key.fhs ? key.fhs : hs0 + kExtraHistRanges);
-  for (int hs = hs_lo; hs <= hs_hi; ++hs) {
+  const int hs_lo = hist_tiles == 0 ? 0 : (fhs ? fhs : (key.fhs == -1 ? 1 : hs0));
+  const int hs_hi = hist_tiles == 0 ? 0 : (fhs ? fhs : (key.fhs == -1 ? 1 : hs0 + kExtraHistRanges));
+  for (int hs = hs_lo; hs <= hs_hi && !(have && best.joint && key.fhs == -1); ++hs) {
     for (int ls = ls_lo; ls <= ls_hi; ++ls) {
       AttnPlan pl{};
       pl.n_ls = ranges_of(loc_tiles, ls, &pl.ls_tiles);
@@ -1024,15 +1140,12 @@ cudaError_t launch_dual_attention(const AttnParams& p0, int head_dim, cudaStream
                                             (size_t)p.n_layers, stream);
     if (e != cudaSuccess) return e;
   }
-  if (head_dim == 64) {
-    cudaFuncSetAttribute(branch_attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    branch_attention_kernel<64><<<units, kThreads, smem, stream>>>(p);
-  } else {
-    cudaFuncSetAttribute(branch_attention_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    branch_attention_kernel<128><<<units, kThreads, smem, stream>>>(p);
-  }
+  auto kernel = head_dim == 64 ? (p.plan.joint ? branch_attention_kernel<64, true>
+                                                : branch_attention_kernel<64, false>)
+                                : (p.plan.joint ? branch_attention_kernel<128, true>
+                                                : branch_attention_kernel<128, false>);
+  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  kernel<<<units, kThreads, smem, stream>>>(p);
   count_launches();
   return cudaGetLastError();
 }

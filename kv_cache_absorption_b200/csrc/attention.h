@@ -19,10 +19,14 @@ constexpr int kMaxSlots = 72;
 // (sink tiles, then the current chunk's) is cut into n_ls ranges of ls_tiles
 // 128-key tiles, the history into n_hs ranges of hs_tiles (n_hs = 0 without
 // a history). Slot k < n_ls is local range k, slot n_ls + k history range k.
+// A joint plan (n_ls = n_hs = 1) runs both branches in one unit per (head,
+// pair): the local keys, then the history from a fresh softmax state; the
+// unit stores A_loc where the history starts and merges in its epilogue.
 struct AttnPlan {
   int n_ls, ls_tiles;
   int n_hs, hs_tiles;
-  __host__ __device__ int n_slots() const { return n_ls + n_hs; }
+  int joint;
+  __host__ __device__ int n_slots() const { return joint ? 1 : n_ls + n_hs; }
 };
 
 // Parameters of one dual-stream attention launch over n_layers layers of the
@@ -67,13 +71,15 @@ struct AttnParams {
 
 // The unit decomposition of a call with these branch lengths over `layers`
 // layers in one launch (see attention.cu for the rule). Cached per shape.
+// allow_joint: the call stores A_loc, which a joint unit needs.
 AttnPlan attention_plan(int64_t nq, int64_t sink_len, int64_t local_len, int64_t hist_len,
-                        int heads, int layers = 1);
+                        int heads, int layers = 1, bool allow_joint = false);
 // Most slots any plan for these branch lengths may use (the candidates'
 // maximum): non-decreasing in hist_len, so a workspace sized for the longest
 // history serves every shorter one with the same sink and local lengths.
 int attention_slot_bound(int64_t sink_len, int64_t local_len, int64_t hist_len);
-// Forces the split counts of later plans (0 = automatic). For measurement.
+// Forces the split counts of later plans (0 = automatic; hist_splits = -1:
+// the joint unit where the call allows it). For measurement and tests.
 void attention_force_splits(int local_splits, int hist_splits);
 // Longest-first order of the plan's slots (grid order of the units).
 void attention_slot_order(const AttnPlan& plan, int64_t loc_tiles, int64_t hist_tiles,

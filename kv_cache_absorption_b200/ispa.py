@@ -328,7 +328,9 @@ def ispa_set_wait_limit_ns(ns: int = 0) -> None:
 
 
 def ispa_attention_set_splits(local_splits: int = 0, hist_splits: int = 0) -> None:
-    """Force the key-range split counts of later attention calls (0 = automatic)."""
+    """Force the key-range split counts of later attention calls (0 = automatic;
+    hist_splits = -1: joint units, one per head and query pair, where a call
+    has a history and returns A_loc)."""
     _check(_load().ispa_attention_set_splits(int(local_splits), int(hist_splits)),
            "ispa_attention_set_splits")
 

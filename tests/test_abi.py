@@ -109,10 +109,16 @@ def test_attention_plan(ispa):
         assert ispa.ispa_attention_units(nq, 1560, 4680, 0, H) == (per * 2, 2, 0)
         # more ranges than tiles: one range per tile
         assert ispa.ispa_attention_units(64, 16, 64, 128, 2)[1:] == (2, 1)
+        # joint units (hist_splits -1) need A_loc as an output, which this
+        # plan query does not assume: one history range then
+        ispa.ispa_attention_set_splits(1, -1)
+        assert ispa.ispa_attention_units(nq, 1560, 4680, 14040, H) == (per * 2, 1, 1)
     finally:
         ispa.ispa_attention_set_splits(0, 0)
     with pytest.raises(ispa.IspaError):
         ispa.ispa_attention_set_splits(-1, 0)
+    with pytest.raises(ispa.IspaError):
+        ispa.ispa_attention_set_splits(1, -2)
 
 
 def _kv(ispa, n, addr=0x10000):

@@ -84,6 +84,35 @@ def _stack_layers(chunks, key, pad_rows=0):
     return t
 
 
+def test_joint_units_equal_the_two_range_plan(lib):
+    """A joint unit per (head, query pair) (the local keys, A_loc stored where
+    the history starts, then the history from a fresh state, merged in the
+    epilogue) gives the same bits as the plan with one local and one history
+    range merged by the later unit: single-layer and over three layers, with
+    ragged query pairs and a partial last tile in every branch."""
+    L, nq, H, hd = 3, 700, 4, 128
+    chunks = [random_chunk(nq, 300, 600, 2000, H, hd, seed=60 + 5 * l) for l in range(L)]
+    keys = ("a_loc", "d", "a_full", "lse_loc", "lse_hist", "lse_full")
+    q = _stack_layers(chunks, "q")
+    kv = [_stack_layers(chunks, k) for k in ("k_sink", "v_sink", "k_loc", "v_loc", "k_hist",
+                                            "v_hist")]
+    outs = {}
+    try:
+        for tag, hs in (("two", 1), ("joint", -1)):
+            lib.ispa_attention_set_splits(1, hs)
+            outs[tag + "1"] = [run_dual(lib, to_dev(ch)) for ch in chunks]
+            outs[tag + "L"] = lib.ispa_dual_attention_layers(q, *kv, lse=True)
+            torch.cuda.synchronize()
+    finally:
+        lib.ispa_attention_set_splits(0, 0)
+    for l in range(L):
+        for key in keys:
+            assert torch.equal(outs["joint1"][l][key], outs["two1"][l][key]), (l, key)
+            assert torch.equal(outs["jointL"][key][l], outs["two1"][l][key]), (l, key)
+    assert lib.read_status(outs["jointL"]["status"]) == 0
+    check_attention(outs["joint1"][0], ref_dual(chunks[0]), "joint unit")
+
+
 @pytest.mark.parametrize("hist", [0, 2000])
 def test_dual_attention_layers_equals_single_layer_calls(lib, hist):
     """One launch over three layers (ragged query pairs; with a history the
