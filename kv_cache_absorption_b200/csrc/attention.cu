@@ -208,42 +208,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
-// 16 consecutive fp32 values: stores (optionally rounded to tf32), loads
-// that bypass L1 (slots written by other SMs in this launch).
-__device__ __forceinline__ void store_f32x16(float* dst, const float (&v)[16], bool tf32) {
-  float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float4 x;
-    x.x = tf32 ? to_tf32(v[4 * i]) : v[4 * i];
-    x.y = tf32 ? to_tf32(v[4 * i + 1]) : v[4 * i + 1];
-    x.z = tf32 ? to_tf32(v[4 * i + 2]) : v[4 * i + 2];
-    x.w = tf32 ? to_tf32(v[4 * i + 3]) : v[4 * i + 3];
-    d4[i] = x;
-  }
-}
-__device__ __forceinline__ void load_f32x16(const float* src, float (&v)[16]) {
-  const float4* s4 = reinterpret_cast<const float4*>(src);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float4 x = __ldcg(s4 + i);
-    v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
-  }
-}
-__device__ __forceinline__ void store_bf16x16(__nv_bfloat16* dst, const float (&v)[16]) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    uint32_t w[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * i + 2 * k], v[8 * i + 2 * k + 1]);
-      w[k] = *reinterpret_cast<uint32_t*>(&b2);
-    }
-    d4[i] = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-}
-
 __device__ __forceinline__ bool finite_f(float x) { return fabsf(x) <= 3.402823466e38f; }
 
 __device__ __forceinline__ float log_add_exp(float x, float y) {
