@@ -194,6 +194,27 @@ def test_dual_attention_layers_host_checks(ispa):
         assert rc in (ispa.ISPA_ERR_CUDA, ispa.ISPA_ERR_NO_DEVICE)
 
 
+def test_dual_attention_layers_binding_checks(ispa):
+    """The binding of the several-layer call rejects inputs the C ABI could
+    not address before any device work: tensors off the GPU, layers that are
+    not contiguous, keys and values at different layer strides, outputs of
+    another shape. CPU tensors are enough to reach these checks."""
+    import torch
+    L, nq, H, hd = 2, 64, 2, 64
+    bf = lambda *shape: torch.zeros(*shape, dtype=torch.bfloat16)
+    q = bf(L, nq, H, hd)
+    with pytest.raises(ValueError):                       # [L, nq, H, hd] expected
+        ispa.ispa_dual_attention_layers(bf(nq, H, hd), bf(L, 16, H, hd), bf(L, 16, H, hd),
+                                        bf(L, nq, H, hd), bf(L, nq, H, hd))
+    with pytest.raises(ValueError):                       # q's layers not contiguous
+        ispa.ispa_dual_attention_layers(q.transpose(1, 2), bf(L, 16, H, hd), bf(L, 16, H, hd),
+                                        bf(L, nq, H, hd), bf(L, nq, H, hd))
+    with pytest.raises(ValueError):                       # keys on the host
+        ispa._kv_layers(bf(L, 16, H, hd), bf(L, 16, H, hd), L, H, hd, "sink")
+    assert ispa._kv_layers(None, None, L, H, hd, "history").len == 0
+    assert ispa._kv_layers(bf(L, 0, H, hd), bf(L, 0, H, hd), L, H, hd, "history").len == 0
+
+
 def test_other_entry_points_host_checks(ispa):
     lib = ispa._load()
     P = 0x1000

@@ -2,6 +2,7 @@
 frame roles of each workload geometry."""
 import math
 
+import pytest
 import torch
 
 from ispa_synth import C0, C1, C2, C3, C4, ar1_stream, layer_streams, projection, scaled
@@ -62,3 +63,44 @@ def test_empty_history_chunk():
     st = layer_streams(cfg, 0)
     ch = st.chunk(0)
     assert ch["k_hist"].shape == (0, 1, 16) and ch["q"].shape == (24, 1, 16)
+
+
+def test_stacked_streams_are_the_per_layer_streams():
+    """All layers' streams in one tensor per Q, K, V: each layer's stream is a
+    view of it with the draws of layer_streams, and stacked_chunk(c) holds
+    chunk c of every layer as [L, tokens, heads, head_dim] views whose layers
+    are contiguous and one stream apart."""
+    import dataclasses
+    from ispa_synth import stacked_chunk, stacked_layer_streams
+    cfg = dataclasses.replace(C0, layers=3)
+    sts, (Q, K, V) = stacked_layer_streams(cfg, [0, 1, 2], seed=5)
+    for i, st in enumerate(sts):
+        ref = layer_streams(cfg, i, seed=5)
+        assert torch.equal(st.q, ref.q) and torch.equal(st.k, ref.k) and torch.equal(st.v, ref.v)
+        assert st.k.data_ptr() == K[i].data_ptr()
+    for c in range(cfg.n_chunks):
+        sc = stacked_chunk(cfg, (Q, K, V), c)
+        for key, x in sc.items():
+            assert x.shape[0] == 3
+            for l in range(3):
+                assert torch.equal(x[l], sts[l].chunk(c)[key]), (c, key)
+                assert x[l].is_contiguous()
+            if x.shape[1]:
+                assert x.untyped_storage().data_ptr() in {t.untyped_storage().data_ptr()
+                                                          for t in (Q, K, V)}
+                assert x.stride(0) == Q[0].numel()
+
+
+def test_warmup_layer_groups():
+    """The warmup driver's groups of layers per attention launch cover every
+    layer once, in order, the last group short (host logic; CPU buffers)."""
+    from kv_cache_absorption_b200.warmup import LayerWarmup
+    mk = lambda L, g: LayerWarmup(2, 64, 64, 16, 64, 256, n_layers=L, device="cpu", n_slots=2,
+                                  group=g)
+    assert mk(30, 10).layer_groups() == [(0, 10), (10, 10), (20, 10)]
+    assert mk(5, 2).layer_groups() == [(0, 2), (2, 2), (4, 1)]
+    assert mk(3, 8).layer_groups() == [(0, 3)]                # a group no larger than the layers
+    r = mk(4, 1)
+    assert r.group == 1 and r.group_slots == []
+    with pytest.raises(ValueError):                           # built without groups
+        r.layers_chunks_stacked([])
