@@ -13,24 +13,24 @@
 //   * one sweep over the 128-column blocks factors A in place and, on the
 //     augmented block [A | Z | Y] with Z = I and Y = B, also yields
 //     Z = L^-1 and Y = L^-1 B (forward substitution). Every step factors and
-//     inverts the diagonal block (one CTA per layer, fp32, shared memory) and
-//     forms the panel L_{>k,k} = A_{>k,k} Linv_kk^T and the block rows
-//     Z_k = Linv_kk Z_k, Y_k = Linv_kk Y_k (one grouped launch).
+//     inverts the diagonal block (fp32, shared memory) and forms the panel
+//     L_{>k,k} = A_{>k,k} Linv_kk^T and the block rows Z_k = Linv_kk Z_k,
+//     Y_k = Linv_kk Y_k.
 //     Several layers: left-looking. Before step k, one grouped launch of
 //     long-K products brings block column k of A and block rows k of Z and Y
 //     up to date (A_{>=k,k} -= L_{>=k,<k} L_{k,<k}^T, Y_k -= L_{k,<k} Y_{<k},
 //     Z_k = -L_{k,<k} Z_{<k}); the finished part is read once per step and
 //     nothing below the block is rewritten, so HBM traffic stays low; these
 //     products sum K in 128-deep chunks (fp32) against accumulator drift.
-//     One layer: right-looking. After step k one grouped launch applies the
-//     rank-128 update to the lower tiles of A and to the rows of Z and Y
-//     below the block: more traffic, but (d/128)^2 tiles per launch where
-//     the left-looking step of a single layer would have ~2 d/128. The
-//     sweep's critical path (factor, panel, the part of each update the
-//     next step needs) runs on a high-priority stream; B = R W and the rest
-//     of each update run on a second stream beside it;
-//   * then one triangular-aware GEMM: Delta W = Z^T Y (for one layer in two
-//     K halves per tile that reduce-add into a zeroed Delta W).
+//     The block factor runs one CTA per layer, the panel as one grouped
+//     launch; finally one triangular-aware GEMM forms Delta W = Z^T Y.
+//     One layer: right-looking, the sweep being a chain of dependent steps
+//     with no other layers to fill the GPU. Each step is one kernel on a
+//     high-priority stream (sweep_step_kernel: the previous step's update of
+//     this block column on the tensor cores, the block factor repeated in
+//     every CTA, each CTA's slice of the panel); the trailing update of A,
+//     the block rows of Z and Y with their updates, and Delta W accumulated
+//     as sum_k Z_k^T Y_k run on three side streams beside the chain.
 // Y is formed by substitution, not as the product Z B: entries of L^-1
 // alternate in sign and |L^-1| |B| can exceed |L^-1 B| by three orders of
 // magnitude, which a product at fp32 precision turns into a 1e-3 relative
@@ -166,15 +166,9 @@ __device__ __forceinline__ void st4(float* d, const float* s) {
 
 // The factor and inverse of steps (1)-(3) above on the block in shared
 // memory: a (lower triangle) is factored in place and z (= I on entry)
-// becomes L^-1, zero above the diagonal. on_idle(J) runs on warps 1-15 once
-// their part of step J's trailing update is done, while warp 0 brings up and
-// factors sub-block J: a hook for the caller's own work, which must leave
-// alone what step J reads (for J = 0: rows and columns 0-31 of a, ljt,
-// rinv, grp). Ends with a barrier.
-template <class Idle>
+// becomes L^-1, zero above the diagonal. Ends with a barrier.
 __device__ __forceinline__ void factor_invert(float* a, float* z, float* pl, float* plT,
-                                              float* ljt, float* rinv, float4* grp, int* status,
-                                              Idle&& on_idle) {
+                                              float* ljt, float* rinv, float4* grp, int* status) {
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   // warp 0: L_JJ of the 32 x 32 diagonal sub-block at J (see step (1) above)
   auto factor32 = [&](int J) {
@@ -306,7 +300,6 @@ __device__ __forceinline__ void factor_invert(float* a, float* z, float* pl, flo
         }
       }
     }
-    if (warp != 0) on_idle(J);                 // warps 1-15, their part of (3) done
     __syncthreads();
     // ---- (2) forward substitution with L_JJ, one 32-vector per thread: the
     // panel rows (x L_JJ^T = a, i.e. L_JJ x^T = a^T) and the columns of the
@@ -392,7 +385,7 @@ __global__ void __launch_bounds__(512, 1) potrf_inv_kernel(const float* __restri
                     i == c + 3 ? 1.f : 0.f);
   }
   __syncthreads();
-  factor_invert(a, z, pl, plT, ljt, rinv, grp, status, [](int) {});
+  factor_invert(a, z, pl, plT, ljt, rinv, grp, status);
   store_linv(z, linv);
 }
 
@@ -597,7 +590,7 @@ __global__ void __launch_bounds__(512, 1) sweep_step_kernel(const __grid_constan
   }
   __syncthreads();
   // ---- (2)
-  factor_invert(a, z, pl, plT, ljt, rinv, grp, p.status, [](int) {});
+  factor_invert(a, z, pl, plT, ljt, rinv, grp, p.status);
   pdl_trigger();
   // ---- (3) L_{S,k}[i][j] = sum_{c <= j} S[i][c] Linv[j][c]: thread = column
   // j and 8 rows; the warp's columns bound c (Linv is zero above the diagonal)
