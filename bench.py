@@ -28,6 +28,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -126,10 +127,16 @@ def absorb_roofline(cfg, gram_ms, solve_ms, bf16_peak, hbm_peak):
 
 
 def source_hash():
+    """Hash of the attention kernel's sources with comments and blank lines
+    removed: a change of the code invalidates the committed traffic figures,
+    a change of the comments does not."""
     h = hashlib.sha256()
     for f in ("attention.cu", "sm100.cuh", "attention.h"):
-        with open(os.path.join(ROOT, "kv_cache_absorption_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "kv_cache_absorption_b200", "csrc", f)) as fh:
+            for line in fh:
+                code = re.sub(r"//.*$", "", line).strip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -21,6 +21,12 @@
 //   A_loc = sum_local e^(LSE_s - LSE_loc) O_s,
 //   D = sum_hist e^(LSE_s - LSE_full) (O_s - A_loc), A_full = A_loc + D.
 // No unit waits for another: whichever finishes last does the merge.
+// A joint plan instead gives each (head, pair) one unit for both branches:
+// the local keys, A_loc and LSE_loc stored when the history starts, the
+// history from a fresh softmax state, and the same merge in its epilogue
+// (a separate kernel instantiation). One launch may cover several layers of
+// one shape (a layer axis in the tensor maps, per-layer output strides): the
+// units of all of them fill whole waves of the SMs.
 //
 // Unit CTA (384 threads), both query tiles t = 0, 1 share every K/V tile:
 //   warp 0      TMA producer: the two Q tiles, then 128-key tiles into a
