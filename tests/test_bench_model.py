@@ -76,3 +76,18 @@ def test_bench_line_config_is_shared_by_both_arms():
     a = bench.config_of(C2, 1, False, 15)
     assert a["workload"] == C2.name and a["layers"] == 30 and a["history"] == [0, 4680, 9360, 14040]
     assert a["parallelism"] == "single GPU"
+
+
+def test_clock_record_rejection():
+    """A timed region is measured again when its clock record shows a slowdown
+    other than the power cap, or SM clocks far below their maximum with no
+    reason active (a clock lock left behind); the power cap alone is kept."""
+    rec = lambda mhz, reasons: {"sm_mhz": mhz, "sm_max_mhz": 1965.0, "reasons": reasons}
+    assert not bench.clocks_rejected(None)
+    assert not bench.clocks_rejected(rec(1700.0, ["sw_power_cap"]))
+    assert not bench.clocks_rejected(rec(1900.0, []))
+    assert bench.clocks_rejected(rec(1900.0, ["hw_slowdown"]))
+    assert bench.clocks_rejected(rec(1500.0, ["sw_power_cap", "sw_thermal_slowdown"]))
+    assert bench.clocks_rejected(rec(1000.0, []))
+    assert not bench.clocks_rejected(rec(1000.0, ["sw_power_cap"]))
+    assert bench.any_over_ranks(True, 1) and not bench.any_over_ranks(False, 1)
