@@ -918,13 +918,15 @@ int64_t attention_key_tiles(int64_t len) { return (len + BN - 1) / BN; }
 
 // ---------------------------------------------------------------- planning
 //
-// Split counts are chosen per shape by simulating the hardware block
-// scheduler on the units: blocks start in grid order (longest key range
-// first), each on the SM that frees first; a unit costs its key tiles plus a
-// fixed per-unit cost (prologue, epilogue, merge). Candidates: the local
-// branch in 1..4 ranges; the history (when present) in n0, n0 + 1, n0 + 2
-// ranges, n0 being about two local branches of keys per range (at most 64).
-// The fewest units win unless more splits shorten the makespan by > 1%.
+// Split counts are chosen per shape and layer count by simulating the
+// hardware block scheduler on the units of the whole launch: blocks start in
+// grid order (longest key range first), each on the SM that frees first; a
+// unit costs its key tiles plus a fixed per-unit cost (prologue, epilogue,
+// merge). Candidates: the local branch in 1..4 ranges; the history (when
+// present) in n0, n0 + 1, n0 + 2 ranges, n0 being about two local branches
+// of keys per range (at most 64); for a launch over several layers whose
+// call stores A_loc, also one joint unit per (head, pair). The fewest units
+// win unless more splits shorten the makespan by > 1%.
 
 namespace {
 
