@@ -84,13 +84,14 @@ def _stack_layers(chunks, key, pad_rows=0):
     return t
 
 
-def test_joint_units_equal_the_two_range_plan(lib):
+@pytest.mark.parametrize("hd", [128, 64])
+def test_joint_units_equal_the_two_range_plan(lib, hd):
     """A joint unit per (head, query pair) (the local keys, A_loc stored where
     the history starts, then the history from a fresh state, merged in the
     epilogue) gives the same bits as the plan with one local and one history
     range merged by the later unit: single-layer and over three layers, with
     ragged query pairs and a partial last tile in every branch."""
-    L, nq, H, hd = 3, 700, 4, 128
+    L, nq, H = 3, 700, 4
     chunks = [random_chunk(nq, 300, 600, 2000, H, hd, seed=60 + 5 * l) for l in range(L)]
     keys = ("a_loc", "d", "a_full", "lse_loc", "lse_hist", "lse_full")
     q = _stack_layers(chunks, "q")
