@@ -108,18 +108,24 @@ def measure_tf32_peak():
 def absorb_roofline(cfg, gram_ms, solve_ms, bf16_peak, hbm_peak):
     """Precision-constrained roofline of the absorb per layer: Gram 4 N d^2 at
     the tf32 rate, solve (1/3 + 4) d^3 at a third of it (three tf32 products
-    per fp32-accurate product), error 6 d^2 fp32 reads at the HBM rate."""
+    per fp32-accurate product), error 6 d^2 fp32 reads at the HBM rate. For
+    context, also the time if every flop ran at the bf16 rate (a bound that
+    ignores the precision the solve needs)."""
     d, L = cfg.d, cfg.layers
     tf32, src = tf32_peak(bf16_peak)
     t_gram = 4.0 * cfg.warmup_rows * d * d / (tf32 * 1e12)
     t_solve = (1.0 / 3.0 + 4.0) * d ** 3 / (tf32 / 3.0 * 1e12)
     t_err = 6.0 * d * d * 4 / (hbm_peak * 1e9)
     t_star = (t_gram + t_solve + t_err) * 1e3
+    t_bf16 = ((4.0 * cfg.warmup_rows * d * d + (1.0 / 3.0 + 4.0) * d ** 3) / (bf16_peak * 1e12)
+              + t_err) * 1e3
     got = (gram_ms + solve_ms) / L
     return {"bound": "tensor (tf32 Gram, 3xTF32 solve) + hbm (error)",
             "t_star_ms_per_layer": round(t_star, 4), "achieved_ms_per_layer": round(got, 4),
             "frac": round(t_star / got, 4), "tf32_peak": tf32, "tf32_peak_source": src,
             "hbm_peak": hbm_peak,
+            "bf16_only": {"t_ms_per_layer": round(t_bf16, 4), "frac": round(t_bf16 / got, 4),
+                          "note": "every flop at the bf16 rate: context, not the target"},
             "parts_ms_per_layer": {"gram": round(gram_ms / L, 4), "solve_error": round(solve_ms / L, 4),
                                    "t_star_gram": round(t_gram * 1e3, 4),
                                    "t_star_solve": round(t_solve * 1e3, 4),

@@ -51,6 +51,11 @@ def test_absorb_roofline_is_the_sum_of_its_parts():
     assert r["t_star_ms_per_layer"] == pytest.approx(t_gram + t_solve + t_err, abs=1e-4)
     assert r["achieved_ms_per_layer"] == pytest.approx(8.5)
     assert r["frac"] == pytest.approx((t_gram + t_solve + t_err) / 8.5, abs=1e-4)
+    # context: the same flops all at the bf16 rate, the error reads unchanged
+    t_bf16 = (4.0 * n * d * d + (1.0 / 3.0 + 4.0) * d ** 3) / (1600.0 * 1e12) * 1e3 + t_err
+    assert r["bf16_only"]["t_ms_per_layer"] == pytest.approx(t_bf16, abs=1e-4)
+    assert r["bf16_only"]["frac"] == pytest.approx(t_bf16 / 8.5, abs=1e-4)
+    assert r["bf16_only"]["t_ms_per_layer"] < r["t_star_ms_per_layer"]
 
 
 @pytest.mark.parametrize("config,layers,k", [("c2", 4, 2), ("c3", 2, 1), ("c2", 30, 15)])
