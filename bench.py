@@ -297,10 +297,13 @@ def oracle_throughput(cfg, budget_s: float):
             acc[s][1] += timing[s][1]
         spent += sum(t for _, t in timing.values())
         n += 1
-    t_full = sum(work[s] * acc[s][1] / max(acc[s][0], 1.0) for s in work if work[s] > 0)
+    stages = {s: work[s] * acc[s][1] / max(acc[s][0], 1.0) for s in work if work[s] > 0}
+    t_full = sum(stages.values())
     total = sum(work.values())
     cores, blas = cpu_cores()
     return {"value": round(total / t_full / 1e12, 6), "unit": "TFLOP/s", "cores": blas or cores,
+            "host_cores": cores, "blas_threads": blas,
+            "stage_seconds_per_full_step": {s: round(t, 3) for s, t in stages.items()},
             "kind": "oracle",
             "sample": (f"{n} x: float64 oracle on 256 query rows of the last chunk for one head "
                        f"(all keys), the Gram and direct error of 1024 rows, one full "
@@ -1026,7 +1029,8 @@ def run_reference(args):
             for s in acc:
                 acc[s][0] += timing[s][0]
                 acc[s][1] += timing[s][1]
-    t_full = sum(work[s] * acc[s][1] / acc[s][0] for s in work if acc[s][0] > 0)
+    stages = {s: work[s] * acc[s][1] / acc[s][0] for s in work if acc[s][0] > 0 and work[s] > 0}
+    t_full = sum(stages.values())
     value = total / t_full / 1e12
     cores, blas = cpu_cores()
     sample = (f"per step: float64 oracle on 256 query rows of the last chunk for one head (all "
@@ -1041,6 +1045,9 @@ def run_reference(args):
            "step_is": "a bounded sample of the workload (see cpu_baseline.sample)",
            "full_step_s_extrapolated": round(t_full, 3),
            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas or cores,
+                            "host_cores": cores, "blas_threads": blas,
+                            "stage_seconds_per_full_step": {k: round(t, 3)
+                                                            for k, t in stages.items()},
                             "kind": "oracle", "sample": sample},
            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}

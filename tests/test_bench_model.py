@@ -96,3 +96,15 @@ def test_clock_record_rejection():
     assert bench.clocks_rejected(rec(1000.0, []))
     assert not bench.clocks_rejected(rec(1000.0, ["sw_power_cap"]))
     assert bench.any_over_ranks(True, 1) and not bench.any_over_ranks(False, 1)
+
+
+def test_oracle_baseline_reports_its_stages_and_threads():
+    """The CPU baseline's per-stage extrapolated seconds add up to its full
+    step, and it states the host cores and BLAS threads it ran with."""
+    from ispa_synth import CONFIGS
+    r = bench.oracle_throughput(CONFIGS["c0"], budget_s=0.0)
+    st = r["stage_seconds_per_full_step"]
+    assert set(st) == {"attention", "gram", "solve"}        # the error stage is credited no flops
+    assert sum(st.values()) == pytest.approx(r["seconds_per_full_step"], abs=5e-3)
+    assert r["host_cores"] >= 1 and r["cores"] >= 1
+    assert r["kind"] == "oracle" and r["value"] > 0
