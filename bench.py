@@ -105,6 +105,15 @@ def measure_tf32_peak():
                       "device": torch.cuda.get_device_name()}), flush=True)
 
 
+def error_bytes(cfg):
+    """Bytes the batched error pass reads per layer (fp32, W W^T resident):
+    the 128 x 128 tiles of G and S on and above the diagonal, R, W W^T,
+    Delta W and B in full."""
+    t = cfg.d // 128
+    upper = t * (t + 1) // 2
+    return int((2 * upper * 128 * 128 + 4 * cfg.d * cfg.d) * 4)
+
+
 def absorb_roofline(cfg, gram_ms, solve_ms, bf16_peak, hbm_peak):
     """Precision-constrained roofline of the absorb per layer: Gram 4 N d^2 at
     the tf32 rate, solve (1/3 + 4) d^3 at a third of it (three tf32 products
@@ -486,7 +495,9 @@ def measure_warmup(args, cfg, world, rank, steps, warmup, with_e2e, with_cpu):
                     else:
                         runner.gram(first=(c == 0), layer=l0 + j)
                 ev["g1"].append(E()); ev["g1"][-1].record()
-        runner.absorb_all(W_all, err_mine)
+        runner.solve_all(W_all)
+        ev["e0"].append(E()); ev["e0"][-1].record()
+        runner.error_all(W_all, err_mine)
         ev["s1"].append(E()); ev["s1"][-1].record()
         err.copy_(gather_errors(err_mine, L, world) if sharded else err_mine)
         rank_layers(err, K, perm, sel)
@@ -528,7 +539,7 @@ def measure_warmup(args, cfg, world, rank, steps, warmup, with_e2e, with_cpu):
 
     # per-stage breakdown: a few more steps on one stream, events around every stage
     n_inst = max(1, min(steps, 5))
-    ev = {"a0": [], "a1": [], "g1": [], "s1": []}
+    ev = {"a0": [], "a1": [], "g1": [], "e0": [], "s1": []}
     for _ in range(n_inst):
         flush.zero_()
         step_instrumented(ev)
@@ -539,6 +550,8 @@ def measure_warmup(args, cfg, world, rank, steps, warmup, with_e2e, with_cpu):
     per_step = len(groups) * cfg.n_chunks
     solve_ms = sum(ev["g1"][(i + 1) * per_step - 1].elapsed_time(ev["s1"][i])
                    for i in range(n_inst)) / n_inst
+    # of which the batched error pass (one read of every layer's matrices)
+    error_ms = sum(a.elapsed_time(b) for a, b in zip(ev["e0"], ev["s1"])) / n_inst
     # the attention calls alone, with the layers in flight on the step's streams
     # (the concurrency the timed step runs them at; no Gram, solve or error)
     def attention_pass():
@@ -618,6 +631,13 @@ def measure_warmup(args, cfg, world, rank, steps, warmup, with_e2e, with_cpu):
         "roofline": roofline,
         "absorb_roofline": absorb_roofline(cfg, gram_ms * L / L_mine, solve_ms * L / L_mine,
                                            bf16_peak, hbm_peak),
+        "error_hbm": {
+            "kernel": "batched layer error from W W^T (dot5_kernel + finalize)",
+            "ms_per_step": round(error_ms, 4),
+            "algorithmic_bytes_per_layer": error_bytes(cfg),
+            "achieved": round(error_bytes(cfg) * L_mine / (error_ms * 1e-3) / 1e9, 1),
+            "peak": hbm_peak, "unit": "GB/s",
+            "frac": round(error_bytes(cfg) * L_mine / (error_ms * 1e-3) / 1e9 / hbm_peak, 4)},
         "gpu_launches": int(launches),
         "device_status": status,
         "clocks": clocks,

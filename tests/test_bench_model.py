@@ -108,3 +108,15 @@ def test_oracle_baseline_reports_its_stages_and_threads():
     assert sum(st.values()) == pytest.approx(r["seconds_per_full_step"], abs=5e-3)
     assert r["host_cores"] >= 1 and r["cores"] >= 1
     assert r["kind"] == "oracle" and r["value"] > 0
+
+
+def test_error_pass_bytes():
+    """The batched error pass reads G and S on and above the tile diagonal and
+    R, W W^T, Delta W and B in full, fp32: about 5 d^2 floats a layer (an ncu
+    capture of the pass over four d = 1536 layers read 191.9 MB)."""
+    for cfg in (C1, C3):
+        d, t = cfg.d, cfg.d // 128
+        tiles_upper = t * (t + 1) // 2
+        assert bench.error_bytes(cfg) == 4 * (2 * tiles_upper * 128 ** 2 + 4 * d * d)
+    assert bench.error_bytes(C1) == pytest.approx(47.97e6, rel=1e-3)     # d = 1536
+    assert bench.error_bytes(C3) == pytest.approx(526.9e6, rel=1e-3)     # d = 5120
